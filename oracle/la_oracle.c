@@ -1,0 +1,381 @@
+/*
+ * la_oracle.c -- plain, slow, fp64 CPU oracle for causal linear attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the CPU
+ * baseline leg of the benchmark may load this library.  It shares no code,
+ * header, table or helper with the CUDA path, and it includes nothing from it.
+ *
+ * What it computes (all arithmetic in double precision, inputs given as
+ * doubles, layouts row-major [B,H,N,D]; every (b,h) slice is independent):
+ *
+ *   phi      -- the feature maps.
+ *               elu(x)+1 ("Transformers are RNNs", the linear-attention
+ *               feature map it proposes; alpha = 1): x+1 for x>0, exp(x) else.
+ *               BASED second-order Taylor map ("Simple linear attention
+ *               language models balance the recall-throughput tradeoff",
+ *               Knowl 3, the equation phi(q).phi(k) = 1 + q.k + (q.k)^2/2):
+ *               [1 | x/d'^(1/4) | x_a x_b / (sqrt(2) sqrt(d'))], the second
+ *               block row-major in (a, b), so 1 + d' + d'^2 features.
+ *   forward_brute      -- the masked parallel form, Knowl 3 eq. for y_i:
+ *               a_ij = phi(q_i).phi(k_j) for j <= i,
+ *               y_i  = sum_j a_ij v_j / sum_j a_ij,           O(N^2 F).
+ *   forward_rows       -- the same, for selected positions of one slice.
+ *   forward_recurrent  -- the recurrent form, Knowl 3 eqs. for s_i, z_i, y_i:
+ *               s_i = s_{i-1} + phi(k_i)^T v_i, z_i = z_{i-1} + phi(k_i)^T,
+ *               y_i = phi(q_i) s_i / phi(q_i) z_i   (state includes token i),
+ *               optionally from a given state, returning the final state
+ *               (Knowl 5: the prefill may write its final state for decode).
+ *   decode_step        -- one step of that recurrence on a given state,
+ *               output taken from the updated state (Knowl 5, recurrent
+ *               generation kernel description).
+ *   backward_brute / backward_recurrent -- gradients of y with respect to
+ *               q, k, v for an upstream gradient dO.  The pages give no
+ *               backward pass; it is the derivative of the Knowl 3 parallel
+ *               form, written out by hand:
+ *                 g_i    = dO_i / den_i,   dden_i = -g_i . y_i,
+ *                 da_ij  = g_i . v_j + dden_i                (j <= i),
+ *                 dv_j   = sum_{i>=j} a_ij g_i,
+ *                 dphiq_i = sum_{j<=i} da_ij phi(k_j),
+ *                 dphik_j = sum_{i>=j} da_ij phi(q_i),
+ *               then dq = J_phi(q)^T dphiq and dk = J_phi(k)^T dphik.
+ *               The recurrent version scans s,z forward for dq and
+ *               R_j = sum_{i>=j} phi(q_i) g_i^T, r_j = sum_{i>=j} phi(q_i) dden_i
+ *               backward for dk, dv.
+ *
+ * Parallelism: OpenMP over (b,h) slices only; each slice is computed in the
+ * plain order above.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_ELU1 0
+#define ORC_TAYLOR2 1
+
+int orc_feature_dim(int fmap, int dqk)
+{
+    if (fmap == ORC_ELU1) return dqk;
+    if (fmap == ORC_TAYLOR2) return 1 + dqk + dqk * dqk;
+    return -1;
+}
+
+/* phi(x) for one vector x[dqk] -> out[F]. */
+void orc_phi(int fmap, int dqk, const double *x, double *out)
+{
+    if (fmap == ORC_ELU1) {
+        for (int a = 0; a < dqk; ++a)
+            out[a] = x[a] > 0.0 ? x[a] + 1.0 : exp(x[a]);
+        return;
+    }
+    /* Taylor: constant, first-order coordinates, then second-order products. */
+    const double c1 = pow((double)dqk, 0.25);            /* d'^(1/4)          */
+    const double c2 = sqrt(2.0) * sqrt((double)dqk);     /* sqrt(2) sqrt(d')  */
+    out[0] = 1.0;
+    for (int a = 0; a < dqk; ++a) out[1 + a] = x[a] / c1;
+    for (int a = 0; a < dqk; ++a)
+        for (int b = 0; b < dqk; ++b)
+            out[1 + dqk + a * dqk + b] = x[a] * x[b] / c2;
+}
+
+/* dx = J_phi(x)^T dphi  (vector-Jacobian product of the feature map). */
+void orc_phi_vjp(int fmap, int dqk, const double *x, const double *dphi, double *dx)
+{
+    if (fmap == ORC_ELU1) {
+        for (int a = 0; a < dqk; ++a)
+            dx[a] = dphi[a] * (x[a] > 0.0 ? 1.0 : exp(x[a]));
+        return;
+    }
+    const double c1 = pow((double)dqk, 0.25);
+    const double c2 = sqrt(2.0) * sqrt((double)dqk);
+    /* phi_{1+a} = x_a / c1;  phi_{1+d'+a d'+b} = x_a x_b / c2. */
+    for (int c = 0; c < dqk; ++c) {
+        double s = dphi[1 + c] / c1;
+        for (int b = 0; b < dqk; ++b) {
+            const double d_cb = dphi[1 + dqk + c * dqk + b];  /* d/dx_c of x_c x_b */
+            const double d_bc = dphi[1 + dqk + b * dqk + c];  /* d/dx_c of x_b x_c */
+            s += (d_cb + d_bc) * x[b] / c2;
+        }
+        dx[c] = s;
+    }
+}
+
+static double dot(const double *a, const double *b, int n)
+{
+    double s = 0.0;
+    for (int i = 0; i < n; ++i) s += a[i] * b[i];
+    return s;
+}
+
+/* Feature vectors of all N rows of one slice: out[N][F]. */
+static double *phi_rows(int fmap, int N, int dqk, const double *x)
+{
+    const int F = orc_feature_dim(fmap, dqk);
+    double *out = (double *)malloc(sizeof(double) * (size_t)N * (size_t)F);
+    for (int i = 0; i < N; ++i) orc_phi(fmap, dqk, x + (size_t)i * dqk, out + (size_t)i * F);
+    return out;
+}
+
+/* ---------------------------------------------------------------- forward */
+
+/* Masked parallel form for one slice at the listed positions. */
+static void brute_slice_rows(int fmap, int N, int dqk, int dv,
+                             const double *q, const double *k, const double *v,
+                             const double *phik, const int64_t *rows, int nrows,
+                             double *o, double *den)
+{
+    const int F = orc_feature_dim(fmap, dqk);
+    double *phiq = (double *)malloc(sizeof(double) * (size_t)F);
+    double *num = (double *)malloc(sizeof(double) * (size_t)dv);
+    for (int r = 0; r < nrows; ++r) {
+        const int64_t i = rows[r];
+        orc_phi(fmap, dqk, q + (size_t)i * dqk, phiq);
+        double d = 0.0;
+        for (int c = 0; c < dv; ++c) num[c] = 0.0;
+        for (int64_t j = 0; j <= i; ++j) {
+            const double a = dot(phiq, phik + (size_t)j * F, F);
+            d += a;
+            for (int c = 0; c < dv; ++c) num[c] += a * v[(size_t)j * dv + c];
+        }
+        for (int c = 0; c < dv; ++c) o[(size_t)r * dv + c] = num[c] / d;
+        if (den) den[r] = d;
+    }
+    (void)N;
+    free(phiq);
+    free(num);
+}
+
+void orc_forward_brute(int fmap, int B, int H, int N, int dqk, int dv,
+                       const double *q, const double *k, const double *v,
+                       double *o, double *den)
+{
+    const int BH = B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int bh = 0; bh < BH; ++bh) {
+        const double *qs = q + (size_t)bh * N * dqk;
+        const double *ks = k + (size_t)bh * N * dqk;
+        const double *vs = v + (size_t)bh * N * dv;
+        double *phik = phi_rows(fmap, N, dqk, ks);
+        int64_t *rows = (int64_t *)malloc(sizeof(int64_t) * (size_t)N);
+        for (int i = 0; i < N; ++i) rows[i] = i;
+        brute_slice_rows(fmap, N, dqk, dv, qs, ks, vs, phik, rows, N,
+                         o + (size_t)bh * N * dv, den ? den + (size_t)bh * N : NULL);
+        free(rows);
+        free(phik);
+    }
+}
+
+/* Brute force at selected positions of slice bh (for sampled checks of
+ * large workloads).  o_rows[nrows][dv], den_rows[nrows] (nullable). */
+void orc_forward_rows(int fmap, int N, int dqk, int dv,
+                      const double *q, const double *k, const double *v,
+                      const int64_t *rows, int nrows, double *o_rows, double *den_rows)
+{
+    /* Only phi(k_j) for j <= max row is needed. */
+    int64_t last = 0;
+    for (int r = 0; r < nrows; ++r) if (rows[r] > last) last = rows[r];
+    double *phik = phi_rows(fmap, (int)(last + 1), dqk, k);
+    brute_slice_rows(fmap, N, dqk, dv, q, k, v, phik, rows, nrows, o_rows, den_rows);
+    free(phik);
+}
+
+static void recurrent_slice(int fmap, int N, int dqk, int dv,
+                            const double *q, const double *k, const double *v,
+                            double *s, double *z, double *o, double *den)
+{
+    const int F = orc_feature_dim(fmap, dqk);
+    double *phiq = (double *)malloc(sizeof(double) * (size_t)F);
+    double *phik = (double *)malloc(sizeof(double) * (size_t)F);
+    for (int i = 0; i < N; ++i) {
+        orc_phi(fmap, dqk, q + (size_t)i * dqk, phiq);
+        orc_phi(fmap, dqk, k + (size_t)i * dqk, phik);
+        const double *vi = v + (size_t)i * dv;
+        /* s_i = s_{i-1} + phi(k_i)^T v_i ; z_i = z_{i-1} + phi(k_i)^T */
+        for (int f = 0; f < F; ++f) {
+            for (int c = 0; c < dv; ++c) s[(size_t)f * dv + c] += phik[f] * vi[c];
+            z[f] += phik[f];
+        }
+        /* y_i = phi(q_i) s_i / phi(q_i) z_i */
+        const double d = dot(phiq, z, F);
+        for (int c = 0; c < dv; ++c) {
+            double n = 0.0;
+            for (int f = 0; f < F; ++f) n += phiq[f] * s[(size_t)f * dv + c];
+            o[(size_t)i * dv + c] = n / d;
+        }
+        if (den) den[i] = d;
+    }
+    free(phiq);
+    free(phik);
+}
+
+/* Recurrent form over all slices.  s0/z0 (nullable) give a starting state
+ * [B,H,F,dv] / [B,H,F]; s_out/z_out (nullable) receive the final state. */
+void orc_forward_recurrent(int fmap, int B, int H, int N, int dqk, int dv,
+                           const double *q, const double *k, const double *v,
+                           const double *s0, const double *z0,
+                           double *o, double *den, double *s_out, double *z_out)
+{
+    const int BH = B * H;
+    const int F = orc_feature_dim(fmap, dqk);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int bh = 0; bh < BH; ++bh) {
+        double *s = (double *)calloc((size_t)F * dv, sizeof(double));
+        double *z = (double *)calloc((size_t)F, sizeof(double));
+        if (s0) memcpy(s, s0 + (size_t)bh * F * dv, sizeof(double) * (size_t)F * dv);
+        if (z0) memcpy(z, z0 + (size_t)bh * F, sizeof(double) * (size_t)F);
+        recurrent_slice(fmap, N, dqk, dv,
+                        q + (size_t)bh * N * dqk, k + (size_t)bh * N * dqk, v + (size_t)bh * N * dv,
+                        s, z, o + (size_t)bh * N * dv, den ? den + (size_t)bh * N : NULL);
+        if (s_out) memcpy(s_out + (size_t)bh * F * dv, s, sizeof(double) * (size_t)F * dv);
+        if (z_out) memcpy(z_out + (size_t)bh * F, z, sizeof(double) * (size_t)F);
+        free(s);
+        free(z);
+    }
+}
+
+/* One decode step for BH independent heads: q,k [BH,dqk], v [BH,dv];
+ * s [BH,F,dv], z [BH,F] updated in place; y [BH,dv] from the updated state. */
+void orc_decode_step(int fmap, int BH, int dqk, int dv,
+                     const double *q, const double *k, const double *v,
+                     double *s, double *z, double *y)
+{
+    const int F = orc_feature_dim(fmap, dqk);
+#pragma omp parallel for schedule(static)
+    for (int bh = 0; bh < BH; ++bh)
+        recurrent_slice(fmap, 1, dqk, dv, q + (size_t)bh * dqk, k + (size_t)bh * dqk,
+                        v + (size_t)bh * dv, s + (size_t)bh * F * dv, z + (size_t)bh * F,
+                        y + (size_t)bh * dv, NULL);
+}
+
+/* --------------------------------------------------------------- backward */
+
+void orc_backward_brute(int fmap, int B, int H, int N, int dqk, int dv,
+                        const double *q, const double *k, const double *v,
+                        const double *dout, double *dq, double *dk, double *dvv)
+{
+    const int BH = B * H;
+    const int F = orc_feature_dim(fmap, dqk);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int bh = 0; bh < BH; ++bh) {
+        const double *qs = q + (size_t)bh * N * dqk;
+        const double *ks = k + (size_t)bh * N * dqk;
+        const double *vs = v + (size_t)bh * N * dv;
+        const double *dos = dout + (size_t)bh * N * dv;
+        double *dqs = dq + (size_t)bh * N * dqk;
+        double *dks = dk + (size_t)bh * N * dqk;
+        double *dvs = dvv + (size_t)bh * N * dv;
+        double *phiq = phi_rows(fmap, N, dqk, qs);
+        double *phik = phi_rows(fmap, N, dqk, ks);
+        double *A = (double *)calloc((size_t)N * N, sizeof(double));   /* a_ij, j<=i */
+        double *dA = (double *)calloc((size_t)N * N, sizeof(double));
+        double *g = (double *)malloc(sizeof(double) * (size_t)N * dv);
+        double *dphiq = (double *)calloc((size_t)N * F, sizeof(double));
+        double *dphik = (double *)calloc((size_t)N * F, sizeof(double));
+        for (int i = 0; i < N; ++i) {
+            double d = 0.0;
+            for (int j = 0; j <= i; ++j) {
+                A[(size_t)i * N + j] = dot(phiq + (size_t)i * F, phik + (size_t)j * F, F);
+                d += A[(size_t)i * N + j];
+            }
+            /* y_i, then g_i = dO_i / den_i and dden_i = -g_i . y_i */
+            double gy = 0.0;
+            for (int c = 0; c < dv; ++c) {
+                double n = 0.0;
+                for (int j = 0; j <= i; ++j) n += A[(size_t)i * N + j] * vs[(size_t)j * dv + c];
+                const double y = n / d;
+                g[(size_t)i * dv + c] = dos[(size_t)i * dv + c] / d;
+                gy += g[(size_t)i * dv + c] * y;
+            }
+            const double dden = -gy;
+            for (int j = 0; j <= i; ++j)
+                dA[(size_t)i * N + j] = dot(g + (size_t)i * dv, vs + (size_t)j * dv, dv) + dden;
+        }
+        for (int j = 0; j < N; ++j)
+            for (int c = 0; c < dv; ++c) {
+                double s = 0.0;
+                for (int i = j; i < N; ++i) s += A[(size_t)i * N + j] * g[(size_t)i * dv + c];
+                dvs[(size_t)j * dv + c] = s;
+            }
+        for (int i = 0; i < N; ++i)
+            for (int j = 0; j <= i; ++j) {
+                const double da = dA[(size_t)i * N + j];
+                for (int f = 0; f < F; ++f) {
+                    dphiq[(size_t)i * F + f] += da * phik[(size_t)j * F + f];
+                    dphik[(size_t)j * F + f] += da * phiq[(size_t)i * F + f];
+                }
+            }
+        for (int i = 0; i < N; ++i) {
+            orc_phi_vjp(fmap, dqk, qs + (size_t)i * dqk, dphiq + (size_t)i * F, dqs + (size_t)i * dqk);
+            orc_phi_vjp(fmap, dqk, ks + (size_t)i * dqk, dphik + (size_t)i * F, dks + (size_t)i * dqk);
+        }
+        free(phiq); free(phik); free(A); free(dA); free(g); free(dphiq); free(dphik);
+    }
+}
+
+void orc_backward_recurrent(int fmap, int B, int H, int N, int dqk, int dv,
+                            const double *q, const double *k, const double *v,
+                            const double *dout, double *dq, double *dk, double *dvv)
+{
+    const int BH = B * H;
+    const int F = orc_feature_dim(fmap, dqk);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int bh = 0; bh < BH; ++bh) {
+        const double *qs = q + (size_t)bh * N * dqk;
+        const double *ks = k + (size_t)bh * N * dqk;
+        const double *vs = v + (size_t)bh * N * dv;
+        const double *dos = dout + (size_t)bh * N * dv;
+        double *dqs = dq + (size_t)bh * N * dqk;
+        double *dks = dk + (size_t)bh * N * dqk;
+        double *dvs = dvv + (size_t)bh * N * dv;
+        double *s = (double *)calloc((size_t)F * dv, sizeof(double));
+        double *z = (double *)calloc((size_t)F, sizeof(double));
+        double *g = (double *)malloc(sizeof(double) * (size_t)N * dv);
+        double *dden = (double *)malloc(sizeof(double) * (size_t)N);
+        double *phiq = (double *)malloc(sizeof(double) * (size_t)F);
+        double *phik = (double *)malloc(sizeof(double) * (size_t)F);
+        double *dphi = (double *)malloc(sizeof(double) * (size_t)F);
+        /* Forward-order scan: s_i, z_i include token i. */
+        for (int i = 0; i < N; ++i) {
+            orc_phi(fmap, dqk, qs + (size_t)i * dqk, phiq);
+            orc_phi(fmap, dqk, ks + (size_t)i * dqk, phik);
+            for (int f = 0; f < F; ++f) {
+                for (int c = 0; c < dv; ++c) s[(size_t)f * dv + c] += phik[f] * vs[(size_t)i * dv + c];
+                z[f] += phik[f];
+            }
+            const double d = dot(phiq, z, F);
+            double gy = 0.0;
+            for (int c = 0; c < dv; ++c) {
+                double n = 0.0;
+                for (int f = 0; f < F; ++f) n += phiq[f] * s[(size_t)f * dv + c];
+                g[(size_t)i * dv + c] = dos[(size_t)i * dv + c] / d;
+                gy += g[(size_t)i * dv + c] * (n / d);
+            }
+            dden[i] = -gy;
+            /* dphi(q_i) = s_i g_i + z_i dden_i */
+            for (int f = 0; f < F; ++f)
+                dphi[f] = dot(s + (size_t)f * dv, g + (size_t)i * dv, dv) + z[f] * dden[i];
+            orc_phi_vjp(fmap, dqk, qs + (size_t)i * dqk, dphi, dqs + (size_t)i * dqk);
+        }
+        /* Reverse-order scan: R_j = sum_{i>=j} phi(q_i) g_i^T (reusing s), r_j (reusing z). */
+        memset(s, 0, sizeof(double) * (size_t)F * dv);
+        memset(z, 0, sizeof(double) * (size_t)F);
+        for (int j = N - 1; j >= 0; --j) {
+            orc_phi(fmap, dqk, qs + (size_t)j * dqk, phiq);
+            orc_phi(fmap, dqk, ks + (size_t)j * dqk, phik);
+            for (int f = 0; f < F; ++f) {
+                for (int c = 0; c < dv; ++c) s[(size_t)f * dv + c] += phiq[f] * g[(size_t)j * dv + c];
+                z[f] += phiq[f] * dden[j];
+            }
+            /* dphi(k_j) = R_j v_j + r_j ; dv_j = R_j^T phi(k_j) */
+            for (int f = 0; f < F; ++f)
+                dphi[f] = dot(s + (size_t)f * dv, vs + (size_t)j * dv, dv) + z[f];
+            orc_phi_vjp(fmap, dqk, ks + (size_t)j * dqk, dphi, dks + (size_t)j * dqk);
+            for (int c = 0; c < dv; ++c) {
+                double a = 0.0;
+                for (int f = 0; f < F; ++f) a += s[(size_t)f * dv + c] * phik[f];
+                dvs[(size_t)j * dv + c] = a;
+            }
+        }
+        free(s); free(z); free(g); free(dden); free(phiq); free(phik); free(dphi);
+    }
+}

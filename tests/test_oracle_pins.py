@@ -1,0 +1,333 @@
+"""Pins of the fp64 CPU oracle against facts that do not come from the oracle.
+
+Each test checks the oracle against something fixed by the pages or by
+mathematics: a library routine for a special case, a closed form, an
+invariant, brute force against a different algorithm, or finite differences.
+Together they are chosen so that a dropped term, a wrong sign, a wrong index
+or a transposed operand anywhere in the oracle fails at least one of them.
+
+Page citations name the page ("Simple linear attention language models
+balance the recall-throughput tradeoff", the BASED page; "Transformers are
+RNNs", the linear-attention page) and the Knowl / section.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+ELU1, TAYLOR2 = 0, 1
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def rnd(seed, *shape, scale=1.0):
+    g = np.random.default_rng(seed)
+    return g.standard_normal(shape) * scale
+
+
+# ----------------------------------------------------------------- feature maps
+
+def test_feature_dims_match_pages(orc):
+    # BASED page, Knowl 5: for projected dimension 16 the unpadded expanded
+    # feature dimension is 273 (= 1 + 16 + 16^2).
+    consts = json.load(open(os.path.join(GOLDEN, "based_page_constants.json")))
+    assert orc.feature_dim(TAYLOR2, 16) == consts["taylor_feature_dim_d16"]["value"]
+    for d in (1, 2, 4, 8, 16, 32):
+        assert orc.feature_dim(ELU1, d) == d
+        assert orc.feature_dim(TAYLOR2, d) == 1 + d + d * d
+
+
+def test_elu1_matches_library_elu():
+    # elu(x)+1 with alpha = 1 is torch's ELU plus one (a library routine).
+    from oracle import oracle as orc
+    x = rnd(1, 7, 32, scale=3.0)
+    x[0, :4] = [0.0, -0.0, 1e-300, -1e-300]
+    ref = torch.nn.functional.elu(torch.from_numpy(x), alpha=1.0).numpy() + 1.0
+    np.testing.assert_allclose(orc.phi(ELU1, x), ref, rtol=1e-15, atol=1e-15)
+    assert (orc.phi(ELU1, x) > 0).all()
+
+
+@pytest.mark.parametrize("d", [1, 2, 3, 4, 16])
+def test_taylor_kernel_closed_form(orc, d):
+    # BASED page, Knowl 3: phi(q).phi(k) = 1 + q.k + (q.k)^2/2 with the scaling
+    # absorbed into q,k; with 1/d'^(1/4) on each side the kernel is
+    # 1 + q.k/sqrt(d') + (q.k)^2/(2 d')  (for d'=16: 1 + q.k/4 + (q.k)^2/32).
+    q = rnd(2, 50, d, scale=1.5)
+    k = rnd(3, 50, d, scale=1.5)
+    pq, pk = orc.phi(TAYLOR2, q), orc.phi(TAYLOR2, k)
+    s = (q * k).sum(-1)
+    ref = 1 + s / math.sqrt(d) + s * s / (2 * d)
+    np.testing.assert_allclose((pq * pk).sum(-1), ref, rtol=1e-12, atol=1e-12)
+
+
+def test_taylor_kernel_d16_constants(orc):
+    # The d'=16 instance printed with the workload: 1 + q.k/4 + (q.k)^2/32.
+    q = rnd(4, 20, 16); k = rnd(5, 20, 16)
+    s = (q * k).sum(-1)
+    got = (orc.phi(TAYLOR2, q) * orc.phi(TAYLOR2, k)).sum(-1)
+    np.testing.assert_allclose(got, 1 + s / 4 + s * s / 32, rtol=1e-12)
+
+
+def test_taylor_feature_order(orc):
+    # Knowl 3: "a constant term, first-order coordinates, and second-order
+    # pairwise products"; the second-order block is row-major in (a, b).
+    d = 5
+    t, u, a, b = 0.7, -1.3, 1, 3
+    x = np.zeros(d); x[a] = t; x[b] = u
+    p = orc.phi(TAYLOR2, x[None])[0]
+    exp = np.zeros(1 + d + d * d)
+    exp[0] = 1.0
+    exp[1 + a] = t / d ** 0.25
+    exp[1 + b] = u / d ** 0.25
+    c2 = math.sqrt(2) * math.sqrt(d)
+    exp[1 + d + a * d + a] = t * t / c2
+    exp[1 + d + b * d + b] = u * u / c2
+    exp[1 + d + a * d + b] = t * u / c2
+    exp[1 + d + b * d + a] = t * u / c2
+    np.testing.assert_allclose(p, exp, rtol=1e-15, atol=1e-16)
+
+
+@pytest.mark.parametrize("fmap", [ELU1, TAYLOR2])
+def test_phi_vjp_finite_difference(orc, fmap):
+    d = 4
+    x = rnd(6, d)
+    F = orc.feature_dim(fmap, d)
+    w = rnd(7, F)
+    got = orc.phi_vjp(fmap, x[None], w[None])[0]
+    h = 1e-6
+    fd = np.empty(d)
+    for a in range(d):
+        xp = x.copy(); xp[a] += h
+        xm = x.copy(); xm[a] -= h
+        fd[a] = ((orc.phi(fmap, xp[None])[0] - orc.phi(fmap, xm[None])[0]) @ w) / (2 * h)
+    np.testing.assert_allclose(got, fd, rtol=1e-7, atol=1e-9)
+
+
+# ----------------------------------------------------------------- forward
+
+@pytest.mark.parametrize("fmap", [ELU1, TAYLOR2])
+def test_first_output_is_first_value(orc, fmap):
+    # The causal sum includes j = i (Knowl 3, sum from j = 1 to i), so the
+    # first output is v_1 exactly, whatever q and k are.
+    q = rnd(8, 2, 3, 1, 4); k = rnd(9, 2, 3, 1, 4); v = rnd(10, 2, 3, 1, 6)
+    o, den = orc.forward_brute(fmap, q, k, v)
+    np.testing.assert_allclose(o, v, rtol=1e-14)
+    o2, _, _, _ = orc.forward_recurrent(fmap, q, k, v)
+    np.testing.assert_allclose(o2, v, rtol=1e-14)
+
+
+def test_two_tokens_one_dim_closed_form(orc):
+    # N=2, D=1, elu+1: q_2 cancels; y_2 = (phi(k1) v1 + phi(k2) v2)/(phi(k1)+phi(k2)).
+    q = np.array([0.3, -2.0]).reshape(1, 1, 2, 1)
+    k = np.array([0.5, -1.0]).reshape(1, 1, 2, 1)
+    v = np.array([2.0, -1.0]).reshape(1, 1, 2, 1)
+    o, den = orc.forward_brute(ELU1, q, k, v)
+    p1, p2 = 1.5, math.exp(-1.0)
+    assert o[0, 0, 0, 0] == pytest.approx(2.0, rel=1e-15)
+    assert o[0, 0, 1, 0] == pytest.approx((p1 * 2.0 + p2 * -1.0) / (p1 + p2), rel=1e-14)
+    # den_2 = phi(q2) (phi(k1) + phi(k2)) with phi(q2) = exp(-2)
+    assert den[0, 0, 1] == pytest.approx(math.exp(-2.0) * (p1 + p2), rel=1e-14)
+
+
+def test_taylor_zero_query_is_running_mean(orc):
+    # With q = 0, phi(q).phi(k) = 1 for every k: y_i = mean(v_1..v_i).
+    N = 40
+    q = np.zeros((1, 2, N, 16)); k = rnd(11, 1, 2, N, 16); v = rnd(12, 1, 2, N, 8)
+    o, den = orc.forward_brute(TAYLOR2, q, k, v)
+    ref = np.cumsum(v, axis=2) / np.arange(1, N + 1)[None, None, :, None]
+    np.testing.assert_allclose(o, ref, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(den, np.broadcast_to(np.arange(1, N + 1), den.shape), rtol=1e-14)
+
+
+def test_elu_equal_keys_is_running_mean(orc):
+    # All keys equal: every weight a_ij is the same, so y_i = mean(v_1..v_i).
+    N = 33
+    q = rnd(13, 1, 1, N, 8); k = np.broadcast_to(rnd(14, 8), (1, 1, N, 8)).copy(); v = rnd(15, 1, 1, N, 5)
+    o, _ = orc.forward_brute(ELU1, q, k, v)
+    ref = np.cumsum(v, axis=2) / np.arange(1, N + 1)[None, None, :, None]
+    np.testing.assert_allclose(o, ref, rtol=1e-12, atol=1e-13)
+
+
+def test_taylor_approximates_causal_softmax(orc):
+    # The Taylor kernel is the second-order expansion of exp(q.k/sqrt(d'))
+    # (Knowl 3), so for small logits the output must match causal softmax
+    # attention (torch's scaled_dot_product_attention, a library routine) to
+    # within the third-order remainder: per weight the relative error is at
+    # most delta = s^3/6 * e^{2|s|}, which moves y by <= 2 delta/(1-delta) max|v|.
+    d, N = 16, 64
+    q = rnd(16, 1, 2, N, d, scale=0.12); k = rnd(17, 1, 2, N, d, scale=0.12); v = rnd(18, 1, 2, N, 8)
+    s = np.einsum("bhid,bhjd->bhij", q, k) / math.sqrt(d)
+    smax = np.abs(s).max()
+    assert smax < 0.2
+    delta = smax ** 3 / 6 * math.exp(2 * smax)
+    bound = 2 * delta / (1 - delta) * np.abs(v).max()
+    o, _ = orc.forward_brute(TAYLOR2, q, k, v)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q), torch.from_numpy(k), torch.from_numpy(v), is_causal=True,
+        scale=1 / math.sqrt(d)).numpy()
+    err = np.abs(o - ref).max()
+    assert err <= bound, (err, bound)
+    # The bound is tight enough to catch a structural mistake: dropping the
+    # diagonal term moves the outputs by far more than it.
+    assert bound < 1e-3 * np.abs(ref).max()
+
+
+@pytest.mark.parametrize("fmap,d,dv", [(ELU1, 8, 5), (ELU1, 32, 32), (TAYLOR2, 4, 6), (TAYLOR2, 16, 16)])
+def test_brute_equals_recurrent(orc, fmap, d, dv):
+    # The parallel form and the recurrent form of Knowl 3 are the same function.
+    for N in (1, 2, 17, 129):
+        q = rnd(20 + N, 2, 2, N, d, scale=0.7); k = rnd(21 + N, 2, 2, N, d, scale=0.7)
+        v = rnd(22 + N, 2, 2, N, dv)
+        ob, db = orc.forward_brute(fmap, q, k, v)
+        orr, dr, s, z = orc.forward_recurrent(fmap, q, k, v)
+        np.testing.assert_allclose(orr, ob, rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(dr, db, rtol=1e-12)
+        # final state is the plain sum of phi(k_j) v_j^T and of phi(k_j)
+        pk = orc.phi(fmap, k)
+        np.testing.assert_allclose(s, np.einsum("bhnf,bhnc->bhfc", pk, v), rtol=1e-11, atol=1e-11)
+        np.testing.assert_allclose(z, pk.sum(2), rtol=1e-12)
+
+
+def test_recurrent_long_sequence_matches_brute(orc):
+    N = 512
+    q = rnd(30, 1, 1, N, 16); k = rnd(31, 1, 1, N, 16); v = rnd(32, 1, 1, N, 8)
+    ob, _ = orc.forward_brute(TAYLOR2, q, k, v)
+    orr, _, _, _ = orc.forward_recurrent(TAYLOR2, q, k, v)
+    np.testing.assert_allclose(orr, ob, rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("fmap", [ELU1, TAYLOR2])
+def test_denominator_positivity(orc, fmap):
+    # elu+1 features are all > 0, so den_i > 0.  Taylor: 1+s+s^2/2 =
+    # ((1+s)^2+1)/2 >= 1/2, so den_i >= i/2 (1-based i).
+    N = 200
+    q = rnd(33, 1, 2, N, 16, scale=2.0); k = rnd(34, 1, 2, N, 16, scale=2.0); v = rnd(35, 1, 2, N, 4)
+    _, den = orc.forward_brute(fmap, q, k, v)
+    assert (den > 0).all()
+    if fmap == TAYLOR2:
+        assert (den >= np.arange(1, N + 1) / 2 - 1e-12).all()
+
+
+def test_forward_rows_matches_brute(orc):
+    N = 100
+    q = rnd(36, 1, 1, N, 16); k = rnd(37, 1, 1, N, 16); v = rnd(38, 1, 1, N, 8)
+    ob, db = orc.forward_brute(TAYLOR2, q, k, v)
+    rows = [0, 5, 63, 64, 99]
+    o, d = orc.forward_rows(TAYLOR2, q[0, 0], k[0, 0], v[0, 0], rows)
+    np.testing.assert_allclose(o, ob[0, 0, rows], rtol=1e-13)
+    np.testing.assert_allclose(d, db[0, 0, rows], rtol=1e-13)
+
+
+@pytest.mark.parametrize("fmap", [ELU1, TAYLOR2])
+def test_forward_from_state_and_decode(orc, fmap):
+    # Knowl 5: the prefill may write its final state for generation; decode
+    # steps from it must continue the same sequence.  Prefill(P) then T steps
+    # == forward over P+T, on the last T outputs and the final state.
+    P, T, d, dv = 23, 9, 16 if fmap == TAYLOR2 else 8, 6
+    q = rnd(40, 2, 3, P + T, d, scale=0.8); k = rnd(41, 2, 3, P + T, d, scale=0.8); v = rnd(42, 2, 3, P + T, dv)
+    ofull, _, sfull, zfull = orc.forward_recurrent(fmap, q, k, v)
+    _, _, s, z = orc.forward_recurrent(fmap, q[:, :, :P], k[:, :, :P], v[:, :, :P])
+    s = np.ascontiguousarray(s); z = np.ascontiguousarray(z)
+    for t in range(T):
+        y = orc.decode_step(fmap, q[:, :, P + t], k[:, :, P + t], v[:, :, P + t], s, z)
+        np.testing.assert_allclose(y, ofull[:, :, P + t], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(s, sfull, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(z, zfull, rtol=1e-12)
+    # starting the recurrent forward from the prefill state gives the same tail
+    _, _, s0, z0 = orc.forward_recurrent(fmap, q[:, :, :P], k[:, :, :P], v[:, :, :P])
+    otail, _, s2, z2 = orc.forward_recurrent(fmap, q[:, :, P:], k[:, :, P:], v[:, :, P:], s0, z0)
+    np.testing.assert_allclose(otail, ofull[:, :, P:], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(s2, sfull, rtol=1e-12, atol=1e-12)
+
+
+# ----------------------------------------------------------------- backward
+
+def _loss_grad_fd(orc, fmap, q, k, v, do, h=1e-6):
+    """Central finite differences of L = sum(dO * y) through the brute forward."""
+    def L(args):
+        o, _ = orc.forward_brute(fmap, *args)
+        return float((o * do).sum())
+    grads = []
+    for pos in range(3):
+        base = [q, k, v]
+        x = base[pos]
+        g = np.zeros_like(x)
+        for idx in np.ndindex(*x.shape):
+            xp = x.copy(); xp[idx] += h
+            xm = x.copy(); xm[idx] -= h
+            ap = list(base); ap[pos] = xp
+            am = list(base); am[pos] = xm
+            g[idx] = (L(ap) - L(am)) / (2 * h)
+        grads.append(g)
+    return grads
+
+
+@pytest.mark.parametrize("fmap,d,dv,N", [(ELU1, 4, 3, 7), (ELU1, 3, 5, 12), (TAYLOR2, 3, 3, 6), (TAYLOR2, 2, 4, 11)])
+def test_backward_finite_differences(orc, fmap, d, dv, N):
+    q = rnd(50, 1, 1, N, d, scale=0.8); k = rnd(51, 1, 1, N, d, scale=0.8)
+    v = rnd(52, 1, 1, N, dv); do = rnd(53, 1, 1, N, dv)
+    dq, dk, dvv = orc.backward_brute(fmap, q, k, v, do)
+    fq, fk, fv = _loss_grad_fd(orc, fmap, q, k, v, do)
+    for got, ref in ((dq, fq), (dk, fk), (dvv, fv)):
+        np.testing.assert_allclose(got, ref, rtol=1e-6, atol=1e-8)
+
+
+@pytest.mark.parametrize("fmap,d,dv", [(ELU1, 8, 6), (ELU1, 16, 16), (TAYLOR2, 4, 5), (TAYLOR2, 16, 8)])
+def test_backward_brute_equals_recurrent(orc, fmap, d, dv):
+    for N in (1, 5, 64, 97):
+        q = rnd(60 + N, 2, 2, N, d, scale=0.6); k = rnd(61 + N, 2, 2, N, d, scale=0.6)
+        v = rnd(62 + N, 2, 2, N, dv); do = rnd(63 + N, 2, 2, N, dv)
+        b = orc.backward_brute(fmap, q, k, v, do)
+        r = orc.backward_recurrent(fmap, q, k, v, do)
+        for x, y in zip(b, r):
+            np.testing.assert_allclose(y, x, rtol=1e-9, atol=1e-11)
+
+
+@pytest.mark.parametrize("fmap", [ELU1, TAYLOR2])
+def test_backward_autograd(orc, fmap):
+    # torch autograd differentiates a plain fp64 torch expression of the
+    # masked form; it checks the hand-derived chain rule, not the forward.
+    d, dv, N = (6, 5, 20) if fmap == ELU1 else (4, 5, 20)
+    q = rnd(70, 1, 2, N, d, scale=0.7); k = rnd(71, 1, 2, N, d, scale=0.7)
+    v = rnd(72, 1, 2, N, dv); do = rnd(73, 1, 2, N, dv)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+
+    def feat(x):
+        if fmap == ELU1:
+            return torch.nn.functional.elu(x) + 1
+        one = torch.ones(*x.shape[:-1], 1, dtype=x.dtype)
+        sec = (x[..., :, None] * x[..., None, :]).flatten(-2) / (math.sqrt(2) * math.sqrt(d))
+        return torch.cat([one, x / d ** 0.25, sec], -1)
+    A = torch.tril(feat(tq) @ feat(tk).transpose(-1, -2))
+    y = (A @ tv) / A.sum(-1, keepdim=True)
+    (y * torch.from_numpy(do)).sum().backward()
+    dq, dk, dvv = orc.backward_recurrent(fmap, q, k, v, do)
+    np.testing.assert_allclose(dq, tq.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dvv, tv.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("fmap", [ELU1, TAYLOR2])
+def test_backward_invariants(orc, fmap):
+    # (a) Each y_i is a convex combination of v_1..v_i (weights sum to 1), so
+    #     adding c to every v shifts every y by c: sum_j dv_j = sum_i dO_i.
+    # (b) Scaling V by alpha scales y by alpha: dq, dk scale by alpha and dv
+    #     does not change.
+    N, d, dv = 50, 16 if fmap == TAYLOR2 else 8, 7
+    q = rnd(80, 1, 2, N, d, scale=0.5); k = rnd(81, 1, 2, N, d, scale=0.5)
+    v = rnd(82, 1, 2, N, dv); do = rnd(83, 1, 2, N, dv)
+    dq, dk, dvv = orc.backward_recurrent(fmap, q, k, v, do)
+    np.testing.assert_allclose(dvv.sum(2), do.sum(2), rtol=1e-10, atol=1e-11)
+    dq2, dk2, dvv2 = orc.backward_recurrent(fmap, q, k, 3.0 * v, do)
+    np.testing.assert_allclose(dq2, 3.0 * dq, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dk2, 3.0 * dk, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dvv2, dvv, rtol=1e-10, atol=1e-12)
+    assert np.abs(dq).max() > 0 and np.abs(dk).max() > 0
+
+
+def test_max_rel_l2_metric(orc):
+    ref = np.ones((2, 3, 4, 5))
+    x = ref.copy(); x[1, 2] *= 1.01
+    assert orc.max_rel_l2(x, ref) == pytest.approx(0.01, rel=1e-12)
