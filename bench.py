@@ -1,0 +1,524 @@
+#!/usr/bin/env python
+"""Throughput benchmark for the B200 causal linear attention library.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-secondary]
+
+One JSON line on stdout (rank 0).  The headline workload is the elu(x)+1 bf16
+chunked prefill, B=4 H=8 N=4096 D=64 (one step = one la_forward over the
+batch); value = prefill tokens/s (B*N per step, all ranks).  The same line
+carries, under "workloads", the BASED Taylor bf16 prefill (B=8 H=16 N=2048
+d'=16), the elu bf16 training step (forward+backward, B=2 H=16 N=16384
+D=128) and the BASED Taylor fp32 decode (256 sequences x 16 heads, 1024
+one-token steps per graph replay), each with its own roofline.
+
+Timing: W untimed warm-up steps, then exactly K steps replayed from a CUDA
+graph, bracketed by a barrier and a device synchronisation, timed with CUDA
+events on the launching stream; the max over ranks is reported.  Inputs that
+fit in L2 rotate through enough copies that every step reads data last
+touched more than L2's capacity ago.  With --gpus N > 1 each rank runs an
+independent replica on its own GPU (the path needs no collective), so
+scaling is weak.
+
+--impl reference times the fp64 CPU oracle on this host's cores on a bounded
+sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------- utilities
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        h.update(open(os.path.join(ROOT, "causal_kernelized_sequence_b200", "csrc", n), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(kernel_key):
+    """DRAM bytes per launch from a committed ncu summary, only if the kernel
+    source is unchanged since the capture (else None)."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(kernel_key)
+    if not d:
+        return None
+    try:
+        if source_hash(*d["sources"]) != d["source_hash"]:
+            return None
+    except OSError:
+        return None
+    return d["bytes_per_launch"]
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    def __init__(self, device_index, period_s=0.005):
+        self.dev = device_index
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.dev)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            return self
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def _run(self):
+        nv = self._nv
+        names = {
+            "hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
+            "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+            "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+            "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4),
+            "hw_power_brake_slowdown": getattr(nv, "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80),
+        }
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for n, bit in names.items():
+                    if mask & bit:
+                        self.reasons.add(n)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *a):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": len(self.samples)}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------- workloads
+
+class Prefill:
+    """One step = la_forward over the whole batch (o only)."""
+
+    def __init__(self, w: W.Workload, dev, seed_offset=0):
+        import causal_kernelized_sequence_b200 as la
+        self.la, self.w, self.dev = la, w, dev
+        g = torch.Generator(device=dev)
+        g.manual_seed(w.index + 1000 * seed_offset)
+        set_bytes = w.B * w.H * w.N * (2 * w.dqk + 2 * w.dv) * 2
+        self.nsets = max(1, math.ceil(2 * L2_BYTES / set_bytes) + 1) if set_bytes < 2 * L2_BYTES else 1
+        mk = lambda d: (torch.randn(w.B, w.H, w.N, d, device=dev, generator=g) * w.scale).to(w.torch_dtype)
+        self.sets = [(mk(w.dqk), mk(w.dqk), mk(w.dv), torch.empty(w.B, w.H, w.N, w.dv, device=dev, dtype=w.torch_dtype))
+                     for _ in range(self.nsets)]
+        self.tokens = w.B * w.N
+        esz = 2 if w.dtype == W.BF16 else 4
+        self.alg_bytes = w.B * w.H * w.N * (2 * w.dqk + 2 * w.dv) * esz
+        F = w.feature_dim
+        self.alg_flops = 4.0 * F * (w.dv + 1) * w.B * w.H * w.N
+        wsb = la.la_forward_workspace_bytes(w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype)
+        self.ws = torch.empty(wsb, dtype=torch.uint8, device=dev) if wsb else None
+
+    def step(self, i):
+        q, k, v, o = self.sets[i % self.nsets]
+        self.la.la_forward(q, k, v, self.w.fmap, out=o, workspace=self.ws)
+
+    def l2_note(self):
+        return (f"{self.nsets} rotating input/output sets of "
+                f"{self.alg_bytes / 1e6:.1f} MB (> 126 MB L2 between reuses)" if self.nsets > 1
+                else f"inputs {self.alg_bytes / 1e6:.0f} MB > 126 MB L2")
+
+
+class Train:
+    """One step = la_forward (o, den) + la_backward (dq, dk, dv)."""
+
+    def __init__(self, w, dev, seed_offset=0):
+        import causal_kernelized_sequence_b200 as la
+        self.la, self.w, self.dev = la, w, dev
+        g = torch.Generator(device=dev)
+        g.manual_seed(w.index + 1000 * seed_offset)
+        mk = lambda d: (torch.randn(w.B, w.H, w.N, d, device=dev, generator=g) * w.scale).to(w.torch_dtype)
+        self.q, self.k, self.v, self.do = mk(w.dqk), mk(w.dqk), mk(w.dv), mk(w.dv)
+        self.o = torch.empty_like(self.v)
+        self.den = torch.empty(w.B, w.H, w.N, device=dev)
+        self.dq, self.dk, self.dvv = torch.empty_like(self.q), torch.empty_like(self.k), torch.empty_like(self.v)
+        self.tokens = w.B * w.N
+        e = 2
+        BHN = w.B * w.H * w.N
+        self.fwd_bytes = BHN * (2 * w.dqk + 2 * w.dv) * e + BHN * 4
+        self.bwd_bytes = BHN * (2 * w.dqk + 3 * w.dv) * e + BHN * 4 + BHN * (2 * w.dqk + w.dv) * e
+        self.alg_bytes = self.fwd_bytes + self.bwd_bytes
+        F = w.feature_dim
+        self.alg_flops = (4.0 * F * (w.dv + 1) + 10.0 * F * w.dv + 6.0 * F) * BHN
+
+    def step(self, i):
+        la = self.la
+        w = self.w
+        lib = la.load_library()
+        import ctypes
+        P = lambda t: ctypes.c_void_p(t.data_ptr())
+        st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        r = lib.la_forward(P(self.q), P(self.k), P(self.v), P(self.o), None, None, P(self.den), None, 0,
+                           w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype, st)
+        assert r == 0, r
+        r = lib.la_backward(P(self.q), P(self.k), P(self.v), P(self.o), P(self.do), P(self.den), P(self.dq),
+                            P(self.dk), P(self.dvv), None, 0, w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype, st)
+        assert r == 0, r
+
+    def l2_note(self):
+        return f"inputs {self.alg_bytes / 1e6:.0f} MB > 126 MB L2"
+
+
+class Decode:
+    """One step = 1024 one-token la_decode_step calls (one new token for each
+    of the B*H heads per call), replayed from a CUDA graph as on the BASED
+    page's generation benchmark."""
+
+    def __init__(self, w, dev, seed_offset=0, steps=None):
+        import causal_kernelized_sequence_b200 as la
+        self.la, self.w, self.dev = la, w, dev
+        T = w.decode_steps if steps is None else steps
+        self.T = T
+        g = torch.Generator(device=dev)
+        g.manual_seed(w.index + 1000 * seed_offset)
+        mk = lambda *s: torch.randn(*s, device=dev, generator=g).to(w.torch_dtype)
+        q, k, v = mk(w.B, w.H, w.N, w.dqk), mk(w.B, w.H, w.N, w.dqk), mk(w.B, w.H, w.N, w.dv)
+        r = la.la_forward(q, k, v, w.fmap, state=True)
+        self.s, self.z = r["s"], r["z"]
+        del q, k, v, r
+        self.sq, self.sk, self.sv = mk(T, w.B, w.H, w.dqk), mk(T, w.B, w.H, w.dqk), mk(T, w.B, w.H, w.dv)
+        self.y = torch.empty(T, w.B, w.H, w.dv, device=dev, dtype=w.torch_dtype)
+        self.tokens = w.B * T
+        F = w.feature_dim
+        esz = 4 if w.dtype == W.F32 else 2
+        self.bytes_per_call = w.B * w.H * (2 * (F * w.dv + F) * 4 + (2 * w.dqk + 2 * w.dv) * esz)
+        self.alg_bytes = self.bytes_per_call * T
+        self.alg_flops = 4.0 * F * (w.dv + 1) * w.B * w.H * T
+
+    def step(self, i):
+        for t in range(self.T):
+            self.la.la_decode_step(self.sq[t], self.sk[t], self.sv[t], self.s, self.z, self.w.fmap, y=self.y[t])
+
+    def l2_note(self):
+        return f"state {self.s.numel() * 4 / 1e6:.0f} MB > 126 MB L2"
+
+
+def make_run(w, dev, seed_offset):
+    if w.decode_steps:
+        return Decode(w, dev, seed_offset)
+    if w.backward:
+        return Train(w, dev, seed_offset)
+    return Prefill(w, dev, seed_offset)
+
+
+def capture(run, nsteps, stream):
+    """CUDA graph of `nsteps` consecutive steps."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(nsteps):
+            run.step(i)
+    return g
+
+
+def timed(run, steps, warmup, dist_on, device_index, graph_len=None):
+    """Run warm-up, then exactly `steps` steps from CUDA graphs; returns
+    (ms per step max over ranks, clocks)."""
+    stream = torch.cuda.Stream()
+    # eager warm-up: also configures kernels before any capture
+    with torch.cuda.stream(stream):
+        for i in range(max(1, warmup)):
+            run.step(i)
+    torch.cuda.synchronize()
+    G = graph_len or min(steps, 100)
+    full, rem = divmod(steps, G)
+    g = capture(run, G, stream) if full else None
+    gr = capture(run, rem, stream) if rem else None
+    # graph warm-up
+    for _ in range(max(1, warmup // G)):
+        (g or gr).replay()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(device_index) as clk:
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for _ in range(full):
+                g.replay()
+            if gr is not None:
+                gr.replay()
+            end.record(stream)
+        torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    ms = start.elapsed_time(end)
+    if dist_on:
+        t = torch.tensor([ms], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    del g, gr
+    return ms / steps, clk.summary()
+
+
+def e2e_prefill(w, dev, steps, warmup):
+    """Same metric through the public API with host buffers: pinned host q,k,v
+    copied in and o copied out inside the timed region, every step."""
+    import causal_kernelized_sequence_b200 as la
+    g = torch.Generator()
+    g.manual_seed(w.index)
+    mk = lambda d: (torch.randn(w.B, w.H, w.N, d, generator=g) * w.scale).to(w.torch_dtype).pin_memory()
+    hq, hk, hv = mk(w.dqk), mk(w.dqk), mk(w.dv)
+    ho = torch.empty(w.B, w.H, w.N, w.dv, dtype=w.torch_dtype).pin_memory()
+    dq_, dk_, dv_ = (torch.empty(t.shape, dtype=t.dtype, device=dev) for t in (hq, hk, hv))
+    do_ = torch.empty(ho.shape, dtype=ho.dtype, device=dev)
+    stream = torch.cuda.Stream()
+
+    def one():
+        dq_.copy_(hq, non_blocking=True)
+        dk_.copy_(hk, non_blocking=True)
+        dv_.copy_(hv, non_blocking=True)
+        la.la_forward(dq_, dk_, dv_, w.fmap, out=do_)
+        ho.copy_(do_, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, warmup)):
+            one()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        s.record(stream)
+        for _ in range(steps):
+            one()
+        e.record(stream)
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = ho.numel() * ho.element_size()
+    return ms, h2d, d2h
+
+
+# ----------------------------------------------------------------- CPU oracle
+
+def oracle_sample(w, heads=None, positions=None):
+    """Time the fp64 oracle on a bounded sample of workload w; returns
+    (tokens/s extrapolated to the full workload, seconds, description)."""
+    from oracle import oracle as orc
+    orc.build()
+    Hs = w.B * w.H if heads is None else heads
+    Ns = w.N if positions is None else positions
+    g = torch.Generator()
+    g.manual_seed(w.index)
+    mk = lambda d: (torch.randn(1, Hs, Ns, d, generator=g) * w.scale).to(w.torch_dtype)
+    q, k, v = mk(w.dqk), mk(w.dqk), mk(w.dv)
+    t0 = time.perf_counter()
+    if w.backward:
+        do = mk(w.dv)
+        orc.forward_recurrent(w.fmap, q, k, v)
+        orc.backward_recurrent(w.fmap, q, k, v, do)
+    elif w.decode_steps:
+        F = w.feature_dim
+        import numpy as np
+        s = np.zeros((Hs, F, w.dv)); z = np.zeros((Hs, F))
+        for t in range(Ns):
+            orc.decode_step(w.fmap, q[0, :, t], k[0, :, t], v[0, :, t], s, z)
+    else:
+        orc.forward_recurrent(w.fmap, q, k, v)
+    dt = time.perf_counter() - t0
+    frac = (Hs * Ns) / (w.B * w.H * (w.decode_steps if w.decode_steps else w.N))
+    full_tokens = w.B * (w.decode_steps if w.decode_steps else w.N)
+    desc = (f"fp64 oracle ({'decode steps' if w.decode_steps else 'recurrent form'}"
+            f"{' + backward' if w.backward else ''}) on {Hs} of {w.B * w.H} heads x {Ns} positions; "
+            f"tokens/s scaled to the full workload by head-token count")
+    return full_tokens * frac / dt, dt, desc
+
+
+def omp_threads():
+    try:
+        return int(os.environ.get("OMP_NUM_THREADS", "")) or os.cpu_count()
+    except ValueError:
+        return os.cpu_count()
+
+
+# ----------------------------------------------------------------- main
+
+def roofline_entry(bound, achieved, peak, unit, traffic):
+    return {"bound": bound, "achieved": round(achieved, 1), "peak": peak, "unit": unit,
+            "frac": round(achieved / peak, 4), "traffic": traffic}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = W.BY_NAME[args.workload]
+    # each step: a bounded sample (8 heads x 256 positions) of the workload
+    heads, pos = min(8, w.B * w.H), min(256, w.N)
+    vals = []
+    total = 0.0
+    for i in range(args.warmup + args.steps):
+        v, dt, desc = oracle_sample(w, heads=heads, positions=pos)
+        if i >= args.warmup:
+            vals.append(v)
+            total += dt
+    value = statistics.median(vals)
+    ms = total / max(1, args.steps) * 1e3
+    line = {
+        "impl": "reference", "metric": "prefill tokens/s", "value": round(value, 2), "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": w.describe()},
+        "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": omp_threads(),
+                         "kind": "oracle", "sample": desc + " per step"},
+        "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="elu_bf16_fwd", choices=list(W.BY_NAME))
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    if args.impl == "reference":
+        return run_reference(args)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist_on = world > 1
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if dist_on:
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+
+    import causal_kernelized_sequence_b200 as la
+    la.load_library()
+    peaks, peak_kind = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+
+    w = W.BY_NAME[args.workload]
+    run = make_run(w, dev, rank)
+    ms, clocks = timed(run, args.steps, args.warmup, dist_on, local)
+    value = run.tokens * world / (ms * 1e-3)
+    kern_ms = ms  # one library launch per step for the prefill workloads
+    achieved = run.alg_bytes / (kern_ms * 1e-3) / 1e9
+    line = {
+        "metric": "prefill tokens/s" if not w.decode_steps else "decode tokens/s",
+        "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 6), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == W.BF16 else "f32", "data": "synthetic",
+        "config": {"workload": w.describe(), "parallelism": f"replicas{world}",
+                   "l2": run.l2_note(), "timing": "CUDA graph of consecutive steps, CUDA events"},
+        "roofline": dict(roofline_entry("hbm", achieved, hbm, "GB/s",
+                                        load_traffic("forward:" + w.name)),
+                         peak_source=peak_kind, alg_bytes_per_launch=run.alg_bytes),
+        "clocks": clocks,
+        "gpu_launches": None,
+    }
+    # e2e through the public API with host buffers
+    if not w.decode_steps and not w.backward:
+        e_ms, h2d, d2h = e2e_prefill(w, dev, min(args.steps, 50), 3)
+        line["e2e"] = {"value": round(run.tokens * world / (e_ms * 1e-3), 1), "unit": "tokens/s",
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    from causal_kernelized_sequence_b200 import kernel_plan
+    kp = kernel_plan(w)
+    line["gpu_launches"] = kp["launches_per_step"] * args.steps
+    line["kernels"] = kp["kernels"]
+
+    if not args.no_secondary and world == 1:
+        sec = {}
+        for name in ("taylor_bf16_fwd", "elu_bf16_train", "taylor_decode"):
+            ws = W.BY_NAME[name]
+            r2 = make_run(ws, dev, 0)
+            st = 3 if ws.decode_steps else 50
+            ms2, clk2 = timed(r2, st, 3, False, local, graph_len=1 if ws.decode_steps else None)
+            v2 = r2.tokens / (ms2 * 1e-3)
+            ach = r2.alg_bytes / (ms2 * 1e-3) / 1e9
+            kp2 = kernel_plan(ws)
+            sec[name] = {"metric": "decode tokens/s" if ws.decode_steps else
+                         ("training tokens/s" if ws.backward else "prefill tokens/s"),
+                         "value": round(v2, 1), "unit": "tokens/s", "ms_per_step": round(ms2, 4),
+                         "steps": st, "config": ws.describe(), "l2": r2.l2_note(),
+                         "roofline": dict(roofline_entry("hbm", ach, hbm, "GB/s",
+                                                         load_traffic("step:" + name)),
+                                          alg_bytes_per_step=r2.alg_bytes,
+                                          tc_frac_alg=round(r2.alg_flops / (ms2 * 1e-3) / 1e12 /
+                                                            float(peaks["bf16_tflops"]), 4)),
+                         "clocks": clk2, "gpu_launches": kp2["launches_per_step"] * st,
+                         "kernels": kp2["kernels"]}
+            del r2
+            torch.cuda.empty_cache()
+        line["workloads"] = sec
+
+    if rank == 0 and world == 1 and not args.no_cpu:
+        v, dt, desc = oracle_sample(w)
+        line["cpu_baseline"] = {"value": round(v, 1), "unit": "tokens/s", "cores": omp_threads(),
+                                "kind": "oracle", "sample": desc + f" ({dt:.1f} s)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist_on:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

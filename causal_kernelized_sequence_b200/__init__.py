@@ -1,0 +1,215 @@
+"""B200 causal linear attention: Python binding of the C-ABI library libla.so.
+
+This module only marshals arguments: it checks shapes and dtypes of torch
+CUDA tensors, passes their device pointers, sizes and the current CUDA stream
+to the C entry points declared in ``include/la.h``, and raises on a non-OK
+status.  Every step of the computation runs in the library's CUDA kernels;
+there is no CPU or PyTorch fallback, and importing the compute functions fails
+loudly when the library has not been built.
+
+Entry points (same names as the C ABI):
+    la_forward(q, k, v, fmap, *, state=False, den=False, out=None) -> dict
+    la_backward(q, k, v, o, dout, den, fmap) -> (dq, dk, dv)
+    la_decode_step(q, k, v, s, z, fmap, y=None) -> y        (s, z in place)
+    la_feature_map(x, fmap) -> phi
+    la_feature_dim(fmap, dqk) -> int
+    la_get_device_status() -> None (raises on a recorded device error)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+LA_FMAP_ELU1 = 0
+LA_FMAP_TAYLOR2 = 1
+LA_F32 = 0
+LA_BF16 = 1
+
+STATUS_NAMES = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED", 3: "LA_ERR_CUDA",
+                4: "LA_ERR_TIMEOUT", 5: "LA_ERR_DEVICE_CHECK"}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_build", "libla.so")
+_lib = None
+
+
+class LAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+
+
+def load_library(path: str | None = None):
+    """Load libla.so (built by ``causal_kernelized_sequence_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = path or LIB_PATH
+    if not os.path.exists(path):
+        raise ImportError(f"libla.so not built ({path}); run python -m causal_kernelized_sequence_b200.build")
+    lib = ctypes.CDLL(path)
+    vp, sz, i, i64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_int64
+    lib.la_version.restype = i
+    lib.la_status_string.argtypes = [i]
+    lib.la_status_string.restype = ctypes.c_char_p
+    lib.la_feature_dim.argtypes = [i, i]
+    lib.la_feature_dim.restype = i64
+    lib.la_forward_workspace_bytes.argtypes = [i] * 7
+    lib.la_forward_workspace_bytes.restype = sz
+    lib.la_backward_workspace_bytes.argtypes = [i] * 7
+    lib.la_backward_workspace_bytes.restype = sz
+    lib.la_forward.argtypes = [vp] * 8 + [sz] + [i] * 7 + [vp]
+    lib.la_forward.restype = i
+    lib.la_backward.argtypes = [vp] * 10 + [sz] + [i] * 7 + [vp]
+    lib.la_backward.restype = i
+    lib.la_decode_step.argtypes = [vp] * 6 + [i] * 6 + [vp]
+    lib.la_decode_step.restype = i
+    lib.la_feature_map.argtypes = [vp, vp, i64, i, i, i, vp]
+    lib.la_feature_map.restype = i
+    lib.la_get_device_status.argtypes = [vp]
+    lib.la_get_device_status.restype = i
+    lib.la_kernel_plan.argtypes = [i] * 8 + [ctypes.c_char_p, sz]
+    lib.la_kernel_plan.restype = i
+    _lib = lib
+    return lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return LA_F32
+    if t.dtype == torch.bfloat16:
+        return LA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise LAError(status, where)
+
+
+def _dev(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def la_feature_dim(fmap: int, dqk: int) -> int:
+    return int(load_library().la_feature_dim(fmap, dqk))
+
+
+def la_forward_workspace_bytes(B, H, N, dqk, dv, fmap, dtype) -> int:
+    return int(load_library().la_forward_workspace_bytes(B, H, N, dqk, dv, fmap, dtype))
+
+
+def la_backward_workspace_bytes(B, H, N, dqk, dv, fmap, dtype) -> int:
+    return int(load_library().la_backward_workspace_bytes(B, H, N, dqk, dv, fmap, dtype))
+
+
+def la_forward(q, k, v, fmap, *, state=False, den=False, out=None, workspace=None):
+    """Causal linear attention forward.  q, k [B,H,N,dqk]; v [B,H,N,dv].
+
+    Returns {"o": [B,H,N,dv], and if requested "s": [B,H,F,dv] fp32,
+    "z": [B,H,F] fp32, "den": [B,H,N] fp32}.
+    """
+    lib = load_library()
+    _dev(q, k, v, out)
+    B, H, N, dqk = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q)
+    F = la_feature_dim(fmap, dqk)
+    o = out if out is not None else torch.empty(B, H, N, dv, dtype=q.dtype, device=q.device)
+    res = {"o": o}
+    if state:
+        res["s"] = torch.empty(B, H, F, dv, dtype=torch.float32, device=q.device)
+        res["z"] = torch.empty(B, H, F, dtype=torch.float32, device=q.device)
+    if den:
+        res["den"] = torch.empty(B, H, N, dtype=torch.float32, device=q.device)
+    wsb = la_forward_workspace_bytes(B, H, N, dqk, dv, fmap, dt)
+    if workspace is None and wsb:
+        workspace = torch.empty(wsb, dtype=torch.uint8, device=q.device)
+    _check(lib.la_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(res.get("s")), _ptr(res.get("z")),
+                          _ptr(res.get("den")), _ptr(workspace), wsb, B, H, N, dqk, dv, fmap, dt,
+                          _stream()), "la_forward")
+    return res
+
+
+def la_backward(q, k, v, o, dout, den, fmap, *, workspace=None):
+    """Gradients (dq, dk, dv) of the forward for upstream gradient dout."""
+    lib = load_library()
+    _dev(q, k, v, o, dout, den)
+    B, H, N, dqk = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q)
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dvv = torch.empty_like(v)
+    wsb = la_backward_workspace_bytes(B, H, N, dqk, dv, fmap, dt)
+    if workspace is None and wsb:
+        workspace = torch.empty(wsb, dtype=torch.uint8, device=q.device)
+    _check(lib.la_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(den), _ptr(dq),
+                           _ptr(dk), _ptr(dvv), _ptr(workspace), wsb, B, H, N, dqk, dv, fmap, dt,
+                           _stream()), "la_backward")
+    return dq, dk, dvv
+
+
+def la_decode_step(q, k, v, s, z, fmap, y=None):
+    """One recurrent step: q, k [B,H,dqk]; v [B,H,dv]; s [B,H,F,dv] and
+    z [B,H,F] fp32 updated in place.  Returns y [B,H,dv]."""
+    lib = load_library()
+    _dev(q, k, v, s, z, y)
+    B, H, dqk = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q)
+    if y is None:
+        y = torch.empty(B, H, dv, dtype=q.dtype, device=q.device)
+    _check(lib.la_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(y), _ptr(s), _ptr(z), B, H, dqk, dv,
+                              fmap, dt, _stream()), "la_decode_step")
+    return y
+
+
+def la_feature_map(x, fmap):
+    """Materialise phi(x) for x [..., dqk] -> [..., F] (test/baseline helper)."""
+    lib = load_library()
+    _dev(x)
+    dqk = x.shape[-1]
+    F = la_feature_dim(fmap, dqk)
+    out = torch.empty(*x.shape[:-1], F, dtype=x.dtype, device=x.device)
+    rows = x.numel() // dqk
+    _check(lib.la_feature_map(_ptr(x), _ptr(out), rows, dqk, fmap, _dtype_code(x), _stream()),
+           "la_feature_map")
+    return out
+
+
+def la_kernel_plan(op: int, B, H, N, dqk, dv, fmap, dtype):
+    """(number of kernel launches, [kernel names]) a call would make."""
+    buf = ctypes.create_string_buffer(512)
+    n = load_library().la_kernel_plan(op, B, H, N, dqk, dv, fmap, dtype, buf, len(buf))
+    return n, [x for x in buf.value.decode().split(",") if x]
+
+
+def kernel_plan(w):
+    """Launches per benchmark step of a workload description (attributes
+    B, H, N, dqk, dv, fmap, dtype, backward, decode_steps)."""
+    if w.decode_steps:
+        n, names = la_kernel_plan(2, w.B, w.H, 1, w.dqk, w.dv, w.fmap, w.dtype)
+        return {"launches_per_step": n * w.decode_steps, "kernels": names}
+    n, names = la_kernel_plan(0, w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype)
+    if w.backward:
+        n2, names2 = la_kernel_plan(1, w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype)
+        n, names = n + n2, names + names2
+    return {"launches_per_step": n, "kernels": names}
+
+
+def la_get_device_status():
+    """Synchronise the current stream and raise if a kernel recorded an error."""
+    _check(load_library().la_get_device_status(_stream()), "la_get_device_status")

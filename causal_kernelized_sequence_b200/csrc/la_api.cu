@@ -1,0 +1,325 @@
+// la_api.cu -- the C ABI of libla (declared in include/la.h): argument
+// validation, kernel selection and launch.  The library is one translation
+// unit: the kernel headers below are included here.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "../../include/la.h"
+#include "la_device.cuh"
+#include "la_simt.cuh"
+
+using namespace la;
+
+namespace {
+
+constexpr size_t kSmemLimit = 227 * 1024;
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+bool valid_enums(int fmap, int dtype)
+{
+    return (fmap == LA_FMAP_ELU1 || fmap == LA_FMAP_TAYLOR2) && (dtype == LA_F32 || dtype == LA_BF16);
+}
+
+// Sizes this build supports (valid but unsupported -> LA_ERR_UNSUPPORTED).
+bool supported_dims(int fmap, int dqk, int dv)
+{
+    if (dv < 1 || dv > 128) return false;
+    if (fmap == LA_FMAP_ELU1) return dqk >= 1 && dqk <= 128;
+    return dqk >= 1 && dqk <= 16;
+}
+
+FmapParams make_fmap(int fmap, int dqk)
+{
+    FmapParams p;
+    p.fmap = fmap;
+    p.dqk = dqk;
+    p.F = (int)la_feature_dim(fmap, dqk);
+    p.inv_c1 = (float)(1.0 / pow((double)dqk, 0.25));
+    p.inv_c2 = (float)(1.0 / (sqrt(2.0) * sqrt((double)dqk)));
+    return p;
+}
+
+// Common shape checks; returns LA_OK or the error to report.
+la_status check_shape(int B, int H, int N, int dqk, int dv, int fmap, int dtype)
+{
+    if (!valid_enums(fmap, dtype)) return LA_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || N < 1 || dqk < 1 || dv < 1) return LA_ERR_INVALID_ARG;
+    const int64_t rows = (int64_t)B * H * N;
+    const int64_t widest = dqk > dv ? dqk : dv;
+    if (rows * widest >= ((int64_t)1 << 31)) return LA_ERR_INVALID_ARG;
+    if (!supported_dims(fmap, dqk, dv)) return LA_ERR_UNSUPPORTED;
+    const int64_t F = la_feature_dim(fmap, dqk);
+    if ((int64_t)B * H * F * dv >= ((int64_t)1 << 31)) return LA_ERR_INVALID_ARG;
+    return LA_OK;
+}
+
+la_status launch_status()
+{
+    return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device) and
+// size; later calls (for example during CUDA-graph capture) make no API call.
+template <auto kernel>
+la_status set_smem(size_t bytes)
+{
+    if (bytes <= 48 * 1024) return LA_OK;
+    static size_t done[64] = {0};  // one table per kernel
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LA_ERR_CUDA;
+    if (done[dev] >= bytes) return LA_OK;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
+        return LA_ERR_CUDA;
+    done[dev] = bytes;
+    return LA_OK;
+}
+
+// Kernel selection, shared by the entry points and la_kernel_plan.
+enum class Path { Invalid, FwdSimt, BwdSimt, DecodeSimt };
+
+Path select_forward(int B, int H, int N, int dqk, int dv, int fmap, int dtype)
+{
+    if (check_shape(B, H, N, dqk, dv, fmap, dtype) != LA_OK) return Path::Invalid;
+    return Path::FwdSimt;
+}
+
+Path select_backward(int B, int H, int N, int dqk, int dv, int fmap, int dtype)
+{
+    if (check_shape(B, H, N, dqk, dv, fmap, dtype) != LA_OK) return Path::Invalid;
+    return Path::BwdSimt;
+}
+
+Path select_decode(int B, int H, int dqk, int dv, int fmap, int dtype)
+{
+    if (check_shape(B, H, 1, dqk, dv, fmap, dtype) != LA_OK) return Path::Invalid;
+    return Path::DecodeSimt;
+}
+
+// Kernel names and launch count of a path.
+int path_kernels(Path p, const char **names)
+{
+    switch (p) {
+    case Path::FwdSimt: names[0] = "fwd_simt_kernel"; return 1;
+    case Path::BwdSimt: names[0] = "bwd_simt_kernel"; return 1;
+    case Path::DecodeSimt: names[0] = "decode_simt_kernel"; return 1;
+    default: return -1;
+    }
+}
+
+// Largest chunk length in {32, 16, 8, 4} whose shared-memory footprint fits.
+template <typename Layout, typename MakeLayout>
+bool pick_chunk(MakeLayout make, int F, int dqk, int dv, Layout *out, size_t *bytes)
+{
+    for (int C = 32; C >= 4; C /= 2) {
+        Layout L = make(C, F, dv);
+        const size_t b = L.floats(F, dqk, dv) * sizeof(float);
+        if (b <= kSmemLimit) {
+            *out = L;
+            *bytes = b;
+            return true;
+        }
+    }
+    return false;
+}
+
+template <typename T>
+la_status forward_simt(const void *q, const void *k, const void *v, void *o, float *s_out,
+                       float *z_out, float *den_out, int B, int H, int N, int dqk, int dv,
+                       int fmap, cudaStream_t stream)
+{
+    const FmapParams fp = make_fmap(fmap, dqk);
+    SimtFwdSmem L;
+    size_t bytes;
+    if (!pick_chunk(simt_fwd_layout, fp.F, dqk, dv, &L, &bytes)) return LA_ERR_UNSUPPORTED;
+    if (set_smem<fwd_simt_kernel<T>>(bytes) != LA_OK) return LA_ERR_CUDA;
+    fwd_simt_kernel<T><<<B * H, kSimtThreads, bytes, stream>>>(
+        (const T *)q, (const T *)k, (const T *)v, (T *)o, s_out, z_out, den_out, N, dv, fp, L);
+    return launch_status();
+}
+
+template <typename T>
+la_status backward_simt(const void *q, const void *k, const void *v, const void *o,
+                        const void *dout, const float *den, void *dq, void *dk, void *dvp,
+                        int B, int H, int N, int dqk, int dv, int fmap, cudaStream_t stream)
+{
+    const FmapParams fp = make_fmap(fmap, dqk);
+    SimtBwdSmem L;
+    size_t bytes;
+    if (!pick_chunk(simt_bwd_layout, fp.F, dqk, dv, &L, &bytes)) return LA_ERR_UNSUPPORTED;
+    if (set_smem<bwd_simt_kernel<T>>(bytes) != LA_OK) return LA_ERR_CUDA;
+    bwd_simt_kernel<T><<<B * H, kSimtThreads, bytes, stream>>>(
+        (const T *)q, (const T *)k, (const T *)v, (const T *)o, (const T *)dout, den, (T *)dq,
+        (T *)dk, (T *)dvp, N, dv, fp, L);
+    return launch_status();
+}
+
+template <typename T>
+la_status decode_simt(const void *q, const void *k, const void *v, void *y, float *s, float *z,
+                      int B, int H, int dqk, int dv, int fmap, cudaStream_t stream)
+{
+    const FmapParams fp = make_fmap(fmap, dqk);
+    const int R = kSimtThreads / dv;
+    const int threads = R * dv;
+    const size_t bytes = sizeof(float) * (2 * (size_t)fp.F + 2 * dqk + dv + (size_t)R * dv + 32);
+    if (set_smem<decode_simt_kernel<T>>(bytes) != LA_OK) return LA_ERR_CUDA;
+    decode_simt_kernel<T><<<B * H, threads, bytes, stream>>>((const T *)q, (const T *)k,
+                                                             (const T *)v, (T *)y, s, z, dv, fp);
+    return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int la_version(void) { return 100; }
+
+const char *la_status_string(int status)
+{
+    switch (status) {
+    case LA_OK: return "LA_OK";
+    case LA_ERR_INVALID_ARG: return "LA_ERR_INVALID_ARG";
+    case LA_ERR_UNSUPPORTED: return "LA_ERR_UNSUPPORTED";
+    case LA_ERR_CUDA: return "LA_ERR_CUDA";
+    case LA_ERR_TIMEOUT: return "LA_ERR_TIMEOUT";
+    case LA_ERR_DEVICE_CHECK: return "LA_ERR_DEVICE_CHECK";
+    default: return "LA_ERR_UNKNOWN";
+    }
+}
+
+int64_t la_feature_dim(int fmap, int dqk)
+{
+    if (dqk < 1) return -1;
+    if (fmap == LA_FMAP_ELU1) return dqk;
+    if (fmap == LA_FMAP_TAYLOR2) return 1 + (int64_t)dqk + (int64_t)dqk * dqk;
+    return -1;
+}
+
+size_t la_forward_workspace_bytes(int B, int H, int N, int dqk, int dv, int fmap, int dtype)
+{
+    if (check_shape(B, H, N, dqk, dv, fmap, dtype) != LA_OK) return 0;
+    return 0;
+}
+
+size_t la_backward_workspace_bytes(int B, int H, int N, int dqk, int dv, int fmap, int dtype)
+{
+    if (check_shape(B, H, N, dqk, dv, fmap, dtype) != LA_OK) return 0;
+    return 0;
+}
+
+la_status la_forward(const void *q, const void *k, const void *v, void *o, float *s_out,
+                     float *z_out, float *den_out, void *workspace, size_t workspace_bytes, int B,
+                     int H, int N, int dqk, int dv, int fmap, int dtype, void *stream)
+{
+    const la_status sh = check_shape(B, H, N, dqk, dv, fmap, dtype);
+    if (sh != LA_OK) return sh;
+    if (!q || !k || !v || !o) return LA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+        !aligned(s_out, 16) || !aligned(z_out, 4) || !aligned(den_out, 4))
+        return LA_ERR_INVALID_ARG;
+    if (workspace_bytes < la_forward_workspace_bytes(B, H, N, dqk, dv, fmap, dtype))
+        return LA_ERR_INVALID_ARG;
+    (void)workspace;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (dtype == LA_F32)
+        return forward_simt<float>(q, k, v, o, s_out, z_out, den_out, B, H, N, dqk, dv, fmap, s);
+    return forward_simt<__nv_bfloat16>(q, k, v, o, s_out, z_out, den_out, B, H, N, dqk, dv, fmap, s);
+}
+
+la_status la_backward(const void *q, const void *k, const void *v, const void *o,
+                      const void *dout, const float *den, void *dq, void *dk, void *dvp,
+                      void *workspace, size_t workspace_bytes, int B, int H, int N, int dqk,
+                      int dv, int fmap, int dtype, void *stream)
+{
+    const la_status sh = check_shape(B, H, N, dqk, dv, fmap, dtype);
+    if (sh != LA_OK) return sh;
+    if (!q || !k || !v || !o || !dout || !den || !dq || !dk || !dvp) return LA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+        !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dvp, 16) ||
+        !aligned(den, 4))
+        return LA_ERR_INVALID_ARG;
+    if (workspace_bytes < la_backward_workspace_bytes(B, H, N, dqk, dv, fmap, dtype))
+        return LA_ERR_INVALID_ARG;
+    (void)workspace;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (dtype == LA_F32)
+        return backward_simt<float>(q, k, v, o, dout, den, dq, dk, dvp, B, H, N, dqk, dv, fmap, s);
+    return backward_simt<__nv_bfloat16>(q, k, v, o, dout, den, dq, dk, dvp, B, H, N, dqk, dv, fmap, s);
+}
+
+la_status la_decode_step(const void *q, const void *k, const void *v, void *y, float *s,
+                         float *z, int B, int H, int dqk, int dv, int fmap, int dtype,
+                         void *stream)
+{
+    const la_status sh = check_shape(B, H, 1, dqk, dv, fmap, dtype);
+    if (sh != LA_OK) return sh;
+    if (!q || !k || !v || !y || !s || !z) return LA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(y, 16) ||
+        !aligned(s, 16) || !aligned(z, 4))
+        return LA_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (dtype == LA_F32) return decode_simt<float>(q, k, v, y, s, z, B, H, dqk, dv, fmap, st);
+    return decode_simt<__nv_bfloat16>(q, k, v, y, s, z, B, H, dqk, dv, fmap, st);
+}
+
+la_status la_feature_map(const void *x, void *phi, int64_t rows, int dqk, int fmap, int dtype,
+                         void *stream)
+{
+    if (!valid_enums(fmap, dtype) || rows < 1 || dqk < 1) return LA_ERR_INVALID_ARG;
+    if (!x || !phi) return LA_ERR_INVALID_ARG;
+    if (!supported_dims(fmap, dqk, 1)) return LA_ERR_UNSUPPORTED;
+    const FmapParams fp = make_fmap(fmap, dqk);
+    if (rows * fp.F >= ((int64_t)1 << 40)) return LA_ERR_INVALID_ARG;
+    const int64_t total = rows * fp.F;
+    const int threads = 256;
+    const int64_t want = (total + threads - 1) / threads;
+    const int blocks = (int)(want < 148 * 16 ? want : 148 * 16);
+    cudaStream_t s = (cudaStream_t)stream;
+    if (dtype == LA_F32)
+        feature_map_kernel<float><<<blocks, threads, 0, s>>>((const float *)x, (float *)phi, rows, fp);
+    else
+        feature_map_kernel<__nv_bfloat16><<<blocks, threads, 0, s>>>(
+            (const __nv_bfloat16 *)x, (__nv_bfloat16 *)phi, rows, fp);
+    return launch_status();
+}
+
+int la_kernel_plan(int op, int B, int H, int N, int dqk, int dv, int fmap, int dtype, char *buf,
+                   size_t buflen)
+{
+    Path p = Path::Invalid;
+    if (op == 0) p = select_forward(B, H, N, dqk, dv, fmap, dtype);
+    else if (op == 1) p = select_backward(B, H, N, dqk, dv, fmap, dtype);
+    else if (op == 2) p = select_decode(B, H, dqk, dv, fmap, dtype);
+    const char *names[8];
+    const int n = path_kernels(p, names);
+    if (buf && buflen) {
+        size_t used = 0;
+        buf[0] = 0;
+        for (int i = 0; i < n; ++i) {
+            const size_t len = strlen(names[i]);
+            if (used + len + (i ? 1 : 0) + 1 > buflen) break;
+            if (i) buf[used++] = ',';
+            memcpy(buf + used, names[i], len);
+            used += len;
+            buf[used] = 0;
+        }
+    }
+    return n;
+}
+
+la_status la_get_device_status(void *stream)
+{
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return LA_ERR_CUDA;
+    unsigned int word = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&word, g_status, sizeof(word)) != cudaSuccess) return LA_ERR_CUDA;
+    if (word && cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return LA_ERR_CUDA;
+    if (word & kStatusTimeout) return LA_ERR_TIMEOUT;
+    if (word & kStatusCheck) return LA_ERR_DEVICE_CHECK;
+    return LA_OK;
+}
+
+}  // extern "C"

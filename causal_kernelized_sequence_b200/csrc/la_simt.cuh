@@ -1,0 +1,396 @@
+// la_simt.cuh -- exact fp32 CUDA-core kernels for every entry point.
+//
+// These kernels compute in fp32 with plain FMA (no tensor cores, no TF32),
+// one thread block per (batch, head) slice, walking the sequence in chunks of
+// C tokens.  They are the path for fp32 I/O (where a 1e-5 relative error
+// rules out bf16/TF32 tensor-core operands) and for the sizes the
+// tensor-core kernels do not cover.  Everything lives in shared memory:
+//
+//   forward  (BASED page, Knowl 3 parallel form, chunked as in Knowl 5):
+//     per chunk, A_ij = phi(q_i).phi(k_j) for j <= i inside the chunk,
+//     num_i = sum_j A_ij v_j + phi(q_i) S,  den_i = sum_j A_ij + phi(q_i).z,
+//     y_i = num_i / den_i, then S += phi(K_c)^T V_c, z += sum_j phi(k_j).
+//   backward (derivative of the same form; see la.h):
+//     forward-order pass for dq, reverse-order pass of R, r for dk, dv.
+//   decode   (Knowl 3 recurrent form): S += phi(k) v^T, z += phi(k),
+//     y = phi(q) S / phi(q).z on the updated state.
+#pragma once
+
+#include "la_device.cuh"
+
+namespace la {
+
+constexpr int kSimtThreads = 256;
+
+// Row strides padded to an odd number of floats so that column walks across
+// a warp hit 32 different banks.
+__host__ __device__ inline int odd_stride(int n) { return n | 1; }
+
+struct SimtFwdSmem {
+    int C, FS, DS;
+    size_t floats(int F, int dqk, int dv) const
+    {
+        return (size_t)F * DS + F + 2 * (size_t)C * dqk + 2 * (size_t)C * FS + (size_t)C * dv +
+               (size_t)C * C + C;
+    }
+};
+
+inline SimtFwdSmem simt_fwd_layout(int C, int F, int dv)
+{
+    return SimtFwdSmem{C, odd_stride(F), odd_stride(dv)};
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kSimtThreads)
+fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+                T *__restrict__ o, float *__restrict__ s_out, float *__restrict__ z_out,
+                float *__restrict__ den_out, int N, int dv, FmapParams fp, SimtFwdSmem L)
+{
+    extern __shared__ float sm[];
+    const int F = fp.F, dqk = fp.dqk, C = L.C, FS = L.FS, DS = L.DS;
+    float *S = sm;                      // [F][DS]
+    float *z = S + (size_t)F * DS;      // [F]
+    float *xq = z + F;                  // [C][dqk]
+    float *xk = xq + C * dqk;           // [C][dqk]
+    float *pq = xk + C * dqk;           // [C][FS]
+    float *pk = pq + (size_t)C * FS;    // [C][FS]
+    float *vs = pk + (size_t)C * FS;    // [C][dv]
+    float *A = vs + C * dv;             // [C][C]
+    float *den = A + C * C;             // [C]
+
+    const int tid = threadIdx.x, nt = blockDim.x;
+    const int lane = tid & 31, warp = tid >> 5, nwarps = nt >> 5;
+    const size_t bh = blockIdx.x;
+    const T *qb = q + bh * N * dqk;
+    const T *kb = k + bh * N * dqk;
+    const T *vb = v + bh * N * dv;
+    T *ob = o + bh * N * dv;
+
+    for (int i = tid; i < F * DS; i += nt) S[i] = 0.f;
+    for (int i = tid; i < F; i += nt) z[i] = 0.f;
+
+    for (int t0 = 0; t0 < N; t0 += C) {
+        const int Lc = min(C, N - t0);
+        __syncthreads();
+        for (int i = tid; i < Lc * dqk; i += nt) {
+            xq[i] = ld(qb + (size_t)t0 * dqk + i);
+            xk[i] = ld(kb + (size_t)t0 * dqk + i);
+        }
+        for (int i = tid; i < Lc * dv; i += nt) vs[i] = ld(vb + (size_t)t0 * dv + i);
+        __syncthreads();
+        for (int idx = tid; idx < Lc * F; idx += nt) {
+            const int i = idx / F, f = idx - i * F;
+            pq[i * FS + f] = phi_feature(fp, xq + i * dqk, f);
+            pk[i * FS + f] = phi_feature(fp, xk + i * dqk, f);
+        }
+        __syncthreads();
+        // Intra-chunk masked weights A_ij, j <= i.
+        for (int idx = tid; idx < Lc * Lc; idx += nt) {
+            const int i = idx / Lc, j = idx - i * Lc;
+            float a = 0.f;
+            if (j <= i)
+                for (int f = 0; f < F; ++f) a = fmaf(pq[i * FS + f], pk[j * FS + f], a);
+            A[i * C + j] = a;
+        }
+        __syncthreads();
+        // den_i = sum_{j<=i} A_ij + phi(q_i).z   (one warp per row)
+        for (int i = warp; i < Lc; i += nwarps) {
+            float acc = 0.f;
+            for (int f = lane; f < F; f += 32) acc = fmaf(pq[i * FS + f], z[f], acc);
+            for (int j = lane; j <= i; j += 32) acc += A[i * C + j];
+            for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+            if (lane == 0) {
+                den[i] = acc;
+                if (den_out) den_out[bh * N + t0 + i] = acc;
+            }
+        }
+        __syncthreads();
+        // num_i = sum_{j<=i} A_ij v_j + phi(q_i) S ; y_i = num_i / den_i
+        for (int idx = tid; idx < Lc * dv; idx += nt) {
+            const int i = idx / dv, c = idx - i * dv;
+            float acc = 0.f;
+            for (int f = 0; f < F; ++f) acc = fmaf(pq[i * FS + f], S[f * DS + c], acc);
+            for (int j = 0; j <= i; ++j) acc = fmaf(A[i * C + j], vs[j * dv + c], acc);
+            st(ob + (size_t)(t0 + i) * dv + c, acc / den[i]);
+        }
+        __syncthreads();
+        // S += phi(K_c)^T V_c ; z += sum_j phi(k_j)
+        for (int idx = tid; idx < F * dv; idx += nt) {
+            const int f = idx / dv, c = idx - f * dv;
+            float acc = S[f * DS + c];
+            for (int j = 0; j < Lc; ++j) acc = fmaf(pk[j * FS + f], vs[j * dv + c], acc);
+            S[f * DS + c] = acc;
+        }
+        for (int f = tid; f < F; f += nt) {
+            float acc = z[f];
+            for (int j = 0; j < Lc; ++j) acc += pk[j * FS + f];
+            z[f] = acc;
+        }
+    }
+    __syncthreads();
+    if (s_out)
+        for (int idx = tid; idx < F * dv; idx += nt) {
+            const int f = idx / dv, c = idx - f * dv;
+            s_out[bh * F * dv + idx] = S[f * DS + c];
+        }
+    if (z_out)
+        for (int f = tid; f < F; f += nt) z_out[bh * F + f] = z[f];
+}
+
+// ------------------------------------------------------------------ backward
+
+struct SimtBwdSmem {
+    int C, FS, DS;
+    size_t floats(int F, int dqk, int dv) const
+    {
+        return (size_t)F * DS + F + 2 * (size_t)C * dqk + 3 * (size_t)C * FS +
+               2 * (size_t)C * dv + 2 * (size_t)C * C + 2 * (size_t)C;
+    }
+};
+
+inline SimtBwdSmem simt_bwd_layout(int C, int F, int dv)
+{
+    return SimtBwdSmem{C, odd_stride(F), odd_stride(dv)};
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kSimtThreads)
+bwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+                const T *__restrict__ o, const T *__restrict__ dout,
+                const float *__restrict__ den_in, T *__restrict__ dq, T *__restrict__ dk,
+                T *__restrict__ dvo, int N, int dv, FmapParams fp, SimtBwdSmem L)
+{
+    extern __shared__ float sm[];
+    const int F = fp.F, dqk = fp.dqk, C = L.C, FS = L.FS, DS = L.DS;
+    float *St = sm;                     // [F][DS]  S (pass 1) / R (pass 2)
+    float *zt = St + (size_t)F * DS;    // [F]      z (pass 1) / r (pass 2)
+    float *xq = zt + F;                 // [C][dqk]
+    float *xk = xq + C * dqk;           // [C][dqk]
+    float *pq = xk + C * dqk;           // [C][FS]
+    float *pk = pq + (size_t)C * FS;    // [C][FS]
+    float *dphi = pk + (size_t)C * FS;  // [C][FS]
+    float *vs = dphi + (size_t)C * FS;  // [C][dv]
+    float *gs = vs + C * dv;            // [C][dv]   g_i = dout_i / den_i
+    float *A = gs + C * dv;             // [C][C]    a_ij
+    float *dA = A + C * C;              // [C][C]    da_ij
+    float *dd = dA + C * C;             // [C]       dden_i = -g_i . y_i
+    float *dn = dd + C;                 // [C]       den_i
+
+    const int tid = threadIdx.x, nt = blockDim.x;
+    const int lane = tid & 31, warp = tid >> 5, nwarps = nt >> 5;
+    const size_t bh = blockIdx.x;
+    const T *qb = q + bh * N * dqk, *kb = k + bh * N * dqk;
+    const T *vb = v + bh * N * dv, *ob = o + bh * N * dv, *gb = dout + bh * N * dv;
+    const float *denb = den_in + bh * N;
+    T *dqb = dq + bh * N * dqk, *dkb = dk + bh * N * dqk, *dvb = dvo + bh * N * dv;
+
+    const int nchunks = (N + C - 1) / C;
+    for (int pass = 0; pass < 2; ++pass) {
+        __syncthreads();
+        for (int i = tid; i < F * DS; i += nt) St[i] = 0.f;
+        for (int i = tid; i < F; i += nt) zt[i] = 0.f;
+        for (int cc = 0; cc < nchunks; ++cc) {
+            const int chunk = pass == 0 ? cc : nchunks - 1 - cc;
+            const int t0 = chunk * C;
+            const int Lc = min(C, N - t0);
+            __syncthreads();
+            for (int i = tid; i < Lc * dqk; i += nt) {
+                xq[i] = ld(qb + (size_t)t0 * dqk + i);
+                xk[i] = ld(kb + (size_t)t0 * dqk + i);
+            }
+            for (int i = tid; i < Lc; i += nt) dn[i] = denb[t0 + i];
+            __syncthreads();
+            for (int i = tid; i < Lc * dv; i += nt) {
+                const int r = i / dv;
+                vs[i] = ld(vb + (size_t)t0 * dv + i);
+                gs[i] = ld(gb + (size_t)t0 * dv + i) / dn[r];
+            }
+            for (int idx = tid; idx < Lc * F; idx += nt) {
+                const int i = idx / F, f = idx - i * F;
+                pq[i * FS + f] = phi_feature(fp, xq + i * dqk, f);
+                pk[i * FS + f] = phi_feature(fp, xk + i * dqk, f);
+            }
+            __syncthreads();
+            // dden_i = -g_i . y_i   (one warp per row; y_i is the forward output)
+            for (int i = warp; i < Lc; i += nwarps) {
+                float acc = 0.f;
+                for (int c = lane; c < dv; c += 32)
+                    acc = fmaf(gs[i * dv + c], ld(ob + (size_t)(t0 + i) * dv + c), acc);
+                for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+                if (lane == 0) dd[i] = -acc;
+            }
+            __syncthreads();
+            // da_ij = g_i . v_j + dden_i, and (pass 2) a_ij, for j <= i
+            for (int idx = tid; idx < Lc * Lc; idx += nt) {
+                const int i = idx / Lc, j = idx - i * Lc;
+                float da = 0.f, a = 0.f;
+                if (j <= i) {
+                    for (int c = 0; c < dv; ++c) da = fmaf(gs[i * dv + c], vs[j * dv + c], da);
+                    da += dd[i];
+                    if (pass == 1)
+                        for (int f = 0; f < F; ++f) a = fmaf(pq[i * FS + f], pk[j * FS + f], a);
+                }
+                dA[i * C + j] = da;
+                A[i * C + j] = a;
+            }
+            __syncthreads();
+            if (pass == 0) {
+                // dphi(q_i) = sum_{j<=i, chunk} da_ij phi(k_j) + S g_i + z dden_i
+                for (int idx = tid; idx < Lc * F; idx += nt) {
+                    const int i = idx / F, f = idx - i * F;
+                    float acc = zt[f] * dd[i];
+                    for (int c = 0; c < dv; ++c) acc = fmaf(St[f * DS + c], gs[i * dv + c], acc);
+                    for (int j = 0; j <= i; ++j) acc = fmaf(dA[i * C + j], pk[j * FS + f], acc);
+                    dphi[i * FS + f] = acc;
+                }
+                __syncthreads();
+                for (int idx = tid; idx < Lc * dqk; idx += nt) {
+                    const int i = idx / dqk, a = idx - i * dqk;
+                    st(dqb + (size_t)t0 * dqk + idx, phi_vjp_component(fp, xq + i * dqk, dphi + i * FS, a));
+                }
+                // S += phi(K_c)^T V_c ; z += sum_j phi(k_j)
+                for (int idx = tid; idx < F * dv; idx += nt) {
+                    const int f = idx / dv, c = idx - f * dv;
+                    float acc = St[f * DS + c];
+                    for (int j = 0; j < Lc; ++j) acc = fmaf(pk[j * FS + f], vs[j * dv + c], acc);
+                    St[f * DS + c] = acc;
+                }
+                for (int f = tid; f < F; f += nt) {
+                    float acc = zt[f];
+                    for (int j = 0; j < Lc; ++j) acc += pk[j * FS + f];
+                    zt[f] = acc;
+                }
+            } else {
+                // dphi(k_j) = sum_{i>=j, chunk} da_ij phi(q_i) + R v_j + r
+                for (int idx = tid; idx < Lc * F; idx += nt) {
+                    const int j = idx / F, f = idx - j * F;
+                    float acc = zt[f];
+                    for (int c = 0; c < dv; ++c) acc = fmaf(St[f * DS + c], vs[j * dv + c], acc);
+                    for (int i = j; i < Lc; ++i) acc = fmaf(dA[i * C + j], pq[i * FS + f], acc);
+                    dphi[j * FS + f] = acc;
+                }
+                // dv_j = sum_{i>=j, chunk} a_ij g_i + R^T phi(k_j)
+                for (int idx = tid; idx < Lc * dv; idx += nt) {
+                    const int j = idx / dv, c = idx - j * dv;
+                    float acc = 0.f;
+                    for (int f = 0; f < F; ++f) acc = fmaf(St[f * DS + c], pk[j * FS + f], acc);
+                    for (int i = j; i < Lc; ++i) acc = fmaf(A[i * C + j], gs[i * dv + c], acc);
+                    st(dvb + (size_t)t0 * dv + idx, acc);
+                }
+                __syncthreads();
+                for (int idx = tid; idx < Lc * dqk; idx += nt) {
+                    const int j = idx / dqk, a = idx - j * dqk;
+                    st(dkb + (size_t)t0 * dqk + idx, phi_vjp_component(fp, xk + j * dqk, dphi + j * FS, a));
+                }
+                // R += sum_i phi(q_i) g_i^T ; r += sum_i phi(q_i) dden_i
+                for (int idx = tid; idx < F * dv; idx += nt) {
+                    const int f = idx / dv, c = idx - f * dv;
+                    float acc = St[f * DS + c];
+                    for (int i = 0; i < Lc; ++i) acc = fmaf(pq[i * FS + f], gs[i * dv + c], acc);
+                    St[f * DS + c] = acc;
+                }
+                for (int f = tid; f < F; f += nt) {
+                    float acc = zt[f];
+                    for (int i = 0; i < Lc; ++i) acc = fmaf(pq[i * FS + f], dd[i], acc);
+                    zt[f] = acc;
+                }
+            }
+        }
+    }
+}
+
+// -------------------------------------------------------------------- decode
+
+// One block per head; blockDim = dv * R threads, thread (r, c) owns column c
+// of the state rows f = r, r + R, ...
+template <typename T>
+__global__ void __launch_bounds__(kSimtThreads)
+decode_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+                   T *__restrict__ y, float *__restrict__ S, float *__restrict__ z, int dv,
+                   FmapParams fp)
+{
+    extern __shared__ float sm[];
+    const int F = fp.F, dqk = fp.dqk;
+    const int tid = threadIdx.x, nt = blockDim.x;
+    const int R = nt / dv;
+    float *pq = sm;            // [F]
+    float *pk = pq + F;        // [F]
+    float *xq = pk + F;        // [dqk]
+    float *xk = xq + dqk;      // [dqk]
+    float *vv = xk + dqk;      // [dv]
+    float *red = vv + dv;      // [R][dv]
+    float *wred = red + R * dv;  // [32]
+    const size_t bh = blockIdx.x;
+
+    for (int i = tid; i < dqk; i += nt) {
+        xq[i] = ld(q + bh * dqk + i);
+        xk[i] = ld(k + bh * dqk + i);
+    }
+    for (int i = tid; i < dv; i += nt) vv[i] = ld(v + bh * dv + i);
+    __syncthreads();
+    for (int f = tid; f < F; f += nt) {
+        pq[f] = phi_feature(fp, xq, f);
+        pk[f] = phi_feature(fp, xk, f);
+    }
+    __syncthreads();
+    float *Sb = S + bh * F * dv;
+    float *zb = z + bh * F;
+    if (tid < R * dv) {
+        const int r = tid / dv, c = tid - r * dv;
+        const float vc = vv[c];
+        float acc = 0.f;
+        for (int f = r; f < F; f += R) {
+            const float s = fmaf(pk[f], vc, Sb[(size_t)f * dv + c]);
+            Sb[(size_t)f * dv + c] = s;
+            acc = fmaf(pq[f], s, acc);
+        }
+        red[r * dv + c] = acc;
+    }
+    float dacc = 0.f;
+    for (int f = tid; f < F; f += nt) {
+        const float zz = zb[f] + pk[f];
+        zb[f] = zz;
+        dacc = fmaf(pq[f], zz, dacc);
+    }
+    for (int off = 16; off; off >>= 1) dacc += __shfl_xor_sync(0xffffffffu, dacc, off);
+    if ((tid & 31) == 0) wred[tid >> 5] = dacc;
+    __syncthreads();
+    if (tid < dv) {
+        float den = 0.f;
+        for (int w = 0; w < (nt + 31) / 32; ++w) den += wred[w];
+        float num = 0.f;
+        for (int r = 0; r < R; ++r) num += red[r * dv + tid];
+        st(y + bh * dv + tid, num / den);
+    }
+}
+
+// --------------------------------------------------------------- feature map
+
+template <typename T>
+__global__ void feature_map_kernel(const T *__restrict__ x, T *__restrict__ phi, int64_t rows,
+                                   FmapParams fp)
+{
+    const int64_t total = rows * fp.F;
+    for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = idx / fp.F;
+        const int f = (int)(idx - r * fp.F);
+        // Only the coordinates this feature reads are loaded.
+        const T *xr = x + r * fp.dqk;
+        float val;
+        if (fp.fmap == LA_FMAP_ELU1) {
+            val = elu1(ld(xr + f));
+        } else if (f == 0) {
+            val = 1.f;
+        } else if (f <= fp.dqk) {
+            val = ld(xr + f - 1) * fp.inv_c1;
+        } else {
+            const int i2 = f - 1 - fp.dqk;
+            const int a = i2 / fp.dqk, b = i2 - a * fp.dqk;
+            val = ld(xr + a) * ld(xr + b) * fp.inv_c2;
+        }
+        st(phi + idx, val);
+    }
+}
+
+}  // namespace la

@@ -1,0 +1,180 @@
+/*
+ * la.h -- C ABI of the B200 causal linear attention library (libla.so).
+ *
+ * Causal linear attention, for every batch b and head h independently:
+ *
+ *     y_i = phi(q_i) S_i / (phi(q_i) . z_i),
+ *     S_i = sum_{j<=i} phi(k_j) v_j^T   [F x Dv],   z_i = sum_{j<=i} phi(k_j)   [F]
+ *
+ * ("Simple linear attention language models balance the recall-throughput
+ * tradeoff", Knowl 3: the masked parallel form for y_i and the recurrent
+ * updates of s_i and z_i; "Transformers are RNNs", abstract: the
+ * associativity that makes the cost linear in N.)  The sum includes j = i and
+ * the denominator has no epsilon.
+ *
+ * Feature maps (phi : R^dqk -> R^F):
+ *   LA_FMAP_ELU1    phi(x)_a = x_a + 1 if x_a > 0 else exp(x_a); F = dqk
+ *                   (the elu(x)+1 map of "Transformers are RNNs", alpha = 1).
+ *   LA_FMAP_TAYLOR2 phi(x) = [1 | x / dqk^(1/4) | x_a x_b / (sqrt(2) sqrt(dqk))],
+ *                   second block row-major in (a, b); F = 1 + dqk + dqk^2.
+ *                   phi(q).phi(k) = 1 + q.k/sqrt(dqk) + (q.k)^2/(2 dqk)
+ *                   (BASED page, Knowl 3, second-order Taylor map with the
+ *                   scaling inside phi; 273 features for dqk = 16, Knowl 5).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *    never allocates or frees device memory and never synchronises, except
+ *    la_get_device_status.  Work is enqueued on `stream` (a cudaStream_t,
+ *    passed as void*; NULL is the legacy default stream) and runs
+ *    asynchronously.
+ *  - Layouts are dense row-major: q, k [B,H,N,dqk]; v, o [B,H,N,dv];
+ *    gradients like their primal; den [B,H,N] fp32; state S [B,H,F,dv] fp32
+ *    and z [B,H,F] fp32 with the feature order above and no padding.
+ *  - dtype selects the element type of q, k, v, o, dout, dq, dk, dv and of the
+ *    decode q, k, v, y: LA_F32 (float) or LA_BF16 (bfloat16).  State, den and
+ *    all accumulation are fp32.
+ *  - Pointers must be 16-byte aligned (z and den need only 4-byte alignment).
+ *  - Argument errors are returned synchronously, before anything is launched:
+ *    LA_ERR_INVALID_ARG (null required pointer, non-positive size, overflow,
+ *    misalignment, workspace too small) or LA_ERR_UNSUPPORTED (a valid
+ *    combination this build has no kernel for).  A failed launch returns
+ *    LA_ERR_CUDA.  Errors detected on the device (a bounded wait that ran out,
+ *    a failed device-side check) are recorded in a per-device status word and
+ *    reported by la_get_device_status.
+ *  - Results are deterministic: the same call on the same inputs gives the
+ *    same bits.
+ *  - Supported sizes: dqk in [1,128] for ELU1 and [1,16] for TAYLOR2;
+ *    dv in [1,128]; N >= 1; B*H*N*max(dqk,dv) < 2^31 elements.  The fast
+ *    tensor-core paths cover bf16 with (ELU1, dqk = dv in {64,128}) and
+ *    (TAYLOR2, dqk = 16, dv = 64); other valid combinations run on exact fp32
+ *    CUDA-core kernels.
+ */
+#ifndef LA_H
+#define LA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LA_API __attribute__((visibility("default")))
+#else
+#define LA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { LA_FMAP_ELU1 = 0, LA_FMAP_TAYLOR2 = 1 } la_fmap;
+typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
+typedef enum {
+    LA_OK = 0,
+    LA_ERR_INVALID_ARG = 1,
+    LA_ERR_UNSUPPORTED = 2,
+    LA_ERR_CUDA = 3,
+    LA_ERR_TIMEOUT = 4,      /* a bounded device-side wait ran out          */
+    LA_ERR_DEVICE_CHECK = 5  /* a device-side bounds/consistency check failed */
+} la_status;
+
+/* Library version as 10000*major + 100*minor + patch. */
+LA_API int la_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+LA_API const char *la_status_string(int status);
+
+/* Feature dimension F of a feature map: dqk for ELU1, 1 + dqk + dqk^2 for
+ * TAYLOR2 (BASED page, Knowl 5: 273 for dqk = 16).  Returns -1 for an
+ * unknown map or dqk < 1. */
+LA_API int64_t la_feature_dim(int fmap, int dqk);
+
+/* Bytes of device workspace la_forward needs for these sizes (0 if none).
+ * The workspace holds per-segment partial states and hand-off flags when a
+ * sequence is split across thread blocks.  The caller allocates it; its
+ * contents need not be initialised (la_forward clears what it uses, on
+ * `stream`).  Returns 0 also for invalid arguments. */
+LA_API size_t la_forward_workspace_bytes(int B, int H, int N, int dqk, int dv, int fmap, int dtype);
+
+/* Bytes of device workspace la_backward needs (0 if none); same rules. */
+LA_API size_t la_backward_workspace_bytes(int B, int H, int N, int dqk, int dv, int fmap, int dtype);
+
+/* Causal linear attention forward (prefill / training forward).
+ * BASED page, Knowl 3 (parallel form for y_i) computed chunk by chunk as in
+ * Knowl 5 (a masked quadratic term inside each chunk plus the product with
+ * the state accumulated over earlier chunks), starting from a zero state.
+ *   q, k      [B,H,N,dqk] dtype, read
+ *   v         [B,H,N,dv]  dtype, read
+ *   o         [B,H,N,dv]  dtype, written (y_i, rounded to nearest even for bf16)
+ *   s_out     [B,H,F,dv]  fp32, nullable: final state S_N (Knowl 5: the
+ *             prefill may write its final state for generation)
+ *   z_out     [B,H,F]     fp32, nullable: final z_N
+ *   den_out   [B,H,N]     fp32, nullable: den_i = phi(q_i).z_i (needed by
+ *             la_backward)
+ *   workspace, workspace_bytes: at least la_forward_workspace_bytes(...)
+ *             bytes of device memory (may be NULL when that is 0).
+ * Outputs must not overlap inputs. */
+LA_API la_status la_forward(const void *q, const void *k, const void *v, void *o,
+                     float *s_out, float *z_out, float *den_out,
+                     void *workspace, size_t workspace_bytes,
+                     int B, int H, int N, int dqk, int dv, int fmap, int dtype,
+                     void *stream);
+
+/* Gradients of the forward with respect to q, k and v for an upstream
+ * gradient dout.  The pages give no backward pass; this is the derivative
+ * of the Knowl 3 parallel form: with g_i = dout_i / den_i and
+ * dden_i = -g_i . o_i, a forward-order scan of (S, z) gives
+ * dphi(q_i) = S_i g_i + z_i dden_i, and a reverse-order scan of
+ * R_j = sum_{i>=j} phi(q_i) g_i^T, r_j = sum_{i>=j} phi(q_i) dden_i gives
+ * dphi(k_j) = R_j v_j + r_j and dv_j = R_j^T phi(k_j); dq, dk then pass
+ * through the Jacobian of phi.
+ *   q, k, v, o, dout  as in la_forward (o = the forward output, read)
+ *   den       [B,H,N] fp32, read: the den_out of the matching la_forward
+ *   dq, dk    [B,H,N,dqk] dtype, written
+ *   dv        [B,H,N,dv]  dtype, written
+ *   workspace, workspace_bytes: at least la_backward_workspace_bytes(...). */
+LA_API la_status la_backward(const void *q, const void *k, const void *v, const void *o,
+                      const void *dout, const float *den,
+                      void *dq, void *dk, void *dv,
+                      void *workspace, size_t workspace_bytes,
+                      int B, int H, int N, int dqk, int dvdim, int fmap, int dtype,
+                      void *stream);
+
+/* One recurrent decode step for B*H heads (BASED page, Knowl 3 recurrent
+ * form; Knowl 5 generation kernel): S += phi(k) v^T, z += phi(k),
+ * y = phi(q) S / phi(q).z using the UPDATED state.
+ *   q, k  [B,H,dqk] dtype, read;  v [B,H,dv] dtype, read
+ *   y     [B,H,dv]  dtype, written
+ *   s     [B,H,F,dv] fp32, read and updated in place
+ *   z     [B,H,F]    fp32, read and updated in place
+ * The state is read once and written once per call. */
+LA_API la_status la_decode_step(const void *q, const void *k, const void *v, void *y,
+                         float *s, float *z,
+                         int B, int H, int dqk, int dv, int fmap, int dtype,
+                         void *stream);
+
+/* Materialise phi for `rows` input vectors: x [rows,dqk] -> phi [rows,F],
+ * both of `dtype` (fp32 arithmetic, rounded once for bf16).  A test and
+ * baseline helper; the attention kernels compute phi on chip instead. */
+LA_API la_status la_feature_map(const void *x, void *phi, int64_t rows, int dqk, int fmap,
+                         int dtype, void *stream);
+
+/* Which kernels a call would launch, without launching anything (for
+ * launch accounting in benchmarks and tests).  op: 0 = la_forward,
+ * 1 = la_backward, 2 = la_decode_step.  Writes a comma-separated list of
+ * kernel names (truncated to buflen-1 characters, NUL-terminated) to buf
+ * when buf is non-NULL, and returns the number of kernel launches the call
+ * makes, or -1 for arguments the call itself would reject. */
+LA_API int la_kernel_plan(int op, int B, int H, int N, int dqk, int dv, int fmap, int dtype,
+                          char *buf, size_t buflen);
+
+/* Synchronise `stream`, then read and clear the calling device's status
+ * word.  Returns LA_OK, LA_ERR_TIMEOUT or LA_ERR_DEVICE_CHECK for errors
+ * recorded by kernels since the last call, or LA_ERR_CUDA if the
+ * synchronisation itself failed. */
+LA_API la_status la_get_device_status(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LA_H */

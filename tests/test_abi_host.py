@@ -1,0 +1,99 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+The library must load without a GPU, export every entry point include/la.h
+declares, and reject bad arguments synchronously before touching the device.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from causal_kernelized_sequence_b200 import build, load_library
+    build.build()
+    return load_library()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "la.h")).read()
+    return sorted(set(re.findall(r"^LA_API\s+[\w\s\*]+?\b(la_\w+)\s*\(", src, re.M)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_feature_dim_and_strings(lib):
+    assert lib.la_feature_dim(0, 64) == 64
+    assert lib.la_feature_dim(1, 16) == 273
+    assert lib.la_feature_dim(1, 0) == -1
+    assert lib.la_feature_dim(7, 4) == -1
+    assert lib.la_status_string(0) == b"LA_OK"
+    assert lib.la_status_string(4) == b"LA_ERR_TIMEOUT"
+    assert lib.la_status_string(99) == b"LA_ERR_UNKNOWN"
+    assert lib.la_version() >= 100
+
+
+def _fwd(lib, q=0x1000, k=0x2000, v=0x3000, o=0x4000, s=None, z=None, den=None, ws=None, wsb=0,
+         B=1, H=1, N=16, dqk=16, dv=16, fmap=0, dtype=0):
+    P = ctypes.c_void_p
+    return lib.la_forward(P(q), P(k), P(v), P(o), P(s), P(z), P(den), P(ws), wsb, B, H, N, dqk, dv,
+                          fmap, dtype, None)
+
+
+def test_forward_argument_errors(lib):
+    assert _fwd(lib, q=None) == 1                      # null input
+    assert _fwd(lib, B=0) == 1                         # non-positive size
+    assert _fwd(lib, N=-3) == 1
+    assert _fwd(lib, fmap=5) == 1                      # unknown feature map
+    assert _fwd(lib, dtype=9) == 1                     # unknown dtype
+    assert _fwd(lib, k=0x2002) == 1                    # misaligned
+    assert _fwd(lib, s=0x5008) == 1                    # misaligned state
+    assert _fwd(lib, fmap=1, dqk=32) == 2              # Taylor beyond d'=16: unsupported
+    assert _fwd(lib, dv=256) == 2
+    assert _fwd(lib, B=1 << 16, H=1 << 10, N=1 << 10) == 1   # element count overflow
+
+
+def test_backward_and_decode_argument_errors(lib):
+    P = ctypes.c_void_p
+    good = [P(0x1000 * (i + 1)) for i in range(9)]
+    args = lambda ptrs, **kw: (*ptrs, P(None), 0, kw.get("B", 1), 1, 16, 16, 16, kw.get("fmap", 0), 0, None)
+    bad = list(good); bad[5] = P(None)                 # den missing
+    assert lib.la_backward(*args(bad)) == 1
+    assert lib.la_backward(*args(good, fmap=3)) == 1
+    assert lib.la_backward(*args(good, B=0)) == 1
+    # decode: q, k, v, y, s, z
+    d = [P(0x1000 * (i + 1)) for i in range(6)]
+    assert lib.la_decode_step(d[0], d[1], d[2], d[3], d[4], P(None), 2, 2, 16, 64, 1, 0, None) == 1
+    assert lib.la_decode_step(d[0], d[1], d[2], d[3], P(0x4004), d[5], 2, 2, 16, 64, 1, 0, None) == 1
+    assert lib.la_decode_step(*d, 2, 2, 17, 64, 1, 0, None) == 2
+
+
+def test_feature_map_argument_errors(lib):
+    P = ctypes.c_void_p
+    assert lib.la_feature_map(P(None), P(0x2000), 4, 16, 1, 0, None) == 1
+    assert lib.la_feature_map(P(0x1000), P(0x2000), 0, 16, 1, 0, None) == 1
+    assert lib.la_feature_map(P(0x1000), P(0x2000), 4, 20, 1, 0, None) == 2
+
+
+def test_workspace_bytes_invalid_is_zero(lib):
+    assert lib.la_forward_workspace_bytes(0, 1, 1, 16, 16, 0, 0) == 0
+    assert lib.la_backward_workspace_bytes(1, 1, 1, 16, 16, 9, 0) == 0
+
+
+def test_product_path_does_not_reference_oracle():
+    # The library package must never import or load the CPU oracle.
+    pkg = os.path.join(ROOT, "causal_kernelized_sequence_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert "la_oracle" not in txt and "import oracle" not in txt and "from oracle" not in txt, f

@@ -1,0 +1,201 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 CPU oracle.
+
+Metric: max over (b,h) slices of ||x - x_ref||_2 / ||x_ref||_2 (decode: per
+step over the heads compared).  Bars: <= 1e-5 for fp32 I/O, <= 1e-2 for bf16
+I/O with fp32 accumulation, gradients included.  For bf16 the oracle runs on
+the bf16-rounded inputs, so only the GPU's internal rounding is measured.
+"""
+import numpy as np
+import pytest
+import torch
+
+import causal_kernelized_sequence_b200 as la
+import workloads as W
+from oracle import oracle as orc
+
+pytestmark = pytest.mark.gpu
+
+TOL = {W.F32: 1e-5, W.BF16: 1e-2}
+ELU1, TAYLOR2 = W.ELU1, W.TAYLOR2
+DEV = "cuda"
+
+NS = [1, 2, 15, 16, 17, 63, 64, 65, 127, 128, 129, 257, 1000]
+DIMS = [(ELU1, 32, 32), (ELU1, 64, 64), (ELU1, 128, 128), (ELU1, 16, 48), (TAYLOR2, 16, 64),
+        (TAYLOR2, 4, 8)]
+
+
+def gpu_forward(q, k, v, fmap, **kw):
+    r = la.la_forward(q.to(DEV), k.to(DEV), v.to(DEV), fmap, **kw)
+    torch.cuda.synchronize()
+    la.la_get_device_status()
+    return {n: t.cpu() for n, t in r.items()}
+
+
+@pytest.mark.parametrize("dtype", [W.F32, W.BF16])
+@pytest.mark.parametrize("fmap,dqk,dv", DIMS)
+def test_forward_small(fmap, dqk, dv, dtype):
+    for N in NS:
+        q, k, v, _ = W.random_qkv(1000 + N, 2, 2, N, dqk, dv, fmap=fmap, dtype=dtype,
+                                  scale=1.0 if fmap == TAYLOR2 else dqk ** -0.5)
+        r = gpu_forward(q, k, v, fmap, state=True, den=True)
+        o_ref, den_ref = orc.forward_brute(fmap, q, k, v)
+        _, _, s_ref, z_ref = orc.forward_recurrent(fmap, q, k, v)
+        tol = TOL[dtype]
+        assert orc.max_rel_l2(r["o"], o_ref) <= tol, (N, orc.max_rel_l2(r["o"], o_ref))
+        assert orc.max_rel_l2(r["den"], den_ref) <= tol, N
+        assert orc.max_rel_l2(r["s"], s_ref) <= tol, N
+        assert orc.max_rel_l2(r["z"], z_ref) <= tol, N
+        assert (r["den"] > 0).all()
+
+
+@pytest.mark.parametrize("dtype", [W.F32, W.BF16])
+@pytest.mark.parametrize("fmap,dqk,dv", DIMS)
+def test_backward_small(fmap, dqk, dv, dtype):
+    for N in (1, 17, 64, 65, 200, 300):
+        q, k, v, do = W.random_qkv(2000 + N, 1, 2, N, dqk, dv, fmap=fmap, dtype=dtype,
+                                   scale=1.0 if fmap == TAYLOR2 else dqk ** -0.5, with_dout=True)
+        qd, kd, vd, dod = (t.to(DEV) for t in (q, k, v, do))
+        fr = la.la_forward(qd, kd, vd, fmap, den=True)
+        dq, dk, dvv = la.la_backward(qd, kd, vd, fr["o"], dod, fr["den"], fmap)
+        torch.cuda.synchronize()
+        la.la_get_device_status()
+        rq, rk, rv = orc.backward_recurrent(fmap, q, k, v, do)
+        tol = TOL[dtype]
+        for got, ref, name in ((dq, rq, "dq"), (dk, rk, "dk"), (dvv, rv, "dv")):
+            err = orc.max_rel_l2(got.cpu(), ref)
+            assert err <= tol, (N, name, err)
+
+
+@pytest.mark.parametrize("dtype", [W.F32, W.BF16])
+@pytest.mark.parametrize("fmap,dqk,dv", [(TAYLOR2, 16, 64), (ELU1, 64, 64), (ELU1, 32, 48)])
+def test_decode_small(fmap, dqk, dv, dtype):
+    P, T = 37, 20
+    q, k, v, _ = W.random_qkv(3000, 3, 2, P + T, dqk, dv, fmap=fmap, dtype=dtype)
+    r = la.la_forward(q[:, :, :P].contiguous().to(DEV), k[:, :, :P].contiguous().to(DEV),
+                      v[:, :, :P].contiguous().to(DEV), fmap, state=True)
+    s, z = r["s"], r["z"]
+    o_ref, _, s_ref, z_ref = orc.forward_recurrent(fmap, q, k, v)
+    tol = TOL[dtype]
+    for t in range(T):
+        y = la.la_decode_step(q[:, :, P + t].contiguous().to(DEV), k[:, :, P + t].contiguous().to(DEV),
+                              v[:, :, P + t].contiguous().to(DEV), s, z, fmap)
+        err = orc.max_rel_l2(y.cpu()[None], o_ref[:, :, P + t][None], slice_dims=1)
+        assert err <= tol, (t, err)
+    torch.cuda.synchronize()
+    la.la_get_device_status()
+    assert orc.max_rel_l2(s.cpu(), s_ref) <= tol
+    assert orc.max_rel_l2(z.cpu(), z_ref) <= tol
+
+
+@pytest.mark.parametrize("dtype", [W.F32, W.BF16])
+@pytest.mark.parametrize("fmap,dqk", [(ELU1, 64), (TAYLOR2, 16), (TAYLOR2, 3)])
+def test_feature_map(fmap, dqk, dtype):
+    x, _, _, _ = W.random_qkv(4000, 1, 3, 50, dqk, 8, dtype=dtype)
+    phi = la.la_feature_map(x.to(DEV), fmap).cpu()
+    ref = orc.phi(fmap, x)
+    tol = 1e-6 if dtype == W.F32 else 4e-3
+    np.testing.assert_allclose(phi.double().numpy(), ref, rtol=tol, atol=tol)
+
+
+def test_forward_deterministic():
+    q, k, v, _ = W.random_qkv(5000, 2, 4, 777, 16, 64, fmap=TAYLOR2, dtype=W.BF16)
+    a = gpu_forward(q, k, v, TAYLOR2, state=True)
+    b = gpu_forward(q, k, v, TAYLOR2, state=True)
+    for n in a:
+        assert torch.equal(a[n], b[n]), n
+
+
+# ------------------------------------------------------------ full workloads
+
+def test_workload_elu_fp32_fwd():
+    w = W.BY_NAME["elu_fp32_fwd"]
+    q, k, v, _ = W.make_inputs(w)
+    r = gpu_forward(q, k, v, w.fmap, den=True)
+    assert r["o"].shape == (1, 1, 256, 32)
+    o_ref, den_ref = orc.forward_brute(w.fmap, q, k, v)
+    assert orc.max_rel_l2(r["o"], o_ref) <= 1e-5
+    assert orc.max_rel_l2(r["den"], den_ref) <= 1e-5
+
+
+def test_workload_elu_bf16_fwd():
+    w = W.BY_NAME["elu_bf16_fwd"]
+    q, k, v, _ = W.make_inputs(w)
+    r = gpu_forward(q, k, v, w.fmap, den=True, state=True)
+    o_ref, den_ref, s_ref, z_ref = orc.forward_recurrent(w.fmap, q, k, v)
+    assert orc.max_rel_l2(r["o"], o_ref) <= 1e-2
+    assert orc.max_rel_l2(r["den"], den_ref) <= 1e-2
+    assert orc.max_rel_l2(r["s"], s_ref) <= 1e-2
+    # brute force on sampled rows cross-checks the recurrent oracle itself
+    rows = [0, 1, 63, 64, 2047, 4095]
+    ob, _ = orc.forward_rows(w.fmap, q[3, 7], k[3, 7], v[3, 7], rows)
+    np.testing.assert_allclose(o_ref[3, 7, rows], ob, rtol=1e-9, atol=1e-12)
+
+
+def test_workload_taylor_bf16_fwd():
+    w = W.BY_NAME["taylor_bf16_fwd"]
+    q, k, v, _ = W.make_inputs(w)
+    r = gpu_forward(q, k, v, w.fmap, den=True, state=True)
+    heads = [(0, 0), (1, 5), (3, 9), (7, 15)]
+    for b, h in heads:
+        o_ref, den_ref, s_ref, z_ref = orc.forward_recurrent(
+            w.fmap, q[b:b + 1, h:h + 1], k[b:b + 1, h:h + 1], v[b:b + 1, h:h + 1])
+        assert orc.max_rel_l2(r["o"][b:b + 1, h:h + 1], o_ref) <= 1e-2
+        assert orc.max_rel_l2(r["den"][b:b + 1, h:h + 1], den_ref) <= 1e-2
+        assert orc.max_rel_l2(r["s"][b:b + 1, h:h + 1], s_ref) <= 1e-2
+        assert orc.max_rel_l2(r["z"][b:b + 1, h:h + 1], z_ref) <= 1e-2
+    # Taylor: den_i >= i/2 for every head (positivity, any size)
+    assert (r["den"] >= torch.arange(1, w.N + 1) / 2 * (1 - 1e-3)).all()
+
+
+def test_workload_elu_bf16_train():
+    w = W.BY_NAME["elu_bf16_train"]
+    q, k, v, do = W.make_inputs(w)
+    qd, kd, vd, dod = (t.to(DEV) for t in (q, k, v, do))
+    fr = la.la_forward(qd, kd, vd, w.fmap, den=True)
+    dq, dk, dvv = la.la_backward(qd, kd, vd, fr["o"], dod, fr["den"], w.fmap)
+    torch.cuda.synchronize()
+    la.la_get_device_status()
+    for b, h in [(0, 0), (1, 11), (0, 15)]:
+        sl = lambda t: t[b:b + 1, h:h + 1]
+        o_ref, den_ref, _, _ = orc.forward_recurrent(w.fmap, sl(q), sl(k), sl(v))
+        rq, rk, rv = orc.backward_recurrent(w.fmap, sl(q), sl(k), sl(v), sl(do))
+        assert orc.max_rel_l2(sl(fr["o"]).cpu(), o_ref) <= 1e-2
+        for got, ref in ((dq, rq), (dk, rk), (dvv, rv)):
+            assert orc.max_rel_l2(sl(got).cpu(), ref) <= 1e-2
+    # any-size invariant: sum_j dv_j = sum_i dO_i per slice
+    lhs = dvv.float().sum(2)
+    rhs = dod.float().sum(2)
+    assert ((lhs - rhs).norm() / rhs.norm()).item() < 1e-2
+
+
+def test_workload_taylor_decode():
+    w = W.BY_NAME["taylor_decode"]
+    (q, k, v), (sq, sk, sv) = W.make_decode_inputs(w)
+    r = la.la_forward(q.to(DEV), k.to(DEV), v.to(DEV), w.fmap, state=True)
+    s, z = r["s"], r["z"]
+    heads = [(0, 0), (17, 3), (128, 8), (255, 15)]
+    hs = lambda t: torch.stack([t[..., b, h, :] for b, h in heads], dim=-2)
+    # oracle: prefill then the same steps, for the sampled heads only
+    qh = torch.stack([q[b, h] for b, h in heads])[None]
+    kh = torch.stack([k[b, h] for b, h in heads])[None]
+    vh = torch.stack([v[b, h] for b, h in heads])[None]
+    _, _, s_o, z_o = orc.forward_recurrent(w.fmap, qh, kh, vh)
+    s_o = np.ascontiguousarray(s_o[0]); z_o = np.ascontiguousarray(z_o[0])
+    # the prefill's final state, for the sampled heads
+    assert orc.max_rel_l2(torch.stack([s[b, h].cpu() for b, h in heads]), s_o, slice_dims=1) <= 1e-5
+    y_all = torch.empty(w.decode_steps, w.B, w.H, w.dv, device=DEV)
+    sqd, skd, svd = sq.to(DEV), sk.to(DEV), sv.to(DEV)
+    for t in range(w.decode_steps):
+        la.la_decode_step(sqd[t], skd[t], svd[t], s, z, w.fmap, y=y_all[t])
+    torch.cuda.synchronize()
+    la.la_get_device_status()
+    y_all = y_all.cpu()
+    worst = 0.0
+    for t in range(w.decode_steps):
+        y_o = orc.decode_step(w.fmap, hs(sq[t]), hs(sk[t]), hs(sv[t]), s_o, z_o)
+        worst = max(worst, orc.max_rel_l2(hs(y_all[t])[None], y_o[None], slice_dims=1))
+    assert worst <= 1e-5, worst
+    s_fin = torch.stack([s[b, h].cpu() for b, h in heads])
+    z_fin = torch.stack([z[b, h].cpu() for b, h in heads])
+    assert orc.max_rel_l2(s_fin, s_o, slice_dims=1) <= 1e-5
+    assert orc.max_rel_l2(z_fin, z_o, slice_dims=1) <= 1e-5
