@@ -318,13 +318,15 @@ def e2e_prefill(w, dev, steps, warmup):
     ho = torch.empty(w.B, w.H, w.N, w.dv, dtype=w.torch_dtype).pin_memory()
     dq_, dk_, dv_ = (torch.empty(t.shape, dtype=t.dtype, device=dev) for t in (hq, hk, hv))
     do_ = torch.empty(ho.shape, dtype=ho.dtype, device=dev)
+    wsb = la.la_forward_workspace_bytes(w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev) if wsb else None
     stream = torch.cuda.Stream()
 
     def one():
         dq_.copy_(hq, non_blocking=True)
         dk_.copy_(hk, non_blocking=True)
         dv_.copy_(hv, non_blocking=True)
-        la.la_forward(dq_, dk_, dv_, w.fmap, out=do_)
+        la.la_forward(dq_, dk_, dv_, w.fmap, out=do_, workspace=ws)
         ho.copy_(do_, non_blocking=True)
 
     with torch.cuda.stream(stream):

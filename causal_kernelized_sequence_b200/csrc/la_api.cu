@@ -5,12 +5,17 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <mutex>
 
 #include "../../include/la.h"
 #include "la_device.cuh"
 #include "la_simt.cuh"
+#include "la_decode.cuh"
+#include "la_prefill_sm100.cuh"
 
 using namespace la;
 
@@ -80,12 +85,47 @@ la_status set_smem(size_t bytes)
 }
 
 // Kernel selection, shared by the entry points and la_kernel_plan.
-enum class Path { Invalid, FwdSimt, BwdSimt, DecodeSimt };
+enum class Path { Invalid, FwdSimt, FwdTc, BwdSimt, DecodeSimt, DecodeVec };
+
+// Shapes with a tensor-core forward: bf16 I/O and (elu, dqk = dv in {64,128})
+// or (Taylor, dqk = 16, dv = 64).
+bool tc_forward_shape(int dqk, int dv, int fmap, int dtype)
+{
+    if (dtype != LA_BF16) return false;
+    if (fmap == LA_FMAP_ELU1) return dqk == dv && (dqk == 64 || dqk == 128);
+    return dqk == 16 && dv == 64;
+}
 
 Path select_forward(int B, int H, int N, int dqk, int dv, int fmap, int dtype)
 {
     if (check_shape(B, H, N, dqk, dv, fmap, dtype) != LA_OK) return Path::Invalid;
+    if (tc_forward_shape(dqk, dv, fmap, dtype)) return Path::FwdTc;
     return Path::FwdSimt;
+}
+
+// Sequence split of the tensor-core forward: P segments of cps chunks each,
+// so that B*H*P thread blocks roughly fill the 148 SMs.
+constexpr int kNumSms = 148;
+constexpr int kChunk = 128;
+
+void tc_segments(int B, int H, int N, int *P, int *cps, int *nchunks)
+{
+    const int BH = B * H;
+    const int nc = (N + kChunk - 1) / kChunk;
+    int p = kNumSms / BH;
+    if (p < 1) p = 1;
+    if (p > nc) p = nc;
+    const int c = (nc + p - 1) / p;
+    *cps = c;
+    *P = (nc + c - 1) / c;
+    *nchunks = nc;
+}
+
+// fp32 elements per segment increment: FP x NA.
+int64_t tc_increment_floats(int dqk, int dv, int fmap)
+{
+    const int FP = fmap == LA_FMAP_TAYLOR2 ? 160 : dqk;
+    return (int64_t)FP * (dv + 16);
 }
 
 Path select_backward(int B, int H, int N, int dqk, int dv, int fmap, int dtype)
@@ -97,6 +137,7 @@ Path select_backward(int B, int H, int N, int dqk, int dv, int fmap, int dtype)
 Path select_decode(int B, int H, int dqk, int dv, int fmap, int dtype)
 {
     if (check_shape(B, H, 1, dqk, dv, fmap, dtype) != LA_OK) return Path::Invalid;
+    if (dv == 32 || dv == 64 || dv == 128) return Path::DecodeVec;
     return Path::DecodeSimt;
 }
 
@@ -105,8 +146,10 @@ int path_kernels(Path p, const char **names)
 {
     switch (p) {
     case Path::FwdSimt: names[0] = "fwd_simt_kernel"; return 1;
+    case Path::FwdTc: names[0] = "fwd_tc_kernel"; return 1;  // plus the segment pass, see below
     case Path::BwdSimt: names[0] = "bwd_simt_kernel"; return 1;
     case Path::DecodeSimt: names[0] = "decode_simt_kernel"; return 1;
+    case Path::DecodeVec: names[0] = "decode_vec_kernel"; return 1;
     default: return -1;
     }
 }
@@ -172,6 +215,100 @@ la_status decode_simt(const void *q, const void *k, const void *v, void *y, floa
     return launch_status();
 }
 
+template <typename T>
+la_status decode_vec(const void *q, const void *k, const void *v, void *y, float *s, float *z,
+                     int B, int H, int dqk, int dv, int fmap, cudaStream_t stream)
+{
+    const FmapParams fp = make_fmap(fmap, dqk);
+    const T *qq = (const T *)q, *kk = (const T *)k, *vv = (const T *)v;
+    T *yy = (T *)y;
+    switch (dv) {
+    case 32: decode_vec_kernel<T, 32, 18><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp); break;
+    case 64: decode_vec_kernel<T, 64, 18><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp); break;
+    case 128: decode_vec_kernel<T, 128, 18><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp); break;
+    default: return LA_ERR_UNSUPPORTED;
+    }
+    return launch_status();
+}
+
+// ---------------------------------------------------------- tensor maps
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// 3D bf16 view [BH][N][inner] of a dense row-major tensor, box
+// {box_inner, 128, 1}; rows past N read as zero.
+bool make_map(CUtensorMap *m, const void *base, int inner, int N, int BH, int box_inner,
+              CUtensorMapSwizzle sw)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)N, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)N * inner * 2};
+    cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)kChunk, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <class Cfg>
+la_status forward_tc_launch(const void *q, const void *k, const void *v, void *o, float *s_out,
+                            float *z_out, float *den_out, void *workspace, int B, int H, int N,
+                            cudaStream_t stream)
+{
+    const int BH = B * H;
+    CUtensorMap tq, tk, tv;
+    const CUtensorMapSwizzle qsw = Cfg::TAYLOR ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_128B;
+    const int qbox = Cfg::TAYLOR ? 16 : 64;
+    if (!make_map(&tq, q, Cfg::DQK, N, BH, qbox, qsw) || !make_map(&tk, k, Cfg::DQK, N, BH, qbox, qsw) ||
+        !make_map(&tv, v, Cfg::DV, N, BH, 16, CU_TENSOR_MAP_SWIZZLE_32B))
+        return LA_ERR_CUDA;
+    FwdParams p;
+    p.s_out = s_out;
+    p.z_out = z_out;
+    p.den_out = den_out;
+    p.ws = (float *)workspace;
+    p.o = o;
+    p.N = N;
+    tc_segments(B, H, N, &p.P, &p.cps, &p.nchunks);
+    const double d = (double)Cfg::DQK;
+    p.inv_c1 = (float)(1.0 / pow(d, 0.25));
+    p.inv_c2 = (float)(1.0 / (sqrt(2.0) * sqrt(d)));
+    p.k1 = (float)(1.0 / sqrt(d));
+    p.k2 = (float)(1.0 / (2.0 * d));
+    if (set_smem<fwd_tc_kernel<Cfg, 0>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
+    if (p.P > 1) {
+        if (set_smem<fwd_tc_kernel<Cfg, 1>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
+        fwd_tc_kernel<Cfg, 1><<<BH * p.P, 128, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+        if (launch_status() != LA_OK) return LA_ERR_CUDA;
+    }
+    fwd_tc_kernel<Cfg, 0><<<BH * p.P, 128, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+    return launch_status();
+}
+
+la_status forward_tc(const void *q, const void *k, const void *v, void *o, float *s_out, float *z_out,
+                     float *den_out, void *workspace, int B, int H, int N, int dqk, int dv, int fmap,
+                     cudaStream_t stream)
+{
+    if (fmap == LA_FMAP_TAYLOR2)
+        return forward_tc_launch<FwdCfg<16, 64, true>>(q, k, v, o, s_out, z_out, den_out, workspace, B, H, N, stream);
+    if (dqk == 64)
+        return forward_tc_launch<FwdCfg<64, 64, false>>(q, k, v, o, s_out, z_out, den_out, workspace, B, H, N, stream);
+    return forward_tc_launch<FwdCfg<128, 128, false>>(q, k, v, o, s_out, z_out, den_out, workspace, B, H, N, stream);
+}
+
 }  // namespace
 
 extern "C" {
@@ -201,8 +338,11 @@ int64_t la_feature_dim(int fmap, int dqk)
 
 size_t la_forward_workspace_bytes(int B, int H, int N, int dqk, int dv, int fmap, int dtype)
 {
-    if (check_shape(B, H, N, dqk, dv, fmap, dtype) != LA_OK) return 0;
-    return 0;
+    if (select_forward(B, H, N, dqk, dv, fmap, dtype) != Path::FwdTc) return 0;
+    int P, cps, nc;
+    tc_segments(B, H, N, &P, &cps, &nc);
+    if (P <= 1) return 0;
+    return (size_t)B * H * P * tc_increment_floats(dqk, dv, fmap) * sizeof(float);
 }
 
 size_t la_backward_workspace_bytes(int B, int H, int N, int dqk, int dv, int fmap, int dtype)
@@ -223,8 +363,12 @@ la_status la_forward(const void *q, const void *k, const void *v, void *o, float
         return LA_ERR_INVALID_ARG;
     if (workspace_bytes < la_forward_workspace_bytes(B, H, N, dqk, dv, fmap, dtype))
         return LA_ERR_INVALID_ARG;
-    (void)workspace;
     cudaStream_t s = (cudaStream_t)stream;
+    if (select_forward(B, H, N, dqk, dv, fmap, dtype) == Path::FwdTc) {
+        if (workspace_bytes && !aligned(workspace, 16)) return LA_ERR_INVALID_ARG;
+        if (la_forward_workspace_bytes(B, H, N, dqk, dv, fmap, dtype) && !workspace) return LA_ERR_INVALID_ARG;
+        return forward_tc(q, k, v, o, s_out, z_out, den_out, workspace, B, H, N, dqk, dv, fmap, s);
+    }
     if (dtype == LA_F32)
         return forward_simt<float>(q, k, v, o, s_out, z_out, den_out, B, H, N, dqk, dv, fmap, s);
     return forward_simt<__nv_bfloat16>(q, k, v, o, s_out, z_out, den_out, B, H, N, dqk, dv, fmap, s);
@@ -262,6 +406,10 @@ la_status la_decode_step(const void *q, const void *k, const void *v, void *y, f
         !aligned(s, 16) || !aligned(z, 4))
         return LA_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
+    if (select_decode(B, H, dqk, dv, fmap, dtype) == Path::DecodeVec) {
+        if (dtype == LA_F32) return decode_vec<float>(q, k, v, y, s, z, B, H, dqk, dv, fmap, st);
+        return decode_vec<__nv_bfloat16>(q, k, v, y, s, z, B, H, dqk, dv, fmap, st);
+    }
     if (dtype == LA_F32) return decode_simt<float>(q, k, v, y, s, z, B, H, dqk, dv, fmap, st);
     return decode_simt<__nv_bfloat16>(q, k, v, y, s, z, B, H, dqk, dv, fmap, st);
 }
@@ -292,6 +440,16 @@ int la_kernel_plan(int op, int B, int H, int N, int dqk, int dv, int fmap, int d
 {
     Path p = Path::Invalid;
     if (op == 0) p = select_forward(B, H, N, dqk, dv, fmap, dtype);
+    if (p == Path::FwdTc) {
+        int P, cps, nc;
+        tc_segments(B, H, N, &P, &cps, &nc);
+        const char *nm = P > 1 ? "fwd_tc_kernel<segment states>,fwd_tc_kernel" : "fwd_tc_kernel";
+        if (buf && buflen) {
+            strncpy(buf, nm, buflen - 1);
+            buf[buflen - 1] = 0;
+        }
+        return P > 1 ? 2 : 1;
+    }
     else if (op == 1) p = select_backward(B, H, N, dqk, dv, fmap, dtype);
     else if (op == 2) p = select_decode(B, H, dqk, dv, fmap, dtype);
     const char *names[8];

@@ -1,0 +1,545 @@
+// la_prefill_sm100.cuh -- chunked causal linear attention forward on the
+// 5th-generation tensor cores (tcgen05 + TMEM), with TMA-staged inputs.
+//
+// The method (BASED page, Knowl 3 parallel form; Knowl 5 chunked prefill):
+// for a chunk c of C = 128 tokens with state (S, z) accumulated over the
+// earlier chunks,
+//     y_i = [ sum_{j<=i in c} a_ij v_j + phi(q_i) S ] / [ sum_{j<=i} a_ij + phi(q_i).z ],
+//     S  += phi(K_c)^T V_c,   z += sum_j phi(k_j).
+// The normaliser rides along as an extra value column: V_aug = [V | 1 | 0..0]
+// (DV + 16 columns), so S_aug = [S | z] and one accumulator row holds both
+// numerator and denominator, rounded identically.
+//
+// Per chunk (one CTA = one 128-thread warpgroup; thread i <-> token i <->
+// TMEM lane i):
+//   TMA     Q_c, K_c (SW128, or SW32 for d'=16) and V_c (SW32) into a
+//           2-stage ring; out-of-range rows of a ragged tail are zero-filled.
+//   phi     elu(x)+1 applied in place to the Q/K tiles; for the Taylor map
+//           the symmetric second-order features (1 + 16 + 136 = 153, padded
+//           to 160) are written to separate phi tiles.  phi(q).phi(k) equals
+//           1 + q.k/sqrt(d') + (q.k)^2/(2 d') exactly as for the 273-feature
+//           map; the state written at the boundary is expanded back to 273.
+//   MMA1    A = phi(Q_c) phi(K_c)^T      (Taylor: Q_c K_c^T, then the closed
+//           form 1 + s/sqrt(d') + s^2/(2d') in the mask pass)   -> TMEM
+//   MMA3    S_aug += phi(K_c)^T V_aug   (feature rows in TMEM lanes)
+//   mask    causal mask j <= i, bf16 -> P tile in shared memory
+//   MMA2    O_aug = P V_aug + phi(Q_c) S_snap   (S_snap = bf16 copy of the
+//           state entering the chunk)                             -> TMEM
+//   out     y = O[:, :DV] / O[:, DV]; S_snap <- bf16(S_aug) for the next chunk.
+//
+// Long sequences with few heads are split into P segments per head: a first
+// kernel computes each segment's state increment (MMA3 only) into the
+// caller's workspace; each segment of the main kernel starts from the sum of
+// the increments of the segments before it.
+#pragma once
+
+#include "la_device.cuh"
+#include "sm100.cuh"
+
+namespace la {
+
+template <int DQK_, int DV_, bool TAYLOR_>
+struct FwdCfg {
+    static constexpr int DQK = DQK_;
+    static constexpr int DV = DV_;
+    static constexpr bool TAYLOR = TAYLOR_;
+    static constexpr int C = 128;                       // tokens per chunk
+    static constexpr int NA = DV + 16;                  // value columns + normaliser block
+    static constexpr int FSYM = TAYLOR ? 1 + DQK + DQK * (DQK + 1) / 2 : DQK;
+    static constexpr int FP = TAYLOR ? 160 : DQK;       // K extent of phi(Q) S_snap
+    static constexpr int FT = TAYLOR ? 192 : DQK;       // feature extent of phi tiles
+    static constexpr int STAGES = (DQK == 128) ? 1 : 2;
+    // State tiles (features in TMEM lanes).  M of each tile:
+    static constexpr int NT = TAYLOR ? 2 : 1;
+    static __host__ __device__ constexpr int tile_m(int t) { return TAYLOR ? (t == 0 ? 128 : 64) : DQK; }
+    static __host__ __device__ constexpr int tile_f0(int t) { return t == 0 ? 0 : 128; }
+    // TMEM columns
+    static constexpr int COL_O = 0;
+    static constexpr int COL_S = (C > NA ? C : NA);
+    static constexpr int TMEM_USED = COL_S + NT * NA;
+    static constexpr int TMEM_COLS = TMEM_USED <= 256 ? 256 : 512;
+    // Shared memory (bytes; every region 1024-aligned)
+    static constexpr int QK_TILE = TAYLOR ? C * 32 : C * DQK * 2;   // one raw Q or K tile
+    static constexpr int V_BLK = C * 32;                            // one 16-column SW32 block
+    static constexpr int V_TILE = (DV / 16 + 1) * V_BLK;            // V blocks + ones block
+    static constexpr int PHI_TILE = TAYLOR ? C * FT * 2 : 0;
+    static constexpr int P_TILE = C * C * 2;
+    static constexpr int S_BLK = FP * 32;                           // one 16-column block of S_snap
+    static constexpr int S_TILE = (NA / 16) * S_BLK;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + STAGES * QK_TILE;
+    static constexpr int OFF_V = OFF_K + STAGES * QK_TILE;
+    static constexpr int OFF_PQ = OFF_V + ((STAGES * V_TILE + 1023) / 1024) * 1024;
+    static constexpr int OFF_PK = OFF_PQ + PHI_TILE;
+    static constexpr int OFF_P = OFF_PK + PHI_TILE;
+    static constexpr int OFF_S = OFF_P + P_TILE;
+    static constexpr int OFF_BAR = OFF_S + ((S_TILE + 1023) / 1024) * 1024;
+    static constexpr int SMEM = OFF_BAR + 128;
+    static constexpr int SMEM_ALLOC = SMEM + 1024;      // slack for 1024-byte alignment
+    static constexpr int TX_BYTES = 2 * C * DQK * 2 + C * DV * 2;
+};
+
+struct FwdParams {
+    float *s_out;       // [BH, F273/F, DV] nullable
+    float *z_out;       // [BH, F] nullable
+    float *den_out;     // [BH, N] nullable
+    float *ws;          // [BH, P, FP, NA] segment increments (P > 1)
+    void *o;            // [BH, N, DV] bf16
+    int N, P, nchunks, cps;
+    float inv_c1, inv_c2;       // Taylor: 1/d'^(1/4), 1/(sqrt(2) sqrt(d'))
+    float k1, k2;               // Taylor closed form: 1/sqrt(d'), 1/(2 d')
+};
+
+namespace fwd_detail {
+
+// Byte offset of element (row r, column col) inside a tile stored as
+// 128-byte swizzled rows (TMA SWIZZLE_128B / UMMA SW128, 64 bf16 per row
+// block, 128 rows per block).
+__device__ __forceinline__ uint32_t sw128_off(int r, int col)
+{
+    const int blk = col >> 6, c = (col >> 3) & 7;
+    return blk * (128 * 128) + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4) + (col & 7) * 2;
+}
+
+// Byte offset of (row r, column col) in a 32-byte swizzled layout made of
+// 16-column blocks of `rows` rows each (TMA SWIZZLE_32B / UMMA SW32).
+__device__ __forceinline__ uint32_t sw32_off(int r, int col, int rows)
+{
+    const int blk = col >> 4, c = (col >> 3) & 1;
+    return blk * (rows * 32) + (r >> 3) * 256 + (r & 7) * 32 + ((c ^ ((r >> 2) & 1)) << 4) + (col & 7) * 2;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b)
+{
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+__device__ __forceinline__ void unpack8(uint4 u, float *f)
+{
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 t = __bfloat1622float2(h[i]);
+        f[2 * i] = t.x;
+        f[2 * i + 1] = t.y;
+    }
+}
+
+// Symmetric second-order Taylor feature f (0 <= f < 192) of x[16]:
+// [1 | x_a/c1 | x_a^2/c2 | sqrt2 x_a x_b / c2 (a < b, row-major) | 0...].
+template <int D>
+__device__ __forceinline__ float taylor_sym_feature(const float *x, int f, float inv_c1, float inv_c2,
+                                                    float r2_inv_c2)
+{
+    if (f == 0) return 1.f;
+    if (f <= D) return x[f - 1] * inv_c1;
+    if (f <= 2 * D) return x[f - 1 - D] * x[f - 1 - D] * inv_c2;
+    int p = f - 1 - 2 * D;
+#pragma unroll
+    for (int a = 0; a < D - 1; ++a) {
+        const int cnt = D - 1 - a;
+        if (p < cnt) return x[a] * x[a + 1 + p] * r2_inv_c2;
+        p -= cnt;
+    }
+    return 0.f;
+}
+
+// Row index in the 273-feature (full outer product) layout of symmetric
+// feature f, and its second position (or -1) and scale.
+template <int D>
+__device__ __forceinline__ void taylor_sym_to_full(int f, int &r1, int &r2, float &scale)
+{
+    r2 = -1;
+    scale = 1.f;
+    if (f <= D) { r1 = f; return; }
+    if (f <= 2 * D) { const int a = f - 1 - D; r1 = 1 + D + a * D + a; return; }
+    int p = f - 1 - 2 * D;
+    for (int a = 0; a < D - 1; ++a) {
+        const int cnt = D - 1 - a;
+        if (p < cnt) {
+            const int b = a + 1 + p;
+            r1 = 1 + D + a * D + b;
+            r2 = 1 + D + b * D + a;
+            scale = 0.70710678118654752440f;  // the packed feature carries sqrt(2)
+            return;
+        }
+        p -= cnt;
+    }
+    r1 = -1;
+}
+
+}  // namespace fwd_detail
+
+// MODE 0: full forward (o, den, final state).  MODE 1: state increments of
+// each segment only (written to p.ws).
+template <class Cfg, int MODE>
+__global__ void __launch_bounds__(128, 1)
+fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v, const FwdParams p)
+{
+    using namespace sm100;
+    using namespace fwd_detail;
+    constexpr int C = Cfg::C, DV = Cfg::DV, NA = Cfg::NA, DQK = Cfg::DQK, FP = Cfg::FP;
+    constexpr int STAGES = Cfg::STAGES;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *tma_bar = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
+    uint64_t *mma_bar = tma_bar + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tma_bar + 3);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tma_bar + 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int bh = blockIdx.x / p.P, seg = blockIdx.x % p.P;
+    if (MODE == 1 && seg == p.P - 1) return;  // the last segment's increment is never read
+    const int c_begin = seg * p.cps;
+    const int c_end = min(p.nchunks, c_begin + p.cps);
+    const int N = p.N;
+
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) mbar_init(&tma_bar[s], 1);
+        mbar_init(mma_bar, 1);
+        *abort_flag = 0;
+        mbar_init_fence();
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+    // Constant normaliser block of every V stage: column DV of V_aug = 1.
+    for (int s = 0; s < STAGES; ++s) {
+        uint8_t *blk = smem + Cfg::OFF_V + s * Cfg::V_TILE + (DV / 16) * Cfg::V_BLK;
+        const int r = tid;  // C == 128 rows, one per thread
+        uint4 *row = reinterpret_cast<uint4 *>(blk + (r >> 3) * 256 + (r & 7) * 32);
+        const int one_chunk = 0 ^ ((r >> 2) & 1);
+        row[one_chunk] = make_uint4(pack_bf16(1.f, 0.f), 0u, 0u, 0u);
+        row[one_chunk ^ 1] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+
+    auto issue_tma = [&](int chunk, int s) {
+        const int t0 = chunk * C;
+        mbar_arrive_expect_tx(&tma_bar[s], MODE == 0 ? Cfg::TX_BYTES : Cfg::TX_BYTES - C * DQK * 2);
+        uint8_t *q_dst = smem + Cfg::OFF_Q + s * Cfg::QK_TILE;
+        uint8_t *k_dst = smem + Cfg::OFF_K + s * Cfg::QK_TILE;
+        constexpr int QBOX = Cfg::TAYLOR ? 16 : 64;
+        for (int x = 0; x < DQK; x += QBOX) {
+            const int off = Cfg::TAYLOR ? 0 : (x / 64) * C * 128;
+            if (MODE == 0) tma_load_3d(q_dst + off, &tm_q, &tma_bar[s], x, t0, bh);
+            tma_load_3d(k_dst + off, &tm_k, &tma_bar[s], x, t0, bh);
+        }
+        uint8_t *v_dst = smem + Cfg::OFF_V + s * Cfg::V_TILE;
+        for (int x = 0; x < DV; x += 16) tma_load_3d(v_dst + (x / 16) * Cfg::V_BLK, &tm_v, &tma_bar[s], x, t0, bh);
+    };
+
+    bool have_state = false;
+    // ---- starting state of this segment: sum of the earlier segments' increments
+    if (MODE == 0 && seg > 0) {
+        for (int t = 0; t < Cfg::NT; ++t) {
+            const int m = Cfg::tile_m(t);
+            const int r = (m == 128) ? tid : ((lane < 16) ? warp * 16 + lane : -1);
+            const int f = r < 0 ? -1 : Cfg::tile_f0(t) + r;
+            for (int c0 = 0; c0 < NA; c0 += 16) {
+                float acc[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+                if (f >= 0 && f < FP) {
+                    for (int s2 = 0; s2 < seg; ++s2) {
+                        const float *src = p.ws + ((size_t)(bh * p.P + s2) * FP + f) * NA + c0;
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) acc[e] += src[e];
+                    }
+                }
+                tmem_st16(tmem + lane_base + Cfg::COL_S + t * NA + c0, acc);
+                if (f >= 0 && f < FP) {
+                    uint8_t *sS = smem + Cfg::OFF_S;
+#pragma unroll
+                    for (int e = 0; e < 16; e += 8) {
+                        uint4 u = make_uint4(pack_bf16(acc[e], acc[e + 1]), pack_bf16(acc[e + 2], acc[e + 3]),
+                                             pack_bf16(acc[e + 4], acc[e + 5]), pack_bf16(acc[e + 6], acc[e + 7]));
+                        *reinterpret_cast<uint4 *>(sS + sw32_off(f, c0 + e, FP)) = u;
+                    }
+                }
+            }
+        }
+        tmem_st_wait();
+        have_state = true;
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    if (tid == 0)
+        for (int s = 0; s < STAGES && c_begin + s < c_end; ++s) issue_tma(c_begin + s, s);
+
+    uint32_t mma_phase = 0;
+    const float inv_c1 = p.inv_c1, inv_c2 = p.inv_c2, r2_inv_c2 = p.inv_c2 * 1.41421356237309504880f;
+
+    for (int chunk = c_begin; chunk < c_end; ++chunk) {
+        const int it = chunk - c_begin;
+        const int s = it % STAGES;
+        const uint32_t tphase = (uint32_t)(it / STAGES) & 1u;
+        const int t0 = chunk * C;
+        const int nvalid = min(C, N - t0);
+        if (!mbar_wait(&tma_bar[s], tphase)) *abort_flag = 1;
+        uint8_t *sQ = smem + Cfg::OFF_Q + s * Cfg::QK_TILE;
+        uint8_t *sK = smem + Cfg::OFF_K + s * Cfg::QK_TILE;
+        uint8_t *sV = smem + Cfg::OFF_V + s * Cfg::V_TILE;
+        uint8_t *sPQ = Cfg::TAYLOR ? smem + Cfg::OFF_PQ : sQ;
+        uint8_t *sPK = Cfg::TAYLOR ? smem + Cfg::OFF_PK : sK;
+
+        // ---- feature maps (thread i owns token row i)
+        {
+            const int i = tid;
+            const bool kvalid = i < nvalid;
+            if (!Cfg::TAYLOR) {
+#pragma unroll 1
+                for (int m = 0; m < (MODE == 0 ? 2 : 1); ++m) {
+                    uint8_t *tile = (MODE == 0 && m == 0) ? sQ : sK;
+                    const bool zero = (tile == sK) && !kvalid;
+#pragma unroll
+                    for (int col = 0; col < DQK; col += 8) {
+                        uint4 *ptr = reinterpret_cast<uint4 *>(tile + sw128_off(i, col));
+                        float x[8];
+                        unpack8(*ptr, x);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) x[e] = zero ? 0.f : (x[e] > 0.f ? x[e] + 1.f : __expf(x[e]));
+                        *ptr = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
+                                          pack_bf16(x[6], x[7]));
+                    }
+                }
+            } else {
+#pragma unroll 1
+                for (int m = (MODE == 0 ? 0 : 1); m < 2; ++m) {
+                    const uint8_t *raw = m == 0 ? sQ : sK;
+                    uint8_t *dst = m == 0 ? sPQ : sPK;
+                    const bool zero = (m == 1) && !kvalid;
+                    float x[16];
+                    unpack8(*reinterpret_cast<const uint4 *>(raw + sw32_off(i, 0, C)), x);
+                    unpack8(*reinterpret_cast<const uint4 *>(raw + sw32_off(i, 8, C)), x + 8);
+#pragma unroll
+                    for (int f0 = 0; f0 < Cfg::FT; f0 += 8) {
+                        float v8[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            v8[e] = zero ? 0.f : taylor_sym_feature<16>(x, f0 + e, inv_c1, inv_c2, r2_inv_c2);
+                        *reinterpret_cast<uint4 *>(dst + sw128_off(i, f0)) =
+                            make_uint4(pack_bf16(v8[0], v8[1]), pack_bf16(v8[2], v8[3]),
+                                       pack_bf16(v8[4], v8[5]), pack_bf16(v8[6], v8[7]));
+                    }
+                }
+            }
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (*abort_flag) break;
+
+        // ---- MMA1 (scores) and MMA3 (state update)
+        if (tid == 0) {
+            const uint32_t aQ = smem_addr(sPQ), aK = smem_addr(sPK), aV = smem_addr(sV);
+            if (MODE == 0) {
+                if (Cfg::TAYLOR) {
+                    const uint32_t qa = smem_addr(sQ), ka = smem_addr(sK);
+                    mma_bf16(tmem + Cfg::COL_O, smem_desc(qa, 16, 256, kSw32), smem_desc(ka, 16, 256, kSw32),
+                             idesc_bf16(128, 128, 0, 0), false);
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < DQK / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * (C * 128) + (kk & 3) * 32;
+                        mma_bf16(tmem + Cfg::COL_O, smem_desc(aQ + off, 16, 1024, kSw128),
+                                 smem_desc(aK + off, 16, 1024, kSw128), idesc_bf16(128, 128, 0, 0), kk > 0);
+                    }
+                }
+            }
+#pragma unroll
+            for (int t = 0; t < Cfg::NT; ++t) {
+                const int m = Cfg::tile_m(t);
+                const uint32_t idesc = idesc_bf16(m, NA, 1, 1);
+                const uint32_t a_base = aK + (Cfg::tile_f0(t) / 64) * (C * 128);
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk) {
+                    mma_bf16(tmem + Cfg::COL_S + t * NA,
+                             smem_desc(a_base + kk * 2048, C * 128, 1024, kSw128),
+                             smem_desc(aV + kk * 512, Cfg::V_BLK, 256, kSw32), idesc,
+                             have_state || kk > 0);
+                }
+            }
+            mma_commit(mma_bar);
+        }
+        if (!mbar_wait(mma_bar, mma_phase)) *abort_flag = 1;
+        mma_phase ^= 1u;
+        tc_fence_after();
+        have_state = true;
+
+        if (MODE == 1) {
+            __syncthreads();
+            if (tid == 0 && it + STAGES < c_end - c_begin) issue_tma(chunk + STAGES, s);
+            if (*abort_flag) break;
+            continue;
+        }
+
+        // ---- causal mask -> P (bf16, K-major SW128)
+        {
+            const int i = tid;
+            uint8_t *sP = smem + Cfg::OFF_P;
+#pragma unroll 1
+            for (int j0 = 0; j0 < C; j0 += 32) {
+                float a[32];
+                tmem_ld32(tmem + lane_base + Cfg::COL_O + j0, a);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int j = j0 + e;
+                    float w = a[e];
+                    if (Cfg::TAYLOR) w = 1.f + w * p.k1 + w * w * p.k2;
+                    a[e] = (j <= i) ? w : 0.f;
+                }
+#pragma unroll
+                for (int e = 0; e < 32; e += 8)
+                    *reinterpret_cast<uint4 *>(sP + sw128_off(i, j0 + e)) =
+                        make_uint4(pack_bf16(a[e], a[e + 1]), pack_bf16(a[e + 2], a[e + 3]),
+                                   pack_bf16(a[e + 4], a[e + 5]), pack_bf16(a[e + 6], a[e + 7]));
+            }
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+
+        // ---- MMA2: O_aug = P V_aug + phi(Q) S_snap
+        if (tid == 0) {
+            const uint32_t aP = smem_addr(smem + Cfg::OFF_P), aV = smem_addr(sV);
+            const uint32_t idesc = idesc_bf16(128, NA, 0, 1);
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * (C * 128) + (kk & 3) * 32;
+                mma_bf16(tmem + Cfg::COL_O, smem_desc(aP + off, 16, 1024, kSw128),
+                         smem_desc(aV + kk * 512, Cfg::V_BLK, 256, kSw32), idesc, kk > 0);
+            }
+            if (chunk > 0) {
+                const uint32_t aQ = smem_addr(sPQ), aS = smem_addr(smem + Cfg::OFF_S);
+#pragma unroll
+                for (int kk = 0; kk < FP / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * (C * 128) + (kk & 3) * 32;
+                    mma_bf16(tmem + Cfg::COL_O, smem_desc(aQ + off, 16, 1024, kSw128),
+                             smem_desc(aS + kk * 512, Cfg::S_BLK, 256, kSw32), idesc, true);
+                }
+            }
+            mma_commit(mma_bar);
+        }
+        if (!mbar_wait(mma_bar, mma_phase)) *abort_flag = 1;
+        mma_phase ^= 1u;
+        tc_fence_after();
+        if (tid == 0 && it + STAGES < c_end - c_begin) issue_tma(chunk + STAGES, s);
+
+        // ---- outputs: y = num / den
+        {
+            const int i = tid;
+            float o[NA];
+#pragma unroll
+            for (int c0 = 0; c0 < NA; c0 += 16) tmem_ld16(tmem + lane_base + Cfg::COL_O + c0, o + c0);
+            tmem_ld_wait();
+            const float den = o[DV];
+            const float inv = 1.f / den;
+            if (i < nvalid) {
+                __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + ((size_t)bh * N + t0 + i) * DV;
+#pragma unroll
+                for (int c0 = 0; c0 < DV; c0 += 8)
+                    *reinterpret_cast<uint4 *>(orow + c0) =
+                        make_uint4(pack_bf16(o[c0] * inv, o[c0 + 1] * inv), pack_bf16(o[c0 + 2] * inv, o[c0 + 3] * inv),
+                                   pack_bf16(o[c0 + 4] * inv, o[c0 + 5] * inv), pack_bf16(o[c0 + 6] * inv, o[c0 + 7] * inv));
+                if (p.den_out) p.den_out[(size_t)bh * N + t0 + i] = den;
+            }
+        }
+        // ---- state snapshot for the next chunk (bf16, MN-major SW32)
+        if (chunk + 1 < c_end) {
+            uint8_t *sS = smem + Cfg::OFF_S;
+#pragma unroll
+            for (int t = 0; t < Cfg::NT; ++t) {
+                const int m = Cfg::tile_m(t);
+                const int r = (m == 128) ? tid : ((lane < 16) ? warp * 16 + lane : -1);
+                const int f = r < 0 ? -1 : Cfg::tile_f0(t) + r;
+#pragma unroll
+                for (int c0 = 0; c0 < NA; c0 += 16) {
+                    float v[16];
+                    tmem_ld16(tmem + lane_base + Cfg::COL_S + t * NA + c0, v);
+                    tmem_ld_wait();
+                    if (f >= 0 && f < FP) {
+                        *reinterpret_cast<uint4 *>(sS + sw32_off(f, c0, FP)) =
+                            make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
+                                       pack_bf16(v[6], v[7]));
+                        *reinterpret_cast<uint4 *>(sS + sw32_off(f, c0 + 8, FP)) =
+                            make_uint4(pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]), pack_bf16(v[12], v[13]),
+                                       pack_bf16(v[14], v[15]));
+                    }
+                }
+            }
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (*abort_flag) break;
+    }
+
+    // ---- segment increment (MODE 1) or final state (MODE 0, last segment)
+    const bool write_ws = (MODE == 1);
+    const bool write_final = (MODE == 0) && (seg == p.P - 1) && (p.s_out || p.z_out) && !*abort_flag;
+    if ((write_ws || write_final) && !*abort_flag) {
+#pragma unroll 1
+        for (int t = 0; t < Cfg::NT; ++t) {
+            const int m = Cfg::tile_m(t);
+            const int r = (m == 128) ? tid : ((lane < 16) ? warp * 16 + lane : -1);
+            const int f = r < 0 ? -1 : Cfg::tile_f0(t) + r;
+#pragma unroll 1
+            for (int c0 = 0; c0 < NA; c0 += 16) {
+                float v[16];
+                tmem_ld16(tmem + lane_base + Cfg::COL_S + t * NA + c0, v);
+                tmem_ld_wait();
+                if (f < 0 || f >= FP) continue;
+                if (write_ws) {
+                    float *dst = p.ws + ((size_t)(bh * p.P + seg) * FP + f) * NA + c0;
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) dst[e] = v[e];
+                    continue;
+                }
+                if (f >= Cfg::FSYM) continue;
+                const int F = Cfg::TAYLOR ? 1 + DQK + DQK * DQK : DQK;
+                int r1, r2;
+                float sc;
+                if (Cfg::TAYLOR) {
+                    taylor_sym_to_full<16>(f, r1, r2, sc);
+                } else {
+                    r1 = f; r2 = -1; sc = 1.f;
+                }
+                for (int e = 0; e < 16; ++e) {
+                    const int col = c0 + e;
+                    const float val = v[e] * sc;
+                    if (col < DV) {
+                        if (p.s_out) {
+                            p.s_out[((size_t)bh * F + r1) * DV + col] = val;
+                            if (r2 >= 0) p.s_out[((size_t)bh * F + r2) * DV + col] = val;
+                        }
+                    } else if (col == DV && p.z_out) {
+                        p.z_out[(size_t)bh * F + r1] = val;
+                        if (r2 >= 0) p.z_out[(size_t)bh * F + r2] = val;
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, Cfg::TMEM_COLS);
+}
+
+}  // namespace la

@@ -61,6 +61,12 @@ def test_backward_small(fmap, dqk, dv, dtype):
         la.la_get_device_status()
         rq, rk, rv = orc.backward_recurrent(fmap, q, k, v, do)
         tol = TOL[dtype]
+        if N == 1:
+            # y_1 = v_1 whatever q and k are: dq and dk vanish exactly (the
+            # relative metric is undefined there), and dv_1 = dO_1.
+            assert dq.abs().max().item() <= 1e-4 and dk.abs().max().item() <= 1e-4
+            assert orc.max_rel_l2(dvv.cpu(), do) <= tol
+            continue
         for got, ref, name in ((dq, rq, "dq"), (dk, rk, "dk"), (dvv, rv, "dv")):
             err = orc.max_rel_l2(got.cpu(), ref)
             assert err <= tol, (N, name, err)
