@@ -187,11 +187,15 @@ class Train:
         self.o = torch.empty_like(self.v)
         self.den = torch.empty(w.B, w.H, w.N, device=dev)
         self.dq, self.dk, self.dvv = torch.empty_like(self.q), torch.empty_like(self.k), torch.empty_like(self.v)
+        self.fws_bytes = la.la_forward_workspace_bytes(w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype)
+        self.bws_bytes = la.la_backward_workspace_bytes(w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype)
+        self.fws = torch.empty(max(1, self.fws_bytes), dtype=torch.uint8, device=dev)
+        self.bws = torch.empty(max(1, self.bws_bytes), dtype=torch.uint8, device=dev)
         self.tokens = w.B * w.N
         e = 2
         BHN = w.B * w.H * w.N
         self.fwd_bytes = BHN * (2 * w.dqk + 2 * w.dv) * e + BHN * 4
-        self.bwd_bytes = BHN * (2 * w.dqk + 3 * w.dv) * e + BHN * 4 + BHN * (2 * w.dqk + w.dv) * e
+        self.bwd_bytes = BHN * (2 * w.dqk + 2 * w.dv) * e + BHN * (2 * w.dqk + w.dv) * e
         self.alg_bytes = self.fwd_bytes + self.bwd_bytes
         F = w.feature_dim
         self.alg_flops = (4.0 * F * (w.dv + 1) + 10.0 * F * w.dv + 6.0 * F) * BHN
@@ -203,11 +207,11 @@ class Train:
         import ctypes
         P = lambda t: ctypes.c_void_p(t.data_ptr())
         st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-        r = lib.la_forward(P(self.q), P(self.k), P(self.v), P(self.o), None, None, P(self.den), None, 0,
-                           w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype, st)
+        r = lib.la_forward(P(self.q), P(self.k), P(self.v), P(self.o), None, None, P(self.den), P(self.fws),
+                           self.fws_bytes, w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype, st)
         assert r == 0, r
-        r = lib.la_backward(P(self.q), P(self.k), P(self.v), P(self.o), P(self.do), P(self.den), P(self.dq),
-                            P(self.dk), P(self.dvv), None, 0, w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype, st)
+        r = lib.la_backward(P(self.q), P(self.k), P(self.v), P(self.do), P(self.dq), P(self.dk), P(self.dvv),
+                            P(self.bws), self.bws_bytes, w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype, st)
         assert r == 0, r
 
     def l2_note(self):

@@ -9,7 +9,7 @@ loudly when the library has not been built.
 
 Entry points (same names as the C ABI):
     la_forward(q, k, v, fmap, *, state=False, den=False, out=None) -> dict
-    la_backward(q, k, v, o, dout, den, fmap) -> (dq, dk, dv)
+    la_backward(q, k, v, dout, fmap) -> (dq, dk, dv)
     la_decode_step(q, k, v, s, z, fmap, y=None) -> y        (s, z in place)
     la_feature_map(x, fmap) -> phi
     la_feature_dim(fmap, dqk) -> int
@@ -62,7 +62,7 @@ def load_library(path: str | None = None):
     lib.la_backward_workspace_bytes.restype = sz
     lib.la_forward.argtypes = [vp] * 8 + [sz] + [i] * 7 + [vp]
     lib.la_forward.restype = i
-    lib.la_backward.argtypes = [vp] * 10 + [sz] + [i] * 7 + [vp]
+    lib.la_backward.argtypes = [vp] * 8 + [sz] + [i] * 7 + [vp]
     lib.la_backward.restype = i
     lib.la_decode_step.argtypes = [vp] * 6 + [i] * 6 + [vp]
     lib.la_decode_step.restype = i
@@ -143,10 +143,10 @@ def la_forward(q, k, v, fmap, *, state=False, den=False, out=None, workspace=Non
     return res
 
 
-def la_backward(q, k, v, o, dout, den, fmap, *, workspace=None):
+def la_backward(q, k, v, dout, fmap, *, workspace=None):
     """Gradients (dq, dk, dv) of the forward for upstream gradient dout."""
     lib = load_library()
-    _dev(q, k, v, o, dout, den)
+    _dev(q, k, v, dout)
     B, H, N, dqk = q.shape
     dv = v.shape[-1]
     dt = _dtype_code(q)
@@ -156,9 +156,8 @@ def la_backward(q, k, v, o, dout, den, fmap, *, workspace=None):
     wsb = la_backward_workspace_bytes(B, H, N, dqk, dv, fmap, dt)
     if workspace is None and wsb:
         workspace = torch.empty(wsb, dtype=torch.uint8, device=q.device)
-    _check(lib.la_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(den), _ptr(dq),
-                           _ptr(dk), _ptr(dvv), _ptr(workspace), wsb, B, H, N, dqk, dv, fmap, dt,
-                           _stream()), "la_backward")
+    _check(lib.la_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dvv),
+                           _ptr(workspace), wsb, B, H, N, dqk, dv, fmap, dt, _stream()), "la_backward")
     return dq, dk, dvv
 
 

@@ -186,9 +186,9 @@ la_status forward_simt(const void *q, const void *k, const void *v, void *o, flo
 }
 
 template <typename T>
-la_status backward_simt(const void *q, const void *k, const void *v, const void *o,
-                        const void *dout, const float *den, void *dq, void *dk, void *dvp,
-                        int B, int H, int N, int dqk, int dv, int fmap, cudaStream_t stream)
+la_status backward_simt(const void *q, const void *k, const void *v, const void *dout, void *dq,
+                        void *dk, void *dvp, float *ws, int B, int H, int N, int dqk, int dv,
+                        int fmap, cudaStream_t stream)
 {
     const FmapParams fp = make_fmap(fmap, dqk);
     SimtBwdSmem L;
@@ -196,8 +196,8 @@ la_status backward_simt(const void *q, const void *k, const void *v, const void 
     if (!pick_chunk(simt_bwd_layout, fp.F, dqk, dv, &L, &bytes)) return LA_ERR_UNSUPPORTED;
     if (set_smem<bwd_simt_kernel<T>>(bytes) != LA_OK) return LA_ERR_CUDA;
     bwd_simt_kernel<T><<<B * H, kSimtThreads, bytes, stream>>>(
-        (const T *)q, (const T *)k, (const T *)v, (const T *)o, (const T *)dout, den, (T *)dq,
-        (T *)dk, (T *)dvp, N, dv, fp, L);
+        (const T *)q, (const T *)k, (const T *)v, (const T *)dout, ws, (T *)dq, (T *)dk, (T *)dvp,
+        N, dv, fp, L);
     return launch_status();
 }
 
@@ -348,7 +348,7 @@ size_t la_forward_workspace_bytes(int B, int H, int N, int dqk, int dv, int fmap
 size_t la_backward_workspace_bytes(int B, int H, int N, int dqk, int dv, int fmap, int dtype)
 {
     if (check_shape(B, H, N, dqk, dv, fmap, dtype) != LA_OK) return 0;
-    return 0;
+    return (size_t)B * H * N * 2 * sizeof(float);  // den_i, dden_i
 }
 
 la_status la_forward(const void *q, const void *k, const void *v, void *o, float *s_out,
@@ -374,25 +374,23 @@ la_status la_forward(const void *q, const void *k, const void *v, void *o, float
     return forward_simt<__nv_bfloat16>(q, k, v, o, s_out, z_out, den_out, B, H, N, dqk, dv, fmap, s);
 }
 
-la_status la_backward(const void *q, const void *k, const void *v, const void *o,
-                      const void *dout, const float *den, void *dq, void *dk, void *dvp,
-                      void *workspace, size_t workspace_bytes, int B, int H, int N, int dqk,
-                      int dv, int fmap, int dtype, void *stream)
+la_status la_backward(const void *q, const void *k, const void *v, const void *dout, void *dq,
+                      void *dk, void *dvp, void *workspace, size_t workspace_bytes, int B, int H,
+                      int N, int dqk, int dv, int fmap, int dtype, void *stream)
 {
     const la_status sh = check_shape(B, H, N, dqk, dv, fmap, dtype);
     if (sh != LA_OK) return sh;
-    if (!q || !k || !v || !o || !dout || !den || !dq || !dk || !dvp) return LA_ERR_INVALID_ARG;
-    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
-        !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dvp, 16) ||
-        !aligned(den, 4))
+    if (!q || !k || !v || !dout || !dq || !dk || !dvp || !workspace) return LA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(dout, 16) ||
+        !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dvp, 16) || !aligned(workspace, 16))
         return LA_ERR_INVALID_ARG;
     if (workspace_bytes < la_backward_workspace_bytes(B, H, N, dqk, dv, fmap, dtype))
         return LA_ERR_INVALID_ARG;
-    (void)workspace;
     cudaStream_t s = (cudaStream_t)stream;
+    float *ws = (float *)workspace;
     if (dtype == LA_F32)
-        return backward_simt<float>(q, k, v, o, dout, den, dq, dk, dvp, B, H, N, dqk, dv, fmap, s);
-    return backward_simt<__nv_bfloat16>(q, k, v, o, dout, den, dq, dk, dvp, B, H, N, dqk, dv, fmap, s);
+        return backward_simt<float>(q, k, v, dout, dq, dk, dvp, ws, B, H, N, dqk, dv, fmap, s);
+    return backward_simt<__nv_bfloat16>(q, k, v, dout, dq, dk, dvp, ws, B, H, N, dqk, dv, fmap, s);
 }
 
 la_status la_decode_step(const void *q, const void *k, const void *v, void *y, float *s,

@@ -156,9 +156,8 @@ inline SimtBwdSmem simt_bwd_layout(int C, int F, int dv)
 template <typename T>
 __global__ void __launch_bounds__(kSimtThreads)
 bwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
-                const T *__restrict__ o, const T *__restrict__ dout,
-                const float *__restrict__ den_in, T *__restrict__ dq, T *__restrict__ dk,
-                T *__restrict__ dvo, int N, int dv, FmapParams fp, SimtBwdSmem L)
+                const T *__restrict__ dout, float *__restrict__ ws, T *__restrict__ dq,
+                T *__restrict__ dk, T *__restrict__ dvo, int N, int dv, FmapParams fp, SimtBwdSmem L)
 {
     extern __shared__ float sm[];
     const int F = fp.F, dqk = fp.dqk, C = L.C, FS = L.FS, DS = L.DS;
@@ -170,7 +169,7 @@ bwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
     float *pk = pq + (size_t)C * FS;    // [C][FS]
     float *dphi = pk + (size_t)C * FS;  // [C][FS]
     float *vs = dphi + (size_t)C * FS;  // [C][dv]
-    float *gs = vs + C * dv;            // [C][dv]   g_i = dout_i / den_i
+    float *gs = vs + C * dv;            // [C][dv]   dout_i, then g_i = dout_i / den_i
     float *A = gs + C * dv;             // [C][C]    a_ij
     float *dA = A + C * C;              // [C][C]    da_ij
     float *dd = dA + C * C;             // [C]       dden_i = -g_i . y_i
@@ -180,8 +179,8 @@ bwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
     const int lane = tid & 31, warp = tid >> 5, nwarps = nt >> 5;
     const size_t bh = blockIdx.x;
     const T *qb = q + bh * N * dqk, *kb = k + bh * N * dqk;
-    const T *vb = v + bh * N * dv, *ob = o + bh * N * dv, *gb = dout + bh * N * dv;
-    const float *denb = den_in + bh * N;
+    const T *vb = v + bh * N * dv, *gb = dout + bh * N * dv;
+    float *wsb = ws + bh * (size_t)N * 2;   // per token: den_i, dden_i (pass 1 -> pass 2)
     T *dqb = dq + bh * N * dqk, *dkb = dk + bh * N * dqk, *dvb = dvo + bh * N * dv;
 
     const int nchunks = (N + C - 1) / C;
@@ -198,40 +197,67 @@ bwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
                 xq[i] = ld(qb + (size_t)t0 * dqk + i);
                 xk[i] = ld(kb + (size_t)t0 * dqk + i);
             }
-            for (int i = tid; i < Lc; i += nt) dn[i] = denb[t0 + i];
-            __syncthreads();
             for (int i = tid; i < Lc * dv; i += nt) {
-                const int r = i / dv;
                 vs[i] = ld(vb + (size_t)t0 * dv + i);
-                gs[i] = ld(gb + (size_t)t0 * dv + i) / dn[r];
+                gs[i] = ld(gb + (size_t)t0 * dv + i);
             }
+            __syncthreads();
             for (int idx = tid; idx < Lc * F; idx += nt) {
                 const int i = idx / F, f = idx - i * F;
                 pq[i * FS + f] = phi_feature(fp, xq + i * dqk, f);
                 pk[i * FS + f] = phi_feature(fp, xk + i * dqk, f);
             }
             __syncthreads();
-            // dden_i = -g_i . y_i   (one warp per row; y_i is the forward output)
-            for (int i = warp; i < Lc; i += nwarps) {
-                float acc = 0.f;
-                for (int c = lane; c < dv; c += 32)
-                    acc = fmaf(gs[i * dv + c], ld(ob + (size_t)(t0 + i) * dv + c), acc);
-                for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-                if (lane == 0) dd[i] = -acc;
-            }
-            __syncthreads();
-            // da_ij = g_i . v_j + dden_i, and (pass 2) a_ij, for j <= i
+            // a_ij = phi(q_i).phi(k_j), j <= i
             for (int idx = tid; idx < Lc * Lc; idx += nt) {
                 const int i = idx / Lc, j = idx - i * Lc;
-                float da = 0.f, a = 0.f;
+                float a = 0.f;
+                if (j <= i)
+                    for (int f = 0; f < F; ++f) a = fmaf(pq[i * FS + f], pk[j * FS + f], a);
+                A[i * C + j] = a;
+            }
+            __syncthreads();
+            if (pass == 0) {
+                // den_i and y_i in fp32 from the state entering the chunk;
+                // dden_i = -(dout_i . num_i) / den_i^2.  One warp per row.
+                for (int i = warp; i < Lc; i += nwarps) {
+                    float d = 0.f;
+                    for (int f = lane; f < F; f += 32) d = fmaf(pq[i * FS + f], zt[f], d);
+                    for (int j = lane; j <= i; j += 32) d += A[i * C + j];
+                    for (int off = 16; off; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+                    float gy = 0.f;
+                    for (int c = lane; c < dv; c += 32) {
+                        float num = 0.f;
+                        for (int f = 0; f < F; ++f) num = fmaf(pq[i * FS + f], St[f * DS + c], num);
+                        for (int j = 0; j <= i; ++j) num = fmaf(A[i * C + j], vs[j * dv + c], num);
+                        gy = fmaf(gs[i * dv + c], num, gy);
+                    }
+                    for (int off = 16; off; off >>= 1) gy += __shfl_xor_sync(0xffffffffu, gy, off);
+                    if (lane == 0) {
+                        dn[i] = d;
+                        dd[i] = -gy / (d * d);
+                        wsb[2 * (t0 + i)] = d;
+                        wsb[2 * (t0 + i) + 1] = dd[i];
+                    }
+                }
+            } else {
+                for (int i = tid; i < Lc; i += nt) {
+                    dn[i] = wsb[2 * (t0 + i)];
+                    dd[i] = wsb[2 * (t0 + i) + 1];
+                }
+            }
+            __syncthreads();
+            for (int i = tid; i < Lc * dv; i += nt) gs[i] = gs[i] / dn[i / dv];
+            __syncthreads();
+            // da_ij = g_i . v_j + dden_i for j <= i
+            for (int idx = tid; idx < Lc * Lc; idx += nt) {
+                const int i = idx / Lc, j = idx - i * Lc;
+                float da = 0.f;
                 if (j <= i) {
                     for (int c = 0; c < dv; ++c) da = fmaf(gs[i * dv + c], vs[j * dv + c], da);
                     da += dd[i];
-                    if (pass == 1)
-                        for (int f = 0; f < F; ++f) a = fmaf(pq[i * FS + f], pk[j * FS + f], a);
                 }
                 dA[i * C + j] = da;
-                A[i * C + j] = a;
             }
             __syncthreads();
             if (pass == 0) {

@@ -108,8 +108,7 @@ LA_API size_t la_backward_workspace_bytes(int B, int H, int N, int dqk, int dv, 
  *   s_out     [B,H,F,dv]  fp32, nullable: final state S_N (Knowl 5: the
  *             prefill may write its final state for generation)
  *   z_out     [B,H,F]     fp32, nullable: final z_N
- *   den_out   [B,H,N]     fp32, nullable: den_i = phi(q_i).z_i (needed by
- *             la_backward)
+ *   den_out   [B,H,N]     fp32, nullable: den_i = phi(q_i).z_i
  *   workspace, workspace_bytes: at least la_forward_workspace_bytes(...)
  *             bytes of device memory (may be NULL when that is 0).
  * Outputs must not overlap inputs. */
@@ -121,23 +120,25 @@ LA_API la_status la_forward(const void *q, const void *k, const void *v, void *o
 
 /* Gradients of the forward with respect to q, k and v for an upstream
  * gradient dout.  The pages give no backward pass; this is the derivative
- * of the Knowl 3 parallel form: with g_i = dout_i / den_i and
- * dden_i = -g_i . o_i, a forward-order scan of (S, z) gives
- * dphi(q_i) = S_i g_i + z_i dden_i, and a reverse-order scan of
- * R_j = sum_{i>=j} phi(q_i) g_i^T, r_j = sum_{i>=j} phi(q_i) dden_i gives
- * dphi(k_j) = R_j v_j + r_j and dv_j = R_j^T phi(k_j); dq, dk then pass
- * through the Jacobian of phi.
- *   q, k, v, o, dout  as in la_forward (o = the forward output, read)
- *   den       [B,H,N] fp32, read: the den_out of the matching la_forward
+ * of the Knowl 3 parallel form: with den_i = phi(q_i).z_i,
+ * y_i = phi(q_i) S_i / den_i, g_i = dout_i / den_i and dden_i = -g_i . y_i,
+ * a forward-order scan of (S, z) gives dphi(q_i) = S_i g_i + z_i dden_i, and
+ * a reverse-order scan of R_j = sum_{i>=j} phi(q_i) g_i^T and
+ * r_j = sum_{i>=j} phi(q_i) dden_i gives dphi(k_j) = R_j v_j + r_j and
+ * dv_j = R_j^T phi(k_j); dq, dk then pass through the Jacobian of phi.
+ * y_i and den_i are recomputed in fp32 inside the call rather than taken
+ * from a rounded forward output: dq is a small difference of large terms
+ * (sum_j a_ij (v_j - y_i) = 0), so a bf16-rounded y would be amplified.
+ *   q, k, dout, v  as in la_forward (dout like o), read
  *   dq, dk    [B,H,N,dqk] dtype, written
  *   dv        [B,H,N,dv]  dtype, written
- *   workspace, workspace_bytes: at least la_backward_workspace_bytes(...). */
-LA_API la_status la_backward(const void *q, const void *k, const void *v, const void *o,
-                      const void *dout, const float *den,
-                      void *dq, void *dk, void *dv,
-                      void *workspace, size_t workspace_bytes,
-                      int B, int H, int N, int dqk, int dvdim, int fmap, int dtype,
-                      void *stream);
+ *   workspace, workspace_bytes: at least la_backward_workspace_bytes(...)
+ *             bytes of device memory (per-token den_i and dden_i, fp32). */
+LA_API la_status la_backward(const void *q, const void *k, const void *v, const void *dout,
+                             void *dq, void *dk, void *dv,
+                             void *workspace, size_t workspace_bytes,
+                             int B, int H, int N, int dqk, int dvdim, int fmap, int dtype,
+                             void *stream);
 
 /* One recurrent decode step for B*H heads (BASED page, Knowl 3 recurrent
  * form; Knowl 5 generation kernel): S += phi(k) v^T, z += phi(k),

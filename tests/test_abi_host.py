@@ -64,12 +64,16 @@ def test_forward_argument_errors(lib):
 
 def test_backward_and_decode_argument_errors(lib):
     P = ctypes.c_void_p
-    good = [P(0x1000 * (i + 1)) for i in range(9)]
-    args = lambda ptrs, **kw: (*ptrs, P(None), 0, kw.get("B", 1), 1, 16, 16, 16, kw.get("fmap", 0), 0, None)
-    bad = list(good); bad[5] = P(None)                 # den missing
+    good = [P(0x1000 * (i + 1)) for i in range(7)]
+    args = lambda ptrs, ws=P(0x9000), wsb=1 << 20, **kw: (*ptrs, ws, wsb, kw.get("B", 1), 1, 16, 16, 16,
+                                                           kw.get("fmap", 0), 0, None)
+    bad = list(good); bad[3] = P(None)                 # dout missing
     assert lib.la_backward(*args(bad)) == 1
     assert lib.la_backward(*args(good, fmap=3)) == 1
     assert lib.la_backward(*args(good, B=0)) == 1
+    assert lib.la_backward(*args(good, ws=P(None))) == 1            # workspace required
+    assert lib.la_backward(*args(good, wsb=16 * 4)) == 1            # too small: 16 tokens x 2 fp32
+    assert lib.la_backward_workspace_bytes(1, 1, 16, 16, 16, 0, 0) == 16 * 2 * 4
     # decode: q, k, v, y, s, z
     d = [P(0x1000 * (i + 1)) for i in range(6)]
     assert lib.la_decode_step(d[0], d[1], d[2], d[3], d[4], P(None), 2, 2, 16, 64, 1, 0, None) == 1

@@ -55,8 +55,7 @@ def test_backward_small(fmap, dqk, dv, dtype):
         q, k, v, do = W.random_qkv(2000 + N, 1, 2, N, dqk, dv, fmap=fmap, dtype=dtype,
                                    scale=1.0 if fmap == TAYLOR2 else dqk ** -0.5, with_dout=True)
         qd, kd, vd, dod = (t.to(DEV) for t in (q, k, v, do))
-        fr = la.la_forward(qd, kd, vd, fmap, den=True)
-        dq, dk, dvv = la.la_backward(qd, kd, vd, fr["o"], dod, fr["den"], fmap)
+        dq, dk, dvv = la.la_backward(qd, kd, vd, dod, fmap)
         torch.cuda.synchronize()
         la.la_get_device_status()
         rq, rk, rv = orc.backward_recurrent(fmap, q, k, v, do)
@@ -158,7 +157,7 @@ def test_workload_elu_bf16_train():
     q, k, v, do = W.make_inputs(w)
     qd, kd, vd, dod = (t.to(DEV) for t in (q, k, v, do))
     fr = la.la_forward(qd, kd, vd, w.fmap, den=True)
-    dq, dk, dvv = la.la_backward(qd, kd, vd, fr["o"], dod, fr["den"], w.fmap)
+    dq, dk, dvv = la.la_backward(qd, kd, vd, dod, w.fmap)
     torch.cuda.synchronize()
     la.la_get_device_status()
     for b, h in [(0, 0), (1, 11), (0, 15)]:
