@@ -28,7 +28,7 @@ LA_F32 = 0
 LA_BF16 = 1
 
 STATUS_NAMES = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED", 3: "LA_ERR_CUDA",
-                4: "LA_ERR_TIMEOUT", 5: "LA_ERR_DEVICE_CHECK"}
+                4: "LA_ERR_TIMEOUT", 5: "LA_ERR_DEVICE_CHECK", 6: "LA_ERR_SCRATCH_LIMIT"}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "_build", "libla.so")
@@ -70,6 +70,8 @@ def load_library(path: str | None = None):
     lib.la_feature_map.restype = i
     lib.la_get_device_status.argtypes = [vp]
     lib.la_get_device_status.restype = i
+    lib.la_forward_noalloc.argtypes = [vp] * 7 + [i] * 7 + [vp]
+    lib.la_forward_noalloc.restype = i
     lib.la_kernel_plan.argtypes = [i] * 8 + [ctypes.c_char_p, sz]
     lib.la_kernel_plan.restype = i
     _lib = lib
@@ -140,6 +142,30 @@ def la_forward(q, k, v, fmap, *, state=False, den=False, out=None, workspace=Non
     _check(lib.la_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(res.get("s")), _ptr(res.get("z")),
                           _ptr(res.get("den")), _ptr(workspace), wsb, B, H, N, dqk, dv, fmap, dt,
                           _stream()), "la_forward")
+    return res
+
+
+def la_forward_noalloc(q, k, v, fmap, *, state=False, den=False, out=None):
+    """la_forward without a workspace argument: the library uses its own
+    built-in device scratch (for callers that cannot allocate device memory;
+    calls must not overlap on the GPU).  Outputs are allocated here only if
+    not given."""
+    lib = load_library()
+    _dev(q, k, v, out)
+    B, H, N, dqk = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q)
+    F = la_feature_dim(fmap, dqk)
+    o = out if out is not None else torch.empty(B, H, N, dv, dtype=q.dtype, device=q.device)
+    res = {"o": o}
+    if state:
+        res["s"] = torch.empty(B, H, F, dv, dtype=torch.float32, device=q.device)
+        res["z"] = torch.empty(B, H, F, dtype=torch.float32, device=q.device)
+    if den:
+        res["den"] = torch.empty(B, H, N, dtype=torch.float32, device=q.device)
+    _check(lib.la_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(res.get("s")), _ptr(res.get("z")),
+                                  _ptr(res.get("den")), B, H, N, dqk, dv, fmap, dt, _stream()),
+           "la_forward_noalloc")
     return res
 
 

@@ -324,6 +324,7 @@ const char *la_status_string(int status)
     case LA_ERR_CUDA: return "LA_ERR_CUDA";
     case LA_ERR_TIMEOUT: return "LA_ERR_TIMEOUT";
     case LA_ERR_DEVICE_CHECK: return "LA_ERR_DEVICE_CHECK";
+    case LA_ERR_SCRATCH_LIMIT: return "LA_ERR_SCRATCH_LIMIT";
     default: return "LA_ERR_UNKNOWN";
     }
 }
@@ -372,6 +373,49 @@ la_status la_forward(const void *q, const void *k, const void *v, void *o, float
     if (dtype == LA_F32)
         return forward_simt<float>(q, k, v, o, s_out, z_out, den_out, B, H, N, dqk, dv, fmap, s);
     return forward_simt<__nv_bfloat16>(q, k, v, o, s_out, z_out, den_out, B, H, N, dqk, dv, fmap, s);
+}
+
+// Allocation-free forward: la_forward with its workspace taken from a
+// scratch array compiled into the library.  Callers without access to a
+// device allocator (a plugin inside a host program that owns all device
+// memory, a fixed-footprint service) use it instead of allocating the
+// workspace themselves.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[LA_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch for the current device, looked up once
+// per device.  In host code the symbol itself is only a host-side stand-in,
+// so kernels must be given this address, never the symbol.
+static la_status noalloc_scratch(void **out)
+{
+    static void *addr[64] = {nullptr};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return LA_ERR_CUDA;
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return LA_OK;
+}
+
+la_status la_forward_noalloc(const void *q, const void *k, const void *v, void *o, float *s_out,
+                             float *z_out, float *den_out, int B, int H, int N, int dqk, int dv,
+                             int fmap, int dtype, void *stream)
+{
+    const la_status sh = check_shape(B, H, N, dqk, dv, fmap, dtype);
+    if (sh != LA_OK) return sh;
+    const size_t need = la_forward_workspace_bytes(B, H, N, dqk, dv, fmap, dtype);
+    if (need > LA_NOALLOC_SCRATCH_BYTES) return LA_ERR_SCRATCH_LIMIT;
+    if (need == 0)
+        return la_forward(q, k, v, o, s_out, z_out, den_out, nullptr, 0, B, H, N, dqk, dv, fmap, dtype, stream);
+    void *scratch = nullptr;
+    const la_status st = noalloc_scratch(&scratch);
+    if (st != LA_OK) return st;
+    return la_forward(q, k, v, o, s_out, z_out, den_out, scratch, LA_NOALLOC_SCRATCH_BYTES, B, H, N, dqk,
+                      dv, fmap, dtype, stream);
 }
 
 la_status la_backward(const void *q, const void *k, const void *v, const void *dout, void *dq,

@@ -74,7 +74,8 @@ typedef enum {
     LA_ERR_UNSUPPORTED = 2,
     LA_ERR_CUDA = 3,
     LA_ERR_TIMEOUT = 4,      /* a bounded device-side wait ran out          */
-    LA_ERR_DEVICE_CHECK = 5  /* a device-side bounds/consistency check failed */
+    LA_ERR_DEVICE_CHECK = 5, /* a device-side bounds/consistency check failed */
+    LA_ERR_SCRATCH_LIMIT = 6 /* la_forward_noalloc: sizes need more than its built-in scratch */
 } la_status;
 
 /* Library version as 10000*major + 100*minor + patch. */
@@ -117,6 +118,37 @@ LA_API la_status la_forward(const void *q, const void *k, const void *v, void *o
                      void *workspace, size_t workspace_bytes,
                      int B, int H, int N, int dqk, int dv, int fmap, int dtype,
                      void *stream);
+
+/* la_forward for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart to this entry point; it is an interface
+ * convenience.  la_forward may need a workspace (la_forward_workspace_bytes)
+ * that the caller allocates.  Some callers have no device allocator to call:
+ * a plugin running inside a host program that owns every device allocation
+ * and hands out none, or a service that keeps a fixed device footprint and
+ * forbids allocating on its serving path.  This variant takes the same
+ * inputs and outputs as la_forward but no workspace: it uses a scratch
+ * array of LA_NOALLOC_SCRATCH_BYTES (8 MiB) compiled into the library as a
+ * static device array, which every GPU that loads the library holds until
+ * the process exits.  It never calls cudaMalloc, cudaFree or any allocating
+ * library routine.
+ *   - Sizes whose workspace would exceed the scratch are rejected with
+ *     LA_ERR_SCRATCH_LIMIT before anything is launched (for example elu
+ *     dqk = dv = 128 with B*H = 32 and N = 16384 needs 9.4 MB).
+ *   - The first call on a device looks up the scratch array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents.
+ *     Nothing in it needs to start at zero (each call writes every value it
+ *     later reads), but calls whose executions overlap on the GPU (on
+ *     different streams, or from different host threads) race on it and
+ *     give wrong results: serialise them.
+ * Other arguments, outputs and errors are those of la_forward. */
+#define LA_NOALLOC_SCRATCH_BYTES (8u << 20)
+LA_API la_status la_forward_noalloc(const void *q, const void *k, const void *v, void *o,
+                                    float *s_out, float *z_out, float *den_out,
+                                    int B, int H, int N, int dqk, int dv, int fmap, int dtype,
+                                    void *stream);
 
 /* Gradients of the forward with respect to q, k and v for an upstream
  * gradient dout.  The pages give no backward pass; this is the derivative

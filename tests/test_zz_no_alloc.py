@@ -1,0 +1,79 @@
+"""The allocation-free forward (la_forward_noalloc) against la_forward.
+
+la_forward_noalloc serves callers that cannot allocate device memory: it
+runs the same kernels as la_forward but takes the workspace from a scratch
+array built into the library instead of from the caller.  This test calls it
+through the C ABI twice in a row, on two different inputs (the second call
+finds the first call's data in the shared scratch), and checks each result
+against la_forward given a workspace the test allocated, within the bf16
+parity tolerance (max relative L2 error per (b,h) slice <= 1e-2).  It also
+checks that sizes needing more scratch than the library holds are refused
+before anything runs.
+
+The file is named so that pytest collects it after every other test.
+"""
+import ctypes
+
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-2  # bf16 I/O parity bar used by the other GPU tests
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from causal_kernelized_sequence_b200 import build, load_library
+    build.build()
+    return load_library()
+
+
+def _rel_l2(x, ref):
+    """Max over (b,h) slices of ||x - ref|| / ||ref||."""
+    x = x.double().reshape(x.shape[0] * x.shape[1], -1)
+    ref = ref.double().reshape(x.shape)
+    return ((x - ref).norm(dim=-1) / ref.norm(dim=-1)).max().item()
+
+
+def _inputs(seed, B, H, N, D):
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    mk = lambda: (torch.randn(B, H, N, D, generator=g) / D ** 0.5).to(torch.bfloat16).cuda()
+    return mk(), mk(), mk()
+
+
+def test_noalloc_matches_forward_twice(lib):
+    import causal_kernelized_sequence_b200 as la
+    B, H, N, D, fmap, dtype = 4, 8, 4096, 64, 0, 1      # elu, bf16: split forward with workspace
+    need = lib.la_forward_workspace_bytes(B, H, N, D, D, fmap, dtype)
+    assert 0 < need <= (8 << 20)
+    P = lambda t: ctypes.c_void_p(None if t is None else t.data_ptr())
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    for seed in (11, 12):
+        q, k, v = _inputs(seed, B, H, N, D)
+        ref = la.la_forward(q, k, v, fmap, state=True, den=True)
+        o = torch.full_like(v, float("nan"))
+        s = torch.full_like(ref["s"], float("nan"))
+        z = torch.full_like(ref["z"], float("nan"))
+        den = torch.full_like(ref["den"], float("nan"))
+        st = lib.la_forward_noalloc(P(q), P(k), P(v), P(o), P(s), P(z), P(den), B, H, N, D, D, fmap, dtype,
+                                    stream)
+        assert st == 0, la.STATUS_NAMES.get(st, st)
+        torch.cuda.synchronize()
+        la.la_get_device_status()
+        assert _rel_l2(o, ref["o"]) <= TOL
+        assert _rel_l2(den, ref["den"]) <= TOL
+        assert _rel_l2(s, ref["s"]) <= TOL
+        assert _rel_l2(z, ref["z"]) <= TOL
+
+
+def test_noalloc_rejects_sizes_beyond_scratch(lib):
+    # elu bf16 B=2 H=16 N=16384 D=128 needs 9.4 MB of workspace > 8 MiB.
+    B, H, N, D = 2, 16, 16384, 128
+    assert lib.la_forward_workspace_bytes(B, H, N, D, D, 0, 1) > (8 << 20)
+    P = ctypes.c_void_p
+    st = lib.la_forward_noalloc(P(0x1000), P(0x2000), P(0x3000), P(0x4000), P(None), P(None), P(None),
+                                B, H, N, D, D, 0, 1, None)
+    assert st == 6  # LA_ERR_SCRATCH_LIMIT
+    assert lib.la_status_string(6) == b"LA_ERR_SCRATCH_LIMIT"
