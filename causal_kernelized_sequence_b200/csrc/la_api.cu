@@ -16,6 +16,7 @@
 #include "la_simt.cuh"
 #include "la_decode.cuh"
 #include "la_prefill_sm100.cuh"
+#include "la_fwd_ws_sm100.cuh"
 
 using namespace la;
 
@@ -298,10 +299,42 @@ la_status forward_tc_launch(const void *q, const void *k, const void *v, void *o
     return launch_status();
 }
 
+// Warp-specialised forward (elu, d_qk = d_v = 64).
+la_status forward_ws64(const void *q, const void *k, const void *v, void *o, float *s_out, float *z_out,
+                       float *den_out, void *workspace, int B, int H, int N, cudaStream_t stream)
+{
+    using Cfg = WsCfg64;
+    const int BH = B * H;
+    CUtensorMap tq, tk, tv;
+    if (!make_map(&tq, q, 64, N, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tk, k, 64, N, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tv, v, 64, N, BH, 16, CU_TENSOR_MAP_SWIZZLE_32B))
+        return LA_ERR_CUDA;
+    FwdParams p;
+    p.s_out = s_out;
+    p.z_out = z_out;
+    p.den_out = den_out;
+    p.ws = (float *)workspace;
+    p.o = o;
+    p.N = N;
+    tc_segments(B, H, N, &p.P, &p.cps, &p.nchunks);
+    p.inv_c1 = p.inv_c2 = p.k1 = p.k2 = 0.f;
+    if (set_smem<fwd_ws_kernel<0>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
+    if (p.P > 1) {
+        if (set_smem<fwd_ws_kernel<1>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
+        fwd_ws_kernel<1><<<BH * p.P, 512, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+        if (launch_status() != LA_OK) return LA_ERR_CUDA;
+    }
+    fwd_ws_kernel<0><<<BH * p.P, 512, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+    return launch_status();
+}
+
 la_status forward_tc(const void *q, const void *k, const void *v, void *o, float *s_out, float *z_out,
                      float *den_out, void *workspace, int B, int H, int N, int dqk, int dv, int fmap,
                      cudaStream_t stream)
 {
+    if (fmap == LA_FMAP_ELU1 && dqk == 64 && dv == 64)
+        return forward_ws64(q, k, v, o, s_out, z_out, den_out, workspace, B, H, N, stream);
     if (fmap == LA_FMAP_TAYLOR2)
         return forward_tc_launch<FwdCfg<16, 64, true>>(q, k, v, o, s_out, z_out, den_out, workspace, B, H, N, stream);
     if (dqk == 64)
@@ -485,7 +518,9 @@ int la_kernel_plan(int op, int B, int H, int N, int dqk, int dv, int fmap, int d
     if (p == Path::FwdTc) {
         int P, cps, nc;
         tc_segments(B, H, N, &P, &cps, &nc);
-        const char *nm = P > 1 ? "fwd_tc_kernel<segment states>,fwd_tc_kernel" : "fwd_tc_kernel";
+        const bool ws64 = fmap == LA_FMAP_ELU1 && dqk == 64 && dv == 64;
+        const char *nm = ws64 ? (P > 1 ? "fwd_ws_kernel<segment states>,fwd_ws_kernel" : "fwd_ws_kernel")
+                              : (P > 1 ? "fwd_tc_kernel<segment states>,fwd_tc_kernel" : "fwd_tc_kernel");
         if (buf && buflen) {
             strncpy(buf, nm, buflen - 1);
             buf[buflen - 1] = 0;

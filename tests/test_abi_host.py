@@ -109,7 +109,7 @@ def test_kernel_plan_and_workspace(lib):
     # chunks; each segment increment is 64 features x (64 + 16) fp32.
     assert la.la_forward_workspace_bytes(4, 8, 4096, 64, 64, 0, 1) == 32 * 4 * 64 * 80 * 4
     n, names = la.la_kernel_plan(0, 4, 8, 4096, 64, 64, 0, 1)
-    assert n == 2 and names[-1] == "fwd_tc_kernel"
+    assert n == 2 and names[-1] == "fwd_ws_kernel"
     # Taylor B=8 H=16: 128 heads -> no split, no workspace
     assert la.la_forward_workspace_bytes(8, 16, 2048, 16, 64, 1, 1) == 0
     assert la.la_kernel_plan(0, 8, 16, 2048, 16, 64, 1, 1)[0] == 1
