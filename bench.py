@@ -437,6 +437,8 @@ def main():
     ap.add_argument("--workload", default="elu_bf16_fwd", choices=list(W.BY_NAME))
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
+    ap.add_argument("--profile-calls", type=int, default=0,
+                    help="run this many untimed steps of --workload and exit (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -461,6 +463,14 @@ def main():
 
     w = W.BY_NAME[args.workload]
     run = make_run(w, dev, rank)
+    if args.profile_calls:
+        for i in range(args.profile_calls):
+            run.step(i)
+        torch.cuda.synchronize()
+        la.la_get_device_status()
+        print(json.dumps({"profile_calls": args.profile_calls, "workload": w.describe(),
+                          "kernels": la.kernel_plan(w)["kernels"]}), flush=True)
+        return 0
     ms, clocks = timed(run, args.steps, args.warmup, dist_on, local)
     value = run.tokens * world / (ms * 1e-3)
     kern_ms = ms  # one library launch per step for the prefill workloads

@@ -303,7 +303,6 @@ la_status forward_tc_launch(const void *q, const void *k, const void *v, void *o
 la_status forward_ws64(const void *q, const void *k, const void *v, void *o, float *s_out, float *z_out,
                        float *den_out, void *workspace, int B, int H, int N, cudaStream_t stream)
 {
-    using Cfg = WsCfg64;
     const int BH = B * H;
     CUtensorMap tq, tk, tv;
     if (!make_map(&tq, q, 64, N, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -319,13 +318,14 @@ la_status forward_ws64(const void *q, const void *k, const void *v, void *o, flo
     p.N = N;
     tc_segments(B, H, N, &p.P, &p.cps, &p.nchunks);
     p.inv_c1 = p.inv_c2 = p.k1 = p.k2 = 0.f;
-    if (set_smem<fwd_ws_kernel<0>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
+    constexpr int smem0 = WsCfg64<0>::SMEM_ALLOC, smem1 = WsCfg64<1>::SMEM_ALLOC;
+    if (set_smem<fwd_ws_kernel<0>>(smem0) != LA_OK) return LA_ERR_CUDA;
     if (p.P > 1) {
-        if (set_smem<fwd_ws_kernel<1>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
-        fwd_ws_kernel<1><<<BH * p.P, 512, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+        if (set_smem<fwd_ws_kernel<1>>(smem1) != LA_OK) return LA_ERR_CUDA;
+        fwd_ws_kernel<1><<<BH * p.P, 512, smem1, stream>>>(tq, tk, tv, p);
         if (launch_status() != LA_OK) return LA_ERR_CUDA;
     }
-    fwd_ws_kernel<0><<<BH * p.P, 512, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+    fwd_ws_kernel<0><<<BH * p.P, 512, smem0, stream>>>(tq, tk, tv, p);
     return launch_status();
 }
 
@@ -545,6 +545,14 @@ int la_kernel_plan(int op, int B, int H, int N, int dqk, int dv, int fmap, int d
     }
     return n;
 }
+
+#ifdef LA_TIMELINE
+// Profiling builds only: copy the block-0 role timeline of the last forward.
+LA_API int la_debug_timeline(long long *host)
+{
+    return cudaMemcpyFromSymbol(host, g_timeline, sizeof(g_timeline)) == cudaSuccess ? 0 : 1;
+}
+#endif
 
 la_status la_get_device_status(void *stream)
 {

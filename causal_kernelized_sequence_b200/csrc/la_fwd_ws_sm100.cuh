@@ -39,27 +39,44 @@
 
 namespace la {
 
+// Optional per-role timeline of block 0 (clock64 at role boundaries, per
+// chunk), for profiling builds that define LA_TIMELINE; compiled out
+// otherwise.
+#ifdef LA_TIMELINE
+__device__ long long g_timeline[2][16][64];
+#define LA_TL(ev, it_)                                                         \
+    do {                                                                       \
+        if (blockIdx.x == 0 && (it_) >= 0 && (it_) < 64) g_timeline[MODE][ev][(it_)] = clock64(); \
+    } while (0)
+#else
+#define LA_TL(ev, it_) do { } while (0)
+#endif
+
+template <int MODE>
 struct WsCfg64 {
     static constexpr int C = 128, DQK = 64, DV = 64, NA = 80;
-    static constexpr int NS = 2;                         // TMA stages
+    // MODE 0 stages hold Q, K and V_aug; MODE 1 (state increments) only K and V_aug.
+    static constexpr int NS = MODE == 0 ? 3 : 4;         // TMA stages
     static constexpr int QK_TILE = C * DQK * 2;          // 16 KB
     static constexpr int V_BLK = C * 32;                 // 4 KB (16 columns)
     static constexpr int V_TILE = (DV / 16 + 1) * V_BLK; // 20 KB incl. the ones block
-    static constexpr int STAGE = 2 * QK_TILE + V_TILE;   // 52 KB
-    static constexpr int P_TILE = C * C * 2;             // 32 KB
+    static constexpr int OFF_Q = 0;                      // within a stage (MODE 0 only)
+    static constexpr int OFF_K = MODE == 0 ? QK_TILE : 0;
+    static constexpr int OFF_V = OFF_K + QK_TILE;
+    static constexpr int STAGE = OFF_V + V_TILE;         // 52 KB / 36 KB
     static constexpr int S_BLK = DQK * 32;               // 2 KB (16 columns x 64 feature rows)
     static constexpr int S_TILE = (NA / 16) * S_BLK;     // 10 KB
     static constexpr int OFF_STAGE = 0;
-    static constexpr int OFF_P = OFF_STAGE + NS * STAGE;         // 104 KB
-    static constexpr int OFF_S = OFF_P + 2 * P_TILE;             // 168 KB
-    static constexpr int OFF_BAR = OFF_S + 2 * S_TILE;           // 188 KB
+    static constexpr int OFF_S = OFF_STAGE + NS * STAGE;
+    static constexpr int OFF_BAR = OFF_S + (MODE == 0 ? 2 * S_TILE : 0);
     static constexpr int SMEM_ALLOC = OFF_BAR + 256 + 1024;
     // TMEM columns
-    static constexpr int COL_A = 0;      // 2 x 128
+    static constexpr int COL_A = 0;      // 2 x 128 (scores fp32; then P bf16 packed in the first 64)
     static constexpr int COL_O = 256;    // 2 x 80
     static constexpr int COL_DS = 416;   // 80 (M = 64 layout: feature f in lane 32*(f/16) + f%16)
     static constexpr int TMEM_COLS = 512;
-    static constexpr int TX_BYTES = 2 * QK_TILE + DV * C * 2;
+    static constexpr int TX_BYTES = (MODE == 0 ? 2 : 1) * QK_TILE + DV * C * 2;
+    static constexpr int PREFETCH = 4;   // chunks ahead whose tiles are pulled into L2
 };
 
 namespace ws_detail {
@@ -70,18 +87,19 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar)
 }
 
 // elu(x)+1 on two packed bf16 values: max(x,0) + 2^(min(x,0) log2 e).  The
-// exponent argument is formed in fp32 and rounded once to bf16; the packed
-// exp2 returns bf16, the precision the MMA consumes.
+// exponent argument min(x,0) * log2 e is formed with log2 e split into a bf16
+// head (1.4453125) and tail (-0.00262451), as fma(n, head, n * tail), so it is
+// rounded once; the packed exp2 returns bf16, the precision the MMA consumes.
 __device__ __forceinline__ uint32_t elu1_bf16x2(uint32_t x)
 {
     const uint32_t zero = 0u;
-    uint32_t neg, pos;
+    const uint32_t l2e_hi = 0x3FB93FB9u;   // bf16(1.4453125) in both halves
+    const uint32_t l2e_lo = 0xBB2CBB2Cu;   // bf16(log2 e - 1.4453125) = -0.00262451 in both halves
+    uint32_t neg, pos, t, arg, ex, r;
     asm("min.bf16x2 %0, %1, %2;" : "=r"(neg) : "r"(x), "r"(zero));
     asm("max.bf16x2 %0, %1, %2;" : "=r"(pos) : "r"(x), "r"(zero));
-    const float lo = __uint_as_float(neg << 16) * 1.4426950408889634f;
-    const float hi = __uint_as_float(neg & 0xFFFF0000u) * 1.4426950408889634f;
-    uint32_t arg, ex, r;
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(arg) : "f"(hi), "f"(lo));
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(t) : "r"(neg), "r"(l2e_lo));
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(arg) : "r"(neg), "r"(l2e_hi), "r"(t));
     asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(ex) : "r"(arg));
     asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(pos), "r"(ex));
     return r;
@@ -110,23 +128,23 @@ fwd_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     using namespace sm100;
     using namespace fwd_detail;
     using namespace ws_detail;
-    using Cfg = WsCfg64;
+    using Cfg = WsCfg64<MODE>;
     constexpr int C = Cfg::C, NA = Cfg::NA, DV = Cfg::DV, NS = Cfg::NS, FP = Cfg::DQK;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
     uint64_t *full = bars + 0;       // [NS] TMA landed
-    uint64_t *empty = bars + 2;      // [NS] stage released by the last MMA reading it
-    uint64_t *phi_done = bars + 4;   // [NS] phi written (4 warp arrivals)
-    uint64_t *a_full = bars + 6;     // [2] MMA1 done
-    uint64_t *p_full = bars + 8;     // [2] P written, A read (4)
-    uint64_t *o_full = bars + 10;    // [2] MMA2 done
-    uint64_t *o_free = bars + 12;    // [2] O read (4)
-    uint64_t *snap_full = bars + 14; // [2] S_snap written (4)
-    uint64_t *ds_full = bars + 16;   // MMA3 done
-    uint64_t *ds_free = bars + 17;   // dS read (4)
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 18);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 19);
+    uint64_t *empty = bars + 4;      // [NS] stage released by the last MMA reading it
+    uint64_t *phi_done = bars + 8;   // [NS] phi written (4 warp arrivals)
+    uint64_t *a_full = bars + 12;    // [2] MMA1 done
+    uint64_t *p_full = bars + 14;    // [2] P written, A read (4)
+    uint64_t *o_full = bars + 16;    // [2] MMA2 done
+    uint64_t *o_free = bars + 18;    // [2] O read (4)
+    uint64_t *snap_full = bars + 20; // [2] S_snap written (4)
+    uint64_t *ds_full = bars + 22;   // MMA3 done
+    uint64_t *ds_free = bars + 23;   // dS read (4)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 24);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 25);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bh = blockIdx.x / p.P, seg = blockIdx.x % p.P;
@@ -140,7 +158,7 @@ fwd_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
-            mbar_init(&phi_done[s], 4);
+            mbar_init(&phi_done[s], MODE == 0 ? 6 : 4);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&a_full[b], 1);
@@ -161,7 +179,7 @@ fwd_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     // Normaliser block of each stage's V_aug: column 0 = 1 (overall column 64).
     if (tid < 128)
         for (int s = 0; s < NS; ++s) {
-            uint8_t *blk = smem + Cfg::OFF_STAGE + s * Cfg::STAGE + 2 * Cfg::QK_TILE + (DV / 16) * Cfg::V_BLK;
+            uint8_t *blk = smem + Cfg::OFF_STAGE + s * Cfg::STAGE + Cfg::OFF_V + (DV / 16) * Cfg::V_BLK;
             const int r = tid;
             uint4 *row = reinterpret_cast<uint4 *>(blk + (r >> 3) * 256 + (r & 7) * 32);
             const int one_chunk = (r >> 2) & 1;
@@ -173,6 +191,7 @@ fwd_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    if (tid == 0) LA_TL(13, 0);
 
     auto stage_ptr = [&](int s) { return smem + Cfg::OFF_STAGE + s * Cfg::STAGE; };
     auto fail = [&]() { *abort_flag = 1; };
@@ -180,16 +199,26 @@ fwd_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
+            auto prefetch = [&](int it) {
+                const int t0 = (c_begin + it) * C;
+                if (MODE == 0) tma_prefetch_3d(&tm_q, 0, t0, bh);
+                tma_prefetch_3d(&tm_k, 0, t0, bh);
+                for (int x = 0; x < DV; x += 16) tma_prefetch_3d(&tm_v, x, t0, bh);
+            };
             for (int it = 0; it < nit && !*abort_flag; ++it) {
+                if (it == NS)
+                    for (int j = NS; j < nit && j < NS + Cfg::PREFETCH; ++j) prefetch(j);
                 const int s = it % NS;
                 if (it >= NS && !mbar_wait(&empty[s], ((it / NS) - 1) & 1)) { fail(); break; }
                 const int t0 = (c_begin + it) * C;
                 uint8_t *st = stage_ptr(s);
-                mbar_arrive_expect_tx(&full[s], MODE == 0 ? Cfg::TX_BYTES : Cfg::TX_BYTES - Cfg::QK_TILE);
-                if (MODE == 0) tma_load_3d(st, &tm_q, &full[s], 0, t0, bh);
-                tma_load_3d(st + Cfg::QK_TILE, &tm_k, &full[s], 0, t0, bh);
+                LA_TL(0, it);
+                mbar_arrive_expect_tx(&full[s], Cfg::TX_BYTES);
+                if (MODE == 0) tma_load_3d(st + Cfg::OFF_Q, &tm_q, &full[s], 0, t0, bh);
+                tma_load_3d(st + Cfg::OFF_K, &tm_k, &full[s], 0, t0, bh);
                 for (int x = 0; x < DV; x += 16)
-                    tma_load_3d(st + 2 * Cfg::QK_TILE + (x / 16) * Cfg::V_BLK, &tm_v, &full[s], x, t0, bh);
+                    tma_load_3d(st + Cfg::OFF_V + (x / 16) * Cfg::V_BLK, &tm_v, &full[s], x, t0, bh);
+                if (it + NS + Cfg::PREFETCH < nit) prefetch(it + NS + Cfg::PREFETCH);
             }
         }
     } else if (warp == 1) {
@@ -203,8 +232,10 @@ fwd_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 const int s = it % NS;
                 if (!mbar_wait(&full[s], (it / NS) & 1)) return false;
                 if (!mbar_wait(&phi_done[s], (it / NS) & 1)) return false;
+                LA_TL(1, it);
                 tc_fence_after();
-                const uint32_t aQ = smem_addr(stage_ptr(s)), aK = aQ + Cfg::QK_TILE, aV = aK + Cfg::QK_TILE;
+                const uint32_t st = smem_addr(stage_ptr(s));
+                const uint32_t aQ = st + Cfg::OFF_Q, aK = st + Cfg::OFF_K, aV = st + Cfg::OFF_V;
                 if (MODE == 0) {
                     const uint32_t dA = tmem + Cfg::COL_A + (it & 1) * 128;
 #pragma unroll
@@ -212,18 +243,18 @@ fwd_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         mma_bf16(dA, smem_desc(aQ + kk * 32, 16, 1024, kSw128), smem_desc(aK + kk * 32, 16, 1024, kSw128),
                                  id_qk, kk > 0);
                     mma_commit(&a_full[it & 1]);
-                    if (it >= 1) {
-                        if (!mbar_wait(ds_free, (it - 1) & 1)) return false;
-                        tc_fence_after();
-                    }
+                    if (!mbar_wait(ds_free, it & 1)) return false;   // S(it-1) read / initial state stored
+                    tc_fence_after();
                 }
-                const bool acc_prev = (MODE == 1) && it > 0;  // MODE 1 sums the whole segment
+                // MODE 0 accumulates onto the state in TMEM; MODE 1 sums the segment from zero
+                const bool acc_prev = (MODE == 0) || it > 0;
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
                     mma_bf16(tmem + Cfg::COL_DS, smem_desc(aK + kk * 2048, C * 128, 1024, kSw128),
                              smem_desc(aV + kk * 512, Cfg::V_BLK, 256, kSw32), id_s, acc_prev || kk > 0);
                 if (MODE == 0) mma_commit(ds_full);
                 else mma_commit(&empty[s]);
+                LA_TL(2, it);
                 return true;
             };
             // Y(it): output of chunk it
@@ -232,71 +263,123 @@ fwd_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 if (!mbar_wait(&p_full[b], (it >> 1) & 1)) return false;
                 if (!mbar_wait(&snap_full[it & 1], (it >> 1) & 1)) return false;   // snapshot index it
                 if (it >= 2 && !mbar_wait(&o_free[b], ((it >> 1) - 1) & 1)) return false;
+                LA_TL(3, it);
                 tc_fence_after();
-                const uint32_t aQ = smem_addr(stage_ptr(s)), aV = aQ + 2 * Cfg::QK_TILE;
-                const uint32_t aP = smem_addr(smem + Cfg::OFF_P + b * Cfg::P_TILE);
+                const uint32_t st = smem_addr(stage_ptr(s));
+                const uint32_t aQ = st + Cfg::OFF_Q, aV = st + Cfg::OFF_V;
+                const uint32_t tP = tmem + Cfg::COL_A + b * 128;   // P(it), bf16 pairs per column
                 const uint32_t aS = smem_addr(smem + Cfg::OFF_S + (it & 1) * Cfg::S_TILE);
                 const uint32_t dO = tmem + Cfg::COL_O + b * NA;
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
-                    mma_bf16(dO, smem_desc(aP + (kk >> 2) * (C * 128) + (kk & 3) * 32, 16, 1024, kSw128),
-                             smem_desc(aV + kk * 512, Cfg::V_BLK, 256, kSw32), id_o, kk > 0);
+                    mma_bf16_ts(dO, tP + kk * 8, smem_desc(aV + kk * 512, Cfg::V_BLK, 256, kSw32), id_o, kk > 0);
 #pragma unroll
                 for (int kk = 0; kk < FP / 16; ++kk)
                     mma_bf16(dO, smem_desc(aQ + kk * 32, 16, 1024, kSw128),
                              smem_desc(aS + kk * 512, Cfg::S_BLK, 256, kSw32), id_o, true);
                 mma_commit(&o_full[b]);
                 mma_commit(&empty[s]);
+                LA_TL(4, it);
                 return true;
             };
-            bool ok = nit > 0 ? issue_x(0) : true;
-            for (int it = 0; it < nit && ok && !*abort_flag; ++it) {
-                if (it + 1 < nit) ok = issue_x(it + 1);
-                if (ok && MODE == 0) ok = issue_y(it);
+            bool ok = true;
+            if (MODE == 1) {
+                for (int it = 0; it < nit && ok && !*abort_flag; ++it) ok = issue_x(it);
+                if (ok) mma_commit(ds_full);   // segment increment complete
+            } else {
+                // Issue whichever of Y(ny) (output of the oldest pending chunk) and
+                // X(nx) (scores and increment of the next chunk) has its inputs
+                // ready, preferring Y; give up after 2 s without progress.
+                auto x_ready = [&](int it) {
+                    const int s = it % NS;
+                    return mbar_test(&full[s], (it / NS) & 1) && mbar_test(&phi_done[s], (it / NS) & 1) &&
+                           mbar_test(ds_free, it & 1);
+                };
+                auto y_ready = [&](int it) {
+                    const int b = it & 1;
+                    return mbar_test(&p_full[b], (it >> 1) & 1) && mbar_test(&snap_full[b], (it >> 1) & 1) &&
+                           (it < 2 || mbar_test(&o_free[b], ((it >> 1) - 1) & 1));
+                };
+                int nx = 0, ny = 0;
+                uint64_t t_last;
+                asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_last));
+                while (ny < nit && ok && !*abort_flag) {
+                    bool progress = false;
+                    if (ny < nx && y_ready(ny)) {
+                        ok = issue_y(ny++);
+                        progress = true;
+                    } else if (nx < nit && nx <= ny + 1 && x_ready(nx)) {
+                        ok = issue_x(nx++);
+                        progress = true;
+                    }
+                    uint64_t t;
+                    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+                    if (progress) {
+                        t_last = t;
+                    } else if (t - t_last > 2000000000ull) {
+                        report(kStatusTimeout);
+                        ok = false;
+                    } else {
+                        __nanosleep(64);   // leave issue slots to the warps sharing this SMSP
+                    }
+                }
             }
-            if (ok && MODE == 1) mma_commit(ds_full);   // segment increment complete
             if (!ok) fail();
         }
-    } else if (warp >= 4 && warp < 8) {
+    } else if ((MODE == 0 && warp >= 2 && warp < 8) || (MODE == 1 && warp >= 4 && warp < 12)) {
         // ---------------------------------------------------------------- phi
-        const int i = tid - 128;
-        for (int it = 0; it < nit && !*abort_flag; ++it) {
+        // elu(x)+1 in place.  MODE 0: warps 2-7 (192 threads) share the 512
+        // half-rows (32 values) of the Q and K tiles of every chunk.  MODE 1:
+        // only K; warps 4-7 take even chunks and warps 8-11 odd ones, a row
+        // per thread.
+        const int first = (MODE == 1 && warp >= 8) ? 1 : 0;
+        const int step = MODE == 1 ? 2 : 1;
+        const int pt = MODE == 0 ? tid - 64 : (tid & 127);   // 0..191 or 0..127
+        for (int it = first; it < nit && !*abort_flag; it += step) {
             const int s = it % NS;
             if (!mbar_wait(&full[s], (it / NS) & 1)) { fail(); break; }
+            if (pt == 0) LA_TL(5, it);
             const int t0 = (c_begin + it) * C;
-            const bool kvalid = t0 + i < N;
             const uint32_t base = smem_addr(stage_ptr(s));
+            auto half_row = [&](int m, int row, int h) {
+                const uint32_t tile = base + (m == 0 ? Cfg::OFF_Q : Cfg::OFF_K);
+                const bool zero = (m == 1) && (t0 + row >= N);
+                uint4 raw[4];
 #pragma unroll
-            for (int m = (MODE == 0 ? 0 : 1); m < 2; ++m) {
-                const uint32_t tile = base + m * Cfg::QK_TILE;
-                const bool zero = (m == 1) && !kvalid;
-                uint4 raw[8];
+                for (int cc = 0; cc < 4; ++cc) raw[cc] = lds128(tile + sw128_off(row, (h * 4 + cc) * 8));
 #pragma unroll
-                for (int cc = 0; cc < 8; ++cc) raw[cc] = lds128(tile + sw128_off(i, cc * 8));
-#pragma unroll
-                for (int cc = 0; cc < 8; ++cc) {
+                for (int cc = 0; cc < 4; ++cc) {
                     uint4 r = raw[cc];
                     r = zero ? make_uint4(0u, 0u, 0u, 0u)
                              : make_uint4(elu1_bf16x2(r.x), elu1_bf16x2(r.y), elu1_bf16x2(r.z), elu1_bf16x2(r.w));
-                    sts128(tile + sw128_off(i, cc * 8), r);
+                    sts128(tile + sw128_off(row, (h * 4 + cc) * 8), r);
                 }
+            };
+            if (MODE == 0) {
+                for (int item = pt; item < 2 * C * 2; item += 192)   // item = (tile, row, half)
+                    half_row(item >> 8, (item >> 1) & (C - 1), item & 1);
+            } else {
+                half_row(1, pt, 0);
+                half_row(1, pt, 1);
             }
             fence_proxy_async();
             __syncwarp();
+            if (pt == 0) LA_TL(6, it);
             if (lane == 0) mbar_arrive(&phi_done[s]);
         }
     } else if (warp >= 8 && warp < 12) {
         // --------------------------------------------------------------- mask
-        if (MODE == 0) {
+        {
             const int i = tid - 256;
             const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
             for (int it = 0; it < nit && !*abort_flag; ++it) {
                 const int b = it & 1;
                 if (!mbar_wait(&a_full[b], (it >> 1) & 1)) { fail(); break; }
-                // P[b] was last read by MMA2(it-2)
-                if (it >= 2 && !mbar_wait(&o_full[b], ((it >> 1) - 1) & 1)) { fail(); break; }
+                // P(it) overwrites the first 64 columns of A[b]: MMA2(it-2), the
+                // last reader of the P in this buffer, finished before MMA1(it)
+                // (MMAs execute in issue order).
+                if (i == 0) LA_TL(7, it);
                 tc_fence_after();
-                const uint32_t aP = smem_addr(smem + Cfg::OFF_P + b * Cfg::P_TILE);
                 const uint32_t tA = tmem + lane_base + Cfg::COL_A + b * 128;
 #pragma unroll 1
                 for (int j0 = 0; j0 < C; j0 += 64) {
@@ -304,108 +387,144 @@ fwd_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     tmem_ld32(tA + j0, a);
                     tmem_ld32(tA + j0 + 32, a + 32);
                     tmem_ld_wait();
+                    uint32_t pk[32];
 #pragma unroll
-                    for (int e = 0; e < 64; e += 8) {
-                        float w[8];
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) w[u] = (j0 + e + u <= i) ? a[e + u] : 0.f;
-                        sts128(aP + sw128_off(i, j0 + e),
-                               make_uint4(pack_bf16(w[0], w[1]), pack_bf16(w[2], w[3]), pack_bf16(w[4], w[5]),
-                                          pack_bf16(w[6], w[7])));
-                    }
+                    for (int e = 0; e < 64; e += 2)
+                        pk[e / 2] = pack_bf16((j0 + e <= i) ? a[e] : 0.f, (j0 + e + 1 <= i) ? a[e + 1] : 0.f);
+                    tmem_st32(tA + j0 / 2, pk);
                 }
-                fence_proxy_async();
+                tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
+                if (i == 0) LA_TL(8, it);
                 if (lane == 0) mbar_arrive(&p_full[b]);
             }
         }
     } else if (warp >= 12) {
         // ------------------------------------------------- state and output
+        // The running state S_aug lives in TMEM (COL_DS, feature rows in the
+        // lanes of the M = 64 layout); MMA3 accumulates each chunk into it.
         const int wq = warp & 3;
         const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
-        const int f = wq * 16 + lane;            // feature row of dS held by this lane (lane < 16)
+        const uint32_t tS = tmem + lane_base + Cfg::COL_DS;
+        const int f = wq * 16 + lane;            // feature row held by this lane (lane < 16)
         const bool frow = lane < 16;
-        float S[NA];
-#pragma unroll
-        for (int e = 0; e < NA; ++e) S[e] = 0.f;
-        if (MODE == 0 && seg > 0 && frow) {
-            for (int s2 = 0; s2 < seg; ++s2) {
-                const float *src = p.ws + ((size_t)(bh * p.P + s2) * FP + f) * NA;
-#pragma unroll
-                for (int e = 0; e < NA; ++e) S[e] += src[e];
-            }
-        }
-        auto write_snap = [&](int j) {   // snapshot j = state before chunk j, buffer j & 1
+        // snapshot j = state before chunk j (bf16, buffer j & 1) from 16-column batches
+        auto snap_cols = [&](int j, int c0, const float *v) {
             if (frow) {
                 const uint32_t aS = smem_addr(smem + Cfg::OFF_S + (j & 1) * Cfg::S_TILE);
-#pragma unroll
-                for (int c0 = 0; c0 < NA; c0 += 8)
-                    sts128(aS + sw32_off(f, c0, FP),
-                           make_uint4(pack_bf16(S[c0], S[c0 + 1]), pack_bf16(S[c0 + 2], S[c0 + 3]),
-                                      pack_bf16(S[c0 + 4], S[c0 + 5]), pack_bf16(S[c0 + 6], S[c0 + 7])));
+                sts128(aS + sw32_off(f, c0, FP), make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
+                                                            pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7])));
+                sts128(aS + sw32_off(f, c0 + 8, FP),
+                       make_uint4(pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]), pack_bf16(v[12], v[13]),
+                                  pack_bf16(v[14], v[15])));
             }
+        };
+        auto snap_done = [&](int j) {
             fence_proxy_async();
             __syncwarp();
             if (lane == 0) mbar_arrive(&snap_full[j & 1]);
         };
         if (MODE == 0) {
-            write_snap(0);
+            // initial state: the sum of the earlier segments' increments, or zero
+            for (int c0 = 0; c0 < NA; c0 += 16) {
+                float v[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) v[e] = 0.f;
+                if (seg > 0 && frow)
+                    for (int s2 = 0; s2 < seg; ++s2) {
+                        const float *src = p.ws + ((size_t)(bh * p.P + s2) * FP + f) * NA + c0;
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) v[e] += src[e];
+                    }
+                tmem_st16(tS + c0, v);
+                snap_cols(0, c0, v);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(ds_free);   // completion 0: initial state in TMEM
+            snap_done(0);
             for (int it = 0; it < nit && !*abort_flag; ++it) {
-                // dS(it) -> S, snapshot it+1 (buffer last read by MMA2(it-1), already complete)
+                // state after chunk it -> snapshot it+1 (its buffer was last read by
+                // MMA2(it-1), complete since the output of chunk it-1 was taken)
                 if (!mbar_wait(ds_full, it & 1)) { fail(); break; }
+                if (tid == 384) LA_TL(9, it);
                 tc_fence_after();
+                if (it + 1 < nit) {
 #pragma unroll
-                for (int c0 = 0; c0 < NA; c0 += 16) {
-                    float d[16];
-                    tmem_ld16(tmem + lane_base + Cfg::COL_DS + c0, d);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) S[c0 + e] += d[e];
+                    for (int c0 = 0; c0 < NA; c0 += 48) {
+                        float v[48];
+                        tmem_ld16(tS + c0, v);
+                        tmem_ld16(tS + c0 + 16, v + 16);
+                        if (c0 + 32 < NA) tmem_ld16(tS + c0 + 32, v + 32);
+                        tmem_ld_wait();
+                        snap_cols(it + 1, c0, v);
+                        snap_cols(it + 1, c0 + 16, v + 16);
+                        if (c0 + 32 < NA) snap_cols(it + 1, c0 + 32, v + 32);
+                    }
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(ds_free);
-                if (it + 1 < nit) write_snap(it + 1);
+                if (lane == 0) mbar_arrive(ds_free);   // completion it+1: S(it) read
+                if (it + 1 < nit) snap_done(it + 1);
+                if (tid == 384) LA_TL(10, it);
                 // output of chunk it
                 const int b = it & 1;
                 if (!mbar_wait(&o_full[b], (it >> 1) & 1)) { fail(); break; }
+                if (tid == 384) LA_TL(11, it);
                 tc_fence_after();
                 const int t0 = (c_begin + it) * C;
                 const int row = wq * 32 + lane;
-                float den[16];
-                tmem_ld16(tmem + lane_base + Cfg::COL_O + b * NA + DV, den);
+                const uint32_t tO = tmem + lane_base + Cfg::COL_O + b * NA;
+                float o[48];
+                tmem_ld16(tO + DV, o + 32);          // den in column 64
+                tmem_ld16(tO, o);
+                tmem_ld16(tO + 16, o + 16);
                 tmem_ld_wait();
-                const float inv = 1.f / den[0];
+                const float den0 = o[32];
+                const float inv = 1.f / den0;
                 __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + ((size_t)bh * N + t0 + row) * DV;
                 const bool valid = t0 + row < N;
 #pragma unroll
-                for (int c0 = 0; c0 < DV; c0 += 16) {
-                    float o[16];
-                    tmem_ld16(tmem + lane_base + Cfg::COL_O + b * NA + c0, o);
-                    tmem_ld_wait();
+                for (int half = 0; half < 2; ++half) {
+                    if (half == 1) {
+                        tmem_ld16(tO + 32, o);
+                        tmem_ld16(tO + 48, o + 16);
+                        tmem_ld_wait();
+                    }
                     if (valid) {
-                        *reinterpret_cast<uint4 *>(orow + c0) =
-                            make_uint4(pack_bf16(o[0] * inv, o[1] * inv), pack_bf16(o[2] * inv, o[3] * inv),
-                                       pack_bf16(o[4] * inv, o[5] * inv), pack_bf16(o[6] * inv, o[7] * inv));
-                        *reinterpret_cast<uint4 *>(orow + c0 + 8) =
-                            make_uint4(pack_bf16(o[8] * inv, o[9] * inv), pack_bf16(o[10] * inv, o[11] * inv),
-                                       pack_bf16(o[12] * inv, o[13] * inv), pack_bf16(o[14] * inv, o[15] * inv));
+#pragma unroll
+                        for (int c0 = 0; c0 < 32; c0 += 8)
+                            *reinterpret_cast<uint4 *>(orow + half * 32 + c0) =
+                                make_uint4(pack_bf16(o[c0] * inv, o[c0 + 1] * inv), pack_bf16(o[c0 + 2] * inv, o[c0 + 3] * inv),
+                                           pack_bf16(o[c0 + 4] * inv, o[c0 + 5] * inv), pack_bf16(o[c0 + 6] * inv, o[c0 + 7] * inv));
                     }
                 }
-                if (valid && p.den_out) p.den_out[(size_t)bh * N + t0 + row] = den[0];
+                if (valid && p.den_out) p.den_out[(size_t)bh * N + t0 + row] = den0;
                 tc_fence_before();
                 __syncwarp();
+                if (tid == 384) LA_TL(12, it);
                 if (lane == 0) mbar_arrive(&o_free[b]);
             }
-            // final state of the sequence (last segment only)
-            if (seg == p.P - 1 && frow && !*abort_flag) {
-                if (p.s_out) {
-                    float *dst = p.s_out + ((size_t)bh * FP + f) * DV;
+            // final state of the sequence (last segment only): S after the last chunk
+            if (seg == p.P - 1 && (p.s_out || p.z_out) && !*abort_flag) {
+#pragma unroll 1
+                for (int c0 = 0; c0 < NA; c0 += 16) {
+                    float v[16];
+                    tmem_ld16(tS + c0, v);
+                    tmem_ld_wait();
+                    if (!frow) continue;
 #pragma unroll
-                    for (int e = 0; e < DV; ++e) dst[e] = S[e];
+                    for (int e = 0; e < 16; ++e) {
+                        const int col = c0 + e;
+                        if (col < DV) {
+                            if (p.s_out) p.s_out[((size_t)bh * FP + f) * DV + col] = v[e];
+                        } else if (col == DV && p.z_out) {
+                            p.z_out[(size_t)bh * FP + f] = v[e];
+                        }
+                    }
                 }
-                if (p.z_out) p.z_out[(size_t)bh * FP + f] = S[DV];
             }
         } else {
             // MODE 1: the accumulated increment of this segment -> workspace
@@ -416,7 +535,7 @@ fwd_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
                     for (int c0 = 0; c0 < NA; c0 += 16) {
                         float d[16];
-                        tmem_ld16(tmem + lane_base + Cfg::COL_DS + c0, d);
+                        tmem_ld16(tS + c0, d);
                         tmem_ld_wait();
                         if (frow)
 #pragma unroll
