@@ -352,7 +352,7 @@ def e2e_prefill(w, dev, steps, warmup):
 
 # ----------------------------------------------------------------- CPU oracle
 
-def oracle_sample(w, heads=None, positions=None):
+def oracle_sample(w, heads=None, positions=None, min_cpu_s=0.0):
     """Time the fp64 oracle on a bounded sample of workload w; returns
     (tokens/s extrapolated to the full workload, seconds, description)."""
     from oracle import oracle as orc
@@ -363,26 +363,37 @@ def oracle_sample(w, heads=None, positions=None):
     g.manual_seed(w.index)
     mk = lambda d: (torch.randn(1, Hs, Ns, d, generator=g) * w.scale).to(w.torch_dtype)
     q, k, v = mk(w.dqk), mk(w.dqk), mk(w.dv)
+    do = mk(w.dv) if w.backward else None
+
+    def once():
+        if w.backward:
+            orc.forward_recurrent(w.fmap, q, k, v)
+            orc.backward_recurrent(w.fmap, q, k, v, do)
+        elif w.decode_steps:
+            F = w.feature_dim
+            import numpy as np
+            s = np.zeros((Hs, F, w.dv)); z = np.zeros((Hs, F))
+            for t in range(Ns):
+                orc.decode_step(w.fmap, q[0, :, t], k[0, :, t], v[0, :, t], s, z)
+        else:
+            orc.forward_recurrent(w.fmap, q, k, v)
+
+    # repeat the sample until it amounts to about min_cpu_s of CPU time
+    reps = 0
     t0 = time.perf_counter()
-    if w.backward:
-        do = mk(w.dv)
-        orc.forward_recurrent(w.fmap, q, k, v)
-        orc.backward_recurrent(w.fmap, q, k, v, do)
-    elif w.decode_steps:
-        F = w.feature_dim
-        import numpy as np
-        s = np.zeros((Hs, F, w.dv)); z = np.zeros((Hs, F))
-        for t in range(Ns):
-            orc.decode_step(w.fmap, q[0, :, t], k[0, :, t], v[0, :, t], s, z)
-    else:
-        orc.forward_recurrent(w.fmap, q, k, v)
-    dt = time.perf_counter() - t0
+    c0 = time.process_time()
+    while True:
+        once()
+        reps += 1
+        if time.process_time() - c0 >= min_cpu_s or time.perf_counter() - t0 >= 60:
+            break
+    dt = (time.perf_counter() - t0) / reps
     frac = (Hs * Ns) / (w.B * w.H * (w.decode_steps if w.decode_steps else w.N))
     full_tokens = w.B * (w.decode_steps if w.decode_steps else w.N)
     desc = (f"fp64 oracle ({'decode steps' if w.decode_steps else 'recurrent form'}"
             f"{' + backward' if w.backward else ''}) on {Hs} of {w.B * w.H} heads x {Ns} positions; "
-            f"tokens/s scaled to the full workload by head-token count")
-    return full_tokens * frac / dt, dt, desc
+            f"tokens/s scaled to the full workload by head-token count; {reps} repetitions")
+    return full_tokens * frac / dt, dt * reps, desc
 
 
 def omp_threads():
@@ -525,9 +536,9 @@ def main():
         line["workloads"] = sec
 
     if rank == 0 and world == 1 and not args.no_cpu:
-        v, dt, desc = oracle_sample(w)
+        v, dt, desc = oracle_sample(w, min_cpu_s=15.0)
         line["cpu_baseline"] = {"value": round(v, 1), "unit": "tokens/s", "cores": omp_threads(),
-                                "kind": "oracle", "sample": desc + f" ({dt:.1f} s)"}
+                                "kind": "oracle", "sample": desc + f" ({dt:.1f} s wall)"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist_on:

@@ -17,6 +17,7 @@
 #include "la_decode.cuh"
 #include "la_prefill_sm100.cuh"
 #include "la_fwd_ws_sm100.cuh"
+#include "la_bwd_sm100.cuh"
 
 using namespace la;
 
@@ -86,7 +87,7 @@ la_status set_smem(size_t bytes)
 }
 
 // Kernel selection, shared by the entry points and la_kernel_plan.
-enum class Path { Invalid, FwdSimt, FwdTc, BwdSimt, DecodeSimt, DecodeVec };
+enum class Path { Invalid, FwdSimt, FwdTc, BwdSimt, BwdTc, DecodeSimt, DecodeVec };
 
 // Shapes with a tensor-core forward: bf16 I/O and (elu, dqk = dv in {64,128})
 // or (Taylor, dqk = 16, dv = 64).
@@ -132,6 +133,7 @@ int64_t tc_increment_floats(int dqk, int dv, int fmap)
 Path select_backward(int B, int H, int N, int dqk, int dv, int fmap, int dtype)
 {
     if (check_shape(B, H, N, dqk, dv, fmap, dtype) != LA_OK) return Path::Invalid;
+    if (dtype == LA_BF16 && fmap == LA_FMAP_ELU1 && dqk == 128 && dv == 128) return Path::BwdTc;
     return Path::BwdSimt;
 }
 
@@ -149,6 +151,7 @@ int path_kernels(Path p, const char **names)
     case Path::FwdSimt: names[0] = "fwd_simt_kernel"; return 1;
     case Path::FwdTc: names[0] = "fwd_tc_kernel"; return 1;  // plus the segment pass, see below
     case Path::BwdSimt: names[0] = "bwd_simt_kernel"; return 1;
+    case Path::BwdTc: names[0] = "bwd_dq_kernel"; names[1] = "bwd_dkdv_kernel"; return 2;
     case Path::DecodeSimt: names[0] = "decode_simt_kernel"; return 1;
     case Path::DecodeVec: names[0] = "decode_vec_kernel"; return 1;
     default: return -1;
@@ -342,6 +345,46 @@ la_status forward_tc(const void *q, const void *k, const void *v, void *o, float
     return forward_tc_launch<FwdCfg<128, 128, false>>(q, k, v, o, s_out, z_out, den_out, workspace, B, H, N, stream);
 }
 
+la_status backward_tc(const void *q, const void *k, const void *v, const void *dout, void *dq, void *dk,
+                      void *dvp, void *workspace, int B, int H, int N, cudaStream_t stream)
+{
+    using Cfg = BwdCfg128;
+    const int BH = B * H;
+    CUtensorMap tq, tk, tv, tdo;
+    if (!make_map(&tq, q, 128, N, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tk, k, 128, N, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tv, v, 128, N, BH, 16, CU_TENSOR_MAP_SWIZZLE_32B) ||
+        !make_map(&tdo, dout, 128, N, BH, 16, CU_TENSOR_MAP_SWIZZLE_32B))
+        return LA_ERR_CUDA;
+    BwdParams p;
+    tc_segments(B, H, N, &p.P, &p.cps, &p.nchunks);
+    p.N = N;
+    p.dd = (float *)workspace;
+    float *ws_s = p.dd + (size_t)BH * N * 2;
+    float *ws_r = ws_s + (size_t)BH * p.P * Cfg::F * Cfg::NA;
+    p.ws_s = ws_s;
+    p.ws_r = ws_r;
+    p.dq = dq;
+    p.dk = dk;
+    p.dv = dvp;
+    if (set_smem<bwd_sstate_kernel>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
+    if (p.P > 1) {
+        bwd_sstate_kernel<<<BH * p.P, 128, Cfg::SMEM_ALLOC, stream>>>(tk, tv, p);
+        if (launch_status() != LA_OK) return LA_ERR_CUDA;
+    }
+    if (set_smem<bwd_dq_kernel>(Cfg::SMEM_ALLOC) != LA_OK || set_smem<bwd_dkdv_kernel>(Cfg::SMEM_ALLOC) != LA_OK ||
+        set_smem<bwd_rstate_kernel>(Cfg::SMEM_ALLOC) != LA_OK)
+        return LA_ERR_CUDA;
+    bwd_dq_kernel<<<BH * p.P, 128, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, p);
+    if (launch_status() != LA_OK) return LA_ERR_CUDA;
+    if (p.P > 1) {
+        bwd_rstate_kernel<<<BH * p.P, 128, Cfg::SMEM_ALLOC, stream>>>(tq, tdo, p);
+        if (launch_status() != LA_OK) return LA_ERR_CUDA;
+    }
+    bwd_dkdv_kernel<<<BH * p.P, 128, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, p);
+    return launch_status();
+}
+
 }  // namespace
 
 extern "C" {
@@ -381,8 +424,15 @@ size_t la_forward_workspace_bytes(int B, int H, int N, int dqk, int dv, int fmap
 
 size_t la_backward_workspace_bytes(int B, int H, int N, int dqk, int dv, int fmap, int dtype)
 {
-    if (check_shape(B, H, N, dqk, dv, fmap, dtype) != LA_OK) return 0;
-    return (size_t)B * H * N * 2 * sizeof(float);  // den_i, dden_i
+    const Path path = select_backward(B, H, N, dqk, dv, fmap, dtype);
+    if (path == Path::Invalid) return 0;
+    size_t bytes = (size_t)B * H * N * 2 * sizeof(float);  // den_i, dden_i
+    if (path == Path::BwdTc) {
+        int P, cps, nc;
+        tc_segments(B, H, N, &P, &cps, &nc);
+        if (P > 1) bytes += 2 * (size_t)B * H * P * BwdCfg128::F * BwdCfg128::NA * sizeof(float);  // S, R increments
+    }
+    return bytes;
 }
 
 la_status la_forward(const void *q, const void *k, const void *v, void *o, float *s_out,
@@ -465,6 +515,8 @@ la_status la_backward(const void *q, const void *k, const void *v, const void *d
         return LA_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
     float *ws = (float *)workspace;
+    if (select_backward(B, H, N, dqk, dv, fmap, dtype) == Path::BwdTc)
+        return backward_tc(q, k, v, dout, dq, dk, dvp, workspace, B, H, N, s);
     if (dtype == LA_F32)
         return backward_simt<float>(q, k, v, dout, dq, dk, dvp, ws, B, H, N, dqk, dv, fmap, s);
     return backward_simt<__nv_bfloat16>(q, k, v, dout, dq, dk, dvp, ws, B, H, N, dqk, dv, fmap, s);
@@ -528,6 +580,17 @@ int la_kernel_plan(int op, int B, int H, int N, int dqk, int dv, int fmap, int d
         return P > 1 ? 2 : 1;
     }
     else if (op == 1) p = select_backward(B, H, N, dqk, dv, fmap, dtype);
+    if (p == Path::BwdTc) {
+        int P, cps, nc;
+        tc_segments(B, H, N, &P, &cps, &nc);
+        const char *nm = P > 1 ? "bwd_sstate_kernel,bwd_dq_kernel,bwd_rstate_kernel,bwd_dkdv_kernel"
+                               : "bwd_dq_kernel,bwd_dkdv_kernel";
+        if (buf && buflen) {
+            strncpy(buf, nm, buflen - 1);
+            buf[buflen - 1] = 0;
+        }
+        return P > 1 ? 4 : 2;
+    }
     else if (op == 2) p = select_decode(B, H, dqk, dv, fmap, dtype);
     const char *names[8];
     const int n = path_kernels(p, names);

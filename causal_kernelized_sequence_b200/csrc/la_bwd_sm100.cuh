@@ -1,0 +1,966 @@
+// la_bwd_sm100.cuh -- tensor-core backward of causal linear attention for the
+// elu(x)+1 map with d_qk = d_v = 128 (bf16 I/O), tcgen05 + TMA.
+//
+// The pages give no backward pass; this is the derivative of the BASED page's
+// Knowl 3 parallel form, computed chunk by chunk (128 tokens) with the same
+// augmented-value trick as the forward: V_aug = [V | 1 | 0..], S_aug = [S | z],
+// G'_i = [g_i | dden_i | 0..] with g_i = dout_i / den_i, dden_i = -g_i . y_i.
+// Then, for a chunk c with state S_aug entering it and R_aug = sum over the
+// later chunks of phi(q_i) G'_i^T,
+//
+//   forward-order pass (dq), in units of den_i per row i:
+//     A   = phi(Q) phi(K)^T, P = A masked to j <= i
+//     O   = P V_aug + phi(Q) S_aug          -> y, den; G'' = den G' = [dO | -dO.y]
+//     dA  = G'' V_aug^T,  dP = dA masked to j <= i
+//     dphi(Q) = (dP phi(K) + G'' S_aug^T) / den   -> dq = dphi(Q) * elu'(q)
+//     S_aug += phi(K)^T V_aug
+//   reverse-order pass (dk, dv):
+//     A^T = phi(K) phi(Q)^T, P^T; dA^T = V_aug G'^T, dP^T (masked to i >= j)
+//     dV  = P^T G + phi(K) R                 (R = first d_v columns of R_aug)
+//     dphi(K) = dP^T phi(Q) + V_aug R_aug^T  -> dk = dphi(K) * elu'(k)
+//     R_aug += phi(Q)^T G'
+//
+// elu'(x) = 1 for x > 0 and exp(x) = phi(x) otherwise, i.e. min(phi(x), 1).
+// den and dden are recomputed in fp32 in the forward-order pass (so no
+// rounded forward output enters the gradient) and kept per token in the
+// workspace for the reverse pass.  Sequences are split into the forward's
+// segments; segment states come from the forward's state pass (S) and from
+// bwd_rstate_kernel (R), summed over the earlier / later segments.
+//
+// These kernels use one 128-thread warpgroup per block (thread i <-> token or
+// feature row i <-> TMEM lane i) and process a chunk's steps in order; every
+// mbarrier wait is bounded.
+#pragma once
+
+#include "la_device.cuh"
+#include "la_fwd_ws_sm100.cuh"
+#include "la_prefill_sm100.cuh"
+#include "sm100.cuh"
+
+namespace la {
+
+struct BwdCfg128 {
+    static constexpr int C = 128, D = 128, DV = 128, NA = 144, F = 128;
+    static constexpr int QK_TILE = C * D * 2;            // 32 KB (two 64-column SW128 blocks)
+    static constexpr int BLK = C * 32;                   // 4 KB: one 16-column SW32 block of 128 rows
+    static constexpr int VG_TILE = (NA / 16) * BLK;      // 36 KB: V_aug or G'
+    static constexpr int S_BLK = F * 32;                 // 4 KB: 16 columns of the F x NA state
+    static constexpr int S_TILE = (NA / 16) * S_BLK;     // 36 KB
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + QK_TILE;
+    static constexpr int OFF_V = OFF_K + QK_TILE;
+    static constexpr int OFF_G = OFF_V + VG_TILE;
+    static constexpr int OFF_S = OFF_G + VG_TILE;
+    static constexpr int OFF_SL = OFF_S + S_TILE;        // low bf16 part of the state (forward-order pass)
+    static constexpr int OFF_BAR = OFF_SL + S_TILE;
+    static constexpr int SMEM_ALLOC = OFF_BAR + 128 + 1024;
+    static constexpr int TMEM_COLS = 512;
+};
+
+struct BwdParams {
+    float *dd;            // [BH, N, 2]: den_i, dden_i
+    float *ws_s;          // [BH, P, F, NA] state increments per segment
+    float *ws_r;          // [BH, P, F, NA] R increments per segment
+    void *dq, *dk, *dv;   // [BH, N, D] bf16
+    int N, P, nchunks, cps;
+};
+
+namespace bwd_detail {
+
+using namespace sm100;
+using namespace fwd_detail;
+using namespace ws_detail;
+
+// Block barrier that also orders tcgen05 and async-proxy accesses around it.
+__device__ __forceinline__ void full_sync()
+{
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+}
+
+// elu(x)+1 in place on row `row` of a [128 x 128] bf16 SW128 tile; rows at or
+// beyond `nvalid` are zeroed when `zero_tail`.
+__device__ __forceinline__ void phi_row_inplace(uint32_t tile, int row, bool zero)
+{
+#pragma unroll
+    for (int blk = 0; blk < 2; ++blk) {
+        uint4 raw[8];
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) raw[cc] = lds128(tile + sw128_off(row, blk * 64 + cc * 8));
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+            uint4 r = raw[cc];
+            r = zero ? make_uint4(0u, 0u, 0u, 0u)
+                     : make_uint4(elu1_bf16x2(r.x), elu1_bf16x2(r.y), elu1_bf16x2(r.z), elu1_bf16x2(r.w));
+            sts128(tile + sw128_off(row, blk * 64 + cc * 8), r);
+        }
+    }
+}
+
+// Ones column (column DV of V_aug = block DV/16, column 0) for all 128 rows.
+__device__ __forceinline__ void write_ones_block(uint8_t *blk, int r)
+{
+    uint4 *row = reinterpret_cast<uint4 *>(blk + (r >> 3) * 256 + (r & 7) * 32);
+    const int c = (r >> 2) & 1;
+    row[c] = make_uint4(pack_bf16(1.f, 0.f), 0u, 0u, 0u);
+    row[c ^ 1] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+// Row r of the augmentation block of G': [dden, 0, ..., 0].
+__device__ __forceinline__ void write_dden(uint8_t *blk, int r, float dden)
+{
+    uint4 *row = reinterpret_cast<uint4 *>(blk + (r >> 3) * 256 + (r & 7) * 32);
+    const int c = (r >> 2) & 1;
+    row[c] = make_uint4(pack_bf16(dden, 0.f), 0u, 0u, 0u);
+    row[c ^ 1] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+// 16 fp32 values of row f of an F x NA state as bf16 into a snapshot tile
+// (SW32 16-column blocks of F rows); with `lo`, also the rounding remainder
+// v - bf16(v) into a second tile, so hi + lo carries ~16 significant bits.
+template <int F>
+__device__ __forceinline__ void snap_cols(uint32_t a_hi, uint32_t a_lo, int f, int c0, const float *v, bool lo)
+{
+    float r[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) r[e] = v[e] - __bfloat162float(__float2bfloat16_rn(v[e]));
+    sts128(a_hi + sw32_off(f, c0, F), make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
+                                                 pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7])));
+    sts128(a_hi + sw32_off(f, c0 + 8, F), make_uint4(pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]),
+                                                     pack_bf16(v[12], v[13]), pack_bf16(v[14], v[15])));
+    if (lo) {
+        sts128(a_lo + sw32_off(f, c0, F), make_uint4(pack_bf16(r[0], r[1]), pack_bf16(r[2], r[3]),
+                                                     pack_bf16(r[4], r[5]), pack_bf16(r[6], r[7])));
+        sts128(a_lo + sw32_off(f, c0 + 8, F), make_uint4(pack_bf16(r[8], r[9]), pack_bf16(r[10], r[11]),
+                                                         pack_bf16(r[12], r[13]), pack_bf16(r[14], r[15])));
+    }
+}
+
+// Row f (thread) of a state tile [F x NA] fp32 in TMEM (M = 128 layout) to its
+// bf16 snapshot(s).
+template <int F, int NA>
+__device__ __forceinline__ void snapshot_state(uint32_t tS_lane, uint8_t *snap, uint8_t *snap_lo, int f)
+{
+#pragma unroll 1
+    for (int c0 = 0; c0 < NA; c0 += 16) {
+        float v[16];
+        tmem_ld16(tS_lane + c0, v);
+        tmem_ld_wait();
+        snap_cols<F>(smem_addr(snap), snap_lo ? smem_addr(snap_lo) : 0u, f, c0, v, snap_lo != nullptr);
+    }
+}
+
+// Masked scores of one TMEM row (128 fp32 columns at `src`) packed as bf16
+// pairs into 64 columns at `dst` (may alias the first half of src).
+// keep(j) decides which entries survive the causal mask.
+template <typename Keep>
+__device__ __forceinline__ void mask_pack_row(uint32_t src, uint32_t dst, Keep keep)
+{
+#pragma unroll 1
+    for (int j0 = 0; j0 < 128; j0 += 64) {
+        float a[64];
+        tmem_ld32(src + j0, a);
+        tmem_ld32(src + j0 + 32, a + 32);
+        tmem_ld_wait();
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 64; e += 2) pk[e / 2] = pack_bf16(keep(j0 + e) ? a[e] : 0.f, keep(j0 + e + 1) ? a[e + 1] : 0.f);
+        tmem_st32(dst + j0 / 2, pk);
+    }
+    tmem_st_wait();
+}
+
+
+// ---- fp16 operand helpers (the forward-order pass runs its MMAs on fp16)
+
+__device__ __forceinline__ uint32_t pack_f16(float a, float b)
+{
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+__device__ __forceinline__ void unpack8_f16(uint4 u, float *f)
+{
+    const __half2 *h = reinterpret_cast<const __half2 *>(&u);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float2 t = __half22float2(h[k]);
+        f[2 * k] = t.x;
+        f[2 * k + 1] = t.y;
+    }
+}
+
+__device__ __forceinline__ float f16_rem(float x) { return x - __half2float(__float2half_rn(x)); }
+
+// Two bf16 values -> the same values as fp16 (exact inside the fp16 range).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t x)
+{
+    return pack_f16(__uint_as_float(x << 16), __uint_as_float(x & 0xFFFF0000u));
+}
+
+// elu(x)+1 of two bf16 values, as fp16: max(x,0) + 2^(min(x,0) log2 e), the
+// exponent argument rounded once to fp16 and the packed exp2 in fp16 (11
+// significant bits, so phi - 1 keeps ~8 bits for |x| ~ 0.1).
+__device__ __forceinline__ uint32_t elu1_f16x2_from_bf16x2(uint32_t x)
+{
+    const float lo = __uint_as_float(x << 16), hi = __uint_as_float(x & 0xFFFF0000u);
+    const uint32_t arg = pack_f16(fminf(lo, 0.f) * 1.4426950408889634f, fminf(hi, 0.f) * 1.4426950408889634f);
+    const uint32_t pos = pack_f16(fmaxf(lo, 0.f), fmaxf(hi, 0.f));
+    uint32_t ex, r;
+    asm("ex2.approx.f16x2 %0, %1;" : "=r"(ex) : "r"(arg));
+    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(pos), "r"(ex));
+    return r;
+}
+
+__device__ __forceinline__ void phi_row_f16(uint32_t tile, int row, bool zero)
+{
+#pragma unroll
+    for (int blk = 0; blk < 2; ++blk) {
+        uint4 raw[8];
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) raw[cc] = lds128(tile + sw128_off(row, blk * 64 + cc * 8));
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+            const uint4 r = raw[cc];
+            sts128(tile + sw128_off(row, blk * 64 + cc * 8),
+                   zero ? make_uint4(0u, 0u, 0u, 0u)
+                        : make_uint4(elu1_f16x2_from_bf16x2(r.x), elu1_f16x2_from_bf16x2(r.y),
+                                     elu1_f16x2_from_bf16x2(r.z), elu1_f16x2_from_bf16x2(r.w)));
+        }
+    }
+}
+
+// Row r of a 16-column SW32 block of 128 rows: [first, 0, ..., 0] in fp16.
+__device__ __forceinline__ void write_first_f16(uint8_t *blk, int r, float first)
+{
+    uint4 *row = reinterpret_cast<uint4 *>(blk + (r >> 3) * 256 + (r & 7) * 32);
+    const int c = (r >> 2) & 1;
+    row[c] = make_uint4(pack_f16(first, 0.f), 0u, 0u, 0u);
+    row[c ^ 1] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+// fp16 hi/lo snapshot of 16 state values of row f.
+template <int F>
+__device__ __forceinline__ void snap_cols_f16(uint32_t a_hi, uint32_t a_lo, int f, int c0, const float *v)
+{
+    sts128(a_hi + sw32_off(f, c0, F), make_uint4(pack_f16(v[0], v[1]), pack_f16(v[2], v[3]),
+                                                 pack_f16(v[4], v[5]), pack_f16(v[6], v[7])));
+    sts128(a_hi + sw32_off(f, c0 + 8, F), make_uint4(pack_f16(v[8], v[9]), pack_f16(v[10], v[11]),
+                                                     pack_f16(v[12], v[13]), pack_f16(v[14], v[15])));
+    sts128(a_lo + sw32_off(f, c0, F), make_uint4(pack_f16(f16_rem(v[0]), f16_rem(v[1])),
+                                                 pack_f16(f16_rem(v[2]), f16_rem(v[3])),
+                                                 pack_f16(f16_rem(v[4]), f16_rem(v[5])),
+                                                 pack_f16(f16_rem(v[6]), f16_rem(v[7]))));
+    sts128(a_lo + sw32_off(f, c0 + 8, F), make_uint4(pack_f16(f16_rem(v[8]), f16_rem(v[9])),
+                                                     pack_f16(f16_rem(v[10]), f16_rem(v[11])),
+                                                     pack_f16(f16_rem(v[12]), f16_rem(v[13])),
+                                                     pack_f16(f16_rem(v[14]), f16_rem(v[15]))));
+}
+
+template <typename Keep>
+__device__ __forceinline__ void mask_pack_row_f16(uint32_t src, uint32_t dst, Keep keep)
+{
+#pragma unroll 1
+    for (int j0 = 0; j0 < 128; j0 += 64) {
+        float a[64];
+        tmem_ld32(src + j0, a);
+        tmem_ld32(src + j0 + 32, a + 32);
+        tmem_ld_wait();
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 64; e += 2) pk[e / 2] = pack_f16(keep(j0 + e) ? a[e] : 0.f, keep(j0 + e + 1) ? a[e + 1] : 0.f);
+        tmem_st32(dst + j0 / 2, pk);
+    }
+    tmem_st_wait();
+}
+
+// Masked scores packed as bf16 hi (at dst_hi) and the bf16 remainder (at
+// dst_lo), 64 columns each.
+template <typename Keep>
+__device__ __forceinline__ void mask_pack_row_hilo(uint32_t src, uint32_t dst_hi, uint32_t dst_lo, Keep keep)
+{
+#pragma unroll 1
+    for (int j0 = 0; j0 < 128; j0 += 64) {
+        float a[64];
+        tmem_ld32(src + j0, a);
+        tmem_ld32(src + j0 + 32, a + 32);
+        tmem_ld_wait();
+        uint32_t hi[32], lo[32];
+#pragma unroll
+        for (int e = 0; e < 64; e += 2) {
+            const float x0 = keep(j0 + e) ? a[e] : 0.f, x1 = keep(j0 + e + 1) ? a[e + 1] : 0.f;
+            hi[e / 2] = pack_bf16(x0, x1);
+            lo[e / 2] = pack_bf16(x0 - __bfloat162float(__float2bfloat16_rn(x0)),
+                                  x1 - __bfloat162float(__float2bfloat16_rn(x1)));
+        }
+        tmem_st32(dst_hi + j0 / 2, hi);
+        tmem_st32(dst_lo + j0 / 2, lo);
+    }
+    tmem_st_wait();
+}
+
+}  // namespace bwd_detail
+
+// ---------------------------------------------------------------------------
+// Forward-order pass: dq, and den_i, dden_i per token.
+//
+// Its MMAs run on fp16 operands (A and B both fp16), not bf16: dq is carried
+// by phi - 1, which is ~0.1 for small inputs, and bf16 keeps only ~5 bits of
+// it (relative error ~2/|phi - 1| x 2^-9 in dq); fp16 keeps 3 more.  V is
+// converted exactly; the state snapshot and G' keep an extra fp16 remainder
+// for the inter-chunk term, and dphi(q) is projected orthogonal to phi(q).
+__global__ void __launch_bounds__(128, 1)
+bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+              const BwdParams p)
+{
+    using namespace bwd_detail;
+    using Cfg = BwdCfg128;
+    constexpr int C = Cfg::C, D = Cfg::D, DV = Cfg::DV, NA = Cfg::NA, F = Cfg::F;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *tma_bar = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
+    uint64_t *mma_bar = tma_bar + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tma_bar + 2);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tma_bar + 3);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int bh = blockIdx.x / p.P, seg = blockIdx.x % p.P;
+    const int c_begin = seg * p.cps, c_end = min(p.nchunks, c_begin + p.cps);
+    const int N = p.N;
+    uint8_t *sQ = smem + Cfg::OFF_Q, *sK = smem + Cfg::OFF_K, *sV = smem + Cfg::OFF_V, *sG = smem + Cfg::OFF_G,
+            *sS = smem + Cfg::OFF_S, *sSL = smem + Cfg::OFF_SL;
+    const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV), aG = smem_addr(sG), aS = smem_addr(sS),
+                   aSL = smem_addr(sSL);
+
+    if (tid == 0) {
+        mbar_init(tma_bar, 1);
+        mbar_init(mma_bar, 1);
+        *abort_flag = 0;
+        mbar_init_fence();
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+    write_first_f16(sV + (DV / 16) * Cfg::BLK, tid, 1.f);   // ones column of V_aug
+    __syncthreads();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane = (uint32_t)(warp * 32) << 16;
+    // TMEM columns: [0,128) scores -> P (first 64) and dP (second 64);
+    // [128,272) O_aug, then dA and dphi(Q); [272,416) state S_aug (M = 128);
+    // [416,488) G'_lo, the bf16 remainder of G' (A operand, packed pairs).
+    const uint32_t tA = tmem, tX = tmem + 128, tS = tmem + 272, tGL = tmem + 416;
+
+    // ---- state entering the segment: sum of the earlier segments' increments
+    for (int c0 = 0; c0 < NA; c0 += 16) {
+        float v[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] = 0.f;
+        for (int s2 = 0; s2 < seg; ++s2) {
+            const float *src = p.ws_s + ((size_t)(bh * p.P + s2) * F + tid) * NA + c0;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] += src[e];
+        }
+        tmem_st16(tS + lane + c0, v);
+        snap_cols_f16<F>(aS, aSL, tid, c0, v);
+    }
+    tmem_st_wait();
+    full_sync();
+
+    uint32_t tph = 0, mph = 0;
+    for (int chunk = c_begin; chunk < c_end && !*abort_flag; ++chunk) {
+        const int t0 = chunk * C, i = tid;
+        const bool valid = t0 + i < N;
+        if (tid == 0) {
+            mbar_arrive_expect_tx(tma_bar, 2 * Cfg::QK_TILE + 2 * C * DV * 2);
+            for (int x = 0; x < D; x += 64) {
+                tma_load_3d(sQ + (x / 64) * C * 128, &tm_q, tma_bar, x, t0, bh);
+                tma_load_3d(sK + (x / 64) * C * 128, &tm_k, tma_bar, x, t0, bh);
+            }
+            for (int x = 0; x < DV; x += 16) {
+                tma_load_3d(sV + (x / 16) * Cfg::BLK, &tm_v, tma_bar, x, t0, bh);
+                tma_load_3d(sG + (x / 16) * Cfg::BLK, &tm_do, tma_bar, x, t0, bh);
+            }
+        }
+        if (!mbar_wait(tma_bar, tph)) *abort_flag = 1;
+        tph ^= 1u;
+        // fp16 operands: phi(Q), phi(K) in place; V converted in place
+        phi_row_f16(aQ, i, false);
+        phi_row_f16(aK, i, !valid);
+#pragma unroll
+        for (int c0 = 0; c0 < DV; c0 += 8) {
+            const uint32_t a = aV + sw32_off(i, c0, C);
+            const uint4 r = lds128(a);
+            sts128(a, make_uint4(bf16x2_to_f16x2(r.x), bf16x2_to_f16x2(r.y), bf16x2_to_f16x2(r.z), bf16x2_to_f16x2(r.w)));
+        }
+        full_sync();
+        if (*abort_flag) break;
+
+        // scores
+        if (tid == 0) {
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * (C * 128) + (kk & 3) * 32;
+                mma_bf16(tA, smem_desc(aQ + off, 16, 1024, kSw128), smem_desc(aK + off, 16, 1024, kSw128),
+                         idesc_f16(128, 128, 0, 0), kk > 0);
+            }
+            mma_commit(mma_bar);
+        }
+        if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
+        mph ^= 1u;
+        tc_fence_after();
+        mask_pack_row_f16(tA + lane, tA + lane, [&](int j) { return j <= i; });
+        full_sync();
+
+        // O_aug = P V_aug + phi(Q) S_aug
+        if (tid == 0) {
+            const uint32_t id_o = idesc_f16(128, NA, 0, 1);
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)
+                mma_bf16_ts(tX, tA + kk * 8, smem_desc(aV + kk * 512, Cfg::BLK, 256, kSw32), id_o, kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < F / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * (C * 128) + (kk & 3) * 32;
+                mma_bf16(tX, smem_desc(aQ + off, 16, 1024, kSw128), smem_desc(aS + kk * 512, Cfg::S_BLK, 256, kSw32),
+                         id_o, true);
+            }
+            mma_commit(mma_bar);
+        }
+        if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
+        mph ^= 1u;
+        tc_fence_after();
+
+        // y, den; G'' = den * G' = [dO | -dO . y] in place over dO (fp16, with its
+        // fp16 remainder in TMEM).  Working with den * g keeps every operand in
+        // fp16's normal range (g itself is ~|dO| / (F i)); the rows of dphi(Q) are
+        // divided by den at the end.  den_i and dden_i = -(dO . y)/den go to the
+        // workspace for the reverse pass.
+        float den_row;
+        {
+            float dv16[16];
+            tmem_ld16(tX + lane + DV, dv16);
+            tmem_ld_wait();
+            const float den = dv16[0];
+            den_row = den;
+            const float inv = valid ? 1.f / den : 0.f;
+            float gy = 0.f;   // dO . y
+#pragma unroll 1
+            for (int half = 0; half < DV; half += 64) {
+                uint32_t glo[32];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int c0 = half + 16 * u;
+                    float num[16], go[16];
+                    tmem_ld16(tX + lane + c0, num);
+                    tmem_ld_wait();
+                    const uint32_t a0 = aG + sw32_off(i, c0, C), a1 = aG + sw32_off(i, c0 + 8, C);
+                    unpack8(lds128(a0), go);
+                    unpack8(lds128(a1), go + 8);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        if (!valid) go[e] = 0.f;
+                        gy = fmaf(go[e], num[e] * inv, gy);
+                    }
+                    sts128(a0, make_uint4(pack_f16(go[0], go[1]), pack_f16(go[2], go[3]), pack_f16(go[4], go[5]),
+                                          pack_f16(go[6], go[7])));
+                    sts128(a1, make_uint4(pack_f16(go[8], go[9]), pack_f16(go[10], go[11]),
+                                          pack_f16(go[12], go[13]), pack_f16(go[14], go[15])));
+#pragma unroll
+                    for (int e = 0; e < 16; e += 2) glo[(16 * u + e) / 2] = pack_f16(f16_rem(go[e]), f16_rem(go[e + 1]));
+                }
+                tmem_st32(tGL + lane + half / 2, glo);
+            }
+            const float ddu = valid ? -gy : 0.f;   // den * dden
+            write_first_f16(sG + (DV / 16) * Cfg::BLK, i, ddu);
+            {
+                uint32_t tail[8];
+                tail[0] = pack_f16(f16_rem(ddu), 0.f);
+#pragma unroll
+                for (int e = 1; e < 8; ++e) tail[e] = 0u;
+                tmem_st8(tGL + lane + DV / 2, tail);
+            }
+            tmem_st_wait();
+            if (valid) {
+                p.dd[((size_t)bh * N + t0 + i) * 2] = den;
+                p.dd[((size_t)bh * N + t0 + i) * 2 + 1] = ddu * inv;
+            }
+        }
+        full_sync();
+
+        // dA = G' V_aug^T  (K = the 144 augmented columns)
+        if (tid == 0) {
+#pragma unroll
+            for (int kk = 0; kk < NA / 16; ++kk)
+                mma_bf16(tX, smem_desc(aG + kk * Cfg::BLK, 16, 256, kSw32), smem_desc(aV + kk * Cfg::BLK, 16, 256, kSw32),
+                         idesc_f16(128, 128, 0, 0), kk > 0);
+            mma_commit(mma_bar);
+        }
+        if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
+        mph ^= 1u;
+        tc_fence_after();
+        mask_pack_row_f16(tX + lane, tA + lane + 64, [&](int j) { return j <= i; });
+        full_sync();
+
+        // dphi(Q) = dP phi(K) + G' S_aug^T ;  then S_aug += phi(K)^T V_aug
+        if (tid == 0) {
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)
+                mma_bf16_ts(tX, tA + 64 + kk * 8, smem_desc(aK + kk * 2048, C * 128, 1024, kSw128),
+                            idesc_f16(128, F, 0, 1), kk > 0);
+            // inter-chunk term in ~16-bit precision: G'_hi S_hi^T + G'_hi S_lo^T + G'_lo S_hi^T
+#pragma unroll
+            for (int kk = 0; kk < NA / 16; ++kk) {
+                mma_bf16(tX, smem_desc(aG + kk * Cfg::BLK, 16, 256, kSw32), smem_desc(aS + kk * Cfg::S_BLK, 16, 256, kSw32),
+                         idesc_f16(128, F, 0, 0), true);
+                mma_bf16(tX, smem_desc(aG + kk * Cfg::BLK, 16, 256, kSw32), smem_desc(aSL + kk * Cfg::S_BLK, 16, 256, kSw32),
+                         idesc_f16(128, F, 0, 0), true);
+                mma_bf16_ts(tX, tGL + kk * 8, smem_desc(aS + kk * Cfg::S_BLK, 16, 256, kSw32), idesc_f16(128, F, 0, 0),
+                            true);
+            }
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)
+                mma_bf16(tS, smem_desc(aK + kk * 2048, C * 128, 1024, kSw128), smem_desc(aV + kk * 512, Cfg::BLK, 256, kSw32),
+                         idesc_f16(128, NA, 1, 1), true);
+            mma_commit(mma_bar);
+        }
+        if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
+        mph ^= 1u;
+        tc_fence_after();
+
+        // dq = dphi(Q) * min(phi(q), 1), with dphi(q_i) first projected onto the
+        // complement of phi(q_i): y_i is homogeneous of degree 0 in phi(q_i), so
+        // the exact dphi(q_i) is orthogonal to phi(q_i); the bf16 operands of the
+        // MMAs above leave an error mostly along phi(q_i) (elu features are
+        // near 1 and the terms cancel), which the projection removes.
+        {
+            __nv_bfloat16 *dqrow = reinterpret_cast<__nv_bfloat16 *>(p.dq) + ((size_t)bh * N + t0 + i) * D;
+            float sd = 0.f, sn = 0.f;
+#pragma unroll 1
+            for (int c0 = 0; c0 < F; c0 += 16) {
+                float g[16], ph[16];
+                tmem_ld16(tX + lane + c0, g);
+                tmem_ld_wait();
+                unpack8_f16(lds128(aQ + sw128_off(i, c0)), ph);
+                unpack8_f16(lds128(aQ + sw128_off(i, c0 + 8)), ph + 8);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    sd = fmaf(g[e], ph[e], sd);
+                    sn = fmaf(ph[e], ph[e], sn);
+                }
+            }
+            const float proj = sd / sn;
+            const float rden = valid ? 1.f / den_row : 0.f;
+#pragma unroll 1
+            for (int c0 = 0; c0 < F; c0 += 16) {
+                float g[16], ph[16];
+                tmem_ld16(tX + lane + c0, g);
+                tmem_ld_wait();
+                unpack8_f16(lds128(aQ + sw128_off(i, c0)), ph);
+                unpack8_f16(lds128(aQ + sw128_off(i, c0 + 8)), ph + 8);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) g[e] = (g[e] - proj * ph[e]) * fminf(ph[e], 1.f) * rden;
+                if (valid) {
+#pragma unroll
+                    for (int e = 0; e < 16; e += 8)
+                        *reinterpret_cast<uint4 *>(dqrow + c0 + e) =
+                            make_uint4(pack_bf16(g[e], g[e + 1]), pack_bf16(g[e + 2], g[e + 3]),
+                                       pack_bf16(g[e + 4], g[e + 5]), pack_bf16(g[e + 6], g[e + 7]));
+                }
+            }
+            if (chunk + 1 < c_end) {
+#pragma unroll 1
+                for (int c0 = 0; c0 < NA; c0 += 16) {
+                    float v[16];
+                    tmem_ld16(tS + lane + c0, v);
+                    tmem_ld_wait();
+                    snap_cols_f16<F>(aS, aSL, tid, c0, v);
+                }
+            }
+        }
+        full_sync();
+    }
+    full_sync();
+    if (warp == 0) tmem_dealloc(tmem, Cfg::TMEM_COLS);
+}
+
+// ---------------------------------------------------------------------------
+// State increments for the forward-order pass: for each segment but the
+// last, sum over its tokens of phi(k_j) [v_j | 1]^T, with fp16 operands like
+// the pass that consumes them.
+__global__ void __launch_bounds__(128, 1)
+bwd_sstate_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  const BwdParams p)
+{
+    using namespace bwd_detail;
+    using Cfg = BwdCfg128;
+    constexpr int C = Cfg::C, D = Cfg::D, DV = Cfg::DV, NA = Cfg::NA, F = Cfg::F;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *tma_bar = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
+    uint64_t *mma_bar = tma_bar + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tma_bar + 2);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tma_bar + 3);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int bh = blockIdx.x / p.P, seg = blockIdx.x % p.P;
+    if (seg == p.P - 1) return;   // the last segment's increment is never read
+    const int c_begin = seg * p.cps, c_end = min(p.nchunks, c_begin + p.cps);
+    const int N = p.N;
+    uint8_t *sK = smem + Cfg::OFF_K, *sV = smem + Cfg::OFF_V;
+    const uint32_t aK = smem_addr(sK), aV = smem_addr(sV);
+    if (tid == 0) {
+        mbar_init(tma_bar, 1);
+        mbar_init(mma_bar, 1);
+        *abort_flag = 0;
+        mbar_init_fence();
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, 256);
+    write_first_f16(sV + (DV / 16) * Cfg::BLK, tid, 1.f);
+    __syncthreads();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane = (uint32_t)(warp * 32) << 16;
+    uint32_t tph = 0, mph = 0;
+    for (int chunk = c_begin; chunk < c_end && !*abort_flag; ++chunk) {
+        const int t0 = chunk * C, i = tid;
+        if (tid == 0) {
+            mbar_arrive_expect_tx(tma_bar, Cfg::QK_TILE + C * DV * 2);
+            for (int x = 0; x < D; x += 64) tma_load_3d(sK + (x / 64) * C * 128, &tm_k, tma_bar, x, t0, bh);
+            for (int x = 0; x < DV; x += 16) tma_load_3d(sV + (x / 16) * Cfg::BLK, &tm_v, tma_bar, x, t0, bh);
+        }
+        if (!mbar_wait(tma_bar, tph)) *abort_flag = 1;
+        tph ^= 1u;
+        phi_row_f16(aK, i, t0 + i >= N);
+#pragma unroll
+        for (int c0 = 0; c0 < DV; c0 += 8) {
+            const uint32_t a = aV + sw32_off(i, c0, C);
+            const uint4 r = lds128(a);
+            sts128(a, make_uint4(bf16x2_to_f16x2(r.x), bf16x2_to_f16x2(r.y), bf16x2_to_f16x2(r.z), bf16x2_to_f16x2(r.w)));
+        }
+        full_sync();
+        if (*abort_flag) break;
+        if (tid == 0) {
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)
+                mma_bf16(tmem, smem_desc(aK + kk * 2048, C * 128, 1024, kSw128), smem_desc(aV + kk * 512, Cfg::BLK, 256, kSw32),
+                         idesc_f16(128, NA, 1, 1), chunk > c_begin || kk > 0);
+            mma_commit(mma_bar);
+        }
+        if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
+        mph ^= 1u;
+        full_sync();
+    }
+    if (!*abort_flag) {
+        float *dst = p.ws_s + ((size_t)(bh * p.P + seg) * F + tid) * NA;
+#pragma unroll 1
+        for (int c0 = 0; c0 < NA; c0 += 16) {
+            float v[16];
+            tmem_ld16(tmem + lane + c0, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) dst[c0 + e] = v[e];
+        }
+    }
+    full_sync();
+    if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+// ---------------------------------------------------------------------------
+// R increments: for each segment but the first, sum over its tokens of
+// phi(q_i) G'_i^T (needs den_i, dden_i from the forward-order pass).
+__global__ void __launch_bounds__(128, 1)
+bwd_rstate_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                  const BwdParams p)
+{
+    using namespace bwd_detail;
+    using Cfg = BwdCfg128;
+    constexpr int C = Cfg::C, D = Cfg::D, DV = Cfg::DV, NA = Cfg::NA, F = Cfg::F;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *tma_bar = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
+    uint64_t *mma_bar = tma_bar + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tma_bar + 2);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tma_bar + 3);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int bh = blockIdx.x / p.P, seg = blockIdx.x % p.P;
+    if (seg == 0) return;   // the first segment's increment is never read
+    const int c_begin = seg * p.cps, c_end = min(p.nchunks, c_begin + p.cps);
+    const int N = p.N;
+    uint8_t *sQ = smem + Cfg::OFF_Q, *sG = smem + Cfg::OFF_G;
+    const uint32_t aQ = smem_addr(sQ), aG = smem_addr(sG);
+    if (tid == 0) {
+        mbar_init(tma_bar, 1);
+        mbar_init(mma_bar, 1);
+        *abort_flag = 0;
+        mbar_init_fence();
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, 256);
+    __syncthreads();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane = (uint32_t)(warp * 32) << 16;
+    uint32_t tph = 0, mph = 0;
+    for (int chunk = c_begin; chunk < c_end && !*abort_flag; ++chunk) {
+        const int t0 = chunk * C, i = tid;
+        const bool valid = t0 + i < N;
+        if (tid == 0) {
+            mbar_arrive_expect_tx(tma_bar, Cfg::QK_TILE + C * DV * 2);
+            for (int x = 0; x < D; x += 64) tma_load_3d(sQ + (x / 64) * C * 128, &tm_q, tma_bar, x, t0, bh);
+            for (int x = 0; x < DV; x += 16) tma_load_3d(sG + (x / 16) * Cfg::BLK, &tm_do, tma_bar, x, t0, bh);
+        }
+        if (!mbar_wait(tma_bar, tph)) *abort_flag = 1;
+        tph ^= 1u;
+        phi_row_inplace(aQ, i, false);
+        {
+            const float den = valid ? p.dd[((size_t)bh * N + t0 + i) * 2] : 1.f;
+            const float dden = valid ? p.dd[((size_t)bh * N + t0 + i) * 2 + 1] : 0.f;
+            const float inv = valid ? 1.f / den : 0.f;
+#pragma unroll 1
+            for (int c0 = 0; c0 < DV; c0 += 8) {
+                float go[8];
+                const uint32_t a = aG + sw32_off(i, c0, C);
+                unpack8(lds128(a), go);
+                sts128(a, make_uint4(pack_bf16(go[0] * inv, go[1] * inv), pack_bf16(go[2] * inv, go[3] * inv),
+                                     pack_bf16(go[4] * inv, go[5] * inv), pack_bf16(go[6] * inv, go[7] * inv)));
+            }
+            write_dden(sG + (DV / 16) * Cfg::BLK, i, dden);
+        }
+        full_sync();
+        if (*abort_flag) break;
+        if (tid == 0) {
+            // R_aug += phi(Q)^T G'   (M = F features, N = NA, K = tokens)
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)
+                mma_bf16(tmem, smem_desc(aQ + kk * 2048, C * 128, 1024, kSw128),
+                         smem_desc(aG + kk * 512, Cfg::BLK, 256, kSw32), idesc_bf16(128, NA, 1, 1),
+                         chunk > c_begin || kk > 0);
+            mma_commit(mma_bar);
+        }
+        if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
+        mph ^= 1u;
+        full_sync();
+    }
+    if (!*abort_flag) {
+        float *dst = p.ws_r + ((size_t)(bh * p.P + seg) * F + tid) * NA;
+#pragma unroll 1
+        for (int c0 = 0; c0 < NA; c0 += 16) {
+            float v[16];
+            tmem_ld16(tmem + lane + c0, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) dst[c0 + e] = v[e];
+        }
+    }
+    full_sync();
+    if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+// ---------------------------------------------------------------------------
+// Reverse-order pass: dk and dv.
+__global__ void __launch_bounds__(128, 1)
+bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                const BwdParams p)
+{
+    using namespace bwd_detail;
+    using Cfg = BwdCfg128;
+    constexpr int C = Cfg::C, D = Cfg::D, DV = Cfg::DV, NA = Cfg::NA, F = Cfg::F;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *tma_bar = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
+    uint64_t *mma_bar = tma_bar + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tma_bar + 2);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tma_bar + 3);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int bh = blockIdx.x / p.P, seg = blockIdx.x % p.P;
+    const int c_begin = seg * p.cps, c_end = min(p.nchunks, c_begin + p.cps);
+    const int N = p.N;
+    uint8_t *sQ = smem + Cfg::OFF_Q, *sK = smem + Cfg::OFF_K, *sV = smem + Cfg::OFF_V, *sG = smem + Cfg::OFF_G,
+            *sR = smem + Cfg::OFF_S, *sGL = smem + Cfg::OFF_SL;   // G' bf16 remainder
+    const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV), aG = smem_addr(sG), aR = smem_addr(sR),
+                   aGL = smem_addr(sGL);
+    if (tid == 0) {
+        mbar_init(tma_bar, 1);
+        mbar_init(mma_bar, 1);
+        *abort_flag = 0;
+        mbar_init_fence();
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+    write_ones_block(sV + (DV / 16) * Cfg::BLK, tid);
+    __syncthreads();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane = (uint32_t)(warp * 32) << 16;
+    // TMEM: [0,64) P^T, [64,128) dP^T (packed); [0,128) holds A^T first;
+    // [128,256) dA^T, then dV, then dphi(K); [256,400) R_aug (M = 128);
+    // [400,464) the bf16 remainder of dP^T.
+    const uint32_t tA = tmem, tX = tmem + 128, tR = tmem + 256, tPL = tmem + 400;
+
+    // ---- R entering the segment: sum of the later segments' increments
+    for (int c0 = 0; c0 < NA; c0 += 16) {
+        float v[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] = 0.f;
+        for (int s2 = seg + 1; s2 < p.P; ++s2) {
+            const float *src = p.ws_r + ((size_t)(bh * p.P + s2) * F + tid) * NA + c0;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] += src[e];
+        }
+        tmem_st16(tR + lane + c0, v);
+        sts128(aR + sw32_off(tid, c0, F), make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
+                                                     pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7])));
+        sts128(aR + sw32_off(tid, c0 + 8, F), make_uint4(pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]),
+                                                         pack_bf16(v[12], v[13]), pack_bf16(v[14], v[15])));
+    }
+    tmem_st_wait();
+    full_sync();
+
+    uint32_t tph = 0, mph = 0;
+    for (int chunk = c_end - 1; chunk >= c_begin && !*abort_flag; --chunk) {
+        const int t0 = chunk * C, j = tid;
+        const bool valid = t0 + j < N;
+        if (tid == 0) {
+            mbar_arrive_expect_tx(tma_bar, 2 * Cfg::QK_TILE + 2 * C * DV * 2);
+            for (int x = 0; x < D; x += 64) {
+                tma_load_3d(sQ + (x / 64) * C * 128, &tm_q, tma_bar, x, t0, bh);
+                tma_load_3d(sK + (x / 64) * C * 128, &tm_k, tma_bar, x, t0, bh);
+            }
+            for (int x = 0; x < DV; x += 16) {
+                tma_load_3d(sV + (x / 16) * Cfg::BLK, &tm_v, tma_bar, x, t0, bh);
+                tma_load_3d(sG + (x / 16) * Cfg::BLK, &tm_do, tma_bar, x, t0, bh);
+            }
+        }
+        if (!mbar_wait(tma_bar, tph)) *abort_flag = 1;
+        tph ^= 1u;
+        phi_row_inplace(aQ, j, false);
+        phi_row_inplace(aK, j, !valid);
+        {
+            // G' row j (this thread's token as a query): [dO/den | dden] as bf16
+            // plus its bf16 remainder (dA^T below uses both)
+            const float den = valid ? p.dd[((size_t)bh * N + t0 + j) * 2] : 1.f;
+            const float dden = valid ? p.dd[((size_t)bh * N + t0 + j) * 2 + 1] : 0.f;
+            const float inv = valid ? 1.f / den : 0.f;
+#pragma unroll 1
+            for (int c0 = 0; c0 < DV; c0 += 8) {
+                float go[8];
+                const uint32_t a = aG + sw32_off(j, c0, C);
+                unpack8(lds128(a), go);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) go[e] *= inv;
+                sts128(a, make_uint4(pack_bf16(go[0], go[1]), pack_bf16(go[2], go[3]), pack_bf16(go[4], go[5]),
+                                     pack_bf16(go[6], go[7])));
+                float r[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) r[e] = go[e] - __bfloat162float(__float2bfloat16_rn(go[e]));
+                sts128(aGL + sw32_off(j, c0, C), make_uint4(pack_bf16(r[0], r[1]), pack_bf16(r[2], r[3]),
+                                                            pack_bf16(r[4], r[5]), pack_bf16(r[6], r[7])));
+            }
+            write_dden(sG + (DV / 16) * Cfg::BLK, j, dden);
+            write_dden(sGL + (DV / 16) * Cfg::BLK, j, dden - __bfloat162float(__float2bfloat16_rn(dden)));
+        }
+        full_sync();
+        if (*abort_flag) break;
+
+        // A^T = phi(K) phi(Q)^T ;  dA^T = V_aug G'^T
+        if (tid == 0) {
+#pragma unroll
+            for (int kk = 0; kk < F / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * (C * 128) + (kk & 3) * 32;
+                mma_bf16(tA, smem_desc(aK + off, 16, 1024, kSw128), smem_desc(aQ + off, 16, 1024, kSw128),
+                         idesc_bf16(128, 128, 0, 0), kk > 0);
+            }
+#pragma unroll
+            for (int kk = 0; kk < NA / 16; ++kk) {
+                mma_bf16(tX, smem_desc(aV + kk * Cfg::BLK, 16, 256, kSw32), smem_desc(aG + kk * Cfg::BLK, 16, 256, kSw32),
+                         idesc_bf16(128, 128, 0, 0), kk > 0);
+                mma_bf16(tX, smem_desc(aV + kk * Cfg::BLK, 16, 256, kSw32), smem_desc(aGL + kk * Cfg::BLK, 16, 256, kSw32),
+                         idesc_bf16(128, 128, 0, 0), true);
+            }
+            mma_commit(mma_bar);
+        }
+        if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
+        mph ^= 1u;
+        tc_fence_after();
+        // row j keeps the queries i >= j
+        mask_pack_row(tA + lane, tA + lane, [&](int i) { return i >= j; });
+        mask_pack_row_hilo(tX + lane, tA + lane + 64, tPL + lane, [&](int i) { return i >= j; });
+        full_sync();
+
+        // dV = P^T G + phi(K) R
+        if (tid == 0) {
+            const uint32_t id = idesc_bf16(128, DV, 0, 1);
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)
+                mma_bf16_ts(tX, tA + kk * 8, smem_desc(aG + kk * 512, Cfg::BLK, 256, kSw32), id, kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < F / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * (C * 128) + (kk & 3) * 32;
+                mma_bf16(tX, smem_desc(aK + off, 16, 1024, kSw128), smem_desc(aR + kk * 512, Cfg::S_BLK, 256, kSw32),
+                         id, true);
+            }
+            mma_commit(mma_bar);
+        }
+        if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
+        mph ^= 1u;
+        tc_fence_after();
+        {
+            __nv_bfloat16 *dvrow = reinterpret_cast<__nv_bfloat16 *>(p.dv) + ((size_t)bh * N + t0 + j) * DV;
+#pragma unroll 1
+            for (int c0 = 0; c0 < DV; c0 += 16) {
+                float g[16];
+                tmem_ld16(tX + lane + c0, g);
+                tmem_ld_wait();
+                if (valid)
+#pragma unroll
+                    for (int e = 0; e < 16; e += 8)
+                        *reinterpret_cast<uint4 *>(dvrow + c0 + e) =
+                            make_uint4(pack_bf16(g[e], g[e + 1]), pack_bf16(g[e + 2], g[e + 3]),
+                                       pack_bf16(g[e + 4], g[e + 5]), pack_bf16(g[e + 6], g[e + 7]));
+            }
+        }
+        full_sync();
+
+        // dphi(K) = dP^T phi(Q) + V_aug R_aug^T ;  then R_aug += phi(Q)^T G'
+        if (tid == 0) {
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk) {
+                mma_bf16_ts(tX, tA + 64 + kk * 8, smem_desc(aQ + kk * 2048, C * 128, 1024, kSw128),
+                            idesc_bf16(128, F, 0, 1), kk > 0);
+                mma_bf16_ts(tX, tPL + kk * 8, smem_desc(aQ + kk * 2048, C * 128, 1024, kSw128),
+                            idesc_bf16(128, F, 0, 1), true);
+            }
+#pragma unroll
+            for (int kk = 0; kk < NA / 16; ++kk)
+                mma_bf16(tX, smem_desc(aV + kk * Cfg::BLK, 16, 256, kSw32), smem_desc(aR + kk * Cfg::S_BLK, 16, 256, kSw32),
+                         idesc_bf16(128, F, 0, 0), true);
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)
+                mma_bf16(tR, smem_desc(aQ + kk * 2048, C * 128, 1024, kSw128),
+                         smem_desc(aG + kk * 512, Cfg::BLK, 256, kSw32), idesc_bf16(128, NA, 1, 1), true);
+            mma_commit(mma_bar);
+        }
+        if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
+        mph ^= 1u;
+        tc_fence_after();
+        {
+            __nv_bfloat16 *dkrow = reinterpret_cast<__nv_bfloat16 *>(p.dk) + ((size_t)bh * N + t0 + j) * D;
+#pragma unroll 1
+            for (int c0 = 0; c0 < F; c0 += 16) {
+                float g[16], ph[16];
+                tmem_ld16(tX + lane + c0, g);
+                tmem_ld_wait();
+                unpack8(lds128(aK + sw128_off(j, c0)), ph);
+                unpack8(lds128(aK + sw128_off(j, c0 + 8)), ph + 8);
+                if (valid)
+#pragma unroll
+                    for (int e = 0; e < 16; e += 8)
+                        *reinterpret_cast<uint4 *>(dkrow + c0 + e) = make_uint4(
+                            pack_bf16(g[e] * fminf(ph[e], 1.f), g[e + 1] * fminf(ph[e + 1], 1.f)),
+                            pack_bf16(g[e + 2] * fminf(ph[e + 2], 1.f), g[e + 3] * fminf(ph[e + 3], 1.f)),
+                            pack_bf16(g[e + 4] * fminf(ph[e + 4], 1.f), g[e + 5] * fminf(ph[e + 5], 1.f)),
+                            pack_bf16(g[e + 6] * fminf(ph[e + 6], 1.f), g[e + 7] * fminf(ph[e + 7], 1.f)));
+            }
+            if (chunk > c_begin) snapshot_state<F, NA>(tR + lane, sR, nullptr, tid);
+        }
+        full_sync();
+    }
+    full_sync();
+    if (warp == 0) tmem_dealloc(tmem, Cfg::TMEM_COLS);
+}
+
+}  // namespace la

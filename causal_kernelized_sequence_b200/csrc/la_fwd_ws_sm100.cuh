@@ -86,38 +86,6 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(sm100::smem_addr(bar)) : "memory");
 }
 
-// elu(x)+1 on two packed bf16 values: max(x,0) + 2^(min(x,0) log2 e).  The
-// exponent argument min(x,0) * log2 e is formed with log2 e split into a bf16
-// head (1.4453125) and tail (-0.00262451), as fma(n, head, n * tail), so it is
-// rounded once; the packed exp2 returns bf16, the precision the MMA consumes.
-__device__ __forceinline__ uint32_t elu1_bf16x2(uint32_t x)
-{
-    const uint32_t zero = 0u;
-    const uint32_t l2e_hi = 0x3FB93FB9u;   // bf16(1.4453125) in both halves
-    const uint32_t l2e_lo = 0xBB2CBB2Cu;   // bf16(log2 e - 1.4453125) = -0.00262451 in both halves
-    uint32_t neg, pos, t, arg, ex, r;
-    asm("min.bf16x2 %0, %1, %2;" : "=r"(neg) : "r"(x), "r"(zero));
-    asm("max.bf16x2 %0, %1, %2;" : "=r"(pos) : "r"(x), "r"(zero));
-    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(t) : "r"(neg), "r"(l2e_lo));
-    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(arg) : "r"(neg), "r"(l2e_hi), "r"(t));
-    asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(ex) : "r"(arg));
-    asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(pos), "r"(ex));
-    return r;
-}
-
-__device__ __forceinline__ uint4 lds128(uint32_t a)
-{
-    uint4 r;
-    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(a));
-    return r;
-}
-
-__device__ __forceinline__ void sts128(uint32_t a, uint4 v)
-{
-    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-                 : "memory");
-}
-
 }  // namespace ws_detail
 
 template <int MODE>

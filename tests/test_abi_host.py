@@ -123,3 +123,10 @@ def test_kernel_plan_and_workspace(lib):
     assert la.la_kernel_plan(2, 256, 16, 1, 16, 64, 1, 0) == (1, ["decode_vec_kernel"])
     assert la.la_kernel_plan(2, 2, 2, 1, 16, 48, 0, 0) == (1, ["decode_simt_kernel"])
     assert la.la_kernel_plan(0, 0, 1, 1, 16, 16, 0, 0)[0] == -1
+    # backward, elu bf16 D=128, B=2 H=16 N=16384: segment states, dq pass, R states, dk/dv pass
+    n, names = la.la_kernel_plan(1, 2, 16, 16384, 128, 128, 0, 1)
+    assert n == 4 and names[1] == "bwd_dq_kernel" and names[-1] == "bwd_dkdv_kernel"
+    # workspace: den/dden per token + S and R increments (4 segments x 128 x 144 fp32 each)
+    assert la.la_backward_workspace_bytes(2, 16, 16384, 128, 128, 0, 1) == \
+        32 * 16384 * 2 * 4 + 2 * 32 * 4 * 128 * 144 * 4
+    assert la.la_kernel_plan(1, 1, 2, 300, 64, 64, 0, 1) == (1, ["bwd_simt_kernel"])
