@@ -49,6 +49,43 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # ----------------------------------------------------------------- utilities
 
+def rank_env():
+    """(world size, rank, local rank) from the torchrun environment; (1, 0, 0)
+    when launched alone."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(x, dist_on, device=None):
+    """The largest of every rank's x.  Every rank calls it at the same point."""
+    if not dist_on:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_seed(w, rank):
+    """Each replica draws its own inputs: the workload's seed, offset by rank."""
+    return w.index + 1000 * rank
+
+
+def metric_name(w):
+    return ("decode tokens/s" if w.decode_steps else
+            "training tokens/s" if w.backward else "prefill tokens/s")
+
+
+def base_config(w, world):
+    """The config keys both arms report for workload w on `world` replicas."""
+    return {"workload": w.describe(), "parallelism": f"replicas{world}"}
+
+
+def whole_job_rate(units_per_rank, world, ms):
+    """Units per second over all ranks for a step of `ms` milliseconds (the
+    max over ranks): every replica processes the same number of units."""
+    return units_per_rank * world / (ms * 1e-3)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -150,7 +187,7 @@ class Prefill:
         import causal_kernelized_sequence_b200 as la
         self.la, self.w, self.dev = la, w, dev
         g = torch.Generator(device=dev)
-        g.manual_seed(w.index + 1000 * seed_offset)
+        g.manual_seed(replica_seed(w, seed_offset))
         set_bytes = w.B * w.H * w.N * (2 * w.dqk + 2 * w.dv) * 2
         self.nsets = max(1, math.ceil(2 * L2_BYTES / set_bytes) + 1) if set_bytes < 2 * L2_BYTES else 1
         mk = lambda d: (torch.randn(w.B, w.H, w.N, d, device=dev, generator=g) * w.scale).to(w.torch_dtype)
@@ -181,7 +218,7 @@ class Train:
         import causal_kernelized_sequence_b200 as la
         self.la, self.w, self.dev = la, w, dev
         g = torch.Generator(device=dev)
-        g.manual_seed(w.index + 1000 * seed_offset)
+        g.manual_seed(replica_seed(w, seed_offset))
         mk = lambda d: (torch.randn(w.B, w.H, w.N, d, device=dev, generator=g) * w.scale).to(w.torch_dtype)
         self.q, self.k, self.v, self.do = mk(w.dqk), mk(w.dqk), mk(w.dv), mk(w.dv)
         self.o = torch.empty_like(self.v)
@@ -229,7 +266,7 @@ class Decode:
         T = w.decode_steps if steps is None else steps
         self.T = T
         g = torch.Generator(device=dev)
-        g.manual_seed(w.index + 1000 * seed_offset)
+        g.manual_seed(replica_seed(w, seed_offset))
         mk = lambda *s: torch.randn(*s, device=dev, generator=g).to(w.torch_dtype)
         q, k, v = mk(w.B, w.H, w.N, w.dqk), mk(w.B, w.H, w.N, w.dqk), mk(w.B, w.H, w.N, w.dv)
         r = la.la_forward(q, k, v, w.fmap, state=True)
@@ -302,21 +339,18 @@ def timed(run, steps, warmup, dist_on, device_index, graph_len=None):
         torch.cuda.synchronize()
     if dist_on:
         torch.distributed.barrier()
-    ms = start.elapsed_time(end)
-    if dist_on:
-        t = torch.tensor([ms], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(start.elapsed_time(end), dist_on, "cuda")
     del g, gr
     return ms / steps, clk.summary()
 
 
-def e2e_prefill(w, dev, steps, warmup):
+def e2e_prefill(w, dev, steps, warmup, dist_on=False, rank=0):
     """Same metric through the public API with host buffers: pinned host q,k,v
-    copied in and o copied out inside the timed region, every step."""
+    copied in and o copied out inside the timed region, every step.  Returns
+    (ms per step, max over ranks; h2d bytes; d2h bytes)."""
     import causal_kernelized_sequence_b200 as la
     g = torch.Generator()
-    g.manual_seed(w.index)
+    g.manual_seed(replica_seed(w, rank))
     mk = lambda d: (torch.randn(w.B, w.H, w.N, d, generator=g) * w.scale).to(w.torch_dtype).pin_memory()
     hq, hk, hv = mk(w.dqk), mk(w.dqk), mk(w.dv)
     ho = torch.empty(w.B, w.H, w.N, w.dv, dtype=w.torch_dtype).pin_memory()
@@ -338,13 +372,18 @@ def e2e_prefill(w, dev, steps, warmup):
             one()
     torch.cuda.synchronize()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
     with torch.cuda.stream(stream):
         s.record(stream)
         for _ in range(steps):
             one()
         e.record(stream)
     torch.cuda.synchronize()
-    ms = s.elapsed_time(e) / steps
+    if dist_on:
+        torch.distributed.barrier()
+    ms = max_over_ranks(s.elapsed_time(e) / steps, dist_on, "cuda")
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
     d2h = ho.numel() * ho.element_size()
     return ms, h2d, d2h
@@ -411,7 +450,8 @@ def roofline_entry(bound, achieved, peak, unit, traffic):
 
 
 def run_reference(args):
-    rank = int(os.environ.get("RANK", "0"))
+    """The oracle arm: rank 0 alone times the fp64 oracle; other ranks exit."""
+    _, rank, _ = rank_env()
     if rank != 0:
         return 0
     w = W.BY_NAME[args.workload]
@@ -427,10 +467,10 @@ def run_reference(args):
     value = statistics.median(vals)
     ms = total / max(1, args.steps) * 1e3
     line = {
-        "impl": "reference", "metric": "prefill tokens/s", "value": round(value, 2), "unit": "tokens/s",
+        "impl": "reference", "metric": metric_name(w), "value": round(value, 2), "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": w.describe()},
+        "data": "synthetic", "config": dict(base_config(w, args.gpus), timing="host wall clock, fp64 oracle"),
         "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": omp_threads(),
                          "kind": "oracle", "sample": desc + " per step"},
         "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -457,9 +497,7 @@ def main():
     if args.impl == "reference":
         return run_reference(args)
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     dist_on = world > 1
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -483,17 +521,17 @@ def main():
                           "kernels": la.kernel_plan(w)["kernels"]}), flush=True)
         return 0
     ms, clocks = timed(run, args.steps, args.warmup, dist_on, local)
-    value = run.tokens * world / (ms * 1e-3)
+    value = whole_job_rate(run.tokens, world, ms)
     kern_ms = ms  # one library launch per step for the prefill workloads
     achieved = run.alg_bytes / (kern_ms * 1e-3) / 1e9
     line = {
-        "metric": "prefill tokens/s" if not w.decode_steps else "decode tokens/s",
+        "metric": metric_name(w),
         "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 6), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if w.dtype == W.BF16 else "f32", "data": "synthetic",
-        "config": {"workload": w.describe(), "parallelism": f"replicas{world}",
-                   "l2": run.l2_note(), "timing": "CUDA graph of consecutive steps, CUDA events"},
+        "config": dict(base_config(w, world), l2=run.l2_note(),
+                       timing="CUDA graph of consecutive steps, CUDA events"),
         "roofline": dict(roofline_entry("hbm", achieved, hbm, "GB/s",
                                         load_traffic("forward:" + w.name)),
                          peak_source=peak_kind, alg_bytes_per_launch=run.alg_bytes),
@@ -502,8 +540,8 @@ def main():
     }
     # e2e through the public API with host buffers
     if not w.decode_steps and not w.backward:
-        e_ms, h2d, d2h = e2e_prefill(w, dev, min(args.steps, 50), 3)
-        line["e2e"] = {"value": round(run.tokens * world / (e_ms * 1e-3), 1), "unit": "tokens/s",
+        e_ms, h2d, d2h = e2e_prefill(w, dev, min(args.steps, 50), 3, dist_on, rank)
+        line["e2e"] = {"value": round(whole_job_rate(run.tokens, world, e_ms), 1), "unit": "tokens/s",
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     from causal_kernelized_sequence_b200 import kernel_plan
     kp = kernel_plan(w)
@@ -520,8 +558,7 @@ def main():
             v2 = r2.tokens / (ms2 * 1e-3)
             ach = r2.alg_bytes / (ms2 * 1e-3) / 1e9
             kp2 = kernel_plan(ws)
-            sec[name] = {"metric": "decode tokens/s" if ws.decode_steps else
-                         ("training tokens/s" if ws.backward else "prefill tokens/s"),
+            sec[name] = {"metric": metric_name(ws),
                          "value": round(v2, 1), "unit": "tokens/s", "ms_per_step": round(ms2, 4),
                          "steps": st, "config": ws.describe(), "l2": r2.l2_note(),
                          "roofline": dict(roofline_entry("hbm", ach, hbm, "GB/s",

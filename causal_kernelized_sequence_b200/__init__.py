@@ -14,6 +14,7 @@ Entry points (same names as the C ABI):
     la_feature_map(x, fmap) -> phi
     la_feature_dim(fmap, dqk) -> int
     la_get_device_status() -> None (raises on a recorded device error)
+    la_selftest_bounded_wait(wait_us) -> None (a wait that runs out, on purpose)
 """
 from __future__ import annotations
 
@@ -74,6 +75,8 @@ def load_library(path: str | None = None):
     lib.la_forward_noalloc.restype = i
     lib.la_kernel_plan.argtypes = [i] * 8 + [ctypes.c_char_p, sz]
     lib.la_kernel_plan.restype = i
+    lib.la_selftest_bounded_wait.argtypes = [ctypes.c_uint, vp]
+    lib.la_selftest_bounded_wait.restype = i
     _lib = lib
     return lib
 
@@ -238,3 +241,10 @@ def kernel_plan(w):
 def la_get_device_status():
     """Synchronise the current stream and raise if a kernel recorded an error."""
     _check(load_library().la_get_device_status(_stream()), "la_get_device_status")
+
+
+def la_selftest_bounded_wait(wait_us):
+    """Enqueue the library's failure-path self-test on the current stream: a
+    wait of `wait_us` microseconds on an mbarrier nobody arrives on.  The
+    following la_get_device_status raises LAError(LA_ERR_TIMEOUT)."""
+    _check(load_library().la_selftest_bounded_wait(int(wait_us), _stream()), "la_selftest_bounded_wait")

@@ -385,6 +385,19 @@ la_status backward_tc(const void *q, const void *k, const void *v, const void *d
     return launch_status();
 }
 
+// One warp; lane 0 waits on an mbarrier that expects one arrival nobody
+// makes, through the kernels' bounded wait with a caller-chosen limit.
+__global__ void selftest_wait_kernel(uint64_t limit_ns)
+{
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        sm100::mbar_init(&bar, 1);
+        sm100::mbar_init_fence();
+        sm100::mbar_wait(&bar, 0, limit_ns);
+    }
+    __syncwarp();
+}
+
 }  // namespace
 
 extern "C" {
@@ -626,6 +639,13 @@ la_status la_get_device_status(void *stream)
     if (word & kStatusTimeout) return LA_ERR_TIMEOUT;
     if (word & kStatusCheck) return LA_ERR_DEVICE_CHECK;
     return LA_OK;
+}
+
+la_status la_selftest_bounded_wait(unsigned int wait_us, void *stream)
+{
+    if (wait_us < 1 || wait_us > 2000000u) return LA_ERR_INVALID_ARG;
+    selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>((uint64_t)wait_us * 1000ull);
+    return launch_status();
 }
 
 }  // extern "C"

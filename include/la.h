@@ -206,6 +206,16 @@ LA_API int la_kernel_plan(int op, int B, int H, int N, int dqk, int dv, int fmap
  * synchronisation itself failed. */
 LA_API la_status la_get_device_status(void *stream);
 
+/* Self-test of the device-side failure path.  Launches one block that waits
+ * on a shared-memory mbarrier nothing ever arrives on, through the same
+ * bounded wait every tensor-core kernel uses, with its limit set to
+ * `wait_us` microseconds instead of the kernels' 2 s.  The wait runs out,
+ * the block records the timeout in the status word and returns, so the
+ * context stays usable: the next la_get_device_status on this device returns
+ * LA_ERR_TIMEOUT, the one after it LA_OK.  wait_us must lie in [1, 2000000];
+ * other values return LA_ERR_INVALID_ARG before any launch. */
+LA_API la_status la_selftest_bounded_wait(unsigned int wait_us, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -130,3 +130,10 @@ def test_kernel_plan_and_workspace(lib):
     assert la.la_backward_workspace_bytes(2, 16, 16384, 128, 128, 0, 1) == \
         32 * 16384 * 2 * 4 + 2 * 32 * 4 * 128 * 144 * 4
     assert la.la_kernel_plan(1, 1, 2, 300, 64, 64, 0, 1) == (1, ["bwd_simt_kernel"])
+
+
+def test_selftest_wait_limit_checked_before_launch(lib):
+    lib.la_selftest_bounded_wait.argtypes = [ctypes.c_uint, ctypes.c_void_p]
+    lib.la_selftest_bounded_wait.restype = ctypes.c_int
+    assert lib.la_selftest_bounded_wait(0, None) == 1
+    assert lib.la_selftest_bounded_wait(2000001, None) == 1
