@@ -24,8 +24,16 @@
 // den and dden are recomputed in fp32 in the forward-order pass (so no
 // rounded forward output enters the gradient) and kept per token in the
 // workspace for the reverse pass.  Sequences are split into the forward's
-// segments; segment states come from the forward's state pass (S) and from
-// bwd_rstate_kernel (R), summed over the earlier / later segments.
+// segments; the state entering a segment is the sum of bwd_sstate_kernel's
+// increments (S) of the earlier segments, and R that of bwd_rstate_kernel's
+// increments of the later ones.
+//
+// dphi(Q) is replaced by its component orthogonal to phi(q_i) before the
+// chain rule.  That is exact: y_i is unchanged when phi(q_i) is scaled, so
+// dphi(q_i) . phi(q_i) = 0 in exact arithmetic and only rounding noise is
+// removed (elu features are all ~1, so that noise is large next to dq).
+// The reverse pass uses bf16 operands, with P^T and G' each split into a
+// bf16 head and a bf16 remainder on the products that carry dk.
 //
 // These kernels use one 128-thread warpgroup per block (thread i <-> token or
 // feature row i <-> TMEM lane i) and process a chunk's steps in order; every
