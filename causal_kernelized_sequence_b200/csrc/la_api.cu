@@ -12,12 +12,15 @@
 #include <mutex>
 
 #include "../../include/la.h"
+#include <cstdio>
+
 #include "la_device.cuh"
 #include "la_simt.cuh"
 #include "la_decode.cuh"
 #include "la_prefill_sm100.cuh"
 #include "la_fwd_ws_sm100.cuh"
 #include "la_bwd_sm100.cuh"
+#include "la_fwd_split_sm100.cuh"
 
 using namespace la;
 
@@ -67,7 +70,11 @@ la_status check_shape(int B, int H, int N, int dqk, int dv, int fmap, int dtype)
 
 la_status launch_status()
 {
-    return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+    const cudaError_t e = cudaGetLastError();
+#ifdef LA_DEBUG_LAUNCH
+    if (e != cudaSuccess) fprintf(stderr, "libla launch error: %s\n", cudaGetErrorString(e));
+#endif
+    return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }
 
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device) and
@@ -87,7 +94,7 @@ la_status set_smem(size_t bytes)
 }
 
 // Kernel selection, shared by the entry points and la_kernel_plan.
-enum class Path { Invalid, FwdSimt, FwdTc, BwdSimt, BwdTc, DecodeSimt, DecodeVec };
+enum class Path { Invalid, FwdSimt, FwdSplit, FwdTc, BwdSimt, BwdTc, DecodeSimt, DecodeVec };
 
 // Shapes with a tensor-core forward: bf16 I/O and (elu, dqk = dv in {64,128})
 // or (Taylor, dqk = 16, dv = 64).
@@ -101,6 +108,7 @@ bool tc_forward_shape(int dqk, int dv, int fmap, int dtype)
 Path select_forward(int B, int H, int N, int dqk, int dv, int fmap, int dtype)
 {
     if (check_shape(B, H, N, dqk, dv, fmap, dtype) != LA_OK) return Path::Invalid;
+    if (dtype == LA_BF16 && fmap == LA_FMAP_ELU1 && dqk == 64 && dv == 64) return Path::FwdSplit;
     if (tc_forward_shape(dqk, dv, fmap, dtype)) return Path::FwdTc;
     return Path::FwdSimt;
 }
@@ -121,6 +129,28 @@ void tc_segments(int B, int H, int N, int *P, int *cps, int *nchunks)
     *cps = c;
     *P = (nc + c - 1) / c;
     *nchunks = nc;
+}
+
+// Chunk ranges of the split forward: T chunks of all heads in (head, chunk)
+// order cut into G contiguous ranges, one per block, G <= 148 and at most
+// SplitCfg64::MAX_PER_HEAD ranges per head.
+void split_grid(int B, int H, int N, long long *T, int *G, int *nc)
+{
+    const long long BH = (long long)B * H;
+    *nc = (N + kChunk - 1) / kChunk;
+    *T = BH * *nc;
+    long long g = *T < kNumSms ? *T : kNumSms;
+    if (g > BH * SplitCfg64::MAX_PER_HEAD) g = BH * SplitCfg64::MAX_PER_HEAD;
+    *G = (int)g;
+}
+
+// Workspace of the split forward: per-chunk phi(K) tiles, per-chunk
+// snapshots, then two fp32 aggregates per range.
+size_t split_phik_bytes(long long T) { return (size_t)T * SplitCfg64::TILE; }
+size_t split_snap_bytes(long long T) { return (size_t)T * SplitCfg64::SNAP; }
+size_t split_ws_bytes(long long T, int G)
+{
+    return split_phik_bytes(T) + split_snap_bytes(T) + (size_t)G * 2 * SplitCfg64::AGG * sizeof(float);
 }
 
 // fp32 elements per segment increment: FP x NA.
@@ -149,6 +179,7 @@ int path_kernels(Path p, const char **names)
 {
     switch (p) {
     case Path::FwdSimt: names[0] = "fwd_simt_kernel"; return 1;
+    case Path::FwdSplit: names[0] = "fwd_split_state_kernel"; names[1] = "fwd_split_out_kernel"; return 2;
     case Path::FwdTc: names[0] = "fwd_tc_kernel"; return 1;  // plus the segment pass, see below
     case Path::BwdSimt: names[0] = "bwd_simt_kernel"; return 1;
     case Path::BwdTc: names[0] = "bwd_dq_kernel"; names[1] = "bwd_dkdv_kernel"; return 2;
@@ -332,6 +363,59 @@ la_status forward_ws64(const void *q, const void *k, const void *v, void *o, flo
     return launch_status();
 }
 
+// Chunk-parallel forward (elu, d_qk = d_v = 64): state launch, then output launch.
+la_status forward_split64(const void *q, const void *k, const void *v, void *o, float *s_out, float *z_out,
+                          float *den_out, void *workspace, int B, int H, int N, cudaStream_t stream)
+{
+    const int BH = B * H;
+    CUtensorMap tq, tk, tv, to;
+    if (!make_map(&tq, q, 64, N, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tk, k, 64, N, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tv, v, 64, N, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&to, o, 64, N, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+        return LA_ERR_CUDA;
+    SplitParams p;
+    split_grid(B, H, N, &p.T, &p.G, &p.nc);
+    p.o = (__nv_bfloat16 *)o;
+    p.den_out = den_out;
+    p.s_out = s_out;
+    p.z_out = z_out;
+    p.phik = (uint8_t *)workspace;
+    p.snap = p.phik + split_phik_bytes(p.T);
+    p.agg = (float *)(p.snap + split_snap_bytes(p.T));
+    p.N = N;
+    using Cfg = SplitCfg64;
+    if (set_smem<fwd_split_state_kernel>(Cfg::S_SMEM_ALLOC) != LA_OK ||
+        set_smem<fwd_split_out_kernel>(Cfg::O_SMEM_ALLOC) != LA_OK) {
+#ifdef LA_DEBUG_LAUNCH
+        fprintf(stderr, "libla: shared-memory attribute of the split forward refused\n");
+#endif
+        return LA_ERR_CUDA;
+    }
+    fwd_split_state_kernel<<<p.G, Cfg::S_THREADS, Cfg::S_SMEM_ALLOC, stream>>>(tk, tv, p);
+    if (launch_status() != LA_OK) return LA_ERR_CUDA;
+    // The output launch may start on SMs the state launch has left (programmatic
+    // dependent launch); it waits for the state launch before using its results.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.G);
+    cfg.blockDim = dim3(Cfg::O_THREADS);
+    cfg.dynamicSmemBytes = Cfg::O_SMEM_ALLOC;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t le = cudaLaunchKernelEx(&cfg, fwd_split_out_kernel, tq, tv, to, p);
+    if (le != cudaSuccess) {
+#ifdef LA_DEBUG_LAUNCH
+        fprintf(stderr, "libla launch error (output launch): %s\n", cudaGetErrorString(le));
+#endif
+        return LA_ERR_CUDA;
+    }
+    return launch_status();
+}
+
 la_status forward_tc(const void *q, const void *k, const void *v, void *o, float *s_out, float *z_out,
                      float *den_out, void *workspace, int B, int H, int N, int dqk, int dv, int fmap,
                      cudaStream_t stream)
@@ -428,7 +512,14 @@ int64_t la_feature_dim(int fmap, int dqk)
 
 size_t la_forward_workspace_bytes(int B, int H, int N, int dqk, int dv, int fmap, int dtype)
 {
-    if (select_forward(B, H, N, dqk, dv, fmap, dtype) != Path::FwdTc) return 0;
+    const Path path = select_forward(B, H, N, dqk, dv, fmap, dtype);
+    if (path == Path::FwdSplit) {
+        long long T;
+        int G, nc;
+        split_grid(B, H, N, &T, &G, &nc);
+        return split_ws_bytes(T, G);
+    }
+    if (path != Path::FwdTc) return 0;
     int P, cps, nc;
     tc_segments(B, H, N, &P, &cps, &nc);
     if (P <= 1) return 0;
@@ -461,7 +552,12 @@ la_status la_forward(const void *q, const void *k, const void *v, void *o, float
     if (workspace_bytes < la_forward_workspace_bytes(B, H, N, dqk, dv, fmap, dtype))
         return LA_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
-    if (select_forward(B, H, N, dqk, dv, fmap, dtype) == Path::FwdTc) {
+    const Path path = select_forward(B, H, N, dqk, dv, fmap, dtype);
+    if (path == Path::FwdSplit) {
+        if (!workspace || !aligned(workspace, 16)) return LA_ERR_INVALID_ARG;
+        return forward_split64(q, k, v, o, s_out, z_out, den_out, workspace, B, H, N, s);
+    }
+    if (path == Path::FwdTc) {
         if (workspace_bytes && !aligned(workspace, 16)) return LA_ERR_INVALID_ARG;
         if (la_forward_workspace_bytes(B, H, N, dqk, dv, fmap, dtype) && !workspace) return LA_ERR_INVALID_ARG;
         return forward_tc(q, k, v, o, s_out, z_out, den_out, workspace, B, H, N, dqk, dv, fmap, s);
@@ -627,6 +723,14 @@ int la_kernel_plan(int op, int B, int H, int N, int dqk, int dv, int fmap, int d
 LA_API int la_debug_timeline(long long *host)
 {
     return cudaMemcpyFromSymbol(host, g_timeline, sizeof(g_timeline)) == cudaSuccess ? 0 : 1;
+}
+
+LA_API int la_debug_timeline_split(long long *events, long long *blocks)
+{
+    return cudaMemcpyFromSymbol(events, g_tl_split, sizeof(g_tl_split)) == cudaSuccess &&
+                   cudaMemcpyFromSymbol(blocks, g_tl_blocks, sizeof(g_tl_blocks)) == cudaSuccess
+               ? 0
+               : 1;
 }
 #endif
 

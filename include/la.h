@@ -128,13 +128,13 @@ LA_API la_status la_forward(const void *q, const void *k, const void *v, void *o
  * and hands out none, or a service that keeps a fixed device footprint and
  * forbids allocating on its serving path.  This variant takes the same
  * inputs and outputs as la_forward but no workspace: it uses a scratch
- * array of LA_NOALLOC_SCRATCH_BYTES (8 MiB) compiled into the library as a
+ * array of LA_NOALLOC_SCRATCH_BYTES (32 MiB) compiled into the library as a
  * static device array, which every GPU that loads the library holds until
  * the process exits.  It never calls cudaMalloc, cudaFree or any allocating
  * library routine.
  *   - Sizes whose workspace would exceed the scratch are rejected with
  *     LA_ERR_SCRATCH_LIMIT before anything is launched (for example elu
- *     dqk = dv = 128 with B*H = 32 and N = 16384 needs 9.4 MB).
+ *     dqk = dv = 64 with B*H = 32 and N = 16384 needs 48 MB).
  *   - The first call on a device looks up the scratch array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
  *     before any stream capture.
@@ -144,7 +144,7 @@ LA_API la_status la_forward(const void *q, const void *k, const void *v, void *o
  *     different streams, or from different host threads) race on it and
  *     give wrong results: serialise them.
  * Other arguments, outputs and errors are those of la_forward. */
-#define LA_NOALLOC_SCRATCH_BYTES (8u << 20)
+#define LA_NOALLOC_SCRATCH_BYTES (32u << 20)
 LA_API la_status la_forward_noalloc(const void *q, const void *k, const void *v, void *o,
                                     float *s_out, float *z_out, float *den_out,
                                     int B, int H, int N, int dqk, int dv, int fmap, int dtype,

@@ -105,20 +105,24 @@ def test_product_path_does_not_reference_oracle():
 
 def test_kernel_plan_and_workspace(lib):
     import causal_kernelized_sequence_b200 as la
-    # elu bf16 B=4 H=8 N=4096 D=64: 32 heads on 148 SMs -> 4 segments of 8
-    # chunks; each segment increment is 64 features x (64 + 16) fp32.
-    assert la.la_forward_workspace_bytes(4, 8, 4096, 64, 64, 0, 1) == 32 * 4 * 64 * 80 * 4
-    n, names = la.la_kernel_plan(0, 4, 8, 4096, 64, 64, 0, 1)
-    assert n == 2 and names[-1] == "fwd_ws_kernel"
+    # elu bf16 B=4 H=8 N=4096 D=64: 32 x 32 = 1024 chunks in 148 ranges; per
+    # chunk a phi(K) tile (128 x 64 bf16) and a state snapshot (64 x 80 bf16),
+    # per range two aggregates of 64 x 80 fp32.
+    assert la.la_forward_workspace_bytes(4, 8, 4096, 64, 64, 0, 1) == \
+        1024 * (128 * 64 * 2 + 64 * 80 * 2) + 148 * 2 * 64 * 80 * 4
+    assert la.la_kernel_plan(0, 4, 8, 4096, 64, 64, 0, 1) == (2, ["fwd_split_state_kernel", "fwd_split_out_kernel"])
     # Taylor B=8 H=16: 128 heads -> no split, no workspace
     assert la.la_forward_workspace_bytes(8, 16, 2048, 16, 64, 1, 1) == 0
     assert la.la_kernel_plan(0, 8, 16, 2048, 16, 64, 1, 1)[0] == 1
     # fp32 I/O runs on the exact CUDA-core kernel
     assert la.la_kernel_plan(0, 1, 1, 256, 32, 32, 0, 0) == (1, ["fwd_simt_kernel"])
     assert la.la_forward_workspace_bytes(1, 1, 256, 32, 32, 0, 0) == 0
-    # short sequences never split into empty segments
-    assert la.la_forward_workspace_bytes(1, 1, 100, 64, 64, 0, 1) == 0
-    assert la.la_forward_workspace_bytes(1, 2, 300, 64, 64, 0, 1) == 2 * 3 * 64 * 80 * 4
+    # short sequences: one range per chunk (T < 148), at most 16 ranges per head
+    assert la.la_forward_workspace_bytes(1, 1, 100, 64, 64, 0, 1) == 1 * (16384 + 10240) + 1 * 2 * 5120 * 4
+    assert la.la_forward_workspace_bytes(1, 2, 300, 64, 64, 0, 1) == 6 * (16384 + 10240) + 6 * 2 * 5120 * 4
+    assert la.la_forward_workspace_bytes(1, 1, 16384, 64, 64, 0, 1) == 128 * (16384 + 10240) + 16 * 2 * 5120 * 4
+    # elu d = 128 (and Taylor) keep the segment split: elu bf16 B=2 H=16 N=16384
+    assert la.la_forward_workspace_bytes(2, 16, 16384, 128, 128, 0, 1) == 32 * 4 * 128 * 144 * 4
     # decode: vectorised kernel for dv in {32, 64, 128}
     assert la.la_kernel_plan(2, 256, 16, 1, 16, 64, 1, 0) == (1, ["decode_vec_kernel"])
     assert la.la_kernel_plan(2, 2, 2, 1, 16, 48, 0, 0) == (1, ["decode_simt_kernel"])
