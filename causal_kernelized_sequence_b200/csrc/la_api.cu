@@ -18,7 +18,6 @@
 #include "la_simt.cuh"
 #include "la_decode.cuh"
 #include "la_prefill_sm100.cuh"
-#include "la_fwd_ws_sm100.cuh"
 #include "la_bwd_sm100.cuh"
 #include "la_fwd_split_sm100.cuh"
 
@@ -333,36 +332,6 @@ la_status forward_tc_launch(const void *q, const void *k, const void *v, void *o
     return launch_status();
 }
 
-// Warp-specialised forward (elu, d_qk = d_v = 64).
-la_status forward_ws64(const void *q, const void *k, const void *v, void *o, float *s_out, float *z_out,
-                       float *den_out, void *workspace, int B, int H, int N, cudaStream_t stream)
-{
-    const int BH = B * H;
-    CUtensorMap tq, tk, tv;
-    if (!make_map(&tq, q, 64, N, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&tk, k, 64, N, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&tv, v, 64, N, BH, 16, CU_TENSOR_MAP_SWIZZLE_32B))
-        return LA_ERR_CUDA;
-    FwdParams p;
-    p.s_out = s_out;
-    p.z_out = z_out;
-    p.den_out = den_out;
-    p.ws = (float *)workspace;
-    p.o = o;
-    p.N = N;
-    tc_segments(B, H, N, &p.P, &p.cps, &p.nchunks);
-    p.inv_c1 = p.inv_c2 = p.k1 = p.k2 = 0.f;
-    constexpr int smem0 = WsCfg64<0>::SMEM_ALLOC, smem1 = WsCfg64<1>::SMEM_ALLOC;
-    if (set_smem<fwd_ws_kernel<0>>(smem0) != LA_OK) return LA_ERR_CUDA;
-    if (p.P > 1) {
-        if (set_smem<fwd_ws_kernel<1>>(smem1) != LA_OK) return LA_ERR_CUDA;
-        fwd_ws_kernel<1><<<BH * p.P, 512, smem1, stream>>>(tq, tk, tv, p);
-        if (launch_status() != LA_OK) return LA_ERR_CUDA;
-    }
-    fwd_ws_kernel<0><<<BH * p.P, 512, smem0, stream>>>(tq, tk, tv, p);
-    return launch_status();
-}
-
 // Chunk-parallel forward (elu, d_qk = d_v = 64): state launch, then output launch.
 la_status forward_split64(const void *q, const void *k, const void *v, void *o, float *s_out, float *z_out,
                           float *den_out, void *workspace, int B, int H, int N, cudaStream_t stream)
@@ -420,8 +389,6 @@ la_status forward_tc(const void *q, const void *k, const void *v, void *o, float
                      float *den_out, void *workspace, int B, int H, int N, int dqk, int dv, int fmap,
                      cudaStream_t stream)
 {
-    if (fmap == LA_FMAP_ELU1 && dqk == 64 && dv == 64)
-        return forward_ws64(q, k, v, o, s_out, z_out, den_out, workspace, B, H, N, stream);
     if (fmap == LA_FMAP_TAYLOR2)
         return forward_tc_launch<FwdCfg<16, 64, true>>(q, k, v, o, s_out, z_out, den_out, workspace, B, H, N, stream);
     if (dqk == 64)
@@ -679,9 +646,7 @@ int la_kernel_plan(int op, int B, int H, int N, int dqk, int dv, int fmap, int d
     if (p == Path::FwdTc) {
         int P, cps, nc;
         tc_segments(B, H, N, &P, &cps, &nc);
-        const bool ws64 = fmap == LA_FMAP_ELU1 && dqk == 64 && dv == 64;
-        const char *nm = ws64 ? (P > 1 ? "fwd_ws_kernel<segment states>,fwd_ws_kernel" : "fwd_ws_kernel")
-                              : (P > 1 ? "fwd_tc_kernel<segment states>,fwd_tc_kernel" : "fwd_tc_kernel");
+        const char *nm = P > 1 ? "fwd_tc_kernel<segment states>,fwd_tc_kernel" : "fwd_tc_kernel";
         if (buf && buflen) {
             strncpy(buf, nm, buflen - 1);
             buf[buflen - 1] = 0;
@@ -720,11 +685,6 @@ int la_kernel_plan(int op, int B, int H, int N, int dqk, int dv, int fmap, int d
 
 #ifdef LA_TIMELINE
 // Profiling builds only: copy the block-0 role timeline of the last forward.
-LA_API int la_debug_timeline(long long *host)
-{
-    return cudaMemcpyFromSymbol(host, g_timeline, sizeof(g_timeline)) == cudaSuccess ? 0 : 1;
-}
-
 LA_API int la_debug_timeline_split(long long *events, long long *blocks)
 {
     return cudaMemcpyFromSymbol(events, g_tl_split, sizeof(g_tl_split)) == cudaSuccess &&

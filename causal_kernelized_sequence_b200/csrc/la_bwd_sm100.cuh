@@ -41,7 +41,6 @@
 #pragma once
 
 #include "la_device.cuh"
-#include "la_fwd_ws_sm100.cuh"
 #include "la_prefill_sm100.cuh"
 #include "sm100.cuh"
 
@@ -77,7 +76,6 @@ namespace bwd_detail {
 
 using namespace sm100;
 using namespace fwd_detail;
-using namespace ws_detail;
 
 // Block barrier that also orders tcgen05 and async-proxy accesses around it.
 __device__ __forceinline__ void full_sync()

@@ -40,7 +40,6 @@
 #pragma once
 
 #include "la_device.cuh"
-#include "la_fwd_ws_sm100.cuh"
 #include "la_prefill_sm100.cuh"
 #include "sm100.cuh"
 
@@ -167,7 +166,6 @@ fwd_split_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
 {
     using namespace sm100;
     using namespace fwd_detail;
-    using namespace ws_detail;
     using namespace split_detail;
     using Cfg = SplitCfg64;
     constexpr int C = Cfg::C, NA = Cfg::NA, DV = Cfg::DV, NS = Cfg::S_NS;
@@ -406,7 +404,6 @@ fwd_split_out_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 {
     using namespace sm100;
     using namespace fwd_detail;
-    using namespace ws_detail;
     using namespace split_detail;
     using Cfg = SplitCfg64;
     constexpr int C = Cfg::C, NA = Cfg::NA, DV = Cfg::DV, NQ = Cfg::O_NQ, NKV = Cfg::O_NKV, NPQ = Cfg::O_NPQ;
