@@ -325,10 +325,10 @@ la_status forward_tc_launch(const void *q, const void *k, const void *v, void *o
     if (set_smem<fwd_tc_kernel<Cfg, 0>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
     if (p.P > 1) {
         if (set_smem<fwd_tc_kernel<Cfg, 1>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
-        fwd_tc_kernel<Cfg, 1><<<BH * p.P, 128, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+        fwd_tc_kernel<Cfg, 1><<<BH * p.P, 256, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
         if (launch_status() != LA_OK) return LA_ERR_CUDA;
     }
-    fwd_tc_kernel<Cfg, 0><<<BH * p.P, 128, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+    fwd_tc_kernel<Cfg, 0><<<BH * p.P, 256, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
     return launch_status();
 }
 

@@ -33,6 +33,8 @@
 // the increments of the segments before it.
 #pragma once
 
+#include <type_traits>
+
 #include "la_device.cuh"
 #include "sm100.cuh"
 
@@ -206,7 +208,7 @@ __device__ __forceinline__ void taylor_sym_to_full(int f, int &r1, int &r2, floa
 // MODE 0: full forward (o, den, final state).  MODE 1: state increments of
 // each segment only (written to p.ws).
 template <class Cfg, int MODE>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(256, 1)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const FwdParams p)
 {
@@ -221,7 +223,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tma_bar + 3);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tma_bar + 4);
 
+    // 256 threads: warp w reaches TMEM lanes 32 (w % 4) .. + 31 and takes
+    // column half w / 4 of the row it owns there.
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wq = warp & 3, half = warp >> 2, row = wq * 32 + lane;
     const int bh = blockIdx.x / p.P, seg = blockIdx.x % p.P;
     if (MODE == 1 && seg == p.P - 1) return;  // the last segment's increment is never read
     const int c_begin = seg * p.cps;
@@ -239,9 +244,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     }
     if (warp == 0) tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
     // Constant normaliser block of every V stage: column DV of V_aug = 1.
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < STAGES && tid < C; ++s) {
         uint8_t *blk = smem + Cfg::OFF_V + s * Cfg::V_TILE + (DV / 16) * Cfg::V_BLK;
-        const int r = tid;  // C == 128 rows, one per thread
+        const int r = tid;  // C == 128 rows
         uint4 *row = reinterpret_cast<uint4 *>(blk + (r >> 3) * 256 + (r & 7) * 32);
         const int one_chunk = 0 ^ ((r >> 2) & 1);
         row[one_chunk] = make_uint4(pack_bf16(1.f, 0.f), 0u, 0u, 0u);
@@ -252,7 +257,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
 
     auto issue_tma = [&](int chunk, int s) {
         const int t0 = chunk * C;
@@ -274,9 +279,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (MODE == 0 && seg > 0) {
         for (int t = 0; t < Cfg::NT; ++t) {
             const int m = Cfg::tile_m(t);
-            const int r = (m == 128) ? tid : ((lane < 16) ? warp * 16 + lane : -1);
+            const int r = (m == 128) ? row : ((lane < 16) ? wq * 16 + lane : -1);
             const int f = r < 0 ? -1 : Cfg::tile_f0(t) + r;
-            for (int c0 = 0; c0 < NA; c0 += 16) {
+            for (int c0 = 16 * half; c0 < NA; c0 += 32) {
                 float acc[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) acc[e] = 0.f;
@@ -326,9 +331,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         uint8_t *sPQ = Cfg::TAYLOR ? smem + Cfg::OFF_PQ : sQ;
         uint8_t *sPK = Cfg::TAYLOR ? smem + Cfg::OFF_PK : sK;
 
-        // ---- feature maps (thread i owns token row i)
+        // ---- feature maps (token row `row`, column half `half`)
         {
-            const int i = tid;
+            const int i = row;
             const bool kvalid = i < nvalid;
             if (!Cfg::TAYLOR) {
 #pragma unroll 1
@@ -336,7 +341,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     uint8_t *tile = (MODE == 0 && m == 0) ? sQ : sK;
                     const bool zero = (tile == sK) && !kvalid;
 #pragma unroll
-                    for (int col = 0; col < DQK; col += 8) {
+                    for (int col = half * (DQK / 2); col < (half + 1) * (DQK / 2); col += 8) {
                         const uint32_t a = smem_addr(tile + sw128_off(i, col));
                         const uint4 r = lds128(a);
                         sts128(a, zero ? make_uint4(0u, 0u, 0u, 0u)
@@ -353,16 +358,22 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     float x[16];
                     unpack8(*reinterpret_cast<const uint4 *>(raw + sw32_off(i, 0, C)), x);
                     unpack8(*reinterpret_cast<const uint4 *>(raw + sw32_off(i, 8, C)), x + 8);
+                    // two unrolled copies so every feature index is a compile-time constant
+                    auto features = [&](auto h) {
+                        constexpr int F0 = decltype(h)::value * (Cfg::FT / 2);
 #pragma unroll
-                    for (int f0 = 0; f0 < Cfg::FT; f0 += 8) {
-                        float v8[8];
+                        for (int f0 = F0; f0 < F0 + Cfg::FT / 2; f0 += 8) {
+                            float v8[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            v8[e] = zero ? 0.f : taylor_sym_feature<16>(x, f0 + e, inv_c1, inv_c2, r2_inv_c2);
-                        *reinterpret_cast<uint4 *>(dst + sw128_off(i, f0)) =
-                            make_uint4(pack_bf16(v8[0], v8[1]), pack_bf16(v8[2], v8[3]),
-                                       pack_bf16(v8[4], v8[5]), pack_bf16(v8[6], v8[7]));
-                    }
+                            for (int e = 0; e < 8; ++e)
+                                v8[e] = zero ? 0.f : taylor_sym_feature<16>(x, f0 + e, inv_c1, inv_c2, r2_inv_c2);
+                            *reinterpret_cast<uint4 *>(dst + sw128_off(i, f0)) =
+                                make_uint4(pack_bf16(v8[0], v8[1]), pack_bf16(v8[2], v8[3]),
+                                           pack_bf16(v8[4], v8[5]), pack_bf16(v8[6], v8[7]));
+                        }
+                    };
+                    if (half == 0) features(std::integral_constant<int, 0>{});
+                    else features(std::integral_constant<int, 1>{});
                 }
             }
         }
@@ -416,12 +427,12 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             continue;
         }
 
-        // ---- causal mask -> P (bf16, K-major SW128)
+        // ---- causal mask -> P (bf16, K-major SW128); keys of this thread's half
         {
-            const int i = tid;
+            const int i = row;
             uint8_t *sP = smem + Cfg::OFF_P;
 #pragma unroll 1
-            for (int j0 = 0; j0 < C; j0 += 32) {
+            for (int j0 = half * (C / 2); j0 < (half + 1) * (C / 2); j0 += 32) {
                 float a[32];
                 tmem_ld32(tmem + lane_base + Cfg::COL_O + j0, a);
                 tmem_ld_wait();
@@ -470,23 +481,25 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tc_fence_after();
         if (tid == 0 && it + STAGES < c_end - c_begin) issue_tma(chunk + STAGES, s);
 
-        // ---- outputs: y = num / den
+        // ---- outputs: y = num / den (this thread's half of the value columns)
         {
-            const int i = tid;
-            float o[NA];
+            const int i = row;
+            constexpr int DH = DV / 2;
+            float o[DH], d16[16];
+            tmem_ld16(tmem + lane_base + Cfg::COL_O + DV, d16);   // den in column DV
 #pragma unroll
-            for (int c0 = 0; c0 < NA; c0 += 16) tmem_ld16(tmem + lane_base + Cfg::COL_O + c0, o + c0);
+            for (int c0 = 0; c0 < DH; c0 += 16) tmem_ld16(tmem + lane_base + Cfg::COL_O + half * DH + c0, o + c0);
             tmem_ld_wait();
-            const float den = o[DV];
+            const float den = d16[0];
             const float inv = 1.f / den;
             if (i < nvalid) {
-                __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + ((size_t)bh * N + t0 + i) * DV;
+                __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + ((size_t)bh * N + t0 + i) * DV + half * DH;
 #pragma unroll
-                for (int c0 = 0; c0 < DV; c0 += 8)
+                for (int c0 = 0; c0 < DH; c0 += 8)
                     *reinterpret_cast<uint4 *>(orow + c0) =
                         make_uint4(pack_bf16(o[c0] * inv, o[c0 + 1] * inv), pack_bf16(o[c0 + 2] * inv, o[c0 + 3] * inv),
                                    pack_bf16(o[c0 + 4] * inv, o[c0 + 5] * inv), pack_bf16(o[c0 + 6] * inv, o[c0 + 7] * inv));
-                if (p.den_out) p.den_out[(size_t)bh * N + t0 + i] = den;
+                if (p.den_out && half == 0) p.den_out[(size_t)bh * N + t0 + i] = den;
             }
         }
         // ---- state snapshot for the next chunk (bf16, MN-major SW32)
@@ -495,10 +508,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
             for (int t = 0; t < Cfg::NT; ++t) {
                 const int m = Cfg::tile_m(t);
-                const int r = (m == 128) ? tid : ((lane < 16) ? warp * 16 + lane : -1);
+                const int r = (m == 128) ? row : ((lane < 16) ? wq * 16 + lane : -1);
                 const int f = r < 0 ? -1 : Cfg::tile_f0(t) + r;
 #pragma unroll
-                for (int c0 = 0; c0 < NA; c0 += 16) {
+                for (int c0 = 16 * half; c0 < NA; c0 += 32) {
                     float v[16];
                     tmem_ld16(tmem + lane_base + Cfg::COL_S + t * NA + c0, v);
                     tmem_ld_wait();
@@ -527,10 +540,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll 1
         for (int t = 0; t < Cfg::NT; ++t) {
             const int m = Cfg::tile_m(t);
-            const int r = (m == 128) ? tid : ((lane < 16) ? warp * 16 + lane : -1);
+            const int r = (m == 128) ? row : ((lane < 16) ? wq * 16 + lane : -1);
             const int f = r < 0 ? -1 : Cfg::tile_f0(t) + r;
 #pragma unroll 1
-            for (int c0 = 0; c0 < NA; c0 += 16) {
+            for (int c0 = 16 * half; c0 < NA; c0 += 32) {
                 float v[16];
                 tmem_ld16(tmem + lane_base + Cfg::COL_S + t * NA + c0, v);
                 tmem_ld_wait();
