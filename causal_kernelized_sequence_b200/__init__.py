@@ -8,7 +8,7 @@ there is no CPU or PyTorch fallback, and importing the compute functions fails
 loudly when the library has not been built.
 
 Entry points (same names as the C ABI):
-    la_forward(q, k, v, fmap, *, state=False, den=False, out=None) -> dict
+    la_forward(q, k, v, fmap, *, state=False, den=False, out=None, s_in=None, z_in=None) -> dict
     la_backward(q, k, v, dout, fmap) -> (dq, dk, dv)
     la_decode_step(q, k, v, s, z, fmap, y=None) -> y        (s, z in place)
     la_feature_map(x, fmap) -> phi
@@ -71,6 +71,8 @@ def load_library(path: str | None = None):
     lib.la_feature_map.restype = i
     lib.la_get_device_status.argtypes = [vp]
     lib.la_get_device_status.restype = i
+    lib.la_forward_from_state.argtypes = [vp] * 10 + [sz] + [i] * 7 + [vp]
+    lib.la_forward_from_state.restype = i
     lib.la_forward_noalloc.argtypes = [vp] * 7 + [i] * 7 + [vp]
     lib.la_forward_noalloc.restype = i
     lib.la_kernel_plan.argtypes = [i] * 8 + [ctypes.c_char_p, sz]
@@ -120,8 +122,11 @@ def la_backward_workspace_bytes(B, H, N, dqk, dv, fmap, dtype) -> int:
     return int(load_library().la_backward_workspace_bytes(B, H, N, dqk, dv, fmap, dtype))
 
 
-def la_forward(q, k, v, fmap, *, state=False, den=False, out=None, workspace=None):
+def la_forward(q, k, v, fmap, *, state=False, den=False, out=None, workspace=None, s_in=None, z_in=None):
     """Causal linear attention forward.  q, k [B,H,N,dqk]; v [B,H,N,dv].
+
+    With s_in [B,H,F,dv] and z_in [B,H,F] (fp32) the sequences start from that
+    state (la_forward_from_state) instead of zero.
 
     Returns {"o": [B,H,N,dv], and if requested "s": [B,H,F,dv] fp32,
     "z": [B,H,F] fp32, "den": [B,H,N] fp32}.
@@ -142,6 +147,18 @@ def la_forward(q, k, v, fmap, *, state=False, den=False, out=None, workspace=Non
     wsb = la_forward_workspace_bytes(B, H, N, dqk, dv, fmap, dt)
     if workspace is None and wsb:
         workspace = torch.empty(wsb, dtype=torch.uint8, device=q.device)
+    if (s_in is None) != (z_in is None):
+        raise ValueError("s_in and z_in go together")
+    if s_in is not None:
+        _dev(s_in, z_in)
+        if s_in.dtype != torch.float32 or z_in.dtype != torch.float32 or not s_in.is_contiguous() \
+                or not z_in.is_contiguous() or tuple(s_in.shape) != (B, H, F, dv) or tuple(z_in.shape) != (B, H, F):
+            raise ValueError("s_in must be fp32 [B,H,F,dv] and z_in fp32 [B,H,F], contiguous")
+        _check(lib.la_forward_from_state(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(s_in), _ptr(z_in),
+                                         _ptr(res.get("s")), _ptr(res.get("z")), _ptr(res.get("den")),
+                                         _ptr(workspace), wsb, B, H, N, dqk, dv, fmap, dt, _stream()),
+               "la_forward_from_state")
+        return res
     _check(lib.la_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(res.get("s")), _ptr(res.get("z")),
                           _ptr(res.get("den")), _ptr(workspace), wsb, B, H, N, dqk, dv, fmap, dt,
                           _stream()), "la_forward")

@@ -205,9 +205,9 @@ bool pick_chunk(MakeLayout make, int F, int dqk, int dv, Layout *out, size_t *by
 }
 
 template <typename T>
-la_status forward_simt(const void *q, const void *k, const void *v, void *o, float *s_out,
-                       float *z_out, float *den_out, int B, int H, int N, int dqk, int dv,
-                       int fmap, cudaStream_t stream)
+la_status forward_simt(const void *q, const void *k, const void *v, void *o, const float *s_in,
+                       const float *z_in, float *s_out, float *z_out, float *den_out, int B, int H, int N,
+                       int dqk, int dv, int fmap, cudaStream_t stream)
 {
     const FmapParams fp = make_fmap(fmap, dqk);
     SimtFwdSmem L;
@@ -215,7 +215,7 @@ la_status forward_simt(const void *q, const void *k, const void *v, void *o, flo
     if (!pick_chunk(simt_fwd_layout, fp.F, dqk, dv, &L, &bytes)) return LA_ERR_UNSUPPORTED;
     if (set_smem<fwd_simt_kernel<T>>(bytes) != LA_OK) return LA_ERR_CUDA;
     fwd_simt_kernel<T><<<B * H, kSimtThreads, bytes, stream>>>(
-        (const T *)q, (const T *)k, (const T *)v, (T *)o, s_out, z_out, den_out, N, dv, fp, L);
+        (const T *)q, (const T *)k, (const T *)v, (T *)o, s_in, z_in, s_out, z_out, den_out, N, dv, fp, L);
     return launch_status();
 }
 
@@ -298,9 +298,9 @@ bool make_map(CUtensorMap *m, const void *base, int inner, int N, int BH, int bo
 }
 
 template <class Cfg>
-la_status forward_tc_launch(const void *q, const void *k, const void *v, void *o, float *s_out,
-                            float *z_out, float *den_out, void *workspace, int B, int H, int N,
-                            cudaStream_t stream)
+la_status forward_tc_launch(const void *q, const void *k, const void *v, void *o, const float *s_in,
+                            const float *z_in, float *s_out, float *z_out, float *den_out, void *workspace, int B,
+                            int H, int N, cudaStream_t stream)
 {
     const int BH = B * H;
     CUtensorMap tq, tk, tv;
@@ -310,6 +310,8 @@ la_status forward_tc_launch(const void *q, const void *k, const void *v, void *o
         !make_map(&tv, v, Cfg::DV, N, BH, 16, CU_TENSOR_MAP_SWIZZLE_32B))
         return LA_ERR_CUDA;
     FwdParams p;
+    p.s_in = s_in;
+    p.z_in = z_in;
     p.s_out = s_out;
     p.z_out = z_out;
     p.den_out = den_out;
@@ -333,7 +335,8 @@ la_status forward_tc_launch(const void *q, const void *k, const void *v, void *o
 }
 
 // Chunk-parallel forward (elu, d_qk = d_v = 64): state launch, then output launch.
-la_status forward_split64(const void *q, const void *k, const void *v, void *o, float *s_out, float *z_out,
+la_status forward_split64(const void *q, const void *k, const void *v, void *o, const float *s_in,
+                          const float *z_in, float *s_out, float *z_out,
                           float *den_out, void *workspace, int B, int H, int N, cudaStream_t stream)
 {
     const int BH = B * H;
@@ -345,6 +348,8 @@ la_status forward_split64(const void *q, const void *k, const void *v, void *o, 
         return LA_ERR_CUDA;
     SplitParams p;
     split_grid(B, H, N, &p.T, &p.G, &p.nc);
+    p.s_in = s_in;
+    p.z_in = z_in;
     p.o = (__nv_bfloat16 *)o;
     p.den_out = den_out;
     p.s_out = s_out;
@@ -385,15 +390,19 @@ la_status forward_split64(const void *q, const void *k, const void *v, void *o, 
     return launch_status();
 }
 
-la_status forward_tc(const void *q, const void *k, const void *v, void *o, float *s_out, float *z_out,
+la_status forward_tc(const void *q, const void *k, const void *v, void *o, const float *s_in, const float *z_in,
+                     float *s_out, float *z_out,
                      float *den_out, void *workspace, int B, int H, int N, int dqk, int dv, int fmap,
                      cudaStream_t stream)
 {
     if (fmap == LA_FMAP_TAYLOR2)
-        return forward_tc_launch<FwdCfg<16, 64, true>>(q, k, v, o, s_out, z_out, den_out, workspace, B, H, N, stream);
+        return forward_tc_launch<FwdCfg<16, 64, true>>(q, k, v, o, s_in, z_in, s_out, z_out, den_out, workspace, B, H, N,
+                                                       stream);
     if (dqk == 64)
-        return forward_tc_launch<FwdCfg<64, 64, false>>(q, k, v, o, s_out, z_out, den_out, workspace, B, H, N, stream);
-    return forward_tc_launch<FwdCfg<128, 128, false>>(q, k, v, o, s_out, z_out, den_out, workspace, B, H, N, stream);
+        return forward_tc_launch<FwdCfg<64, 64, false>>(q, k, v, o, s_in, z_in, s_out, z_out, den_out, workspace, B, H,
+                                                        N, stream);
+    return forward_tc_launch<FwdCfg<128, 128, false>>(q, k, v, o, s_in, z_in, s_out, z_out, den_out, workspace, B, H,
+                                                      N, stream);
 }
 
 la_status backward_tc(const void *q, const void *k, const void *v, const void *dout, void *dq, void *dk,
@@ -506,9 +515,10 @@ size_t la_backward_workspace_bytes(int B, int H, int N, int dqk, int dv, int fma
     return bytes;
 }
 
-la_status la_forward(const void *q, const void *k, const void *v, void *o, float *s_out,
-                     float *z_out, float *den_out, void *workspace, size_t workspace_bytes, int B,
-                     int H, int N, int dqk, int dv, int fmap, int dtype, void *stream)
+static la_status forward_impl(const void *q, const void *k, const void *v, void *o, const float *s_in,
+                              const float *z_in, float *s_out, float *z_out, float *den_out, void *workspace,
+                              size_t workspace_bytes, int B, int H, int N, int dqk, int dv, int fmap, int dtype,
+                              void *stream)
 {
     const la_status sh = check_shape(B, H, N, dqk, dv, fmap, dtype);
     if (sh != LA_OK) return sh;
@@ -522,16 +532,49 @@ la_status la_forward(const void *q, const void *k, const void *v, void *o, float
     const Path path = select_forward(B, H, N, dqk, dv, fmap, dtype);
     if (path == Path::FwdSplit) {
         if (!workspace || !aligned(workspace, 16)) return LA_ERR_INVALID_ARG;
-        return forward_split64(q, k, v, o, s_out, z_out, den_out, workspace, B, H, N, s);
+        return forward_split64(q, k, v, o, s_in, z_in, s_out, z_out, den_out, workspace, B, H, N, s);
     }
     if (path == Path::FwdTc) {
         if (workspace_bytes && !aligned(workspace, 16)) return LA_ERR_INVALID_ARG;
         if (la_forward_workspace_bytes(B, H, N, dqk, dv, fmap, dtype) && !workspace) return LA_ERR_INVALID_ARG;
-        return forward_tc(q, k, v, o, s_out, z_out, den_out, workspace, B, H, N, dqk, dv, fmap, s);
+        return forward_tc(q, k, v, o, s_in, z_in, s_out, z_out, den_out, workspace, B, H, N, dqk, dv, fmap, s);
     }
     if (dtype == LA_F32)
-        return forward_simt<float>(q, k, v, o, s_out, z_out, den_out, B, H, N, dqk, dv, fmap, s);
-    return forward_simt<__nv_bfloat16>(q, k, v, o, s_out, z_out, den_out, B, H, N, dqk, dv, fmap, s);
+        return forward_simt<float>(q, k, v, o, s_in, z_in, s_out, z_out, den_out, B, H, N, dqk, dv, fmap, s);
+    return forward_simt<__nv_bfloat16>(q, k, v, o, s_in, z_in, s_out, z_out, den_out, B, H, N, dqk, dv, fmap, s);
+}
+
+la_status la_forward(const void *q, const void *k, const void *v, void *o, float *s_out,
+                     float *z_out, float *den_out, void *workspace, size_t workspace_bytes, int B,
+                     int H, int N, int dqk, int dv, int fmap, int dtype, void *stream)
+{
+    return forward_impl(q, k, v, o, nullptr, nullptr, s_out, z_out, den_out, workspace, workspace_bytes, B, H, N,
+                        dqk, dv, fmap, dtype, stream);
+}
+
+// Byte ranges [a, a + na) and [b, b + nb) overlap (null never overlaps).
+static bool overlaps(const void *a, size_t na, const void *b, size_t nb)
+{
+    if (!a || !b) return false;
+    const uintptr_t x = (uintptr_t)a, y = (uintptr_t)b;
+    return x < y + nb && y < x + na;
+}
+
+la_status la_forward_from_state(const void *q, const void *k, const void *v, void *o, const float *s_in,
+                                const float *z_in, float *s_out, float *z_out, float *den_out, void *workspace,
+                                size_t workspace_bytes, int B, int H, int N, int dqk, int dv, int fmap,
+                                int dtype, void *stream)
+{
+    const la_status sh = check_shape(B, H, N, dqk, dv, fmap, dtype);
+    if (sh != LA_OK) return sh;
+    if (!s_in || !z_in || !aligned(s_in, 16) || !aligned(z_in, 4)) return LA_ERR_INVALID_ARG;
+    const size_t F = (size_t)la_feature_dim(fmap, dqk);
+    const size_t sb = (size_t)B * H * F * dv * sizeof(float), zb = (size_t)B * H * F * sizeof(float);
+    if (overlaps(s_in, sb, s_out, sb) || overlaps(s_in, sb, z_out, zb) || overlaps(z_in, zb, s_out, sb) ||
+        overlaps(z_in, zb, z_out, zb))
+        return LA_ERR_INVALID_ARG;
+    return forward_impl(q, k, v, o, s_in, z_in, s_out, z_out, den_out, workspace, workspace_bytes, B, H, N, dqk,
+                        dv, fmap, dtype, stream);
 }
 
 // Allocation-free forward: la_forward with its workspace taken from a

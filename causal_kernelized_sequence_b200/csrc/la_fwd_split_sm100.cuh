@@ -80,6 +80,7 @@ struct SplitCfg64 {
 };
 
 struct SplitParams {
+    const float *s_in, *z_in;         // nullable: state entering each sequence, [BH][64][64], [BH][64]
     __nv_bfloat16 *o;
     float *den_out, *s_out, *z_out;   // nullable
     uint8_t *phik;                    // [T][TILE] phi(K) tiles, swizzled as in shared memory
@@ -308,13 +309,48 @@ fwd_split_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
         float run[NA];
 #pragma unroll
         for (int e = 0; e < NA; ++e) run[e] = 0.f;
+        // bf16 copy of `run` as the snapshot of range chunk j, in the MMA operand
+        // layout: staged in shared memory (double-buffered), then one bulk store
+        // by thread 320
+        auto write_snap = [&](int j) -> bool {
+            const int sb = ns & 1;
+            if (ns >= 2 && !mbar_wait(&sn_free[sb], ((ns >> 1) - 1) & 1)) return false;
+            const uint32_t stg = smem_addr(smem + Cfg::S_OFF_SNAP + sb * Cfg::SNAP);
+            if (frow) {
+#pragma unroll
+                for (int q = 0; q < NA / 8; ++q)
+                    sts128(stg + sw32_off(f, 8 * q, 64),
+                           make_uint4(pack_bf16(run[8 * q], run[8 * q + 1]), pack_bf16(run[8 * q + 2], run[8 * q + 3]),
+                                      pack_bf16(run[8 * q + 4], run[8 * q + 5]), pack_bf16(run[8 * q + 6], run[8 * q + 7])));
+            }
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sn_full[sb]);
+            if (tid == 320) {
+                if (!mbar_wait(&sn_full[sb], (ns >> 1) & 1)) return false;
+                bulk_store_hint(p.snap + (size_t)(rg.tb + j) * Cfg::SNAP, smem + Cfg::S_OFF_SNAP + sb * Cfg::SNAP, Cfg::SNAP,
+                                keep);
+                bulk_commit();
+                bulk_wait_read_le1();   // the previous snapshot's store has read its tile
+                if (ns >= 1) mbar_arrive(&sn_free[sb ^ 1]);
+            }
+            ++ns;
+            return true;
+        };
         for (int it = 0; it < nit && !*abort_flag; ++it) {
             const int b = it & 1;
             int h, c;
             rg.at(it, nc, h, c);
             if (c == 0) {
+                // a head opens: its entering state (zero unless given)
 #pragma unroll
                 for (int e = 0; e < NA; ++e) run[e] = 0.f;
+                if (p.s_in && frow) {
+#pragma unroll
+                    for (int e = 0; e < DV; ++e) run[e] = p.s_in[((size_t)h * 64 + f) * DV + e];
+                    run[DV] = p.z_in[(size_t)h * 64 + f];
+                }
+                if (p.s_in && !write_snap(it)) { fail(); break; }   // S_snap of this chunk
             }
             if (!mbar_wait(&ds_full[b], (it >> 1) & 1)) { fail(); break; }
             __syncwarp();
@@ -334,32 +370,7 @@ fwd_split_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
             if (lane == 0) mbar_arrive(&ds_free[b]);
             const bool head_end = c == nc - 1, last = it == nit - 1;
             if (!head_end && !last) {
-                // local state before chunk t+1, bf16, in the MMA operand layout:
-                // staged in shared memory (double-buffered), then one bulk store
-                // by thread 320
-                const int sb = ns & 1;
-                if (ns >= 2 && !mbar_wait(&sn_free[sb], ((ns >> 1) - 1) & 1)) { fail(); break; }
-                const uint32_t stg = smem_addr(smem + Cfg::S_OFF_SNAP + sb * Cfg::SNAP);
-                if (frow) {
-#pragma unroll
-                    for (int j = 0; j < NA / 8; ++j)
-                        sts128(stg + sw32_off(f, 8 * j, 64),
-                               make_uint4(pack_bf16(run[8 * j], run[8 * j + 1]), pack_bf16(run[8 * j + 2], run[8 * j + 3]),
-                                          pack_bf16(run[8 * j + 4], run[8 * j + 5]),
-                                          pack_bf16(run[8 * j + 6], run[8 * j + 7])));
-                }
-                fence_proxy_async();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sn_full[sb]);
-                if (tid == 320) {
-                    if (!mbar_wait(&sn_full[sb], (ns >> 1) & 1)) { fail(); break; }
-                    bulk_store_hint(p.snap + (size_t)(rg.tb + it + 1) * Cfg::SNAP, smem + Cfg::S_OFF_SNAP + sb * Cfg::SNAP,
-                                    Cfg::SNAP, keep);
-                    bulk_commit();
-                    bulk_wait_read_le1();   // the previous snapshot's store has read its tile
-                    if (ns >= 1) mbar_arrive(&sn_free[sb ^ 1]);
-                }
-                ++ns;
+                if (!write_snap(it + 1)) { fail(); break; }   // local state before chunk it+1
                 continue;
             }
             if (!frow) continue;
@@ -469,8 +480,12 @@ fwd_split_out_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     auto fail = [&]() { *abort_flag = 1; };
-    // local snapshot exists unless the chunk opens a head segment of the range
-    auto has_loc = [&](int it) { return it > 0 && (rg.c0 + it) % nc != 0; };
+    // local snapshot exists unless the chunk opens a head segment of the range;
+    // where a head opens, it exists when the heads start from a given state
+    auto has_loc = [&](int it) {
+        const bool opens = (rg.c0 + it) % nc == 0;
+        return opens ? p.s_in != nullptr : it > 0;
+    };
     auto has_carry = [&](int it) { return carry_in && it < first_len; };
     LA_TLB(1, 0);
     if (tid == 0) LA_TLS(1, 15, 0);

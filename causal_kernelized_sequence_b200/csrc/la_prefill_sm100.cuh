@@ -82,6 +82,8 @@ struct FwdCfg {
 };
 
 struct FwdParams {
+    const float *s_in;  // [BH, F273/F, DV] nullable: state entering the sequence
+    const float *z_in;  // [BH, F273/F]
     float *s_out;       // [BH, F273/F, DV] nullable
     float *z_out;       // [BH, F] nullable
     float *den_out;     // [BH, N] nullable
@@ -275,8 +277,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     };
 
     bool have_state = false;
-    // ---- starting state of this segment: sum of the earlier segments' increments
-    if (MODE == 0 && seg > 0) {
+    // ---- starting state of this segment: the state entering the sequence (if
+    // given) plus the sum of the earlier segments' increments
+    if (MODE == 0 && (seg > 0 || p.s_in)) {
         for (int t = 0; t < Cfg::NT; ++t) {
             const int m = Cfg::tile_m(t);
             const int r = (m == 128) ? row : ((lane < 16) ? wq * 16 + lane : -1);
@@ -290,6 +293,26 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         const float *src = p.ws + ((size_t)(bh * p.P + s2) * FP + f) * NA + c0;
 #pragma unroll
                         for (int e = 0; e < 16; ++e) acc[e] += src[e];
+                    }
+                    if (p.s_in && f < Cfg::FSYM) {
+                        // boundary rows of internal row f (Taylor: the symmetric pair, scaled)
+                        const int F = Cfg::TAYLOR ? 1 + DQK + DQK * DQK : DQK;
+                        int r1 = f, r2 = -1;
+                        float sc = 1.f;
+                        if (Cfg::TAYLOR) taylor_sym_to_full<16>(f, r1, r2, sc);
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const int col = c0 + e;
+                            float x = 0.f;
+                            if (col < DV) {
+                                x = p.s_in[((size_t)bh * F + r1) * DV + col];
+                                if (r2 >= 0) x += p.s_in[((size_t)bh * F + r2) * DV + col];
+                            } else if (col == DV) {
+                                x = p.z_in[(size_t)bh * F + r1];
+                                if (r2 >= 0) x += p.z_in[(size_t)bh * F + r2];
+                            }
+                            acc[e] += sc * x;
+                        }
                     }
                 }
                 tmem_st16(tmem + lane_base + Cfg::COL_S + t * NA + c0, acc);
@@ -465,7 +488,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 mma_bf16(tmem + Cfg::COL_O, smem_desc(aP + off, 16, 1024, kSw128),
                          smem_desc(aV + kk * 512, Cfg::V_BLK, 256, kSw32), idesc, kk > 0);
             }
-            if (chunk > 0) {
+            if (chunk > 0 || p.s_in) {
                 const uint32_t aQ = smem_addr(sPQ), aS = smem_addr(smem + Cfg::OFF_S);
 #pragma unroll
                 for (int kk = 0; kk < FP / 16; ++kk) {
@@ -566,14 +589,23 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 for (int e = 0; e < 16; ++e) {
                     const int col = c0 + e;
                     const float val = v[e] * sc;
+                    // a packed row holds the symmetric part of a given entering state;
+                    // its antisymmetric part (zero for any state a prefill produces) is
+                    // added back so the returned state is exact
+                    float skew = 0.f;
+                    if (r2 >= 0 && p.s_in)
+                        skew = 0.5f * (col < DV ? p.s_in[((size_t)bh * F + r1) * DV + col] -
+                                                      p.s_in[((size_t)bh * F + r2) * DV + col]
+                                                : (col == DV ? p.z_in[(size_t)bh * F + r1] - p.z_in[(size_t)bh * F + r2]
+                                                             : 0.f));
                     if (col < DV) {
                         if (p.s_out) {
-                            p.s_out[((size_t)bh * F + r1) * DV + col] = val;
-                            if (r2 >= 0) p.s_out[((size_t)bh * F + r2) * DV + col] = val;
+                            p.s_out[((size_t)bh * F + r1) * DV + col] = val + skew;
+                            if (r2 >= 0) p.s_out[((size_t)bh * F + r2) * DV + col] = val - skew;
                         }
                     } else if (col == DV && p.z_out) {
-                        p.z_out[(size_t)bh * F + r1] = val;
-                        if (r2 >= 0) p.z_out[(size_t)bh * F + r2] = val;
+                        p.z_out[(size_t)bh * F + r1] = val + skew;
+                        if (r2 >= 0) p.z_out[(size_t)bh * F + r2] = val - skew;
                     }
                 }
             }

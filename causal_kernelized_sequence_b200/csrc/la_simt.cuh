@@ -43,7 +43,8 @@ inline SimtFwdSmem simt_fwd_layout(int C, int F, int dv)
 template <typename T>
 __global__ void __launch_bounds__(kSimtThreads)
 fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
-                T *__restrict__ o, float *__restrict__ s_out, float *__restrict__ z_out,
+                T *__restrict__ o, const float *__restrict__ s_in, const float *__restrict__ z_in,
+                float *__restrict__ s_out, float *__restrict__ z_out,
                 float *__restrict__ den_out, int N, int dv, FmapParams fp, SimtFwdSmem L)
 {
     extern __shared__ float sm[];
@@ -66,8 +67,12 @@ fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
     const T *vb = v + bh * N * dv;
     T *ob = o + bh * N * dv;
 
-    for (int i = tid; i < F * DS; i += nt) S[i] = 0.f;
-    for (int i = tid; i < F; i += nt) z[i] = 0.f;
+    // state entering the sequence: zero, or the given (s_in, z_in)
+    for (int i = tid; i < F * DS; i += nt) {
+        const int f = i / DS, c = i - f * DS;
+        S[i] = (s_in && c < dv) ? s_in[bh * F * dv + (size_t)f * dv + c] : 0.f;
+    }
+    for (int i = tid; i < F; i += nt) z[i] = z_in ? z_in[bh * F + i] : 0.f;
 
     for (int t0 = 0; t0 < N; t0 += C) {
         const int Lc = min(C, N - t0);

@@ -119,6 +119,33 @@ LA_API la_status la_forward(const void *q, const void *k, const void *v, void *o
                      int B, int H, int N, int dqk, int dv, int fmap, int dtype,
                      void *stream);
 
+/* la_forward starting from a given state instead of zero: resumes a prefill
+ * (chunked prompt processing) from the state a previous la_forward,
+ * la_forward_from_state or la_decode_step left.
+ *
+ *   S_i = S0 + sum_{j<=i} phi(k_j) v_j^T,   z_i = z0 + sum_{j<=i} phi(k_j),
+ *   y_i = phi(q_i) S_i / phi(q_i) . z_i
+ *
+ * (the recurrence of the BASED page, Knowl 3, with s_0 = S0 and z_0 = z0;
+ * running a sequence in two calls gives the outputs and final state of one
+ * call over the whole sequence.)
+ *   s_in [B,H,F,dv] fp32, z_in [B,H,F] fp32: S0 and z0 per (b, h), in the
+ *          layout of s_out / z_out; read only.  Required (NULL is
+ *          LA_ERR_INVALID_ARG) and must not overlap s_out or z_out
+ *          (LA_ERR_INVALID_ARG).  For the Taylor map the state pairs
+ *          rows (a, b) and (b, a) of the second-order block: any state this
+ *          library returns has them equal, and the outputs depend only on
+ *          their sum; the returned state keeps any difference between them
+ *          unchanged.
+ * Every other argument, the workspace size (la_forward_workspace_bytes) and
+ * the errors are those of la_forward. */
+LA_API la_status la_forward_from_state(const void *q, const void *k, const void *v, void *o,
+                                       const float *s_in, const float *z_in,
+                                       float *s_out, float *z_out, float *den_out,
+                                       void *workspace, size_t workspace_bytes,
+                                       int B, int H, int N, int dqk, int dv, int fmap, int dtype,
+                                       void *stream);
+
 /* la_forward for callers that cannot allocate device memory.
  *
  * The pages have no counterpart to this entry point; it is an interface

@@ -141,3 +141,21 @@ def test_selftest_wait_limit_checked_before_launch(lib):
     lib.la_selftest_bounded_wait.restype = ctypes.c_int
     assert lib.la_selftest_bounded_wait(0, None) == 1
     assert lib.la_selftest_bounded_wait(2000001, None) == 1
+
+
+def test_forward_from_state_argument_errors(lib):
+    P = ctypes.c_void_p
+    f = lib.la_forward_from_state
+    f.argtypes = [P] * 10 + [ctypes.c_size_t] + [ctypes.c_int] * 7 + [P]
+    f.restype = ctypes.c_int
+    q, k, v, o, s_in, z_in, s_out, z_out = (0x1000 * (i + 1) for i in range(8))
+    call = lambda s_in=s_in, z_in=z_in, s_out=s_out, z_out=z_out, fmap=0: \
+        f(P(q), P(k), P(v), P(o), P(s_in), P(z_in), P(s_out), P(z_out), None, None, 0,
+          1, 1, 16, 16, 16, fmap, 0, None)
+    assert call(s_in=None) == 1                        # start state required
+    assert call(z_in=None) == 1
+    assert call(s_in=0x6004) == 1                      # misaligned
+    assert call(s_out=s_in) == 1                       # in-place update not allowed
+    assert call(z_out=z_in + 16) == 1                  # z_out overlaps z_in (16 floats)
+    assert call(s_out=s_in + 16 * 16 * 4 - 16) == 1    # tail of s_in overlaps s_out
+    assert call(fmap=4) == 1

@@ -48,6 +48,62 @@ def test_forward_small(fmap, dqk, dv, dtype):
         assert (r["den"] > 0).all()
 
 
+FROM_STATE = [(ELU1, 64, 64, W.BF16), (ELU1, 128, 128, W.BF16), (ELU1, 16, 48, W.BF16),
+              (ELU1, 32, 32, W.F32), (TAYLOR2, 16, 64, W.BF16), (TAYLOR2, 16, 64, W.F32)]
+
+
+def _start_state(fmap, dqk, dv, dtype, seed, B, H, skew):
+    """A realistic state: the recurrence's state after 300 tokens of other
+    random data (fp64), optionally with noise that breaks the symmetry of the
+    Taylor pair features (S[(a,b)] != S[(b,a)])."""
+    q0, k0, v0, _ = W.random_qkv(seed, B, H, 300, dqk, dv, fmap=fmap, dtype=dtype,
+                                 scale=1.0 if fmap == TAYLOR2 else dqk ** -0.5)
+    _, _, s0, z0 = orc.forward_recurrent(fmap, q0, k0, v0)
+    if skew:
+        g = np.random.default_rng(seed)
+        s0 = s0 + 0.1 * np.abs(s0).mean() * g.standard_normal(s0.shape)
+    return torch.from_numpy(s0).float(), torch.from_numpy(z0).float()
+
+
+@pytest.mark.parametrize("fmap,dqk,dv,dtype", FROM_STATE)
+def test_forward_from_state(fmap, dqk, dv, dtype):
+    """la_forward_from_state against the oracle's recurrence started from the
+    same state: outputs, denominators and the final state."""
+    for B, H, N in ((1, 1, 1), (1, 2, 129), (2, 3, 1000), (1, 2, 3000)):
+        s0, z0 = _start_state(fmap, dqk, dv, dtype, 4000 + N, B, H, skew=fmap == TAYLOR2)
+        q, k, v, _ = W.random_qkv(5000 + N, B, H, N, dqk, dv, fmap=fmap, dtype=dtype,
+                                  scale=1.0 if fmap == TAYLOR2 else dqk ** -0.5)
+        r = gpu_forward(q, k, v, fmap, state=True, den=True, s_in=s0.to(DEV), z_in=z0.to(DEV))
+        o_ref, den_ref, s_ref, z_ref = orc.forward_recurrent(fmap, q, k, v, s0, z0)
+        tol = TOL[dtype]
+        for name, ref in (("o", o_ref), ("den", den_ref), ("s", s_ref), ("z", z_ref)):
+            err = orc.max_rel_l2(r[name], ref)
+            assert err <= tol, (B, H, N, name, err)
+
+
+@pytest.mark.parametrize("fmap,dqk,dv,dtype", FROM_STATE)
+def test_chunked_prefill_matches_one_call(fmap, dqk, dv, dtype):
+    """A prompt prefilled in pieces (la_forward, then la_forward_from_state on
+    the rest with the returned state) equals the one-call forward."""
+    B, H, N = 2, 2, 1100
+    q, k, v, _ = W.random_qkv(6000, B, H, N, dqk, dv, fmap=fmap, dtype=dtype,
+                              scale=1.0 if fmap == TAYLOR2 else dqk ** -0.5)
+    o_ref, den_ref, s_ref, z_ref = orc.forward_recurrent(fmap, q, k, v)
+    cuts = [0, 1, 130, 640, N]
+    s = z = None
+    outs, dens = [], []
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        part = [t[:, :, a:b].contiguous() for t in (q, k, v)]
+        kw = {} if s is None else {"s_in": s.to(DEV), "z_in": z.to(DEV)}
+        r = gpu_forward(*part, fmap, state=True, den=True, **kw)
+        outs.append(r["o"]); dens.append(r["den"]); s, z = r["s"], r["z"]
+    tol = TOL[dtype]
+    assert orc.max_rel_l2(torch.cat(outs, 2), o_ref) <= tol
+    assert orc.max_rel_l2(torch.cat(dens, 2), den_ref) <= tol
+    assert orc.max_rel_l2(s, s_ref) <= tol
+    assert orc.max_rel_l2(z, z_ref) <= tol
+
+
 @pytest.mark.parametrize("dtype", [W.F32, W.BF16])
 @pytest.mark.parametrize("fmap,dqk,dv", DIMS)
 def test_backward_small(fmap, dqk, dv, dtype):
