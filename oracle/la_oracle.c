@@ -16,6 +16,12 @@
  *               Knowl 3, the equation phi(q).phi(k) = 1 + q.k + (q.k)^2/2):
  *               [1 | x/d'^(1/4) | x_a x_b / (sqrt(2) sqrt(d'))], the second
  *               block row-major in (a, b), so 1 + d' + d'^2 features.
+ *               The same map with each symmetric pair of second-order
+ *               features folded into one (the count behind the BASED page's
+ *               state-size expression, Knowl 7: 1 + 3d'/2 + d'^2/2 features):
+ *               [1 | x/d'^(1/4) | x_a^2 / (sqrt(2) sqrt(d')) for each a |
+ *               x_a x_b / sqrt(d') for a < b, row-major], so that
+ *               phi_sym(q).phi_sym(k) = phi(q).phi(k) term by term.
  *   forward_brute      -- the masked parallel form, Knowl 3 eq. for y_i:
  *               a_ij = phi(q_i).phi(k_j) for j <= i,
  *               y_i  = sum_j a_ij v_j / sum_j a_ij,           O(N^2 F).
@@ -52,11 +58,13 @@
 
 #define ORC_ELU1 0
 #define ORC_TAYLOR2 1
+#define ORC_TAYLOR2_SYM 2
 
 int orc_feature_dim(int fmap, int dqk)
 {
     if (fmap == ORC_ELU1) return dqk;
     if (fmap == ORC_TAYLOR2) return 1 + dqk + dqk * dqk;
+    if (fmap == ORC_TAYLOR2_SYM) return 1 + dqk + dqk + dqk * (dqk - 1) / 2;
     return -1;
 }
 
@@ -73,6 +81,16 @@ void orc_phi(int fmap, int dqk, const double *x, double *out)
     const double c2 = sqrt(2.0) * sqrt((double)dqk);     /* sqrt(2) sqrt(d')  */
     out[0] = 1.0;
     for (int a = 0; a < dqk; ++a) out[1 + a] = x[a] / c1;
+    if (fmap == ORC_TAYLOR2_SYM) {
+        /* squares, then each unordered pair a < b once; the pair feature
+           stands for the two equal features (a,b), (b,a) of the full map,
+           so it carries sqrt(2) times their value: sqrt(2)/c2 = 1/sqrt(d'). */
+        for (int a = 0; a < dqk; ++a) out[1 + dqk + a] = x[a] * x[a] / c2;
+        int f = 1 + 2 * dqk;
+        for (int a = 0; a < dqk; ++a)
+            for (int b = a + 1; b < dqk; ++b) out[f++] = x[a] * x[b] / sqrt((double)dqk);
+        return;
+    }
     for (int a = 0; a < dqk; ++a)
         for (int b = 0; b < dqk; ++b)
             out[1 + dqk + a * dqk + b] = x[a] * x[b] / c2;
@@ -88,6 +106,18 @@ void orc_phi_vjp(int fmap, int dqk, const double *x, const double *dphi, double 
     }
     const double c1 = pow((double)dqk, 0.25);
     const double c2 = sqrt(2.0) * sqrt((double)dqk);
+    if (fmap == ORC_TAYLOR2_SYM) {
+        /* d/dx_c of x_c^2/c2 is 2 x_c/c2; of x_a x_b/sqrt(d') it is
+           x_b/sqrt(d') for c = a and x_a/sqrt(d') for c = b. */
+        for (int c = 0; c < dqk; ++c) dx[c] = dphi[1 + c] / c1 + dphi[1 + dqk + c] * 2.0 * x[c] / c2;
+        int f = 1 + 2 * dqk;
+        for (int a = 0; a < dqk; ++a)
+            for (int b = a + 1; b < dqk; ++b, ++f) {
+                dx[a] += dphi[f] * x[b] / sqrt((double)dqk);
+                dx[b] += dphi[f] * x[a] / sqrt((double)dqk);
+            }
+        return;
+    }
     /* phi_{1+a} = x_a / c1;  phi_{1+d'+a d'+b} = x_a x_b / c2. */
     for (int c = 0; c < dqk; ++c) {
         double s = dphi[1 + c] / c1;

@@ -18,6 +18,7 @@ import numpy as np
 
 ELU1 = 0
 TAYLOR2 = 1
+TAYLOR2_SYM = 2   # Taylor map with symmetric second-order pairs folded (153 features for d' = 16)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "la_oracle.c")

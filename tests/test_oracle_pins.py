@@ -18,7 +18,7 @@ import numpy as np
 import pytest
 import torch
 
-ELU1, TAYLOR2 = 0, 1
+ELU1, TAYLOR2, TAYLOR2_SYM = 0, 1, 2
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
 
@@ -37,6 +37,14 @@ def test_feature_dims_match_pages(orc):
     for d in (1, 2, 4, 8, 16, 32):
         assert orc.feature_dim(ELU1, d) == d
         assert orc.feature_dim(TAYLOR2, d) == 1 + d + d * d
+    # Knowl 7: the state-size expression (d+1)(1 + 3d'/2 + d'^2/2) for model
+    # dimension d = 64 and d' = 16 counts (d+1) x 153 numbers: the symmetric
+    # feature count of the folded map.
+    st = consts["state_size_d64_dprime16"]
+    assert (st["d"] + 1) * orc.feature_dim(TAYLOR2_SYM, st["dprime"]) == st["value"]
+    for d in (2, 4, 8, 16):
+        assert orc.feature_dim(TAYLOR2_SYM, d) == 1 + 3 * d // 2 + d * d // 2
+    assert orc.feature_dim(TAYLOR2_SYM, 1) == 3 and orc.feature_dim(TAYLOR2_SYM, 3) == 10   # [1, x, x^2]; 1+3+3+3
 
 
 def test_elu1_matches_library_elu():
@@ -49,14 +57,15 @@ def test_elu1_matches_library_elu():
     assert (orc.phi(ELU1, x) > 0).all()
 
 
+@pytest.mark.parametrize("fmap", [TAYLOR2, TAYLOR2_SYM])
 @pytest.mark.parametrize("d", [1, 2, 3, 4, 16])
-def test_taylor_kernel_closed_form(orc, d):
+def test_taylor_kernel_closed_form(orc, d, fmap):
     # BASED page, Knowl 3: phi(q).phi(k) = 1 + q.k + (q.k)^2/2 with the scaling
     # absorbed into q,k; with 1/d'^(1/4) on each side the kernel is
     # 1 + q.k/sqrt(d') + (q.k)^2/(2 d')  (for d'=16: 1 + q.k/4 + (q.k)^2/32).
     q = rnd(2, 50, d, scale=1.5)
     k = rnd(3, 50, d, scale=1.5)
-    pq, pk = orc.phi(TAYLOR2, q), orc.phi(TAYLOR2, k)
+    pq, pk = orc.phi(fmap, q), orc.phi(fmap, k)
     s = (q * k).sum(-1)
     ref = 1 + s / math.sqrt(d) + s * s / (2 * d)
     np.testing.assert_allclose((pq * pk).sum(-1), ref, rtol=1e-12, atol=1e-12)
@@ -89,7 +98,53 @@ def test_taylor_feature_order(orc):
     np.testing.assert_allclose(p, exp, rtol=1e-15, atol=1e-16)
 
 
-@pytest.mark.parametrize("fmap", [ELU1, TAYLOR2])
+def test_taylor_sym_feature_order(orc):
+    # The folded map: constant, first-order coordinates, the d' squares, then
+    # each pair a < b once, row-major; a pair carries both equal features
+    # (a,b), (b,a) of the full map, so sqrt(2) x their value, x_a x_b/sqrt(d').
+    d = 5
+    t, u, a, b = 0.7, -1.3, 1, 3
+    x = np.zeros(d); x[a] = t; x[b] = u
+    p = orc.phi(TAYLOR2_SYM, x[None])[0]
+    exp = np.zeros(1 + 2 * d + d * (d - 1) // 2)
+    exp[0] = 1.0
+    exp[1 + a] = t / d ** 0.25
+    exp[1 + b] = u / d ** 0.25
+    c2 = math.sqrt(2) * math.sqrt(d)
+    exp[1 + d + a] = t * t / c2
+    exp[1 + d + b] = u * u / c2
+    # pairs in order (0,1),(0,2),(0,3),(0,4),(1,2),(1,3): (1,3) is pair number 5
+    exp[1 + 2 * d + 5] = t * u / math.sqrt(d)
+    np.testing.assert_allclose(p, exp, rtol=1e-15, atol=1e-16)
+
+
+def test_taylor_sym_state_is_folded_full_state(orc):
+    # S_sym = sum_j phi_sym(k_j) v_j^T, and phi_sym folds phi's rows (a,b), (b,a)
+    # into one row scaled by 1/sqrt(2): so the folded state's pair row is
+    # (S[a,b] + S[b,a]) / sqrt(2), its square rows are S[a,a], and the
+    # constant and first-order rows are equal.  The outputs are equal.
+    d, dv, N = 4, 3, 30
+    q = rnd(90, 1, 2, N, d); k = rnd(91, 1, 2, N, d); v = rnd(92, 1, 2, N, dv)
+    o1, den1, s1, z1 = orc.forward_recurrent(TAYLOR2, q, k, v)
+    o2, den2, s2, z2 = orc.forward_recurrent(TAYLOR2_SYM, q, k, v)
+    np.testing.assert_allclose(o2, o1, rtol=1e-12)
+    np.testing.assert_allclose(den2, den1, rtol=1e-12)
+    full = lambda a, b: 1 + d + a * d + b
+    rows = list(range(1 + d)) + [full(a, a) for a in range(d)]
+    np.testing.assert_allclose(s2[:, :, :1 + 2 * d], s1[:, :, rows], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(z2[:, :, :1 + 2 * d], z1[:, :, rows], rtol=1e-12, atol=1e-13)
+    f = 1 + 2 * d
+    for a in range(d):
+        for b in range(a + 1, d):
+            np.testing.assert_allclose(s2[:, :, f], (s1[:, :, full(a, b)] + s1[:, :, full(b, a)]) / math.sqrt(2),
+                                       rtol=1e-12, atol=1e-13)
+            np.testing.assert_allclose(z2[:, :, f], (z1[:, :, full(a, b)] + z1[:, :, full(b, a)]) / math.sqrt(2),
+                                       rtol=1e-12, atol=1e-13)
+            f += 1
+    assert f == s2.shape[2]
+
+
+@pytest.mark.parametrize("fmap", [ELU1, TAYLOR2, TAYLOR2_SYM])
 def test_phi_vjp_finite_difference(orc, fmap):
     d = 4
     x = rnd(6, d)
@@ -174,7 +229,8 @@ def test_taylor_approximates_causal_softmax(orc):
     assert bound < 1e-3 * np.abs(ref).max()
 
 
-@pytest.mark.parametrize("fmap,d,dv", [(ELU1, 8, 5), (ELU1, 32, 32), (TAYLOR2, 4, 6), (TAYLOR2, 16, 16)])
+@pytest.mark.parametrize("fmap,d,dv", [(ELU1, 8, 5), (ELU1, 32, 32), (TAYLOR2, 4, 6), (TAYLOR2, 16, 16),
+                                        (TAYLOR2_SYM, 16, 16)])
 def test_brute_equals_recurrent(orc, fmap, d, dv):
     # The parallel form and the recurrent form of Knowl 3 are the same function.
     for N in (1, 2, 17, 129):
@@ -220,12 +276,12 @@ def test_forward_rows_matches_brute(orc):
     np.testing.assert_allclose(d, db[0, 0, rows], rtol=1e-13)
 
 
-@pytest.mark.parametrize("fmap", [ELU1, TAYLOR2])
+@pytest.mark.parametrize("fmap", [ELU1, TAYLOR2, TAYLOR2_SYM])
 def test_forward_from_state_and_decode(orc, fmap):
     # Knowl 5: the prefill may write its final state for generation; decode
     # steps from it must continue the same sequence.  Prefill(P) then T steps
     # == forward over P+T, on the last T outputs and the final state.
-    P, T, d, dv = 23, 9, 16 if fmap == TAYLOR2 else 8, 6
+    P, T, d, dv = 23, 9, 8 if fmap == ELU1 else 16, 6
     q = rnd(40, 2, 3, P + T, d, scale=0.8); k = rnd(41, 2, 3, P + T, d, scale=0.8); v = rnd(42, 2, 3, P + T, dv)
     ofull, _, sfull, zfull = orc.forward_recurrent(fmap, q, k, v)
     _, _, s, z = orc.forward_recurrent(fmap, q[:, :, :P], k[:, :, :P], v[:, :, :P])
@@ -264,7 +320,8 @@ def _loss_grad_fd(orc, fmap, q, k, v, do, h=1e-6):
     return grads
 
 
-@pytest.mark.parametrize("fmap,d,dv,N", [(ELU1, 4, 3, 7), (ELU1, 3, 5, 12), (TAYLOR2, 3, 3, 6), (TAYLOR2, 2, 4, 11)])
+@pytest.mark.parametrize("fmap,d,dv,N", [(ELU1, 4, 3, 7), (ELU1, 3, 5, 12), (TAYLOR2, 3, 3, 6), (TAYLOR2, 2, 4, 11),
+                                          (TAYLOR2_SYM, 3, 3, 6), (TAYLOR2_SYM, 4, 2, 9)])
 def test_backward_finite_differences(orc, fmap, d, dv, N):
     q = rnd(50, 1, 1, N, d, scale=0.8); k = rnd(51, 1, 1, N, d, scale=0.8)
     v = rnd(52, 1, 1, N, dv); do = rnd(53, 1, 1, N, dv)
@@ -274,7 +331,8 @@ def test_backward_finite_differences(orc, fmap, d, dv, N):
         np.testing.assert_allclose(got, ref, rtol=1e-6, atol=1e-8)
 
 
-@pytest.mark.parametrize("fmap,d,dv", [(ELU1, 8, 6), (ELU1, 16, 16), (TAYLOR2, 4, 5), (TAYLOR2, 16, 8)])
+@pytest.mark.parametrize("fmap,d,dv", [(ELU1, 8, 6), (ELU1, 16, 16), (TAYLOR2, 4, 5), (TAYLOR2, 16, 8),
+                                       (TAYLOR2_SYM, 16, 8)])
 def test_backward_brute_equals_recurrent(orc, fmap, d, dv):
     for N in (1, 5, 64, 97):
         q = rnd(60 + N, 2, 2, N, d, scale=0.6); k = rnd(61 + N, 2, 2, N, d, scale=0.6)
@@ -285,7 +343,7 @@ def test_backward_brute_equals_recurrent(orc, fmap, d, dv):
             np.testing.assert_allclose(y, x, rtol=1e-9, atol=1e-11)
 
 
-@pytest.mark.parametrize("fmap", [ELU1, TAYLOR2])
+@pytest.mark.parametrize("fmap", [ELU1, TAYLOR2, TAYLOR2_SYM])
 def test_backward_autograd(orc, fmap):
     # torch autograd differentiates a plain fp64 torch expression of the
     # masked form; it checks the hand-derived chain rule, not the forward.
@@ -298,8 +356,13 @@ def test_backward_autograd(orc, fmap):
         if fmap == ELU1:
             return torch.nn.functional.elu(x) + 1
         one = torch.ones(*x.shape[:-1], 1, dtype=x.dtype)
-        sec = (x[..., :, None] * x[..., None, :]).flatten(-2) / (math.sqrt(2) * math.sqrt(d))
-        return torch.cat([one, x / d ** 0.25, sec], -1)
+        outer = x[..., :, None] * x[..., None, :] / (math.sqrt(2) * math.sqrt(d))
+        if fmap == TAYLOR2:
+            return torch.cat([one, x / d ** 0.25, outer.flatten(-2)], -1)
+        # folded: the diagonal, then the strict upper triangle times sqrt(2)
+        iu = torch.triu_indices(d, d, offset=1)
+        diag = torch.diagonal(outer, dim1=-2, dim2=-1)
+        return torch.cat([one, x / d ** 0.25, diag, math.sqrt(2) * outer[..., iu[0], iu[1]]], -1)
     A = torch.tril(feat(tq) @ feat(tk).transpose(-1, -2))
     y = (A @ tv) / A.sum(-1, keepdim=True)
     (y * torch.from_numpy(do)).sum().backward()
