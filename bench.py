@@ -550,7 +550,7 @@ def main():
 
     if not args.no_secondary and world == 1:
         sec = {}
-        for name in ("taylor_bf16_fwd", "elu_bf16_train", "taylor_decode"):
+        for name in ("taylor_bf16_fwd", "elu_bf16_train", "taylor_decode", "taylor_decode_sym"):
             ws = W.BY_NAME[name]
             r2 = make_run(ws, dev, 0)
             st = 3 if ws.decode_steps else 50

@@ -25,6 +25,7 @@ import torch
 
 LA_FMAP_ELU1 = 0
 LA_FMAP_TAYLOR2 = 1
+LA_FMAP_TAYLOR2_SYM = 2
 LA_F32 = 0
 LA_BF16 = 1
 

@@ -31,7 +31,8 @@ bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
 bool valid_enums(int fmap, int dtype)
 {
-    return (fmap == LA_FMAP_ELU1 || fmap == LA_FMAP_TAYLOR2) && (dtype == LA_F32 || dtype == LA_BF16);
+    return (fmap == LA_FMAP_ELU1 || fmap == LA_FMAP_TAYLOR2 || fmap == LA_FMAP_TAYLOR2_SYM) &&
+           (dtype == LA_F32 || dtype == LA_BF16);
 }
 
 // Sizes this build supports (valid but unsupported -> LA_ERR_UNSUPPORTED).
@@ -50,6 +51,7 @@ FmapParams make_fmap(int fmap, int dqk)
     p.F = (int)la_feature_dim(fmap, dqk);
     p.inv_c1 = (float)(1.0 / pow((double)dqk, 0.25));
     p.inv_c2 = (float)(1.0 / (sqrt(2.0) * sqrt((double)dqk)));
+    p.inv_c3 = (float)(1.0 / sqrt((double)dqk));
     return p;
 }
 
@@ -96,7 +98,7 @@ la_status set_smem(size_t bytes)
 enum class Path { Invalid, FwdSimt, FwdSplit, FwdTc, BwdSimt, BwdTc, DecodeSimt, DecodeVec };
 
 // Shapes with a tensor-core forward: bf16 I/O and (elu, dqk = dv in {64,128})
-// or (Taylor, dqk = 16, dv = 64).
+// or (either Taylor map, dqk = 16, dv = 64).
 bool tc_forward_shape(int dqk, int dv, int fmap, int dtype)
 {
     if (dtype != LA_BF16) return false;
@@ -155,7 +157,7 @@ size_t split_ws_bytes(long long T, int G)
 // fp32 elements per segment increment: FP x NA.
 int64_t tc_increment_floats(int dqk, int dv, int fmap)
 {
-    const int FP = fmap == LA_FMAP_TAYLOR2 ? 160 : dqk;
+    const int FP = fmap == LA_FMAP_ELU1 ? dqk : 160;
     return (int64_t)FP * (dv + 16);
 }
 
@@ -224,7 +226,10 @@ la_status backward_simt(const void *q, const void *k, const void *v, const void 
                         void *dk, void *dvp, float *ws, int B, int H, int N, int dqk, int dv,
                         int fmap, cudaStream_t stream)
 {
-    const FmapParams fp = make_fmap(fmap, dqk);
+    // The backward reads no state, and both Taylor maps give the same
+    // phi(q).phi(k), hence the same gradients: run the 273-feature map on the
+    // folded features (1 + 2d' + d'(d'-1)/2 of them), 44 % less work.
+    const FmapParams fp = make_fmap(fmap == LA_FMAP_TAYLOR2 ? LA_FMAP_TAYLOR2_SYM : fmap, dqk);
     SimtBwdSmem L;
     size_t bytes;
     if (!pick_chunk(simt_bwd_layout, fp.F, dqk, dv, &L, &bytes)) return LA_ERR_UNSUPPORTED;
@@ -256,10 +261,22 @@ la_status decode_vec(const void *q, const void *k, const void *v, void *y, float
     const FmapParams fp = make_fmap(fmap, dqk);
     const T *qq = (const T *)q, *kk = (const T *)k, *vv = (const T *)v;
     T *yy = (T *)y;
+    // state rows per pass: 256 threads / (dv / 4) float4 groups per row
+    const int passes = (fp.F + kDecodeThreads / (dv / 4) - 1) / (kDecodeThreads / (dv / 4));
+    const bool short_state = passes <= 10;
     switch (dv) {
-    case 32: decode_vec_kernel<T, 32, 18><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp); break;
-    case 64: decode_vec_kernel<T, 64, 18><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp); break;
-    case 128: decode_vec_kernel<T, 128, 18><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp); break;
+    case 32:
+        if (short_state) decode_vec_kernel<T, 32, 10, 3><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp);
+        else decode_vec_kernel<T, 32, 18, 2><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp);
+        break;
+    case 64:
+        if (short_state) decode_vec_kernel<T, 64, 10, 3><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp);
+        else decode_vec_kernel<T, 64, 18, 2><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp);
+        break;
+    case 128:
+        if (short_state) decode_vec_kernel<T, 128, 10, 3><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp);
+        else decode_vec_kernel<T, 128, 18, 2><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp);
+        break;
     default: return LA_ERR_UNSUPPORTED;
     }
     return launch_status();
@@ -300,7 +317,7 @@ bool make_map(CUtensorMap *m, const void *base, int inner, int N, int BH, int bo
 template <class Cfg>
 la_status forward_tc_launch(const void *q, const void *k, const void *v, void *o, const float *s_in,
                             const float *z_in, float *s_out, float *z_out, float *den_out, void *workspace, int B,
-                            int H, int N, cudaStream_t stream)
+                            int H, int N, cudaStream_t stream, bool sym_state = false)
 {
     const int BH = B * H;
     CUtensorMap tq, tk, tv;
@@ -315,6 +332,7 @@ la_status forward_tc_launch(const void *q, const void *k, const void *v, void *o
     p.s_out = s_out;
     p.z_out = z_out;
     p.den_out = den_out;
+    p.sym_state = sym_state ? 1 : 0;
     p.ws = (float *)workspace;
     p.o = o;
     p.N = N;
@@ -395,9 +413,9 @@ la_status forward_tc(const void *q, const void *k, const void *v, void *o, const
                      float *den_out, void *workspace, int B, int H, int N, int dqk, int dv, int fmap,
                      cudaStream_t stream)
 {
-    if (fmap == LA_FMAP_TAYLOR2)
+    if (fmap != LA_FMAP_ELU1)
         return forward_tc_launch<FwdCfg<16, 64, true>>(q, k, v, o, s_in, z_in, s_out, z_out, den_out, workspace, B, H, N,
-                                                       stream);
+                                                       stream, fmap == LA_FMAP_TAYLOR2_SYM);
     if (dqk == 64)
         return forward_tc_launch<FwdCfg<64, 64, false>>(q, k, v, o, s_in, z_in, s_out, z_out, den_out, workspace, B, H,
                                                         N, stream);
@@ -483,6 +501,7 @@ int64_t la_feature_dim(int fmap, int dqk)
     if (dqk < 1) return -1;
     if (fmap == LA_FMAP_ELU1) return dqk;
     if (fmap == LA_FMAP_TAYLOR2) return 1 + (int64_t)dqk + (int64_t)dqk * dqk;
+    if (fmap == LA_FMAP_TAYLOR2_SYM) return 1 + 2 * (int64_t)dqk + (int64_t)dqk * (dqk - 1) / 2;
     return -1;
 }
 

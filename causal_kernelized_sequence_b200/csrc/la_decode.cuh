@@ -8,6 +8,9 @@
 //  - one 256-thread block per head; thread (r0, c4) owns the float4 column
 //    group c4 of rows r0, r0 + RPP, r0 + 2 RPP, ... (RPP = 256 / (DV/4)), so
 //    each warp moves whole 128-byte lines with 16-byte loads and stores;
+//  - MINB blocks per SM: 2 for the 273-row Taylor state, more for states of
+//    at most MAXP = 10 passes (the 153-row folded state), whose blocks are
+//    shorter, so that more of them keep loads in flight;
 //  - every state load of a batch of up to MAXP row passes is issued before
 //    the block computes phi(q), phi(k) (the feature-map prologue overlaps the
 //    first DRAM round trip) and before any of them is consumed, keeping
@@ -25,8 +28,8 @@ namespace la {
 constexpr int kDecodeThreads = 256;
 constexpr int kDecodeMaxF = 288;
 
-template <typename T, int DV, int MAXP>
-__global__ void __launch_bounds__(kDecodeThreads, 2)
+template <typename T, int DV, int MAXP, int MINB>
+__global__ void __launch_bounds__(kDecodeThreads, MINB)
 decode_vec_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                   T *__restrict__ y, float *__restrict__ S, float *__restrict__ z, FmapParams fp)
 {
@@ -52,6 +55,11 @@ decode_vec_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__r
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float4 vc = acc;
     float4 sreg[MAXP];
+    // z entries of this thread (F <= kDecodeMaxF < 2 x 256), loaded with the
+    // first batch of state rows rather than after the last one.
+    static_assert(kDecodeMaxF <= 2 * kDecodeThreads, "two z entries per thread");
+    const float z0 = tid < F ? __ldcs(zb + tid) : 0.f;
+    const float z1 = tid + kDecodeThreads < F ? __ldcs(zb + tid + kDecodeThreads) : 0.f;
     for (int p0 = 0; p0 < passes; p0 += MAXP) {
 #pragma unroll
         for (int b = 0; b < MAXP; ++b) {
@@ -93,10 +101,15 @@ decode_vec_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__r
     }
     // z update and the denominator phi(q).z (z rows are 4-byte aligned only).
     float dacc = 0.f;
-    for (int f = tid; f < F; f += kDecodeThreads) {
-        const float zz = zb[f] + pk[f];
-        zb[f] = zz;
-        dacc = fmaf(pq[f], zz, dacc);
+    if (tid < F) {
+        const float zz = z0 + pk[tid];
+        __stcs(zb + tid, zz);
+        dacc = pq[tid] * zz;
+    }
+    if (tid + kDecodeThreads < F) {
+        const float zz = z1 + pk[tid + kDecodeThreads];
+        __stcs(zb + tid + kDecodeThreads, zz);
+        dacc = fmaf(pq[tid + kDecodeThreads], zz, dacc);
     }
     // Numerator: reduce row groups inside the warp, then across warps.
     if (CPR < 32) {

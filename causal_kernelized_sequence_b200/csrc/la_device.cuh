@@ -37,27 +37,54 @@ template <> __device__ __forceinline__ void st<__nv_bfloat16>(__nv_bfloat16 *p, 
 
 // ------------------------------------------------------------ feature maps
 // Constants of the Taylor map, computed on the host in double precision and
-// rounded once: inv_c1 = 1/dqk^(1/4), inv_c2 = 1/(sqrt(2) sqrt(dqk)).
+// rounded once: inv_c1 = 1/dqk^(1/4), inv_c2 = 1/(sqrt(2) sqrt(dqk)),
+// inv_c3 = 1/sqrt(dqk) (the folded map's pair features).
 struct FmapParams {
-    int fmap;   // LA_FMAP_ELU1 or LA_FMAP_TAYLOR2
+    int fmap;   // LA_FMAP_ELU1, LA_FMAP_TAYLOR2 or LA_FMAP_TAYLOR2_SYM
     int dqk;
     int F;
     float inv_c1;
     float inv_c2;
+    float inv_c3;
 };
 
 // elu(x)+1 with alpha = 1 ("Transformers are RNNs").
 __device__ __forceinline__ float elu1(float x) { return x > 0.f ? x + 1.f : expf(x); }
 __device__ __forceinline__ float elu1_grad(float x) { return x > 0.f ? 1.f : expf(x); }
 
+// Pair number p of the folded Taylor map's cross block -> (a, b), a < b,
+// pairs in row-major order (0,1), (0,2), ..., (1,2), ...
+__host__ __device__ __forceinline__ void sym_pair(int p, int d, int &a, int &b)
+{
+    a = 0;
+    while (p >= d - 1 - a) {
+        p -= d - 1 - a;
+        ++a;
+    }
+    b = a + 1 + p;
+}
+
+// Inverse of sym_pair for a < b.
+__host__ __device__ __forceinline__ int sym_pair_index(int a, int b, int d)
+{
+    return a * d - a * (a + 1) / 2 + (b - a - 1);
+}
+
 // Feature f of phi(x) for a vector x held in shared/local memory.
-// Taylor order: [1 | x_a * inv_c1 | x_a x_b * inv_c2 (row-major a, b)].
+// TAYLOR2:     [1 | x_a * inv_c1 | x_a x_b * inv_c2 (row-major a, b)].
+// TAYLOR2_SYM: [1 | x_a * inv_c1 | x_a^2 * inv_c2 | x_a x_b * inv_c3 (a < b)].
 __device__ __forceinline__ float phi_feature(const FmapParams &fp, const float *x, int f)
 {
     if (fp.fmap == LA_FMAP_ELU1) return elu1(x[f]);
     if (f == 0) return 1.f;
     if (f <= fp.dqk) return x[f - 1] * fp.inv_c1;
     const int idx = f - 1 - fp.dqk;
+    if (fp.fmap == LA_FMAP_TAYLOR2_SYM) {
+        if (idx < fp.dqk) return x[idx] * x[idx] * fp.inv_c2;
+        int a, b;
+        sym_pair(idx - fp.dqk, fp.dqk, a, b);
+        return x[a] * x[b] * fp.inv_c3;
+    }
     const int a = idx / fp.dqk, b = idx - a * fp.dqk;
     return x[a] * x[b] * fp.inv_c2;
 }
@@ -68,6 +95,15 @@ __device__ __forceinline__ float phi_vjp_component(const FmapParams &fp, const f
 {
     if (fp.fmap == LA_FMAP_ELU1) return dphi[c] * elu1_grad(x[c]);
     const int d = fp.dqk;
+    if (fp.fmap == LA_FMAP_TAYLOR2_SYM) {
+        // d/dx_c: x_c^2 inv_c2 -> 2 x_c inv_c2;  x_a x_b inv_c3 -> x_b inv_c3 (c = a) or x_a inv_c3 (c = b)
+        const float *dp = dphi + 1 + 2 * d;
+        float t = 0.f;
+        for (int b = 0; b < d; ++b)
+            if (b != c) t = fmaf(dp[b < c ? sym_pair_index(b, c, d) : sym_pair_index(c, b, d)], x[b], t);
+        const float s = fmaf(dphi[1 + d + c] * 2.f * x[c], fp.inv_c2, dphi[1 + c] * fp.inv_c1);
+        return fmaf(t, fp.inv_c3, s);
+    }
     float s = dphi[1 + c] * fp.inv_c1;
     float t = 0.f;
     for (int b = 0; b < d; ++b)

@@ -18,7 +18,8 @@
 //           the symmetric second-order features (1 + 16 + 136 = 153, padded
 //           to 160) are written to separate phi tiles.  phi(q).phi(k) equals
 //           1 + q.k/sqrt(d') + (q.k)^2/(2 d') exactly as for the 273-feature
-//           map; the state written at the boundary is expanded back to 273.
+//           map.  The state at the boundary is either expanded back to 273
+//           rows or, for the folded map, is these 153 rows as they are.
 //   MMA1    A = phi(Q_c) phi(K_c)^T      (Taylor: Q_c K_c^T, then the closed
 //           form 1 + s/sqrt(d') + s^2/(2d') in the mask pass)   -> TMEM
 //   MMA3    S_aug += phi(K_c)^T V_aug   (feature rows in TMEM lanes)
@@ -82,10 +83,14 @@ struct FwdCfg {
 };
 
 struct FwdParams {
-    const float *s_in;  // [BH, F273/F, DV] nullable: state entering the sequence
-    const float *z_in;  // [BH, F273/F]
-    float *s_out;       // [BH, F273/F, DV] nullable
+    const float *s_in;  // [BH, F, DV] nullable: state entering the sequence
+    const float *z_in;  // [BH, F]
+    float *s_out;       // [BH, F, DV] nullable
     float *z_out;       // [BH, F] nullable
+    // Taylor boundary layout of s_in/z_in/s_out/z_out: 0 = 273 features (row
+    // pairs (a,b), (b,a) unfolded), 1 = the 153 folded features, which are
+    // the kernel's own rows 0..152.
+    int sym_state;
     float *den_out;     // [BH, N] nullable
     float *ws;          // [BH, P, FP, NA] segment increments (P > 1)
     void *o;            // [BH, N, DV] bf16
@@ -296,10 +301,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     }
                     if (p.s_in && f < Cfg::FSYM) {
                         // boundary rows of internal row f (Taylor: the symmetric pair, scaled)
-                        const int F = Cfg::TAYLOR ? 1 + DQK + DQK * DQK : DQK;
+                        const int F = !Cfg::TAYLOR ? DQK : p.sym_state ? Cfg::FSYM : 1 + DQK + DQK * DQK;
                         int r1 = f, r2 = -1;
                         float sc = 1.f;
-                        if (Cfg::TAYLOR) taylor_sym_to_full<16>(f, r1, r2, sc);
+                        if (Cfg::TAYLOR && !p.sym_state) taylor_sym_to_full<16>(f, r1, r2, sc);
 #pragma unroll
                         for (int e = 0; e < 16; ++e) {
                             const int col = c0 + e;
@@ -578,10 +583,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     continue;
                 }
                 if (f >= Cfg::FSYM) continue;
-                const int F = Cfg::TAYLOR ? 1 + DQK + DQK * DQK : DQK;
+                const int F = !Cfg::TAYLOR ? DQK : p.sym_state ? Cfg::FSYM : 1 + DQK + DQK * DQK;
                 int r1, r2;
                 float sc;
-                if (Cfg::TAYLOR) {
+                if (Cfg::TAYLOR && !p.sym_state) {
                     taylor_sym_to_full<16>(f, r1, r2, sc);
                 } else {
                     r1 = f; r2 = -1; sc = 1.f;

@@ -415,6 +415,16 @@ __global__ void feature_map_kernel(const T *__restrict__ x, T *__restrict__ phi,
             val = 1.f;
         } else if (f <= fp.dqk) {
             val = ld(xr + f - 1) * fp.inv_c1;
+        } else if (fp.fmap == LA_FMAP_TAYLOR2_SYM) {
+            const int i2 = f - 1 - fp.dqk;
+            if (i2 < fp.dqk) {
+                const float xa = ld(xr + i2);
+                val = xa * xa * fp.inv_c2;
+            } else {
+                int a, b;
+                sym_pair(i2 - fp.dqk, fp.dqk, a, b);
+                val = ld(xr + a) * ld(xr + b) * fp.inv_c3;
+            }
         } else {
             const int i2 = f - 1 - fp.dqk;
             const int a = i2 / fp.dqk, b = i2 - a * fp.dqk;

@@ -20,6 +20,17 @@
  *                   phi(q).phi(k) = 1 + q.k/sqrt(dqk) + (q.k)^2/(2 dqk)
  *                   (BASED page, Knowl 3, second-order Taylor map with the
  *                   scaling inside phi; 273 features for dqk = 16, Knowl 5).
+ *   LA_FMAP_TAYLOR2_SYM the same map with each pair of equal second-order
+ *                   features (a,b), (b,a) folded into one:
+ *                   phi(x) = [1 | x / dqk^(1/4) | x_a^2 / (sqrt(2) sqrt(dqk)) for
+ *                   each a | x_a x_b / sqrt(dqk) for a < b, row-major];
+ *                   F = 1 + 2 dqk + dqk (dqk - 1) / 2 (153 for dqk = 16, the
+ *                   count in the BASED page's state-size expression
+ *                   (d+1)(1 + 3d'/2 + d'^2/2), Knowl 7).  phi(q).phi(k) is the
+ *                   same as for TAYLOR2, so o, den and gradients are the same;
+ *                   only the state S, z is smaller: its pair row (a,b) holds
+ *                   (S[a,b] + S[b,a]) / sqrt(2) of the TAYLOR2 state.  A decode
+ *                   step moves 44 % fewer state bytes.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -44,11 +55,11 @@
  *    reported by la_get_device_status.
  *  - Results are deterministic: the same call on the same inputs gives the
  *    same bits.
- *  - Supported sizes: dqk in [1,128] for ELU1 and [1,16] for TAYLOR2;
+ *  - Supported sizes: dqk in [1,128] for ELU1 and [1,16] for the Taylor maps;
  *    dv in [1,128]; N >= 1; B*H*N*max(dqk,dv) < 2^31 elements.  The fast
  *    tensor-core paths cover bf16 with (ELU1, dqk = dv in {64,128}) and
- *    (TAYLOR2, dqk = 16, dv = 64); other valid combinations run on exact fp32
- *    CUDA-core kernels.
+ *    (TAYLOR2 or TAYLOR2_SYM, dqk = 16, dv = 64); other valid combinations run
+ *    on exact fp32 CUDA-core kernels.
  */
 #ifndef LA_H
 #define LA_H
@@ -66,7 +77,7 @@
 extern "C" {
 #endif
 
-typedef enum { LA_FMAP_ELU1 = 0, LA_FMAP_TAYLOR2 = 1 } la_fmap;
+typedef enum { LA_FMAP_ELU1 = 0, LA_FMAP_TAYLOR2 = 1, LA_FMAP_TAYLOR2_SYM = 2 } la_fmap;
 typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
 typedef enum {
     LA_OK = 0,
@@ -85,8 +96,9 @@ LA_API int la_version(void);
 LA_API const char *la_status_string(int status);
 
 /* Feature dimension F of a feature map: dqk for ELU1, 1 + dqk + dqk^2 for
- * TAYLOR2 (BASED page, Knowl 5: 273 for dqk = 16).  Returns -1 for an
- * unknown map or dqk < 1. */
+ * TAYLOR2 (BASED page, Knowl 5: 273 for dqk = 16), 1 + 2 dqk + dqk (dqk-1)/2
+ * for TAYLOR2_SYM (153 for dqk = 16).  Returns -1 for an unknown map or
+ * dqk < 1. */
 LA_API int64_t la_feature_dim(int fmap, int dqk);
 
 /* Bytes of device workspace la_forward needs for these sizes (0 if none).

@@ -36,6 +36,8 @@ def test_feature_dim_and_strings(lib):
     assert lib.la_feature_dim(1, 16) == 273
     assert lib.la_feature_dim(1, 0) == -1
     assert lib.la_feature_dim(7, 4) == -1
+    assert lib.la_feature_dim(2, 16) == 153           # folded Taylor map
+    assert lib.la_feature_dim(2, 1) == 3
     assert lib.la_status_string(0) == b"LA_OK"
     assert lib.la_status_string(4) == b"LA_ERR_TIMEOUT"
     assert lib.la_status_string(99) == b"LA_ERR_UNKNOWN"
@@ -114,6 +116,11 @@ def test_kernel_plan_and_workspace(lib):
     # Taylor B=8 H=16: 128 heads -> no split, no workspace
     assert la.la_forward_workspace_bytes(8, 16, 2048, 16, 64, 1, 1) == 0
     assert la.la_kernel_plan(0, 8, 16, 2048, 16, 64, 1, 1)[0] == 1
+    # the folded Taylor map takes the same tensor-core forward and workspace
+    assert la.la_kernel_plan(0, 8, 16, 2048, 16, 64, 2, 1)[0] == 1
+    assert la.la_kernel_plan(0, 1, 1, 65536, 16, 64, 2, 1) == la.la_kernel_plan(0, 1, 1, 65536, 16, 64, 1, 1)
+    assert la.la_forward_workspace_bytes(1, 1, 65536, 16, 64, 2, 1) == \
+        la.la_forward_workspace_bytes(1, 1, 65536, 16, 64, 1, 1) > 0
     # fp32 I/O runs on the exact CUDA-core kernel
     assert la.la_kernel_plan(0, 1, 1, 256, 32, 32, 0, 0) == (1, ["fwd_simt_kernel"])
     assert la.la_forward_workspace_bytes(1, 1, 256, 32, 32, 0, 0) == 0

@@ -16,12 +16,12 @@ from oracle import oracle as orc
 pytestmark = pytest.mark.gpu
 
 TOL = {W.F32: 1e-5, W.BF16: 1e-2}
-ELU1, TAYLOR2 = W.ELU1, W.TAYLOR2
+ELU1, TAYLOR2, TAYLOR2_SYM = W.ELU1, W.TAYLOR2, W.TAYLOR2_SYM
 DEV = "cuda"
 
 NS = [1, 2, 15, 16, 17, 63, 64, 65, 127, 128, 129, 257, 1000]
 DIMS = [(ELU1, 32, 32), (ELU1, 64, 64), (ELU1, 128, 128), (ELU1, 16, 48), (TAYLOR2, 16, 64),
-        (TAYLOR2, 4, 8)]
+        (TAYLOR2, 4, 8), (TAYLOR2_SYM, 16, 64), (TAYLOR2_SYM, 4, 8)]
 
 
 def gpu_forward(q, k, v, fmap, **kw):
@@ -36,7 +36,7 @@ def gpu_forward(q, k, v, fmap, **kw):
 def test_forward_small(fmap, dqk, dv, dtype):
     for N in NS:
         q, k, v, _ = W.random_qkv(1000 + N, 2, 2, N, dqk, dv, fmap=fmap, dtype=dtype,
-                                  scale=1.0 if fmap == TAYLOR2 else dqk ** -0.5)
+                                  scale=1.0 if fmap != ELU1 else dqk ** -0.5)
         r = gpu_forward(q, k, v, fmap, state=True, den=True)
         o_ref, den_ref = orc.forward_brute(fmap, q, k, v)
         _, _, s_ref, z_ref = orc.forward_recurrent(fmap, q, k, v)
@@ -49,7 +49,8 @@ def test_forward_small(fmap, dqk, dv, dtype):
 
 
 FROM_STATE = [(ELU1, 64, 64, W.BF16), (ELU1, 128, 128, W.BF16), (ELU1, 16, 48, W.BF16),
-              (ELU1, 32, 32, W.F32), (TAYLOR2, 16, 64, W.BF16), (TAYLOR2, 16, 64, W.F32)]
+              (ELU1, 32, 32, W.F32), (TAYLOR2, 16, 64, W.BF16), (TAYLOR2, 16, 64, W.F32),
+              (TAYLOR2_SYM, 16, 64, W.BF16), (TAYLOR2_SYM, 16, 64, W.F32)]
 
 
 def _start_state(fmap, dqk, dv, dtype, seed, B, H, skew):
@@ -57,7 +58,7 @@ def _start_state(fmap, dqk, dv, dtype, seed, B, H, skew):
     random data (fp64), optionally with noise that breaks the symmetry of the
     Taylor pair features (S[(a,b)] != S[(b,a)])."""
     q0, k0, v0, _ = W.random_qkv(seed, B, H, 300, dqk, dv, fmap=fmap, dtype=dtype,
-                                 scale=1.0 if fmap == TAYLOR2 else dqk ** -0.5)
+                                 scale=1.0 if fmap != ELU1 else dqk ** -0.5)
     _, _, s0, z0 = orc.forward_recurrent(fmap, q0, k0, v0)
     if skew:
         g = np.random.default_rng(seed)
@@ -70,9 +71,9 @@ def test_forward_from_state(fmap, dqk, dv, dtype):
     """la_forward_from_state against the oracle's recurrence started from the
     same state: outputs, denominators and the final state."""
     for B, H, N in ((1, 1, 1), (1, 2, 129), (2, 3, 1000), (1, 2, 3000)):
-        s0, z0 = _start_state(fmap, dqk, dv, dtype, 4000 + N, B, H, skew=fmap == TAYLOR2)
+        s0, z0 = _start_state(fmap, dqk, dv, dtype, 4000 + N, B, H, skew=fmap != ELU1)
         q, k, v, _ = W.random_qkv(5000 + N, B, H, N, dqk, dv, fmap=fmap, dtype=dtype,
-                                  scale=1.0 if fmap == TAYLOR2 else dqk ** -0.5)
+                                  scale=1.0 if fmap != ELU1 else dqk ** -0.5)
         r = gpu_forward(q, k, v, fmap, state=True, den=True, s_in=s0.to(DEV), z_in=z0.to(DEV))
         o_ref, den_ref, s_ref, z_ref = orc.forward_recurrent(fmap, q, k, v, s0, z0)
         tol = TOL[dtype]
@@ -87,7 +88,7 @@ def test_chunked_prefill_matches_one_call(fmap, dqk, dv, dtype):
     the rest with the returned state) equals the one-call forward."""
     B, H, N = 2, 2, 1100
     q, k, v, _ = W.random_qkv(6000, B, H, N, dqk, dv, fmap=fmap, dtype=dtype,
-                              scale=1.0 if fmap == TAYLOR2 else dqk ** -0.5)
+                              scale=1.0 if fmap != ELU1 else dqk ** -0.5)
     o_ref, den_ref, s_ref, z_ref = orc.forward_recurrent(fmap, q, k, v)
     cuts = [0, 1, 130, 640, N]
     s = z = None
@@ -109,7 +110,7 @@ def test_chunked_prefill_matches_one_call(fmap, dqk, dv, dtype):
 def test_backward_small(fmap, dqk, dv, dtype):
     for N in (1, 17, 64, 65, 200, 300):
         q, k, v, do = W.random_qkv(2000 + N, 1, 2, N, dqk, dv, fmap=fmap, dtype=dtype,
-                                   scale=1.0 if fmap == TAYLOR2 else dqk ** -0.5, with_dout=True)
+                                   scale=1.0 if fmap != ELU1 else dqk ** -0.5, with_dout=True)
         qd, kd, vd, dod = (t.to(DEV) for t in (q, k, v, do))
         dq, dk, dvv = la.la_backward(qd, kd, vd, dod, fmap)
         torch.cuda.synchronize()
@@ -128,7 +129,7 @@ def test_backward_small(fmap, dqk, dv, dtype):
 
 
 @pytest.mark.parametrize("dtype", [W.F32, W.BF16])
-@pytest.mark.parametrize("fmap,dqk,dv", [(TAYLOR2, 16, 64), (ELU1, 64, 64), (ELU1, 32, 48)])
+@pytest.mark.parametrize("fmap,dqk,dv", [(TAYLOR2, 16, 64), (TAYLOR2_SYM, 16, 64), (ELU1, 64, 64), (ELU1, 32, 48)])
 def test_decode_small(fmap, dqk, dv, dtype):
     P, T = 37, 20
     q, k, v, _ = W.random_qkv(3000, 3, 2, P + T, dqk, dv, fmap=fmap, dtype=dtype)
@@ -149,13 +150,31 @@ def test_decode_small(fmap, dqk, dv, dtype):
 
 
 @pytest.mark.parametrize("dtype", [W.F32, W.BF16])
-@pytest.mark.parametrize("fmap,dqk", [(ELU1, 64), (TAYLOR2, 16), (TAYLOR2, 3)])
+@pytest.mark.parametrize("fmap,dqk", [(ELU1, 64), (TAYLOR2, 16), (TAYLOR2, 3), (TAYLOR2_SYM, 16), (TAYLOR2_SYM, 3)])
 def test_feature_map(fmap, dqk, dtype):
     x, _, _, _ = W.random_qkv(4000, 1, 3, 50, dqk, 8, dtype=dtype)
     phi = la.la_feature_map(x.to(DEV), fmap).cpu()
     ref = orc.phi(fmap, x)
     tol = 1e-6 if dtype == W.F32 else 4e-3
     np.testing.assert_allclose(phi.double().numpy(), ref, rtol=tol, atol=tol)
+
+
+@pytest.mark.parametrize("dtype", [W.F32, W.BF16])
+def test_folded_state_is_folded_full_state(dtype):
+    # The two Taylor maps give the same outputs; the folded state's pair row is
+    # (S[a,b] + S[b,a]) / sqrt(2) of the 273-row state, its square rows S[a,a].
+    q, k, v, _ = W.random_qkv(7000, 2, 3, 700, 16, 64, fmap=TAYLOR2, dtype=dtype)
+    full = gpu_forward(q, k, v, TAYLOR2, state=True, den=True)
+    sym = gpu_forward(q, k, v, TAYLOR2_SYM, state=True, den=True)
+    tol = TOL[dtype]
+    assert orc.max_rel_l2(sym["o"].double(), full["o"].double()) <= tol
+    assert orc.max_rel_l2(sym["den"], full["den"]) <= tol
+    d = 16
+    sf = full["s"].double()
+    rows = [sf[:, :, :1 + d]] + [sf[:, :, 1 + d + a * d + a][:, :, None] for a in range(d)]
+    rows += [((sf[:, :, 1 + d + a * d + b] + sf[:, :, 1 + d + b * d + a]) / 2 ** 0.5)[:, :, None]
+             for a in range(d) for b in range(a + 1, d)]
+    assert orc.max_rel_l2(sym["s"], torch.cat(rows, 2)) <= tol
 
 
 def test_forward_deterministic():
@@ -229,8 +248,9 @@ def test_workload_elu_bf16_train():
     assert ((lhs - rhs).norm() / rhs.norm()).item() < 1e-2
 
 
-def test_workload_taylor_decode():
-    w = W.BY_NAME["taylor_decode"]
+@pytest.mark.parametrize("name", ["taylor_decode", "taylor_decode_sym"])
+def test_workload_taylor_decode(name):
+    w = W.BY_NAME[name]
     (q, k, v), (sq, sk, sv) = W.make_decode_inputs(w)
     r = la.la_forward(q.to(DEV), k.to(DEV), v.to(DEV), w.fmap, state=True)
     s, z = r["s"], r["z"]

@@ -38,6 +38,7 @@ import torch
 
 ELU1 = 0
 TAYLOR2 = 1
+TAYLOR2_SYM = 2
 F32 = 0
 BF16 = 1
 
@@ -65,11 +66,16 @@ class Workload:
 
     @property
     def feature_dim(self) -> int:
-        # ELU: one feature per input coordinate; Taylor: 1 + d' + d'^2.
-        return self.dqk if self.fmap == ELU1 else 1 + self.dqk + self.dqk * self.dqk
+        # ELU: one feature per input coordinate; Taylor: 1 + d' + d'^2; the
+        # folded Taylor map: 1 + 2d' + d'(d'-1)/2.
+        if self.fmap == ELU1:
+            return self.dqk
+        if self.fmap == TAYLOR2:
+            return 1 + self.dqk + self.dqk * self.dqk
+        return 1 + 2 * self.dqk + self.dqk * (self.dqk - 1) // 2
 
     def describe(self) -> str:
-        fm = "elu1" if self.fmap == ELU1 else "taylor2"
+        fm = {ELU1: "elu1", TAYLOR2: "taylor2", TAYLOR2_SYM: "taylor2sym"}[self.fmap]
         dt = "f32" if self.dtype == F32 else "bf16"
         s = f"{self.name}: {fm} {dt} B={self.B} H={self.H} N={self.N} dqk={self.dqk} dv={self.dv}"
         if self.decode_steps:
@@ -83,6 +89,8 @@ WORKLOADS = [
     Workload("taylor_bf16_fwd", 2, TAYLOR2, BF16, 8, 16, 2048, 16, 64, 1.0),
     Workload("elu_bf16_train", 3, ELU1, BF16, 2, 16, 16384, 128, 128, 1.0 / math.sqrt(128), backward=True),
     Workload("taylor_decode", 4, TAYLOR2, F32, 256, 16, 2048, 16, 64, 1.0, decode_steps=1024),
+    # the same decode with the folded Taylor state (153 rows instead of 273)
+    Workload("taylor_decode_sym", 4, TAYLOR2_SYM, F32, 256, 16, 2048, 16, 64, 1.0, decode_steps=1024),
 ]
 BY_NAME = {w.name: w for w in WORKLOADS}
 
