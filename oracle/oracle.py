@@ -157,6 +157,38 @@ def forward_recurrent(fmap: int, q, k, v, s0=None, z0=None):
     return o, den, s, z
 
 
+def forward_varlen(fmap: int, q, k, v, cu_seqlens, s0=None, z0=None):
+    """A batch of sequences of different lengths packed along the token axis:
+    q, k [H, T, dqk], v [H, T, dv], sequence n holding tokens
+    cu_seqlens[n] .. cu_seqlens[n+1] - 1 of every head.  Each sequence runs
+    the recurrence of Knowl 3 on its own (from zero, or from s0[n], z0[n]);
+    nothing crosses a boundary.  Returns (o [H,T,dv], den [H,T],
+    s_final [nseq,H,F,dv], z_final [nseq,H,F]); an empty sequence returns its
+    starting state."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    H, T, dqk = q.shape
+    dv = v.shape[-1]
+    F = feature_dim(fmap, dqk)
+    cu = [int(c) for c in np.asarray(cu_seqlens).reshape(-1)]
+    nseq = len(cu) - 1
+    assert cu[0] == 0 and cu[-1] == T and all(a <= b for a, b in zip(cu[:-1], cu[1:]))
+    s0 = None if s0 is None else _f64(s0)
+    z0 = None if z0 is None else _f64(z0)
+    o = np.zeros((H, T, dv))
+    den = np.zeros((H, T))
+    s = np.zeros((nseq, H, F, dv)) if s0 is None else s0.copy()
+    z = np.zeros((nseq, H, F)) if z0 is None else z0.copy()
+    for n in range(nseq):
+        a, b = cu[n], cu[n + 1]
+        if b == a:
+            continue
+        on, dn, sn, zn = forward_recurrent(fmap, q[None, :, a:b], k[None, :, a:b], v[None, :, a:b],
+                                           None if s0 is None else s0[n:n + 1],
+                                           None if z0 is None else z0[n:n + 1])
+        o[:, a:b], den[:, a:b], s[n], z[n] = on[0], dn[0], sn[0], zn[0]
+    return o, den, s, z
+
+
 def decode_step(fmap: int, q, k, v, s, z):
     """One recurrent step on the state (s, z), updated in place (float64
     arrays [BH,F,dv] / [BH,F]); output from the updated state (Knowl 5)."""

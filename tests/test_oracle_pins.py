@@ -298,6 +298,45 @@ def test_forward_from_state_and_decode(orc, fmap):
     np.testing.assert_allclose(s2, sfull, rtol=1e-12, atol=1e-12)
 
 
+@pytest.mark.parametrize("fmap", [ELU1, TAYLOR2_SYM])
+def test_varlen_sequences_are_independent(orc, fmap):
+    # Packed sequences: each is its own recurrence (Knowl 3 per sequence).
+    # (a) A sequence's outputs and final state are those of a separate forward
+    #     over it alone, by brute force (a different algorithm);
+    # (b) two packed copies of one sequence give identical outputs, so no
+    #     state crosses a boundary;
+    # (c) an empty sequence returns its starting state.
+    d, dv, H = (6, 5, 2) if fmap == ELU1 else (3, 4, 2)
+    lens = [7, 0, 1, 12, 7]
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    T = int(cu[-1])
+    q = rnd(100, H, T, d); k = rnd(101, H, T, d); v = rnd(102, H, T, dv)
+    # the last sequence repeats the first
+    q[:, cu[4]:cu[5]] = q[:, :7]; k[:, cu[4]:cu[5]] = k[:, :7]; v[:, cu[4]:cu[5]] = v[:, :7]
+    F = orc.feature_dim(fmap, d)
+    s0 = rnd(103, 5, H, F, dv); z0 = np.abs(rnd(104, 5, H, F)) + 1.0
+    o, den, s, z = orc.forward_varlen(fmap, q, k, v, cu)
+    for n in range(5):
+        a, b = cu[n], cu[n + 1]
+        if a == b:
+            assert (s[n] == 0).all() and (z[n] == 0).all()
+            continue
+        ob, db = orc.forward_brute(fmap, q[None, :, a:b], k[None, :, a:b], v[None, :, a:b])
+        np.testing.assert_allclose(o[:, a:b], ob[0], rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(den[:, a:b], db[0], rtol=1e-12)
+        pk = orc.phi(fmap, k[:, a:b])
+        np.testing.assert_allclose(s[n], np.einsum("htf,htc->hfc", pk, v[:, a:b]), rtol=1e-11, atol=1e-12)
+    np.testing.assert_array_equal(o[:, cu[4]:cu[5]], o[:, :7])
+    # from a given state: the empty sequence keeps it, the others continue it
+    o2, _, s2, z2 = orc.forward_varlen(fmap, q, k, v, cu, s0, z0)
+    np.testing.assert_array_equal(s2[1], s0[1])
+    np.testing.assert_array_equal(z2[1], z0[1])
+    a, b = cu[3], cu[4]
+    ref, _, sr, _ = orc.forward_recurrent(fmap, q[None, :, a:b], k[None, :, a:b], v[None, :, a:b], s0[3:4], z0[3:4])
+    np.testing.assert_allclose(o2[:, a:b], ref[0], rtol=1e-12)
+    np.testing.assert_allclose(s2[3], sr[0], rtol=1e-12)
+
+
 # ----------------------------------------------------------------- backward
 
 def _loss_grad_fd(orc, fmap, q, k, v, do, h=1e-6):
