@@ -75,6 +75,10 @@ def load_library(path: str | None = None):
     lib.la_forward_from_state.argtypes = [vp] * 10 + [sz] + [i] * 7 + [vp]
     lib.la_forward_from_state.restype = i
     lib.la_forward_noalloc.argtypes = [vp] * 7 + [i] * 7 + [vp]
+    lib.la_forward_varlen.argtypes = [vp] * 5 + [i] * 3 + [vp] * 6 + [sz] + [i] * 5 + [vp]
+    lib.la_forward_varlen.restype = i
+    lib.la_forward_varlen_workspace_bytes.argtypes = [i] * 7
+    lib.la_forward_varlen_workspace_bytes.restype = sz
     lib.la_forward_noalloc.restype = i
     lib.la_kernel_plan.argtypes = [i] * 8 + [ctypes.c_char_p, sz]
     lib.la_kernel_plan.restype = i
@@ -163,6 +167,52 @@ def la_forward(q, k, v, fmap, *, state=False, den=False, out=None, workspace=Non
     _check(lib.la_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(res.get("s")), _ptr(res.get("z")),
                           _ptr(res.get("den")), _ptr(workspace), wsb, B, H, N, dqk, dv, fmap, dt,
                           _stream()), "la_forward")
+    return res
+
+
+def la_forward_varlen_workspace_bytes(nseq, H, max_seqlen, dqk, dv, fmap, dtype) -> int:
+    return int(load_library().la_forward_varlen_workspace_bytes(nseq, H, max_seqlen, dqk, dv, fmap, dtype))
+
+
+def la_forward_varlen(q, k, v, cu_seqlens, max_seqlen, fmap, *, state=False, den=False, out=None,
+                      workspace=None, s_in=None, z_in=None):
+    """Forward over sequences packed along the token axis: q, k [H,T,dqk],
+    v [H,T,dv]; cu_seqlens int32 [nseq+1] on the device (sequence n is tokens
+    cu_seqlens[n] .. cu_seqlens[n+1]-1); max_seqlen bounds every length.
+
+    Returns {"o": [H,T,dv], and if requested "s": [nseq,H,F,dv], "z": [nseq,H,F],
+    "den": [H,T]}.  s_in/z_in [nseq,H,F,dv]/[nseq,H,F] start each sequence.
+    """
+    lib = load_library()
+    _dev(q, k, v, out, cu_seqlens)
+    H, T, dqk = q.shape
+    dv = v.shape[-1]
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or not cu_seqlens.is_contiguous():
+        raise ValueError("cu_seqlens must be a contiguous int32 vector")
+    nseq = cu_seqlens.numel() - 1
+    dt = _dtype_code(q)
+    F = la_feature_dim(fmap, dqk)
+    o = out if out is not None else torch.empty(H, T, dv, dtype=q.dtype, device=q.device)
+    res = {"o": o}
+    if state:
+        res["s"] = torch.empty(nseq, H, F, dv, dtype=torch.float32, device=q.device)
+        res["z"] = torch.empty(nseq, H, F, dtype=torch.float32, device=q.device)
+    if den:
+        res["den"] = torch.empty(H, T, dtype=torch.float32, device=q.device)
+    if (s_in is None) != (z_in is None):
+        raise ValueError("s_in and z_in go together")
+    if s_in is not None:
+        _dev(s_in, z_in)
+        if s_in.dtype != torch.float32 or z_in.dtype != torch.float32 or not s_in.is_contiguous() \
+                or not z_in.is_contiguous() or tuple(s_in.shape) != (nseq, H, F, dv) or tuple(z_in.shape) != (nseq, H, F):
+            raise ValueError("s_in must be fp32 [nseq,H,F,dv] and z_in fp32 [nseq,H,F], contiguous")
+    wsb = la_forward_varlen_workspace_bytes(nseq, H, min(max_seqlen, T), dqk, dv, fmap, dt)
+    if workspace is None and wsb:
+        workspace = torch.empty(wsb, dtype=torch.uint8, device=q.device)
+    _check(lib.la_forward_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(cu_seqlens), nseq, max_seqlen, T,
+                                 _ptr(s_in), _ptr(z_in), _ptr(res.get("s")), _ptr(res.get("z")),
+                                 _ptr(res.get("den")), _ptr(workspace), wsb, H, dqk, dv, fmap, dt, _stream()),
+           "la_forward_varlen")
     return res
 
 

@@ -209,7 +209,7 @@ bool pick_chunk(MakeLayout make, int F, int dqk, int dv, Layout *out, size_t *by
 template <typename T>
 la_status forward_simt(const void *q, const void *k, const void *v, void *o, const float *s_in,
                        const float *z_in, float *s_out, float *z_out, float *den_out, int B, int H, int N,
-                       int dqk, int dv, int fmap, cudaStream_t stream)
+                       int dqk, int dv, int fmap, cudaStream_t stream, const int *cu = nullptr, int T_total = 0)
 {
     const FmapParams fp = make_fmap(fmap, dqk);
     SimtFwdSmem L;
@@ -217,7 +217,8 @@ la_status forward_simt(const void *q, const void *k, const void *v, void *o, con
     if (!pick_chunk(simt_fwd_layout, fp.F, dqk, dv, &L, &bytes)) return LA_ERR_UNSUPPORTED;
     if (set_smem<fwd_simt_kernel<T>>(bytes) != LA_OK) return LA_ERR_CUDA;
     fwd_simt_kernel<T><<<B * H, kSimtThreads, bytes, stream>>>(
-        (const T *)q, (const T *)k, (const T *)v, (T *)o, s_in, z_in, s_out, z_out, den_out, N, dv, fp, L);
+        (const T *)q, (const T *)k, (const T *)v, (T *)o, s_in, z_in, s_out, z_out, den_out, N, dv, fp, L, cu, H,
+        T_total);
     return launch_status();
 }
 
@@ -317,14 +318,19 @@ bool make_map(CUtensorMap *m, const void *base, int inner, int N, int BH, int bo
 template <class Cfg>
 la_status forward_tc_launch(const void *q, const void *k, const void *v, void *o, const float *s_in,
                             const float *z_in, float *s_out, float *z_out, float *den_out, void *workspace, int B,
-                            int H, int N, cudaStream_t stream, bool sym_state = false)
+                            int H, int N, cudaStream_t stream, bool sym_state = false, const int *cu = nullptr,
+                            int T = 0)
 {
+    // Fixed length: B*H slices of N tokens, tensors [B*H, N, *].  Packed
+    // sequences (cu != null): B sequences of at most N tokens, tensors [H, T, *].
     const int BH = B * H;
+    const int map_rows = cu ? T : N, map_slices = cu ? H : BH;
     CUtensorMap tq, tk, tv;
     const CUtensorMapSwizzle qsw = Cfg::TAYLOR ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_128B;
     const int qbox = Cfg::TAYLOR ? 16 : 64;
-    if (!make_map(&tq, q, Cfg::DQK, N, BH, qbox, qsw) || !make_map(&tk, k, Cfg::DQK, N, BH, qbox, qsw) ||
-        !make_map(&tv, v, Cfg::DV, N, BH, 16, CU_TENSOR_MAP_SWIZZLE_32B))
+    if (!make_map(&tq, q, Cfg::DQK, map_rows, map_slices, qbox, qsw) ||
+        !make_map(&tk, k, Cfg::DQK, map_rows, map_slices, qbox, qsw) ||
+        !make_map(&tv, v, Cfg::DV, map_rows, map_slices, 16, CU_TENSOR_MAP_SWIZZLE_32B))
         return LA_ERR_CUDA;
     FwdParams p;
     p.s_in = s_in;
@@ -336,6 +342,10 @@ la_status forward_tc_launch(const void *q, const void *k, const void *v, void *o
     p.ws = (float *)workspace;
     p.o = o;
     p.N = N;
+    p.cu = cu;
+    p.H = H;
+    p.T = T;
+    p.max_len = N;
     tc_segments(B, H, N, &p.P, &p.cps, &p.nchunks);
     const double d = (double)Cfg::DQK;
     p.inv_c1 = (float)(1.0 / pow(d, 0.25));
@@ -411,16 +421,16 @@ la_status forward_split64(const void *q, const void *k, const void *v, void *o, 
 la_status forward_tc(const void *q, const void *k, const void *v, void *o, const float *s_in, const float *z_in,
                      float *s_out, float *z_out,
                      float *den_out, void *workspace, int B, int H, int N, int dqk, int dv, int fmap,
-                     cudaStream_t stream)
+                     cudaStream_t stream, const int *cu = nullptr, int T = 0)
 {
     if (fmap != LA_FMAP_ELU1)
         return forward_tc_launch<FwdCfg<16, 64, true>>(q, k, v, o, s_in, z_in, s_out, z_out, den_out, workspace, B, H, N,
-                                                       stream, fmap == LA_FMAP_TAYLOR2_SYM);
+                                                       stream, fmap == LA_FMAP_TAYLOR2_SYM, cu, T);
     if (dqk == 64)
         return forward_tc_launch<FwdCfg<64, 64, false>>(q, k, v, o, s_in, z_in, s_out, z_out, den_out, workspace, B, H,
-                                                        N, stream);
+                                                        N, stream, false, cu, T);
     return forward_tc_launch<FwdCfg<128, 128, false>>(q, k, v, o, s_in, z_in, s_out, z_out, den_out, workspace, B, H,
-                                                      N, stream);
+                                                      N, stream, false, cu, T);
 }
 
 la_status backward_tc(const void *q, const void *k, const void *v, const void *dout, void *dq, void *dk,
@@ -594,6 +604,53 @@ la_status la_forward_from_state(const void *q, const void *k, const void *v, voi
         return LA_ERR_INVALID_ARG;
     return forward_impl(q, k, v, o, s_in, z_in, s_out, z_out, den_out, workspace, workspace_bytes, B, H, N, dqk,
                         dv, fmap, dtype, stream);
+}
+
+size_t la_forward_varlen_workspace_bytes(int nseq, int H, int max_seqlen, int dqk, int dv, int fmap, int dtype)
+{
+    if (check_shape(nseq, H, max_seqlen, dqk, dv, fmap, dtype) != LA_OK) return 0;
+    if (!tc_forward_shape(dqk, dv, fmap, dtype)) return 0;
+    int P, cps, nc;
+    tc_segments(nseq, H, max_seqlen, &P, &cps, &nc);
+    if (P <= 1) return 0;
+    return (size_t)nseq * H * P * tc_increment_floats(dqk, dv, fmap) * sizeof(float);
+}
+
+la_status la_forward_varlen(const void *q, const void *k, const void *v, void *o, const int32_t *cu_seqlens,
+                            int nseq, int max_seqlen, int T, const float *s_in, const float *z_in, float *s_out,
+                            float *z_out, float *den_out, void *workspace, size_t workspace_bytes, int H, int dqk,
+                            int dv, int fmap, int dtype, void *stream)
+{
+    if (T < 1) return LA_ERR_INVALID_ARG;
+    if (max_seqlen > T) max_seqlen = T;   // no sequence is longer than the batch
+    la_status sh = check_shape(nseq, H, max_seqlen, dqk, dv, fmap, dtype);
+    if (sh != LA_OK) return sh;
+    sh = check_shape(1, H, T, dqk, dv, fmap, dtype);   // element counts of the packed tensors
+    if (sh != LA_OK) return sh;
+    if (!q || !k || !v || !o || !cu_seqlens || !aligned(cu_seqlens, 4)) return LA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(s_out, 16) ||
+        !aligned(z_out, 4) || !aligned(den_out, 4))
+        return LA_ERR_INVALID_ARG;
+    if ((s_in == nullptr) != (z_in == nullptr)) return LA_ERR_INVALID_ARG;
+    const size_t F = (size_t)la_feature_dim(fmap, dqk);
+    if (s_in) {
+        if (!aligned(s_in, 16) || !aligned(z_in, 4)) return LA_ERR_INVALID_ARG;
+        const size_t sb = (size_t)nseq * H * F * dv * sizeof(float), zb = (size_t)nseq * H * F * sizeof(float);
+        if (overlaps(s_in, sb, s_out, sb) || overlaps(s_in, sb, z_out, zb) || overlaps(z_in, zb, s_out, sb) ||
+            overlaps(z_in, zb, z_out, zb))
+            return LA_ERR_INVALID_ARG;
+    }
+    const size_t need = la_forward_varlen_workspace_bytes(nseq, H, max_seqlen, dqk, dv, fmap, dtype);
+    if (workspace_bytes < need || (need && (!workspace || !aligned(workspace, 16)))) return LA_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (tc_forward_shape(dqk, dv, fmap, dtype))
+        return forward_tc(q, k, v, o, s_in, z_in, s_out, z_out, den_out, workspace, nseq, H, max_seqlen, dqk, dv,
+                          fmap, st, cu_seqlens, T);
+    if (dtype == LA_F32)
+        return forward_simt<float>(q, k, v, o, s_in, z_in, s_out, z_out, den_out, nseq, H, max_seqlen, dqk, dv,
+                                   fmap, st, cu_seqlens, T);
+    return forward_simt<__nv_bfloat16>(q, k, v, o, s_in, z_in, s_out, z_out, den_out, nseq, H, max_seqlen, dqk, dv,
+                                       fmap, st, cu_seqlens, T);
 }
 
 // Allocation-free forward: la_forward with its workspace taken from a

@@ -95,6 +95,12 @@ struct FwdParams {
     float *ws;          // [BH, P, FP, NA] segment increments (P > 1)
     void *o;            // [BH, N, DV] bf16
     int N, P, nchunks, cps;
+    // Packed sequences (nullable): sequence n holds tokens cu[n] .. cu[n+1]-1
+    // of every head of a [H, T, *] batch; the grid is nseq x H x P blocks and
+    // the state slices are (n, h).  N, nchunks and cps are then those of the
+    // longest allowed sequence, max_len.
+    const int *cu;
+    int H, T, max_len;
     float inv_c1, inv_c2;       // Taylor: 1/d'^(1/4), 1/(sqrt(2) sqrt(d'))
     float k1, k2;               // Taylor closed form: 1/sqrt(d'), 1/(2 d')
 };
@@ -234,11 +240,30 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     // column half w / 4 of the row it owns there.
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wq = warp & 3, half = warp >> 2, row = wq * 32 + lane;
-    const int bh = blockIdx.x / p.P, seg = blockIdx.x % p.P;
-    if (MODE == 1 && seg == p.P - 1) return;  // the last segment's increment is never read
+    const int bh = blockIdx.x / p.P, seg = blockIdx.x % p.P;   // bh: the state slice
+    // This slice's tokens: fixed length N at rows bh*N.. of a [BH, N, *] tensor
+    // (TMA coordinates (x, t, bh)), or packed sequence n at rows h*T + cu[n]..
+    // of a [H, T, *] tensor (TMA coordinates (x, cu[n] + t, h)).
+    int N = p.N, nchunks = p.nchunks, nseg = p.P, tz = bh, t_base = 0;
+    long long row0 = (long long)bh * p.N;
+    if (p.cu) {
+        const int n = bh / p.H, h = bh - n * p.H;
+        const int a = p.cu[n], b = p.cu[n + 1];
+        if (a < 0 || b < a || b > p.T || b - a > p.max_len) {
+            if (tid == 0 && seg == 0) report(kStatusCheck);
+            return;
+        }
+        N = b - a;
+        nchunks = (N + C - 1) / C;
+        nseg = max(1, (nchunks + p.cps - 1) / p.cps);
+        if (seg >= nseg) return;   // a shorter sequence: no chunks for this segment
+        tz = h;
+        t_base = a;
+        row0 = (long long)h * p.T + a;
+    }
+    if (MODE == 1 && seg == nseg - 1) return;  // the last segment's increment is never read
     const int c_begin = seg * p.cps;
-    const int c_end = min(p.nchunks, c_begin + p.cps);
-    const int N = p.N;
+    const int c_end = min(nchunks, c_begin + p.cps);
 
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) mbar_init(&tma_bar[s], 1);
@@ -274,11 +299,12 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         constexpr int QBOX = Cfg::TAYLOR ? 16 : 64;
         for (int x = 0; x < DQK; x += QBOX) {
             const int off = Cfg::TAYLOR ? 0 : (x / 64) * C * 128;
-            if (MODE == 0) tma_load_3d(q_dst + off, &tm_q, &tma_bar[s], x, t0, bh);
-            tma_load_3d(k_dst + off, &tm_k, &tma_bar[s], x, t0, bh);
+            if (MODE == 0) tma_load_3d(q_dst + off, &tm_q, &tma_bar[s], x, t_base + t0, tz);
+            tma_load_3d(k_dst + off, &tm_k, &tma_bar[s], x, t_base + t0, tz);
         }
         uint8_t *v_dst = smem + Cfg::OFF_V + s * Cfg::V_TILE;
-        for (int x = 0; x < DV; x += 16) tma_load_3d(v_dst + (x / 16) * Cfg::V_BLK, &tm_v, &tma_bar[s], x, t0, bh);
+        for (int x = 0; x < DV; x += 16)
+            tma_load_3d(v_dst + (x / 16) * Cfg::V_BLK, &tm_v, &tma_bar[s], x, t_base + t0, tz);
     };
 
     bool have_state = false;
@@ -521,13 +547,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const float den = d16[0];
             const float inv = 1.f / den;
             if (i < nvalid) {
-                __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + ((size_t)bh * N + t0 + i) * DV + half * DH;
+                __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + (size_t)(row0 + t0 + i) * DV + half * DH;
 #pragma unroll
                 for (int c0 = 0; c0 < DH; c0 += 8)
                     *reinterpret_cast<uint4 *>(orow + c0) =
                         make_uint4(pack_bf16(o[c0] * inv, o[c0 + 1] * inv), pack_bf16(o[c0 + 2] * inv, o[c0 + 3] * inv),
                                    pack_bf16(o[c0 + 4] * inv, o[c0 + 5] * inv), pack_bf16(o[c0 + 6] * inv, o[c0 + 7] * inv));
-                if (p.den_out && half == 0) p.den_out[(size_t)bh * N + t0 + i] = den;
+                if (p.den_out && half == 0) p.den_out[row0 + t0 + i] = den;
             }
         }
         // ---- state snapshot for the next chunk (bf16, MN-major SW32)
@@ -563,7 +589,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
     // ---- segment increment (MODE 1) or final state (MODE 0, last segment)
     const bool write_ws = (MODE == 1);
-    const bool write_final = (MODE == 0) && (seg == p.P - 1) && (p.s_out || p.z_out) && !*abort_flag;
+    const bool write_final = (MODE == 0) && (seg == nseg - 1) && (p.s_out || p.z_out) && !*abort_flag;
     if ((write_ws || write_final) && !*abort_flag) {
 #pragma unroll 1
         for (int t = 0; t < Cfg::NT; ++t) {
@@ -575,6 +601,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 float v[16];
                 tmem_ld16(tmem + lane_base + Cfg::COL_S + t * NA + c0, v);
                 tmem_ld_wait();
+                if (!have_state) {   // an empty packed sequence with no entering state
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) v[e] = 0.f;
+                }
                 if (f < 0 || f >= FP) continue;
                 if (write_ws) {
                     float *dst = p.ws + ((size_t)(bh * p.P + seg) * FP + f) * NA + c0;

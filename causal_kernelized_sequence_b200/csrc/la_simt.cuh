@@ -45,7 +45,8 @@ __global__ void __launch_bounds__(kSimtThreads)
 fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                 T *__restrict__ o, const float *__restrict__ s_in, const float *__restrict__ z_in,
                 float *__restrict__ s_out, float *__restrict__ z_out,
-                float *__restrict__ den_out, int N, int dv, FmapParams fp, SimtFwdSmem L)
+                float *__restrict__ den_out, int N, int dv, FmapParams fp, SimtFwdSmem L,
+                const int *__restrict__ cu = nullptr, int H = 0, int T_total = 0)
 {
     extern __shared__ float sm[];
     const int F = fp.F, dqk = fp.dqk, C = L.C, FS = L.FS, DS = L.DS;
@@ -61,11 +62,24 @@ fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
 
     const int tid = threadIdx.x, nt = blockDim.x;
     const int lane = tid & 31, warp = tid >> 5, nwarps = nt >> 5;
-    const size_t bh = blockIdx.x;
-    const T *qb = q + bh * N * dqk;
-    const T *kb = k + bh * N * dqk;
-    const T *vb = v + bh * N * dv;
-    T *ob = o + bh * N * dv;
+    const size_t bh = blockIdx.x;   // the state slice
+    // token rows of this slice: bh*N.. of [BH, N, *], or for packed sequences
+    // (cu != null; slice = (n, h)) h*T_total + cu[n] .. of [H, T_total, *]
+    size_t row0 = bh * N;
+    if (cu) {
+        const int n = (int)bh / H, h = (int)bh - n * H;
+        const int a = cu[n], b = cu[n + 1];
+        if (a < 0 || b < a || b > T_total || b - a > N) {   // N: the caller's max_seqlen
+            if (tid == 0) report(kStatusCheck);
+            return;
+        }
+        N = b - a;
+        row0 = (size_t)h * T_total + a;
+    }
+    const T *qb = q + row0 * dqk;
+    const T *kb = k + row0 * dqk;
+    const T *vb = v + row0 * dv;
+    T *ob = o + row0 * dv;
 
     // state entering the sequence: zero, or the given (s_in, z_in)
     for (int i = tid; i < F * DS; i += nt) {
@@ -106,7 +120,7 @@ fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
             for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
             if (lane == 0) {
                 den[i] = acc;
-                if (den_out) den_out[bh * N + t0 + i] = acc;
+                if (den_out) den_out[row0 + t0 + i] = acc;
             }
         }
         __syncthreads();

@@ -158,6 +158,47 @@ LA_API la_status la_forward_from_state(const void *q, const void *k, const void 
                                        int B, int H, int N, int dqk, int dv, int fmap, int dtype,
                                        void *stream);
 
+/* Bytes of device workspace la_forward_varlen needs for nseq sequences of at
+ * most max_seqlen tokens (0 if none); the rules of la_forward_workspace_bytes. */
+LA_API size_t la_forward_varlen_workspace_bytes(int nseq, int H, int max_seqlen, int dqk, int dv,
+                                                int fmap, int dtype);
+
+/* Forward over a batch of sequences of different lengths, packed along the
+ * token axis without padding.  Each sequence is its own causal recurrence
+ * (BASED page, Knowl 3, one state per sequence and head), started from zero
+ * or from s_in; no state crosses from one sequence to the next.  It is
+ * la_forward (or la_forward_from_state) on B = 1, N = T with the state reset at
+ * every sequence boundary.
+ *   q, k        [H, T, dqk] dtype, read; v [H, T, dv] dtype, read
+ *   o           [H, T, dv]  dtype, written
+ *   cu_seqlens  [nseq + 1] int32, DEVICE memory, read: sequence n holds tokens
+ *               cu_seqlens[n] .. cu_seqlens[n+1] - 1 of every head;
+ *               0 = cu_seqlens[0] <= cu_seqlens[1] <= ... <= cu_seqlens[nseq] = T.
+ *               Empty sequences are allowed (their final state is their
+ *               starting state).
+ *   max_seqlen  a bound on every sequence's length, >= 1; a bound above T is
+ *               taken as T (it sizes the grid and the workspace, which
+ *               la_forward_varlen_workspace_bytes(nseq, H, min(max_seqlen, T),
+ *               ...) gives; a tight bound is fastest)
+ *   s_in, z_in  [nseq, H, F, dv], [nseq, H, F] fp32, nullable (both or neither):
+ *               the state entering each sequence; must not overlap s_out/z_out
+ *   s_out, z_out [nseq, H, F, dv], [nseq, H, F] fp32, nullable: final states
+ *   den_out     [H, T] fp32, nullable
+ *   workspace   at least la_forward_varlen_workspace_bytes(...) bytes
+ * The lengths live on the device, so they are checked there: a sequence with
+ * cu_seqlens[n] < 0, a decreasing pair, an end beyond T or a length above
+ * max_seqlen writes nothing and sets LA_ERR_DEVICE_CHECK in the device
+ * status word.  Host-side argument errors are those of la_forward.  The
+ * bf16 shapes with a tensor-core forward use it (the elu d = 64 shape takes
+ * the one-launch chunked kernel rather than the split forward); every other
+ * combination runs on the exact fp32 CUDA-core kernel. */
+LA_API la_status la_forward_varlen(const void *q, const void *k, const void *v, void *o,
+                                   const int32_t *cu_seqlens, int nseq, int max_seqlen, int T,
+                                   const float *s_in, const float *z_in,
+                                   float *s_out, float *z_out, float *den_out,
+                                   void *workspace, size_t workspace_bytes,
+                                   int H, int dqk, int dv, int fmap, int dtype, void *stream);
+
 /* la_forward for callers that cannot allocate device memory.
  *
  * The pages have no counterpart to this entry point; it is an interface

@@ -166,3 +166,32 @@ def test_forward_from_state_argument_errors(lib):
     assert call(z_out=z_in + 16) == 1                  # z_out overlaps z_in (16 floats)
     assert call(s_out=s_in + 16 * 16 * 4 - 16) == 1    # tail of s_in overlaps s_out
     assert call(fmap=4) == 1
+
+
+def test_forward_varlen_argument_errors(lib):
+    import causal_kernelized_sequence_b200 as la
+    la.load_library()
+    P = ctypes.c_void_p
+    f = lib.la_forward_varlen
+    q, k, v, o, cu = (0x1000 * (i + 1) for i in range(5))
+
+    def call(cu=cu, nseq=2, max_len=64, T=100, s_in=None, z_in=None, ws=None, wsb=0, H=2, dqk=16, dv=64,
+             fmap=1, dtype=1):
+        return f(P(q), P(k), P(v), P(o), P(cu), nseq, max_len, T, P(s_in), P(z_in), None, None, None,
+                 P(ws), wsb, H, dqk, dv, fmap, dtype, None)
+    assert call(cu=None) == 1                          # lengths required
+    assert call(cu=0x5002) == 1                        # misaligned int32 array
+    assert call(T=0) == 1
+    assert call(max_len=0) == 1
+    assert call(nseq=0) == 1
+    assert call(s_in=0x9000) == 1                      # s_in without z_in
+    assert call(fmap=9) == 1
+    assert call(dqk=32) == 2                           # Taylor beyond d'=16
+    # one long sequence needs segment increments: the workspace is required
+    need = la.la_forward_varlen_workspace_bytes(1, 1, 65536, 16, 64, 1, 1)
+    assert need == la.la_forward_workspace_bytes(1, 1, 65536, 16, 64, 1, 1) > 0
+    assert call(nseq=1, H=1, max_len=65536, T=65536) == 1
+    assert call(nseq=1, H=1, max_len=65536, T=65536, ws=0x10000, wsb=need - 16) == 1
+    # fp32 runs on the CUDA-core kernel: no workspace
+    assert la.la_forward_varlen_workspace_bytes(1, 1, 65536, 16, 64, 1, 0) == 0
+

@@ -105,6 +105,96 @@ def test_chunked_prefill_matches_one_call(fmap, dqk, dv, dtype):
     assert orc.max_rel_l2(z, z_ref) <= tol
 
 
+VARLEN = [(ELU1, 64, 64, W.BF16), (ELU1, 128, 128, W.BF16), (TAYLOR2, 16, 64, W.BF16),
+          (TAYLOR2_SYM, 16, 64, W.BF16), (ELU1, 16, 48, W.BF16), (ELU1, 32, 32, W.F32),
+          (TAYLOR2, 16, 64, W.F32)]
+
+
+def _packed(seed, lens, H, dqk, dv, fmap, dtype):
+    """Packed [H, T, *] inputs for sequences of the given lengths."""
+    T = int(sum(lens))
+    q, k, v, _ = W.random_qkv(seed, 1, H, T, dqk, dv, fmap=fmap, dtype=dtype,
+                              scale=1.0 if fmap != ELU1 else dqk ** -0.5)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32)
+    return q[0].contiguous(), k[0].contiguous(), v[0].contiguous(), cu
+
+
+@pytest.mark.parametrize("fmap,dqk,dv,dtype", VARLEN)
+def test_forward_varlen(fmap, dqk, dv, dtype):
+    """Packed sequences of mixed lengths (empty, one token, chunk edges, a
+    long one that takes several segments) against the oracle's per-sequence
+    recurrence, from zero and from given states."""
+    H = 3
+    for lens, max_len in (([129, 0, 1, 127, 128, 1000, 300], 1000), ([5, 2000], 2048), ([1], 1)):
+        q, k, v, cu = _packed(8000 + len(lens), lens, H, dqk, dv, fmap, dtype)
+        nseq = len(lens)
+        F = la.la_feature_dim(fmap, dqk)
+        tol = TOL[dtype]
+        for start in (False, True):
+            kw = {}
+            s0 = z0 = None
+            if start:
+                s0, z0 = _start_state(fmap, dqk, dv, dtype, 8100 + nseq, nseq, H, skew=fmap != ELU1)
+                kw = {"s_in": s0.to(DEV), "z_in": z0.to(DEV)}
+            r = la.la_forward_varlen(q.to(DEV), k.to(DEV), v.to(DEV), cu.to(DEV), max_len, fmap,
+                                     state=True, den=True, **kw)
+            torch.cuda.synchronize()
+            la.la_get_device_status()
+            o_ref, den_ref, s_ref, z_ref = orc.forward_varlen(fmap, q, k, v, cu.numpy(), s0, z0)
+            o, den, s, z = (r[n].cpu() for n in ("o", "den", "s", "z"))
+            for n_, (a, b) in enumerate(zip(cu[:-1].tolist(), cu[1:].tolist())):
+                if b > a:
+                    err = orc.max_rel_l2(o[:, a:b], o_ref[:, a:b], slice_dims=1)
+                    assert err <= tol, (lens, start, n_, "o", err)
+                    assert orc.max_rel_l2(den[:, a:b], den_ref[:, a:b], slice_dims=1) <= tol
+                if b > a or start:
+                    assert orc.max_rel_l2(s[n_], s_ref[n_], slice_dims=1) <= tol, (lens, start, n_, "s")
+                    assert orc.max_rel_l2(z[n_], z_ref[n_], slice_dims=1) <= tol, (lens, start, n_, "z")
+                else:
+                    assert (s[n_] == 0).all() and (z[n_] == 0).all()
+
+
+def test_forward_varlen_matches_fixed_length():
+    """Equal lengths packed are the fixed-length batch: same bits from the
+    same kernel (Taylor bf16, one launch either way)."""
+    B, H, N = 3, 2, 700
+    q, k, v, _ = W.random_qkv(8200, B, H, N, 16, 64, fmap=TAYLOR2, dtype=W.BF16)
+    fixed = gpu_forward(q, k, v, TAYLOR2, state=True, den=True)
+    pk = lambda t: t.permute(1, 0, 2, 3).reshape(H, B * N, t.shape[-1]).contiguous().to(DEV)
+    cu = torch.arange(0, B * N + 1, N, dtype=torch.int32, device=DEV)
+    r = la.la_forward_varlen(pk(q), pk(k), pk(v), cu, N, TAYLOR2, state=True, den=True)
+    torch.cuda.synchronize()
+    unpk = lambda t: t.cpu().reshape(H, B, N, -1).permute(1, 0, 2, 3)
+    assert torch.equal(unpk(r["o"]), fixed["o"])
+    assert torch.equal(r["s"].cpu().reshape(B, H, *r["s"].shape[2:]), fixed["s"])
+
+
+def test_forward_varlen_bad_lengths_reported():
+    """Lengths live on the device: a decreasing pair or a length above
+    max_seqlen is reported through the status word, and nothing is written
+    for that sequence; the context stays usable."""
+    H, dqk, dv = 2, 16, 64
+    q, k, v, _ = _packed(8300, [100, 100], H, dqk, dv, TAYLOR2, W.BF16)
+    bad = torch.tensor([0, 150, 120], dtype=torch.int32, device=DEV)     # 150 > 120: decreasing
+    o = torch.full((H, 200, dv), 7.0, dtype=torch.bfloat16, device=DEV)
+    la.la_forward_varlen(q.to(DEV), k.to(DEV), v.to(DEV), bad, 150, TAYLOR2, out=o)
+    torch.cuda.synchronize()
+    with pytest.raises(RuntimeError, match="DEVICE_CHECK"):
+        la.la_get_device_status()
+    assert (o[:, 150:].float() == 7.0).all()                               # sequence 1 untouched
+    long = torch.tensor([0, 190, 200], dtype=torch.int32, device=DEV)      # 190 > max_seqlen 100
+    la.la_forward_varlen(q.to(DEV), k.to(DEV), v.to(DEV), long, 100, TAYLOR2, out=o)
+    torch.cuda.synchronize()
+    with pytest.raises(RuntimeError, match="DEVICE_CHECK"):
+        la.la_get_device_status()
+    ok = torch.tensor([0, 100, 200], dtype=torch.int32, device=DEV)
+    r = la.la_forward_varlen(q.to(DEV), k.to(DEV), v.to(DEV), ok, 100, TAYLOR2)
+    torch.cuda.synchronize()
+    la.la_get_device_status()
+    o_ref, _, _, _ = orc.forward_varlen(TAYLOR2, q, k, v, ok.cpu().numpy())
+    assert orc.max_rel_l2(r["o"].cpu(), o_ref, slice_dims=1) <= 1e-2
+
+
 @pytest.mark.parametrize("dtype", [W.F32, W.BF16])
 @pytest.mark.parametrize("fmap,dqk,dv", DIMS)
 def test_backward_small(fmap, dqk, dv, dtype):
