@@ -211,6 +211,40 @@ class Prefill:
                 else f"inputs {self.alg_bytes / 1e6:.0f} MB > 126 MB L2")
 
 
+class VarlenPrefill:
+    """One step = la_forward_varlen over a packed batch of mixed-length
+    sequences (o only)."""
+
+    def __init__(self, w: W.Workload, dev, seed_offset=0):
+        import causal_kernelized_sequence_b200 as la
+        self.la, self.w, self.dev = la, w, dev
+        lens = W.varlen_lengths(w)
+        self.T = T = sum(lens)
+        self.max_len = max(lens)
+        g = torch.Generator(device=dev)
+        g.manual_seed(replica_seed(w, seed_offset))
+        set_bytes = w.H * T * (2 * w.dqk + 2 * w.dv) * 2
+        self.nsets = max(1, math.ceil(2 * L2_BYTES / set_bytes) + 1) if set_bytes < 2 * L2_BYTES else 1
+        mk = lambda d: (torch.randn(w.H, T, d, device=dev, generator=g) * w.scale).to(w.torch_dtype)
+        self.sets = [(mk(w.dqk), mk(w.dqk), mk(w.dv), torch.empty(w.H, T, w.dv, device=dev, dtype=w.torch_dtype))
+                     for _ in range(self.nsets)]
+        self.cu = torch.tensor([0] + torch.tensor(lens).cumsum(0).tolist(), dtype=torch.int32, device=dev)
+        self.tokens = T
+        esz = 2 if w.dtype == W.BF16 else 4
+        self.alg_bytes = w.H * T * (2 * w.dqk + 2 * w.dv) * esz
+        self.alg_flops = 4.0 * w.feature_dim * (w.dv + 1) * w.H * T
+        wsb = la.la_forward_varlen_workspace_bytes(w.B, w.H, self.max_len, w.dqk, w.dv, w.fmap, w.dtype)
+        self.ws = torch.empty(wsb, dtype=torch.uint8, device=dev) if wsb else None
+
+    def step(self, i):
+        q, k, v, o = self.sets[i % self.nsets]
+        self.la.la_forward_varlen(q, k, v, self.cu, self.max_len, self.w.fmap, out=o, workspace=self.ws)
+
+    def l2_note(self):
+        return (f"{self.nsets} rotating input/output sets of "
+                f"{self.alg_bytes / 1e6:.1f} MB (> 126 MB L2 between reuses)")
+
+
 class Train:
     """One step = la_forward (o, den) + la_backward (dq, dk, dv)."""
 
@@ -294,6 +328,8 @@ def make_run(w, dev, seed_offset):
         return Decode(w, dev, seed_offset)
     if w.backward:
         return Train(w, dev, seed_offset)
+    if w.varlen:
+        return VarlenPrefill(w, dev, seed_offset)
     return Prefill(w, dev, seed_offset)
 
 
@@ -550,7 +586,7 @@ def main():
 
     if not args.no_secondary and world == 1:
         sec = {}
-        for name in ("taylor_bf16_fwd", "elu_bf16_train", "taylor_decode", "taylor_decode_sym"):
+        for name in ("taylor_bf16_fwd", "elu_bf16_train", "taylor_decode", "taylor_decode_sym", "elu_bf16_varlen"):
             ws = W.BY_NAME[name]
             r2 = make_run(ws, dev, 0)
             st = 3 if ws.decode_steps else 50

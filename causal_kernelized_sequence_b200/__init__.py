@@ -299,7 +299,7 @@ def kernel_plan(w):
     if w.decode_steps:
         n, names = la_kernel_plan(2, w.B, w.H, 1, w.dqk, w.dv, w.fmap, w.dtype)
         return {"launches_per_step": n * w.decode_steps, "kernels": names}
-    n, names = la_kernel_plan(0, w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype)
+    n, names = la_kernel_plan(3 if getattr(w, "varlen", False) else 0, w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype)
     if w.backward:
         n2, names2 = la_kernel_plan(1, w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype)
         n, names = n + n2, names + names2

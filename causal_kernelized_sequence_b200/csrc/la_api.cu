@@ -762,6 +762,8 @@ int la_kernel_plan(int op, int B, int H, int N, int dqk, int dv, int fmap, int d
 {
     Path p = Path::Invalid;
     if (op == 0) p = select_forward(B, H, N, dqk, dv, fmap, dtype);
+    if (op == 3 && check_shape(B, H, N, dqk, dv, fmap, dtype) == LA_OK)
+        p = tc_forward_shape(dqk, dv, fmap, dtype) ? Path::FwdTc : Path::FwdSimt;
     if (p == Path::FwdTc) {
         int P, cps, nc;
         tc_segments(B, H, N, &P, &cps, &nc);

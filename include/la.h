@@ -273,7 +273,8 @@ LA_API la_status la_feature_map(const void *x, void *phi, int64_t rows, int dqk,
 
 /* Which kernels a call would launch, without launching anything (for
  * launch accounting in benchmarks and tests).  op: 0 = la_forward,
- * 1 = la_backward, 2 = la_decode_step.  Writes a comma-separated list of
+ * 1 = la_backward, 2 = la_decode_step, 3 = la_forward_varlen (B = nseq,
+ * N = max_seqlen).  Writes a comma-separated list of
  * kernel names (truncated to buflen-1 characters, NUL-terminated) to buf
  * when buf is non-NULL, and returns the number of kernel launches the call
  * makes, or -1 for arguments the call itself would reject. */

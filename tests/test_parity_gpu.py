@@ -338,6 +338,27 @@ def test_workload_elu_bf16_train():
     assert ((lhs - rhs).norm() / rhs.norm()).item() < 1e-2
 
 
+def test_workload_elu_bf16_varlen():
+    w = W.BY_NAME["elu_bf16_varlen"]
+    q, k, v, cu = W.make_varlen_inputs(w)
+    lens = W.varlen_lengths(w)
+    r = la.la_forward_varlen(q.to(DEV), k.to(DEV), v.to(DEV), cu.to(DEV), max(lens), w.fmap, den=True, state=True)
+    torch.cuda.synchronize()
+    la.la_get_device_status()
+    o, den, s = r["o"].cpu(), r["den"].cpu(), r["s"].cpu()
+    # sampled sequences (the longest, a short one, the last) and heads, one by one
+    longest = int(np.argmax(lens))
+    for n in (longest, int(np.argmin(lens)), len(lens) - 1):
+        a, b = int(cu[n]), int(cu[n + 1])
+        for h in (0, 5):
+            sl = lambda t: t[h:h + 1, a:b][None]
+            o_ref, den_ref, s_ref, _ = orc.forward_recurrent(w.fmap, sl(q), sl(k), sl(v))
+            assert orc.max_rel_l2(o[h, a:b][None, None], o_ref) <= 1e-2, (n, h)
+            assert orc.max_rel_l2(den[h, a:b][None, None], den_ref) <= 1e-2
+            assert orc.max_rel_l2(s[n, h][None, None], s_ref) <= 1e-2
+    assert (den > 0).all()   # elu+1 features are positive: any size
+
+
 @pytest.mark.parametrize("name", ["taylor_decode", "taylor_decode_sym"])
 def test_workload_taylor_decode(name):
     w = W.BY_NAME[name]

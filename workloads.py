@@ -59,6 +59,7 @@ class Workload:
     scale: float
     backward: bool = False
     decode_steps: int = 0
+    varlen: bool = False   # B sequences of seeded lengths in [1, N], packed [H, T, *]
 
     @property
     def torch_dtype(self):
@@ -80,6 +81,9 @@ class Workload:
         s = f"{self.name}: {fm} {dt} B={self.B} H={self.H} N={self.N} dqk={self.dqk} dv={self.dv}"
         if self.decode_steps:
             s += f" decode_steps={self.decode_steps}"
+        if self.varlen:
+            s = (f"{self.name}: {fm} {dt} {self.B} packed sequences of 1..{self.N} tokens "
+                 f"(T={sum(varlen_lengths(self))}) H={self.H} dqk={self.dqk} dv={self.dv}")
         return s
 
 
@@ -91,6 +95,8 @@ WORKLOADS = [
     Workload("taylor_decode", 4, TAYLOR2, F32, 256, 16, 2048, 16, 64, 1.0, decode_steps=1024),
     # the same decode with the folded Taylor state (153 rows instead of 273)
     Workload("taylor_decode_sym", 4, TAYLOR2_SYM, F32, 256, 16, 2048, 16, 64, 1.0, decode_steps=1024),
+    # a serving-style batch: 16 prompts of mixed lengths, elu d=64, packed
+    Workload("elu_bf16_varlen", 5, ELU1, BF16, 16, 8, 2048, 64, 64, 1.0 / math.sqrt(64), varlen=True),
 ]
 BY_NAME = {w.name: w for w in WORKLOADS}
 
@@ -148,6 +154,29 @@ def make_decode_inputs(w: Workload, *, B=None, H=None, prefill_N=None, steps=Non
         sk[t] = _draw(gen, (B, H, w.dqk), w.scale, dt)
         sv[t] = _draw(gen, (B, H, w.dv), w.scale, dt)
     return (q, k, v), (sq, sk, sv)
+
+
+def varlen_lengths(w: Workload) -> list:
+    """Sequence lengths of a packed workload: B integers drawn uniformly from
+    [1, N] by a generator seeded with the workload's seed + 1000."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(w.index + 1000)
+    return [int(x) for x in torch.randint(1, w.N + 1, (w.B,), generator=gen)]
+
+
+def make_varlen_inputs(w: Workload, dtype=None):
+    """Packed q, k [H, T, dqk], v [H, T, dv] and cu_seqlens [B+1] (int32) on the
+    CPU, drawn in the order q, k, v like make_inputs."""
+    lens = varlen_lengths(w)
+    T = sum(lens)
+    dt = w.torch_dtype if dtype is None else _DT[dtype]
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(w.index)
+    q = _draw(gen, (w.H, T, w.dqk), w.scale, dt)
+    k = _draw(gen, (w.H, T, w.dqk), w.scale, dt)
+    v = _draw(gen, (w.H, T, w.dv), w.scale, dt)
+    cu = torch.tensor([0] + list(torch.tensor(lens).cumsum(0).tolist()), dtype=torch.int32)
+    return q, k, v, cu
 
 
 def random_qkv(seed, B, H, N, dqk, dv, *, fmap=ELU1, dtype=F32, scale=1.0, with_dout=False):
