@@ -31,6 +31,18 @@
  *               y_i = phi(q_i) s_i / phi(q_i) z_i   (state includes token i),
  *               optionally from a given state, returning the final state
  *               (Knowl 5: the prefill may write its final state for decode).
+ *   forward_recurrent_decay / forward_brute_decay / decode_step_decay --
+ *               the gated form: a scalar forget gate a_i = exp(g_i) per
+ *               token multiplies the state before token i is added,
+ *               s_i = a_i s_{i-1} + phi(k_i)^T v_i, z_i = a_i z_{i-1} + phi(k_i)^T
+ *               (the gated update C_t = F_t C_{t-1} + k_t v_t^T of the reader
+ *               comment on linear RNNs, and the scalar-times-identity state
+ *               matrix a_t I of the comment on the state-space duality, on the
+ *               'Transformers are RNNs' discussion page; the input-dependent
+ *               decay of the BASED page, Knowl 10).  The pages give no
+ *               normaliser for it; the same gate decays z, so y_i stays a
+ *               weighted mean of the v_j with weights
+ *               (prod_{l=j+1..i} a_l) phi(q_i).phi(k_j).
  *   decode_step        -- one step of that recurrence on a given state,
  *               output taken from the updated state (Knowl 5, recurrent
  *               generation kernel description).
@@ -209,8 +221,10 @@ void orc_forward_rows(int fmap, int N, int dqk, int dv,
     free(phik);
 }
 
+/* The recurrence over one slice.  g (nullable) holds a log-decay per token:
+ * with it the state is first multiplied by a_i = exp(g_i) (the gated form). */
 static void recurrent_slice(int fmap, int N, int dqk, int dv,
-                            const double *q, const double *k, const double *v,
+                            const double *q, const double *k, const double *v, const double *g,
                             double *s, double *z, double *o, double *den)
 {
     const int F = orc_feature_dim(fmap, dqk);
@@ -220,6 +234,14 @@ static void recurrent_slice(int fmap, int N, int dqk, int dv,
         orc_phi(fmap, dqk, q + (size_t)i * dqk, phiq);
         orc_phi(fmap, dqk, k + (size_t)i * dqk, phik);
         const double *vi = v + (size_t)i * dv;
+        if (g) {
+            /* gated: s_{i-1} <- a_i s_{i-1}, z_{i-1} <- a_i z_{i-1} */
+            const double a = exp(g[i]);
+            for (int f = 0; f < F; ++f) {
+                for (int c = 0; c < dv; ++c) s[(size_t)f * dv + c] *= a;
+                z[f] *= a;
+            }
+        }
         /* s_i = s_{i-1} + phi(k_i)^T v_i ; z_i = z_{i-1} + phi(k_i)^T */
         for (int f = 0; f < F; ++f) {
             for (int c = 0; c < dv; ++c) s[(size_t)f * dv + c] += phik[f] * vi[c];
@@ -240,10 +262,24 @@ static void recurrent_slice(int fmap, int N, int dqk, int dv,
 
 /* Recurrent form over all slices.  s0/z0 (nullable) give a starting state
  * [B,H,F,dv] / [B,H,F]; s_out/z_out (nullable) receive the final state. */
+void orc_forward_recurrent_decay(int fmap, int B, int H, int N, int dqk, int dv,
+                                 const double *q, const double *k, const double *v, const double *g,
+                                 const double *s0, const double *z0,
+                                 double *o, double *den, double *s_out, double *z_out);
+
 void orc_forward_recurrent(int fmap, int B, int H, int N, int dqk, int dv,
                            const double *q, const double *k, const double *v,
                            const double *s0, const double *z0,
                            double *o, double *den, double *s_out, double *z_out)
+{
+    orc_forward_recurrent_decay(fmap, B, H, N, dqk, dv, q, k, v, NULL, s0, z0, o, den, s_out, z_out);
+}
+
+/* The same with a log-decay per token, g [B,H,N] (nullable: no decay). */
+void orc_forward_recurrent_decay(int fmap, int B, int H, int N, int dqk, int dv,
+                                 const double *q, const double *k, const double *v, const double *g,
+                                 const double *s0, const double *z0,
+                                 double *o, double *den, double *s_out, double *z_out)
 {
     const int BH = B * H;
     const int F = orc_feature_dim(fmap, dqk);
@@ -255,6 +291,7 @@ void orc_forward_recurrent(int fmap, int B, int H, int N, int dqk, int dv,
         if (z0) memcpy(z, z0 + (size_t)bh * F, sizeof(double) * (size_t)F);
         recurrent_slice(fmap, N, dqk, dv,
                         q + (size_t)bh * N * dqk, k + (size_t)bh * N * dqk, v + (size_t)bh * N * dv,
+                        g ? g + (size_t)bh * N : NULL,
                         s, z, o + (size_t)bh * N * dv, den ? den + (size_t)bh * N : NULL);
         if (s_out) memcpy(s_out + (size_t)bh * F * dv, s, sizeof(double) * (size_t)F * dv);
         if (z_out) memcpy(z_out + (size_t)bh * F, z, sizeof(double) * (size_t)F);
@@ -265,16 +302,58 @@ void orc_forward_recurrent(int fmap, int B, int H, int N, int dqk, int dv,
 
 /* One decode step for BH independent heads: q,k [BH,dqk], v [BH,dv];
  * s [BH,F,dv], z [BH,F] updated in place; y [BH,dv] from the updated state. */
-void orc_decode_step(int fmap, int BH, int dqk, int dv,
-                     const double *q, const double *k, const double *v,
-                     double *s, double *z, double *y)
+void orc_decode_step_decay(int fmap, int BH, int dqk, int dv,
+                           const double *q, const double *k, const double *v, const double *g,
+                           double *s, double *z, double *y)
 {
     const int F = orc_feature_dim(fmap, dqk);
 #pragma omp parallel for schedule(static)
     for (int bh = 0; bh < BH; ++bh)
         recurrent_slice(fmap, 1, dqk, dv, q + (size_t)bh * dqk, k + (size_t)bh * dqk,
-                        v + (size_t)bh * dv, s + (size_t)bh * F * dv, z + (size_t)bh * F,
+                        v + (size_t)bh * dv, g ? g + bh : NULL, s + (size_t)bh * F * dv, z + (size_t)bh * F,
                         y + (size_t)bh * dv, NULL);
+}
+
+void orc_decode_step(int fmap, int BH, int dqk, int dv,
+                     const double *q, const double *k, const double *v,
+                     double *s, double *z, double *y)
+{
+    orc_decode_step_decay(fmap, BH, dqk, dv, q, k, v, NULL, s, z, y);
+}
+
+/* Gated masked form by brute force, one slice per (b,h):
+ *   w_ij = (prod_{l=j+1..i} exp(g_l)) phi(q_i).phi(k_j)   (j <= i),
+ *   y_i  = sum_j w_ij v_j / sum_j w_ij.
+ * The product is taken factor by factor, walking j down from i. */
+void orc_forward_brute_decay(int fmap, int B, int H, int N, int dqk, int dv,
+                             const double *q, const double *k, const double *v, const double *g,
+                             double *o, double *den)
+{
+    const int BH = B * H;
+    const int F = orc_feature_dim(fmap, dqk);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int bh = 0; bh < BH; ++bh) {
+        const double *qs = q + (size_t)bh * N * dqk, *vs = v + (size_t)bh * N * dv, *gs = g + (size_t)bh * N;
+        double *phik = phi_rows(fmap, N, dqk, k + (size_t)bh * N * dqk);
+        double *phiq = (double *)malloc(sizeof(double) * (size_t)F);
+        double *num = (double *)malloc(sizeof(double) * (size_t)dv);
+        for (int i = 0; i < N; ++i) {
+            orc_phi(fmap, dqk, qs + (size_t)i * dqk, phiq);
+            double d = 0.0, prod = 1.0;
+            for (int c = 0; c < dv; ++c) num[c] = 0.0;
+            for (int j = i; j >= 0; --j) {
+                if (j < i) prod *= exp(gs[j + 1]);
+                const double w = prod * dot(phiq, phik + (size_t)j * F, F);
+                d += w;
+                for (int c = 0; c < dv; ++c) num[c] += w * vs[(size_t)j * dv + c];
+            }
+            for (int c = 0; c < dv; ++c) o[((size_t)bh * N + i) * dv + c] = num[c] / d;
+            if (den) den[(size_t)bh * N + i] = d;
+        }
+        free(phik);
+        free(phiq);
+        free(num);
+    }
 }
 
 /* --------------------------------------------------------------- backward */

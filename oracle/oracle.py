@@ -56,10 +56,14 @@ def _load():
             lib.orc_forward_recurrent.argtypes = [I, I, I, I, I, I, _d, _d, _d, _d, _d, _d, _d, _d, _d]
             lib.orc_decode_step.argtypes = [I, I, I, I, _d, _d, _d, _d, _d, _d]
             lib.orc_backward_brute.argtypes = [I, I, I, I, I, I, _d, _d, _d, _d, _d, _d, _d]
+            lib.orc_forward_recurrent_decay.argtypes = [I, I, I, I, I, I] + [_d] * 10
+            lib.orc_forward_brute_decay.argtypes = [I, I, I, I, I, I] + [_d] * 6
+            lib.orc_decode_step_decay.argtypes = [I, I, I, I] + [_d] * 7
             lib.orc_backward_recurrent.argtypes = [I, I, I, I, I, I, _d, _d, _d, _d, _d, _d, _d]
             for f in (lib.orc_phi, lib.orc_phi_vjp, lib.orc_forward_brute, lib.orc_forward_rows,
                       lib.orc_forward_recurrent, lib.orc_decode_step, lib.orc_backward_brute,
-                      lib.orc_backward_recurrent):
+                      lib.orc_backward_recurrent, lib.orc_forward_recurrent_decay,
+                      lib.orc_forward_brute_decay, lib.orc_decode_step_decay):
                 f.restype = None
             _lib = lib
     return _lib
@@ -187,6 +191,51 @@ def forward_varlen(fmap: int, q, k, v, cu_seqlens, s0=None, z0=None):
                                            None if z0 is None else z0[n:n + 1])
         o[:, a:b], den[:, a:b], s[n], z[n] = on[0], dn[0], sn[0], zn[0]
     return o, den, s, z
+
+
+def forward_recurrent_decay(fmap: int, q, k, v, g, s0=None, z0=None):
+    """Gated recurrent form: a_i = exp(g_i) per token (g [B,H,N]) multiplies
+    the state before token i is added (the gated update of the reader
+    comments on the 'Transformers are RNNs' discussion page; the BASED page's
+    input-dependent decay, Knowl 10).  Returns (o, den, s_final, z_final)."""
+    q, k, v, g = _f64(q), _f64(k), _f64(v), _f64(g)
+    B, H, N, dqk = q.shape
+    dv = v.shape[-1]
+    F = feature_dim(fmap, dqk)
+    assert g.shape == (B, H, N)
+    s0 = None if s0 is None else _f64(s0)
+    z0 = None if z0 is None else _f64(z0)
+    o = np.empty((B, H, N, dv))
+    den = np.empty((B, H, N))
+    s = np.empty((B, H, F, dv))
+    z = np.empty((B, H, F))
+    _load().orc_forward_recurrent_decay(fmap, B, H, N, dqk, dv, _p(q), _p(k), _p(v), _p(g), _p(s0), _p(z0),
+                                        _p(o), _p(den), _p(s), _p(z))
+    return o, den, s, z
+
+
+def forward_brute_decay(fmap: int, q, k, v, g):
+    """Gated masked form by brute force: weights
+    (prod_{l=j+1..i} exp(g_l)) phi(q_i).phi(k_j) for j <= i.  Returns (o, den)."""
+    q, k, v, g = _f64(q), _f64(k), _f64(v), _f64(g)
+    B, H, N, dqk = q.shape
+    dv = v.shape[-1]
+    o = np.empty((B, H, N, dv))
+    den = np.empty((B, H, N))
+    _load().orc_forward_brute_decay(fmap, B, H, N, dqk, dv, _p(q), _p(k), _p(v), _p(g), _p(o), _p(den))
+    return o, den
+
+
+def decode_step_decay(fmap: int, q, k, v, g, s, z):
+    """One gated decode step: s <- exp(g) s + phi(k) v^T, z <- exp(g) z + phi(k),
+    y = phi(q) s / phi(q) z.  g [..heads]; s, z updated in place (float64)."""
+    q, k, v, g = _f64(q), _f64(k), _f64(v), _f64(g)
+    dqk, dv = q.shape[-1], v.shape[-1]
+    BH = int(np.prod(q.shape[:-1]))
+    assert s.dtype == np.float64 and z.dtype == np.float64 and s.flags.c_contiguous and z.flags.c_contiguous
+    y = np.empty(q.shape[:-1] + (dv,))
+    _load().orc_decode_step_decay(fmap, BH, dqk, dv, _p(q), _p(k), _p(v), _p(g), _p(s), _p(z), _p(y))
+    return y
 
 
 def decode_step(fmap: int, q, k, v, s, z):

@@ -337,6 +337,89 @@ def test_varlen_sequences_are_independent(orc, fmap):
     np.testing.assert_allclose(s2[3], sr[0], rtol=1e-12)
 
 
+# ------------------------------------------------------------ gated (decay)
+
+def _gates(seed, *shape, lo=-1.0):
+    # log-decays g <= 0 (forget gates a = exp(g) in (e^lo, 1])
+    return rnd(seed, *shape) ** 2 * (lo / 4.0)
+
+
+@pytest.mark.parametrize("fmap", [ELU1, TAYLOR2, TAYLOR2_SYM])
+def test_decay_zero_gate_is_plain_form(orc, fmap):
+    # g = 0 (a = 1) is the ungated recurrence, already pinned above.
+    d, dv, N = (6, 4, 40) if fmap == ELU1 else (4, 4, 40)
+    q = rnd(110, 2, 2, N, d); k = rnd(111, 2, 2, N, d); v = rnd(112, 2, 2, N, dv)
+    g = np.zeros((2, 2, N))
+    got = orc.forward_recurrent_decay(fmap, q, k, v, g)
+    ref = orc.forward_recurrent(fmap, q, k, v)
+    for x, y in zip(got, ref):
+        np.testing.assert_array_equal(x, y)
+    ob, db = orc.forward_brute_decay(fmap, q, k, v, g)
+    np.testing.assert_allclose(ob, ref[0], rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("fmap,d,dv", [(ELU1, 8, 5), (TAYLOR2, 4, 6), (TAYLOR2_SYM, 16, 8)])
+def test_decay_brute_equals_recurrent(orc, fmap, d, dv):
+    # The product-weight masked form and the gated recurrence are one function.
+    for N in (1, 2, 33, 130):
+        q = rnd(120 + N, 2, 2, N, d, scale=0.7); k = rnd(121 + N, 2, 2, N, d, scale=0.7)
+        v = rnd(122 + N, 2, 2, N, dv); g = _gates(123 + N, 2, 2, N)
+        ob, db = orc.forward_brute_decay(fmap, q, k, v, g)
+        orr, dr, s, z = orc.forward_recurrent_decay(fmap, q, k, v, g)
+        np.testing.assert_allclose(orr, ob, rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(dr, db, rtol=1e-11)
+        # final state: sum_j (prod_{l>j} a_l) phi(k_j) v_j^T
+        pk = orc.phi(fmap, k)
+        tail = np.exp(np.cumsum(g[..., ::-1], -1)[..., ::-1] - g)   # prod_{l=j+1..N-1} a_l
+        np.testing.assert_allclose(s, np.einsum("bhn,bhnf,bhnc->bhfc", tail, pk, v), rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(z, np.einsum("bhn,bhnf->bhf", tail, pk), rtol=1e-10)
+
+
+def test_decay_geometric_weights_closed_form(orc):
+    # Equal keys make phi(q_i).phi(k_j) the same for every j, so with a
+    # constant gate a the output is the geometric mean
+    # y_i = sum_j a^(i-j) v_j / sum_j a^(i-j).
+    N, a = 6, 0.5
+    q = rnd(130, 1, 1, N, 3); k = np.tile(rnd(131, 1, 1, 1, 3), (1, 1, N, 1)); v = rnd(132, 1, 1, N, 2)
+    g = np.full((1, 1, N), math.log(a))
+    o, _, _, _ = orc.forward_recurrent_decay(ELU1, q, k, v, g)
+    for i in range(N):
+        w = np.array([a ** (i - j) for j in range(i + 1)])
+        np.testing.assert_allclose(o[0, 0, i], (w[:, None] * v[0, 0, :i + 1]).sum(0) / w.sum(), rtol=1e-13)
+
+
+def test_decay_full_forgetting_returns_current_value(orc):
+    # a_i = 0 (g = -inf) wipes the state before token i: y_i = v_i exactly and
+    # the state is phi(k_i) v_i^T alone.
+    N = 9
+    q = rnd(140, 1, 2, N, 4); k = rnd(141, 1, 2, N, 4); v = rnd(142, 1, 2, N, 3)
+    g = np.full((1, 2, N), -np.inf)
+    o, den, s, z = orc.forward_recurrent_decay(TAYLOR2, q, k, v, g)
+    np.testing.assert_allclose(o, v, rtol=1e-14)
+    pk = orc.phi(TAYLOR2, k[:, :, -1])
+    np.testing.assert_allclose(s, pk[..., None] * v[:, :, -1, None, :], rtol=1e-14)
+
+
+@pytest.mark.parametrize("fmap", [ELU1, TAYLOR2_SYM])
+def test_decay_decode_and_start_state_continue_the_sequence(orc, fmap):
+    # Prefill(P) then gated decode steps, or a gated forward started from the
+    # prefill's state, continue the gated forward over P + T.
+    P, T, d, dv = 21, 8, 8 if fmap == ELU1 else 16, 5
+    q = rnd(150, 2, 2, P + T, d, scale=0.8); k = rnd(151, 2, 2, P + T, d, scale=0.8)
+    v = rnd(152, 2, 2, P + T, dv); g = _gates(153, 2, 2, P + T)
+    ofull, _, sfull, zfull = orc.forward_recurrent_decay(fmap, q, k, v, g)
+    _, _, s, z = orc.forward_recurrent_decay(fmap, q[:, :, :P], k[:, :, :P], v[:, :, :P], g[:, :, :P])
+    s = np.ascontiguousarray(s); z = np.ascontiguousarray(z)
+    s0, z0 = s.copy(), z.copy()
+    for t in range(T):
+        y = orc.decode_step_decay(fmap, q[:, :, P + t], k[:, :, P + t], v[:, :, P + t], g[:, :, P + t], s, z)
+        np.testing.assert_allclose(y, ofull[:, :, P + t], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(s, sfull, rtol=1e-11, atol=1e-12)
+    ot, _, s2, _ = orc.forward_recurrent_decay(fmap, q[:, :, P:], k[:, :, P:], v[:, :, P:], g[:, :, P:], s0, z0)
+    np.testing.assert_allclose(ot, ofull[:, :, P:], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(s2, sfull, rtol=1e-11, atol=1e-12)
+
+
 # ----------------------------------------------------------------- backward
 
 def _loss_grad_fd(orc, fmap, q, k, v, do, h=1e-6):
