@@ -8,9 +8,12 @@ there is no CPU or PyTorch fallback, and importing the compute functions fails
 loudly when the library has not been built.
 
 Entry points (same names as the C ABI):
-    la_forward(q, k, v, fmap, *, state=False, den=False, out=None, s_in=None, z_in=None) -> dict
+    la_forward(q, k, v, fmap, *, state=False, den=False, out=None, s_in=None, z_in=None,
+               log_decay=None) -> dict   (la_forward / _from_state / _decay)
+    la_forward_varlen(q, k, v, cu_seqlens, max_seqlen, fmap, ...) -> dict
+    la_forward_noalloc(q, k, v, fmap, ...) -> dict
     la_backward(q, k, v, dout, fmap) -> (dq, dk, dv)
-    la_decode_step(q, k, v, s, z, fmap, y=None) -> y        (s, z in place)
+    la_decode_step(q, k, v, s, z, fmap, y=None, log_decay=None) -> y   (s, z in place)
     la_feature_map(x, fmap) -> phi
     la_feature_dim(fmap, dqk) -> int
     la_get_device_status() -> None (raises on a recorded device error)
@@ -77,8 +80,14 @@ def load_library(path: str | None = None):
     lib.la_forward_noalloc.argtypes = [vp] * 7 + [i] * 7 + [vp]
     lib.la_forward_varlen.argtypes = [vp] * 5 + [i] * 3 + [vp] * 6 + [sz] + [i] * 5 + [vp]
     lib.la_forward_varlen.restype = i
+    lib.la_forward_decay.argtypes = [vp] * 11 + [sz] + [i] * 7 + [vp]
+    lib.la_forward_decay.restype = i
+    lib.la_decode_step_decay.argtypes = [vp] * 7 + [i] * 6 + [vp]
+    lib.la_decode_step_decay.restype = i
     lib.la_forward_varlen_workspace_bytes.argtypes = [i] * 7
     lib.la_forward_varlen_workspace_bytes.restype = sz
+    lib.la_forward_decay_workspace_bytes.argtypes = [i] * 7
+    lib.la_forward_decay_workspace_bytes.restype = sz
     lib.la_forward_noalloc.restype = i
     lib.la_kernel_plan.argtypes = [i] * 8 + [ctypes.c_char_p, sz]
     lib.la_kernel_plan.restype = i
@@ -127,11 +136,13 @@ def la_backward_workspace_bytes(B, H, N, dqk, dv, fmap, dtype) -> int:
     return int(load_library().la_backward_workspace_bytes(B, H, N, dqk, dv, fmap, dtype))
 
 
-def la_forward(q, k, v, fmap, *, state=False, den=False, out=None, workspace=None, s_in=None, z_in=None):
+def la_forward(q, k, v, fmap, *, state=False, den=False, out=None, workspace=None, s_in=None, z_in=None,
+               log_decay=None):
     """Causal linear attention forward.  q, k [B,H,N,dqk]; v [B,H,N,dv].
 
     With s_in [B,H,F,dv] and z_in [B,H,F] (fp32) the sequences start from that
-    state (la_forward_from_state) instead of zero.
+    state (la_forward_from_state) instead of zero.  With log_decay [B,H,N]
+    (fp32) the gated form runs (la_forward_decay).
 
     Returns {"o": [B,H,N,dv], and if requested "s": [B,H,F,dv] fp32,
     "z": [B,H,F] fp32, "den": [B,H,N] fp32}.
@@ -159,6 +170,17 @@ def la_forward(q, k, v, fmap, *, state=False, den=False, out=None, workspace=Non
         if s_in.dtype != torch.float32 or z_in.dtype != torch.float32 or not s_in.is_contiguous() \
                 or not z_in.is_contiguous() or tuple(s_in.shape) != (B, H, F, dv) or tuple(z_in.shape) != (B, H, F):
             raise ValueError("s_in must be fp32 [B,H,F,dv] and z_in fp32 [B,H,F], contiguous")
+    if log_decay is not None:
+        _dev(log_decay)
+        if log_decay.dtype != torch.float32 or tuple(log_decay.shape) != (B, H, N):
+            raise ValueError("log_decay must be fp32 [B,H,N]")
+        wsd = int(lib.la_forward_decay_workspace_bytes(B, H, N, dqk, dv, fmap, dt))
+        wsd_t = torch.empty(wsd, dtype=torch.uint8, device=q.device) if wsd else None
+        _check(lib.la_forward_decay(_ptr(q), _ptr(k), _ptr(v), _ptr(log_decay), _ptr(o), _ptr(s_in), _ptr(z_in),
+                                    _ptr(res.get("s")), _ptr(res.get("z")), _ptr(res.get("den")),
+                                    _ptr(wsd_t), wsd, B, H, N, dqk, dv, fmap, dt, _stream()), "la_forward_decay")
+        return res
+    if s_in is not None:
         _check(lib.la_forward_from_state(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(s_in), _ptr(z_in),
                                          _ptr(res.get("s")), _ptr(res.get("z")), _ptr(res.get("den")),
                                          _ptr(workspace), wsb, B, H, N, dqk, dv, fmap, dt, _stream()),
@@ -258,16 +280,24 @@ def la_backward(q, k, v, dout, fmap, *, workspace=None):
     return dq, dk, dvv
 
 
-def la_decode_step(q, k, v, s, z, fmap, y=None):
+def la_decode_step(q, k, v, s, z, fmap, y=None, log_decay=None):
     """One recurrent step: q, k [B,H,dqk]; v [B,H,dv]; s [B,H,F,dv] and
-    z [B,H,F] fp32 updated in place.  Returns y [B,H,dv]."""
+    z [B,H,F] fp32 updated in place.  Returns y [B,H,dv].  With log_decay
+    [B,H] fp32 the state is first multiplied by exp(log_decay)
+    (la_decode_step_decay)."""
     lib = load_library()
-    _dev(q, k, v, s, z, y)
+    _dev(q, k, v, s, z, y, log_decay)
     B, H, dqk = q.shape
     dv = v.shape[-1]
     dt = _dtype_code(q)
     if y is None:
         y = torch.empty(B, H, dv, dtype=q.dtype, device=q.device)
+    if log_decay is not None:
+        if log_decay.dtype != torch.float32 or tuple(log_decay.shape) != (B, H):
+            raise ValueError("log_decay must be fp32 [B,H]")
+        _check(lib.la_decode_step_decay(_ptr(q), _ptr(k), _ptr(v), _ptr(log_decay), _ptr(y), _ptr(s), _ptr(z),
+                                        B, H, dqk, dv, fmap, dt, _stream()), "la_decode_step_decay")
+        return y
     _check(lib.la_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(y), _ptr(s), _ptr(z), B, H, dqk, dv,
                               fmap, dt, _stream()), "la_decode_step")
     return y

@@ -209,7 +209,8 @@ bool pick_chunk(MakeLayout make, int F, int dqk, int dv, Layout *out, size_t *by
 template <typename T>
 la_status forward_simt(const void *q, const void *k, const void *v, void *o, const float *s_in,
                        const float *z_in, float *s_out, float *z_out, float *den_out, int B, int H, int N,
-                       int dqk, int dv, int fmap, cudaStream_t stream, const int *cu = nullptr, int T_total = 0)
+                       int dqk, int dv, int fmap, cudaStream_t stream, const int *cu = nullptr, int T_total = 0,
+                       const float *logdecay = nullptr)
 {
     const FmapParams fp = make_fmap(fmap, dqk);
     SimtFwdSmem L;
@@ -218,7 +219,7 @@ la_status forward_simt(const void *q, const void *k, const void *v, void *o, con
     if (set_smem<fwd_simt_kernel<T>>(bytes) != LA_OK) return LA_ERR_CUDA;
     fwd_simt_kernel<T><<<B * H, kSimtThreads, bytes, stream>>>(
         (const T *)q, (const T *)k, (const T *)v, (T *)o, s_in, z_in, s_out, z_out, den_out, N, dv, fp, L, cu, H,
-        T_total);
+        T_total, logdecay);
     return launch_status();
 }
 
@@ -243,7 +244,7 @@ la_status backward_simt(const void *q, const void *k, const void *v, const void 
 
 template <typename T>
 la_status decode_simt(const void *q, const void *k, const void *v, void *y, float *s, float *z,
-                      int B, int H, int dqk, int dv, int fmap, cudaStream_t stream)
+                      int B, int H, int dqk, int dv, int fmap, cudaStream_t stream, const float *g = nullptr)
 {
     const FmapParams fp = make_fmap(fmap, dqk);
     const int R = kSimtThreads / dv;
@@ -251,13 +252,13 @@ la_status decode_simt(const void *q, const void *k, const void *v, void *y, floa
     const size_t bytes = sizeof(float) * (2 * (size_t)fp.F + 2 * dqk + dv + (size_t)R * dv + 32);
     if (set_smem<decode_simt_kernel<T>>(bytes) != LA_OK) return LA_ERR_CUDA;
     decode_simt_kernel<T><<<B * H, threads, bytes, stream>>>((const T *)q, (const T *)k,
-                                                             (const T *)v, (T *)y, s, z, dv, fp);
+                                                             (const T *)v, (T *)y, s, z, dv, fp, g);
     return launch_status();
 }
 
 template <typename T>
 la_status decode_vec(const void *q, const void *k, const void *v, void *y, float *s, float *z,
-                     int B, int H, int dqk, int dv, int fmap, cudaStream_t stream)
+                     int B, int H, int dqk, int dv, int fmap, cudaStream_t stream, const float *g = nullptr)
 {
     const FmapParams fp = make_fmap(fmap, dqk);
     const T *qq = (const T *)q, *kk = (const T *)k, *vv = (const T *)v;
@@ -267,16 +268,16 @@ la_status decode_vec(const void *q, const void *k, const void *v, void *y, float
     const bool short_state = passes <= 10;
     switch (dv) {
     case 32:
-        if (short_state) decode_vec_kernel<T, 32, 10, 3><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp);
-        else decode_vec_kernel<T, 32, 18, 2><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp);
+        if (short_state) decode_vec_kernel<T, 32, 10, 3><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp, g);
+        else decode_vec_kernel<T, 32, 18, 2><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp, g);
         break;
     case 64:
-        if (short_state) decode_vec_kernel<T, 64, 10, 3><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp);
-        else decode_vec_kernel<T, 64, 18, 2><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp);
+        if (short_state) decode_vec_kernel<T, 64, 10, 3><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp, g);
+        else decode_vec_kernel<T, 64, 18, 2><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp, g);
         break;
     case 128:
-        if (short_state) decode_vec_kernel<T, 128, 10, 3><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp);
-        else decode_vec_kernel<T, 128, 18, 2><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp);
+        if (short_state) decode_vec_kernel<T, 128, 10, 3><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp, g);
+        else decode_vec_kernel<T, 128, 18, 2><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp, g);
         break;
     default: return LA_ERR_UNSUPPORTED;
     }
@@ -717,23 +718,72 @@ la_status la_backward(const void *q, const void *k, const void *v, const void *d
     return backward_simt<__nv_bfloat16>(q, k, v, dout, dq, dk, dvp, ws, B, H, N, dqk, dv, fmap, s);
 }
 
-la_status la_decode_step(const void *q, const void *k, const void *v, void *y, float *s,
-                         float *z, int B, int H, int dqk, int dv, int fmap, int dtype,
-                         void *stream)
+static la_status decode_impl(const void *q, const void *k, const void *v, const float *g, void *y, float *s,
+                             float *z, int B, int H, int dqk, int dv, int fmap, int dtype, void *stream)
 {
     const la_status sh = check_shape(B, H, 1, dqk, dv, fmap, dtype);
     if (sh != LA_OK) return sh;
     if (!q || !k || !v || !y || !s || !z) return LA_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(y, 16) ||
-        !aligned(s, 16) || !aligned(z, 4))
+        !aligned(s, 16) || !aligned(z, 4) || !aligned(g, 4))
         return LA_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
     if (select_decode(B, H, dqk, dv, fmap, dtype) == Path::DecodeVec) {
-        if (dtype == LA_F32) return decode_vec<float>(q, k, v, y, s, z, B, H, dqk, dv, fmap, st);
-        return decode_vec<__nv_bfloat16>(q, k, v, y, s, z, B, H, dqk, dv, fmap, st);
+        if (dtype == LA_F32) return decode_vec<float>(q, k, v, y, s, z, B, H, dqk, dv, fmap, st, g);
+        return decode_vec<__nv_bfloat16>(q, k, v, y, s, z, B, H, dqk, dv, fmap, st, g);
     }
-    if (dtype == LA_F32) return decode_simt<float>(q, k, v, y, s, z, B, H, dqk, dv, fmap, st);
-    return decode_simt<__nv_bfloat16>(q, k, v, y, s, z, B, H, dqk, dv, fmap, st);
+    if (dtype == LA_F32) return decode_simt<float>(q, k, v, y, s, z, B, H, dqk, dv, fmap, st, g);
+    return decode_simt<__nv_bfloat16>(q, k, v, y, s, z, B, H, dqk, dv, fmap, st, g);
+}
+
+la_status la_decode_step(const void *q, const void *k, const void *v, void *y, float *s,
+                         float *z, int B, int H, int dqk, int dv, int fmap, int dtype,
+                         void *stream)
+{
+    return decode_impl(q, k, v, nullptr, y, s, z, B, H, dqk, dv, fmap, dtype, stream);
+}
+
+la_status la_decode_step_decay(const void *q, const void *k, const void *v, const float *log_decay, void *y,
+                               float *s, float *z, int B, int H, int dqk, int dv, int fmap, int dtype,
+                               void *stream)
+{
+    if (!log_decay) return LA_ERR_INVALID_ARG;
+    return decode_impl(q, k, v, log_decay, y, s, z, B, H, dqk, dv, fmap, dtype, stream);
+}
+
+size_t la_forward_decay_workspace_bytes(int B, int H, int N, int dqk, int dv, int fmap, int dtype)
+{
+    (void)B; (void)H; (void)N; (void)dqk; (void)dv; (void)fmap; (void)dtype;
+    return 0;   // the gated forward runs one block per slice, with no segment split
+}
+
+la_status la_forward_decay(const void *q, const void *k, const void *v, const float *log_decay, void *o,
+                           const float *s_in, const float *z_in, float *s_out, float *z_out, float *den_out,
+                           void *workspace, size_t workspace_bytes, int B, int H, int N, int dqk, int dv,
+                           int fmap, int dtype, void *stream)
+{
+    (void)workspace; (void)workspace_bytes;
+    const la_status sh = check_shape(B, H, N, dqk, dv, fmap, dtype);
+    if (sh != LA_OK) return sh;
+    if (!q || !k || !v || !o || !log_decay) return LA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(log_decay, 4) ||
+        !aligned(s_out, 16) || !aligned(z_out, 4) || !aligned(den_out, 4))
+        return LA_ERR_INVALID_ARG;
+    if ((s_in == nullptr) != (z_in == nullptr)) return LA_ERR_INVALID_ARG;
+    if (s_in) {
+        if (!aligned(s_in, 16) || !aligned(z_in, 4)) return LA_ERR_INVALID_ARG;
+        const size_t F = (size_t)la_feature_dim(fmap, dqk);
+        const size_t sb = (size_t)B * H * F * dv * sizeof(float), zb = (size_t)B * H * F * sizeof(float);
+        if (overlaps(s_in, sb, s_out, sb) || overlaps(s_in, sb, z_out, zb) || overlaps(z_in, zb, s_out, sb) ||
+            overlaps(z_in, zb, z_out, zb))
+            return LA_ERR_INVALID_ARG;
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    if (dtype == LA_F32)
+        return forward_simt<float>(q, k, v, o, s_in, z_in, s_out, z_out, den_out, B, H, N, dqk, dv, fmap, st,
+                                   nullptr, 0, log_decay);
+    return forward_simt<__nv_bfloat16>(q, k, v, o, s_in, z_in, s_out, z_out, den_out, B, H, N, dqk, dv, fmap, st,
+                                       nullptr, 0, log_decay);
 }
 
 la_status la_feature_map(const void *x, void *phi, int64_t rows, int dqk, int fmap, int dtype,

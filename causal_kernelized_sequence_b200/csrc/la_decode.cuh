@@ -2,7 +2,9 @@
 //
 // BASED page, Knowl 3 recurrent form and Knowl 5 generation kernel: for each
 // head, S += phi(k) v^T, z += phi(k), y = phi(q) S / phi(q).z on the updated
-// state.  The state (F x DV fp32 plus F fp32) is read once and written once
+// state; with a forget gate a = exp(g) per head, S = a S + phi(k) v^T and
+// z = a z + phi(k) (the gated update of the 'Transformers are RNNs'
+// discussion page).  The state (F x DV fp32 plus F fp32) is read once and written once
 // per call; everything else is noise, so the kernel is organised around HBM:
 //
 //  - one 256-thread block per head; thread (r0, c4) owns the float4 column
@@ -31,7 +33,8 @@ constexpr int kDecodeMaxF = 288;
 template <typename T, int DV, int MAXP, int MINB>
 __global__ void __launch_bounds__(kDecodeThreads, MINB)
 decode_vec_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
-                  T *__restrict__ y, float *__restrict__ S, float *__restrict__ z, FmapParams fp)
+                  T *__restrict__ y, float *__restrict__ S, float *__restrict__ z, FmapParams fp,
+                  const float *__restrict__ logdecay)
 {
     constexpr int CPR = DV / 4;                  // float4 groups per state row
     constexpr int RPP = kDecodeThreads / CPR;    // rows per pass
@@ -60,6 +63,8 @@ decode_vec_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__r
     static_assert(kDecodeMaxF <= 2 * kDecodeThreads, "two z entries per thread");
     const float z0 = tid < F ? __ldcs(zb + tid) : 0.f;
     const float z1 = tid + kDecodeThreads < F ? __ldcs(zb + tid + kDecodeThreads) : 0.f;
+    // gated form: the head's forget gate a = exp(g) scales the state first (1 ungated)
+    const float gate = logdecay ? expf(logdecay[bh]) : 1.f;
     for (int p0 = 0; p0 < passes; p0 += MAXP) {
 #pragma unroll
         for (int b = 0; b < MAXP; ++b) {
@@ -87,10 +92,10 @@ decode_vec_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__r
             if (p0 + b < passes && f < F) {
                 const float a = pk[f], w = pq[f];
                 float4 s = sreg[b];
-                s.x = fmaf(a, vc.x, s.x);
-                s.y = fmaf(a, vc.y, s.y);
-                s.z = fmaf(a, vc.z, s.z);
-                s.w = fmaf(a, vc.w, s.w);
+                s.x = fmaf(a, vc.x, gate * s.x);
+                s.y = fmaf(a, vc.y, gate * s.y);
+                s.z = fmaf(a, vc.z, gate * s.z);
+                s.w = fmaf(a, vc.w, gate * s.w);
                 __stcs(Sb + (size_t)f * CPR + c4, s);
                 acc.x = fmaf(w, s.x, acc.x);
                 acc.y = fmaf(w, s.y, acc.y);
@@ -102,12 +107,12 @@ decode_vec_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__r
     // z update and the denominator phi(q).z (z rows are 4-byte aligned only).
     float dacc = 0.f;
     if (tid < F) {
-        const float zz = z0 + pk[tid];
+        const float zz = fmaf(gate, z0, pk[tid]);
         __stcs(zb + tid, zz);
         dacc = pq[tid] * zz;
     }
     if (tid + kDecodeThreads < F) {
-        const float zz = z1 + pk[tid + kDecodeThreads];
+        const float zz = fmaf(gate, z1, pk[tid + kDecodeThreads]);
         __stcs(zb + tid + kDecodeThreads, zz);
         dacc = fmaf(pq[tid + kDecodeThreads], zz, dacc);
     }

@@ -31,7 +31,7 @@ struct SimtFwdSmem {
     size_t floats(int F, int dqk, int dv) const
     {
         return (size_t)F * DS + F + 2 * (size_t)C * dqk + 2 * (size_t)C * FS + (size_t)C * dv +
-               (size_t)C * C + C;
+               (size_t)C * C + 3 * (size_t)C;
     }
 };
 
@@ -46,7 +46,8 @@ fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
                 T *__restrict__ o, const float *__restrict__ s_in, const float *__restrict__ z_in,
                 float *__restrict__ s_out, float *__restrict__ z_out,
                 float *__restrict__ den_out, int N, int dv, FmapParams fp, SimtFwdSmem L,
-                const int *__restrict__ cu = nullptr, int H = 0, int T_total = 0)
+                const int *__restrict__ cu = nullptr, int H = 0, int T_total = 0,
+                const float *__restrict__ logdecay = nullptr)
 {
     extern __shared__ float sm[];
     const int F = fp.F, dqk = fp.dqk, C = L.C, FS = L.FS, DS = L.DS;
@@ -59,6 +60,8 @@ fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
     float *vs = pk + (size_t)C * FS;    // [C][dv]
     float *A = vs + C * dv;             // [C][C]
     float *den = A + C * C;             // [C]
+    float *cum = den + C;               // [C]  gated form: L_i = sum_{l=t0..t0+i} g_l
+    float *wk = cum + C;                // [C]  exp(L_last - L_j): weight of key j in the state update
 
     const int tid = threadIdx.x, nt = blockDim.x;
     const int lane = tid & 31, warp = tid >> 5, nwarps = nt >> 5;
@@ -96,6 +99,18 @@ fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
             xk[i] = ld(kb + (size_t)t0 * dqk + i);
         }
         for (int i = tid; i < Lc * dv; i += nt) vs[i] = ld(vb + (size_t)t0 * dv + i);
+        if (logdecay && warp == 0) {
+            // inclusive prefix sum of the chunk's log-gates (C <= 32: one warp)
+            float x = lane < Lc ? logdecay[row0 + t0 + lane] : 0.f;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, x, off);
+                if (lane >= off) x += y;
+            }
+            if (lane < Lc) cum[lane] = x;
+            const float last = __shfl_sync(0xffffffffu, x, Lc - 1);
+            if (lane < Lc) wk[lane] = expf(last - x);
+        }
         __syncthreads();
         for (int idx = tid; idx < Lc * F; idx += nt) {
             const int i = idx / F, f = idx - i * F;
@@ -103,19 +118,22 @@ fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
             pk[i * FS + f] = phi_feature(fp, xk + i * dqk, f);
         }
         __syncthreads();
-        // Intra-chunk masked weights A_ij, j <= i.
+        // Intra-chunk masked weights A_ij, j <= i (gated: times exp(L_i - L_j)).
         for (int idx = tid; idx < Lc * Lc; idx += nt) {
             const int i = idx / Lc, j = idx - i * Lc;
             float a = 0.f;
-            if (j <= i)
+            if (j <= i) {
                 for (int f = 0; f < F; ++f) a = fmaf(pq[i * FS + f], pk[j * FS + f], a);
+                if (logdecay) a *= expf(cum[i] - cum[j]);
+            }
             A[i * C + j] = a;
         }
         __syncthreads();
-        // den_i = sum_{j<=i} A_ij + phi(q_i).z   (one warp per row)
+        // den_i = sum_{j<=i} A_ij + e_i phi(q_i).z, e_i = exp(L_i) (1 ungated)  (one warp per row)
         for (int i = warp; i < Lc; i += nwarps) {
             float acc = 0.f;
             for (int f = lane; f < F; f += 32) acc = fmaf(pq[i * FS + f], z[f], acc);
+            if (logdecay) acc *= expf(cum[i]);
             for (int j = lane; j <= i; j += 32) acc += A[i * C + j];
             for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
             if (lane == 0) {
@@ -124,25 +142,33 @@ fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
             }
         }
         __syncthreads();
-        // num_i = sum_{j<=i} A_ij v_j + phi(q_i) S ; y_i = num_i / den_i
+        // num_i = sum_{j<=i} A_ij v_j + e_i phi(q_i) S ; y_i = num_i / den_i
         for (int idx = tid; idx < Lc * dv; idx += nt) {
             const int i = idx / dv, c = idx - i * dv;
             float acc = 0.f;
             for (int f = 0; f < F; ++f) acc = fmaf(pq[i * FS + f], S[f * DS + c], acc);
+            if (logdecay) acc *= expf(cum[i]);
             for (int j = 0; j <= i; ++j) acc = fmaf(A[i * C + j], vs[j * dv + c], acc);
             st(ob + (size_t)(t0 + i) * dv + c, acc / den[i]);
         }
         __syncthreads();
-        // S += phi(K_c)^T V_c ; z += sum_j phi(k_j)
+        // S = e_last S + sum_j w_j phi(k_j) v_j^T ; z likewise (ungated: e = w = 1)
+        const float e_last = logdecay ? expf(cum[Lc - 1]) : 1.f;
         for (int idx = tid; idx < F * dv; idx += nt) {
             const int f = idx / dv, c = idx - f * dv;
-            float acc = S[f * DS + c];
-            for (int j = 0; j < Lc; ++j) acc = fmaf(pk[j * FS + f], vs[j * dv + c], acc);
+            float acc = S[f * DS + c] * e_last;
+            if (logdecay)
+                for (int j = 0; j < Lc; ++j) acc = fmaf(pk[j * FS + f] * wk[j], vs[j * dv + c], acc);
+            else
+                for (int j = 0; j < Lc; ++j) acc = fmaf(pk[j * FS + f], vs[j * dv + c], acc);
             S[f * DS + c] = acc;
         }
         for (int f = tid; f < F; f += nt) {
-            float acc = z[f];
-            for (int j = 0; j < Lc; ++j) acc += pk[j * FS + f];
+            float acc = z[f] * e_last;
+            if (logdecay)
+                for (int j = 0; j < Lc; ++j) acc = fmaf(pk[j * FS + f], wk[j], acc);
+            else
+                for (int j = 0; j < Lc; ++j) acc += pk[j * FS + f];
             z[f] = acc;
         }
     }
@@ -352,7 +378,7 @@ template <typename T>
 __global__ void __launch_bounds__(kSimtThreads)
 decode_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                    T *__restrict__ y, float *__restrict__ S, float *__restrict__ z, int dv,
-                   FmapParams fp)
+                   FmapParams fp, const float *__restrict__ logdecay)
 {
     extern __shared__ float sm[];
     const int F = fp.F, dqk = fp.dqk;
@@ -380,12 +406,13 @@ decode_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__
     __syncthreads();
     float *Sb = S + bh * F * dv;
     float *zb = z + bh * F;
+    const float gate = logdecay ? expf(logdecay[bh]) : 1.f;   // forget gate (1 ungated)
     if (tid < R * dv) {
         const int r = tid / dv, c = tid - r * dv;
         const float vc = vv[c];
         float acc = 0.f;
         for (int f = r; f < F; f += R) {
-            const float s = fmaf(pk[f], vc, Sb[(size_t)f * dv + c]);
+            const float s = fmaf(pk[f], vc, gate * Sb[(size_t)f * dv + c]);
             Sb[(size_t)f * dv + c] = s;
             acc = fmaf(pq[f], s, acc);
         }
@@ -393,7 +420,7 @@ decode_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__
     }
     float dacc = 0.f;
     for (int f = tid; f < F; f += nt) {
-        const float zz = zb[f] + pk[f];
+        const float zz = fmaf(gate, zb[f], pk[f]);
         zb[f] = zz;
         dacc = fmaf(pq[f], zz, dacc);
     }

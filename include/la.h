@@ -199,6 +199,41 @@ LA_API la_status la_forward_varlen(const void *q, const void *k, const void *v, 
                                    void *workspace, size_t workspace_bytes,
                                    int H, int dqk, int dv, int fmap, int dtype, void *stream);
 
+/* Gated (decayed) causal linear attention: a scalar forget gate per token,
+ * a_t = exp(g_t), multiplies the state before the token is added:
+ *
+ *   S_t = a_t S_{t-1} + phi(k_t) v_t^T,   z_t = a_t z_{t-1} + phi(k_t),
+ *   y_t = phi(q_t) S_t / phi(q_t) . z_t
+ *
+ * (the gated update C_t = F_t C_{t-1} + k_t v_t^T and the scalar-times-
+ * identity state matrix a_t I of the reader comments on the 'Transformers
+ * are RNNs' discussion page; the input-dependent decay of the BASED page,
+ * Knowl 10).  The pages give no normaliser for the gated form; the same gate
+ * decays z, so y_t is the mean of v_1..v_t weighted by
+ * (a_{j+1} ... a_t) phi(q_t).phi(k_j).  With g = 0 everywhere this is
+ * la_forward / la_forward_from_state.
+ *   log_decay  [B,H,N] fp32, read: g_t = log a_t.  Gates are forget gates,
+ *              g_t <= 0 (a_t in [0, 1]); -inf forgets everything before t.
+ *              Positive g is computed by the same formulas but can overflow.
+ *   s_in, z_in nullable (both or neither): the state entering each slice.
+ * The other arguments, layouts and errors are those of la_forward_from_state.
+ * Every shape runs on the exact fp32 CUDA-core forward. */
+LA_API size_t la_forward_decay_workspace_bytes(int B, int H, int N, int dqk, int dv, int fmap, int dtype);
+
+LA_API la_status la_forward_decay(const void *q, const void *k, const void *v, const float *log_decay,
+                                  void *o, const float *s_in, const float *z_in,
+                                  float *s_out, float *z_out, float *den_out,
+                                  void *workspace, size_t workspace_bytes,
+                                  int B, int H, int N, int dqk, int dv, int fmap, int dtype,
+                                  void *stream);
+
+/* One gated decode step: S = a S + phi(k) v^T, z = a z + phi(k), then y as in
+ * la_decode_step, with a = exp(log_decay[b,h]) per head (log_decay [B,H]
+ * fp32, read).  Arguments and errors otherwise those of la_decode_step. */
+LA_API la_status la_decode_step_decay(const void *q, const void *k, const void *v, const float *log_decay,
+                                      void *y, float *s, float *z, int B, int H, int dqk, int dv,
+                                      int fmap, int dtype, void *stream);
+
 /* la_forward for callers that cannot allocate device memory.
  *
  * The pages have no counterpart to this entry point; it is an interface

@@ -195,3 +195,25 @@ def test_forward_varlen_argument_errors(lib):
     # fp32 runs on the CUDA-core kernel: no workspace
     assert la.la_forward_varlen_workspace_bytes(1, 1, 65536, 16, 64, 1, 0) == 0
 
+
+def test_decay_argument_errors(lib):
+    P = ctypes.c_void_p
+    f = lib.la_forward_decay
+    f.argtypes = [P] * 11 + [ctypes.c_size_t] + [ctypes.c_int] * 7 + [P]
+    f.restype = ctypes.c_int
+    q, k, v, g, o = (0x1000 * (i + 1) for i in range(5))
+    call = lambda g=g, s_in=None, z_in=None, N=16, fmap=0: \
+        f(P(q), P(k), P(v), P(g), P(o), P(s_in), P(z_in), None, None, None, None, 0, 1, 1, N, 16, 16, fmap, 0, None)
+    assert call(g=None) == 1                           # gates required
+    assert call(g=0x5002) == 1                         # misaligned fp32
+    assert call(s_in=0x9000) == 1                      # s_in without z_in
+    assert call(N=0) == 1
+    assert call(fmap=3) == 1
+    d = lib.la_decode_step_decay
+    d.argtypes = [P] * 7 + [ctypes.c_int] * 6 + [P]
+    d.restype = ctypes.c_int
+    ptr = [P(0x1000 * (i + 1)) for i in range(7)]
+    assert d(ptr[0], ptr[1], ptr[2], P(None), ptr[4], ptr[5], ptr[6], 2, 2, 16, 64, 1, 0, None) == 1
+    assert d(*ptr, 2, 2, 17, 64, 1, 0, None) == 2
+    assert lib.la_forward_decay_workspace_bytes(2, 2, 100, 16, 64, 1, 1) == 0
+

@@ -195,6 +195,74 @@ def test_forward_varlen_bad_lengths_reported():
     assert orc.max_rel_l2(r["o"].cpu(), o_ref, slice_dims=1) <= 1e-2
 
 
+def _log_gates(seed, *shape, lo=-0.5):
+    """Seeded log forget gates g <= 0 (a = exp(g) in [e^lo, 1]), some exactly 0."""
+    g = torch.Generator().manual_seed(seed)
+    x = torch.rand(*shape, generator=g) * lo
+    x[..., ::7] = 0.0
+    return x
+
+
+@pytest.mark.parametrize("dtype", [W.F32, W.BF16])
+@pytest.mark.parametrize("fmap,dqk,dv", [(ELU1, 32, 32), (ELU1, 64, 64), (TAYLOR2, 16, 64), (TAYLOR2_SYM, 16, 64),
+                                         (ELU1, 16, 48)])
+def test_forward_decay(fmap, dqk, dv, dtype):
+    """The gated forward against the oracle's gated recurrence, from zero and
+    from a given state, with ragged lengths; and a strong gate (e^-8 per
+    token) that makes the far past vanish."""
+    for N, lo in ((1, -0.5), (33, -0.5), (257, -0.5), (700, -8.0)):
+        q, k, v, _ = W.random_qkv(9000 + N, 2, 2, N, dqk, dv, fmap=fmap, dtype=dtype,
+                                  scale=1.0 if fmap != ELU1 else dqk ** -0.5)
+        g = _log_gates(9100 + N, 2, 2, N, lo=lo)
+        tol = TOL[dtype]
+        for start in (False, True):
+            kw = {}
+            s0 = z0 = None
+            if start:
+                s0, z0 = _start_state(fmap, dqk, dv, dtype, 9200 + N, 2, 2, skew=fmap != ELU1)
+                kw = {"s_in": s0.to(DEV), "z_in": z0.to(DEV)}
+            r = gpu_forward(q, k, v, fmap, state=True, den=True, log_decay=g.to(DEV), **kw)
+            o_ref, den_ref, s_ref, z_ref = orc.forward_recurrent_decay(fmap, q, k, v, g, s0, z0)
+            for name, ref in (("o", o_ref), ("den", den_ref), ("s", s_ref), ("z", z_ref)):
+                err = orc.max_rel_l2(r[name], ref)
+                assert err <= tol, (N, lo, start, name, err)
+
+
+def test_forward_decay_zero_gate_is_plain_forward():
+    """g = 0 gives the ungated exact forward bit for bit (fp32, same kernel)."""
+    q, k, v, _ = W.random_qkv(9300, 2, 3, 300, 32, 32, dtype=W.F32, scale=32 ** -0.5)
+    a = gpu_forward(q, k, v, ELU1, state=True, den=True)
+    b = gpu_forward(q, k, v, ELU1, state=True, den=True, log_decay=torch.zeros(2, 3, 300, device=DEV))
+    for n in a:
+        assert torch.equal(a[n], b[n]), n
+
+
+@pytest.mark.parametrize("dtype", [W.F32, W.BF16])
+@pytest.mark.parametrize("fmap,dqk,dv", [(TAYLOR2, 16, 64), (TAYLOR2_SYM, 16, 64), (ELU1, 64, 64), (ELU1, 32, 48)])
+def test_decode_decay(fmap, dqk, dv, dtype):
+    """Gated decode steps continue the gated forward (oracle steps from the
+    oracle prefill state)."""
+    P, T = 37, 20
+    q, k, v, _ = W.random_qkv(9400, 3, 2, P + T, dqk, dv, fmap=fmap, dtype=dtype)
+    g = _log_gates(9401, 3, 2, P + T)
+    r = la.la_forward(q[:, :, :P].contiguous().to(DEV), k[:, :, :P].contiguous().to(DEV),
+                      v[:, :, :P].contiguous().to(DEV), fmap, state=True, log_decay=g[:, :, :P].contiguous().to(DEV))
+    s, z = r["s"], r["z"]
+    _, _, s_o, z_o = orc.forward_recurrent_decay(fmap, q[:, :, :P], k[:, :, :P], v[:, :, :P], g[:, :, :P])
+    s_o = np.ascontiguousarray(s_o.reshape(6, *s_o.shape[2:])); z_o = np.ascontiguousarray(z_o.reshape(6, -1))
+    tol = TOL[dtype]
+    for t in range(T):
+        y = la.la_decode_step(q[:, :, P + t].contiguous().to(DEV), k[:, :, P + t].contiguous().to(DEV),
+                              v[:, :, P + t].contiguous().to(DEV), s, z, fmap,
+                              log_decay=g[:, :, P + t].contiguous().to(DEV))
+        torch.cuda.synchronize()
+        y_o = orc.decode_step_decay(fmap, q[:, :, P + t], k[:, :, P + t], v[:, :, P + t], g[:, :, P + t], s_o, z_o)
+        err = orc.max_rel_l2(y.cpu().reshape(6, dv)[None], y_o.reshape(6, dv)[None], slice_dims=1)
+        assert err <= tol, (t, err)
+    la.la_get_device_status()
+    assert orc.max_rel_l2(s.cpu().reshape(6, -1), s_o.reshape(6, -1), slice_dims=1) <= tol
+
+
 @pytest.mark.parametrize("dtype", [W.F32, W.BF16])
 @pytest.mark.parametrize("fmap,dqk,dv", DIMS)
 def test_backward_small(fmap, dqk, dv, dtype):
