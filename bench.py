@@ -193,17 +193,24 @@ class Prefill:
         mk = lambda d: (torch.randn(w.B, w.H, w.N, d, device=dev, generator=g) * w.scale).to(w.torch_dtype)
         self.sets = [(mk(w.dqk), mk(w.dqk), mk(w.dv), torch.empty(w.B, w.H, w.N, w.dv, device=dev, dtype=w.torch_dtype))
                      for _ in range(self.nsets)]
+        # gated form: one log gate per head-token (fp32), one tensor per set
+        self.gates = [W.make_gates(w, device=dev, seed=replica_seed(w, seed_offset) + i) for i in range(self.nsets)] \
+            if w.decay else None
         self.tokens = w.B * w.N
         esz = 2 if w.dtype == W.BF16 else 4
-        self.alg_bytes = w.B * w.H * w.N * (2 * w.dqk + 2 * w.dv) * esz
+        self.alg_bytes = w.B * w.H * w.N * ((2 * w.dqk + 2 * w.dv) * esz + (4 if w.decay else 0))
         F = w.feature_dim
         self.alg_flops = 4.0 * F * (w.dv + 1) * w.B * w.H * w.N
-        wsb = la.la_forward_workspace_bytes(w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype)
+        wsb = (la.load_library().la_forward_decay_workspace_bytes if w.decay else la.la_forward_workspace_bytes)(
+            w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype)
         self.ws = torch.empty(wsb, dtype=torch.uint8, device=dev) if wsb else None
 
     def step(self, i):
         q, k, v, o = self.sets[i % self.nsets]
-        self.la.la_forward(q, k, v, self.w.fmap, out=o, workspace=self.ws)
+        if self.gates is not None:
+            self.la.la_forward(q, k, v, self.w.fmap, out=o, log_decay=self.gates[i % self.nsets], workspace=self.ws)
+        else:
+            self.la.la_forward(q, k, v, self.w.fmap, out=o, workspace=self.ws)
 
     def l2_note(self):
         return (f"{self.nsets} rotating input/output sets of "
@@ -586,7 +593,8 @@ def main():
 
     if not args.no_secondary and world == 1:
         sec = {}
-        for name in ("taylor_bf16_fwd", "elu_bf16_train", "taylor_decode", "taylor_decode_sym", "elu_bf16_varlen"):
+        for name in ("taylor_bf16_fwd", "elu_bf16_train", "taylor_decode", "taylor_decode_sym", "elu_bf16_varlen",
+                     "elu_bf16_decay_fwd"):
             ws = W.BY_NAME[name]
             r2 = make_run(ws, dev, 0)
             st = 3 if ws.decode_steps else 50

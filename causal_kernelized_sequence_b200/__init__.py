@@ -160,7 +160,10 @@ def la_forward(q, k, v, fmap, *, state=False, den=False, out=None, workspace=Non
         res["z"] = torch.empty(B, H, F, dtype=torch.float32, device=q.device)
     if den:
         res["den"] = torch.empty(B, H, N, dtype=torch.float32, device=q.device)
-    wsb = la_forward_workspace_bytes(B, H, N, dqk, dv, fmap, dt)
+    if log_decay is not None:
+        wsb = int(lib.la_forward_decay_workspace_bytes(B, H, N, dqk, dv, fmap, dt))
+    else:
+        wsb = la_forward_workspace_bytes(B, H, N, dqk, dv, fmap, dt)
     if workspace is None and wsb:
         workspace = torch.empty(wsb, dtype=torch.uint8, device=q.device)
     if (s_in is None) != (z_in is None):
@@ -174,11 +177,9 @@ def la_forward(q, k, v, fmap, *, state=False, den=False, out=None, workspace=Non
         _dev(log_decay)
         if log_decay.dtype != torch.float32 or tuple(log_decay.shape) != (B, H, N):
             raise ValueError("log_decay must be fp32 [B,H,N]")
-        wsd = int(lib.la_forward_decay_workspace_bytes(B, H, N, dqk, dv, fmap, dt))
-        wsd_t = torch.empty(wsd, dtype=torch.uint8, device=q.device) if wsd else None
         _check(lib.la_forward_decay(_ptr(q), _ptr(k), _ptr(v), _ptr(log_decay), _ptr(o), _ptr(s_in), _ptr(z_in),
                                     _ptr(res.get("s")), _ptr(res.get("z")), _ptr(res.get("den")),
-                                    _ptr(wsd_t), wsd, B, H, N, dqk, dv, fmap, dt, _stream()), "la_forward_decay")
+                                    _ptr(workspace), wsb, B, H, N, dqk, dv, fmap, dt, _stream()), "la_forward_decay")
         return res
     if s_in is not None:
         _check(lib.la_forward_from_state(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(s_in), _ptr(z_in),
@@ -329,7 +330,8 @@ def kernel_plan(w):
     if w.decode_steps:
         n, names = la_kernel_plan(2, w.B, w.H, 1, w.dqk, w.dv, w.fmap, w.dtype)
         return {"launches_per_step": n * w.decode_steps, "kernels": names}
-    n, names = la_kernel_plan(3 if getattr(w, "varlen", False) else 0, w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype)
+    op = 3 if getattr(w, "varlen", False) else 4 if getattr(w, "decay", False) else 0
+    n, names = la_kernel_plan(op, w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype)
     if w.backward:
         n2, names2 = la_kernel_plan(1, w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype)
         n, names = n + n2, names + names2

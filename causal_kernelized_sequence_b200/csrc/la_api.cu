@@ -316,11 +316,26 @@ bool make_map(CUtensorMap *m, const void *base, int inner, int N, int BH, int bo
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The segment-state launch (P > 1) and the main launch of fwd_tc_kernel.
+template <class Cfg, bool GATED>
+la_status forward_tc_run(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv, const FwdParams &p,
+                         int BH, cudaStream_t stream)
+{
+    if (set_smem<fwd_tc_kernel<Cfg, 0, GATED>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
+    if (p.P > 1) {
+        if (set_smem<fwd_tc_kernel<Cfg, 1, GATED>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
+        fwd_tc_kernel<Cfg, 1, GATED><<<BH * p.P, 256, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+        if (launch_status() != LA_OK) return LA_ERR_CUDA;
+    }
+    fwd_tc_kernel<Cfg, 0, GATED><<<BH * p.P, 256, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+    return launch_status();
+}
+
 template <class Cfg>
 la_status forward_tc_launch(const void *q, const void *k, const void *v, void *o, const float *s_in,
                             const float *z_in, float *s_out, float *z_out, float *den_out, void *workspace, int B,
                             int H, int N, cudaStream_t stream, bool sym_state = false, const int *cu = nullptr,
-                            int T = 0)
+                            int T = 0, const float *logdecay = nullptr)
 {
     // Fixed length: B*H slices of N tokens, tensors [B*H, N, *].  Packed
     // sequences (cu != null): B sequences of at most N tokens, tensors [H, T, *].
@@ -347,20 +362,15 @@ la_status forward_tc_launch(const void *q, const void *k, const void *v, void *o
     p.H = H;
     p.T = T;
     p.max_len = N;
+    p.logdecay = logdecay;
     tc_segments(B, H, N, &p.P, &p.cps, &p.nchunks);
     const double d = (double)Cfg::DQK;
     p.inv_c1 = (float)(1.0 / pow(d, 0.25));
     p.inv_c2 = (float)(1.0 / (sqrt(2.0) * sqrt(d)));
     p.k1 = (float)(1.0 / sqrt(d));
     p.k2 = (float)(1.0 / (2.0 * d));
-    if (set_smem<fwd_tc_kernel<Cfg, 0>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
-    if (p.P > 1) {
-        if (set_smem<fwd_tc_kernel<Cfg, 1>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
-        fwd_tc_kernel<Cfg, 1><<<BH * p.P, 256, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
-        if (launch_status() != LA_OK) return LA_ERR_CUDA;
-    }
-    fwd_tc_kernel<Cfg, 0><<<BH * p.P, 256, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
-    return launch_status();
+    if (logdecay) return forward_tc_run<Cfg, true>(tq, tk, tv, p, BH, stream);
+    return forward_tc_run<Cfg, false>(tq, tk, tv, p, BH, stream);
 }
 
 // Chunk-parallel forward (elu, d_qk = d_v = 64): state launch, then output launch.
@@ -422,16 +432,16 @@ la_status forward_split64(const void *q, const void *k, const void *v, void *o, 
 la_status forward_tc(const void *q, const void *k, const void *v, void *o, const float *s_in, const float *z_in,
                      float *s_out, float *z_out,
                      float *den_out, void *workspace, int B, int H, int N, int dqk, int dv, int fmap,
-                     cudaStream_t stream, const int *cu = nullptr, int T = 0)
+                     cudaStream_t stream, const int *cu = nullptr, int T = 0, const float *logdecay = nullptr)
 {
     if (fmap != LA_FMAP_ELU1)
         return forward_tc_launch<FwdCfg<16, 64, true>>(q, k, v, o, s_in, z_in, s_out, z_out, den_out, workspace, B, H, N,
-                                                       stream, fmap == LA_FMAP_TAYLOR2_SYM, cu, T);
+                                                       stream, fmap == LA_FMAP_TAYLOR2_SYM, cu, T, logdecay);
     if (dqk == 64)
         return forward_tc_launch<FwdCfg<64, 64, false>>(q, k, v, o, s_in, z_in, s_out, z_out, den_out, workspace, B, H,
-                                                        N, stream, false, cu, T);
+                                                        N, stream, false, cu, T, logdecay);
     return forward_tc_launch<FwdCfg<128, 128, false>>(q, k, v, o, s_in, z_in, s_out, z_out, den_out, workspace, B, H,
-                                                      N, stream, false, cu, T);
+                                                      N, stream, false, cu, T, logdecay);
 }
 
 la_status backward_tc(const void *q, const void *k, const void *v, const void *dout, void *dq, void *dk,
@@ -753,8 +763,12 @@ la_status la_decode_step_decay(const void *q, const void *k, const void *v, cons
 
 size_t la_forward_decay_workspace_bytes(int B, int H, int N, int dqk, int dv, int fmap, int dtype)
 {
-    (void)B; (void)H; (void)N; (void)dqk; (void)dv; (void)fmap; (void)dtype;
-    return 0;   // the gated forward runs one block per slice, with no segment split
+    if (check_shape(B, H, N, dqk, dv, fmap, dtype) != LA_OK || !tc_forward_shape(dqk, dv, fmap, dtype)) return 0;
+    int P, cps, nc;
+    tc_segments(B, H, N, &P, &cps, &nc);
+    if (P <= 1) return 0;
+    // segment increments, then each segment's sum of log gates
+    return (size_t)B * H * P * (tc_increment_floats(dqk, dv, fmap) + 1) * sizeof(float);
 }
 
 la_status la_forward_decay(const void *q, const void *k, const void *v, const float *log_decay, void *o,
@@ -762,10 +776,11 @@ la_status la_forward_decay(const void *q, const void *k, const void *v, const fl
                            void *workspace, size_t workspace_bytes, int B, int H, int N, int dqk, int dv,
                            int fmap, int dtype, void *stream)
 {
-    (void)workspace; (void)workspace_bytes;
     const la_status sh = check_shape(B, H, N, dqk, dv, fmap, dtype);
     if (sh != LA_OK) return sh;
     if (!q || !k || !v || !o || !log_decay) return LA_ERR_INVALID_ARG;
+    const size_t need = la_forward_decay_workspace_bytes(B, H, N, dqk, dv, fmap, dtype);
+    if (workspace_bytes < need || (need && (!workspace || !aligned(workspace, 16)))) return LA_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(log_decay, 4) ||
         !aligned(s_out, 16) || !aligned(z_out, 4) || !aligned(den_out, 4))
         return LA_ERR_INVALID_ARG;
@@ -779,6 +794,9 @@ la_status la_forward_decay(const void *q, const void *k, const void *v, const fl
             return LA_ERR_INVALID_ARG;
     }
     cudaStream_t st = (cudaStream_t)stream;
+    if (tc_forward_shape(dqk, dv, fmap, dtype))
+        return forward_tc(q, k, v, o, s_in, z_in, s_out, z_out, den_out, workspace, B, H, N, dqk, dv, fmap, st,
+                          nullptr, 0, log_decay);
     if (dtype == LA_F32)
         return forward_simt<float>(q, k, v, o, s_in, z_in, s_out, z_out, den_out, B, H, N, dqk, dv, fmap, st,
                                    nullptr, 0, log_decay);
@@ -812,7 +830,7 @@ int la_kernel_plan(int op, int B, int H, int N, int dqk, int dv, int fmap, int d
 {
     Path p = Path::Invalid;
     if (op == 0) p = select_forward(B, H, N, dqk, dv, fmap, dtype);
-    if (op == 3 && check_shape(B, H, N, dqk, dv, fmap, dtype) == LA_OK)
+    if ((op == 3 || op == 4) && check_shape(B, H, N, dqk, dv, fmap, dtype) == LA_OK)
         p = tc_forward_shape(dqk, dv, fmap, dtype) ? Path::FwdTc : Path::FwdSimt;
     if (p == Path::FwdTc) {
         int P, cps, nc;

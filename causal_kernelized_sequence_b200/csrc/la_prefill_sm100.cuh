@@ -77,8 +77,10 @@ struct FwdCfg {
     static constexpr int OFF_P = OFF_PK + PHI_TILE;
     static constexpr int OFF_S = OFF_P + P_TILE;
     static constexpr int OFF_BAR = OFF_S + ((S_TILE + 1023) / 1024) * 1024;
-    static constexpr int SMEM = OFF_BAR + 128;
+    static constexpr int OFF_G = OFF_BAR + 128;         // gated form: C prefix sums + 4 warp totals
+    static constexpr int SMEM = OFF_G + (C + 4) * 4;
     static constexpr int SMEM_ALLOC = SMEM + 1024;      // slack for 1024-byte alignment
+    static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory per block");
     static constexpr int TX_BYTES = 2 * C * DQK * 2 + C * DV * 2;
 };
 
@@ -103,6 +105,9 @@ struct FwdParams {
     int H, T, max_len;
     float inv_c1, inv_c2;       // Taylor: 1/d'^(1/4), 1/(sqrt(2) sqrt(d'))
     float k1, k2;               // Taylor closed form: 1/sqrt(d'), 1/(2 d')
+    // Gated form (nullable): log forget gate g_t per token, at the token's row
+    // (row0 + t).  Needs P == 1: segments would have to carry their decay.
+    const float *logdecay;
 };
 
 namespace fwd_detail {
@@ -219,8 +224,9 @@ __device__ __forceinline__ void taylor_sym_to_full(int f, int &r1, int &r2, floa
 }  // namespace fwd_detail
 
 // MODE 0: full forward (o, den, final state).  MODE 1: state increments of
-// each segment only (written to p.ws).
-template <class Cfg, int MODE>
+// each segment only (written to p.ws).  GATED: the gated form (p.logdecay);
+// a template flag, so the ungated kernels carry none of its work.
+template <class Cfg, int MODE, bool GATED>
 __global__ void __launch_bounds__(256, 1)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const FwdParams p)
@@ -308,23 +314,27 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     };
 
     bool have_state = false;
+    constexpr bool gated = GATED;
+    // gated form: per-segment sums of the log gates follow the increments in
+    // the workspace, [slices, P]
+    float *ws_log = p.ws ? p.ws + (size_t)(gridDim.x / p.P) * p.P * FP * NA : nullptr;
+    float lsum_before = 0.f;   // gated: sum of the gates of the earlier segments
+    if (MODE == 0 && gated)
+        for (int s2 = 0; s2 < seg; ++s2) lsum_before += ws_log[(size_t)bh * p.P + s2];
     // ---- starting state of this segment: the state entering the sequence (if
-    // given) plus the sum of the earlier segments' increments
+    // given) plus the sum of the earlier segments' increments; gated, each
+    // earlier term first decays by the gates of the segments after it:
+    // acc <- exp(L_seg) acc + dS_seg, from the entering state through seg - 1
     if (MODE == 0 && (seg > 0 || p.s_in)) {
         for (int t = 0; t < Cfg::NT; ++t) {
             const int m = Cfg::tile_m(t);
             const int r = (m == 128) ? row : ((lane < 16) ? wq * 16 + lane : -1);
             const int f = r < 0 ? -1 : Cfg::tile_f0(t) + r;
             for (int c0 = 16 * half; c0 < NA; c0 += 32) {
-                float acc[16];
+                float acc[16], sin16[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+                for (int e = 0; e < 16; ++e) acc[e] = sin16[e] = 0.f;
                 if (f >= 0 && f < FP) {
-                    for (int s2 = 0; s2 < seg; ++s2) {
-                        const float *src = p.ws + ((size_t)(bh * p.P + s2) * FP + f) * NA + c0;
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) acc[e] += src[e];
-                    }
                     if (p.s_in && f < Cfg::FSYM) {
                         // boundary rows of internal row f (Taylor: the symmetric pair, scaled)
                         const int F = !Cfg::TAYLOR ? DQK : p.sym_state ? Cfg::FSYM : 1 + DQK + DQK * DQK;
@@ -342,8 +352,26 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                                 x = p.z_in[(size_t)bh * F + r1];
                                 if (r2 >= 0) x += p.z_in[(size_t)bh * F + r2];
                             }
-                            acc[e] += sc * x;
+                            sin16[e] = sc * x;
                         }
+                    }
+                    if (gated) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) acc[e] = sin16[e];
+                        for (int s2 = 0; s2 < seg; ++s2) {
+                            const float d = __expf(ws_log[(size_t)bh * p.P + s2]);
+                            const float *src = p.ws + ((size_t)(bh * p.P + s2) * FP + f) * NA + c0;
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) acc[e] = fmaf(acc[e], d, src[e]);
+                        }
+                    } else {
+                        for (int s2 = 0; s2 < seg; ++s2) {
+                            const float *src = p.ws + ((size_t)(bh * p.P + s2) * FP + f) * NA + c0;
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) acc[e] += src[e];
+                        }
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) acc[e] += sin16[e];
                     }
                 }
                 tmem_st16(tmem + lane_base + Cfg::COL_S + t * NA + c0, acc);
@@ -371,6 +399,54 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
     uint32_t mma_phase = 0;
     const float inv_c1 = p.inv_c1, inv_c2 = p.inv_c2, r2_inv_c2 = p.inv_c2 * 1.41421356237309504880f;
+    float seg_log = 0.f;   // gated: sum of this segment's gates so far
+    float *gL = reinterpret_cast<float *>(smem + Cfg::OFF_G);   // [C] prefix sums of the chunk's gates
+    float *gTot = gL + C;                                         // [4] per-warp totals
+
+    // Gated form, elu: multiply this thread's half of row `row` of a phi tile by rs.
+    auto scale_row_half = [&](uint8_t *tile, float rs) {
+#pragma unroll
+        for (int col = half * (DQK / 2); col < (half + 1) * (DQK / 2); col += 8) {
+            const uint32_t a = smem_addr(tile + sw128_off(row, col));
+            float x8[8];
+            unpack8(lds128(a), x8);
+            sts128(a, make_uint4(pack_bf16(rs * x8[0], rs * x8[1]), pack_bf16(rs * x8[2], rs * x8[3]),
+                                 pack_bf16(rs * x8[4], rs * x8[5]), pack_bf16(rs * x8[6], rs * x8[7])));
+        }
+    };
+    // Gated form: S_aug in TMEM <- exp(l) S_aug (this thread's lanes and columns).
+    auto decay_state = [&](float l) {
+        const float dl = __expf(l);
+#pragma unroll 1
+        for (int t = 0; t < Cfg::NT; ++t) {
+#pragma unroll 1
+            for (int c0 = 16 * half; c0 < NA; c0 += 32) {
+                float v[16];
+                tmem_ld16(tmem + lane_base + Cfg::COL_S + t * NA + c0, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) v[e] *= dl;
+                tmem_st16(tmem + lane_base + Cfg::COL_S + t * NA + c0, v);
+            }
+        }
+        tmem_st_wait();
+    };
+
+    // MMA3: S_aug (+)= phi(K_c)^T V_aug, issued by one thread.
+    auto issue_state_mma = [&](uint32_t aK, uint32_t aV, bool acc0) {
+#pragma unroll
+        for (int t = 0; t < Cfg::NT; ++t) {
+            const int m = Cfg::tile_m(t);
+            const uint32_t idesc = idesc_bf16(m, NA, 1, 1);
+            const uint32_t a_base = aK + (Cfg::tile_f0(t) / 64) * (C * 128);
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk) {
+                mma_bf16(tmem + Cfg::COL_S + t * NA,
+                         smem_desc(a_base + kk * 2048, C * 128, 1024, kSw128),
+                         smem_desc(aV + kk * 512, Cfg::V_BLK, 256, kSw32), idesc, acc0 || kk > 0);
+            }
+        }
+    };
 
     for (int chunk = c_begin; chunk < c_end; ++chunk) {
         const int it = chunk - c_begin;
@@ -378,6 +454,33 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const uint32_t tphase = (uint32_t)(it / STAGES) & 1u;
         const int t0 = chunk * C;
         const int nvalid = min(C, N - t0);
+        // ---- gated form: L_i = g_{t0} + ... + g_{t0+i} over the chunk (rows past
+        // the end add 0), e_i = exp(L_i) scales phi(q_i) for the carried state,
+        // w_i = exp(L_last - L_i) scales phi(k_i) for the state update.
+        float gate_e = 1.f, gate_w = 1.f, gate_last = 0.f, gate_L = 0.f;
+        if (gated) {
+            // gates below e^-80 count as e^-80: zero next to any surviving term
+            // in fp32, and it keeps L finite, so differences of L never meet inf - inf
+            float x = row < nvalid ? fmaxf(p.logdecay[row0 + t0 + row], -80.f) : 0.f;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, x, off);
+                if (lane >= off) x += y;
+            }
+            if (half == 0 && lane == 31) gTot[wq] = x;
+            __syncthreads();
+            float before = 0.f;
+#pragma unroll
+            for (int w2 = 0; w2 < 4; ++w2) {
+                if (w2 < wq) before += gTot[w2];
+                gate_last += gTot[w2];
+            }
+            gate_L = x + before;
+            if (half == 0) gL[row] = gate_L;
+            gate_e = __expf(gate_L);
+            gate_w = __expf(gate_last - gate_L);
+            seg_log += gate_last;
+        }
         if (!mbar_wait(&tma_bar[s], tphase)) *abort_flag = 1;
         uint8_t *sQ = smem + Cfg::OFF_Q + s * Cfg::QK_TILE;
         uint8_t *sK = smem + Cfg::OFF_K + s * Cfg::QK_TILE;
@@ -403,12 +506,15 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                                                     elu1_bf16x2(r.w)));
                     }
                 }
+                // segment pass, gated: phi(K) feeds only MMA3 here, scale it now
+                if (MODE == 1 && gated) scale_row_half(sK, gate_w);
             } else {
 #pragma unroll 1
                 for (int m = (MODE == 0 ? 0 : 1); m < 2; ++m) {
                     const uint8_t *raw = m == 0 ? sQ : sK;
                     uint8_t *dst = m == 0 ? sPQ : sPK;
                     const bool zero = (m == 1) && !kvalid;
+                    const float rs = m == 0 ? gate_e : gate_w;   // 1 ungated
                     float x[16];
                     unpack8(*reinterpret_cast<const uint4 *>(raw + sw32_off(i, 0, C)), x);
                     unpack8(*reinterpret_cast<const uint4 *>(raw + sw32_off(i, 8, C)), x + 8);
@@ -420,7 +526,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                             float v8[8];
 #pragma unroll
                             for (int e = 0; e < 8; ++e)
-                                v8[e] = zero ? 0.f : taylor_sym_feature<16>(x, f0 + e, inv_c1, inv_c2, r2_inv_c2);
+                                v8[e] = zero ? 0.f : rs * taylor_sym_feature<16>(x, f0 + e, inv_c1, inv_c2, r2_inv_c2);
                             *reinterpret_cast<uint4 *>(dst + sw128_off(i, f0)) =
                                 make_uint4(pack_bf16(v8[0], v8[1]), pack_bf16(v8[2], v8[3]),
                                            pack_bf16(v8[4], v8[5]), pack_bf16(v8[6], v8[7]));
@@ -431,6 +537,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 }
             }
         }
+        // segment pass, gated: the carried state decays before MMA3 adds to it
+        if (MODE == 1 && gated && have_state) decay_state(gate_last);
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
@@ -454,25 +562,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     }
                 }
             }
-#pragma unroll
-            for (int t = 0; t < Cfg::NT; ++t) {
-                const int m = Cfg::tile_m(t);
-                const uint32_t idesc = idesc_bf16(m, NA, 1, 1);
-                const uint32_t a_base = aK + (Cfg::tile_f0(t) / 64) * (C * 128);
-#pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk) {
-                    mma_bf16(tmem + Cfg::COL_S + t * NA,
-                             smem_desc(a_base + kk * 2048, C * 128, 1024, kSw128),
-                             smem_desc(aV + kk * 512, Cfg::V_BLK, 256, kSw32), idesc,
-                             have_state || kk > 0);
-                }
-            }
+            if (!gated || MODE == 1) issue_state_mma(aK, aV, have_state);
             mma_commit(mma_bar);
         }
         if (!mbar_wait(mma_bar, mma_phase)) *abort_flag = 1;
         mma_phase ^= 1u;
         tc_fence_after();
-        have_state = true;
+        if (!gated || MODE == 1) have_state = true;
 
         if (MODE == 1) {
             __syncthreads();
@@ -495,6 +591,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     const int j = j0 + e;
                     float w = a[e];
                     if (Cfg::TAYLOR) w = 1.f + w * p.k1 + w * w * p.k2;
+                    if (gated) w *= __expf(gate_L - gL[j]);   // a_{j+1} ... a_i
                     a[e] = (j <= i) ? w : 0.f;
                 }
 #pragma unroll
@@ -503,6 +600,16 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         make_uint4(pack_bf16(a[e], a[e + 1]), pack_bf16(a[e + 2], a[e + 3]),
                                    pack_bf16(a[e + 4], a[e + 5]), pack_bf16(a[e + 6], a[e + 7]));
             }
+        }
+        if (gated) {
+            // elu: phi tiles are also MMA1's operands, so they are scaled only
+            // now that MMA1 has completed (Taylor scaled them when computing them)
+            if (!Cfg::TAYLOR) {
+                scale_row_half(sPQ, gate_e);
+                scale_row_half(sPK, gate_w);
+            }
+            // the carried state decays by the chunk's whole gate before MMA3 adds to it
+            if (have_state) decay_state(gate_last);
         }
         fence_proxy_async();
         tc_fence_before();
@@ -528,11 +635,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                              smem_desc(aS + kk * 512, Cfg::S_BLK, 256, kSw32), idesc, true);
                 }
             }
+            if (gated) issue_state_mma(smem_addr(sPK), aV, have_state);
             mma_commit(mma_bar);
         }
         if (!mbar_wait(mma_bar, mma_phase)) *abort_flag = 1;
         mma_phase ^= 1u;
         tc_fence_after();
+        if (gated) have_state = true;
         if (tid == 0 && it + STAGES < c_end - c_begin) issue_tma(chunk + STAGES, s);
 
         // ---- outputs: y = num / den (this thread's half of the value columns)
@@ -590,6 +699,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     // ---- segment increment (MODE 1) or final state (MODE 0, last segment)
     const bool write_ws = (MODE == 1);
     const bool write_final = (MODE == 0) && (seg == nseg - 1) && (p.s_out || p.z_out) && !*abort_flag;
+    if (write_ws && gated && tid == 0 && !*abort_flag) ws_log[(size_t)bh * p.P + seg] = seg_log;
+    // gated: the entering state's antisymmetric part (restored below) has
+    // decayed by every gate of the sequence
+    const float skew_decay = gated ? __expf(lsum_before + seg_log) : 1.f;
     if ((write_ws || write_final) && !*abort_flag) {
 #pragma unroll 1
         for (int t = 0; t < Cfg::NT; ++t) {
@@ -629,7 +742,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     // added back so the returned state is exact
                     float skew = 0.f;
                     if (r2 >= 0 && p.s_in)
-                        skew = 0.5f * (col < DV ? p.s_in[((size_t)bh * F + r1) * DV + col] -
+                        skew = 0.5f * skew_decay * (col < DV ? p.s_in[((size_t)bh * F + r1) * DV + col] -
                                                       p.s_in[((size_t)bh * F + r2) * DV + col]
                                                 : (col == DV ? p.z_in[(size_t)bh * F + r1] - p.z_in[(size_t)bh * F + r2]
                                                              : 0.f));

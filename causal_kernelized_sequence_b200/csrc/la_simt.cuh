@@ -31,7 +31,7 @@ struct SimtFwdSmem {
     size_t floats(int F, int dqk, int dv) const
     {
         return (size_t)F * DS + F + 2 * (size_t)C * dqk + 2 * (size_t)C * FS + (size_t)C * dv +
-               (size_t)C * C + 3 * (size_t)C;
+               (size_t)C * C + 4 * (size_t)C;
     }
 };
 
@@ -60,8 +60,9 @@ fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
     float *vs = pk + (size_t)C * FS;    // [C][dv]
     float *A = vs + C * dv;             // [C][C]
     float *den = A + C * C;             // [C]
-    float *cum = den + C;               // [C]  gated form: L_i = sum_{l=t0..t0+i} g_l
-    float *wk = cum + C;                // [C]  exp(L_last - L_j): weight of key j in the state update
+    float *cum = den + C;               // [C]  gated form: L_i = g_{t0} + ... + g_{t0+i}
+    float *wk = cum + C;                // [C]  exp(g_{t0+j+1} + ... + g_last): key j's weight in the state update
+    float *graw = wk + C;               // [C]  the chunk's gates g_{t0+j}
 
     const int tid = threadIdx.x, nt = blockDim.x;
     const int lane = tid & 31, warp = tid >> 5, nwarps = nt >> 5;
@@ -100,16 +101,28 @@ fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
         }
         for (int i = tid; i < Lc * dv; i += nt) vs[i] = ld(vb + (size_t)t0 * dv + i);
         if (logdecay && warp == 0) {
-            // inclusive prefix sum of the chunk's log-gates (C <= 32: one warp)
-            float x = lane < Lc ? logdecay[row0 + t0 + lane] : 0.f;
+            // the chunk's gates (C <= 32: one warp).  Every decay factor is a
+            // plain sum of gates, never a difference of prefix sums, so a gate
+            // of -inf gives exact zeros and large gates lose no precision.
+            const float gj = lane < Lc ? logdecay[row0 + t0 + lane] : 0.f;
+            float x = gj;   // inclusive prefix
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
                 const float y = __shfl_up_sync(0xffffffffu, x, off);
                 if (lane >= off) x += y;
             }
-            if (lane < Lc) cum[lane] = x;
-            const float last = __shfl_sync(0xffffffffu, x, Lc - 1);
-            if (lane < Lc) wk[lane] = expf(last - x);
+            float r = __shfl_down_sync(0xffffffffu, gj, 1);   // exclusive suffix over lanes j+1 .. Lc-1
+            if (lane + 1 >= Lc) r = 0.f;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float y = __shfl_down_sync(0xffffffffu, r, off);
+                if (lane + off < 32) r += y;
+            }
+            if (lane < Lc) {
+                cum[lane] = x;
+                wk[lane] = expf(r);
+                graw[lane] = gj;
+            }
         }
         __syncthreads();
         for (int idx = tid; idx < Lc * F; idx += nt) {
@@ -124,7 +137,11 @@ fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
             float a = 0.f;
             if (j <= i) {
                 for (int f = 0; f < F; ++f) a = fmaf(pq[i * FS + f], pk[j * FS + f], a);
-                if (logdecay) a *= expf(cum[i] - cum[j]);
+                if (logdecay) {
+                    float gsum = 0.f;   // g_{j+1} + ... + g_i
+                    for (int l = j + 1; l <= i; ++l) gsum += graw[l];
+                    a *= expf(gsum);
+                }
             }
             A[i * C + j] = a;
         }

@@ -217,7 +217,11 @@ LA_API la_status la_forward_varlen(const void *q, const void *k, const void *v, 
  *              Positive g is computed by the same formulas but can overflow.
  *   s_in, z_in nullable (both or neither): the state entering each slice.
  * The other arguments, layouts and errors are those of la_forward_from_state.
- * Every shape runs on the exact fp32 CUDA-core forward. */
+ * The bf16 shapes with a tensor-core forward run on it (long sequences split
+ * into segments whose increments and summed gates go through the workspace,
+ * la_forward_decay_workspace_bytes); there a gate below e^-80 counts as
+ * e^-80, which is zero next to any surviving term in fp32.  Every other combination runs on the
+ * exact fp32 CUDA-core forward, which takes -inf as it is. */
 LA_API size_t la_forward_decay_workspace_bytes(int B, int H, int N, int dqk, int dv, int fmap, int dtype);
 
 LA_API la_status la_forward_decay(const void *q, const void *k, const void *v, const float *log_decay,
@@ -309,7 +313,7 @@ LA_API la_status la_feature_map(const void *x, void *phi, int64_t rows, int dqk,
 /* Which kernels a call would launch, without launching anything (for
  * launch accounting in benchmarks and tests).  op: 0 = la_forward,
  * 1 = la_backward, 2 = la_decode_step, 3 = la_forward_varlen (B = nseq,
- * N = max_seqlen).  Writes a comma-separated list of
+ * N = max_seqlen), 4 = la_forward_decay.  Writes a comma-separated list of
  * kernel names (truncated to buflen-1 characters, NUL-terminated) to buf
  * when buf is non-NULL, and returns the number of kernel launches the call
  * makes, or -1 for arguments the call itself would reject. */

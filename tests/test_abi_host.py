@@ -216,4 +216,12 @@ def test_decay_argument_errors(lib):
     assert d(ptr[0], ptr[1], ptr[2], P(None), ptr[4], ptr[5], ptr[6], 2, 2, 16, 64, 1, 0, None) == 1
     assert d(*ptr, 2, 2, 17, 64, 1, 0, None) == 2
     assert lib.la_forward_decay_workspace_bytes(2, 2, 100, 16, 64, 1, 1) == 0
+    # a long gated sequence splits into segments: increments plus one summed gate each
+    import causal_kernelized_sequence_b200 as la
+    la.load_library()
+    lib.la_forward_decay_workspace_bytes.argtypes = [ctypes.c_int] * 7
+    lib.la_forward_decay_workspace_bytes.restype = ctypes.c_size_t
+    P = 148
+    assert lib.la_forward_decay_workspace_bytes(1, 1, 148 * 128, 16, 64, 1, 1) == P * (160 * 80 + 1) * 4
+    assert lib.la_forward_decay_workspace_bytes(1, 1, 148 * 128, 16, 64, 1, 0) == 0      # fp32: CUDA cores
 

@@ -204,8 +204,8 @@ def _log_gates(seed, *shape, lo=-0.5):
 
 
 @pytest.mark.parametrize("dtype", [W.F32, W.BF16])
-@pytest.mark.parametrize("fmap,dqk,dv", [(ELU1, 32, 32), (ELU1, 64, 64), (TAYLOR2, 16, 64), (TAYLOR2_SYM, 16, 64),
-                                         (ELU1, 16, 48)])
+@pytest.mark.parametrize("fmap,dqk,dv", [(ELU1, 32, 32), (ELU1, 64, 64), (ELU1, 128, 128), (TAYLOR2, 16, 64),
+                                         (TAYLOR2_SYM, 16, 64), (ELU1, 16, 48)])
 def test_forward_decay(fmap, dqk, dv, dtype):
     """The gated forward against the oracle's gated recurrence, from zero and
     from a given state, with ragged lengths; and a strong gate (e^-8 per
@@ -226,6 +226,25 @@ def test_forward_decay(fmap, dqk, dv, dtype):
             for name, ref in (("o", o_ref), ("den", den_ref), ("s", s_ref), ("z", z_ref)):
                 err = orc.max_rel_l2(r[name], ref)
                 assert err <= tol, (N, lo, start, name, err)
+
+
+@pytest.mark.parametrize("dtype,fmap,dqk,dv", [(W.F32, ELU1, 32, 32), (W.BF16, ELU1, 64, 64),
+                                               (W.BF16, TAYLOR2, 16, 64)])
+def test_forward_decay_full_forgetting(dtype, fmap, dqk, dv):
+    """Gates of -inf (a = 0) wipe the state: the token after one starts over.
+    The oracle takes -inf exactly; the tensor-core path counts it as e^-80."""
+    N = 300
+    q, k, v, _ = W.random_qkv(9500, 2, 2, N, dqk, dv, fmap=fmap, dtype=dtype,
+                              scale=1.0 if fmap != ELU1 else dqk ** -0.5)
+    g = _log_gates(9501, 2, 2, N)
+    g[..., [0, 5, 127, 128, 200]] = -float("inf")
+    r = gpu_forward(q, k, v, fmap, state=True, den=True, log_decay=g.to(DEV))
+    o_ref, den_ref, s_ref, _ = orc.forward_recurrent_decay(fmap, q, k, v, g)
+    tol = TOL[dtype]
+    assert orc.max_rel_l2(r["o"], o_ref) <= tol
+    assert orc.max_rel_l2(r["den"], den_ref) <= tol
+    assert orc.max_rel_l2(r["s"], s_ref) <= tol
+    assert torch.isfinite(r["o"].float()).all()
 
 
 def test_forward_decay_zero_gate_is_plain_forward():
@@ -404,6 +423,20 @@ def test_workload_elu_bf16_train():
     lhs = dvv.float().sum(2)
     rhs = dod.float().sum(2)
     assert ((lhs - rhs).norm() / rhs.norm()).item() < 1e-2
+
+
+def test_workload_elu_bf16_decay_fwd():
+    w = W.BY_NAME["elu_bf16_decay_fwd"]
+    q, k, v, _ = W.make_inputs(w)
+    g = W.make_gates(w)
+    r = gpu_forward(q, k, v, w.fmap, den=True, state=True, log_decay=g.to(DEV))
+    for b, h in [(0, 0), (2, 5), (3, 7)]:
+        sl = lambda t: t[b:b + 1, h:h + 1]
+        o_ref, den_ref, s_ref, _ = orc.forward_recurrent_decay(w.fmap, sl(q), sl(k), sl(v), sl(g))
+        assert orc.max_rel_l2(sl(r["o"]), o_ref) <= 1e-2, (b, h)
+        assert orc.max_rel_l2(sl(r["den"]), den_ref) <= 1e-2
+        assert orc.max_rel_l2(sl(r["s"]), s_ref) <= 1e-2
+    assert (r["den"] > 0).all()
 
 
 def test_workload_elu_bf16_varlen():

@@ -60,6 +60,7 @@ class Workload:
     backward: bool = False
     decode_steps: int = 0
     varlen: bool = False   # B sequences of seeded lengths in [1, N], packed [H, T, *]
+    decay: bool = False    # gated form: log forget gates g ~ U(-0.05, 0) per token
 
     @property
     def torch_dtype(self):
@@ -79,6 +80,8 @@ class Workload:
         fm = {ELU1: "elu1", TAYLOR2: "taylor2", TAYLOR2_SYM: "taylor2sym"}[self.fmap]
         dt = "f32" if self.dtype == F32 else "bf16"
         s = f"{self.name}: {fm} {dt} B={self.B} H={self.H} N={self.N} dqk={self.dqk} dv={self.dv}"
+        if self.decay:
+            s += " gated (g ~ U(-0.05, 0))"
         if self.decode_steps:
             s += f" decode_steps={self.decode_steps}"
         if self.varlen:
@@ -97,6 +100,8 @@ WORKLOADS = [
     Workload("taylor_decode_sym", 4, TAYLOR2_SYM, F32, 256, 16, 2048, 16, 64, 1.0, decode_steps=1024),
     # a serving-style batch: 16 prompts of mixed lengths, elu d=64, packed
     Workload("elu_bf16_varlen", 5, ELU1, BF16, 16, 8, 2048, 64, 64, 1.0 / math.sqrt(64), varlen=True),
+    # the headline shape with per-token forget gates
+    Workload("elu_bf16_decay_fwd", 6, ELU1, BF16, 4, 8, 4096, 64, 64, 1.0 / math.sqrt(64), decay=True),
 ]
 BY_NAME = {w.name: w for w in WORKLOADS}
 
@@ -177,6 +182,17 @@ def make_varlen_inputs(w: Workload, dtype=None):
     v = _draw(gen, (w.H, T, w.dv), w.scale, dt)
     cu = torch.tensor([0] + list(torch.tensor(lens).cumsum(0).tolist()), dtype=torch.int32)
     return q, k, v, cu
+
+
+def make_gates(w: Workload, B=None, H=None, N=None, device="cpu", seed=None):
+    """Log forget gates [B, H, N] fp32, uniform on [-0.05, 0), from a generator
+    seeded with the workload's seed + 2000 (decay about 2.5 % per token)."""
+    B = w.B if B is None else B
+    H = w.H if H is None else H
+    N = w.N if N is None else N
+    gen = torch.Generator(device=device)
+    gen.manual_seed((w.index if seed is None else seed) + 2000)
+    return -0.05 * torch.rand(B, H, N, generator=gen, device=device)
 
 
 def random_qkv(seed, B, H, N, dqk, dv, *, fmap=ELU1, dtype=F32, scale=1.0, with_dout=False):
