@@ -43,6 +43,9 @@
  *               normaliser for it; the same gate decays z, so y_i stays a
  *               weighted mean of the v_j with weights
  *               (prod_{l=j+1..i} a_l) phi(q_i).phi(k_j).
+ *   swa_forward        -- causal sliding-window softmax attention (Knowl 4):
+ *               query i attends to keys max(0,i-w+1)..i with softmax weights
+ *               of scale q_i.k_j, and the log-sum-exp of those scores.
  *   decode_step        -- one step of that recurrence on a given state,
  *               output taken from the updated state (Knowl 5, recurrent
  *               generation kernel description).
@@ -486,5 +489,43 @@ void orc_backward_recurrent(int fmap, int B, int H, int N, int dqk, int dv,
             }
         }
         free(s); free(z); free(g); free(dden); free(phiq); free(phik); free(dphi);
+    }
+}
+
+/* ------------------------------------------------ sliding-window attention */
+
+/* Causal sliding-window softmax attention ("Simple linear attention language
+ * models balance the recall-throughput tradeoff", Knowl 4): query i attends
+ * to keys max(0, i-w+1) .. i (0-based),
+ *   o_i = sum_j exp(s_ij - m_i) v_j / sum_j exp(s_ij - m_i),
+ *   s_ij = scale q_i.k_j,  m_i = max_j s_ij,  lse_i = m_i + log sum_j exp(s_ij - m_i).
+ * One slice per (b,h); plain loops. */
+void orc_swa_forward(int B, int H, int N, int dqk, int dv, int w, double scale,
+                     const double *q, const double *k, const double *v, double *o, double *lse)
+{
+    const int BH = B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int bh = 0; bh < BH; ++bh) {
+        const double *qs = q + (size_t)bh * N * dqk, *ks = k + (size_t)bh * N * dqk, *vs = v + (size_t)bh * N * dv;
+        double *os = o + (size_t)bh * N * dv;
+        double *sc = (double *)malloc(sizeof(double) * (size_t)w);
+        for (int i = 0; i < N; ++i) {
+            const int j0 = i - w + 1 > 0 ? i - w + 1 : 0;
+            double m = -INFINITY;
+            for (int j = j0; j <= i; ++j) {
+                sc[j - j0] = scale * dot(qs + (size_t)i * dqk, ks + (size_t)j * dqk, dqk);
+                if (sc[j - j0] > m) m = sc[j - j0];
+            }
+            double den = 0.0;
+            for (int c = 0; c < dv; ++c) os[(size_t)i * dv + c] = 0.0;
+            for (int j = j0; j <= i; ++j) {
+                const double e = exp(sc[j - j0] - m);
+                den += e;
+                for (int c = 0; c < dv; ++c) os[(size_t)i * dv + c] += e * vs[(size_t)j * dv + c];
+            }
+            for (int c = 0; c < dv; ++c) os[(size_t)i * dv + c] /= den;
+            if (lse) lse[(size_t)bh * N + i] = m + log(den);
+        }
+        free(sc);
     }
 }

@@ -59,11 +59,12 @@ def _load():
             lib.orc_forward_recurrent_decay.argtypes = [I, I, I, I, I, I] + [_d] * 10
             lib.orc_forward_brute_decay.argtypes = [I, I, I, I, I, I] + [_d] * 6
             lib.orc_decode_step_decay.argtypes = [I, I, I, I] + [_d] * 7
+            lib.orc_swa_forward.argtypes = [I, I, I, I, I, I, ctypes.c_double] + [_d] * 5
             lib.orc_backward_recurrent.argtypes = [I, I, I, I, I, I, _d, _d, _d, _d, _d, _d, _d]
             for f in (lib.orc_phi, lib.orc_phi_vjp, lib.orc_forward_brute, lib.orc_forward_rows,
                       lib.orc_forward_recurrent, lib.orc_decode_step, lib.orc_backward_brute,
                       lib.orc_backward_recurrent, lib.orc_forward_recurrent_decay,
-                      lib.orc_forward_brute_decay, lib.orc_decode_step_decay):
+                      lib.orc_forward_brute_decay, lib.orc_decode_step_decay, lib.orc_swa_forward):
                 f.restype = None
             _lib = lib
     return _lib
@@ -236,6 +237,28 @@ def decode_step_decay(fmap: int, q, k, v, g, s, z):
     y = np.empty(q.shape[:-1] + (dv,))
     _load().orc_decode_step_decay(fmap, BH, dqk, dv, _p(q), _p(k), _p(v), _p(g), _p(s), _p(z), _p(y))
     return y
+
+
+def swa_forward(q, k, v, window: int, scale=None):
+    """Causal sliding-window softmax attention (BASED page, Knowl 4): query i
+    attends to keys max(0, i-w+1) .. i with softmax weights of scale q_i.k_j,
+    scale = 1/sqrt(dqk) unless given.  Returns (o [B,H,N,dv], lse [B,H,N])."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, N, dqk = q.shape
+    dv = v.shape[-1]
+    scale = 1.0 / np.sqrt(dqk) if scale is None else float(scale)
+    o = np.empty((B, H, N, dv))
+    lse = np.empty((B, H, N))
+    _load().orc_swa_forward(B, H, N, dqk, dv, int(window), scale, _p(q), _p(k), _p(v), _p(o), _p(lse))
+    return o, lse
+
+
+def swa_decode(q, k, v, window: int):
+    """Decode-step outputs for tokens q [B,H,T,dqk] arriving one at a time after
+    nothing: token t attends to the last min(t+1, w) keys, which is the
+    sliding-window forward itself (Knowl 4: a w-token key-value cache during
+    generation holds exactly those keys)."""
+    return swa_forward(q, k, v, window)[0]
 
 
 def decode_step(fmap: int, q, k, v, s, z):

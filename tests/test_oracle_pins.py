@@ -420,6 +420,49 @@ def test_decay_decode_and_start_state_continue_the_sequence(orc, fmap):
     np.testing.assert_allclose(s2, sfull, rtol=1e-11, atol=1e-12)
 
 
+# ------------------------------------------------- sliding-window attention
+
+def test_swa_wide_window_is_causal_softmax_attention(orc):
+    # A window at least as long as the sequence is full causal softmax
+    # attention: torch's scaled_dot_product_attention (a library routine).
+    q = rnd(160, 2, 3, 50, 16); k = rnd(161, 2, 3, 50, 16); v = rnd(162, 2, 3, 50, 8)
+    o, _ = orc.swa_forward(q, k, v, 64)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q), torch.from_numpy(k), torch.from_numpy(v), is_causal=True).numpy()
+    np.testing.assert_allclose(o, ref, rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("w", [1, 16, 64])
+def test_swa_band_mask_softmax(orc, w):
+    # The window is the band max(0, i-w+1) <= j <= i: an explicit boolean mask
+    # with torch's softmax, and the log-sum-exp of the same scores.
+    N, d = 90, 8
+    q = rnd(170 + w, 1, 2, N, d); k = rnd(171 + w, 1, 2, N, d); v = rnd(172 + w, 1, 2, N, 5)
+    o, lse = orc.swa_forward(q, k, v, w)
+    i = np.arange(N)[:, None]; j = np.arange(N)[None, :]
+    band = torch.from_numpy((j <= i) & (j > i - w))
+    sc = torch.from_numpy(q) @ torch.from_numpy(k).transpose(-1, -2) / math.sqrt(d)
+    sc = sc.masked_fill(~band, -float("inf"))
+    np.testing.assert_allclose(o, (torch.softmax(sc, -1) @ torch.from_numpy(v)).numpy(), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse, torch.logsumexp(sc, -1).numpy(), rtol=1e-13)
+    if w == 1:
+        np.testing.assert_array_equal(o, v)      # one key: the query's own value
+
+
+def test_swa_value_shift_and_recency(orc):
+    # The weights of each row sum to one: adding c to every value adds c to
+    # every output.  A key far outside the window changes nothing.
+    N, d, w = 70, 8, 16
+    q = rnd(180, 1, 1, N, d); k = rnd(181, 1, 1, N, d); v = rnd(182, 1, 1, N, 4)
+    o, _ = orc.swa_forward(q, k, v, w)
+    o2, _ = orc.swa_forward(q, k, v + 2.5, w)
+    np.testing.assert_allclose(o2, o + 2.5, rtol=1e-13, atol=1e-13)
+    k2 = k.copy(); v2 = v.copy(); k2[0, 0, 3] *= 7; v2[0, 0, 3] += 100.0
+    o3, _ = orc.swa_forward(q, k2, v2, w)
+    np.testing.assert_array_equal(o3[0, 0, 3 + w:], o[0, 0, 3 + w:])
+    assert np.abs(o3[0, 0, 3:3 + w] - o[0, 0, 3:3 + w]).max() > 1e-3
+
+
 # ----------------------------------------------------------------- backward
 
 def _loss_grad_fd(orc, fmap, q, k, v, do, h=1e-6):
