@@ -14,6 +14,9 @@ Entry points (same names as the C ABI):
     la_forward_noalloc(q, k, v, fmap, ...) -> dict
     la_backward(q, k, v, dout, fmap) -> (dq, dk, dv)
     la_decode_step(q, k, v, s, z, fmap, y=None, log_decay=None) -> y   (s, z in place)
+    la_swa_forward(q, k, v, window, *, out=None, lse=False) -> dict
+    la_swa_cache_fill(k, v, window) -> (k_cache, v_cache)
+    la_swa_decode_step(q, k, v, k_cache, v_cache, pos, window, y=None) -> y
     la_feature_map(x, fmap) -> phi
     la_feature_dim(fmap, dqk) -> int
     la_get_device_status() -> None (raises on a recorded device error)
@@ -89,6 +92,12 @@ def load_library(path: str | None = None):
     lib.la_forward_decay_workspace_bytes.argtypes = [i] * 7
     lib.la_forward_decay_workspace_bytes.restype = sz
     lib.la_forward_noalloc.restype = i
+    lib.la_swa_forward.argtypes = [vp] * 5 + [i] * 7 + [vp]
+    lib.la_swa_forward.restype = i
+    lib.la_swa_cache_fill.argtypes = [vp] * 4 + [i] * 7 + [vp]
+    lib.la_swa_cache_fill.restype = i
+    lib.la_swa_decode_step.argtypes = [vp] * 7 + [i] * 6 + [vp]
+    lib.la_swa_decode_step.restype = i
     lib.la_kernel_plan.argtypes = [i] * 8 + [ctypes.c_char_p, sz]
     lib.la_kernel_plan.restype = i
     lib.la_selftest_bounded_wait.argtypes = [ctypes.c_uint, vp]
@@ -301,6 +310,56 @@ def la_decode_step(q, k, v, s, z, fmap, y=None, log_decay=None):
         return y
     _check(lib.la_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(y), _ptr(s), _ptr(z), B, H, dqk, dv,
                               fmap, dt, _stream()), "la_decode_step")
+    return y
+
+
+def la_swa_forward(q, k, v, window, *, out=None, lse=False):
+    """Causal sliding-window softmax attention (query i attends to keys
+    max(0, i-w+1) .. i).  q, k [B,H,N,dqk]; v [B,H,N,dv].
+    Returns {"o": [B,H,N,dv], and if requested "lse": [B,H,N] fp32}."""
+    lib = load_library()
+    _dev(q, k, v, out)
+    B, H, N, dqk = q.shape
+    dv = v.shape[-1]
+    o = out if out is not None else torch.empty(B, H, N, dv, dtype=q.dtype, device=q.device)
+    res = {"o": o}
+    if lse:
+        res["lse"] = torch.empty(B, H, N, dtype=torch.float32, device=q.device)
+    _check(lib.la_swa_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(res.get("lse")), B, H, N, dqk, dv,
+                              int(window), _dtype_code(q), _stream()), "la_swa_forward")
+    return res
+
+
+def la_swa_cache_fill(k, v, window, *, k_cache=None, v_cache=None):
+    """The w-token cache of a prefill: the last min(N, w) tokens of k, v
+    [B,H,N,*] in slots t mod w.  Returns (k_cache [B,H,w,dqk], v_cache [B,H,w,dv])."""
+    lib = load_library()
+    _dev(k, v, k_cache, v_cache)
+    B, H, N, dqk = k.shape
+    dv = v.shape[-1]
+    if k_cache is None:
+        k_cache = torch.zeros(B, H, window, dqk, dtype=k.dtype, device=k.device)
+    if v_cache is None:
+        v_cache = torch.zeros(B, H, window, dv, dtype=v.dtype, device=v.device)
+    _check(lib.la_swa_cache_fill(_ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), B, H, N, dqk, dv, int(window),
+                                 _dtype_code(k), _stream()), "la_swa_cache_fill")
+    return k_cache, v_cache
+
+
+def la_swa_decode_step(q, k, v, k_cache, v_cache, pos, window, y=None):
+    """One sliding-window decode step: q, k [B,H,dqk], v [B,H,dv]; the caches
+    are updated in place; pos int32 [B] on the device = tokens held before
+    this one (not advanced here).  Returns y [B,H,dv]."""
+    lib = load_library()
+    _dev(q, k, v, k_cache, v_cache, pos, y)
+    B, H, dqk = q.shape
+    dv = v.shape[-1]
+    if pos.dtype != torch.int32 or tuple(pos.shape) != (B,):
+        raise ValueError("pos must be int32 [B]")
+    if y is None:
+        y = torch.empty(B, H, dv, dtype=q.dtype, device=q.device)
+    _check(lib.la_swa_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(y), _ptr(k_cache), _ptr(v_cache), _ptr(pos),
+                                  B, H, dqk, dv, int(window), _dtype_code(q), _stream()), "la_swa_decode_step")
     return y
 
 

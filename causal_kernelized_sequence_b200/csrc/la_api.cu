@@ -20,6 +20,7 @@
 #include "la_prefill_sm100.cuh"
 #include "la_bwd_sm100.cuh"
 #include "la_fwd_split_sm100.cuh"
+#include "la_swa.cuh"
 
 using namespace la;
 
@@ -303,13 +304,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 // 3D bf16 view [BH][N][inner] of a dense row-major tensor, box
 // {box_inner, 128, 1}; rows past N read as zero.
 bool make_map(CUtensorMap *m, const void *base, int inner, int N, int BH, int box_inner,
-              CUtensorMapSwizzle sw)
+              CUtensorMapSwizzle sw, int box_rows = kChunk)
 {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)N, (cuuint64_t)BH};
     cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)N * inner * 2};
-    cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)kChunk, 1};
+    cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -498,6 +499,62 @@ __global__ void selftest_wait_kernel(uint64_t limit_ns)
 }
 
 }  // namespace
+
+// ------------------------------------------------ sliding-window attention
+
+static la_status check_swa(int B, int H, int N, int dqk, int dv, int window, int dtype)
+{
+    if (B < 1 || H < 1 || N < 1 || dqk < 1 || dv < 1 || window < 1) return LA_ERR_INVALID_ARG;
+    if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
+    if ((int64_t)B * H * N * (dqk > dv ? dqk : dv) >= (int64_t)1 << 31) return LA_ERR_INVALID_ARG;
+    if (dqk > 128 || dv > 128 || window > kSwaMaxWindow) return LA_ERR_UNSUPPORTED;
+    return LA_OK;
+}
+
+static bool swa_tc_shape(int dqk, int dv, int window, int dtype)
+{
+    return dtype == LA_BF16 && dqk == 64 && dv == 64 && window % 16 == 0 && window >= 16 && window <= 128;
+}
+
+template <int W>
+static la_status swa_tc_launch(const void *q, const void *k, const void *v, void *o, float *lse, int BH, int N,
+                               cudaStream_t stream)
+{
+    using Cfg = SwaCfg<W>;
+    CUtensorMap tq, tk, tv;
+    if (!make_map(&tq, q, 64, N, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tk, k, 64, N, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B, Cfg::KW) ||
+        !make_map(&tv, v, 64, N, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B, Cfg::KW))
+        return LA_ERR_CUDA;
+    SwaParams p;
+    p.o = (__nv_bfloat16 *)o;
+    p.lse = lse;
+    p.N = N;
+    p.BH = BH;
+    p.tiles_per_bh = (N + Cfg::C - 1) / Cfg::C;
+    p.scale = (float)(1.0 / sqrt(64.0));
+    p.scale_log2 = (float)(1.4426950408889634 / sqrt(64.0));
+    const long long ntiles = (long long)BH * p.tiles_per_bh;
+    const int per_sm = Cfg::TMEM_COLS == 256 ? 2 : 1;   // TMEM: 512 columns per SM
+    const int grid = (int)(ntiles < (long long)per_sm * kNumSms ? ntiles : per_sm * kNumSms);
+    if (set_smem<swa_fwd_tc_kernel<Cfg>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
+    swa_fwd_tc_kernel<Cfg><<<grid, 128, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+    return launch_status();
+}
+
+template <typename T>
+static la_status swa_simt_launch(const void *q, const void *k, const void *v, void *o, float *lse, int BH, int N,
+                                 int dqk, int dv, int window, cudaStream_t stream)
+{
+    const int rblocks = (N + kSwaSimtWarps - 1) / kSwaSimtWarps;
+    const long long blocks = (long long)BH * rblocks;
+    if (blocks >= ((long long)1 << 31)) return LA_ERR_UNSUPPORTED;
+    const size_t bytes = (size_t)kSwaSimtWarps * (window + dqk) * sizeof(float);
+    if (set_smem<swa_fwd_simt_kernel<T>>(bytes) != LA_OK) return LA_ERR_CUDA;
+    swa_fwd_simt_kernel<T><<<(unsigned)blocks, 32 * kSwaSimtWarps, bytes, stream>>>(
+        (const T *)q, (const T *)k, (const T *)v, (T *)o, lse, N, dqk, dv, window, (float)(1.0 / sqrt((double)dqk)));
+    return launch_status();
+}
 
 extern "C" {
 
@@ -802,6 +859,72 @@ la_status la_forward_decay(const void *q, const void *k, const void *v, const fl
                                    nullptr, 0, log_decay);
     return forward_simt<__nv_bfloat16>(q, k, v, o, s_in, z_in, s_out, z_out, den_out, B, H, N, dqk, dv, fmap, st,
                                        nullptr, 0, log_decay);
+}
+
+la_status la_swa_forward(const void *q, const void *k, const void *v, void *o, float *lse_out, int B, int H, int N,
+                         int dqk, int dv, int window, int dtype, void *stream)
+{
+    const la_status sh = check_swa(B, H, N, dqk, dv, window, dtype);
+    if (sh != LA_OK) return sh;
+    if (!q || !k || !v || !o) return LA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse_out, 4))
+        return LA_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    const int BH = B * H;
+    if (swa_tc_shape(dqk, dv, window, dtype)) {
+        switch (window) {
+        case 16: return swa_tc_launch<16>(q, k, v, o, lse_out, BH, N, st);
+        case 32: return swa_tc_launch<32>(q, k, v, o, lse_out, BH, N, st);
+        case 48: return swa_tc_launch<48>(q, k, v, o, lse_out, BH, N, st);
+        case 64: return swa_tc_launch<64>(q, k, v, o, lse_out, BH, N, st);
+        case 80: return swa_tc_launch<80>(q, k, v, o, lse_out, BH, N, st);
+        case 96: return swa_tc_launch<96>(q, k, v, o, lse_out, BH, N, st);
+        case 112: return swa_tc_launch<112>(q, k, v, o, lse_out, BH, N, st);
+        default: return swa_tc_launch<128>(q, k, v, o, lse_out, BH, N, st);
+        }
+    }
+    if (dtype == LA_F32) return swa_simt_launch<float>(q, k, v, o, lse_out, BH, N, dqk, dv, window, st);
+    return swa_simt_launch<__nv_bfloat16>(q, k, v, o, lse_out, BH, N, dqk, dv, window, st);
+}
+
+la_status la_swa_cache_fill(const void *k, const void *v, void *k_cache, void *v_cache, int B, int H, int N,
+                            int dqk, int dv, int window, int dtype, void *stream)
+{
+    const la_status sh = check_swa(B, H, N, dqk, dv, window, dtype);
+    if (sh != LA_OK) return sh;
+    if (!k || !v || !k_cache || !v_cache) return LA_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (dtype == LA_F32)
+        swa_cache_fill_kernel<float><<<B * H, 256, 0, st>>>((const float *)k, (const float *)v, (float *)k_cache,
+                                                            (float *)v_cache, N, dqk, dv, window);
+    else
+        swa_cache_fill_kernel<__nv_bfloat16><<<B * H, 256, 0, st>>>(
+            (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, (__nv_bfloat16 *)k_cache, (__nv_bfloat16 *)v_cache,
+            N, dqk, dv, window);
+    return launch_status();
+}
+
+la_status la_swa_decode_step(const void *q, const void *k, const void *v, void *y, void *k_cache, void *v_cache,
+                             const int32_t *pos, int B, int H, int dqk, int dv, int window, int dtype, void *stream)
+{
+    const la_status sh = check_swa(B, H, 1, dqk, dv, window, dtype);
+    if (sh != LA_OK) return sh;
+    if (!q || !k || !v || !y || !k_cache || !v_cache || !pos || !aligned(pos, 4)) return LA_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t bytes = sizeof(float) * ((size_t)window + dqk + 8);
+    const float scale = (float)(1.0 / sqrt((double)dqk));
+    if (dtype == LA_F32) {
+        if (set_smem<swa_decode_kernel<float>>(bytes) != LA_OK) return LA_ERR_CUDA;
+        swa_decode_kernel<float><<<B * H, kSwaDecodeThreads, bytes, st>>>(
+            (const float *)q, (const float *)k, (const float *)v, (float *)y, (float *)k_cache, (float *)v_cache, pos,
+            H, dqk, dv, window, scale);
+    } else {
+        if (set_smem<swa_decode_kernel<__nv_bfloat16>>(bytes) != LA_OK) return LA_ERR_CUDA;
+        swa_decode_kernel<__nv_bfloat16><<<B * H, kSwaDecodeThreads, bytes, st>>>(
+            (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, (__nv_bfloat16 *)y,
+            (__nv_bfloat16 *)k_cache, (__nv_bfloat16 *)v_cache, pos, H, dqk, dv, window, scale);
+    }
+    return launch_status();
 }
 
 la_status la_feature_map(const void *x, void *phi, int64_t rows, int dqk, int fmap, int dtype,

@@ -238,6 +238,42 @@ LA_API la_status la_decode_step_decay(const void *q, const void *k, const void *
                                       void *y, float *s, float *z, int B, int H, int dqk, int dv,
                                       int fmap, int dtype, void *stream);
 
+/* Causal sliding-window softmax attention, BASED's local exact mixer
+ * (BASED page, Knowl 4): query i attends only to keys max(0, i-w+1) .. i,
+ *
+ *     o_i = sum_j softmax_j(s_ij) v_j,   s_ij = q_i . k_j / sqrt(dqk)
+ *
+ * (the pages give no scale; the standard 1/sqrt(dqk) of scaled dot-product
+ * attention is used).
+ *   q, k [B,H,N,dqk], v, o [B,H,N,dv] dtype; lse_out [B,H,N] fp32 nullable:
+ *   log sum_j exp(s_ij) over the window.
+ *   window  w >= 1 (up to 1024).  bf16 with dqk = dv = 64 and w a multiple of
+ *   16 up to 128 (Knowl 4: widths that are multiples of 16, generally no
+ *   larger than 128) runs on the tensor cores; every other combination on an
+ *   exact fp32 CUDA-core kernel.  Errors as for la_forward. */
+LA_API la_status la_swa_forward(const void *q, const void *k, const void *v, void *o, float *lse_out,
+                                int B, int H, int N, int dqk, int dv, int window, int dtype,
+                                void *stream);
+
+/* The w-token key/value cache of sliding-window generation (Knowl 4):
+ * k_cache [B,H,w,dqk], v_cache [B,H,w,dv] of dtype; token t of a sequence
+ * lives in slot t mod w.  la_swa_cache_fill copies the last min(N, w) tokens
+ * of a prefill's k, v [B,H,N,*] into their slots. */
+LA_API la_status la_swa_cache_fill(const void *k, const void *v, void *k_cache, void *v_cache,
+                                   int B, int H, int N, int dqk, int dv, int window, int dtype,
+                                   void *stream);
+
+/* One sliding-window decode step (Knowl 5, the sliding-window generation
+ * kernel): for each (b,h), store the new k, v [B,H,*] in slot pos[b] mod w
+ * of the cache, then y [B,H,dv] = softmax attention of q over the
+ * min(pos[b] + 1, w) cached tokens.  pos [B] int32, DEVICE memory, read: the
+ * number of tokens sequence b held before this one; the caller advances it.
+ * A negative pos[b] writes nothing for that sequence and sets
+ * LA_ERR_DEVICE_CHECK in the device status word. */
+LA_API la_status la_swa_decode_step(const void *q, const void *k, const void *v, void *y,
+                                    void *k_cache, void *v_cache, const int32_t *pos,
+                                    int B, int H, int dqk, int dv, int window, int dtype, void *stream);
+
 /* la_forward for callers that cannot allocate device memory.
  *
  * The pages have no counterpart to this entry point; it is an interface

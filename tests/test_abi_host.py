@@ -225,3 +225,32 @@ def test_decay_argument_errors(lib):
     assert lib.la_forward_decay_workspace_bytes(1, 1, 148 * 128, 16, 64, 1, 1) == P * (160 * 80 + 1) * 4
     assert lib.la_forward_decay_workspace_bytes(1, 1, 148 * 128, 16, 64, 1, 0) == 0      # fp32: CUDA cores
 
+
+def test_swa_argument_errors(lib):
+    P = ctypes.c_void_p
+    f = lib.la_swa_forward
+    f.argtypes = [P] * 5 + [ctypes.c_int] * 7 + [P]
+    f.restype = ctypes.c_int
+    q, k, v, o = (0x1000 * (i + 1) for i in range(4))
+    call = lambda q=q, N=16, dqk=64, dv=64, w=64, dt=1, lse=None: f(P(q), P(k), P(v), P(o), P(lse), 1, 1, N, dqk, dv,
+                                                                    w, dt, None)
+    assert call(q=None) == 1
+    assert call(w=0) == 1
+    assert call(N=0) == 1
+    assert call(dt=5) == 1
+    assert call(q=0x1008) == 1                         # misaligned
+    assert call(lse=0x9002) == 1
+    assert call(w=2048) == 2                           # beyond the exact kernel's window
+    assert call(dqk=256) == 2
+    d = lib.la_swa_decode_step
+    d.argtypes = [P] * 7 + [ctypes.c_int] * 6 + [P]
+    d.restype = ctypes.c_int
+    ptr = [P(0x1000 * (i + 1)) for i in range(7)]
+    assert d(*ptr[:6], P(None), 1, 1, 64, 64, 64, 1, None) == 1       # positions required
+    assert d(*ptr[:6], P(0x7002), 1, 1, 64, 64, 64, 1, None) == 1     # misaligned int32
+    assert d(*ptr, 1, 1, 64, 64, 0, 1, None) == 1
+    c = lib.la_swa_cache_fill
+    c.argtypes = [P] * 4 + [ctypes.c_int] * 7 + [P]
+    c.restype = ctypes.c_int
+    assert c(P(None), *ptr[1:4], 1, 1, 16, 64, 64, 64, 1, None) == 1
+

@@ -282,6 +282,76 @@ def test_decode_decay(fmap, dqk, dv, dtype):
     assert orc.max_rel_l2(s.cpu().reshape(6, -1), s_o.reshape(6, -1), slice_dims=1) <= tol
 
 
+SWA = [(W.BF16, 64, 64, 64), (W.BF16, 64, 64, 16), (W.BF16, 64, 64, 128), (W.BF16, 64, 64, 48),
+       (W.BF16, 64, 64, 50), (W.F32, 32, 48, 64), (W.F32, 64, 64, 1), (W.BF16, 16, 32, 300)]
+
+
+@pytest.mark.parametrize("dtype,dqk,dv,w", SWA)
+def test_swa_forward(dtype, dqk, dv, w):
+    """Sliding-window attention against the oracle: tensor-core tiles (bf16,
+    d = 64, w a multiple of 16) with ragged tails and windows reaching before
+    the sequence start, and the exact kernel for the other shapes."""
+    for N in (1, 15, 127, 128, 129, 300, 1000):
+        q, k, v, _ = W.random_qkv(9600 + N + w, 2, 3, N, dqk, dv, dtype=dtype)
+        r = la.la_swa_forward(q.to(DEV), k.to(DEV), v.to(DEV), w, lse=True)
+        torch.cuda.synchronize()
+        la.la_get_device_status()
+        o_ref, lse_ref = orc.swa_forward(q, k, v, w)
+        tol = TOL[dtype]
+        err = orc.max_rel_l2(r["o"].cpu(), o_ref)
+        assert err <= tol, (N, err)
+        assert orc.max_rel_l2(r["lse"].cpu(), lse_ref) <= tol, N
+
+
+@pytest.mark.parametrize("dtype,dqk,dv,w", [(W.BF16, 64, 64, 64), (W.F32, 32, 48, 16)])
+def test_swa_decode(dtype, dqk, dv, w):
+    """Prefill, cache fill, then decode steps: each step equals the oracle's
+    sliding-window forward at that position; prompts shorter and longer than
+    the window, and sequences at different positions."""
+    B, H, T = 2, 3, 40
+    for P in (5, w + 37):
+        q, k, v, _ = W.random_qkv(9700 + P, B, H, P + T, dqk, dv, dtype=dtype)
+        o_ref, _ = orc.swa_forward(q, k, v, w)
+        kc, vc = la.la_swa_cache_fill(k[:, :, :P].contiguous().to(DEV), v[:, :, :P].contiguous().to(DEV), w)
+        pos = torch.full((B,), P, dtype=torch.int32, device=DEV)
+        tol = TOL[dtype]
+        for t in range(T):
+            y = la.la_swa_decode_step(q[:, :, P + t].contiguous().to(DEV), k[:, :, P + t].contiguous().to(DEV),
+                                      v[:, :, P + t].contiguous().to(DEV), kc, vc, pos, w)
+            pos += 1
+            torch.cuda.synchronize()
+            err = orc.max_rel_l2(y.cpu(), o_ref[:, :, P + t])
+            assert err <= tol, (P, t, err)
+        la.la_get_device_status()
+    # sequences at different positions in one call: sequence 1 is one token behind
+    q, k, v, _ = W.random_qkv(9800, B, H, 30, dqk, dv, dtype=dtype)
+    o_ref, _ = orc.swa_forward(q, k, v, w)
+    kc, vc = la.la_swa_cache_fill(k[:, :, :20].contiguous().to(DEV), v[:, :, :20].contiguous().to(DEV), w)
+    kc1, vc1 = la.la_swa_cache_fill(k[1:, :, :19].contiguous().to(DEV), v[1:, :, :19].contiguous().to(DEV), w)
+    kc[1:], vc[1:] = kc1, vc1
+    pos = torch.tensor([20, 19], dtype=torch.int32, device=DEV)
+    qt = torch.stack([q[0, :, 20], q[1, :, 19]]).contiguous().to(DEV)
+    kt = torch.stack([k[0, :, 20], k[1, :, 19]]).contiguous().to(DEV)
+    vt = torch.stack([v[0, :, 20], v[1, :, 19]]).contiguous().to(DEV)
+    y = la.la_swa_decode_step(qt, kt, vt, kc, vc, pos, w).cpu()
+    ref = torch.stack([torch.from_numpy(o_ref[0, :, 20]), torch.from_numpy(o_ref[1, :, 19])])
+    assert orc.max_rel_l2(y, ref) <= TOL[dtype]
+
+
+def test_swa_decode_bad_position_reported():
+    """A negative position writes nothing and is reported; the context stays usable."""
+    q, k, v, _ = W.random_qkv(9900, 1, 2, 1, 64, 64, dtype=W.BF16)
+    kc = torch.full((1, 2, 64, 64), 3.0, dtype=torch.bfloat16, device=DEV)
+    vc = kc.clone()
+    pos = torch.tensor([-1], dtype=torch.int32, device=DEV)
+    la.la_swa_decode_step(q[:, :, 0].contiguous().to(DEV), k[:, :, 0].contiguous().to(DEV),
+                          v[:, :, 0].contiguous().to(DEV), kc, vc, pos, 64)
+    torch.cuda.synchronize()
+    with pytest.raises(RuntimeError, match="DEVICE_CHECK"):
+        la.la_get_device_status()
+    assert (kc.float() == 3.0).all()
+
+
 @pytest.mark.parametrize("dtype", [W.F32, W.BF16])
 @pytest.mark.parametrize("fmap,dqk,dv", DIMS)
 def test_backward_small(fmap, dqk, dv, dtype):
