@@ -330,7 +330,72 @@ class Decode:
         return f"state {self.s.numel() * 4 / 1e6:.0f} MB > 126 MB L2"
 
 
+class SwaPrefill:
+    """One step = la_swa_forward over the whole batch (o only)."""
+
+    def __init__(self, w: W.Workload, dev, seed_offset=0):
+        import causal_kernelized_sequence_b200 as la
+        self.la, self.w, self.dev = la, w, dev
+        g = torch.Generator(device=dev)
+        g.manual_seed(replica_seed(w, seed_offset))
+        set_bytes = w.B * w.H * w.N * (2 * w.dqk + 2 * w.dv) * 2
+        self.nsets = max(1, math.ceil(2 * L2_BYTES / set_bytes) + 1) if set_bytes < 2 * L2_BYTES else 1
+        mk = lambda d: (torch.randn(w.B, w.H, w.N, d, device=dev, generator=g) * w.scale).to(w.torch_dtype)
+        self.sets = [(mk(w.dqk), mk(w.dqk), mk(w.dv), torch.empty(w.B, w.H, w.N, w.dv, device=dev, dtype=w.torch_dtype))
+                     for _ in range(self.nsets)]
+        self.tokens = w.B * w.N
+        self.alg_bytes = w.B * w.H * w.N * (2 * w.dqk + 2 * w.dv) * 2
+        # flops of the band only: 2 w (dqk + dv) per head-token (QK^T and PV)
+        self.alg_flops = 2.0 * w.window * (w.dqk + w.dv) * w.B * w.H * w.N
+
+    def step(self, i):
+        q, k, v, o = self.sets[i % self.nsets]
+        self.la.la_swa_forward(q, k, v, self.w.window, out=o)
+
+    def l2_note(self):
+        return (f"{self.nsets} rotating input/output sets of "
+                f"{self.alg_bytes / 1e6:.1f} MB (> 126 MB L2 between reuses)")
+
+
+class SwaDecode:
+    """One step = 1024 sliding-window decode steps (one token for each of the
+    B*H heads per call) on w-token caches filled from an N-token prompt."""
+
+    def __init__(self, w, dev, seed_offset=0, steps=None):
+        import causal_kernelized_sequence_b200 as la
+        self.la, self.w, self.dev = la, w, dev
+        T = w.decode_steps if steps is None else steps
+        self.T = T
+        g = torch.Generator(device=dev)
+        g.manual_seed(replica_seed(w, seed_offset))
+        mk = lambda *s: torch.randn(*s, device=dev, generator=g).to(w.torch_dtype)
+        k, v = mk(w.B, w.H, w.N, w.dqk), mk(w.B, w.H, w.N, w.dv)
+        self.kc, self.vc = la.la_swa_cache_fill(k, v, w.window)
+        del k, v
+        self.sq, self.sk, self.sv = mk(T, w.B, w.H, w.dqk), mk(T, w.B, w.H, w.dqk), mk(T, w.B, w.H, w.dv)
+        self.y = torch.empty(T, w.B, w.H, w.dv, device=dev, dtype=w.torch_dtype)
+        # positions per step, precomputed so a step launches only the decode kernels
+        self.pos = (w.N + torch.arange(T, device=dev, dtype=torch.int32))[:, None].expand(T, w.B).contiguous()
+        self.tokens = w.B * T
+        esz = 2 if w.dtype == W.BF16 else 4
+        per_head = (w.window * (w.dqk + w.dv) + (w.dqk + w.dv) + 2 * w.dqk + 2 * w.dv) * esz
+        self.alg_bytes = per_head * w.B * w.H * T
+        self.alg_flops = 2.0 * w.window * (w.dqk + w.dv) * w.B * w.H * T
+
+    def step(self, i):
+        for t in range(self.T):
+            self.la.la_swa_decode_step(self.sq[t], self.sk[t], self.sv[t], self.kc, self.vc, self.pos[t],
+                                       self.w.window, y=self.y[t])
+
+    def l2_note(self):
+        return f"caches {(self.kc.numel() + self.vc.numel()) * self.kc.element_size() / 1e6:.0f} MB > 126 MB L2"
+
+
 def make_run(w, dev, seed_offset):
+    if w.window and w.decode_steps:
+        return SwaDecode(w, dev, seed_offset)
+    if w.window:
+        return SwaPrefill(w, dev, seed_offset)
     if w.decode_steps:
         return Decode(w, dev, seed_offset)
     if w.backward:
@@ -594,7 +659,7 @@ def main():
     if not args.no_secondary and world == 1:
         sec = {}
         for name in ("taylor_bf16_fwd", "elu_bf16_train", "taylor_decode", "taylor_decode_sym", "elu_bf16_varlen",
-                     "elu_bf16_decay_fwd"):
+                     "elu_bf16_decay_fwd", "swa_bf16_fwd", "swa_bf16_decode"):
             ws = W.BY_NAME[name]
             r2 = make_run(ws, dev, 0)
             st = 3 if ws.decode_steps else 50

@@ -98,6 +98,8 @@ def load_library(path: str | None = None):
     lib.la_swa_cache_fill.restype = i
     lib.la_swa_decode_step.argtypes = [vp] * 7 + [i] * 6 + [vp]
     lib.la_swa_decode_step.restype = i
+    lib.la_swa_kernel_plan.argtypes = [i] * 8 + [ctypes.c_char_p, sz]
+    lib.la_swa_kernel_plan.restype = i
     lib.la_kernel_plan.argtypes = [i] * 8 + [ctypes.c_char_p, sz]
     lib.la_kernel_plan.restype = i
     lib.la_selftest_bounded_wait.argtypes = [ctypes.c_uint, vp]
@@ -386,6 +388,11 @@ def la_kernel_plan(op: int, B, H, N, dqk, dv, fmap, dtype):
 def kernel_plan(w):
     """Launches per benchmark step of a workload description (attributes
     B, H, N, dqk, dv, fmap, dtype, backward, decode_steps)."""
+    if getattr(w, "window", 0):
+        buf = ctypes.create_string_buffer(256)
+        n = load_library().la_swa_kernel_plan(1 if w.decode_steps else 0, w.B, w.H, w.N, w.dqk, w.dv, w.window,
+                                              w.dtype, buf, len(buf))
+        return {"launches_per_step": n * max(1, w.decode_steps), "kernels": buf.value.decode().split(",")}
     if w.decode_steps:
         n, names = la_kernel_plan(2, w.B, w.H, 1, w.dqk, w.dv, w.fmap, w.dtype)
         return {"launches_per_step": n * w.decode_steps, "kernels": names}

@@ -887,6 +887,19 @@ la_status la_swa_forward(const void *q, const void *k, const void *v, void *o, f
     return swa_simt_launch<__nv_bfloat16>(q, k, v, o, lse_out, BH, N, dqk, dv, window, st);
 }
 
+int la_swa_kernel_plan(int decode, int B, int H, int N, int dqk, int dv, int window, int dtype, char *buf,
+                       size_t buflen)
+{
+    if (check_swa(B, H, decode ? 1 : N, dqk, dv, window, dtype) != LA_OK) return -1;
+    const char *nm = decode ? (dqk == 64 && dv == 64 && window <= 64 ? "swa_decode64_kernel" : "swa_decode_kernel")
+                            : (swa_tc_shape(dqk, dv, window, dtype) ? "swa_fwd_tc_kernel" : "swa_fwd_simt_kernel");
+    if (buf && buflen) {
+        strncpy(buf, nm, buflen - 1);
+        buf[buflen - 1] = 0;
+    }
+    return 1;
+}
+
 la_status la_swa_cache_fill(const void *k, const void *v, void *k_cache, void *v_cache, int B, int H, int N,
                             int dqk, int dv, int window, int dtype, void *stream)
 {
@@ -913,6 +926,19 @@ la_status la_swa_decode_step(const void *q, const void *k, const void *v, void *
     cudaStream_t st = (cudaStream_t)stream;
     const size_t bytes = sizeof(float) * ((size_t)window + dqk + 8);
     const float scale = (float)(1.0 / sqrt((double)dqk));
+    const bool vec = dqk == 64 && dv == 64 && window <= 64 && aligned(q, 16) && aligned(k, 16) && aligned(v, 16) &&
+                     aligned(k_cache, 16) && aligned(v_cache, 16);
+    if (vec) {
+        if (dtype == LA_F32)
+            swa_decode64_kernel<float><<<B * H, 128, 0, st>>>((const float *)q, (const float *)k, (const float *)v,
+                                                              (float *)y, (float *)k_cache, (float *)v_cache, pos,
+                                                              H, window, scale);
+        else
+            swa_decode64_kernel<__nv_bfloat16><<<B * H, 128, 0, st>>>(
+                (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, (__nv_bfloat16 *)y,
+                (__nv_bfloat16 *)k_cache, (__nv_bfloat16 *)v_cache, pos, H, window, scale);
+        return launch_status();
+    }
     if (dtype == LA_F32) {
         if (set_smem<swa_decode_kernel<float>>(bytes) != LA_OK) return LA_ERR_CUDA;
         swa_decode_kernel<float><<<B * H, kSwaDecodeThreads, bytes, st>>>(

@@ -356,4 +356,113 @@ swa_decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__r
     }
 }
 
+// 8 consecutive elements as floats (16-byte loads; rows are 16-byte aligned).
+__device__ __forceinline__ void load8(const float *p, float *f)
+{
+    const float4 a = *reinterpret_cast<const float4 *>(p), b = *reinterpret_cast<const float4 *>(p + 4);
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16 *p, float *f)
+{
+    fwd_detail::unpack8(*reinterpret_cast<const uint4 *>(p), f);
+}
+__device__ __forceinline__ void copy8(float *dst, const float *src)
+{
+    reinterpret_cast<float4 *>(dst)[0] = reinterpret_cast<const float4 *>(src)[0];
+    reinterpret_cast<float4 *>(dst)[1] = reinterpret_cast<const float4 *>(src)[1];
+}
+__device__ __forceinline__ void copy8(__nv_bfloat16 *dst, const __nv_bfloat16 *src)
+{
+    *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(src);
+}
+
+// Decode step for d = dv = 64 and windows up to 64, one 128-thread block per
+// (b, h).  Every load is issued up front with 16-byte accesses: thread pair
+// (2j, 2j+1) holds key j (one half of d each) and thread (g, c) the value
+// columns 8c..8c+7 of keys g, g+16, g+32, g+48.  The new token's k and v
+// are read from the inputs, not from its cache slot, so the slot can be
+// written without a barrier before the scores.
+template <typename T>
+__global__ void __launch_bounds__(128, 4)
+swa_decode64_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, T *__restrict__ y,
+                    T *__restrict__ kc, T *__restrict__ vc, const int *__restrict__ pos, int H, int w, float scale)
+{
+    __shared__ float p_s[64];
+    __shared__ float part[16][64];
+    __shared__ float red[8];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const size_t bh = blockIdx.x;
+    const int t = pos[bh / H];
+    if (t < 0) {
+        if (tid == 0) report(kStatusCheck);
+        return;
+    }
+    const int slot = t % w, n = min(t + 1, w);
+    const T *kin = k + bh * 64, *vin = v + bh * 64;
+    T *kb = kc + bh * (size_t)w * 64, *vb = vc + bh * (size_t)w * 64;
+    // keys
+    const int j = tid >> 1, h = tid & 1;
+    float kf[32], qf[32];
+    const bool kvalid = j < n;
+    const T *krow = (j == slot ? kin : kb + (size_t)j * 64) + h * 32;
+#pragma unroll
+    for (int e = 0; e < 32; e += 8) {
+        if (kvalid) load8(krow + e, kf + e);
+        load8(q + bh * 64 + h * 32 + e, qf + e);
+    }
+    // values
+    const int g = tid >> 3, c8 = (tid & 7) * 8;
+    float vf[4][8];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const int jj = g + 16 * r;
+        if (jj < n) load8((jj == slot ? vin : vb + (size_t)jj * 64) + c8, vf[r]);
+    }
+    // the new token into its slot (no thread reads the slot from the cache)
+    if (tid < 8) copy8(kb + (size_t)slot * 64 + tid * 8, kin + tid * 8);
+    else if (tid < 16) copy8(vb + (size_t)slot * 64 + (tid - 8) * 8, vin + (tid - 8) * 8);
+    // scores and softmax
+    float s = 0.f;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) s = fmaf(qf[e], kvalid ? kf[e] : 0.f, s);
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    s = kvalid ? s * scale : -INFINITY;
+    float m = s;
+#pragma unroll
+    for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    m = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    const float e = kvalid ? expf(s - m) : 0.f;
+    if (h == 0) p_s[j] = e;
+    float den = h == 0 ? e : 0.f;
+#pragma unroll
+    for (int off = 16; off; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+    if (lane == 0) red[4 + warp] = den;
+    __syncthreads();
+    den = (red[4] + red[5]) + (red[6] + red[7]);
+    // outputs: partial sums of 16 key groups, then one column per thread
+    float acc[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const int jj = g + 16 * r;
+        if (jj < n) {
+            const float pj = p_s[jj];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) acc[c] = fmaf(pj, vf[r][c], acc[c]);
+        }
+    }
+#pragma unroll
+    for (int c = 0; c < 8; ++c) part[g][c8 + c] = acc[c];
+    __syncthreads();
+    if (tid < 64) {
+        float o = 0.f;
+#pragma unroll
+        for (int gg = 0; gg < 16; ++gg) o += part[gg][tid];
+        st(y + bh * 64 + tid, o / den);
+    }
+}
+
 }  // namespace la

@@ -255,6 +255,11 @@ LA_API la_status la_swa_forward(const void *q, const void *k, const void *v, voi
                                 int B, int H, int N, int dqk, int dv, int window, int dtype,
                                 void *stream);
 
+/* la_kernel_plan for the sliding-window calls: decode = 0 for
+ * la_swa_forward, 1 for la_swa_decode_step (N ignored).  Same output rules. */
+LA_API int la_swa_kernel_plan(int decode, int B, int H, int N, int dqk, int dv, int window, int dtype,
+                              char *buf, size_t buflen);
+
 /* The w-token key/value cache of sliding-window generation (Knowl 4):
  * k_cache [B,H,w,dqk], v_cache [B,H,w,dv] of dtype; token t of a sequence
  * lives in slot t mod w.  la_swa_cache_fill copies the last min(N, w) tokens

@@ -509,6 +509,42 @@ def test_workload_elu_bf16_decay_fwd():
     assert (r["den"] > 0).all()
 
 
+def test_workload_swa_bf16_fwd():
+    w = W.BY_NAME["swa_bf16_fwd"]
+    q, k, v, _ = W.make_inputs(w)
+    r = la.la_swa_forward(q.to(DEV), k.to(DEV), v.to(DEV), w.window, lse=True)
+    torch.cuda.synchronize()
+    la.la_get_device_status()
+    for b, h in [(0, 0), (2, 5), (3, 7)]:
+        sl = lambda t: t[b:b + 1, h:h + 1]
+        o_ref, lse_ref = orc.swa_forward(sl(q), sl(k), sl(v), w.window)
+        assert orc.max_rel_l2(sl(r["o"]).cpu(), o_ref) <= 1e-2, (b, h)
+        assert orc.max_rel_l2(sl(r["lse"]).cpu(), lse_ref) <= 1e-2
+    assert torch.isfinite(r["o"].float()).all()
+
+
+def test_workload_swa_bf16_decode():
+    """The decode workload's shapes (1024 x 16 heads, 64-token caches filled
+    by a 64-token prompt), 16 steps, sampled heads against the oracle."""
+    w = W.BY_NAME["swa_bf16_decode"]
+    (q, k, v), (sq, sk, sv) = W.make_decode_inputs(w, steps=16)
+    kc, vc = la.la_swa_cache_fill(k.to(DEV), v.to(DEV), w.window)
+    pos = torch.full((w.B,), w.N, dtype=torch.int32, device=DEV)
+    ys = []
+    for t in range(16):
+        ys.append(la.la_swa_decode_step(sq[t].to(DEV), sk[t].to(DEV), sv[t].to(DEV), kc, vc, pos, w.window).cpu())
+        pos += 1
+    torch.cuda.synchronize()
+    la.la_get_device_status()
+    for b, h in [(0, 0), (100, 7), (1023, 15)]:
+        qf = torch.cat([q[b, h], sq[:, b, h]])[None, None]
+        kf = torch.cat([k[b, h], sk[:, b, h]])[None, None]
+        vf = torch.cat([v[b, h], sv[:, b, h]])[None, None]
+        o_ref, _ = orc.swa_forward(qf, kf, vf, w.window)
+        got = torch.stack([y[b, h] for y in ys])[None, None]
+        assert orc.max_rel_l2(got, o_ref[:, :, w.N:]) <= 1e-2, (b, h)
+
+
 def test_workload_elu_bf16_varlen():
     w = W.BY_NAME["elu_bf16_varlen"]
     q, k, v, cu = W.make_varlen_inputs(w)

@@ -61,6 +61,7 @@ class Workload:
     decode_steps: int = 0
     varlen: bool = False   # B sequences of seeded lengths in [1, N], packed [H, T, *]
     decay: bool = False    # gated form: log forget gates g ~ U(-0.05, 0) per token
+    window: int = 0        # sliding-window softmax attention with this window (no feature map)
 
     @property
     def torch_dtype(self):
@@ -78,6 +79,8 @@ class Workload:
 
     def describe(self) -> str:
         fm = {ELU1: "elu1", TAYLOR2: "taylor2", TAYLOR2_SYM: "taylor2sym"}[self.fmap]
+        if self.window:
+            fm = f"sliding-window softmax w={self.window}"
         dt = "f32" if self.dtype == F32 else "bf16"
         s = f"{self.name}: {fm} {dt} B={self.B} H={self.H} N={self.N} dqk={self.dqk} dv={self.dv}"
         if self.decay:
@@ -102,6 +105,12 @@ WORKLOADS = [
     Workload("elu_bf16_varlen", 5, ELU1, BF16, 16, 8, 2048, 64, 64, 1.0 / math.sqrt(64), varlen=True),
     # the headline shape with per-token forget gates
     Workload("elu_bf16_decay_fwd", 6, ELU1, BF16, 4, 8, 4096, 64, 64, 1.0 / math.sqrt(64), decay=True),
+    # BASED's local mixer: sliding-window attention, w = 64, d = 64 (the width and head dimension
+    # of the page's generation benchmark), on the headline shape; and its decode with a 64-token cache
+    Workload("swa_bf16_fwd", 7, ELU1, BF16, 4, 8, 4096, 64, 64, 1.0, window=64),
+    # (decode: 1024 sequences so that the 64-token bf16 caches, 268 MB, exceed L2; a 64-token
+    # prompt fills each window, and a longer prompt would leave the same cache)
+    Workload("swa_bf16_decode", 8, ELU1, BF16, 1024, 16, 64, 64, 64, 1.0, decode_steps=1024, window=64),
 ]
 BY_NAME = {w.name: w for w in WORKLOADS}
 
