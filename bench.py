@@ -534,12 +534,14 @@ def oracle_sample(w, heads=None, positions=None, min_cpu_s=0.0):
         reps += 1
         if time.process_time() - c0 >= min_cpu_s or time.perf_counter() - t0 >= 60:
             break
+    cpu_s = time.process_time() - c0
     dt = (time.perf_counter() - t0) / reps
     frac = (Hs * Ns) / (w.B * w.H * (w.decode_steps if w.decode_steps else w.N))
     full_tokens = w.B * (w.decode_steps if w.decode_steps else w.N)
     desc = (f"fp64 oracle ({'decode steps' if w.decode_steps else 'recurrent form'}"
             f"{' + backward' if w.backward else ''}) on {Hs} of {w.B * w.H} heads x {Ns} positions; "
-            f"tokens/s scaled to the full workload by head-token count; {reps} repetitions")
+            f"tokens/s scaled to the full workload by head-token count; {reps} repetitions, "
+            f"{cpu_s:.1f} s of CPU time over the oracle's threads")
     return full_tokens * frac / dt, dt * reps, desc
 
 
