@@ -239,6 +239,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *tma_bar = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
     uint64_t *mma_bar = tma_bar + 2;
+    uint64_t *x_bar = tma_bar + 5;   // MODE 0: the scores (MMA1) alone, so the mask need not wait for MMA3
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tma_bar + 3);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tma_bar + 4);
 
@@ -274,6 +275,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) mbar_init(&tma_bar[s], 1);
         mbar_init(mma_bar, 1);
+        mbar_init(x_bar, 1);
         *abort_flag = 0;
         mbar_init_fence();
         prefetch_tensormap(&tm_q);
@@ -397,7 +399,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (tid == 0)
         for (int s = 0; s < STAGES && c_begin + s < c_end; ++s) issue_tma(c_begin + s, s);
 
-    uint32_t mma_phase = 0;
+    uint32_t mma_phase = 0, x_phase = 0;
     const float inv_c1 = p.inv_c1, inv_c2 = p.inv_c2, r2_inv_c2 = p.inv_c2 * 1.41421356237309504880f;
     float seg_log = 0.f;   // gated: sum of this segment's gates so far
     float *gL = reinterpret_cast<float *>(smem + Cfg::OFF_G);   // [C] prefix sums of the chunk's gates
@@ -562,11 +564,18 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     }
                 }
             }
+            if (MODE == 0) mma_commit(x_bar);
+            // MMA3 runs under the mask step; the commit after MMA2 covers it
             if (!gated || MODE == 1) issue_state_mma(aK, aV, have_state);
-            mma_commit(mma_bar);
+            if (MODE == 1) mma_commit(mma_bar);
         }
-        if (!mbar_wait(mma_bar, mma_phase)) *abort_flag = 1;
-        mma_phase ^= 1u;
+        if (MODE == 0) {
+            if (!mbar_wait(x_bar, x_phase)) *abort_flag = 1;
+            x_phase ^= 1u;
+        } else {
+            if (!mbar_wait(mma_bar, mma_phase)) *abort_flag = 1;
+            mma_phase ^= 1u;
+        }
         tc_fence_after();
         if (!gated || MODE == 1) have_state = true;
 
