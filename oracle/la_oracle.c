@@ -529,3 +529,71 @@ void orc_swa_forward(int B, int H, int N, int dqk, int dv, int w, double scale,
         free(sc);
     }
 }
+
+/* Gradients of the gated masked form by brute force, one slice per (b,h):
+ *   w_ij = (prod_{l=j+1..i} exp(g_l)) phi(q_i).phi(k_j),  y_i = sum_j w_ij v_j / sum_j w_ij,
+ *   g_i = dO_i / den_i,  dden_i = -g_i . y_i,  dw_ij = g_i . v_j + dden_i,
+ *   dv_j = sum_{i>=j} w_ij g_i,
+ *   dphiq_i = sum_{j<=i} dw_ij e_ij phi(k_j),  dphik_j = sum_{i>=j} dw_ij e_ij phi(q_i)   (e_ij = w_ij / a_ij),
+ *   dg_l = sum over the pairs j < l <= i of dw_ij w_ij   (g_l scales every such w_ij),
+ * then dq, dk through the feature map's Jacobian.  O(N^3) for dg. */
+void orc_backward_brute_decay(int fmap, int B, int H, int N, int dqk, int dv,
+                              const double *q, const double *k, const double *v, const double *g,
+                              const double *dout, double *dq, double *dk, double *dvo, double *dg)
+{
+    const int BH = B * H;
+    const int F = orc_feature_dim(fmap, dqk);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int bh = 0; bh < BH; ++bh) {
+        const double *qs = q + (size_t)bh * N * dqk, *ks = k + (size_t)bh * N * dqk;
+        const double *vs = v + (size_t)bh * N * dv, *gs = g + (size_t)bh * N, *dos = dout + (size_t)bh * N * dv;
+        double *phiq = phi_rows(fmap, N, dqk, qs), *phik = phi_rows(fmap, N, dqk, ks);
+        double *e = (double *)calloc((size_t)N * N, sizeof(double));   /* e_ij, j <= i */
+        double *w = (double *)calloc((size_t)N * N, sizeof(double));   /* w_ij */
+        double *gi = (double *)malloc(sizeof(double) * (size_t)N * dv);
+        double *dd = (double *)malloc(sizeof(double) * (size_t)N);
+        double *dphiq = (double *)calloc((size_t)N * F, sizeof(double));
+        double *dphik = (double *)calloc((size_t)N * F, sizeof(double));
+        for (int i = 0; i < N; ++i) {
+            double prod = 1.0;
+            for (int j = i; j >= 0; --j) {
+                if (j < i) prod *= exp(gs[j + 1]);
+                e[(size_t)i * N + j] = prod;
+                w[(size_t)i * N + j] = prod * dot(phiq + (size_t)i * F, phik + (size_t)j * F, F);
+            }
+            double den = 0.0;
+            for (int j = 0; j <= i; ++j) den += w[(size_t)i * N + j];
+            double gy = 0.0;
+            for (int c = 0; c < dv; ++c) {
+                double num = 0.0;
+                for (int j = 0; j <= i; ++j) num += w[(size_t)i * N + j] * vs[(size_t)j * dv + c];
+                gi[(size_t)i * dv + c] = dos[(size_t)i * dv + c] / den;
+                gy += gi[(size_t)i * dv + c] * (num / den);
+            }
+            dd[i] = -gy;
+        }
+        double *dgs = dg + (size_t)bh * N;
+        for (int l = 0; l < N; ++l) dgs[l] = 0.0;
+        for (int i = 0; i < N; ++i)
+            for (int j = 0; j <= i; ++j) {
+                const double dw = dot(gi + (size_t)i * dv, vs + (size_t)j * dv, dv) + dd[i];
+                const double ee = e[(size_t)i * N + j], ww = w[(size_t)i * N + j];
+                for (int f = 0; f < F; ++f) {
+                    dphiq[(size_t)i * F + f] += dw * ee * phik[(size_t)j * F + f];
+                    dphik[(size_t)j * F + f] += dw * ee * phiq[(size_t)i * F + f];
+                }
+                for (int l = j + 1; l <= i; ++l) dgs[l] += dw * ww;
+            }
+        for (int j = 0; j < N; ++j)
+            for (int c = 0; c < dv; ++c) {
+                double acc = 0.0;
+                for (int i = j; i < N; ++i) acc += w[(size_t)i * N + j] * gi[(size_t)i * dv + c];
+                dvo[((size_t)bh * N + j) * dv + c] = acc;
+            }
+        for (int i = 0; i < N; ++i) {
+            orc_phi_vjp(fmap, dqk, qs + (size_t)i * dqk, dphiq + (size_t)i * F, dq + ((size_t)bh * N + i) * dqk);
+            orc_phi_vjp(fmap, dqk, ks + (size_t)i * dqk, dphik + (size_t)i * F, dk + ((size_t)bh * N + i) * dqk);
+        }
+        free(phiq); free(phik); free(e); free(w); free(gi); free(dd); free(dphiq); free(dphik);
+    }
+}

@@ -60,11 +60,13 @@ def _load():
             lib.orc_forward_brute_decay.argtypes = [I, I, I, I, I, I] + [_d] * 6
             lib.orc_decode_step_decay.argtypes = [I, I, I, I] + [_d] * 7
             lib.orc_swa_forward.argtypes = [I, I, I, I, I, I, ctypes.c_double] + [_d] * 5
+            lib.orc_backward_brute_decay.argtypes = [I, I, I, I, I, I] + [_d] * 9
             lib.orc_backward_recurrent.argtypes = [I, I, I, I, I, I, _d, _d, _d, _d, _d, _d, _d]
             for f in (lib.orc_phi, lib.orc_phi_vjp, lib.orc_forward_brute, lib.orc_forward_rows,
                       lib.orc_forward_recurrent, lib.orc_decode_step, lib.orc_backward_brute,
                       lib.orc_backward_recurrent, lib.orc_forward_recurrent_decay,
-                      lib.orc_forward_brute_decay, lib.orc_decode_step_decay, lib.orc_swa_forward):
+                      lib.orc_forward_brute_decay, lib.orc_decode_step_decay, lib.orc_swa_forward,
+                      lib.orc_backward_brute_decay):
                 f.restype = None
             _lib = lib
     return _lib
@@ -259,6 +261,19 @@ def swa_decode(q, k, v, window: int):
     sliding-window forward itself (Knowl 4: a w-token key-value cache during
     generation holds exactly those keys)."""
     return swa_forward(q, k, v, window)[0]
+
+
+def backward_brute_decay(fmap: int, q, k, v, g, dout):
+    """Gradients (dq, dk, dv, dg) of the gated forward by brute force: the
+    chain rule through the gated masked form, with dg_l the sum over the pairs
+    j < l <= i of dL/dw_ij w_ij (g_l scales each such weight)."""
+    q, k, v, g, dout = _f64(q), _f64(k), _f64(v), _f64(g), _f64(dout)
+    B, H, N, dqk = q.shape
+    dv = v.shape[-1]
+    dq = np.empty_like(q); dk = np.empty_like(k); dvv = np.empty_like(v); dg = np.empty_like(g)
+    _load().orc_backward_brute_decay(fmap, B, H, N, dqk, dv, _p(q), _p(k), _p(v), _p(g), _p(dout),
+                                     _p(dq), _p(dk), _p(dvv), _p(dg))
+    return dq, dk, dvv, dg
 
 
 def decode_step(fmap: int, q, k, v, s, z):

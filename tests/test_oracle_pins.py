@@ -420,6 +420,52 @@ def test_decay_decode_and_start_state_continue_the_sequence(orc, fmap):
     np.testing.assert_allclose(s2, sfull, rtol=1e-11, atol=1e-12)
 
 
+def test_decay_backward_zero_gate_is_plain_backward(orc):
+    # g = 0: the gated gradients of q, k, v are the ungated ones (pinned above).
+    q = rnd(190, 1, 2, 20, 4, scale=0.7); k = rnd(191, 1, 2, 20, 4, scale=0.7)
+    v = rnd(192, 1, 2, 20, 3); do = rnd(193, 1, 2, 20, 3)
+    dq, dk, dvv, dg = orc.backward_brute_decay(TAYLOR2, q, k, v, np.zeros((1, 2, 20)), do)
+    for a, b in zip((dq, dk, dvv), orc.backward_recurrent(TAYLOR2, q, k, v, do)):
+        np.testing.assert_allclose(a, b, rtol=1e-10, atol=1e-12)
+    assert np.abs(dg[..., 1:]).max() > 1e-6 and np.abs(dg[..., 0]).max() < 1e-12   # g_0 scales an empty state
+
+
+@pytest.mark.parametrize("fmap", [ELU1, TAYLOR2_SYM])
+def test_decay_backward_finite_differences(orc, fmap):
+    d, dv, N = (3, 2, 9) if fmap == ELU1 else (3, 3, 7)
+    q = rnd(200, 1, 1, N, d, scale=0.8); k = rnd(201, 1, 1, N, d, scale=0.8)
+    v = rnd(202, 1, 1, N, dv); do = rnd(203, 1, 1, N, dv); g = -np.abs(rnd(204, 1, 1, N)) * 0.5
+    got = orc.backward_brute_decay(fmap, q, k, v, g, do)
+    L = lambda q, k, v, g: (orc.forward_brute_decay(fmap, q, k, v, g)[0] * do).sum()
+    h = 1e-6
+    args = [q, k, v, g]
+    for which in range(4):
+        fd = np.zeros_like(args[which])
+        for idx in np.ndindex(*args[which].shape):
+            ap = [a.copy() for a in args]; am = [a.copy() for a in args]
+            ap[which][idx] += h; am[which][idx] -= h
+            fd[idx] = (L(*ap) - L(*am)) / (2 * h)
+        np.testing.assert_allclose(got[which], fd, rtol=1e-6, atol=1e-8)
+
+
+def test_decay_backward_autograd(orc):
+    # torch autograd through a plain fp64 torch expression of the gated masked
+    # form (decay factors from a cumulative sum of the gates).
+    N, d, dv = 16, 4, 3
+    q = rnd(210, 1, 2, N, d, scale=0.7); k = rnd(211, 1, 2, N, d, scale=0.7)
+    v = rnd(212, 1, 2, N, dv); do = rnd(213, 1, 2, N, dv); g = -np.abs(rnd(214, 1, 2, N)) * 0.3
+    tq, tk, tv, tg = (torch.tensor(x, requires_grad=True) for x in (q, k, v, g))
+    A = (torch.nn.functional.elu(tq) + 1) @ (torch.nn.functional.elu(tk) + 1).transpose(-1, -2)
+    cs = torch.cumsum(tg, -1)
+    decay = torch.exp(cs[..., :, None] - cs[..., None, :])      # prod_{l=j+1..i} a_l for j <= i
+    W = torch.tril(A * torch.tril(decay))
+    y = (W @ tv) / W.sum(-1, keepdim=True)
+    (y * torch.from_numpy(do)).sum().backward()
+    got = orc.backward_brute_decay(ELU1, q, k, v, g, do)
+    for a, t in zip(got, (tq, tk, tv, tg)):
+        np.testing.assert_allclose(a, t.grad.numpy(), rtol=1e-9, atol=1e-11)
+
+
 # ------------------------------------------------- sliding-window attention
 
 def test_swa_wide_window_is_causal_softmax_attention(orc):
