@@ -13,6 +13,7 @@ Entry points (same names as the C ABI):
     la_forward_varlen(q, k, v, cu_seqlens, max_seqlen, fmap, ...) -> dict
     la_forward_noalloc(q, k, v, fmap, ...) -> dict
     la_backward(q, k, v, dout, fmap) -> (dq, dk, dv)
+    la_backward_decay(q, k, v, log_decay, dout, fmap) -> (dq, dk, dv, dlog_decay)
     la_decode_step(q, k, v, s, z, fmap, y=None, log_decay=None) -> y   (s, z in place)
     la_swa_forward(q, k, v, window, *, out=None, lse=False) -> dict
     la_swa_cache_fill(k, v, window) -> (k_cache, v_cache)
@@ -86,6 +87,10 @@ def load_library(path: str | None = None):
     lib.la_forward_decay.argtypes = [vp] * 11 + [sz] + [i] * 7 + [vp]
     lib.la_forward_decay.restype = i
     lib.la_decode_step_decay.argtypes = [vp] * 7 + [i] * 6 + [vp]
+    lib.la_backward_decay.argtypes = [vp] * 10 + [sz] + [i] * 7 + [vp]
+    lib.la_backward_decay.restype = i
+    lib.la_backward_decay_workspace_bytes.argtypes = [i] * 7
+    lib.la_backward_decay_workspace_bytes.restype = sz
     lib.la_decode_step_decay.restype = i
     lib.la_forward_varlen_workspace_bytes.argtypes = [i] * 7
     lib.la_forward_varlen_workspace_bytes.restype = sz
@@ -290,6 +295,27 @@ def la_backward(q, k, v, dout, fmap, *, workspace=None):
     _check(lib.la_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dvv),
                            _ptr(workspace), wsb, B, H, N, dqk, dv, fmap, dt, _stream()), "la_backward")
     return dq, dk, dvv
+
+
+def la_backward_decay(q, k, v, log_decay, dout, fmap, *, workspace=None):
+    """Gradients (dq, dk, dv, dlog_decay) of the gated forward (la_forward with
+    log_decay) for upstream gradient dout."""
+    lib = load_library()
+    _dev(q, k, v, dout, log_decay)
+    B, H, N, dqk = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q)
+    if log_decay.dtype != torch.float32 or tuple(log_decay.shape) != (B, H, N):
+        raise ValueError("log_decay must be fp32 [B,H,N]")
+    dq, dk, dvv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dg = torch.empty(B, H, N, dtype=torch.float32, device=q.device)
+    wsb = int(lib.la_backward_decay_workspace_bytes(B, H, N, dqk, dv, fmap, dt))
+    if workspace is None:
+        workspace = torch.empty(wsb, dtype=torch.uint8, device=q.device)
+    _check(lib.la_backward_decay(_ptr(q), _ptr(k), _ptr(v), _ptr(log_decay), _ptr(dout), _ptr(dq), _ptr(dk),
+                                 _ptr(dvv), _ptr(dg), _ptr(workspace), wsb, B, H, N, dqk, dv, fmap, dt, _stream()),
+           "la_backward_decay")
+    return dq, dk, dvv, dg
 
 
 def la_decode_step(q, k, v, s, z, fmap, y=None, log_decay=None):

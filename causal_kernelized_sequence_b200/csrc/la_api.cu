@@ -227,7 +227,8 @@ la_status forward_simt(const void *q, const void *k, const void *v, void *o, con
 template <typename T>
 la_status backward_simt(const void *q, const void *k, const void *v, const void *dout, void *dq,
                         void *dk, void *dvp, float *ws, int B, int H, int N, int dqk, int dv,
-                        int fmap, cudaStream_t stream)
+                        int fmap, cudaStream_t stream, const float *logdecay = nullptr,
+                        float *dlogdecay = nullptr)
 {
     // The backward reads no state, and both Taylor maps give the same
     // phi(q).phi(k), hence the same gradients: run the 273-feature map on the
@@ -239,7 +240,7 @@ la_status backward_simt(const void *q, const void *k, const void *v, const void 
     if (set_smem<bwd_simt_kernel<T>>(bytes) != LA_OK) return LA_ERR_CUDA;
     bwd_simt_kernel<T><<<B * H, kSimtThreads, bytes, stream>>>(
         (const T *)q, (const T *)k, (const T *)v, (const T *)dout, ws, (T *)dq, (T *)dk, (T *)dvp,
-        N, dv, fp, L);
+        N, dv, fp, L, logdecay, dlogdecay);
     return launch_status();
 }
 
@@ -826,6 +827,34 @@ size_t la_forward_decay_workspace_bytes(int B, int H, int N, int dqk, int dv, in
     if (P <= 1) return 0;
     // segment increments, then each segment's sum of log gates
     return (size_t)B * H * P * (tc_increment_floats(dqk, dv, fmap) + 1) * sizeof(float);
+}
+
+size_t la_backward_decay_workspace_bytes(int B, int H, int N, int dqk, int dv, int fmap, int dtype)
+{
+    if (check_shape(B, H, N, dqk, dv, fmap, dtype) != LA_OK) return 0;
+    return (size_t)B * H * N * 2 * sizeof(float);   // den_i, dden_i per token
+}
+
+la_status la_backward_decay(const void *q, const void *k, const void *v, const float *log_decay,
+                            const void *dout, void *dq, void *dk, void *dvp, float *dlog_decay, void *workspace,
+                            size_t workspace_bytes, int B, int H, int N, int dqk, int dv, int fmap, int dtype,
+                            void *stream)
+{
+    const la_status sh = check_shape(B, H, N, dqk, dv, fmap, dtype);
+    if (sh != LA_OK) return sh;
+    if (!q || !k || !v || !log_decay || !dout || !dq || !dk || !dvp || !dlog_decay || !workspace)
+        return LA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(dout, 16) || !aligned(dq, 16) ||
+        !aligned(dk, 16) || !aligned(dvp, 16) || !aligned(log_decay, 4) || !aligned(dlog_decay, 4) ||
+        !aligned(workspace, 4))
+        return LA_ERR_INVALID_ARG;
+    if (workspace_bytes < la_backward_decay_workspace_bytes(B, H, N, dqk, dv, fmap, dtype)) return LA_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    float *ws = (float *)workspace;
+    if (dtype == LA_F32)
+        return backward_simt<float>(q, k, v, dout, dq, dk, dvp, ws, B, H, N, dqk, dv, fmap, st, log_decay, dlog_decay);
+    return backward_simt<__nv_bfloat16>(q, k, v, dout, dq, dk, dvp, ws, B, H, N, dqk, dv, fmap, st, log_decay,
+                                        dlog_decay);
 }
 
 la_status la_forward_decay(const void *q, const void *k, const void *v, const float *log_decay, void *o,

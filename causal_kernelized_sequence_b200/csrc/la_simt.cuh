@@ -206,7 +206,7 @@ struct SimtBwdSmem {
     size_t floats(int F, int dqk, int dv) const
     {
         return (size_t)F * DS + F + 2 * (size_t)C * dqk + 3 * (size_t)C * FS +
-               2 * (size_t)C * dv + 2 * (size_t)C * C + 2 * (size_t)C;
+               2 * (size_t)C * dv + 3 * (size_t)C * C + 6 * (size_t)C;
     }
 };
 
@@ -219,7 +219,8 @@ template <typename T>
 __global__ void __launch_bounds__(kSimtThreads)
 bwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                 const T *__restrict__ dout, float *__restrict__ ws, T *__restrict__ dq,
-                T *__restrict__ dk, T *__restrict__ dvo, int N, int dv, FmapParams fp, SimtBwdSmem L)
+                T *__restrict__ dk, T *__restrict__ dvo, int N, int dv, FmapParams fp, SimtBwdSmem L,
+                const float *__restrict__ logdecay = nullptr, float *__restrict__ dlogdecay = nullptr)
 {
     extern __shared__ float sm[];
     const int F = fp.F, dqk = fp.dqk, C = L.C, FS = L.FS, DS = L.DS;
@@ -236,6 +237,15 @@ bwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
     float *dA = A + C * C;              // [C][C]    da_ij
     float *dd = dA + C * C;             // [C]       dden_i = -g_i . y_i
     float *dn = dd + C;                 // [C]       den_i
+    // gated form (logdecay != null): w_ij = D_ij a_ij with D_ij = exp(g_{j+1} + ... + g_i)
+    float *Dm = dn + C;                 // [C][C]    D_ij, j <= i
+    float *cum = Dm + C * C;            // [C]       e_i: exp(g_{t0} + ... + g_{t0+i})
+    float *wk = cum + C;                // [C]       f_j: exp(g_{t0+j+1} + ... + g_{last})
+    float *graw = wk + C;               // [C]       the chunk's gates
+    float *ub = graw + C;               // [C]       u_j = phi(k_j) . dphi(k_j)  (pass 2)
+    double ucarry = 0.0;                // sum of u_j over the later chunks (pass 2); double:
+                                        // the full sum is zero, so the partial sums cancel
+    float elast = 1.f;                  // exp of the chunk's gate sum
 
     const int tid = threadIdx.x, nt = blockDim.x;
     const int lane = tid & 31, warp = tid >> 5, nwarps = nt >> 5;
@@ -263,19 +273,52 @@ bwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
                 vs[i] = ld(vb + (size_t)t0 * dv + i);
                 gs[i] = ld(gb + (size_t)t0 * dv + i);
             }
+            if (logdecay && warp == 0) {
+                // gate factors as plain sums of gates (as in the gated forward)
+                const float gj = lane < Lc ? logdecay[bh * N + t0 + lane] : 0.f;
+                float x = gj;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, x, off);
+                    if (lane >= off) x += y;
+                }
+                float r = __shfl_down_sync(0xffffffffu, gj, 1);
+                if (lane + 1 >= Lc) r = 0.f;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float y = __shfl_down_sync(0xffffffffu, r, off);
+                    if (lane + off < 32) r += y;
+                }
+                if (lane < Lc) {
+                    cum[lane] = expf(x);
+                    wk[lane] = expf(r);
+                    graw[lane] = gj;
+                }
+            }
             __syncthreads();
+            if (logdecay) {
+                for (int idx = tid; idx < Lc * Lc; idx += nt) {
+                    const int i = idx / Lc, j = idx - i * Lc;
+                    float gsum = 0.f;
+                    for (int l = j + 1; l <= i; ++l) gsum += graw[l];
+                    Dm[i * C + j] = j <= i ? expf(gsum) : 0.f;
+                }
+                elast = cum[Lc - 1];
+            }
             for (int idx = tid; idx < Lc * F; idx += nt) {
                 const int i = idx / F, f = idx - i * F;
                 pq[i * FS + f] = phi_feature(fp, xq + i * dqk, f);
                 pk[i * FS + f] = phi_feature(fp, xk + i * dqk, f);
             }
             __syncthreads();
-            // a_ij = phi(q_i).phi(k_j), j <= i
+            // a_ij = phi(q_i).phi(k_j), j <= i (gated: w_ij = D_ij a_ij)
             for (int idx = tid; idx < Lc * Lc; idx += nt) {
                 const int i = idx / Lc, j = idx - i * Lc;
                 float a = 0.f;
-                if (j <= i)
+                if (j <= i) {
                     for (int f = 0; f < F; ++f) a = fmaf(pq[i * FS + f], pk[j * FS + f], a);
+                    if (logdecay) a *= Dm[i * C + j];
+                }
                 A[i * C + j] = a;
             }
             __syncthreads();
@@ -283,14 +326,17 @@ bwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
                 // den_i and y_i in fp32 from the state entering the chunk;
                 // dden_i = -(dout_i . num_i) / den_i^2.  One warp per row.
                 for (int i = warp; i < Lc; i += nwarps) {
+                    const float ei = logdecay ? cum[i] : 1.f;
                     float d = 0.f;
                     for (int f = lane; f < F; f += 32) d = fmaf(pq[i * FS + f], zt[f], d);
+                    d *= ei;
                     for (int j = lane; j <= i; j += 32) d += A[i * C + j];
                     for (int off = 16; off; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
                     float gy = 0.f;
                     for (int c = lane; c < dv; c += 32) {
                         float num = 0.f;
                         for (int f = 0; f < F; ++f) num = fmaf(pq[i * FS + f], St[f * DS + c], num);
+                        num *= ei;
                         for (int j = 0; j <= i; ++j) num = fmaf(A[i * C + j], vs[j * dv + c], num);
                         gy = fmaf(gs[i * dv + c], num, gy);
                     }
@@ -318,6 +364,7 @@ bwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
                 if (j <= i) {
                     for (int c = 0; c < dv; ++c) da = fmaf(gs[i * dv + c], vs[j * dv + c], da);
                     da += dd[i];
+                    if (logdecay) da *= Dm[i * C + j];   // dL/da_ij = D_ij dL/dw_ij
                 }
                 dA[i * C + j] = da;
             }
@@ -328,6 +375,7 @@ bwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
                     const int i = idx / F, f = idx - i * F;
                     float acc = zt[f] * dd[i];
                     for (int c = 0; c < dv; ++c) acc = fmaf(St[f * DS + c], gs[i * dv + c], acc);
+                    if (logdecay) acc *= cum[i];
                     for (int j = 0; j <= i; ++j) acc = fmaf(dA[i * C + j], pk[j * FS + f], acc);
                     dphi[i * FS + f] = acc;
                 }
@@ -336,16 +384,17 @@ bwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
                     const int i = idx / dqk, a = idx - i * dqk;
                     st(dqb + (size_t)t0 * dqk + idx, phi_vjp_component(fp, xq + i * dqk, dphi + i * FS, a));
                 }
-                // S += phi(K_c)^T V_c ; z += sum_j phi(k_j)
+                // S = e_last S + sum_j f_j phi(k_j) v_j^T ; z likewise (ungated: factors 1)
                 for (int idx = tid; idx < F * dv; idx += nt) {
                     const int f = idx / dv, c = idx - f * dv;
-                    float acc = St[f * DS + c];
-                    for (int j = 0; j < Lc; ++j) acc = fmaf(pk[j * FS + f], vs[j * dv + c], acc);
+                    float acc = St[f * DS + c] * elast;
+                    for (int j = 0; j < Lc; ++j)
+                        acc = fmaf(logdecay ? pk[j * FS + f] * wk[j] : pk[j * FS + f], vs[j * dv + c], acc);
                     St[f * DS + c] = acc;
                 }
                 for (int f = tid; f < F; f += nt) {
-                    float acc = zt[f];
-                    for (int j = 0; j < Lc; ++j) acc += pk[j * FS + f];
+                    float acc = zt[f] * elast;
+                    for (int j = 0; j < Lc; ++j) acc += logdecay ? pk[j * FS + f] * wk[j] : pk[j * FS + f];
                     zt[f] = acc;
                 }
             } else {
@@ -354,32 +403,56 @@ bwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
                     const int j = idx / F, f = idx - j * F;
                     float acc = zt[f];
                     for (int c = 0; c < dv; ++c) acc = fmaf(St[f * DS + c], vs[j * dv + c], acc);
+                    if (logdecay) acc *= wk[j];
                     for (int i = j; i < Lc; ++i) acc = fmaf(dA[i * C + j], pq[i * FS + f], acc);
                     dphi[j * FS + f] = acc;
                 }
-                // dv_j = sum_{i>=j, chunk} a_ij g_i + R^T phi(k_j)
+                // dv_j = sum_{i>=j, chunk} a_ij g_i + R^T phi(k_j)   (gated: w_ij, f_j R)
                 for (int idx = tid; idx < Lc * dv; idx += nt) {
                     const int j = idx / dv, c = idx - j * dv;
                     float acc = 0.f;
                     for (int f = 0; f < F; ++f) acc = fmaf(St[f * DS + c], pk[j * FS + f], acc);
+                    if (logdecay) acc *= wk[j];
                     for (int i = j; i < Lc; ++i) acc = fmaf(A[i * C + j], gs[i * dv + c], acc);
                     st(dvb + (size_t)t0 * dv + idx, acc);
                 }
                 __syncthreads();
+                if (logdecay) {
+                    // dL/dg_l = -sum_{j>=l} phi(k_j) . dphi(k_j): the weights of each
+                    // output row sum to one, so only the pairs crossing l remain
+                    for (int j = warp; j < Lc; j += nwarps) {
+                        float u = 0.f;
+                        for (int f = lane; f < F; f += 32) u = fmaf(pk[j * FS + f], dphi[j * FS + f], u);
+#pragma unroll
+                        for (int off = 16; off; off >>= 1) u += __shfl_xor_sync(0xffffffffu, u, off);
+                        if (lane == 0) ub[j] = u;
+                    }
+                    __syncthreads();
+                    if (tid == 0) {
+                        double acc = ucarry;
+                        for (int j = Lc - 1; j >= 0; --j) {
+                            acc += (double)ub[j];
+                            dlogdecay[bh * N + t0 + j] = (float)-acc;
+                        }
+                        ucarry = acc;   // only thread 0 carries the running sum
+                    }
+                }
                 for (int idx = tid; idx < Lc * dqk; idx += nt) {
                     const int j = idx / dqk, a = idx - j * dqk;
                     st(dkb + (size_t)t0 * dqk + idx, phi_vjp_component(fp, xk + j * dqk, dphi + j * FS, a));
                 }
-                // R += sum_i phi(q_i) g_i^T ; r += sum_i phi(q_i) dden_i
+                // R = e_last R + sum_i e_i phi(q_i) g_i^T ; r likewise with dden_i (ungated: factors 1)
                 for (int idx = tid; idx < F * dv; idx += nt) {
                     const int f = idx / dv, c = idx - f * dv;
-                    float acc = St[f * DS + c];
-                    for (int i = 0; i < Lc; ++i) acc = fmaf(pq[i * FS + f], gs[i * dv + c], acc);
+                    float acc = St[f * DS + c] * elast;
+                    for (int i = 0; i < Lc; ++i)
+                        acc = fmaf(logdecay ? pq[i * FS + f] * cum[i] : pq[i * FS + f], gs[i * dv + c], acc);
                     St[f * DS + c] = acc;
                 }
                 for (int f = tid; f < F; f += nt) {
-                    float acc = zt[f];
-                    for (int i = 0; i < Lc; ++i) acc = fmaf(pq[i * FS + f], dd[i], acc);
+                    float acc = zt[f] * elast;
+                    for (int i = 0; i < Lc; ++i)
+                        acc = fmaf(logdecay ? pq[i * FS + f] * cum[i] : pq[i * FS + f], dd[i], acc);
                     zt[f] = acc;
                 }
             }

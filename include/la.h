@@ -231,6 +231,21 @@ LA_API la_status la_forward_decay(const void *q, const void *k, const void *v, c
                                   int B, int H, int N, int dqk, int dv, int fmap, int dtype,
                                   void *stream);
 
+/* Gradients of la_forward_decay (from a zero state) for an upstream gradient
+ * dout: dq, dk, dv as in la_backward, and dlog_decay [B,H,N] fp32 = dL/dg_t.
+ * The weights of each output row sum to one, so
+ *     dL/dg_l = sum over the pairs j < l <= i of w_ij dL/dw_ij
+ *             = -sum_{j>=l} phi(k_j) . dL/dphi(k_j),
+ * a suffix sum that the reverse-order pass accumulates.  Every shape runs on
+ * the exact fp32 CUDA-core backward; workspace: la_backward_decay_workspace_bytes. */
+LA_API size_t la_backward_decay_workspace_bytes(int B, int H, int N, int dqk, int dv, int fmap, int dtype);
+
+LA_API la_status la_backward_decay(const void *q, const void *k, const void *v, const float *log_decay,
+                                   const void *dout, void *dq, void *dk, void *dv, float *dlog_decay,
+                                   void *workspace, size_t workspace_bytes,
+                                   int B, int H, int N, int dqk, int dv_dim, int fmap, int dtype,
+                                   void *stream);
+
 /* One gated decode step: S = a S + phi(k) v^T, z = a z + phi(k), then y as in
  * la_decode_step, with a = exp(log_decay[b,h]) per head (log_decay [B,H]
  * fp32, read).  Arguments and errors otherwise those of la_decode_step. */

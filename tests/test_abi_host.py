@@ -254,3 +254,21 @@ def test_swa_argument_errors(lib):
     c.restype = ctypes.c_int
     assert c(P(None), *ptr[1:4], 1, 1, 16, 64, 64, 64, 1, None) == 1
 
+
+def test_backward_decay_argument_errors(lib):
+    P = ctypes.c_void_p
+    f = lib.la_backward_decay
+    f.argtypes = [P] * 10 + [ctypes.c_size_t] + [ctypes.c_int] * 7 + [P]
+    f.restype = ctypes.c_int
+    ptr = [0x1000 * (i + 1) for i in range(10)]   # q k v g dout dq dk dv dg ws
+    def call(i_null=None, wsb=16 * 2 * 4, N=16):
+        args = [P(None) if i == i_null else P(x) for i, x in enumerate(ptr)]
+        return f(*args, wsb, 1, 1, N, 16, 16, 0, 0, None)
+    for i in range(10):
+        assert call(i_null=i) == 1, i              # every pointer is required
+    assert call(wsb=16 * 2 * 4 - 4) == 1           # workspace too small
+    assert call(N=0) == 1
+    lib.la_backward_decay_workspace_bytes.argtypes = [ctypes.c_int] * 7
+    lib.la_backward_decay_workspace_bytes.restype = ctypes.c_size_t
+    assert lib.la_backward_decay_workspace_bytes(2, 3, 100, 16, 16, 0, 1) == 2 * 3 * 100 * 2 * 4
+

@@ -247,6 +247,31 @@ def test_forward_decay_full_forgetting(dtype, fmap, dqk, dv):
     assert torch.isfinite(r["o"].float()).all()
 
 
+@pytest.mark.parametrize("dtype", [W.F32, W.BF16])
+@pytest.mark.parametrize("fmap,dqk,dv", [(ELU1, 32, 32), (ELU1, 64, 64), (TAYLOR2_SYM, 16, 64), (TAYLOR2, 4, 8)])
+def test_backward_decay(fmap, dqk, dv, dtype):
+    """Gated gradients, the gate's included, against the oracle's brute force."""
+    for N in (1, 17, 64, 65, 200):
+        q, k, v, do = W.random_qkv(9950 + N, 1, 2, N, dqk, dv, fmap=fmap, dtype=dtype,
+                                   scale=1.0 if fmap != ELU1 else dqk ** -0.5, with_dout=True)
+        g = _log_gates(9960 + N, 1, 2, N)
+        dq, dk, dvv, dg = la.la_backward_decay(q.to(DEV), k.to(DEV), v.to(DEV), g.to(DEV), do.to(DEV), fmap)
+        torch.cuda.synchronize()
+        la.la_get_device_status()
+        rq, rk, rv, rg = orc.backward_brute_decay(fmap, q, k, v, g, do)
+        tol = TOL[dtype]
+        if N == 1:
+            # one token: y_1 = v_1, so dq, dk and the gate gradient vanish
+            assert dq.abs().max().item() <= 1e-4 and dk.abs().max().item() <= 1e-4
+            assert dg.abs().max().item() <= 1e-4   # fp32 rounding of phi(k).dphi(k), exactly 0 in exact arithmetic
+            assert orc.max_rel_l2(dvv.cpu(), do) <= tol
+            continue
+        for got, ref, name in ((dq, rq, "dq"), (dk, rk, "dk"), (dvv, rv, "dv"), (dg, rg, "dg")):
+            err = orc.max_rel_l2(got.cpu(), ref)
+            assert err <= tol, (N, name, err)
+        assert dg[..., 0].abs().max().item() <= 1e-4 * dg.abs().max().item()   # g_1 scales an empty state
+
+
 def test_forward_decay_zero_gate_is_plain_forward():
     """g = 0 gives the ungated exact forward bit for bit (fp32, same kernel)."""
     q, k, v, _ = W.random_qkv(9300, 2, 3, 300, 32, 32, dtype=W.F32, scale=32 ** -0.5)
