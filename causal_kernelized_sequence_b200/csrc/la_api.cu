@@ -539,7 +539,7 @@ static la_status swa_tc_launch(const void *q, const void *k, const void *v, void
     const int per_sm = Cfg::TMEM_COLS == 256 ? 2 : 1;   // TMEM: 512 columns per SM
     const int grid = (int)(ntiles < (long long)per_sm * kNumSms ? ntiles : per_sm * kNumSms);
     if (set_smem<swa_fwd_tc_kernel<Cfg>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
-    swa_fwd_tc_kernel<Cfg><<<grid, 128, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+    swa_fwd_tc_kernel<Cfg><<<grid, Cfg::THREADS, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
     return launch_status();
 }
 

@@ -10,14 +10,15 @@
 // (Knowl 4 and the sliding-window generation kernel of Knowl 5).
 //
 // Tensor-core prefill (bf16, dqk = dv = 64, w a multiple of 16 up to 128):
-// one CTA of 128 threads per 128-query tile, persistent over tiles.
+// one CTA of 256 threads (two per query row) per 128-query tile, persistent
+// over tiles.
 //   TMA     Q tile [128 x 64] and K, V spans [128 + w x 64] starting w keys
 //           before the tile (a negative start reads zeros), SW128.
 //   MMA1    S = Q K^T  [128 x (128 + w)] fp32 -> TMEM.
-//   softmax thread i reads the band of its row (columns i+1 .. i+w of the
-//           span, the keys t0+i-w+1 .. t0+i), takes max and exp2 in fp32 and
-//           writes P (bf16, zero off the band) over the Q/K buffer, which
-//           MMA1 no longer needs.
+//   softmax the two threads of row i read the band of the row (columns
+//           i+1 .. i+w of the span, the keys t0+i-w+1 .. t0+i) in two parts,
+//           combine max and sum through shared memory, and write P (bf16,
+//           zero off the band) over the Q/K buffer, which MMA1 no longer needs.
 //   MMA2    O = P V  [128 x 64] -> TMEM; then o = O / rowsum, bf16.
 // The next tile's loads are issued as soon as MMA2 completes, under the
 // epilogue.  For w <= 64 a CTA takes 256 TMEM columns and 80 KB of shared
@@ -44,7 +45,8 @@ struct SwaCfg {
     static constexpr int OFF_Q = 0, OFF_K = Q_TILE, OFF_P = 0;
     static constexpr int OFF_V = REGION_A;
     static constexpr int OFF_BAR = OFF_V + (KV_TILE + 1023) / 1024 * 1024;
-    static constexpr int SMEM = OFF_BAR + 64;
+    static constexpr int OFF_RED = OFF_BAR + 64;     // row max and row sum of each half: 4 x 128 floats
+    static constexpr int SMEM = OFF_RED + 4 * C * 4;
     static constexpr int COL_S = 0;
     static constexpr int COL_O = (KW + 31) / 32 * 32;
     static constexpr int TMEM_COLS = COL_O + D <= 256 ? 256 : 512;
@@ -54,6 +56,11 @@ struct SwaCfg {
     static constexpr int SMEM_FLOOR = TMEM_COLS == 256 ? 80 * 1024 : 120 * 1024;
     static constexpr int SMEM_ALLOC = SMEM + 1024 > SMEM_FLOOR ? SMEM + 1024 : SMEM_FLOOR;
     static constexpr int NCOL = 32 + W;              // span columns a warp's rows can touch
+    // two threads per query row (warps w and w + 4 reach the same TMEM lanes):
+    // the first takes H0 of those columns, the second the other H1
+    static constexpr int H0 = 16 * ((NCOL + 31) / 32), H1 = NCOL - H0;
+    static constexpr int THREADS = 256;
+    static constexpr int MIN_BLOCKS = TMEM_COLS == 256 ? 2 : 1;
     static_assert(W % 16 == 0 && W >= 16 && W <= 128, "window: a multiple of 16 up to 128");
     static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory");
 };
@@ -67,7 +74,7 @@ struct SwaParams {
 };
 
 template <class Cfg>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(Cfg::THREADS, Cfg::MIN_BLOCKS)
 swa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const SwaParams p)
 {
@@ -81,8 +88,11 @@ swa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(load_bar + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(load_bar + 3);
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, row = tid;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wq = warp & 3, hh = warp >> 2, row = wq * 32 + lane;   // TMEM lane quadrant, row half
     const int ntiles = p.BH * p.tiles_per_bh;
+    float *red_m = reinterpret_cast<float *>(smem + Cfg::OFF_RED);   // [2][C] row max per half
+    float *red_s = red_m + 2 * C;                                    // [2][C] row sum per half
 
     if (tid == 0) {
         mbar_init(load_bar, 1);
@@ -98,7 +108,7 @@ swa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
     const uint32_t aQ = smem_addr(smem + Cfg::OFF_Q), aK = smem_addr(smem + Cfg::OFF_K);
     const uint32_t aV = smem_addr(smem + Cfg::OFF_V), aP = smem_addr(smem + Cfg::OFF_P);
 
@@ -137,37 +147,47 @@ swa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         tc_fence_after();
 
         // ---- softmax over the band of row i: span columns i+1 .. i+W, and
-        // only keys at index >= 0 (column >= W - t0)
-        float rowsum = 0.f, rowmax = -INFINITY;
+        // only keys at index >= 0 (column >= W - t0).  The two threads of a row
+        // take the columns [c0, c0 + nh) of the warp's span (nh = H0 or H1; the
+        // guard c < nh is the same across a warp).
+        float rowmax, rowsum;
         {
-            const int i = row, c_base = warp * 32;
-            float sv[Cfg::NCOL];
-#pragma unroll
-            for (int c = 0; c < Cfg::NCOL; c += 16) tmem_ld16(tmem + lane_base + Cfg::COL_S + c_base + c, sv + c);
-            tmem_ld_wait();
+            const int i = row, c_base = wq * 32;
+            const int c0 = c_base + (hh ? Cfg::H0 : 0), nh = hh ? Cfg::H1 : Cfg::H0;
             const int lo = max(i + 1, W - t0), hi = i + W;   // inclusive band in span columns
+            float sv[Cfg::H0];
 #pragma unroll
-            for (int c = 0; c < Cfg::NCOL; ++c) {
-                const int jc = c_base + c;
-                if (jc >= lo && jc <= hi) rowmax = fmaxf(rowmax, sv[c]);
-            }
+            for (int c = 0; c < Cfg::H0; c += 16)
+                if (c < nh) tmem_ld16(tmem + lane_base + Cfg::COL_S + c0 + c, sv + c);
+            tmem_ld_wait();
+            float m = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < Cfg::NCOL; ++c) {
-                const int jc = c_base + c;
-                const float e = (jc >= lo && jc <= hi) ? exp2f((sv[c] - rowmax) * p.scale_log2) : 0.f;
+            for (int c = 0; c < Cfg::H0; ++c)
+                if (c < nh && c0 + c >= lo && c0 + c <= hi) m = fmaxf(m, sv[c]);
+            red_m[hh * C + i] = m;
+            __syncthreads();
+            rowmax = fmaxf(red_m[i], red_m[C + i]);
+            float sum = 0.f;
+#pragma unroll
+            for (int c = 0; c < Cfg::H0; ++c) {
+                const float e = (c < nh && c0 + c >= lo && c0 + c <= hi) ? exp2f((sv[c] - rowmax) * p.scale_log2) : 0.f;
                 sv[c] = e;
-                rowsum += e;
+                sum += e;
             }
-            // P row i over all KW columns, K-major SW128 blocks of 64 keys: the
-            // warp's span from the registers, zeros elsewhere
+            red_s[hh * C + i] = sum;
+            // P row i over these columns (K-major SW128 blocks of 64 keys), zeros
+            // off the warp's span: the first half left of it, the second right of it
 #pragma unroll
-            for (int c = 0; c < Cfg::NCOL; c += 8)
-                sts128(aP + sw128_off(i, c_base + c),
-                       make_uint4(pack_bf16(sv[c], sv[c + 1]), pack_bf16(sv[c + 2], sv[c + 3]),
-                                  pack_bf16(sv[c + 4], sv[c + 5]), pack_bf16(sv[c + 6], sv[c + 7])));
-            for (int col = 0; col < c_base; col += 8) sts128(aP + sw128_off(i, col), make_uint4(0u, 0u, 0u, 0u));
-            for (int col = c_base + Cfg::NCOL; col < KW; col += 8)
-                sts128(aP + sw128_off(i, col), make_uint4(0u, 0u, 0u, 0u));
+            for (int c = 0; c < Cfg::H0; c += 8)
+                if (c < nh)
+                    sts128(aP + sw128_off(i, c0 + c),
+                           make_uint4(pack_bf16(sv[c], sv[c + 1]), pack_bf16(sv[c + 2], sv[c + 3]),
+                                      pack_bf16(sv[c + 4], sv[c + 5]), pack_bf16(sv[c + 6], sv[c + 7])));
+            if (hh == 0)
+                for (int col = 0; col < c_base; col += 8) sts128(aP + sw128_off(i, col), make_uint4(0u, 0u, 0u, 0u));
+            else
+                for (int col = c_base + Cfg::NCOL; col < KW; col += 8)
+                    sts128(aP + sw128_off(i, col), make_uint4(0u, 0u, 0u, 0u));
         }
         fence_proxy_async();
         tc_fence_before();
@@ -195,22 +215,24 @@ swa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             load_pending = true;
         }
 
-        // ---- epilogue: o = O / rowsum (bf16), lse
+        // ---- epilogue: o = O / rowsum (bf16; this thread's 32 of the 64 columns), lse
         {
             const int i = row;
-            float ov[Cfg::D];
+            constexpr int DH = Cfg::D / 2;
+            rowsum = red_s[i] + red_s[C + i];   // both halves, written before the barrier above
+            float ov[DH];
 #pragma unroll
-            for (int c = 0; c < Cfg::D; c += 16) tmem_ld16(tmem + lane_base + Cfg::COL_O + c, ov + c);
+            for (int c = 0; c < DH; c += 16) tmem_ld16(tmem + lane_base + Cfg::COL_O + hh * DH + c, ov + c);
             tmem_ld_wait();
             if (t0 + i < p.N) {
                 const float inv = 1.f / rowsum;
-                __nv_bfloat16 *orow = p.o + ((size_t)bh * p.N + t0 + i) * Cfg::D;
+                __nv_bfloat16 *orow = p.o + ((size_t)bh * p.N + t0 + i) * Cfg::D + hh * DH;
 #pragma unroll
-                for (int c = 0; c < Cfg::D; c += 8)
+                for (int c = 0; c < DH; c += 8)
                     *reinterpret_cast<uint4 *>(orow + c) =
                         make_uint4(pack_bf16(ov[c] * inv, ov[c + 1] * inv), pack_bf16(ov[c + 2] * inv, ov[c + 3] * inv),
                                    pack_bf16(ov[c + 4] * inv, ov[c + 5] * inv), pack_bf16(ov[c + 6] * inv, ov[c + 7] * inv));
-                if (p.lse) p.lse[(size_t)bh * p.N + t0 + i] = rowmax * p.scale + logf(rowsum);
+                if (p.lse && hh == 0) p.lse[(size_t)bh * p.N + t0 + i] = rowmax * p.scale + logf(rowsum);
             }
         }
         tc_fence_before();
