@@ -476,13 +476,13 @@ la_status backward_tc(const void *q, const void *k, const void *v, const void *d
     if (set_smem<bwd_dq_kernel>(Cfg::SMEM_ALLOC) != LA_OK || set_smem<bwd_dkdv_kernel>(Cfg::SMEM_ALLOC) != LA_OK ||
         set_smem<bwd_rstate_kernel>(Cfg::SMEM_ALLOC) != LA_OK)
         return LA_ERR_CUDA;
-    bwd_dq_kernel<<<BH * p.P, 128, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, p);
+    bwd_dq_kernel<<<BH * p.P, 256, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, p);
     if (launch_status() != LA_OK) return LA_ERR_CUDA;
     if (p.P > 1) {
         bwd_rstate_kernel<<<BH * p.P, 128, Cfg::SMEM_ALLOC, stream>>>(tq, tdo, p);
         if (launch_status() != LA_OK) return LA_ERR_CUDA;
     }
-    bwd_dkdv_kernel<<<BH * p.P, 128, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, p);
+    bwd_dkdv_kernel<<<BH * p.P, 256, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, p);
     return launch_status();
 }
 

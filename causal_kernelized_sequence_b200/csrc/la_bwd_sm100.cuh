@@ -60,7 +60,8 @@ struct BwdCfg128 {
     static constexpr int OFF_S = OFF_G + VG_TILE;
     static constexpr int OFF_SL = OFF_S + S_TILE;        // low bf16 part of the state (forward-order pass)
     static constexpr int OFF_BAR = OFF_SL + S_TILE;
-    static constexpr int SMEM_ALLOC = OFF_BAR + 128 + 1024;
+    static constexpr int OFF_RED = OFF_BAR + 128;        // forward-order pass: per-row partial sums of its two threads
+    static constexpr int SMEM_ALLOC = OFF_RED + 3 * 2 * C * 4 + 1024;
     static constexpr int TMEM_COLS = 512;
 };
 
@@ -102,6 +103,22 @@ __device__ __forceinline__ void phi_row_inplace(uint32_t tile, int row, bool zer
                      : make_uint4(elu1_bf16x2(r.x), elu1_bf16x2(r.y), elu1_bf16x2(r.z), elu1_bf16x2(r.w));
             sts128(tile + sw128_off(row, blk * 64 + cc * 8), r);
         }
+    }
+}
+
+// elu(x)+1 in place on the 64-column block `blk` of row `row` (one half of
+// phi_row_inplace, for two threads per row).
+__device__ __forceinline__ void phi_block_inplace(uint32_t tile, int row, bool zero, int blk)
+{
+    uint4 raw[8];
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) raw[cc] = lds128(tile + sw128_off(row, blk * 64 + cc * 8));
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) {
+        uint4 r = raw[cc];
+        r = zero ? make_uint4(0u, 0u, 0u, 0u)
+                 : make_uint4(elu1_bf16x2(r.x), elu1_bf16x2(r.y), elu1_bf16x2(r.z), elu1_bf16x2(r.w));
+        sts128(tile + sw128_off(row, blk * 64 + cc * 8), r);
     }
 }
 
@@ -147,10 +164,11 @@ __device__ __forceinline__ void snap_cols(uint32_t a_hi, uint32_t a_lo, int f, i
 // Row f (thread) of a state tile [F x NA] fp32 in TMEM (M = 128 layout) to its
 // bf16 snapshot(s).
 template <int F, int NA>
-__device__ __forceinline__ void snapshot_state(uint32_t tS_lane, uint8_t *snap, uint8_t *snap_lo, int f)
+__device__ __forceinline__ void snapshot_state(uint32_t tS_lane, uint8_t *snap, uint8_t *snap_lo, int f,
+                                               int c_lo = 0, int c_hi = NA)
 {
 #pragma unroll 1
-    for (int c0 = 0; c0 < NA; c0 += 16) {
+    for (int c0 = c_lo; c0 < c_hi; c0 += 16) {
         float v[16];
         tmem_ld16(tS_lane + c0, v);
         tmem_ld_wait();
@@ -238,6 +256,45 @@ __device__ __forceinline__ void phi_row_f16(uint32_t tile, int row, bool zero)
     }
 }
 
+// phi_row_f16 on the 64-column block `blk` only (two threads per row).
+__device__ __forceinline__ void phi_block_f16(uint32_t tile, int row, bool zero, int blk)
+{
+    uint4 raw[8];
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) raw[cc] = lds128(tile + sw128_off(row, blk * 64 + cc * 8));
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) {
+        const uint4 r = raw[cc];
+        sts128(tile + sw128_off(row, blk * 64 + cc * 8),
+               zero ? make_uint4(0u, 0u, 0u, 0u)
+                    : make_uint4(elu1_f16x2_from_bf16x2(r.x), elu1_f16x2_from_bf16x2(r.y),
+                                 elu1_f16x2_from_bf16x2(r.z), elu1_f16x2_from_bf16x2(r.w)));
+    }
+}
+
+// mask_pack_row_f16 for two threads per row: the 64 source columns from j0.
+// With `aliased` the packed columns may overlap source columns the other
+// thread has not read yet, so the block meets at a barrier between the loads
+// and the stores (every thread must then call this).
+template <typename Keep>
+__device__ __forceinline__ void mask_pack_half_f16(uint32_t src, uint32_t dst, int j0, bool aliased, Keep keep)
+{
+    float a[64];
+    tmem_ld32(src + j0, a);
+    tmem_ld32(src + j0 + 32, a + 32);
+    tmem_ld_wait();
+    if (aliased) {
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
+    uint32_t pk[32];
+#pragma unroll
+    for (int e = 0; e < 64; e += 2) pk[e / 2] = pack_f16(keep(j0 + e) ? a[e] : 0.f, keep(j0 + e + 1) ? a[e + 1] : 0.f);
+    tmem_st32(dst + j0 / 2, pk);
+    tmem_st_wait();
+}
+
 // Row r of a 16-column SW32 block of 128 rows: [first, 0, ..., 0] in fp16.
 __device__ __forceinline__ void write_first_f16(uint8_t *blk, int r, float first)
 {
@@ -282,6 +339,50 @@ __device__ __forceinline__ void mask_pack_row_f16(uint32_t src, uint32_t dst, Ke
     tmem_st_wait();
 }
 
+// mask_pack_row for two threads per row: this thread takes the 64 source
+// columns from j0 and writes 32 packed columns at dst + j0/2.  The packed
+// columns may alias source columns the other thread has not read yet, so the
+// whole block meets at a barrier between the loads and the stores (every
+// thread must call this).
+template <typename Keep>
+__device__ __forceinline__ void mask_pack_half(uint32_t src, uint32_t dst, int j0, Keep keep)
+{
+    float a[64];
+    tmem_ld32(src + j0, a);
+    tmem_ld32(src + j0 + 32, a + 32);
+    tmem_ld_wait();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    uint32_t pk[32];
+#pragma unroll
+    for (int e = 0; e < 64; e += 2) pk[e / 2] = pack_bf16(keep(j0 + e) ? a[e] : 0.f, keep(j0 + e + 1) ? a[e + 1] : 0.f);
+    tmem_st32(dst + j0 / 2, pk);
+    tmem_st_wait();
+}
+
+// mask_pack_row_hilo for two threads per row: the 64 source columns from j0
+// (destinations do not alias the source).
+template <typename Keep>
+__device__ __forceinline__ void mask_pack_half_hilo(uint32_t src, uint32_t dst_hi, uint32_t dst_lo, int j0, Keep keep)
+{
+    float a[64];
+    tmem_ld32(src + j0, a);
+    tmem_ld32(src + j0 + 32, a + 32);
+    tmem_ld_wait();
+    uint32_t hi[32], lo[32];
+#pragma unroll
+    for (int e = 0; e < 64; e += 2) {
+        const float x0 = keep(j0 + e) ? a[e] : 0.f, x1 = keep(j0 + e + 1) ? a[e + 1] : 0.f;
+        hi[e / 2] = pack_bf16(x0, x1);
+        lo[e / 2] = pack_bf16(x0 - __bfloat162float(__float2bfloat16_rn(x0)),
+                              x1 - __bfloat162float(__float2bfloat16_rn(x1)));
+    }
+    tmem_st32(dst_hi + j0 / 2, hi);
+    tmem_st32(dst_lo + j0 / 2, lo);
+    tmem_st_wait();
+}
+
 // Masked scores packed as bf16 hi (at dst_hi) and the bf16 remainder (at
 // dst_lo), 64 columns each.
 template <typename Keep>
@@ -317,7 +418,7 @@ __device__ __forceinline__ void mask_pack_row_hilo(uint32_t src, uint32_t dst_hi
 // it (relative error ~2/|phi - 1| x 2^-9 in dq); fp16 keeps 3 more.  V is
 // converted exactly; the state snapshot and G' keep an extra fp16 remainder
 // for the inter-chunk term, and dphi(q) is projected orthogonal to phi(q).
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(256, 1)
 bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
               const BwdParams p)
@@ -331,7 +432,11 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     uint64_t *mma_bar = tma_bar + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tma_bar + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tma_bar + 3);
-    const int tid = threadIdx.x, warp = tid >> 5;
+    // 256 threads: warps w and w + 4 share the TMEM lanes of rows 32 (w % 4) ..
+    // + 31 and split every per-row step by columns; row sums meet in red[]
+    const int tid = threadIdx.x, warp = tid >> 5, wq = warp & 3, hh = warp >> 2;
+    const int row = wq * 32 + (tid & 31);
+    float *red = reinterpret_cast<float *>(smem + Cfg::OFF_RED);   // [3][2][C]
     const int bh = blockIdx.x / p.P, seg = blockIdx.x % p.P;
     const int c_begin = seg * p.cps, c_end = min(p.nchunks, c_begin + p.cps);
     const int N = p.N;
@@ -347,34 +452,35 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         mbar_init_fence();
     }
     if (warp == 0) tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
-    write_first_f16(sV + (DV / 16) * Cfg::BLK, tid, 1.f);   // ones column of V_aug
+    if (hh == 0) write_first_f16(sV + (DV / 16) * Cfg::BLK, row, 1.f);   // ones column of V_aug
     __syncthreads();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t lane = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane = (uint32_t)(wq * 32) << 16;
+    const int na_lo = hh ? 80 : 0, na_hi = hh ? NA : 80;   // this thread's 16-column groups of S_aug
     // TMEM columns: [0,128) scores -> P (first 64) and dP (second 64);
     // [128,272) O_aug, then dA and dphi(Q); [272,416) state S_aug (M = 128);
     // [416,488) G'_lo, the bf16 remainder of G' (A operand, packed pairs).
     const uint32_t tA = tmem, tX = tmem + 128, tS = tmem + 272, tGL = tmem + 416;
 
     // ---- state entering the segment: sum of the earlier segments' increments
-    for (int c0 = 0; c0 < NA; c0 += 16) {
+    for (int c0 = na_lo; c0 < na_hi; c0 += 16) {
         float v[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) v[e] = 0.f;
         for (int s2 = 0; s2 < seg; ++s2) {
-            const float *src = p.ws_s + ((size_t)(bh * p.P + s2) * F + tid) * NA + c0;
+            const float *src = p.ws_s + ((size_t)(bh * p.P + s2) * F + row) * NA + c0;
 #pragma unroll
             for (int e = 0; e < 16; ++e) v[e] += src[e];
         }
         tmem_st16(tS + lane + c0, v);
-        snap_cols_f16<F>(aS, aSL, tid, c0, v);
+        snap_cols_f16<F>(aS, aSL, row, c0, v);
     }
     tmem_st_wait();
     full_sync();
 
     uint32_t tph = 0, mph = 0;
     for (int chunk = c_begin; chunk < c_end && !*abort_flag; ++chunk) {
-        const int t0 = chunk * C, i = tid;
+        const int t0 = chunk * C, i = row;
         const bool valid = t0 + i < N;
         if (tid == 0) {
             mbar_arrive_expect_tx(tma_bar, 2 * Cfg::QK_TILE + 2 * C * DV * 2);
@@ -390,10 +496,10 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (!mbar_wait(tma_bar, tph)) *abort_flag = 1;
         tph ^= 1u;
         // fp16 operands: phi(Q), phi(K) in place; V converted in place
-        phi_row_f16(aQ, i, false);
-        phi_row_f16(aK, i, !valid);
+        phi_block_f16(aQ, i, false, hh);
+        phi_block_f16(aK, i, !valid, hh);
 #pragma unroll
-        for (int c0 = 0; c0 < DV; c0 += 8) {
+        for (int c0 = hh * (DV / 2); c0 < (hh + 1) * (DV / 2); c0 += 8) {
             const uint32_t a = aV + sw32_off(i, c0, C);
             const uint4 r = lds128(a);
             sts128(a, make_uint4(bf16x2_to_f16x2(r.x), bf16x2_to_f16x2(r.y), bf16x2_to_f16x2(r.z), bf16x2_to_f16x2(r.w)));
@@ -414,7 +520,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
         mph ^= 1u;
         tc_fence_after();
-        mask_pack_row_f16(tA + lane, tA + lane, [&](int j) { return j <= i; });
+        mask_pack_half_f16(tA + lane, tA + lane, 64 * hh, true, [&](int j) { return j <= i; });
         full_sync();
 
         // O_aug = P V_aug + phi(Q) S_aug
@@ -448,9 +554,9 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const float den = dv16[0];
             den_row = den;
             const float inv = valid ? 1.f / den : 0.f;
-            float gy = 0.f;   // dO . y
-#pragma unroll 1
-            for (int half = 0; half < DV; half += 64) {
+            float gy = 0.f;   // dO . y over this thread's half of the columns
+            {
+                const int half = 64 * hh;
                 uint32_t glo[32];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
@@ -475,20 +581,23 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 }
                 tmem_st32(tGL + lane + half / 2, glo);
             }
+            red[hh * C + i] = gy;
+            __syncthreads();
+            gy = red[i] + red[C + i];
             const float ddu = valid ? -gy : 0.f;   // den * dden
-            write_first_f16(sG + (DV / 16) * Cfg::BLK, i, ddu);
-            {
+            if (hh == 0) {
+                write_first_f16(sG + (DV / 16) * Cfg::BLK, i, ddu);
                 uint32_t tail[8];
                 tail[0] = pack_f16(f16_rem(ddu), 0.f);
 #pragma unroll
                 for (int e = 1; e < 8; ++e) tail[e] = 0u;
                 tmem_st8(tGL + lane + DV / 2, tail);
+                if (valid) {
+                    p.dd[((size_t)bh * N + t0 + i) * 2] = den;
+                    p.dd[((size_t)bh * N + t0 + i) * 2 + 1] = ddu * inv;
+                }
             }
             tmem_st_wait();
-            if (valid) {
-                p.dd[((size_t)bh * N + t0 + i) * 2] = den;
-                p.dd[((size_t)bh * N + t0 + i) * 2 + 1] = ddu * inv;
-            }
         }
         full_sync();
 
@@ -503,7 +612,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
         mph ^= 1u;
         tc_fence_after();
-        mask_pack_row_f16(tX + lane, tA + lane + 64, [&](int j) { return j <= i; });
+        mask_pack_half_f16(tX + lane, tA + lane + 64, 64 * hh, false, [&](int j) { return j <= i; });
         full_sync();
 
         // dphi(Q) = dP phi(K) + G' S_aug^T ;  then S_aug += phi(K)^T V_aug
@@ -541,7 +650,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             __nv_bfloat16 *dqrow = reinterpret_cast<__nv_bfloat16 *>(p.dq) + ((size_t)bh * N + t0 + i) * D;
             float sd = 0.f, sn = 0.f;
 #pragma unroll 1
-            for (int c0 = 0; c0 < F; c0 += 16) {
+            for (int c0 = hh * (F / 2); c0 < (hh + 1) * (F / 2); c0 += 16) {
                 float g[16], ph[16];
                 tmem_ld16(tX + lane + c0, g);
                 tmem_ld_wait();
@@ -553,10 +662,15 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     sn = fmaf(ph[e], ph[e], sn);
                 }
             }
+            red[2 * C + hh * C + i] = sd;
+            red[4 * C + hh * C + i] = sn;
+            __syncthreads();
+            sd = red[2 * C + i] + red[3 * C + i];
+            sn = red[4 * C + i] + red[5 * C + i];
             const float proj = sd / sn;
             const float rden = valid ? 1.f / den_row : 0.f;
 #pragma unroll 1
-            for (int c0 = 0; c0 < F; c0 += 16) {
+            for (int c0 = hh * (F / 2); c0 < (hh + 1) * (F / 2); c0 += 16) {
                 float g[16], ph[16];
                 tmem_ld16(tX + lane + c0, g);
                 tmem_ld_wait();
@@ -574,11 +688,11 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             if (chunk + 1 < c_end) {
 #pragma unroll 1
-                for (int c0 = 0; c0 < NA; c0 += 16) {
+                for (int c0 = na_lo; c0 < na_hi; c0 += 16) {
                     float v[16];
                     tmem_ld16(tS + lane + c0, v);
                     tmem_ld_wait();
-                    snap_cols_f16<F>(aS, aSL, tid, c0, v);
+                    snap_cols_f16<F>(aS, aSL, row, c0, v);
                 }
             }
         }
@@ -758,8 +872,10 @@ bwd_rstate_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 }
 
 // ---------------------------------------------------------------------------
-// Reverse-order pass: dk and dv.
-__global__ void __launch_bounds__(128, 1)
+// Reverse-order pass: dk and dv.  256 threads: warps w and w + 4 share the
+// TMEM lanes of rows 32 (w % 4) .. + 31, and every per-row step is split
+// between them by columns (the first half of the columns to warps 0-3).
+__global__ void __launch_bounds__(256, 1)
 bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                 const BwdParams p)
@@ -773,7 +889,8 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint64_t *mma_bar = tma_bar + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tma_bar + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tma_bar + 3);
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, wq = warp & 3, hh = warp >> 2;
+    const int row = wq * 32 + (tid & 31);   // this thread's token row / TMEM lane
     const int bh = blockIdx.x / p.P, seg = blockIdx.x % p.P;
     const int c_begin = seg * p.cps, c_end = min(p.nchunks, c_begin + p.cps);
     const int N = p.N;
@@ -788,29 +905,30 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_init_fence();
     }
     if (warp == 0) tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
-    write_ones_block(sV + (DV / 16) * Cfg::BLK, tid);
+    if (hh == 0) write_ones_block(sV + (DV / 16) * Cfg::BLK, row);
     __syncthreads();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t lane = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane = (uint32_t)(wq * 32) << 16;
+    const int na_lo = hh ? 80 : 0, na_hi = hh ? NA : 80;   // this thread's 16-column groups of R_aug
     // TMEM: [0,64) P^T, [64,128) dP^T (packed); [0,128) holds A^T first;
     // [128,256) dA^T, then dV, then dphi(K); [256,400) R_aug (M = 128);
     // [400,464) the bf16 remainder of dP^T.
     const uint32_t tA = tmem, tX = tmem + 128, tR = tmem + 256, tPL = tmem + 400;
 
     // ---- R entering the segment: sum of the later segments' increments
-    for (int c0 = 0; c0 < NA; c0 += 16) {
+    for (int c0 = na_lo; c0 < na_hi; c0 += 16) {
         float v[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) v[e] = 0.f;
         for (int s2 = seg + 1; s2 < p.P; ++s2) {
-            const float *src = p.ws_r + ((size_t)(bh * p.P + s2) * F + tid) * NA + c0;
+            const float *src = p.ws_r + ((size_t)(bh * p.P + s2) * F + row) * NA + c0;
 #pragma unroll
             for (int e = 0; e < 16; ++e) v[e] += src[e];
         }
         tmem_st16(tR + lane + c0, v);
-        sts128(aR + sw32_off(tid, c0, F), make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
+        sts128(aR + sw32_off(row, c0, F), make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
                                                      pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7])));
-        sts128(aR + sw32_off(tid, c0 + 8, F), make_uint4(pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]),
+        sts128(aR + sw32_off(row, c0 + 8, F), make_uint4(pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]),
                                                          pack_bf16(v[12], v[13]), pack_bf16(v[14], v[15])));
     }
     tmem_st_wait();
@@ -818,7 +936,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     uint32_t tph = 0, mph = 0;
     for (int chunk = c_end - 1; chunk >= c_begin && !*abort_flag; --chunk) {
-        const int t0 = chunk * C, j = tid;
+        const int t0 = chunk * C, j = row;
         const bool valid = t0 + j < N;
         if (tid == 0) {
             mbar_arrive_expect_tx(tma_bar, 2 * Cfg::QK_TILE + 2 * C * DV * 2);
@@ -833,8 +951,8 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         if (!mbar_wait(tma_bar, tph)) *abort_flag = 1;
         tph ^= 1u;
-        phi_row_inplace(aQ, j, false);
-        phi_row_inplace(aK, j, !valid);
+        phi_block_inplace(aQ, j, false, hh);
+        phi_block_inplace(aK, j, !valid, hh);
         {
             // G' row j (this thread's token as a query): [dO/den | dden] as bf16
             // plus its bf16 remainder (dA^T below uses both)
@@ -842,7 +960,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const float dden = valid ? p.dd[((size_t)bh * N + t0 + j) * 2 + 1] : 0.f;
             const float inv = valid ? 1.f / den : 0.f;
 #pragma unroll 1
-            for (int c0 = 0; c0 < DV; c0 += 8) {
+            for (int c0 = hh * (DV / 2); c0 < (hh + 1) * (DV / 2); c0 += 8) {
                 float go[8];
                 const uint32_t a = aG + sw32_off(j, c0, C);
                 unpack8(lds128(a), go);
@@ -856,8 +974,10 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 sts128(aGL + sw32_off(j, c0, C), make_uint4(pack_bf16(r[0], r[1]), pack_bf16(r[2], r[3]),
                                                             pack_bf16(r[4], r[5]), pack_bf16(r[6], r[7])));
             }
-            write_dden(sG + (DV / 16) * Cfg::BLK, j, dden);
-            write_dden(sGL + (DV / 16) * Cfg::BLK, j, dden - __bfloat162float(__float2bfloat16_rn(dden)));
+            if (hh == 0) {
+                write_dden(sG + (DV / 16) * Cfg::BLK, j, dden);
+                write_dden(sGL + (DV / 16) * Cfg::BLK, j, dden - __bfloat162float(__float2bfloat16_rn(dden)));
+            }
         }
         full_sync();
         if (*abort_flag) break;
@@ -883,8 +1003,8 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mph ^= 1u;
         tc_fence_after();
         // row j keeps the queries i >= j
-        mask_pack_row(tA + lane, tA + lane, [&](int i) { return i >= j; });
-        mask_pack_row_hilo(tX + lane, tA + lane + 64, tPL + lane, [&](int i) { return i >= j; });
+        mask_pack_half(tA + lane, tA + lane, 64 * hh, [&](int i) { return i >= j; });
+        mask_pack_half_hilo(tX + lane, tA + lane + 64, tPL + lane, 64 * hh, [&](int i) { return i >= j; });
         full_sync();
 
         // dV = P^T G + phi(K) R
@@ -907,7 +1027,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         {
             __nv_bfloat16 *dvrow = reinterpret_cast<__nv_bfloat16 *>(p.dv) + ((size_t)bh * N + t0 + j) * DV;
 #pragma unroll 1
-            for (int c0 = 0; c0 < DV; c0 += 16) {
+            for (int c0 = hh * (DV / 2); c0 < (hh + 1) * (DV / 2); c0 += 16) {
                 float g[16];
                 tmem_ld16(tX + lane + c0, g);
                 tmem_ld_wait();
@@ -946,7 +1066,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         {
             __nv_bfloat16 *dkrow = reinterpret_cast<__nv_bfloat16 *>(p.dk) + ((size_t)bh * N + t0 + j) * D;
 #pragma unroll 1
-            for (int c0 = 0; c0 < F; c0 += 16) {
+            for (int c0 = hh * (F / 2); c0 < (hh + 1) * (F / 2); c0 += 16) {
                 float g[16], ph[16];
                 tmem_ld16(tX + lane + c0, g);
                 tmem_ld_wait();
@@ -961,7 +1081,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                             pack_bf16(g[e + 4] * fminf(ph[e + 4], 1.f), g[e + 5] * fminf(ph[e + 5], 1.f)),
                             pack_bf16(g[e + 6] * fminf(ph[e + 6], 1.f), g[e + 7] * fminf(ph[e + 7], 1.f)));
             }
-            if (chunk > c_begin) snapshot_state<F, NA>(tR + lane, sR, nullptr, tid);
+            if (chunk > c_begin) snapshot_state<F, NA>(tR + lane, sR, nullptr, row, na_lo, na_hi);
         }
         full_sync();
     }
