@@ -724,29 +724,39 @@ bwd_sstate_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     if (seg == p.P - 1) return;   // the last segment's increment is never read
     const int c_begin = seg * p.cps, c_end = min(p.nchunks, c_begin + p.cps);
     const int N = p.N;
-    uint8_t *sK = smem + Cfg::OFF_K, *sV = smem + Cfg::OFF_V;
-    const uint32_t aK = smem_addr(sK), aV = smem_addr(sV);
+    // two stages of [K | V_aug]: the Q and dO buffers, unused here, hold the second
+    uint8_t *sKs[2] = {smem + Cfg::OFF_K, smem + Cfg::OFF_Q}, *sVs[2] = {smem + Cfg::OFF_V, smem + Cfg::OFF_G};
+    uint64_t *tma_b[2] = {tma_bar, tma_bar + 4};
     if (tid == 0) {
-        mbar_init(tma_bar, 1);
+        mbar_init(tma_b[0], 1);
+        mbar_init(tma_b[1], 1);
         mbar_init(mma_bar, 1);
         *abort_flag = 0;
         mbar_init_fence();
     }
     if (warp == 0) tmem_alloc(tmem_slot, 256);
-    write_first_f16(sV + (DV / 16) * Cfg::BLK, tid, 1.f);
+    write_first_f16(sVs[0] + (DV / 16) * Cfg::BLK, tid, 1.f);
+    write_first_f16(sVs[1] + (DV / 16) * Cfg::BLK, tid, 1.f);
     __syncthreads();
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane = (uint32_t)(warp * 32) << 16;
-    uint32_t tph = 0, mph = 0;
+    // chunk c uses stage (c - c_begin) & 1; its loads go out when chunk c - 2's
+    // MMA has finished with the stage, a whole chunk ahead of their use
+    auto issue = [&](int chunk) {
+        const int st = (chunk - c_begin) & 1, t0 = chunk * C;
+        mbar_arrive_expect_tx(tma_b[st], Cfg::QK_TILE + C * DV * 2);
+        for (int x = 0; x < D; x += 64) tma_load_3d(sKs[st] + (x / 64) * C * 128, &tm_k, tma_b[st], x, t0, bh);
+        for (int x = 0; x < DV; x += 16) tma_load_3d(sVs[st] + (x / 16) * Cfg::BLK, &tm_v, tma_b[st], x, t0, bh);
+    };
+    int issued = c_begin, waited = c_begin;   // thread 0: chunks whose loads went out / were waited for
+    if (tid == 0)
+        for (; issued < c_end && issued < c_begin + 2; ++issued) issue(issued);
+    uint32_t mph = 0;
     for (int chunk = c_begin; chunk < c_end && !*abort_flag; ++chunk) {
-        const int t0 = chunk * C, i = tid;
-        if (tid == 0) {
-            mbar_arrive_expect_tx(tma_bar, Cfg::QK_TILE + C * DV * 2);
-            for (int x = 0; x < D; x += 64) tma_load_3d(sK + (x / 64) * C * 128, &tm_k, tma_bar, x, t0, bh);
-            for (int x = 0; x < DV; x += 16) tma_load_3d(sV + (x / 16) * Cfg::BLK, &tm_v, tma_bar, x, t0, bh);
-        }
-        if (!mbar_wait(tma_bar, tph)) *abort_flag = 1;
-        tph ^= 1u;
+        const int t0 = chunk * C, i = tid, st = (chunk - c_begin) & 1;
+        const uint32_t aK = smem_addr(sKs[st]), aV = smem_addr(sVs[st]);
+        if (!mbar_wait(tma_b[st], (uint32_t)((chunk - c_begin) >> 1) & 1u)) *abort_flag = 1;
+        waited = chunk + 1;
         phi_row_f16(aK, i, t0 + i >= N);
 #pragma unroll
         for (int c0 = 0; c0 < DV; c0 += 8) {
@@ -765,8 +775,13 @@ bwd_sstate_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         }
         if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
         mph ^= 1u;
+        if (tid == 0 && !*abort_flag && issued < c_end) issue(issued++);
         full_sync();
     }
+    // after an early exit, let this block's own copies land (bounded)
+    if (tid == 0 && *abort_flag)
+        for (int c = waited; c < issued; ++c)
+            mbar_wait(tma_b[(c - c_begin) & 1], (uint32_t)((c - c_begin) >> 1) & 1u, 100000000ull);
     if (!*abort_flag) {
         float *dst = p.ws_s + ((size_t)(bh * p.P + seg) * F + tid) * NA;
 #pragma unroll 1
@@ -803,10 +818,12 @@ bwd_rstate_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (seg == 0) return;   // the first segment's increment is never read
     const int c_begin = seg * p.cps, c_end = min(p.nchunks, c_begin + p.cps);
     const int N = p.N;
-    uint8_t *sQ = smem + Cfg::OFF_Q, *sG = smem + Cfg::OFF_G;
-    const uint32_t aQ = smem_addr(sQ), aG = smem_addr(sG);
+    // two stages of [Q | G'_aug]: the K and V buffers, unused here, hold the second
+    uint8_t *sQs[2] = {smem + Cfg::OFF_Q, smem + Cfg::OFF_K}, *sGs[2] = {smem + Cfg::OFF_G, smem + Cfg::OFF_V};
+    uint64_t *tma_b[2] = {tma_bar, tma_bar + 4};
     if (tid == 0) {
-        mbar_init(tma_bar, 1);
+        mbar_init(tma_b[0], 1);
+        mbar_init(tma_b[1], 1);
         mbar_init(mma_bar, 1);
         *abort_flag = 0;
         mbar_init_fence();
@@ -815,17 +832,25 @@ bwd_rstate_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     __syncthreads();
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane = (uint32_t)(warp * 32) << 16;
-    uint32_t tph = 0, mph = 0;
+    // chunk c uses stage (c - c_begin) & 1; its loads go out when chunk c - 2's
+    // MMA has finished with the stage
+    auto issue = [&](int chunk) {
+        const int st = (chunk - c_begin) & 1, t0 = chunk * C;
+        mbar_arrive_expect_tx(tma_b[st], Cfg::QK_TILE + C * DV * 2);
+        for (int x = 0; x < D; x += 64) tma_load_3d(sQs[st] + (x / 64) * C * 128, &tm_q, tma_b[st], x, t0, bh);
+        for (int x = 0; x < DV; x += 16) tma_load_3d(sGs[st] + (x / 16) * Cfg::BLK, &tm_do, tma_b[st], x, t0, bh);
+    };
+    int issued = c_begin, waited = c_begin;
+    if (tid == 0)
+        for (; issued < c_end && issued < c_begin + 2; ++issued) issue(issued);
+    uint32_t mph = 0;
     for (int chunk = c_begin; chunk < c_end && !*abort_flag; ++chunk) {
-        const int t0 = chunk * C, i = tid;
+        const int t0 = chunk * C, i = tid, st = (chunk - c_begin) & 1;
         const bool valid = t0 + i < N;
-        if (tid == 0) {
-            mbar_arrive_expect_tx(tma_bar, Cfg::QK_TILE + C * DV * 2);
-            for (int x = 0; x < D; x += 64) tma_load_3d(sQ + (x / 64) * C * 128, &tm_q, tma_bar, x, t0, bh);
-            for (int x = 0; x < DV; x += 16) tma_load_3d(sG + (x / 16) * Cfg::BLK, &tm_do, tma_bar, x, t0, bh);
-        }
-        if (!mbar_wait(tma_bar, tph)) *abort_flag = 1;
-        tph ^= 1u;
+        uint8_t *sG = sGs[st];
+        const uint32_t aQ = smem_addr(sQs[st]), aG = smem_addr(sG);
+        if (!mbar_wait(tma_b[st], (uint32_t)((chunk - c_begin) >> 1) & 1u)) *abort_flag = 1;
+        waited = chunk + 1;
         phi_row_inplace(aQ, i, false);
         {
             const float den = valid ? p.dd[((size_t)bh * N + t0 + i) * 2] : 1.f;
@@ -854,8 +879,12 @@ bwd_rstate_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
         mph ^= 1u;
+        if (tid == 0 && !*abort_flag && issued < c_end) issue(issued++);
         full_sync();
     }
+    if (tid == 0 && *abort_flag)
+        for (int c = waited; c < issued; ++c)
+            mbar_wait(tma_b[(c - c_begin) & 1], (uint32_t)((c - c_begin) >> 1) & 1u, 100000000ull);
     if (!*abort_flag) {
         float *dst = p.ws_r + ((size_t)(bh * p.P + seg) * F + tid) * NA;
 #pragma unroll 1
