@@ -216,12 +216,16 @@ LA_API la_status la_forward_varlen(const void *q, const void *k, const void *v, 
  *              g_t <= 0 (a_t in [0, 1]); -inf forgets everything before t.
  *              Positive g is computed by the same formulas but can overflow.
  *   s_in, z_in nullable (both or neither): the state entering each slice.
+ *              (For a Taylor start state, the difference between the paired
+ *              rows (a, b) and (b, a) decays with the gates like the rest of
+ *              the state.)
  * The other arguments, layouts and errors are those of la_forward_from_state.
  * The bf16 shapes with a tensor-core forward run on it (long sequences split
  * into segments whose increments and summed gates go through the workspace,
  * la_forward_decay_workspace_bytes); there a gate below e^-80 counts as
- * e^-80, which is zero next to any surviving term in fp32.  Every other combination runs on the
- * exact fp32 CUDA-core forward, which takes -inf as it is. */
+ * e^-80, which is zero next to any surviving term in fp32.  Every other
+ * combination runs on the exact fp32 CUDA-core forward, which takes -inf as
+ * it is. */
 LA_API size_t la_forward_decay_workspace_bytes(int B, int H, int N, int dqk, int dv, int fmap, int dtype);
 
 LA_API la_status la_forward_decay(const void *q, const void *k, const void *v, const float *log_decay,
@@ -265,7 +269,10 @@ LA_API la_status la_decode_step_decay(const void *q, const void *k, const void *
  *   window  w >= 1 (up to 1024).  bf16 with dqk = dv = 64 and w a multiple of
  *   16 up to 128 (Knowl 4: widths that are multiples of 16, generally no
  *   larger than 128) runs on the tensor cores; every other combination on an
- *   exact fp32 CUDA-core kernel.  Errors as for la_forward. */
+ *   exact fp32 CUDA-core kernel.
+ * Errors: LA_ERR_INVALID_ARG for a size below 1, an unknown dtype or more
+ * than 2^31 elements in one tensor; LA_ERR_UNSUPPORTED for dqk or dv above
+ * 128 or w above 1024.  The cache and decode calls below check the same. */
 LA_API la_status la_swa_forward(const void *q, const void *k, const void *v, void *o, float *lse_out,
                                 int B, int H, int N, int dqk, int dv, int window, int dtype,
                                 void *stream);
@@ -372,7 +379,9 @@ LA_API la_status la_feature_map(const void *x, void *phi, int64_t rows, int dqk,
  * N = max_seqlen), 4 = la_forward_decay.  Writes a comma-separated list of
  * kernel names (truncated to buflen-1 characters, NUL-terminated) to buf
  * when buf is non-NULL, and returns the number of kernel launches the call
- * makes, or -1 for arguments the call itself would reject. */
+ * makes, or -1 for arguments the call itself would reject.  The gated
+ * calls outside this list launch fixed kernels: la_decode_step_decay the
+ * one op 2 reports for its shape, la_backward_decay one bwd_simt_kernel. */
 LA_API int la_kernel_plan(int op, int B, int H, int N, int dqk, int dv, int fmap, int dtype,
                           char *buf, size_t buflen);
 
