@@ -38,3 +38,57 @@ def test_cpu_tensors_rejected(call):
     la.load_library()
     with pytest.raises(ValueError, match="CUDA"):
         call()
+
+
+def _header_signatures():
+    """{name: (return kind, [parameter kinds])} of every LA_API declaration in
+    include/la.h, each kind one of ptr, int, size_t, int64, uint."""
+    import os
+    import re
+    src = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "la.h")).read()
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+
+    def kind(decl):
+        decl = " ".join(decl.split())
+        if "*" in decl:
+            return "ptr"
+        for word, k in (("size_t", "size_t"), ("int64_t", "int64"), ("unsigned int", "uint"),
+                        ("la_status", "int"), ("int", "int")):
+            if re.search(r"\b" + word + r"\b", decl):
+                return k
+        raise AssertionError(f"unclassified declaration {decl!r}")
+
+    sigs = {}
+    for m in re.finditer(r"\bLA_API\s+([^;(]*?)\b(la_\w+)\s*\(([^)]*)\)\s*;", src):
+        ret, name, params = m.group(1), m.group(2), m.group(3).strip()
+        plist = [] if params in ("", "void") else [kind(p) for p in params.split(",")]
+        sigs[name] = (kind(ret + " x"), plist)
+    return sigs
+
+
+def _ctypes_kind(t):
+    import ctypes
+    if t in (ctypes.c_void_p, ctypes.c_char_p):
+        return "ptr"
+    table = {ctypes.c_int: "int", ctypes.c_size_t: "size_t", ctypes.c_int64: "int64", ctypes.c_uint: "uint"}
+    return table[t]
+
+
+def test_binding_signatures_match_header(monkeypatch):
+    # The ctypes declarations in the binding must agree with include/la.h
+    # argument by argument: a wrong width or a missing argument is not an
+    # error ctypes can see, the call would just pass garbage.
+    from causal_kernelized_sequence_b200 import build
+    build.build()
+    monkeypatch.setattr(la, "_lib", None)   # a fresh CDLL with only the binding's own declarations
+    lib = la.load_library()
+    sigs = _header_signatures()
+    assert len(sigs) >= 25
+    for name, (ret, params) in sigs.items():
+        fn = getattr(lib, name)
+        assert _ctypes_kind(fn.restype) == ret, name
+        if params:
+            assert fn.argtypes is not None, f"{name}: no argtypes"
+            assert [_ctypes_kind(t) for t in fn.argtypes] == params, name
+        else:
+            assert not fn.argtypes, name
