@@ -106,7 +106,9 @@ struct FwdParams {
     float inv_c1, inv_c2;       // Taylor: 1/d'^(1/4), 1/(sqrt(2) sqrt(d'))
     float k1, k2;               // Taylor closed form: 1/sqrt(d'), 1/(2 d')
     // Gated form (nullable): log forget gate g_t per token, at the token's row
-    // (row0 + t).  Needs P == 1: segments would have to carry their decay.
+    // (row0 + t).  With P > 1 the segment-state launch also writes each
+    // segment's summed gate after the increments in ws, and a segment starts
+    // from the increments before it, each decayed by the gates after it.
     const float *logdecay;
 };
 
