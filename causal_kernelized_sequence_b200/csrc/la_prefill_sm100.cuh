@@ -10,10 +10,13 @@
 // (DV + 16 columns), so S_aug = [S | z] and one accumulator row holds both
 // numerator and denominator, rounded identically.
 //
-// Per chunk (one CTA = one 128-thread warpgroup; thread i <-> token i <->
-// TMEM lane i):
+// Per chunk (one CTA of 256 threads; token i <-> TMEM lane i, whose row two
+// threads share, warps w and w + 4 each taking half of its columns):
 //   TMA     Q_c, K_c (SW128, or SW32 for d'=16) and V_c (SW32) into a
-//           2-stage ring; out-of-range rows of a ragged tail are zero-filled.
+//           2-stage ring (one stage for d = 128).  Rows past the slice's
+//           end read as zeros (fixed length) or hold the next packed
+//           sequence's tokens; either way they are kept out of the state
+//           and out of every stored row.
 //   phi     elu(x)+1 applied in place to the Q/K tiles; for the Taylor map
 //           the symmetric second-order features (1 + 16 + 136 = 153, padded
 //           to 160) are written to separate phi tiles.  phi(q).phi(k) equals
@@ -21,8 +24,11 @@
 //           map.  The state at the boundary is either expanded back to 273
 //           rows or, for the folded map, is these 153 rows as they are.
 //   MMA1    A = phi(Q_c) phi(K_c)^T      (Taylor: Q_c K_c^T, then the closed
-//           form 1 + s/sqrt(d') + s^2/(2d') in the mask pass)   -> TMEM
-//   MMA3    S_aug += phi(K_c)^T V_aug   (feature rows in TMEM lanes)
+//           form 1 + s/sqrt(d') + s^2/(2d') in the mask pass)   -> TMEM,
+//           with a commit of its own so the mask pass need not wait for MMA3
+//   MMA3    S_aug += phi(K_c)^T V_aug   (feature rows in TMEM lanes); issued
+//           right after MMA1, or with MMA2 in the gated form, whose phi(K)
+//           rows are first scaled by their decay to the chunk's end
 //   mask    causal mask j <= i, bf16 -> P tile in shared memory
 //   MMA2    O_aug = P V_aug + phi(Q_c) S_snap   (S_snap = bf16 copy of the
 //           state entering the chunk)                             -> TMEM
