@@ -35,9 +35,12 @@
 // The reverse pass uses bf16 operands, with P^T and G' each split into a
 // bf16 head and a bf16 remainder on the products that carry dk.
 //
-// These kernels use one 128-thread warpgroup per block (thread i <-> token or
-// feature row i <-> TMEM lane i) and process a chunk's steps in order; every
-// mbarrier wait is bounded.
+// Token or feature row i <-> TMEM lane i.  bwd_dq_kernel and bwd_dkdv_kernel
+// run 256 threads: warps w and w + 4 share the lanes of one 32-row quadrant
+// and split every per-row step by columns, exchanging row reductions through
+// shared memory.  bwd_sstate_kernel and bwd_rstate_kernel run 128 threads, one
+// per row, and load the next chunk while the current one is summed.  Each
+// block takes a chunk's steps in order; every mbarrier wait is bounded.
 #pragma once
 
 #include "la_device.cuh"

@@ -14,6 +14,13 @@
 //     forward-order pass for dq, reverse-order pass of R, r for dk, dv.
 //   decode   (Knowl 3 recurrent form): S += phi(k) v^T, z += phi(k),
 //     y = phi(q) S / phi(q).z on the updated state.
+// The forward also takes a start state, packed sequences (a block per
+// (sequence, head) of a [H, T, *] batch cut by cu_seqlens) and the gated form
+// S_t = exp(g_t) S_{t-1} + phi(k_t) v_t^T.  Gated, every decay factor is the
+// exponential of a plain sum of gates (a prefix, a suffix or a pair range),
+// never a difference of prefix sums, so g = -inf gives exact zeros and no
+// inf - inf.  The gated backward adds the gate gradient
+// dL/dg_l = -sum_{j>=l} phi(k_j) . dL/dphi(k_j), summed in double.
 #pragma once
 
 #include "la_device.cuh"
