@@ -605,3 +605,26 @@ def test_max_rel_l2_metric(orc):
     ref = np.ones((2, 3, 4, 5))
     x = ref.copy(); x[1, 2] *= 1.01
     assert orc.max_rel_l2(x, ref) == pytest.approx(0.01, rel=1e-12)
+
+
+# ------------------------------------------------------------ full-size inputs
+
+@pytest.mark.parametrize("name", ["elu_bf16_fwd", "taylor_bf16_fwd", "elu_bf16_train"])
+def test_full_size_recurrence_matches_brute_rows(orc, name):
+    # The full-size GPU parity tests compare against the recurrent oracle.  On
+    # the same full-size inputs, brute force (the masked form, a different
+    # algorithm) at 64 random rows of every (b, h) slice gives the same outputs
+    # and denominators, so the recurrence carries its state correctly over
+    # thousands of tokens.
+    import workloads as W
+    w = W.BY_NAME[name]
+    q, k, v, _ = W.make_inputs(w)
+    o, den, _, _ = orc.forward_recurrent(w.fmap, q, k, v)
+    B, H, N = q.shape[0], q.shape[1], q.shape[2]
+    g = np.random.default_rng(11)
+    for b in range(B):
+        for h in range(H):
+            rows = np.sort(g.choice(N, 64, replace=False))
+            ob, db = orc.forward_rows(w.fmap, q[b, h], k[b, h], v[b, h], rows)
+            np.testing.assert_allclose(ob, o[b, h, rows], rtol=1e-11, atol=1e-12 * np.abs(ob).max())
+            np.testing.assert_allclose(db, den[b, h, rows], rtol=1e-12)
