@@ -452,20 +452,25 @@ def timed(run, steps, warmup, dist_on, device_index, graph_len=None):
     return ms / steps, clk.summary()
 
 
-def e2e_prefill(w, dev, steps, warmup, dist_on=False, rank=0):
-    """Same metric through the public API with host buffers: pinned host q,k,v
-    copied in and o copied out inside the timed region, every step.  Returns
-    (ms per step, max over ranks; h2d bytes; d2h bytes)."""
+def _e2e_buffers(w, dev, rank, nsets):
+    """Pinned host q, k, v (the step's inputs) and o (its result), and `nsets`
+    device buffer sets plus the forward's workspace."""
     import causal_kernelized_sequence_b200 as la
     g = torch.Generator()
     g.manual_seed(replica_seed(w, rank))
     mk = lambda d: (torch.randn(w.B, w.H, w.N, d, generator=g) * w.scale).to(w.torch_dtype).pin_memory()
     hq, hk, hv = mk(w.dqk), mk(w.dqk), mk(w.dv)
     ho = torch.empty(w.B, w.H, w.N, w.dv, dtype=w.torch_dtype).pin_memory()
-    dq_, dk_, dv_ = (torch.empty(t.shape, dtype=t.dtype, device=dev) for t in (hq, hk, hv))
-    do_ = torch.empty(ho.shape, dtype=ho.dtype, device=dev)
+    sets = [tuple(torch.empty(t.shape, dtype=t.dtype, device=dev) for t in (hq, hk, hv, ho)) for _ in range(nsets)]
     wsb = la.la_forward_workspace_bytes(w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype)
     ws = torch.empty(wsb, dtype=torch.uint8, device=dev) if wsb else None
+    return (hq, hk, hv, ho), sets, ws
+
+
+def _e2e_serial(w, dev, steps, warmup, dist_on, rank):
+    """Every step on one stream: copy q, k, v in, forward, copy o out."""
+    import causal_kernelized_sequence_b200 as la
+    (hq, hk, hv, ho), [(dq_, dk_, dv_, do_)], ws = _e2e_buffers(w, dev, rank, 1)
     stream = torch.cuda.Stream()
 
     def one():
@@ -492,9 +497,82 @@ def e2e_prefill(w, dev, steps, warmup, dist_on=False, rank=0):
     if dist_on:
         torch.distributed.barrier()
     ms = max_over_ranks(s.elapsed_time(e) / steps, dist_on, "cuda")
+    return ms, (hq, hk, hv, ho)
+
+
+def _e2e_pipelined(w, dev, steps, warmup, dist_on, rank):
+    """The same steps on three streams with two device buffer sets: step t's
+    inputs are copied in while step t-1 computes and step t-2's output is
+    copied out, as a serving loop would run them.  Every step still copies all
+    of its inputs in and its whole result out inside the timed region.  Also
+    checks that the result copied out last is that step's forward."""
+    import causal_kernelized_sequence_b200 as la
+    (hq, hk, hv, ho), sets, ws = _e2e_buffers(w, dev, rank, 2)
+    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: [torch.cuda.Event() for _ in range(2)]
+    copied_in, computed, copied_out = ev(), ev(), ev()
+    used = [False, False]
+
+    def step(t):
+        b = t & 1
+        dq_, dk_, dv_, do_ = sets[b]
+        with torch.cuda.stream(s_in):
+            if used[b]:
+                s_in.wait_event(computed[b])        # step t-2 has read this set's inputs
+            dq_.copy_(hq, non_blocking=True)
+            dk_.copy_(hk, non_blocking=True)
+            dv_.copy_(hv, non_blocking=True)
+            copied_in[b].record(s_in)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(copied_in[b])
+            if used[b]:
+                s_comp.wait_event(copied_out[b])    # step t-2's output has left this set
+            la.la_forward(dq_, dk_, dv_, w.fmap, out=do_, workspace=ws)
+            computed[b].record(s_comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(computed[b])
+            ho.copy_(do_, non_blocking=True)
+            copied_out[b].record(s_out)
+        used[b] = True
+
+    for t in range(max(1, warmup)):
+        step(t)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    start.record(s_in)
+    for t in range(steps):
+        step(t)
+    end.record(s_out)   # after the last output copy, which follows every other step's work
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    ms = max_over_ranks(start.elapsed_time(end) / steps, dist_on, "cuda")
+    last = sets[(steps - 1) & 1]
+    ok = torch.equal(ho, last[3].cpu())
+    return ms, (hq, hk, hv, ho), ok
+
+
+def e2e_prefill(w, dev, steps, warmup, dist_on=False, rank=0):
+    """Same metric through the public API with host buffers: pinned host q,k,v
+    copied in and o copied out inside the timed region, every step.  Runs the
+    pipelined loop; the serial one-stream loop is the fallback if the pipelined
+    one fails or its last output does not check out.  Returns (ms per step, max
+    over ranks; h2d bytes; d2h bytes; mode)."""
+    mode = "pipelined: copy-in, forward and copy-out on three streams, two buffer sets"
+    try:
+        ms, host, ok = _e2e_pipelined(w, dev, steps, warmup, dist_on, rank)
+        if not ok:
+            raise RuntimeError("last output copied out differs from the device result")
+    except Exception as exc:   # noqa: BLE001 - any failure falls back to the serial loop
+        mode = f"serial: one stream (pipelined loop failed: {exc})"
+        ms, host = _e2e_serial(w, dev, steps, warmup, dist_on, rank)
+    hq, hk, hv, ho = host
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
     d2h = ho.numel() * ho.element_size()
-    return ms, h2d, d2h
+    return ms, h2d, d2h, mode
 
 
 # ----------------------------------------------------------------- CPU oracle
@@ -650,9 +728,9 @@ def main():
     }
     # e2e through the public API with host buffers
     if not w.decode_steps and not w.backward:
-        e_ms, h2d, d2h = e2e_prefill(w, dev, min(args.steps, 50), 3, dist_on, rank)
+        e_ms, h2d, d2h, e_mode = e2e_prefill(w, dev, min(args.steps, 50), 3, dist_on, rank)
         line["e2e"] = {"value": round(whole_job_rate(run.tokens, world, e_ms), 1), "unit": "tokens/s",
-                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "mode": e_mode}
     from causal_kernelized_sequence_b200 import kernel_plan
     kp = kernel_plan(w)
     line["gpu_launches"] = kp["launches_per_step"] * args.steps
