@@ -9,6 +9,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/la.h"
@@ -81,17 +82,19 @@ la_status launch_status()
 
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device) and
 // size; later calls (for example during CUDA-graph capture) make no API call.
+// The table is atomic because calls may come from several host threads; two
+// threads racing on a first call both set the same attribute, which is harmless.
 template <auto kernel>
 la_status set_smem(size_t bytes)
 {
     if (bytes <= 48 * 1024) return LA_OK;
-    static size_t done[64] = {0};  // one table per kernel
+    static std::atomic<size_t> done[64];  // one table per kernel, zero-initialised
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LA_ERR_CUDA;
-    if (done[dev] >= bytes) return LA_OK;
+    if (done[dev].load(std::memory_order_acquire) >= bytes) return LA_OK;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
         return LA_ERR_CUDA;
-    done[dev] = bytes;
+    done[dev].store(bytes, std::memory_order_release);
     return LA_OK;
 }
 
