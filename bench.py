@@ -94,10 +94,36 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def _code_only(text):
+    """C/CUDA source with comments removed and whitespace runs collapsed, so
+    that an edit to comments alone keeps a kernel's hash (string literals,
+    such as inline PTX, are kept as they are)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        if text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        elif text[i] in "\"'":
+            q, j = text[i], i + 1
+            while j < n and text[j] != q:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        else:
+            out.append(text[i])
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def source_hash(*names):
+    """Hash of the code (comments and layout aside) of kernel sources."""
     h = hashlib.sha256()
     for n in names:
-        h.update(open(os.path.join(ROOT, "causal_kernelized_sequence_b200", "csrc", n), "rb").read())
+        text = open(os.path.join(ROOT, "causal_kernelized_sequence_b200", "csrc", n), encoding="utf-8").read()
+        h.update(_code_only(text).encode())
     return h.hexdigest()[:16]
 
 
