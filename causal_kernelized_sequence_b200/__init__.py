@@ -140,6 +140,31 @@ def _dev(*ts):
             raise ValueError("tensors must be contiguous CUDA tensors")
 
 
+def _expect(name, t, shape, dtype, device):
+    """The library sees only pointers: a tensor of another shape, dtype or
+    device than the call implies would be read or written out of bounds, so
+    it is refused here (None passes: the argument is optional)."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype:
+        raise ValueError(f"{name}: expected {dtype} {list(shape)}, got {t.dtype} {list(t.shape)}")
+    if t.device != device:
+        raise ValueError(f"{name}: on {t.device}, expected {device}")
+
+
+def _workspace(ws, need, device):
+    """(workspace tensor, its size in bytes): a new one of `need` bytes, or the
+    caller's after checking it is large enough and on the right device."""
+    if ws is None:
+        return (torch.empty(need, dtype=torch.uint8, device=device) if need else None), need
+    if ws.device != device or not ws.is_contiguous():
+        raise ValueError(f"workspace must be a contiguous tensor on {device}")
+    have = ws.numel() * ws.element_size()
+    if have < need:
+        raise ValueError(f"workspace holds {have} bytes, the call needs {need}")
+    return ws, have
+
+
 def la_feature_dim(fmap: int, dqk: int) -> int:
     return int(load_library().la_feature_dim(fmap, dqk))
 
@@ -164,11 +189,24 @@ def la_forward(q, k, v, fmap, *, state=False, den=False, out=None, workspace=Non
     "z": [B,H,F] fp32, "den": [B,H,N] fp32}.
     """
     lib = load_library()
-    _dev(q, k, v, out)
     B, H, N, dqk = q.shape
     dv = v.shape[-1]
     dt = _dtype_code(q)
     F = la_feature_dim(fmap, dqk)
+    if (s_in is None) != (z_in is None):
+        raise ValueError("s_in and z_in go together")
+    _expect("k", k, (B, H, N, dqk), q.dtype, q.device)
+    _expect("v", v, (B, H, N, dv), q.dtype, q.device)
+    _expect("out", out, (B, H, N, dv), q.dtype, q.device)
+    _expect("s_in", s_in, (B, H, F, dv), torch.float32, q.device)
+    _expect("z_in", z_in, (B, H, F), torch.float32, q.device)
+    _expect("log_decay", log_decay, (B, H, N), torch.float32, q.device)
+    if log_decay is not None:
+        wsb = int(lib.la_forward_decay_workspace_bytes(B, H, N, dqk, dv, fmap, dt))
+    else:
+        wsb = la_forward_workspace_bytes(B, H, N, dqk, dv, fmap, dt)
+    workspace, wsb = _workspace(workspace, wsb, q.device)
+    _dev(q, k, v, out, s_in, z_in, log_decay)
     o = out if out is not None else torch.empty(B, H, N, dv, dtype=q.dtype, device=q.device)
     res = {"o": o}
     if state:
@@ -177,22 +215,6 @@ def la_forward(q, k, v, fmap, *, state=False, den=False, out=None, workspace=Non
     if den:
         res["den"] = torch.empty(B, H, N, dtype=torch.float32, device=q.device)
     if log_decay is not None:
-        wsb = int(lib.la_forward_decay_workspace_bytes(B, H, N, dqk, dv, fmap, dt))
-    else:
-        wsb = la_forward_workspace_bytes(B, H, N, dqk, dv, fmap, dt)
-    if workspace is None and wsb:
-        workspace = torch.empty(wsb, dtype=torch.uint8, device=q.device)
-    if (s_in is None) != (z_in is None):
-        raise ValueError("s_in and z_in go together")
-    if s_in is not None:
-        _dev(s_in, z_in)
-        if s_in.dtype != torch.float32 or z_in.dtype != torch.float32 or not s_in.is_contiguous() \
-                or not z_in.is_contiguous() or tuple(s_in.shape) != (B, H, F, dv) or tuple(z_in.shape) != (B, H, F):
-            raise ValueError("s_in must be fp32 [B,H,F,dv] and z_in fp32 [B,H,F], contiguous")
-    if log_decay is not None:
-        _dev(log_decay)
-        if log_decay.dtype != torch.float32 or tuple(log_decay.shape) != (B, H, N):
-            raise ValueError("log_decay must be fp32 [B,H,N]")
         _check(lib.la_forward_decay(_ptr(q), _ptr(k), _ptr(v), _ptr(log_decay), _ptr(o), _ptr(s_in), _ptr(z_in),
                                     _ptr(res.get("s")), _ptr(res.get("z")), _ptr(res.get("den")),
                                     _ptr(workspace), wsb, B, H, N, dqk, dv, fmap, dt, _stream()), "la_forward_decay")
@@ -223,14 +245,23 @@ def la_forward_varlen(q, k, v, cu_seqlens, max_seqlen, fmap, *, state=False, den
     "den": [H,T]}.  s_in/z_in [nseq,H,F,dv]/[nseq,H,F] start each sequence.
     """
     lib = load_library()
-    _dev(q, k, v, out, cu_seqlens)
     H, T, dqk = q.shape
     dv = v.shape[-1]
-    if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or not cu_seqlens.is_contiguous():
-        raise ValueError("cu_seqlens must be a contiguous int32 vector")
+    _expect("k", k, (H, T, dqk), q.dtype, q.device)
+    _expect("v", v, (H, T, dv), q.dtype, q.device)
+    _expect("out", out, (H, T, dv), q.dtype, q.device)
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or cu_seqlens.device != q.device:
+        raise ValueError("cu_seqlens must be an int32 vector on the device of q")
     nseq = cu_seqlens.numel() - 1
     dt = _dtype_code(q)
     F = la_feature_dim(fmap, dqk)
+    if (s_in is None) != (z_in is None):
+        raise ValueError("s_in and z_in go together")
+    _expect("s_in", s_in, (nseq, H, F, dv), torch.float32, q.device)
+    _expect("z_in", z_in, (nseq, H, F), torch.float32, q.device)
+    wsb = la_forward_varlen_workspace_bytes(nseq, H, min(max_seqlen, T), dqk, dv, fmap, dt)
+    workspace, wsb = _workspace(workspace, wsb, q.device)
+    _dev(q, k, v, out, cu_seqlens, s_in, z_in)
     o = out if out is not None else torch.empty(H, T, dv, dtype=q.dtype, device=q.device)
     res = {"o": o}
     if state:
@@ -238,16 +269,6 @@ def la_forward_varlen(q, k, v, cu_seqlens, max_seqlen, fmap, *, state=False, den
         res["z"] = torch.empty(nseq, H, F, dtype=torch.float32, device=q.device)
     if den:
         res["den"] = torch.empty(H, T, dtype=torch.float32, device=q.device)
-    if (s_in is None) != (z_in is None):
-        raise ValueError("s_in and z_in go together")
-    if s_in is not None:
-        _dev(s_in, z_in)
-        if s_in.dtype != torch.float32 or z_in.dtype != torch.float32 or not s_in.is_contiguous() \
-                or not z_in.is_contiguous() or tuple(s_in.shape) != (nseq, H, F, dv) or tuple(z_in.shape) != (nseq, H, F):
-            raise ValueError("s_in must be fp32 [nseq,H,F,dv] and z_in fp32 [nseq,H,F], contiguous")
-    wsb = la_forward_varlen_workspace_bytes(nseq, H, min(max_seqlen, T), dqk, dv, fmap, dt)
-    if workspace is None and wsb:
-        workspace = torch.empty(wsb, dtype=torch.uint8, device=q.device)
     _check(lib.la_forward_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(cu_seqlens), nseq, max_seqlen, T,
                                  _ptr(s_in), _ptr(z_in), _ptr(res.get("s")), _ptr(res.get("z")),
                                  _ptr(res.get("den")), _ptr(workspace), wsb, H, dqk, dv, fmap, dt, _stream()),
@@ -261,9 +282,12 @@ def la_forward_noalloc(q, k, v, fmap, *, state=False, den=False, out=None):
     calls must not overlap on the GPU).  Outputs are allocated here only if
     not given."""
     lib = load_library()
-    _dev(q, k, v, out)
     B, H, N, dqk = q.shape
     dv = v.shape[-1]
+    _expect("k", k, (B, H, N, dqk), q.dtype, q.device)
+    _expect("v", v, (B, H, N, dv), q.dtype, q.device)
+    _expect("out", out, (B, H, N, dv), q.dtype, q.device)
+    _dev(q, k, v, out)
     dt = _dtype_code(q)
     F = la_feature_dim(fmap, dqk)
     o = out if out is not None else torch.empty(B, H, N, dv, dtype=q.dtype, device=q.device)
@@ -282,16 +306,18 @@ def la_forward_noalloc(q, k, v, fmap, *, state=False, den=False, out=None):
 def la_backward(q, k, v, dout, fmap, *, workspace=None):
     """Gradients (dq, dk, dv) of the forward for upstream gradient dout."""
     lib = load_library()
-    _dev(q, k, v, dout)
     B, H, N, dqk = q.shape
     dv = v.shape[-1]
+    _expect("k", k, (B, H, N, dqk), q.dtype, q.device)
+    _expect("v", v, (B, H, N, dv), q.dtype, q.device)
+    _expect("dout", dout, (B, H, N, dv), q.dtype, q.device)
     dt = _dtype_code(q)
+    wsb = la_backward_workspace_bytes(B, H, N, dqk, dv, fmap, dt)
+    workspace, wsb = _workspace(workspace, wsb, q.device)
+    _dev(q, k, v, dout)
     dq = torch.empty_like(q)
     dk = torch.empty_like(k)
     dvv = torch.empty_like(v)
-    wsb = la_backward_workspace_bytes(B, H, N, dqk, dv, fmap, dt)
-    if workspace is None and wsb:
-        workspace = torch.empty(wsb, dtype=torch.uint8, device=q.device)
     _check(lib.la_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dvv),
                            _ptr(workspace), wsb, B, H, N, dqk, dv, fmap, dt, _stream()), "la_backward")
     return dq, dk, dvv
@@ -301,17 +327,18 @@ def la_backward_decay(q, k, v, log_decay, dout, fmap, *, workspace=None):
     """Gradients (dq, dk, dv, dlog_decay) of the gated forward (la_forward with
     log_decay) for upstream gradient dout."""
     lib = load_library()
-    _dev(q, k, v, dout, log_decay)
     B, H, N, dqk = q.shape
     dv = v.shape[-1]
+    _expect("k", k, (B, H, N, dqk), q.dtype, q.device)
+    _expect("v", v, (B, H, N, dv), q.dtype, q.device)
+    _expect("dout", dout, (B, H, N, dv), q.dtype, q.device)
+    _expect("log_decay", log_decay, (B, H, N), torch.float32, q.device)
     dt = _dtype_code(q)
-    if log_decay.dtype != torch.float32 or tuple(log_decay.shape) != (B, H, N):
-        raise ValueError("log_decay must be fp32 [B,H,N]")
+    wsb = int(lib.la_backward_decay_workspace_bytes(B, H, N, dqk, dv, fmap, dt))
+    workspace, wsb = _workspace(workspace, wsb, q.device)
+    _dev(q, k, v, dout, log_decay)
     dq, dk, dvv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     dg = torch.empty(B, H, N, dtype=torch.float32, device=q.device)
-    wsb = int(lib.la_backward_decay_workspace_bytes(B, H, N, dqk, dv, fmap, dt))
-    if workspace is None:
-        workspace = torch.empty(wsb, dtype=torch.uint8, device=q.device)
     _check(lib.la_backward_decay(_ptr(q), _ptr(k), _ptr(v), _ptr(log_decay), _ptr(dout), _ptr(dq), _ptr(dk),
                                  _ptr(dvv), _ptr(dg), _ptr(workspace), wsb, B, H, N, dqk, dv, fmap, dt, _stream()),
            "la_backward_decay")
@@ -324,15 +351,20 @@ def la_decode_step(q, k, v, s, z, fmap, y=None, log_decay=None):
     [B,H] fp32 the state is first multiplied by exp(log_decay)
     (la_decode_step_decay)."""
     lib = load_library()
-    _dev(q, k, v, s, z, y, log_decay)
     B, H, dqk = q.shape
     dv = v.shape[-1]
+    F = la_feature_dim(fmap, dqk)
+    _expect("k", k, (B, H, dqk), q.dtype, q.device)
+    _expect("v", v, (B, H, dv), q.dtype, q.device)
+    _expect("s", s, (B, H, F, dv), torch.float32, q.device)
+    _expect("z", z, (B, H, F), torch.float32, q.device)
+    _expect("y", y, (B, H, dv), q.dtype, q.device)
+    _expect("log_decay", log_decay, (B, H), torch.float32, q.device)
+    _dev(q, k, v, s, z, y, log_decay)
     dt = _dtype_code(q)
     if y is None:
         y = torch.empty(B, H, dv, dtype=q.dtype, device=q.device)
     if log_decay is not None:
-        if log_decay.dtype != torch.float32 or tuple(log_decay.shape) != (B, H):
-            raise ValueError("log_decay must be fp32 [B,H]")
         _check(lib.la_decode_step_decay(_ptr(q), _ptr(k), _ptr(v), _ptr(log_decay), _ptr(y), _ptr(s), _ptr(z),
                                         B, H, dqk, dv, fmap, dt, _stream()), "la_decode_step_decay")
         return y
@@ -346,9 +378,12 @@ def la_swa_forward(q, k, v, window, *, out=None, lse=False):
     max(0, i-w+1) .. i).  q, k [B,H,N,dqk]; v [B,H,N,dv].
     Returns {"o": [B,H,N,dv], and if requested "lse": [B,H,N] fp32}."""
     lib = load_library()
-    _dev(q, k, v, out)
     B, H, N, dqk = q.shape
     dv = v.shape[-1]
+    _expect("k", k, (B, H, N, dqk), q.dtype, q.device)
+    _expect("v", v, (B, H, N, dv), q.dtype, q.device)
+    _expect("out", out, (B, H, N, dv), q.dtype, q.device)
+    _dev(q, k, v, out)
     o = out if out is not None else torch.empty(B, H, N, dv, dtype=q.dtype, device=q.device)
     res = {"o": o}
     if lse:
@@ -362,9 +397,13 @@ def la_swa_cache_fill(k, v, window, *, k_cache=None, v_cache=None):
     """The w-token cache of a prefill: the last min(N, w) tokens of k, v
     [B,H,N,*] in slots t mod w.  Returns (k_cache [B,H,w,dqk], v_cache [B,H,w,dv])."""
     lib = load_library()
-    _dev(k, v, k_cache, v_cache)
     B, H, N, dqk = k.shape
     dv = v.shape[-1]
+    window = int(window)
+    _expect("v", v, (B, H, N, dv), k.dtype, k.device)
+    _expect("k_cache", k_cache, (B, H, window, dqk), k.dtype, k.device)
+    _expect("v_cache", v_cache, (B, H, window, dv), k.dtype, k.device)
+    _dev(k, v, k_cache, v_cache)
     if k_cache is None:
         k_cache = torch.zeros(B, H, window, dqk, dtype=k.dtype, device=k.device)
     if v_cache is None:
@@ -379,11 +418,16 @@ def la_swa_decode_step(q, k, v, k_cache, v_cache, pos, window, y=None):
     are updated in place; pos int32 [B] on the device = tokens held before
     this one (not advanced here).  Returns y [B,H,dv]."""
     lib = load_library()
-    _dev(q, k, v, k_cache, v_cache, pos, y)
     B, H, dqk = q.shape
     dv = v.shape[-1]
-    if pos.dtype != torch.int32 or tuple(pos.shape) != (B,):
-        raise ValueError("pos must be int32 [B]")
+    window = int(window)
+    _expect("k", k, (B, H, dqk), q.dtype, q.device)
+    _expect("v", v, (B, H, dv), q.dtype, q.device)
+    _expect("k_cache", k_cache, (B, H, window, dqk), q.dtype, q.device)
+    _expect("v_cache", v_cache, (B, H, window, dv), q.dtype, q.device)
+    _expect("pos", pos, (B,), torch.int32, q.device)
+    _expect("y", y, (B, H, dv), q.dtype, q.device)
+    _dev(q, k, v, k_cache, v_cache, pos, y)
     if y is None:
         y = torch.empty(B, H, dv, dtype=q.dtype, device=q.device)
     _check(lib.la_swa_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(y), _ptr(k_cache), _ptr(v_cache), _ptr(pos),

@@ -92,3 +92,62 @@ def test_binding_signatures_match_header(monkeypatch):
             assert [_ctypes_kind(t) for t in fn.argtypes] == params, name
         else:
             assert not fn.argtypes, name
+
+
+def _f32(*shape):
+    return torch.zeros(*shape, dtype=torch.float32)
+
+
+# Correctly shaped (CPU) tensors pass the binding's shape checks and are then
+# refused only for not being CUDA tensors.
+@pytest.mark.parametrize("call", [
+    lambda: la.la_forward(_cpu(1, 2, 8, 16), _cpu(1, 2, 8, 16), _cpu(1, 2, 8, 64), la.LA_FMAP_TAYLOR2,
+                          s_in=_f32(1, 2, 273, 64), z_in=_f32(1, 2, 273), out=_cpu(1, 2, 8, 64)),
+    lambda: la.la_forward(_cpu(1, 2, 8, 16), _cpu(1, 2, 8, 16), _cpu(1, 2, 8, 64), la.LA_FMAP_ELU1,
+                          log_decay=_f32(1, 2, 8)),
+    lambda: la.la_decode_step(_f32(2, 3, 16), _f32(2, 3, 16), _f32(2, 3, 64), _f32(2, 3, 153, 64), _f32(2, 3, 153),
+                              la.LA_FMAP_TAYLOR2_SYM, y=_f32(2, 3, 64), log_decay=_f32(2, 3)),
+    lambda: la.la_forward_varlen(_cpu(2, 8, 16), _cpu(2, 8, 16), _cpu(2, 8, 64),
+                                 torch.tensor([0, 3, 8], dtype=torch.int32), 5, la.LA_FMAP_ELU1,
+                                 s_in=_f32(2, 2, 16, 64), z_in=_f32(2, 2, 16), out=_cpu(2, 8, 64)),
+    lambda: la.la_swa_cache_fill(_cpu(1, 2, 8, 64), _cpu(1, 2, 8, 64), 16, k_cache=_cpu(1, 2, 16, 64),
+                                 v_cache=_cpu(1, 2, 16, 64)),
+    lambda: la.la_swa_decode_step(_cpu(1, 2, 64), _cpu(1, 2, 64), _cpu(1, 2, 64), _cpu(1, 2, 16, 64),
+                                  _cpu(1, 2, 16, 64), torch.zeros(1, dtype=torch.int32), 16, y=_cpu(1, 2, 64)),
+    lambda: la.la_backward(_cpu(1, 1, 8, 16), _cpu(1, 1, 8, 16), _cpu(1, 1, 8, 32), _cpu(1, 1, 8, 32),
+                           la.LA_FMAP_ELU1, workspace=torch.zeros(1 << 16, dtype=torch.uint8)),
+])
+def test_consistent_shapes_reach_the_device_check(call):
+    la.load_library()
+    with pytest.raises(ValueError, match="CUDA"):
+        call()
+
+
+# A tensor whose shape, dtype or size disagrees with the call is refused before
+# its pointer could reach a kernel.
+@pytest.mark.parametrize("call,what", [
+    (lambda: la.la_forward(_cpu(1, 2, 8, 16), _cpu(1, 2, 7, 16), _cpu(1, 2, 8, 64), la.LA_FMAP_ELU1), "k"),
+    (lambda: la.la_forward(_cpu(1, 2, 8, 16), _f32(1, 2, 8, 16), _cpu(1, 2, 8, 64), la.LA_FMAP_ELU1), "k"),
+    (lambda: la.la_forward(_cpu(1, 2, 8, 16), _cpu(1, 2, 8, 16), _cpu(1, 2, 8, 64), la.LA_FMAP_ELU1,
+                           out=_cpu(1, 2, 8, 32)), "out"),
+    (lambda: la.la_forward(_cpu(1, 2, 8, 16), _cpu(1, 2, 8, 16), _cpu(1, 2, 8, 64), la.LA_FMAP_TAYLOR2,
+                           s_in=_f32(1, 2, 153, 64), z_in=_f32(1, 2, 153)), "s_in"),
+    (lambda: la.la_forward(_cpu(1, 2, 8, 16), _cpu(1, 2, 8, 16), _cpu(1, 2, 8, 64), la.LA_FMAP_ELU1,
+                           log_decay=_cpu(1, 2, 8)), "log_decay"),
+    (lambda: la.la_decode_step(_f32(2, 3, 16), _f32(2, 3, 16), _f32(2, 3, 64), _f32(2, 3, 273, 64),
+                               _f32(2, 3, 273), la.LA_FMAP_TAYLOR2_SYM), "s"),
+    (lambda: la.la_decode_step(_f32(2, 3, 16), _f32(2, 3, 16), _f32(2, 3, 64), _f32(2, 3, 16, 64),
+                               _f32(2, 3, 16), la.LA_FMAP_ELU1, y=_f32(2, 3, 63)), "y"),
+    (lambda: la.la_forward_varlen(_cpu(2, 8, 16), _cpu(2, 8, 16), _cpu(2, 9, 64),
+                                  torch.tensor([0, 8], dtype=torch.int32), 8, la.LA_FMAP_ELU1), "v"),
+    (lambda: la.la_swa_decode_step(_cpu(1, 2, 64), _cpu(1, 2, 64), _cpu(1, 2, 64), _cpu(1, 2, 32, 64),
+                                   _cpu(1, 2, 16, 64), torch.zeros(1, dtype=torch.int32), 16), "k_cache"),
+    (lambda: la.la_swa_decode_step(_cpu(1, 2, 64), _cpu(1, 2, 64), _cpu(1, 2, 64), _cpu(1, 2, 16, 64),
+                                   _cpu(1, 2, 16, 64), torch.zeros(2, dtype=torch.int32), 16), "pos"),
+    (lambda: la.la_backward(_cpu(1, 1, 8, 16), _cpu(1, 1, 8, 16), _cpu(1, 1, 8, 32), _cpu(1, 1, 8, 32),
+                            la.LA_FMAP_ELU1, workspace=torch.zeros(16, dtype=torch.uint8)), "workspace"),
+])
+def test_mismatched_tensors_rejected(call, what):
+    la.load_library()
+    with pytest.raises(ValueError, match=what):
+        call()
