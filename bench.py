@@ -588,13 +588,22 @@ def e2e_prefill(w, dev, steps, warmup, dist_on=False, rank=0):
     one fails or its last output does not check out.  Returns (ms per step, max
     over ranks; h2d bytes; d2h bytes; mode)."""
     mode = "pipelined: copy-in, forward and copy-out on three streams, two buffer sets"
-    try:
+    if dist_on:
+        # Every rank must take the same collective steps: an exception here
+        # ends the job rather than leaving the ranks at different barriers,
+        # and a failed check falls back on all ranks together.
         ms, host, ok = _e2e_pipelined(w, dev, steps, warmup, dist_on, rank)
-        if not ok:
-            raise RuntimeError("last output copied out differs from the device result")
-    except Exception as exc:   # noqa: BLE001 - any failure falls back to the serial loop
-        mode = f"serial: one stream (pipelined loop failed: {exc})"
-        ms, host = _e2e_serial(w, dev, steps, warmup, dist_on, rank)
+        if max_over_ranks(0.0 if ok else 1.0, dist_on, "cuda") > 0:
+            mode = "serial: one stream (the pipelined loop's last output did not check out on some rank)"
+            ms, host = _e2e_serial(w, dev, steps, warmup, dist_on, rank)
+    else:
+        try:
+            ms, host, ok = _e2e_pipelined(w, dev, steps, warmup, dist_on, rank)
+            if not ok:
+                raise RuntimeError("last output copied out differs from the device result")
+        except Exception as exc:   # noqa: BLE001 - any failure falls back to the serial loop
+            mode = f"serial: one stream (pipelined loop failed: {exc})"
+            ms, host = _e2e_serial(w, dev, steps, warmup, dist_on, rank)
     hq, hk, hv, ho = host
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
     d2h = ho.numel() * ho.element_size()
