@@ -91,3 +91,40 @@ def test_range_bookkeeping(B, H, N):
             if first_len < begin(T, G, kb + 1) - tb or c0 + first_len == nc:
                 finals[tb // nc] = finals.get(tb // nc, 0) + 1
     assert finals == {h: 1 for h in range(B * H)}
+
+
+# ------------------------------------------------------------------ segments
+# The one-launch forward (elu d=128, Taylor) and the tensor-core backward split
+# a sequence into P segments of cps chunks so that B*H*P blocks roughly fill
+# the 148 SMs; segment s covers chunks [s*cps, min(nc, (s+1)*cps)).
+
+def segments(B, H, N):
+    nc = (N + C - 1) // C
+    p = max(1, NSM // (B * H))
+    p = min(p, nc)
+    cps = (nc + p - 1) // p
+    return (nc + cps - 1) // cps, cps, nc
+
+
+SEG_SHAPES = [(B, H, N) for B, H in [(1, 1), (1, 2), (2, 3), (2, 16), (8, 16), (1, 200)]
+              for N in [1, 100, 128, 129, 1000, 4097, 16384, 65536]]
+
+
+@pytest.mark.parametrize("B,H,N", SEG_SHAPES)
+def test_segment_plan(B, H, N):
+    la.load_library()
+    P, cps, nc = segments(B, H, N)
+    # every chunk in exactly one segment, none empty
+    chunks = [c for s in range(P) for c in range(s * cps, min(nc, (s + 1) * cps))]
+    assert chunks == list(range(nc)) and all(s * cps < nc for s in range(P))
+    assert B * H * P <= max(NSM, B * H)
+    # the workspaces the library asks for hold one increment per (head, segment)
+    inc128 = 128 * 144 * 4                   # elu d=128: F x (d_v + 16) fp32
+    incT = 160 * 80 * 4                      # Taylor: 160 packed features x (64 + 16)
+    assert la.la_forward_workspace_bytes(B, H, N, 128, 128, la.LA_FMAP_ELU1, la.LA_BF16) == \
+        (B * H * P * inc128 if P > 1 else 0)
+    assert la.la_forward_workspace_bytes(B, H, N, 16, 64, la.LA_FMAP_TAYLOR2, la.LA_BF16) == \
+        (B * H * P * incT if P > 1 else 0)
+    # backward: den_i, dden_i per token, plus S and R increments when split
+    assert la.la_backward_workspace_bytes(B, H, N, 128, 128, la.LA_FMAP_ELU1, la.LA_BF16) == \
+        B * H * N * 2 * 4 + (2 * B * H * P * 128 * 144 * 4 if P > 1 else 0)
