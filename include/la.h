@@ -102,13 +102,19 @@ LA_API const char *la_status_string(int status);
 LA_API int64_t la_feature_dim(int fmap, int dqk);
 
 /* Bytes of device workspace la_forward needs for these sizes (0 if none).
- * The workspace holds per-segment partial states and hand-off flags when a
- * sequence is split across thread blocks.  The caller allocates it; its
- * contents need not be initialised (la_forward clears what it uses, on
- * `stream`).  Returns 0 also for invalid arguments. */
+ * The workspace carries what one launch of the call hands to the next: for
+ * the bf16 elu dqk = dv = 64 forward, the phi(K) tiles, a state snapshot per
+ * 128-token chunk and two partial sums per block; for the other tensor-core
+ * shapes, when a long sequence is split across thread blocks, one state
+ * increment per segment.  The caller allocates it.  Its contents need not be
+ * initialised: every value a call reads from it was written earlier in the
+ * same call.  Calls that may run at the same time need separate workspaces.
+ * Returns 0 also for invalid arguments. */
 LA_API size_t la_forward_workspace_bytes(int B, int H, int N, int dqk, int dv, int fmap, int dtype);
 
-/* Bytes of device workspace la_backward needs (0 if none); same rules. */
+/* Bytes of device workspace la_backward needs: den_i and dden_i per token
+ * (fp32), plus, when a sequence is split across thread blocks, one S and one
+ * R increment per segment.  Same rules as la_forward_workspace_bytes. */
 LA_API size_t la_backward_workspace_bytes(int B, int H, int N, int dqk, int dv, int fmap, int dtype);
 
 /* Causal linear attention forward (prefill / training forward).
