@@ -455,171 +455,3 @@ def test_forward_deterministic():
     b = gpu_forward(q, k, v, TAYLOR2, state=True)
     for n in a:
         assert torch.equal(a[n], b[n]), n
-
-
-# ------------------------------------------------------------ full workloads
-
-def test_workload_elu_fp32_fwd():
-    w = W.BY_NAME["elu_fp32_fwd"]
-    q, k, v, _ = W.make_inputs(w)
-    r = gpu_forward(q, k, v, w.fmap, den=True)
-    assert r["o"].shape == (1, 1, 256, 32)
-    o_ref, den_ref = orc.forward_brute(w.fmap, q, k, v)
-    assert orc.max_rel_l2(r["o"], o_ref) <= 1e-5
-    assert orc.max_rel_l2(r["den"], den_ref) <= 1e-5
-
-
-def test_workload_elu_bf16_fwd():
-    w = W.BY_NAME["elu_bf16_fwd"]
-    q, k, v, _ = W.make_inputs(w)
-    r = gpu_forward(q, k, v, w.fmap, den=True, state=True)
-    o_ref, den_ref, s_ref, z_ref = orc.forward_recurrent(w.fmap, q, k, v)
-    assert orc.max_rel_l2(r["o"], o_ref) <= 1e-2
-    assert orc.max_rel_l2(r["den"], den_ref) <= 1e-2
-    assert orc.max_rel_l2(r["s"], s_ref) <= 1e-2
-    # brute force on sampled rows cross-checks the recurrent oracle itself
-    rows = [0, 1, 63, 64, 2047, 4095]
-    ob, _ = orc.forward_rows(w.fmap, q[3, 7], k[3, 7], v[3, 7], rows)
-    np.testing.assert_allclose(o_ref[3, 7, rows], ob, rtol=1e-9, atol=1e-12)
-
-
-def test_workload_taylor_bf16_fwd():
-    w = W.BY_NAME["taylor_bf16_fwd"]
-    q, k, v, _ = W.make_inputs(w)
-    r = gpu_forward(q, k, v, w.fmap, den=True, state=True)
-    heads = [(0, 0), (1, 5), (3, 9), (7, 15)]
-    for b, h in heads:
-        o_ref, den_ref, s_ref, z_ref = orc.forward_recurrent(
-            w.fmap, q[b:b + 1, h:h + 1], k[b:b + 1, h:h + 1], v[b:b + 1, h:h + 1])
-        assert orc.max_rel_l2(r["o"][b:b + 1, h:h + 1], o_ref) <= 1e-2
-        assert orc.max_rel_l2(r["den"][b:b + 1, h:h + 1], den_ref) <= 1e-2
-        assert orc.max_rel_l2(r["s"][b:b + 1, h:h + 1], s_ref) <= 1e-2
-        assert orc.max_rel_l2(r["z"][b:b + 1, h:h + 1], z_ref) <= 1e-2
-    # Taylor: den_i >= i/2 for every head (positivity, any size)
-    assert (r["den"] >= torch.arange(1, w.N + 1) / 2 * (1 - 1e-3)).all()
-
-
-def test_workload_elu_bf16_train():
-    w = W.BY_NAME["elu_bf16_train"]
-    q, k, v, do = W.make_inputs(w)
-    qd, kd, vd, dod = (t.to(DEV) for t in (q, k, v, do))
-    fr = la.la_forward(qd, kd, vd, w.fmap, den=True)
-    dq, dk, dvv = la.la_backward(qd, kd, vd, dod, w.fmap)
-    torch.cuda.synchronize()
-    la.la_get_device_status()
-    for b, h in [(0, 0), (1, 11), (0, 15)]:
-        sl = lambda t: t[b:b + 1, h:h + 1]
-        o_ref, den_ref, _, _ = orc.forward_recurrent(w.fmap, sl(q), sl(k), sl(v))
-        rq, rk, rv = orc.backward_recurrent(w.fmap, sl(q), sl(k), sl(v), sl(do))
-        assert orc.max_rel_l2(sl(fr["o"]).cpu(), o_ref) <= 1e-2
-        for got, ref in ((dq, rq), (dk, rk), (dvv, rv)):
-            assert orc.max_rel_l2(sl(got).cpu(), ref) <= 1e-2
-    # any-size invariant: sum_j dv_j = sum_i dO_i per slice
-    lhs = dvv.float().sum(2)
-    rhs = dod.float().sum(2)
-    assert ((lhs - rhs).norm() / rhs.norm()).item() < 1e-2
-
-
-def test_workload_elu_bf16_decay_fwd():
-    w = W.BY_NAME["elu_bf16_decay_fwd"]
-    q, k, v, _ = W.make_inputs(w)
-    g = W.make_gates(w)
-    r = gpu_forward(q, k, v, w.fmap, den=True, state=True, log_decay=g.to(DEV))
-    for b, h in [(0, 0), (2, 5), (3, 7)]:
-        sl = lambda t: t[b:b + 1, h:h + 1]
-        o_ref, den_ref, s_ref, _ = orc.forward_recurrent_decay(w.fmap, sl(q), sl(k), sl(v), sl(g))
-        assert orc.max_rel_l2(sl(r["o"]), o_ref) <= 1e-2, (b, h)
-        assert orc.max_rel_l2(sl(r["den"]), den_ref) <= 1e-2
-        assert orc.max_rel_l2(sl(r["s"]), s_ref) <= 1e-2
-    assert (r["den"] > 0).all()
-
-
-def test_workload_swa_bf16_fwd():
-    w = W.BY_NAME["swa_bf16_fwd"]
-    q, k, v, _ = W.make_inputs(w)
-    r = la.la_swa_forward(q.to(DEV), k.to(DEV), v.to(DEV), w.window, lse=True)
-    torch.cuda.synchronize()
-    la.la_get_device_status()
-    for b, h in [(0, 0), (2, 5), (3, 7)]:
-        sl = lambda t: t[b:b + 1, h:h + 1]
-        o_ref, lse_ref = orc.swa_forward(sl(q), sl(k), sl(v), w.window)
-        assert orc.max_rel_l2(sl(r["o"]).cpu(), o_ref) <= 1e-2, (b, h)
-        assert orc.max_rel_l2(sl(r["lse"]).cpu(), lse_ref) <= 1e-2
-    assert torch.isfinite(r["o"].float()).all()
-
-
-def test_workload_swa_bf16_decode():
-    """The decode workload's shapes (1024 x 16 heads, 64-token caches filled
-    by a 64-token prompt), 16 steps, sampled heads against the oracle."""
-    w = W.BY_NAME["swa_bf16_decode"]
-    (q, k, v), (sq, sk, sv) = W.make_decode_inputs(w, steps=16)
-    kc, vc = la.la_swa_cache_fill(k.to(DEV), v.to(DEV), w.window)
-    pos = torch.full((w.B,), w.N, dtype=torch.int32, device=DEV)
-    ys = []
-    for t in range(16):
-        ys.append(la.la_swa_decode_step(sq[t].to(DEV), sk[t].to(DEV), sv[t].to(DEV), kc, vc, pos, w.window).cpu())
-        pos += 1
-    torch.cuda.synchronize()
-    la.la_get_device_status()
-    for b, h in [(0, 0), (100, 7), (1023, 15)]:
-        qf = torch.cat([q[b, h], sq[:, b, h]])[None, None]
-        kf = torch.cat([k[b, h], sk[:, b, h]])[None, None]
-        vf = torch.cat([v[b, h], sv[:, b, h]])[None, None]
-        o_ref, _ = orc.swa_forward(qf, kf, vf, w.window)
-        got = torch.stack([y[b, h] for y in ys])[None, None]
-        assert orc.max_rel_l2(got, o_ref[:, :, w.N:]) <= 1e-2, (b, h)
-
-
-def test_workload_elu_bf16_varlen():
-    w = W.BY_NAME["elu_bf16_varlen"]
-    q, k, v, cu = W.make_varlen_inputs(w)
-    lens = W.varlen_lengths(w)
-    r = la.la_forward_varlen(q.to(DEV), k.to(DEV), v.to(DEV), cu.to(DEV), max(lens), w.fmap, den=True, state=True)
-    torch.cuda.synchronize()
-    la.la_get_device_status()
-    o, den, s = r["o"].cpu(), r["den"].cpu(), r["s"].cpu()
-    # sampled sequences (the longest, a short one, the last) and heads, one by one
-    longest = int(np.argmax(lens))
-    for n in (longest, int(np.argmin(lens)), len(lens) - 1):
-        a, b = int(cu[n]), int(cu[n + 1])
-        for h in (0, 5):
-            sl = lambda t: t[h:h + 1, a:b][None]
-            o_ref, den_ref, s_ref, _ = orc.forward_recurrent(w.fmap, sl(q), sl(k), sl(v))
-            assert orc.max_rel_l2(o[h, a:b][None, None], o_ref) <= 1e-2, (n, h)
-            assert orc.max_rel_l2(den[h, a:b][None, None], den_ref) <= 1e-2
-            assert orc.max_rel_l2(s[n, h][None, None], s_ref) <= 1e-2
-    assert (den > 0).all()   # elu+1 features are positive: any size
-
-
-@pytest.mark.parametrize("name", ["taylor_decode", "taylor_decode_sym"])
-def test_workload_taylor_decode(name):
-    w = W.BY_NAME[name]
-    (q, k, v), (sq, sk, sv) = W.make_decode_inputs(w)
-    r = la.la_forward(q.to(DEV), k.to(DEV), v.to(DEV), w.fmap, state=True)
-    s, z = r["s"], r["z"]
-    heads = [(0, 0), (17, 3), (128, 8), (255, 15)]
-    hs = lambda t: torch.stack([t[..., b, h, :] for b, h in heads], dim=-2)
-    # oracle: prefill then the same steps, for the sampled heads only
-    qh = torch.stack([q[b, h] for b, h in heads])[None]
-    kh = torch.stack([k[b, h] for b, h in heads])[None]
-    vh = torch.stack([v[b, h] for b, h in heads])[None]
-    _, _, s_o, z_o = orc.forward_recurrent(w.fmap, qh, kh, vh)
-    s_o = np.ascontiguousarray(s_o[0]); z_o = np.ascontiguousarray(z_o[0])
-    # the prefill's final state, for the sampled heads
-    assert orc.max_rel_l2(torch.stack([s[b, h].cpu() for b, h in heads]), s_o, slice_dims=1) <= 1e-5
-    y_all = torch.empty(w.decode_steps, w.B, w.H, w.dv, device=DEV)
-    sqd, skd, svd = sq.to(DEV), sk.to(DEV), sv.to(DEV)
-    for t in range(w.decode_steps):
-        la.la_decode_step(sqd[t], skd[t], svd[t], s, z, w.fmap, y=y_all[t])
-    torch.cuda.synchronize()
-    la.la_get_device_status()
-    y_all = y_all.cpu()
-    worst = 0.0
-    for t in range(w.decode_steps):
-        y_o = orc.decode_step(w.fmap, hs(sq[t]), hs(sk[t]), hs(sv[t]), s_o, z_o)
-        worst = max(worst, orc.max_rel_l2(hs(y_all[t])[None], y_o[None], slice_dims=1))
-    assert worst <= 1e-5, worst
-    s_fin = torch.stack([s[b, h].cpu() for b, h in heads])
-    z_fin = torch.stack([z[b, h].cpu() for b, h in heads])
-    assert orc.max_rel_l2(s_fin, s_o, slice_dims=1) <= 1e-5
-    assert orc.max_rel_l2(z_fin, z_o, slice_dims=1) <= 1e-5
