@@ -1,9 +1,9 @@
 """B200 causal linear attention: Python binding of the C-ABI library libla.so.
 
 This module only marshals arguments: it checks shapes and dtypes of torch
-CUDA tensors, passes their device pointers, sizes and the current CUDA stream
-to the C entry points declared in ``include/la.h``, and raises on a non-OK
-status.  Every step of the computation runs in the library's CUDA kernels;
+CUDA tensors, makes their device the current one for the call, passes their
+device pointers, sizes and that device's current stream to the C entry points
+declared in ``include/la.h``, and raises on a non-OK status.  Every step of the computation runs in the library's CUDA kernels;
 there is no CPU or PyTorch fallback, and importing the compute functions fails
 loudly when the library has not been built.
 
@@ -117,8 +117,17 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream():
-    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+def _device(device):
+    return torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+
+
+def _call(fn, where, device, *args):
+    """One library call for tensors on `device`: that device is made current
+    for the call (the library launches on the current device) and its
+    current stream is passed as the last argument."""
+    with torch.cuda.device(device):
+        stream = ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+        _check(fn(*args, stream), where)
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -215,19 +224,18 @@ def la_forward(q, k, v, fmap, *, state=False, den=False, out=None, workspace=Non
     if den:
         res["den"] = torch.empty(B, H, N, dtype=torch.float32, device=q.device)
     if log_decay is not None:
-        _check(lib.la_forward_decay(_ptr(q), _ptr(k), _ptr(v), _ptr(log_decay), _ptr(o), _ptr(s_in), _ptr(z_in),
-                                    _ptr(res.get("s")), _ptr(res.get("z")), _ptr(res.get("den")),
-                                    _ptr(workspace), wsb, B, H, N, dqk, dv, fmap, dt, _stream()), "la_forward_decay")
+        _call(lib.la_forward_decay, "la_forward_decay", q.device,
+              _ptr(q), _ptr(k), _ptr(v), _ptr(log_decay), _ptr(o), _ptr(s_in), _ptr(z_in), _ptr(res.get("s")),
+              _ptr(res.get("z")), _ptr(res.get("den")), _ptr(workspace), wsb, B, H, N, dqk, dv, fmap, dt)
         return res
     if s_in is not None:
-        _check(lib.la_forward_from_state(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(s_in), _ptr(z_in),
-                                         _ptr(res.get("s")), _ptr(res.get("z")), _ptr(res.get("den")),
-                                         _ptr(workspace), wsb, B, H, N, dqk, dv, fmap, dt, _stream()),
-               "la_forward_from_state")
+        _call(lib.la_forward_from_state, "la_forward_from_state", q.device,
+              _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(s_in), _ptr(z_in), _ptr(res.get("s")), _ptr(res.get("z")),
+              _ptr(res.get("den")), _ptr(workspace), wsb, B, H, N, dqk, dv, fmap, dt)
         return res
-    _check(lib.la_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(res.get("s")), _ptr(res.get("z")),
-                          _ptr(res.get("den")), _ptr(workspace), wsb, B, H, N, dqk, dv, fmap, dt,
-                          _stream()), "la_forward")
+    _call(lib.la_forward, "la_forward", q.device,
+          _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(res.get("s")), _ptr(res.get("z")), _ptr(res.get("den")),
+          _ptr(workspace), wsb, B, H, N, dqk, dv, fmap, dt)
     return res
 
 
@@ -269,10 +277,9 @@ def la_forward_varlen(q, k, v, cu_seqlens, max_seqlen, fmap, *, state=False, den
         res["z"] = torch.empty(nseq, H, F, dtype=torch.float32, device=q.device)
     if den:
         res["den"] = torch.empty(H, T, dtype=torch.float32, device=q.device)
-    _check(lib.la_forward_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(cu_seqlens), nseq, max_seqlen, T,
-                                 _ptr(s_in), _ptr(z_in), _ptr(res.get("s")), _ptr(res.get("z")),
-                                 _ptr(res.get("den")), _ptr(workspace), wsb, H, dqk, dv, fmap, dt, _stream()),
-           "la_forward_varlen")
+    _call(lib.la_forward_varlen, "la_forward_varlen", q.device,
+          _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(cu_seqlens), nseq, max_seqlen, T, _ptr(s_in), _ptr(z_in),
+          _ptr(res.get("s")), _ptr(res.get("z")), _ptr(res.get("den")), _ptr(workspace), wsb, H, dqk, dv, fmap, dt)
     return res
 
 
@@ -297,9 +304,9 @@ def la_forward_noalloc(q, k, v, fmap, *, state=False, den=False, out=None):
         res["z"] = torch.empty(B, H, F, dtype=torch.float32, device=q.device)
     if den:
         res["den"] = torch.empty(B, H, N, dtype=torch.float32, device=q.device)
-    _check(lib.la_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(res.get("s")), _ptr(res.get("z")),
-                                  _ptr(res.get("den")), B, H, N, dqk, dv, fmap, dt, _stream()),
-           "la_forward_noalloc")
+    _call(lib.la_forward_noalloc, "la_forward_noalloc", q.device,
+          _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(res.get("s")), _ptr(res.get("z")), _ptr(res.get("den")), B, H, N,
+          dqk, dv, fmap, dt)
     return res
 
 
@@ -318,8 +325,9 @@ def la_backward(q, k, v, dout, fmap, *, workspace=None):
     dq = torch.empty_like(q)
     dk = torch.empty_like(k)
     dvv = torch.empty_like(v)
-    _check(lib.la_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dvv),
-                           _ptr(workspace), wsb, B, H, N, dqk, dv, fmap, dt, _stream()), "la_backward")
+    _call(lib.la_backward, "la_backward", q.device,
+          _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dvv), _ptr(workspace), wsb, B, H, N, dqk,
+          dv, fmap, dt)
     return dq, dk, dvv
 
 
@@ -339,9 +347,9 @@ def la_backward_decay(q, k, v, log_decay, dout, fmap, *, workspace=None):
     _dev(q, k, v, dout, log_decay)
     dq, dk, dvv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     dg = torch.empty(B, H, N, dtype=torch.float32, device=q.device)
-    _check(lib.la_backward_decay(_ptr(q), _ptr(k), _ptr(v), _ptr(log_decay), _ptr(dout), _ptr(dq), _ptr(dk),
-                                 _ptr(dvv), _ptr(dg), _ptr(workspace), wsb, B, H, N, dqk, dv, fmap, dt, _stream()),
-           "la_backward_decay")
+    _call(lib.la_backward_decay, "la_backward_decay", q.device,
+          _ptr(q), _ptr(k), _ptr(v), _ptr(log_decay), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dvv), _ptr(dg),
+          _ptr(workspace), wsb, B, H, N, dqk, dv, fmap, dt)
     return dq, dk, dvv, dg
 
 
@@ -365,11 +373,11 @@ def la_decode_step(q, k, v, s, z, fmap, y=None, log_decay=None):
     if y is None:
         y = torch.empty(B, H, dv, dtype=q.dtype, device=q.device)
     if log_decay is not None:
-        _check(lib.la_decode_step_decay(_ptr(q), _ptr(k), _ptr(v), _ptr(log_decay), _ptr(y), _ptr(s), _ptr(z),
-                                        B, H, dqk, dv, fmap, dt, _stream()), "la_decode_step_decay")
+        _call(lib.la_decode_step_decay, "la_decode_step_decay", q.device,
+              _ptr(q), _ptr(k), _ptr(v), _ptr(log_decay), _ptr(y), _ptr(s), _ptr(z), B, H, dqk, dv, fmap, dt)
         return y
-    _check(lib.la_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(y), _ptr(s), _ptr(z), B, H, dqk, dv,
-                              fmap, dt, _stream()), "la_decode_step")
+    _call(lib.la_decode_step, "la_decode_step", q.device,
+          _ptr(q), _ptr(k), _ptr(v), _ptr(y), _ptr(s), _ptr(z), B, H, dqk, dv, fmap, dt)
     return y
 
 
@@ -388,8 +396,8 @@ def la_swa_forward(q, k, v, window, *, out=None, lse=False):
     res = {"o": o}
     if lse:
         res["lse"] = torch.empty(B, H, N, dtype=torch.float32, device=q.device)
-    _check(lib.la_swa_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(res.get("lse")), B, H, N, dqk, dv,
-                              int(window), _dtype_code(q), _stream()), "la_swa_forward")
+    _call(lib.la_swa_forward, "la_swa_forward", q.device,
+          _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(res.get("lse")), B, H, N, dqk, dv, int(window), _dtype_code(q))
     return res
 
 
@@ -408,8 +416,8 @@ def la_swa_cache_fill(k, v, window, *, k_cache=None, v_cache=None):
         k_cache = torch.zeros(B, H, window, dqk, dtype=k.dtype, device=k.device)
     if v_cache is None:
         v_cache = torch.zeros(B, H, window, dv, dtype=v.dtype, device=v.device)
-    _check(lib.la_swa_cache_fill(_ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), B, H, N, dqk, dv, int(window),
-                                 _dtype_code(k), _stream()), "la_swa_cache_fill")
+    _call(lib.la_swa_cache_fill, "la_swa_cache_fill", k.device,
+          _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), B, H, N, dqk, dv, int(window), _dtype_code(k))
     return k_cache, v_cache
 
 
@@ -430,8 +438,9 @@ def la_swa_decode_step(q, k, v, k_cache, v_cache, pos, window, y=None):
     _dev(q, k, v, k_cache, v_cache, pos, y)
     if y is None:
         y = torch.empty(B, H, dv, dtype=q.dtype, device=q.device)
-    _check(lib.la_swa_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(y), _ptr(k_cache), _ptr(v_cache), _ptr(pos),
-                                  B, H, dqk, dv, int(window), _dtype_code(q), _stream()), "la_swa_decode_step")
+    _call(lib.la_swa_decode_step, "la_swa_decode_step", q.device,
+          _ptr(q), _ptr(k), _ptr(v), _ptr(y), _ptr(k_cache), _ptr(v_cache), _ptr(pos), B, H, dqk, dv, int(window),
+          _dtype_code(q))
     return y
 
 
@@ -443,8 +452,8 @@ def la_feature_map(x, fmap):
     F = la_feature_dim(fmap, dqk)
     out = torch.empty(*x.shape[:-1], F, dtype=x.dtype, device=x.device)
     rows = x.numel() // dqk
-    _check(lib.la_feature_map(_ptr(x), _ptr(out), rows, dqk, fmap, _dtype_code(x), _stream()),
-           "la_feature_map")
+    _call(lib.la_feature_map, "la_feature_map", x.device,
+          _ptr(x), _ptr(out), rows, dqk, fmap, _dtype_code(x))
     return out
 
 
@@ -474,13 +483,15 @@ def kernel_plan(w):
     return {"launches_per_step": n, "kernels": names}
 
 
-def la_get_device_status():
-    """Synchronise the current stream and raise if a kernel recorded an error."""
-    _check(load_library().la_get_device_status(_stream()), "la_get_device_status")
+def la_get_device_status(device=None):
+    """Synchronise the current stream of `device` (default: the current CUDA
+    device) and raise if a kernel on that device recorded an error."""
+    _call(load_library().la_get_device_status, "la_get_device_status", _device(device))
 
 
-def la_selftest_bounded_wait(wait_us):
-    """Enqueue the library's failure-path self-test on the current stream: a
+def la_selftest_bounded_wait(wait_us, device=None):
+    """Enqueue the library's failure-path self-test on the current stream of
+    `device` (default: the current CUDA device): a
     wait of `wait_us` microseconds on an mbarrier nobody arrives on.  The
     following la_get_device_status raises LAError(LA_ERR_TIMEOUT)."""
-    _check(load_library().la_selftest_bounded_wait(int(wait_us), _stream()), "la_selftest_bounded_wait")
+    _call(load_library().la_selftest_bounded_wait, "la_selftest_bounded_wait", _device(device), int(wait_us))

@@ -71,6 +71,25 @@ la_status check_shape(int B, int H, int N, int dqk, int dv, int fmap, int dtype)
     return LA_OK;
 }
 
+// The kernels run on the calling thread's current device and dereference
+// the pointers they are given there.  A first operand that lives on another
+// device, or in host memory the device cannot address, is refused before any
+// launch (a launch would read another device's addresses through this one's
+// page tables).  Device memory of the current device and managed memory pass.
+la_status check_on_current_device(const void *p)
+{
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        (void)cudaGetLastError();   // the query's error is the caller's argument, not a sticky state
+        return LA_ERR_INVALID_ARG;
+    }
+    if (a.type == cudaMemoryTypeManaged) return LA_OK;
+    if (a.type != cudaMemoryTypeDevice) return LA_ERR_INVALID_ARG;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LA_ERR_CUDA;
+    return a.device == dev ? LA_OK : LA_ERR_INVALID_ARG;
+}
+
 la_status launch_status()
 {
     const cudaError_t e = cudaGetLastError();
@@ -627,6 +646,7 @@ static la_status forward_impl(const void *q, const void *k, const void *v, void 
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
         !aligned(s_out, 16) || !aligned(z_out, 4) || !aligned(den_out, 4))
         return LA_ERR_INVALID_ARG;
+    if (check_on_current_device(q) != LA_OK) return LA_ERR_INVALID_ARG;
     if (workspace_bytes < la_forward_workspace_bytes(B, H, N, dqk, dv, fmap, dtype))
         return LA_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
@@ -700,6 +720,7 @@ la_status la_forward_varlen(const void *q, const void *k, const void *v, void *o
     sh = check_shape(1, H, T, dqk, dv, fmap, dtype);   // element counts of the packed tensors
     if (sh != LA_OK) return sh;
     if (!q || !k || !v || !o || !cu_seqlens || !aligned(cu_seqlens, 4)) return LA_ERR_INVALID_ARG;
+    if (check_on_current_device(q) != LA_OK) return LA_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(s_out, 16) ||
         !aligned(z_out, 4) || !aligned(den_out, 4))
         return LA_ERR_INVALID_ARG;
@@ -775,6 +796,7 @@ la_status la_backward(const void *q, const void *k, const void *v, const void *d
     const la_status sh = check_shape(B, H, N, dqk, dv, fmap, dtype);
     if (sh != LA_OK) return sh;
     if (!q || !k || !v || !dout || !dq || !dk || !dvp || !workspace) return LA_ERR_INVALID_ARG;
+    if (check_on_current_device(q) != LA_OK) return LA_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(dout, 16) ||
         !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dvp, 16) || !aligned(workspace, 16))
         return LA_ERR_INVALID_ARG;
@@ -795,6 +817,7 @@ static la_status decode_impl(const void *q, const void *k, const void *v, const 
     const la_status sh = check_shape(B, H, 1, dqk, dv, fmap, dtype);
     if (sh != LA_OK) return sh;
     if (!q || !k || !v || !y || !s || !z) return LA_ERR_INVALID_ARG;
+    if (check_on_current_device(s) != LA_OK) return LA_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(y, 16) ||
         !aligned(s, 16) || !aligned(z, 4) || !aligned(g, 4))
         return LA_ERR_INVALID_ARG;
@@ -847,6 +870,7 @@ la_status la_backward_decay(const void *q, const void *k, const void *v, const f
     if (sh != LA_OK) return sh;
     if (!q || !k || !v || !log_decay || !dout || !dq || !dk || !dvp || !dlog_decay || !workspace)
         return LA_ERR_INVALID_ARG;
+    if (check_on_current_device(q) != LA_OK) return LA_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(dout, 16) || !aligned(dq, 16) ||
         !aligned(dk, 16) || !aligned(dvp, 16) || !aligned(log_decay, 4) || !aligned(dlog_decay, 4) ||
         !aligned(workspace, 4))
@@ -868,6 +892,7 @@ la_status la_forward_decay(const void *q, const void *k, const void *v, const fl
     const la_status sh = check_shape(B, H, N, dqk, dv, fmap, dtype);
     if (sh != LA_OK) return sh;
     if (!q || !k || !v || !o || !log_decay) return LA_ERR_INVALID_ARG;
+    if (check_on_current_device(q) != LA_OK) return LA_ERR_INVALID_ARG;
     const size_t need = la_forward_decay_workspace_bytes(B, H, N, dqk, dv, fmap, dtype);
     if (workspace_bytes < need || (need && (!workspace || !aligned(workspace, 16)))) return LA_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(log_decay, 4) ||
@@ -901,6 +926,7 @@ la_status la_swa_forward(const void *q, const void *k, const void *v, void *o, f
     if (!q || !k || !v || !o) return LA_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse_out, 4))
         return LA_ERR_INVALID_ARG;
+    if (check_on_current_device(q) != LA_OK) return LA_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
     const int BH = B * H;
     if (swa_tc_shape(dqk, dv, window, dtype)) {
@@ -938,6 +964,7 @@ la_status la_swa_cache_fill(const void *k, const void *v, void *k_cache, void *v
     const la_status sh = check_swa(B, H, N, dqk, dv, window, dtype);
     if (sh != LA_OK) return sh;
     if (!k || !v || !k_cache || !v_cache) return LA_ERR_INVALID_ARG;
+    if (check_on_current_device(k_cache) != LA_OK) return LA_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
     if (dtype == LA_F32)
         swa_cache_fill_kernel<float><<<B * H, 256, 0, st>>>((const float *)k, (const float *)v, (float *)k_cache,
@@ -955,6 +982,7 @@ la_status la_swa_decode_step(const void *q, const void *k, const void *v, void *
     const la_status sh = check_swa(B, H, 1, dqk, dv, window, dtype);
     if (sh != LA_OK) return sh;
     if (!q || !k || !v || !y || !k_cache || !v_cache || !pos || !aligned(pos, 4)) return LA_ERR_INVALID_ARG;
+    if (check_on_current_device(k_cache) != LA_OK) return LA_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
     const size_t bytes = sizeof(float) * ((size_t)window + dqk + 8);
     const float scale = (float)(1.0 / sqrt((double)dqk));
@@ -991,6 +1019,7 @@ la_status la_feature_map(const void *x, void *phi, int64_t rows, int dqk, int fm
     if (!valid_enums(fmap, dtype) || rows < 1 || dqk < 1) return LA_ERR_INVALID_ARG;
     if (!x || !phi) return LA_ERR_INVALID_ARG;
     if (!supported_dims(fmap, dqk, 1)) return LA_ERR_UNSUPPORTED;
+    if (check_on_current_device(x) != LA_OK) return LA_ERR_INVALID_ARG;
     const FmapParams fp = make_fmap(fmap, dqk);
     if (rows * fp.F >= ((int64_t)1 << 40)) return LA_ERR_INVALID_ARG;
     const int64_t total = rows * fp.F;
