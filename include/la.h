@@ -48,7 +48,10 @@
  *  - Pointers must be 16-byte aligned (z and den need only 4-byte alignment).
  *  - Argument errors are returned synchronously, before anything is launched:
  *    LA_ERR_INVALID_ARG (null required pointer, non-positive size, overflow,
- *    misalignment, workspace too small) or LA_ERR_UNSUPPORTED (a valid
+ *    misalignment, workspace too small, or a first tensor operand that is not
+ *    memory of the calling thread's current device -- another device's
+ *    memory or pageable host memory; the kernels run on the current device)
+ *    or LA_ERR_UNSUPPORTED (a valid
  *    combination this build has no kernel for).  A failed launch returns
  *    LA_ERR_CUDA.  Errors detected on the device (a bounded wait that ran out,
  *    a failed device-side check) are recorded in a per-device status word and
@@ -325,7 +328,10 @@ LA_API la_status la_swa_decode_step(const void *q, const void *k, const void *v,
  *     dqk = dv = 64 with B*H = 32 and N = 16384 needs 48 MB).
  *   - The first call on a device looks up the scratch array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is kept for the life of the
+ *     process: after cudaDeviceReset on a device the array goes with the old
+ *     context, and this entry point must not be called on that device again
+ *     in the same process.
  *   - All calls share the one array and it keeps the last call's contents.
  *     Nothing in it needs to start at zero (each call writes every value it
  *     later reads), but calls whose executions overlap on the GPU (on
