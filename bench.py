@@ -440,9 +440,12 @@ def capture(run, nsteps, stream):
     return g
 
 
-def timed(run, steps, warmup, dist_on, device_index, graph_len=None):
-    """Run warm-up, then exactly `steps` steps from CUDA graphs; returns
-    (ms per step max over ranks, clocks)."""
+def timed(run, steps, warmup, dist_on, device_index, graph_len=None, repeats=1):
+    """Run warm-up, then `repeats` timed regions of exactly `steps` steps each,
+    replayed from CUDA graphs, each bracketed by a barrier and a device
+    synchronisation and timed with CUDA events on the launching stream (max
+    over ranks).  Returns (median ms per step, [min, max] ms per step over the
+    repeats, clocks sampled over all of them)."""
     stream = torch.cuda.Stream()
     # eager warm-up: also configures kernels before any capture
     with torch.cuda.stream(stream):
@@ -459,23 +462,25 @@ def timed(run, steps, warmup, dist_on, device_index, graph_len=None):
     torch.cuda.synchronize()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
-    if dist_on:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
+    per_step = []
     with ClockSampler(device_index) as clk:
-        with torch.cuda.stream(stream):
-            start.record(stream)
-            for _ in range(full):
-                g.replay()
-            if gr is not None:
-                gr.replay()
-            end.record(stream)
-        torch.cuda.synchronize()
-    if dist_on:
-        torch.distributed.barrier()
-    ms = max_over_ranks(start.elapsed_time(end), dist_on, "cuda")
+        for _ in range(max(1, repeats)):
+            if dist_on:
+                torch.distributed.barrier()
+            torch.cuda.synchronize()
+            with torch.cuda.stream(stream):
+                start.record(stream)
+                for _ in range(full):
+                    g.replay()
+                if gr is not None:
+                    gr.replay()
+                end.record(stream)
+            torch.cuda.synchronize()
+            if dist_on:
+                torch.distributed.barrier()
+            per_step.append(max_over_ranks(start.elapsed_time(end), dist_on, "cuda") / steps)
     del g, gr
-    return ms / steps, clk.summary()
+    return statistics.median(per_step), [min(per_step), max(per_step)], clk.summary()
 
 
 def _e2e_buffers(w, dev, rank, nsets):
@@ -612,50 +617,82 @@ def e2e_prefill(w, dev, steps, warmup, dist_on=False, rank=0):
 
 # ----------------------------------------------------------------- CPU oracle
 
-def oracle_sample(w, heads=None, positions=None, min_cpu_s=0.0):
-    """Time the fp64 oracle on a bounded sample of workload w; returns
-    (tokens/s extrapolated to the full workload, seconds, description)."""
-    from oracle import oracle as orc
-    orc.build()
-    Hs = w.B * w.H if heads is None else heads
-    Ns = w.N if positions is None else positions
-    g = torch.Generator()
-    g.manual_seed(w.index)
-    mk = lambda d: (torch.randn(1, Hs, Ns, d, generator=g) * w.scale).to(w.torch_dtype)
-    q, k, v = mk(w.dqk), mk(w.dqk), mk(w.dv)
-    do = mk(w.dv) if w.backward else None
+class OracleSample:
+    """The fp64 oracle on a bounded sample of workload w: every one of the
+    B*H heads (so OpenMP has all of them to share out, as on the full
+    workload) for the first `positions` tokens (decode: that many one-token
+    steps from a zero state).  The recurrence's cost per head-token does not
+    depend on the position, so tokens/s scales to the full workload by the
+    head-token count."""
 
-    def once():
+    def __init__(self, w, positions):
+        from oracle import oracle as orc
+        orc.build()
+        self.orc, self.w = orc, w
+        self.full_positions = w.decode_steps if w.decode_steps else w.N
+        self.Ns = max(1, min(int(positions), self.full_positions))
+        Hs = w.B * w.H
+        g = torch.Generator()
+        g.manual_seed(w.index)
+        mk = lambda d: (torch.randn(1, Hs, self.Ns, d, generator=g) * w.scale).to(w.torch_dtype)
+        self.q, self.k, self.v = mk(w.dqk), mk(w.dqk), mk(w.dv)
+        self.do = mk(w.dv) if w.backward else None
+
+    def once(self):
+        orc, w = self.orc, self.w
+        q, k, v = self.q, self.k, self.v
         if w.backward:
             orc.forward_recurrent(w.fmap, q, k, v)
-            orc.backward_recurrent(w.fmap, q, k, v, do)
+            orc.backward_recurrent(w.fmap, q, k, v, self.do)
         elif w.decode_steps:
-            F = w.feature_dim
             import numpy as np
-            s = np.zeros((Hs, F, w.dv)); z = np.zeros((Hs, F))
-            for t in range(Ns):
+            s = np.zeros((w.B * w.H, w.feature_dim, w.dv))
+            z = np.zeros((w.B * w.H, w.feature_dim))
+            for t in range(self.Ns):
                 orc.decode_step(w.fmap, q[0, :, t], k[0, :, t], v[0, :, t], s, z)
         else:
             orc.forward_recurrent(w.fmap, q, k, v)
 
-    # repeat the sample until it amounts to about min_cpu_s of CPU time
+    def tokens_per_s(self, seconds_per_run):
+        """Tokens/s of the full workload (B sequences x all positions) at
+        this sample's speed."""
+        return self.w.B * self.Ns / seconds_per_run
+
+    def describe(self):
+        w = self.w
+        what = "decode steps" if w.decode_steps else "recurrent form" + (" + backward" if w.backward else "")
+        unit = "steps" if w.decode_steps else "positions"
+        return (f"fp64 oracle ({what}) on all {w.B * w.H} heads x {self.Ns} of {self.full_positions} {unit}; "
+                f"tokens/s scaled to the full workload by head-token count")
+
+
+def sized_oracle_sample(w, seconds):
+    """An OracleSample whose one run takes about `seconds` of wall time on
+    this host (at most the full workload), sized from a 32-position probe."""
+    probe = OracleSample(w, 32)
+    t0 = time.perf_counter()
+    probe.once()
+    dt = max(time.perf_counter() - t0, 1e-6)
+    return OracleSample(w, int(32 * seconds / dt))
+
+
+def oracle_baseline(w, min_cpu_s):
+    """(tokens/s, wall seconds, description): the full-workload oracle run
+    (or a sample of about 3 s wall per run) repeated until it has used about
+    `min_cpu_s` of CPU time."""
+    smp = sized_oracle_sample(w, 3.0)
     reps = 0
     t0 = time.perf_counter()
     c0 = time.process_time()
     while True:
-        once()
+        smp.once()
         reps += 1
         if time.process_time() - c0 >= min_cpu_s or time.perf_counter() - t0 >= 60:
             break
+    wall = time.perf_counter() - t0
     cpu_s = time.process_time() - c0
-    dt = (time.perf_counter() - t0) / reps
-    frac = (Hs * Ns) / (w.B * w.H * (w.decode_steps if w.decode_steps else w.N))
-    full_tokens = w.B * (w.decode_steps if w.decode_steps else w.N)
-    desc = (f"fp64 oracle ({'decode steps' if w.decode_steps else 'recurrent form'}"
-            f"{' + backward' if w.backward else ''}) on {Hs} of {w.B * w.H} heads x {Ns} positions; "
-            f"tokens/s scaled to the full workload by head-token count; {reps} repetitions, "
-            f"{cpu_s:.1f} s of CPU time over the oracle's threads")
-    return full_tokens * frac / dt, dt * reps, desc
+    desc = smp.describe() + f"; {reps} runs, {cpu_s:.1f} s of CPU time over the oracle's threads"
+    return smp.tokens_per_s(wall / reps), wall, desc
 
 
 def omp_threads():
@@ -673,29 +710,34 @@ def roofline_entry(bound, achieved, peak, unit, traffic):
 
 
 def run_reference(args):
-    """The oracle arm: rank 0 alone times the fp64 oracle; other ranks exit."""
+    """The oracle arm: rank 0 alone times the fp64 oracle; other ranks exit.
+    Each step is one run of the same all-head sample the other arm's
+    cpu_baseline uses (the full workload when one run of it takes a few
+    seconds at most), sized so that warm-up and steps together take about
+    two minutes."""
     _, rank, _ = rank_env()
     if rank != 0:
         return 0
     w = W.BY_NAME[args.workload]
-    # each step: a bounded sample (8 heads x 256 positions) of the workload
-    heads, pos = min(8, w.B * w.H), min(256, w.N)
-    vals = []
-    total = 0.0
+    per_step_s = min(3.0, 120.0 / (args.warmup + args.steps))
+    smp = sized_oracle_sample(w, per_step_s)
+    times = []
     for i in range(args.warmup + args.steps):
-        v, dt, desc = oracle_sample(w, heads=heads, positions=pos)
+        t0 = time.perf_counter()
+        smp.once()
         if i >= args.warmup:
-            vals.append(v)
-            total += dt
-    value = statistics.median(vals)
-    ms = total / max(1, args.steps) * 1e3
+            times.append(time.perf_counter() - t0)
+    sec = statistics.median(times)
+    value = smp.tokens_per_s(sec)
+    desc = smp.describe() + ", one run per step, median over the steps"
     line = {
         "impl": "reference", "metric": metric_name(w), "value": round(value, 2), "unit": "tokens/s",
-        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(sum(times) / len(times) * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": dict(base_config(w, args.gpus), timing="host wall clock, fp64 oracle"),
+        "data": "synthetic", "config": base_config(w, args.gpus), "timing": "host wall clock, fp64 oracle",
         "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": omp_threads(),
-                         "kind": "oracle", "sample": desc + " per step"},
+                         "kind": "oracle", "sample": desc},
         "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -710,6 +752,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="elu_bf16_fwd", choices=list(W.BY_NAME))
     ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--repeats", type=int, default=5,
+                    help="timed regions of --steps steps each; the line reports their median")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
     ap.add_argument("--profile-calls", type=int, default=0,
                     help="run this many untimed steps of --workload and exit (for ncu captures)")
@@ -743,63 +787,69 @@ def main():
         print(json.dumps({"profile_calls": args.profile_calls, "workload": w.describe(),
                           "kernels": la.kernel_plan(w)["kernels"]}), flush=True)
         return 0
-    ms, clocks = timed(run, args.steps, args.warmup, dist_on, local)
+    ms, spread, clocks = timed(run, args.steps, args.warmup, dist_on, local, repeats=args.repeats)
     value = whole_job_rate(run.tokens, world, ms)
-    kern_ms = ms  # one library launch per step for the prefill workloads
-    achieved = run.alg_bytes / (kern_ms * 1e-3) / 1e9
+    achieved = run.alg_bytes / (ms * 1e-3) / 1e9
+    from causal_kernelized_sequence_b200 import kernel_plan
+    kp = kernel_plan(w)
     line = {
         "metric": metric_name(w),
         "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 6), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if w.dtype == W.BF16 else "f32", "data": "synthetic",
-        "config": dict(base_config(w, world), l2=run.l2_note(),
-                       timing="CUDA graph of consecutive steps, CUDA events"),
-        "roofline": dict(roofline_entry("hbm", achieved, hbm, "GB/s",
-                                        load_traffic("forward:" + w.name)),
-                         peak_source=peak_kind, alg_bytes_per_launch=run.alg_bytes),
+        "config": base_config(w, world),
+        "repeats": args.repeats, "ms_per_step_min_max": [round(x, 6) for x in spread],
+        "timing": f"median of {args.repeats} timed regions of {args.steps} steps (CUDA graphs, CUDA events)",
+        "l2": run.l2_note(),
+        "roofline": dict(roofline_entry("hbm", achieved, hbm, "GB/s", load_traffic("forward:" + w.name)),
+                         peak_source=peak_kind, alg_bytes_per_step=run.alg_bytes,
+                         launches_per_step=kp["launches_per_step"]),
         "clocks": clocks,
-        "gpu_launches": None,
+        "gpu_launches": kp["launches_per_step"] * args.steps * args.repeats,
+        "kernels": kp["kernels"],
     }
     # e2e through the public API with host buffers
     if not w.decode_steps and not w.backward:
         e_ms, h2d, d2h, e_mode = e2e_prefill(w, dev, min(args.steps, 50), 3, dist_on, rank)
         line["e2e"] = {"value": round(whole_job_rate(run.tokens, world, e_ms), 1), "unit": "tokens/s",
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "mode": e_mode}
-    from causal_kernelized_sequence_b200 import kernel_plan
-    kp = kernel_plan(w)
-    line["gpu_launches"] = kp["launches_per_step"] * args.steps
-    line["kernels"] = kp["kernels"]
+
+    if rank == 0 and world == 1 and not args.no_cpu:
+        v, dt, desc = oracle_baseline(w, min_cpu_s=15.0)
+        line["cpu_baseline"] = {"value": round(v, 1), "unit": "tokens/s", "cores": omp_threads(),
+                                "kind": "oracle", "sample": desc + f" ({dt:.1f} s wall)"}
 
     if not args.no_secondary and world == 1:
+        # The other workloads, each with its own roofline.  Compact keys, and
+        # the configs with a published target last, so that a reader keeping
+        # only the end of the line still has them: v = tokens/s, ms = per step,
+        # hbm = fraction of measured HBM bandwidth on the algorithmic bytes,
+        # tc = fraction of measured dense bf16 peak on the algorithmic FLOPs,
+        # dram_x = DRAM bytes over algorithmic bytes (recorded ncu capture of
+        # the current code, else absent).
         sec = {}
-        for name in ("taylor_bf16_fwd", "elu_bf16_train", "taylor_decode", "taylor_decode_sym", "elu_bf16_varlen",
-                     "elu_bf16_decay_fwd", "swa_bf16_fwd", "swa_bf16_decode"):
+        for name in ("elu_bf16_varlen", "elu_bf16_decay_fwd", "swa_bf16_fwd", "swa_bf16_decode",
+                     "taylor_decode_sym", "taylor_decode", "elu_bf16_train", "taylor_bf16_fwd"):
             ws = W.BY_NAME[name]
             r2 = make_run(ws, dev, 0)
             st = 3 if ws.decode_steps else 50
-            ms2, clk2 = timed(r2, st, 3, False, local, graph_len=1 if ws.decode_steps else None)
-            v2 = r2.tokens / (ms2 * 1e-3)
-            ach = r2.alg_bytes / (ms2 * 1e-3) / 1e9
-            kp2 = kernel_plan(ws)
-            sec[name] = {"metric": metric_name(ws),
-                         "value": round(v2, 1), "unit": "tokens/s", "ms_per_step": round(ms2, 4),
-                         "steps": st, "config": ws.describe(), "l2": r2.l2_note(),
-                         "roofline": dict(roofline_entry("hbm", ach, hbm, "GB/s",
-                                                         load_traffic("step:" + name)),
-                                          alg_bytes_per_step=r2.alg_bytes,
-                                          tc_frac_alg=round(r2.alg_flops / (ms2 * 1e-3) / 1e12 /
-                                                            float(peaks["bf16_tflops"]), 4)),
-                         "clocks": clk2, "gpu_launches": kp2["launches_per_step"] * st,
-                         "kernels": kp2["kernels"]}
+            ms2, spread2, clk2 = timed(r2, st, 3, False, local, graph_len=1 if ws.decode_steps else None,
+                                       repeats=3)
+            ent = {"v": round(r2.tokens / (ms2 * 1e-3), 1), "ms": round(ms2, 4),
+                   "hbm": round(r2.alg_bytes / (ms2 * 1e-3) / 1e9 / hbm, 4),
+                   "tc": round(r2.alg_flops / (ms2 * 1e-3) / 1e12 / float(peaks["bf16_tflops"]), 4)}
+            tr = load_traffic("step:" + name)
+            if tr:
+                ent["dram_x"] = round(tr / r2.alg_bytes, 3)
+            sec[name] = ent
+            print(f"[bench] {ws.describe()}: {ent['v'] / 1e6:.2f} M tokens/s, {ms2:.4f} ms/step "
+                  f"(min {spread2[0]:.4f}, max {spread2[1]:.4f}), {ent['hbm'] * 100:.1f} % HBM, "
+                  f"{ent['tc'] * 100:.1f} % bf16 peak, clocks {clk2.get('sm_mhz')} MHz {clk2.get('reasons')}",
+                  file=sys.stderr, flush=True)
             del r2
             torch.cuda.empty_cache()
         line["workloads"] = sec
-
-    if rank == 0 and world == 1 and not args.no_cpu:
-        v, dt, desc = oracle_sample(w, min_cpu_s=15.0)
-        line["cpu_baseline"] = {"value": round(v, 1), "unit": "tokens/s", "cores": omp_threads(),
-                                "kind": "oracle", "sample": desc + f" ({dt:.1f} s wall)"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist_on:
