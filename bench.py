@@ -830,7 +830,7 @@ def main():
         # the current code, else absent).
         sec = {}
         for name in ("elu_bf16_varlen", "elu_bf16_decay_fwd", "swa_bf16_fwd", "swa_bf16_decode",
-                     "taylor_decode_sym", "taylor_decode", "elu_bf16_train", "taylor_bf16_fwd"):
+                     "taylor_decode_sym", "taylor_bf16_train", "taylor_decode", "elu_bf16_train", "taylor_bf16_fwd"):
             ws = W.BY_NAME[name]
             r2 = make_run(ws, dev, 0)
             st = 3 if ws.decode_steps else 50

@@ -184,10 +184,32 @@ int64_t tc_increment_floats(int dqk, int dv, int fmap)
     return (int64_t)FP * (dv + 16);
 }
 
+// Which tensor-core backward serves a shape: 0 none, 1 elu d = 128,
+// 2 elu d = 64, 3 Taylor d' = 16 with d_v = 64 (either Taylor map).
+int bwd_tc_kind(int dqk, int dv, int fmap, int dtype)
+{
+    if (dtype != LA_BF16) return 0;
+    if (fmap == LA_FMAP_ELU1 && dqk == 128 && dv == 128) return 1;
+    if (fmap == LA_FMAP_ELU1 && dqk == 64 && dv == 64) return 2;
+    if (fmap != LA_FMAP_ELU1 && dqk == 16 && dv == 64) return 3;
+    return 0;
+}
+
+// fp32 elements of one segment increment (S or R) of the tensor-core backward.
+size_t bwd_increment_floats(int kind)
+{
+    switch (kind) {
+    case 1: return (size_t)BwdCfg128::F * BwdCfg128::NA;
+    case 2: return (size_t)BwdCfg64::F * BwdCfg64::NA;
+    case 3: return (size_t)BwdCfgT16::F * BwdCfgT16::NA;
+    default: return 0;
+    }
+}
+
 Path select_backward(int B, int H, int N, int dqk, int dv, int fmap, int dtype)
 {
     if (check_shape(B, H, N, dqk, dv, fmap, dtype) != LA_OK) return Path::Invalid;
-    if (dtype == LA_BF16 && fmap == LA_FMAP_ELU1 && dqk == 128 && dv == 128) return Path::BwdTc;
+    if (bwd_tc_kind(dqk, dv, fmap, dtype)) return Path::BwdTc;
     return Path::BwdSimt;
 }
 
@@ -468,16 +490,17 @@ la_status forward_tc(const void *q, const void *k, const void *v, void *o, const
                                                       N, stream, false, cu, T, logdecay);
 }
 
+template <class Cfg>
 la_status backward_tc(const void *q, const void *k, const void *v, const void *dout, void *dq, void *dk,
                       void *dvp, void *workspace, int B, int H, int N, cudaStream_t stream)
 {
-    using Cfg = BwdCfg128;
     const int BH = B * H;
     CUtensorMap tq, tk, tv, tdo;
-    if (!make_map(&tq, q, 128, N, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&tk, k, 128, N, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&tv, v, 128, N, BH, 16, CU_TENSOR_MAP_SWIZZLE_32B) ||
-        !make_map(&tdo, dout, 128, N, BH, 16, CU_TENSOR_MAP_SWIZZLE_32B))
+    const int qbox = Cfg::TAYLOR ? 16 : 64;
+    const CUtensorMapSwizzle qsw = Cfg::TAYLOR ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_128B;
+    if (!make_map(&tq, q, Cfg::D, N, BH, qbox, qsw) || !make_map(&tk, k, Cfg::D, N, BH, qbox, qsw) ||
+        !make_map(&tv, v, Cfg::DV, N, BH, 16, CU_TENSOR_MAP_SWIZZLE_32B) ||
+        !make_map(&tdo, dout, Cfg::DV, N, BH, 16, CU_TENSOR_MAP_SWIZZLE_32B))
         return LA_ERR_CUDA;
     BwdParams p;
     tc_segments(B, H, N, &p.P, &p.cps, &p.nchunks);
@@ -490,21 +513,27 @@ la_status backward_tc(const void *q, const void *k, const void *v, const void *d
     p.dq = dq;
     p.dk = dk;
     p.dv = dvp;
-    if (set_smem<bwd_sstate_kernel>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
+    const double d = (double)Cfg::D;
+    p.inv_c1 = (float)(1.0 / pow(d, 0.25));
+    p.inv_c2 = (float)(1.0 / (sqrt(2.0) * sqrt(d)));
+    p.inv_c3 = (float)(1.0 / sqrt(d));
+    p.k2 = (float)(1.0 / (2.0 * d));
+    if (set_smem<bwd_sstate_kernel<Cfg>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
     if (p.P > 1) {
-        bwd_sstate_kernel<<<BH * p.P, 128, Cfg::SMEM_ALLOC, stream>>>(tk, tv, p);
+        bwd_sstate_kernel<Cfg><<<BH * p.P, 128, Cfg::SMEM_ALLOC, stream>>>(tk, tv, p);
         if (launch_status() != LA_OK) return LA_ERR_CUDA;
     }
-    if (set_smem<bwd_dq_kernel>(Cfg::SMEM_ALLOC) != LA_OK || set_smem<bwd_dkdv_kernel>(Cfg::SMEM_ALLOC) != LA_OK ||
-        set_smem<bwd_rstate_kernel>(Cfg::SMEM_ALLOC) != LA_OK)
+    if (set_smem<bwd_dq_kernel<Cfg>>(Cfg::SMEM_ALLOC) != LA_OK ||
+        set_smem<bwd_dkdv_kernel<Cfg>>(Cfg::SMEM_ALLOC) != LA_OK ||
+        set_smem<bwd_rstate_kernel<Cfg>>(Cfg::SMEM_ALLOC) != LA_OK)
         return LA_ERR_CUDA;
-    bwd_dq_kernel<<<BH * p.P, 256, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, p);
+    bwd_dq_kernel<Cfg><<<BH * p.P, 256, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, p);
     if (launch_status() != LA_OK) return LA_ERR_CUDA;
     if (p.P > 1) {
-        bwd_rstate_kernel<<<BH * p.P, 128, Cfg::SMEM_ALLOC, stream>>>(tq, tdo, p);
+        bwd_rstate_kernel<Cfg><<<BH * p.P, 128, Cfg::SMEM_ALLOC, stream>>>(tq, tdo, p);
         if (launch_status() != LA_OK) return LA_ERR_CUDA;
     }
-    bwd_dkdv_kernel<<<BH * p.P, 256, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, p);
+    bwd_dkdv_kernel<Cfg><<<BH * p.P, 256, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, p);
     return launch_status();
 }
 
@@ -630,7 +659,8 @@ size_t la_backward_workspace_bytes(int B, int H, int N, int dqk, int dv, int fma
     if (path == Path::BwdTc) {
         int P, cps, nc;
         tc_segments(B, H, N, &P, &cps, &nc);
-        if (P > 1) bytes += 2 * (size_t)B * H * P * BwdCfg128::F * BwdCfg128::NA * sizeof(float);  // S, R increments
+        if (P > 1) bytes += 2 * (size_t)B * H * P * bwd_increment_floats(bwd_tc_kind(dqk, dv, fmap, dtype)) *
+                                sizeof(float);   // S, R increments
     }
     return bytes;
 }
@@ -804,8 +834,12 @@ la_status la_backward(const void *q, const void *k, const void *v, const void *d
         return LA_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
     float *ws = (float *)workspace;
-    if (select_backward(B, H, N, dqk, dv, fmap, dtype) == Path::BwdTc)
-        return backward_tc(q, k, v, dout, dq, dk, dvp, workspace, B, H, N, s);
+    switch (select_backward(B, H, N, dqk, dv, fmap, dtype) == Path::BwdTc ? bwd_tc_kind(dqk, dv, fmap, dtype) : 0) {
+    case 1: return backward_tc<BwdCfg128>(q, k, v, dout, dq, dk, dvp, workspace, B, H, N, s);
+    case 2: return backward_tc<BwdCfg64>(q, k, v, dout, dq, dk, dvp, workspace, B, H, N, s);
+    case 3: return backward_tc<BwdCfgT16>(q, k, v, dout, dq, dk, dvp, workspace, B, H, N, s);
+    default: break;
+    }
     if (dtype == LA_F32)
         return backward_simt<float>(q, k, v, dout, dq, dk, dvp, ws, B, H, N, dqk, dv, fmap, s);
     return backward_simt<__nv_bfloat16>(q, k, v, dout, dq, dk, dvp, ws, B, H, N, dqk, dv, fmap, s);

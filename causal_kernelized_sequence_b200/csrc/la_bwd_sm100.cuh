@@ -1,5 +1,8 @@
-// la_bwd_sm100.cuh -- tensor-core backward of causal linear attention for the
-// elu(x)+1 map with d_qk = d_v = 128 (bf16 I/O), tcgen05 + TMA.
+// la_bwd_sm100.cuh -- tensor-core backward of causal linear attention (bf16
+// I/O), tcgen05 + TMA, for three shapes: the elu(x)+1 map with
+// d_qk = d_v = 128 or 64, and the BASED second-order Taylor map with d' = 16
+// and d_v = 64 (both the full and the folded map: their phi(q).phi(k) and so
+// their gradients are the same).
 //
 // The pages give no backward pass; this is the derivative of the BASED page's
 // Knowl 3 parallel form, computed chunk by chunk (128 tokens) with the same
@@ -12,15 +15,23 @@
 //     A   = phi(Q) phi(K)^T, P = A masked to j <= i
 //     O   = P V_aug + phi(Q) S_aug          -> y, den; G'' = den G' = [dO | -dO.y]
 //     dA  = G'' V_aug^T,  dP = dA masked to j <= i
-//     dphi(Q) = (dP phi(K) + G'' S_aug^T) / den   -> dq = dphi(Q) * elu'(q)
+//     dphi(Q) = (dP phi(K) + G'' S_aug^T) / den   -> dq = J_phi(q)^T dphi(q)
 //     S_aug += phi(K)^T V_aug
 //   reverse-order pass (dk, dv):
 //     A^T = phi(K) phi(Q)^T, P^T; dA^T = V_aug G'^T, dP^T (masked to i >= j)
 //     dV  = P^T G + phi(K) R                 (R = first d_v columns of R_aug)
-//     dphi(K) = dP^T phi(Q) + V_aug R_aug^T  -> dk = dphi(K) * elu'(k)
+//     dphi(K) = dP^T phi(Q) + V_aug R_aug^T  -> dk = J_phi(k)^T dphi(k)
 //     R_aug += phi(Q)^T G'
 //
-// elu'(x) = 1 for x > 0 and exp(x) = phi(x) otherwise, i.e. min(phi(x), 1).
+// The maps.  elu: J_phi(x)^T is the diagonal elu'(x) = 1 for x > 0 and
+// exp(x) = phi(x) otherwise, i.e. min(phi(x), 1).  Taylor: the scores come
+// from the raw Q K^T (K = 16) through the closed form
+// 1 + s/sqrt(d') + s^2/(2 d') (BASED page, Knowl 3), and phi is the folded
+// map's 153 features (padded to 160 with zeros) in a separate shared-memory
+// tile; J_phi(x)^T dphi maps the 160 feature derivatives back to the 16
+// coordinates on the CUDA cores (linear features 1/d'^(1/4), squares
+// 2 x_a / (sqrt2 sqrt d'), pairs x_b / sqrt(d') and x_a / sqrt(d')).
+//
 // den and dden are recomputed in fp32 in the forward-order pass (so no
 // rounded forward output enters the gradient) and kept per token in the
 // workspace for the reverse pass.  Sequences are split into the forward's
@@ -31,17 +42,30 @@
 // dphi(Q) is replaced by its component orthogonal to phi(q_i) before the
 // chain rule.  That is exact: y_i is unchanged when phi(q_i) is scaled, so
 // dphi(q_i) . phi(q_i) = 0 in exact arithmetic and only rounding noise is
-// removed (elu features are all ~1, so that noise is large next to dq).
-// The reverse pass uses bf16 operands, with P^T and G' each split into a
-// bf16 head and a bf16 remainder on the products that carry dk.
+// removed (elu features are all ~1, so that noise is large next to dq).  For
+// the Taylor map the projection is applied after the chain rule, with
+// |phi(x)|^2 = 1 + |x|^2/sqrt(d') + |x|^4/(2 d') and
+// J_phi(x)^T phi(x) = x (1/sqrt(d') + |x|^2/d') in closed form.
+// The elu forward-order pass runs its MMAs on fp16 operands (phi - 1 carries
+// dq and keeps 3 more bits in fp16); the Taylor map, whose features are not
+// clustered near one value, runs on bf16 with a bf16 remainder on the state
+// and on G'' for the inter-chunk term.  The reverse pass uses bf16 operands,
+// with P^T and G' each split into a bf16 head and a bf16 remainder on the
+// products that carry dk.
 //
-// Token or feature row i <-> TMEM lane i.  bwd_dq_kernel and bwd_dkdv_kernel
-// run 256 threads: warps w and w + 4 share the lanes of one 32-row quadrant
-// and split every per-row step by columns, exchanging row reductions through
-// shared memory.  bwd_sstate_kernel and bwd_rstate_kernel run 128 threads, one
-// per row, and load the next chunk while the current one is summed.  Each
-// block takes a chunk's steps in order; every mbarrier wait is bounded.
+// Token or feature row i <-> TMEM lane i.  The Taylor state (160 feature
+// rows) is two TMEM tiles, M = 128 (features 0..127) and M = 64 (features
+// 128..191, of which 128..159 are kept: row 128 + 16 q + l in lane 32 q + l,
+// l < 16); the elu d = 64 state is one M = 64 tile in the same layout.
+// bwd_dq_kernel and bwd_dkdv_kernel run 256 threads: warps w and w + 4 share
+// the lanes of one 32-row quadrant and split every per-row step by columns,
+// exchanging row reductions through shared memory.  bwd_sstate_kernel and
+// bwd_rstate_kernel run 128 threads, one per row, and load the next chunk
+// while the current one is summed.  Each block takes a chunk's steps in
+// order; every mbarrier wait is bounded.
 #pragma once
+
+#include <type_traits>
 
 #include "la_device.cuh"
 #include "la_prefill_sm100.cuh"
@@ -49,31 +73,69 @@
 
 namespace la {
 
-struct BwdCfg128 {
-    static constexpr int C = 128, D = 128, DV = 128, NA = 144, F = 128;
-    static constexpr int QK_TILE = C * D * 2;            // 32 KB (two 64-column SW128 blocks)
-    static constexpr int BLK = C * 32;                   // 4 KB: one 16-column SW32 block of 128 rows
-    static constexpr int VG_TILE = (NA / 16) * BLK;      // 36 KB: V_aug or G'
-    static constexpr int S_BLK = F * 32;                 // 4 KB: 16 columns of the F x NA state
-    static constexpr int S_TILE = (NA / 16) * S_BLK;     // 36 KB
+template <int D_, int DV_, bool TAYLOR_>
+struct BwdCfg {
+    static constexpr int D = D_, DV = DV_;
+    static constexpr bool TAYLOR = TAYLOR_;
+    static constexpr bool F16 = !TAYLOR;                 // fp16 operands in the forward-order pass
+    static constexpr int C = 128;
+    static constexpr int NA = DV + 16;                   // value columns + normaliser block
+    static constexpr int F = TAYLOR ? 160 : D;           // feature rows of the state
+    static constexpr int FT = TAYLOR ? 192 : D;          // width of a phi tile (64-feature SW128 blocks)
+    static constexpr int NT = TAYLOR ? 2 : 1;            // state tiles in TMEM
+    static __host__ __device__ constexpr int tile_m(int t) { return TAYLOR ? (t == 0 ? 128 : 64) : (D == 128 ? 128 : 64); }
+    static __host__ __device__ constexpr int tile_f0(int t) { return 128 * t; }
+    static constexpr int NA_SPLIT = ((NA / 16 + 1) / 2) * 16;   // a row's first thread takes columns [0, NA_SPLIT)
+    // shared memory (bytes; SW128 regions 1024-aligned, SW32 regions 256-aligned)
+    static constexpr int PHI_TILE = C * FT * 2;          // phi(Q) or phi(K) (elu: the loaded tile, phi in place)
+    static constexpr int RAW = TAYLOR ? C * 32 : 0;      // raw Q or K tile (Taylor, one 16-column SW32 block)
+    static constexpr int BLK = C * 32;                   // one 16-column SW32 block of 128 rows
+    static constexpr int VG_TILE = (NA / 16) * BLK;      // V_aug or G'
+    static constexpr int S_BLK = F * 32;                 // 16 columns of the F x NA state
+    static constexpr int S_TILE = (NA / 16) * S_BLK;
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = OFF_Q + QK_TILE;
-    static constexpr int OFF_V = OFF_K + QK_TILE;
+    static constexpr int OFF_K = OFF_Q + PHI_TILE;
+    static constexpr int OFF_V = OFF_K + PHI_TILE;
     static constexpr int OFF_G = OFF_V + VG_TILE;
     static constexpr int OFF_S = OFF_G + VG_TILE;
-    static constexpr int OFF_SL = OFF_S + S_TILE;        // low bf16 part of the state (forward-order pass)
-    static constexpr int OFF_BAR = OFF_SL + S_TILE;
-    static constexpr int OFF_RED = OFF_BAR + 128;        // forward-order pass: per-row partial sums of its two threads
-    static constexpr int SMEM_ALLOC = OFF_RED + 3 * 2 * C * 4 + 1024;
+    static constexpr int OFF_SL = OFF_S + S_TILE;        // low part of the state (forward-order pass) or of G'
+    static constexpr int OFF_RQ = OFF_SL + S_TILE;       // raw Q (Taylor)
+    static constexpr int OFF_RK = OFF_RQ + RAW;          // raw K (Taylor)
+    static constexpr int OFF_BAR = OFF_RK + RAW;
+    static constexpr int OFF_RED = OFF_BAR + 128;        // per-row partial sums of the two threads of a row
+    static constexpr int RED_FLOATS = 6 * C + (TAYLOR ? 2 * C * 16 : 0);
+    static constexpr int SMEM_ALLOC = OFF_RED + RED_FLOATS * 4 + 1024;
+    // TMEM columns.  Forward-order pass: [0, 128) scores -> P | dP; X: O_aug,
+    // then dA, then dphi(Q); S: the state tiles; GL: the remainder of G''.
+    // Reverse pass: [0, 128) scores -> P^T | dP^T; X: dA^T, then dV, then
+    // dphi(K); R: the R_aug tiles; PL: the remainder of dP^T.
+    static constexpr int cmax(int a, int b) { return a > b ? a : b; }
+    static constexpr int COL_X = C;
+    static constexpr int COL_S = COL_X + cmax(cmax(NA, C), F);
+    static constexpr int COL_GL = COL_S + NT * NA;
+    static constexpr int COL_R = COL_X + cmax(cmax(C, DV), F);
+    static constexpr int COL_PL = COL_R + NT * NA;
     static constexpr int TMEM_COLS = 512;
+    static_assert(COL_GL + NA / 2 <= 512 && COL_PL + C / 2 <= 512, "TMEM columns");
+    static_assert(NT * NA <= 256, "state tiles of the state passes");
+    static_assert(PHI_TILE % 1024 == 0 && VG_TILE % 1024 == 0 && S_TILE % 256 == 0 && OFF_RQ % 1024 == 0,
+                  "shared-memory alignment");
+    static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory");
 };
+
+using BwdCfg128 = BwdCfg<128, 128, false>;
+using BwdCfg64 = BwdCfg<64, 64, false>;
+using BwdCfgT16 = BwdCfg<16, 64, true>;
 
 struct BwdParams {
     float *dd;            // [BH, N, 2]: den_i, dden_i
     float *ws_s;          // [BH, P, F, NA] state increments per segment
     float *ws_r;          // [BH, P, F, NA] R increments per segment
-    void *dq, *dk, *dv;   // [BH, N, D] bf16
+    void *dq, *dk, *dv;   // [BH, N, D] / [BH, N, DV] bf16
     int N, P, nchunks, cps;
+    // Taylor map: 1/d'^(1/4), 1/(sqrt2 sqrt d'), 1/sqrt(d') (pair features and
+    // the score's linear term), 1/(2 d') (its square term)
+    float inv_c1, inv_c2, inv_c3, k2;
 };
 
 namespace bwd_detail {
@@ -411,24 +473,233 @@ __device__ __forceinline__ void mask_pack_row_hilo(uint32_t src, uint32_t dst_hi
     tmem_st_wait();
 }
 
+// ---- state tiles
+
+// Feature row held by lane l of quadrant wq in state tile t, or -1 (M = 128:
+// row = lane; M = 64: row 16 wq + l in lane 32 wq + l, l < 16).
+template <class Cfg>
+__device__ __forceinline__ int state_row(int t, int wq, int l)
+{
+    const int f = Cfg::tile_m(t) == 128 ? Cfg::tile_f0(t) + 32 * wq + l
+                                        : (l < 16 ? Cfg::tile_f0(t) + 16 * wq + l : Cfg::F);
+    return f < Cfg::F ? f : -1;
+}
+
+// Whether quadrant wq holds a kept row of state tile t (warp-uniform).
+template <class Cfg>
+__device__ __forceinline__ bool state_quadrant(int t, int wq)
+{
+    return Cfg::tile_f0(t) + (Cfg::tile_m(t) == 128 ? 32 : 16) * wq < Cfg::F;
+}
+
+// bf16 or fp16 pair, as the pass's MMA kind wants.
+template <bool F16>
+__device__ __forceinline__ uint32_t pack2(float a, float b)
+{
+    if constexpr (F16) return pack_f16(a, b);
+    else return pack_bf16(a, b);
+}
+
+// Row r of a 16-column SW32 block of 128 rows: [first, 0, ..., 0].
+template <bool F16>
+__device__ __forceinline__ void write_first(uint8_t *blk, int r, float first)
+{
+    if constexpr (F16) write_first_f16(blk, r, first);
+    else write_dden(blk, r, first);
+}
+
+// Masked scores of this thread's 64 columns from j0, packed as pairs at
+// dst + j0/2.  With `aliased` the packed columns may overlap source columns
+// the other thread of the row has not read yet, so the whole block meets at
+// a barrier between the loads and the stores (every thread must call this).
+// With TAY the raw scores s become 1 + s k1 + s^2 k2 first.
+template <bool F16, bool TAY, typename Keep>
+__device__ __forceinline__ void mask_pack_half_g(uint32_t src, uint32_t dst, int j0, bool aliased, float k1, float k2,
+                                                 Keep keep)
+{
+    float a[64];
+    tmem_ld32(src + j0, a);
+    tmem_ld32(src + j0 + 32, a + 32);
+    tmem_ld_wait();
+    if (aliased) {
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
+    if constexpr (TAY) {
+#pragma unroll
+        for (int e = 0; e < 64; ++e) a[e] = fmaf(a[e], fmaf(a[e], k2, k1), 1.f);
+    }
+    uint32_t pk[32];
+#pragma unroll
+    for (int e = 0; e < 64; e += 2) pk[e / 2] = pack2<F16>(keep(j0 + e) ? a[e] : 0.f, keep(j0 + e + 1) ? a[e + 1] : 0.f);
+    tmem_st32(dst + j0 / 2, pk);
+    tmem_st_wait();
+}
+
+// ---- the Taylor map, d' = 16: the folded features packed to 160
+//   0: 1;  1..16: x_a / d'^(1/4);  17..32: x_a^2 / (sqrt2 sqrt d');
+//   33..152: x_a x_b / sqrt(d'), a < b, row-major pairs;  153..159: 0.
+
+__host__ __device__ constexpr int tay_kind(int f) { return f == 0 ? 0 : f <= 16 ? 1 : f <= 32 ? 2 : f < 153 ? 3 : 4; }
+__host__ __device__ constexpr int tay_a(int f)
+{
+    if (f <= 16) return f - 1;
+    if (f <= 32) return f - 17;
+    int p = f - 33, a = 0;
+    while (p >= 15 - a) {
+        p -= 15 - a;
+        ++a;
+    }
+    return a;
+}
+__host__ __device__ constexpr int tay_b(int f)
+{
+    int p = f - 33, a = 0;
+    while (p >= 15 - a) {
+        p -= 15 - a;
+        ++a;
+    }
+    return a + 1 + p;
+}
+
+template <int f>
+__device__ __forceinline__ float tay_feat(const float *x, const BwdParams &p)
+{
+    constexpr int kind = tay_kind(f);
+    if constexpr (kind == 0) return 1.f;
+    else if constexpr (kind == 1) return x[tay_a(f)] * p.inv_c1;
+    else if constexpr (kind == 2) return x[tay_a(f)] * x[tay_a(f)] * p.inv_c2;
+    else if constexpr (kind == 3) return x[tay_a(f)] * x[tay_b(f)] * p.inv_c3;
+    else return 0.f;
+}
+
+template <int F0>
+__device__ __forceinline__ uint4 tay_feat8(const float *x, const BwdParams &p)
+{
+    return make_uint4(pack_bf16(tay_feat<F0>(x, p), tay_feat<F0 + 1>(x, p)),
+                      pack_bf16(tay_feat<F0 + 2>(x, p), tay_feat<F0 + 3>(x, p)),
+                      pack_bf16(tay_feat<F0 + 4>(x, p), tay_feat<F0 + 5>(x, p)),
+                      pack_bf16(tay_feat<F0 + 6>(x, p), tay_feat<F0 + 7>(x, p)));
+}
+
+template <int FB, int... G>
+__device__ __forceinline__ void tay_phi_groups(uint32_t tile, int r, const float *x, bool zero, const BwdParams &p,
+                                               std::integer_sequence<int, G...>)
+{
+    ((sts128(tile + sw128_off(r, FB + 8 * G), zero ? make_uint4(0u, 0u, 0u, 0u) : tay_feat8<FB + 8 * G>(x, p))), ...);
+}
+
+// Features [FB, FB + 8 NG) of row r of a phi tile (SW128 blocks of 64
+// features), from the raw row x; zeros when `zero`.
+template <int FB, int NG>
+__device__ __forceinline__ void tay_phi_row(uint32_t tile, int r, const float *x, bool zero, const BwdParams &p)
+{
+    tay_phi_groups<FB>(tile, r, x, zero, p, std::make_integer_sequence<int, NG>{});
+}
+
+// Row r's 16 raw values from a [128 x 16] bf16 SW32 tile.
+__device__ __forceinline__ void raw_row16(uint32_t tile, int r, float *x)
+{
+    unpack8(lds128(tile + sw32_off(r, 0, 128)), x);
+    unpack8(lds128(tile + sw32_off(r, 8, 128)), x + 8);
+}
+
+// dx += J_phi(x)^T e_f g (the derivative of feature f, weighted by g), and
+// sd += g phi_f(x).
+template <int f>
+__device__ __forceinline__ void tay_vjp_one(float g, const float *x, float *dx, float &sd, const BwdParams &p)
+{
+    constexpr int kind = tay_kind(f);
+    if constexpr (kind == 0) {
+        sd += g;
+    } else if constexpr (kind == 1) {
+        constexpr int a = tay_a(f);
+        dx[a] = fmaf(g, p.inv_c1, dx[a]);
+        sd = fmaf(g, x[a] * p.inv_c1, sd);
+    } else if constexpr (kind == 2) {
+        constexpr int a = tay_a(f);
+        const float gx = g * x[a] * p.inv_c2;
+        dx[a] = fmaf(2.f, gx, dx[a]);
+        sd = fmaf(gx, x[a], sd);
+    } else if constexpr (kind == 3) {
+        constexpr int a = tay_a(f), b = tay_b(f);
+        const float gc = g * p.inv_c3;
+        dx[a] = fmaf(gc, x[b], dx[a]);
+        dx[b] = fmaf(gc, x[a], dx[b]);
+        sd = fmaf(gc * x[a], x[b], sd);
+    }
+}
+
+template <int F0, int... E>
+__device__ __forceinline__ void tay_vjp_seq(const float *g, const float *x, float *dx, float &sd, const BwdParams &p,
+                                            std::integer_sequence<int, E...>)
+{
+    (tay_vjp_one<F0 + E>(g[E], x, dx, sd, p), ...);
+}
+
+template <int F0>
+__device__ __forceinline__ void tay_vjp16(uint32_t tcol, const float *x, float *dx, float &sd, const BwdParams &p)
+{
+    float g[16];
+    tmem_ld16(tcol + F0, g);
+    tmem_ld_wait();
+    tay_vjp_seq<F0>(g, x, dx, sd, p, std::make_integer_sequence<int, 16>{});
+}
+
+template <int FB, int... G>
+__device__ __forceinline__ void tay_vjp_groups(uint32_t tcol, const float *x, float *dx, float &sd, const BwdParams &p,
+                                               std::integer_sequence<int, G...>)
+{
+    (tay_vjp16<FB + 16 * G>(tcol, x, dx, sd, p), ...);
+}
+
+// J_phi(x)^T dphi over features [80 HALF, 80 HALF + 80), dphi read from TMEM
+// columns tcol + f; also sd = dphi . phi(x) over the same features.
+template <int HALF>
+__device__ __forceinline__ void tay_vjp_half(uint32_t tcol, const float *x, float *dx, float &sd, const BwdParams &p)
+{
+    tay_vjp_groups<80 * HALF>(tcol, x, dx, sd, p, std::make_integer_sequence<int, 5>{});
+}
+
+// The two threads of row i combine their halves of J^T dphi (and of
+// dphi . phi) through shared memory; thread hh gets coordinates 8 hh .. 8 hh + 7
+// of the whole.  Every thread of the block must call this.
+__device__ __forceinline__ void tay_combine(float *xred, float *sred, int hh, int i, const float *dx, float sd,
+                                            float *out8, float &sd_all)
+{
+    float *mine = xred + (hh * 128 + i) * 16;
+#pragma unroll
+    for (int c = 0; c < 16; c += 4) *reinterpret_cast<float4 *>(mine + c) = make_float4(dx[c], dx[c + 1], dx[c + 2], dx[c + 3]);
+    sred[hh * 128 + i] = sd;
+    __syncthreads();
+    const float *a = xred + i * 16 + 8 * hh, *b = xred + (128 + i) * 16 + 8 * hh;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) out8[c] = a[c] + b[c];
+    sd_all = sred[i] + sred[128 + i];
+}
+
 }  // namespace bwd_detail
 
 // ---------------------------------------------------------------------------
 // Forward-order pass: dq, and den_i, dden_i per token.
 //
-// Its MMAs run on fp16 operands (A and B both fp16), not bf16: dq is carried
-// by phi - 1, which is ~0.1 for small inputs, and bf16 keeps only ~5 bits of
-// it (relative error ~2/|phi - 1| x 2^-9 in dq); fp16 keeps 3 more.  V is
-// converted exactly; the state snapshot and G' keep an extra fp16 remainder
+// elu: the MMAs run on fp16 operands (A and B both fp16), not bf16: dq is
+// carried by phi - 1, which is ~0.1 for small inputs, and bf16 keeps only ~5
+// bits of it (relative error ~2/|phi - 1| x 2^-9 in dq); fp16 keeps 3 more.
+// V is converted exactly; the state snapshot and G'' keep an extra remainder
 // for the inter-chunk term, and dphi(q) is projected orthogonal to phi(q).
+// Taylor: the same steps on bf16 operands, with the raw scores and the
+// feature-to-coordinate chain rule described at the top of the file.
+template <class Cfg>
 __global__ void __launch_bounds__(256, 1)
 bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
               const BwdParams p)
 {
     using namespace bwd_detail;
-    using Cfg = BwdCfg128;
-    constexpr int C = Cfg::C, D = Cfg::D, DV = Cfg::DV, NA = Cfg::NA, F = Cfg::F;
+    constexpr int C = Cfg::C, D = Cfg::D, DV = Cfg::DV, NA = Cfg::NA, F = Cfg::F, NT = Cfg::NT;
+    constexpr bool TAY = Cfg::TAYLOR, F16 = Cfg::F16;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *tma_bar = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
@@ -437,16 +708,16 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tma_bar + 3);
     // 256 threads: warps w and w + 4 share the TMEM lanes of rows 32 (w % 4) ..
     // + 31 and split every per-row step by columns; row sums meet in red[]
-    const int tid = threadIdx.x, warp = tid >> 5, wq = warp & 3, hh = warp >> 2;
-    const int row = wq * 32 + (tid & 31);
-    float *red = reinterpret_cast<float *>(smem + Cfg::OFF_RED);   // [3][2][C]
+    const int tid = threadIdx.x, warp = tid >> 5, wq = warp & 3, hh = warp >> 2, l = tid & 31;
+    const int row = wq * 32 + l;
+    float *red = reinterpret_cast<float *>(smem + Cfg::OFF_RED);   // [3][2][C], then (Taylor) [2][C][16]
     const int bh = blockIdx.x / p.P, seg = blockIdx.x % p.P;
     const int c_begin = seg * p.cps, c_end = min(p.nchunks, c_begin + p.cps);
     const int N = p.N;
     uint8_t *sQ = smem + Cfg::OFF_Q, *sK = smem + Cfg::OFF_K, *sV = smem + Cfg::OFF_V, *sG = smem + Cfg::OFF_G,
             *sS = smem + Cfg::OFF_S, *sSL = smem + Cfg::OFF_SL;
     const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV), aG = smem_addr(sG), aS = smem_addr(sS),
-                   aSL = smem_addr(sSL);
+                   aSL = smem_addr(sSL), aRQ = smem_addr(smem + Cfg::OFF_RQ), aRK = smem_addr(smem + Cfg::OFF_RK);
 
     if (tid == 0) {
         mbar_init(tma_bar, 1);
@@ -455,28 +726,41 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         mbar_init_fence();
     }
     if (warp == 0) tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
-    if (hh == 0) write_first_f16(sV + (DV / 16) * Cfg::BLK, row, 1.f);   // ones column of V_aug
+    if (hh == 0) write_first<F16>(sV + (DV / 16) * Cfg::BLK, row, 1.f);   // ones column of V_aug
+    if constexpr (TAY) {
+        // features 160..191 of both phi tiles stay zero (the M = 64 state tile reads them)
+#pragma unroll
+        for (int f0 = F; f0 < Cfg::FT; f0 += 8)
+            sts128((hh ? aK : aQ) + sw128_off(row, f0), make_uint4(0u, 0u, 0u, 0u));
+    }
     __syncthreads();
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane = (uint32_t)(wq * 32) << 16;
-    const int na_lo = hh ? 80 : 0, na_hi = hh ? NA : 80;   // this thread's 16-column groups of S_aug
-    // TMEM columns: [0,128) scores -> P (first 64) and dP (second 64);
-    // [128,272) O_aug, then dA and dphi(Q); [272,416) state S_aug (M = 128);
-    // [416,488) G'_lo, the bf16 remainder of G' (A operand, packed pairs).
-    const uint32_t tA = tmem, tX = tmem + 128, tS = tmem + 272, tGL = tmem + 416;
+    const int na_lo = hh ? Cfg::NA_SPLIT : 0, na_hi = hh ? NA : Cfg::NA_SPLIT;   // this thread's columns of S_aug
+    const uint32_t tA = tmem, tX = tmem + Cfg::COL_X, tS = tmem + Cfg::COL_S, tGL = tmem + Cfg::COL_GL;
+    auto snap = [&](int f, int c0, const float *v) {
+        if constexpr (F16) snap_cols_f16<F>(aS, aSL, f, c0, v);
+        else snap_cols<F>(aS, aSL, f, c0, v, true);
+    };
 
     // ---- state entering the segment: sum of the earlier segments' increments
-    for (int c0 = na_lo; c0 < na_hi; c0 += 16) {
-        float v[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) v[e] = 0.f;
-        for (int s2 = 0; s2 < seg; ++s2) {
-            const float *src = p.ws_s + ((size_t)(bh * p.P + s2) * F + row) * NA + c0;
+    for (int t = 0; t < NT; ++t) {
+        if (!state_quadrant<Cfg>(t, wq)) continue;
+        const int f = state_row<Cfg>(t, wq, l);
+        for (int c0 = na_lo; c0 < na_hi; c0 += 16) {
+            float v[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] += src[e];
+            for (int e = 0; e < 16; ++e) v[e] = 0.f;
+            if (f >= 0)
+                for (int s2 = 0; s2 < seg; ++s2) {
+                    const float *src = p.ws_s + ((size_t)(bh * p.P + s2) * F + f) * NA + c0;
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) v[e] += src[e];
+                }
+            tmem_st16(tS + t * NA + lane + c0, v);
+            if (f >= 0) snap(f, c0, v);
         }
-        tmem_st16(tS + lane + c0, v);
-        snap_cols_f16<F>(aS, aSL, row, c0, v);
     }
     tmem_st_wait();
     full_sync();
@@ -486,10 +770,15 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const int t0 = chunk * C, i = row;
         const bool valid = t0 + i < N;
         if (tid == 0) {
-            mbar_arrive_expect_tx(tma_bar, 2 * Cfg::QK_TILE + 2 * C * DV * 2);
-            for (int x = 0; x < D; x += 64) {
-                tma_load_3d(sQ + (x / 64) * C * 128, &tm_q, tma_bar, x, t0, bh);
-                tma_load_3d(sK + (x / 64) * C * 128, &tm_k, tma_bar, x, t0, bh);
+            mbar_arrive_expect_tx(tma_bar, TAY ? 2 * Cfg::RAW + 2 * C * DV * 2 : 2 * C * D * 2 + 2 * C * DV * 2);
+            if constexpr (TAY) {
+                tma_load_3d(smem + Cfg::OFF_RQ, &tm_q, tma_bar, 0, t0, bh);
+                tma_load_3d(smem + Cfg::OFF_RK, &tm_k, tma_bar, 0, t0, bh);
+            } else {
+                for (int x = 0; x < D; x += 64) {
+                    tma_load_3d(sQ + (x / 64) * C * 128, &tm_q, tma_bar, x, t0, bh);
+                    tma_load_3d(sK + (x / 64) * C * 128, &tm_k, tma_bar, x, t0, bh);
+                }
             }
             for (int x = 0; x < DV; x += 16) {
                 tma_load_3d(sV + (x / 16) * Cfg::BLK, &tm_v, tma_bar, x, t0, bh);
@@ -498,37 +787,63 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
         if (!mbar_wait(tma_bar, tph)) *abort_flag = 1;
         tph ^= 1u;
-        // fp16 operands: phi(Q), phi(K) in place; V converted in place
-        phi_block_f16(aQ, i, false, hh);
-        phi_block_f16(aK, i, !valid, hh);
+        if constexpr (TAY) {
+            // phi(Q), phi(K): this thread's 80 of the 160 features of row i
+            float xq[16], xk[16];
+            raw_row16(aRQ, i, xq);
+            raw_row16(aRK, i, xk);
+            if (hh == 0) {
+                tay_phi_row<0, 10>(aQ, i, xq, false, p);
+                tay_phi_row<0, 10>(aK, i, xk, !valid, p);
+            } else {
+                tay_phi_row<80, 10>(aQ, i, xq, false, p);
+                tay_phi_row<80, 10>(aK, i, xk, !valid, p);
+            }
+        } else {
+            // fp16 operands: phi(Q), phi(K) in place; V converted in place
+            if (D == 128) {
+                phi_block_f16(aQ, i, false, hh);
+                phi_block_f16(aK, i, !valid, hh);
+            } else if (hh == 0) {
+                phi_block_f16(aQ, i, false, 0);
+            } else {
+                phi_block_f16(aK, i, !valid, 0);
+            }
 #pragma unroll
-        for (int c0 = hh * (DV / 2); c0 < (hh + 1) * (DV / 2); c0 += 8) {
-            const uint32_t a = aV + sw32_off(i, c0, C);
-            const uint4 r = lds128(a);
-            sts128(a, make_uint4(bf16x2_to_f16x2(r.x), bf16x2_to_f16x2(r.y), bf16x2_to_f16x2(r.z), bf16x2_to_f16x2(r.w)));
+            for (int c0 = hh * (DV / 2); c0 < (hh + 1) * (DV / 2); c0 += 8) {
+                const uint32_t a = aV + sw32_off(i, c0, C);
+                const uint4 r = lds128(a);
+                sts128(a, make_uint4(bf16x2_to_f16x2(r.x), bf16x2_to_f16x2(r.y), bf16x2_to_f16x2(r.z),
+                                     bf16x2_to_f16x2(r.w)));
+            }
         }
         full_sync();
         if (*abort_flag) break;
 
         // scores
         if (tid == 0) {
+            if constexpr (TAY) {
+                mma_bf16(tA, smem_desc(aRQ, 16, 256, kSw32), smem_desc(aRK, 16, 256, kSw32), idesc_bf16(128, 128, 0, 0),
+                         false);
+            } else {
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off = (kk >> 2) * (C * 128) + (kk & 3) * 32;
-                mma_bf16(tA, smem_desc(aQ + off, 16, 1024, kSw128), smem_desc(aK + off, 16, 1024, kSw128),
-                         idesc_f16(128, 128, 0, 0), kk > 0);
+                for (int kk = 0; kk < F / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * (C * 128) + (kk & 3) * 32;
+                    mma_bf16(tA, smem_desc(aQ + off, 16, 1024, kSw128), smem_desc(aK + off, 16, 1024, kSw128),
+                             idesc_f16(128, 128, 0, 0), kk > 0);
+                }
             }
             mma_commit(mma_bar);
         }
         if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
         mph ^= 1u;
         tc_fence_after();
-        mask_pack_half_f16(tA + lane, tA + lane, 64 * hh, true, [&](int j) { return j <= i; });
+        mask_pack_half_g<F16, TAY>(tA + lane, tA + lane, 64 * hh, true, p.inv_c3, p.k2, [&](int j) { return j <= i; });
         full_sync();
 
         // O_aug = P V_aug + phi(Q) S_aug
         if (tid == 0) {
-            const uint32_t id_o = idesc_f16(128, NA, 0, 1);
+            const uint32_t id_o = F16 ? idesc_f16(128, NA, 0, 1) : idesc_bf16(128, NA, 0, 1);
 #pragma unroll
             for (int kk = 0; kk < C / 16; ++kk)
                 mma_bf16_ts(tX, tA + kk * 8, smem_desc(aV + kk * 512, Cfg::BLK, 256, kSw32), id_o, kk > 0);
@@ -544,8 +859,8 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         mph ^= 1u;
         tc_fence_after();
 
-        // y, den; G'' = den * G' = [dO | -dO . y] in place over dO (fp16, with its
-        // fp16 remainder in TMEM).  Working with den * g keeps every operand in
+        // y, den; G'' = den * G' = [dO | -dO . y] in place over dO (with its
+        // remainder in TMEM).  Working with den * g keeps every operand in
         // fp16's normal range (g itself is ~|dO| / (F i)); the rows of dphi(Q) are
         // divided by den at the end.  den_i and dden_i = -(dO . y)/den go to the
         // workspace for the reverse pass.
@@ -559,10 +874,10 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const float inv = valid ? 1.f / den : 0.f;
             float gy = 0.f;   // dO . y over this thread's half of the columns
             {
-                const int half = 64 * hh;
-                uint32_t glo[32];
+                const int half = (DV / 2) * hh;
+                uint32_t glo[DV / 4];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < DV / 32; ++u) {
                     const int c0 = half + 16 * u;
                     float num[16], go[16];
                     tmem_ld16(tX + lane + c0, num);
@@ -575,23 +890,32 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         if (!valid) go[e] = 0.f;
                         gy = fmaf(go[e], num[e] * inv, gy);
                     }
-                    sts128(a0, make_uint4(pack_f16(go[0], go[1]), pack_f16(go[2], go[3]), pack_f16(go[4], go[5]),
-                                          pack_f16(go[6], go[7])));
-                    sts128(a1, make_uint4(pack_f16(go[8], go[9]), pack_f16(go[10], go[11]),
-                                          pack_f16(go[12], go[13]), pack_f16(go[14], go[15])));
+                    sts128(a0, make_uint4(pack2<F16>(go[0], go[1]), pack2<F16>(go[2], go[3]), pack2<F16>(go[4], go[5]),
+                                          pack2<F16>(go[6], go[7])));
+                    sts128(a1, make_uint4(pack2<F16>(go[8], go[9]), pack2<F16>(go[10], go[11]),
+                                          pack2<F16>(go[12], go[13]), pack2<F16>(go[14], go[15])));
 #pragma unroll
-                    for (int e = 0; e < 16; e += 2) glo[(16 * u + e) / 2] = pack_f16(f16_rem(go[e]), f16_rem(go[e + 1]));
+                    for (int e = 0; e < 16; e += 2) {
+                        if constexpr (F16) {
+                            glo[(16 * u + e) / 2] = pack_f16(f16_rem(go[e]), f16_rem(go[e + 1]));
+                        } else {
+                            glo[(16 * u + e) / 2] = pack_bf16(go[e] - __bfloat162float(__float2bfloat16_rn(go[e])),
+                                                              go[e + 1] - __bfloat162float(__float2bfloat16_rn(go[e + 1])));
+                        }
+                    }
                 }
-                tmem_st32(tGL + lane + half / 2, glo);
+                if constexpr (DV / 4 == 32) tmem_st32(tGL + lane + half / 2, glo);
+                else tmem_st16(tGL + lane + half / 2, reinterpret_cast<const float *>(glo));
             }
             red[hh * C + i] = gy;
             __syncthreads();
             gy = red[i] + red[C + i];
             const float ddu = valid ? -gy : 0.f;   // den * dden
             if (hh == 0) {
-                write_first_f16(sG + (DV / 16) * Cfg::BLK, i, ddu);
+                write_first<F16>(sG + (DV / 16) * Cfg::BLK, i, ddu);
                 uint32_t tail[8];
-                tail[0] = pack_f16(f16_rem(ddu), 0.f);
+                if constexpr (F16) tail[0] = pack_f16(f16_rem(ddu), 0.f);
+                else tail[0] = pack_bf16(ddu - __bfloat162float(__float2bfloat16_rn(ddu)), 0.f);
 #pragma unroll
                 for (int e = 1; e < 8; ++e) tail[e] = 0u;
                 tmem_st8(tGL + lane + DV / 2, tail);
@@ -604,98 +928,133 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
         full_sync();
 
-        // dA = G' V_aug^T  (K = the 144 augmented columns)
+        // dA = G'' V_aug^T  (K = the NA augmented columns)
         if (tid == 0) {
 #pragma unroll
             for (int kk = 0; kk < NA / 16; ++kk)
                 mma_bf16(tX, smem_desc(aG + kk * Cfg::BLK, 16, 256, kSw32), smem_desc(aV + kk * Cfg::BLK, 16, 256, kSw32),
-                         idesc_f16(128, 128, 0, 0), kk > 0);
+                         F16 ? idesc_f16(128, 128, 0, 0) : idesc_bf16(128, 128, 0, 0), kk > 0);
             mma_commit(mma_bar);
         }
         if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
         mph ^= 1u;
         tc_fence_after();
-        mask_pack_half_f16(tX + lane, tA + lane + 64, 64 * hh, false, [&](int j) { return j <= i; });
+        mask_pack_half_g<F16, false>(tX + lane, tA + lane + 64, 64 * hh, false, 0.f, 0.f, [&](int j) { return j <= i; });
         full_sync();
 
-        // dphi(Q) = dP phi(K) + G' S_aug^T ;  then S_aug += phi(K)^T V_aug
+        // dphi(Q) = dP phi(K) + G'' S_aug^T ;  then S_aug += phi(K)^T V_aug
         if (tid == 0) {
+            const uint32_t id_f = F16 ? idesc_f16(128, F, 0, 1) : idesc_bf16(128, F, 0, 1);
+            const uint32_t id_fk = F16 ? idesc_f16(128, F, 0, 0) : idesc_bf16(128, F, 0, 0);
 #pragma unroll
             for (int kk = 0; kk < C / 16; ++kk)
-                mma_bf16_ts(tX, tA + 64 + kk * 8, smem_desc(aK + kk * 2048, C * 128, 1024, kSw128),
-                            idesc_f16(128, F, 0, 1), kk > 0);
-            // inter-chunk term in ~16-bit precision: G'_hi S_hi^T + G'_hi S_lo^T + G'_lo S_hi^T
+                mma_bf16_ts(tX, tA + 64 + kk * 8, smem_desc(aK + kk * 2048, C * 128, 1024, kSw128), id_f, kk > 0);
+            // inter-chunk term in ~16-bit precision: G''_hi S_hi^T + G''_hi S_lo^T + G''_lo S_hi^T
 #pragma unroll
             for (int kk = 0; kk < NA / 16; ++kk) {
                 mma_bf16(tX, smem_desc(aG + kk * Cfg::BLK, 16, 256, kSw32), smem_desc(aS + kk * Cfg::S_BLK, 16, 256, kSw32),
-                         idesc_f16(128, F, 0, 0), true);
+                         id_fk, true);
                 mma_bf16(tX, smem_desc(aG + kk * Cfg::BLK, 16, 256, kSw32), smem_desc(aSL + kk * Cfg::S_BLK, 16, 256, kSw32),
-                         idesc_f16(128, F, 0, 0), true);
-                mma_bf16_ts(tX, tGL + kk * 8, smem_desc(aS + kk * Cfg::S_BLK, 16, 256, kSw32), idesc_f16(128, F, 0, 0),
-                            true);
+                         id_fk, true);
+                mma_bf16_ts(tX, tGL + kk * 8, smem_desc(aS + kk * Cfg::S_BLK, 16, 256, kSw32), id_fk, true);
             }
 #pragma unroll
-            for (int kk = 0; kk < C / 16; ++kk)
-                mma_bf16(tS, smem_desc(aK + kk * 2048, C * 128, 1024, kSw128), smem_desc(aV + kk * 512, Cfg::BLK, 256, kSw32),
-                         idesc_f16(128, NA, 1, 1), true);
+            for (int t = 0; t < NT; ++t) {
+                const int m = Cfg::tile_m(t);
+                const uint32_t a_base = aK + (Cfg::tile_f0(t) / 64) * (C * 128);
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    mma_bf16(tS + t * NA, smem_desc(a_base + kk * 2048, C * 128, 1024, kSw128),
+                             smem_desc(aV + kk * 512, Cfg::BLK, 256, kSw32),
+                             F16 ? idesc_f16(m, NA, 1, 1) : idesc_bf16(m, NA, 1, 1), true);
+            }
             mma_commit(mma_bar);
         }
         if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
         mph ^= 1u;
         tc_fence_after();
 
-        // dq = dphi(Q) * min(phi(q), 1), with dphi(q_i) first projected onto the
+        // dq = J_phi(q)^T dphi(Q), with dphi(q_i) first projected onto the
         // complement of phi(q_i): y_i is homogeneous of degree 0 in phi(q_i), so
-        // the exact dphi(q_i) is orthogonal to phi(q_i); the bf16 operands of the
-        // MMAs above leave an error mostly along phi(q_i) (elu features are
+        // the exact dphi(q_i) is orthogonal to phi(q_i); the rounded operands of
+        // the MMAs above leave an error mostly along phi(q_i) (elu features are
         // near 1 and the terms cancel), which the projection removes.
         {
-            __nv_bfloat16 *dqrow = reinterpret_cast<__nv_bfloat16 *>(p.dq) + ((size_t)bh * N + t0 + i) * D;
-            float sd = 0.f, sn = 0.f;
-#pragma unroll 1
-            for (int c0 = hh * (F / 2); c0 < (hh + 1) * (F / 2); c0 += 16) {
-                float g[16], ph[16];
-                tmem_ld16(tX + lane + c0, g);
-                tmem_ld_wait();
-                unpack8_f16(lds128(aQ + sw128_off(i, c0)), ph);
-                unpack8_f16(lds128(aQ + sw128_off(i, c0 + 8)), ph + 8);
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    sd = fmaf(g[e], ph[e], sd);
-                    sn = fmaf(ph[e], ph[e], sn);
-                }
-            }
-            red[2 * C + hh * C + i] = sd;
-            red[4 * C + hh * C + i] = sn;
-            __syncthreads();
-            sd = red[2 * C + i] + red[3 * C + i];
-            sn = red[4 * C + i] + red[5 * C + i];
-            const float proj = sd / sn;
             const float rden = valid ? 1.f / den_row : 0.f;
+            if constexpr (TAY) {
+                __nv_bfloat16 *dqrow = reinterpret_cast<__nv_bfloat16 *>(p.dq) + ((size_t)bh * N + t0 + i) * D;
+                float x[16], dx[16], sd = 0.f;
+                raw_row16(aRQ, i, x);
+#pragma unroll
+                for (int c = 0; c < 16; ++c) dx[c] = 0.f;
+                if (hh == 0) tay_vjp_half<0>(tX + lane, x, dx, sd, p);
+                else tay_vjp_half<1>(tX + lane, x, dx, sd, p);
+                float d8[8], sd_all;
+                tay_combine(red + 6 * C, red + 2 * C, hh, i, dx, sd, d8, sd_all);
+                float xx = 0.f;
+#pragma unroll
+                for (int c = 0; c < 16; ++c) xx = fmaf(x[c], x[c], xx);
+                // |phi|^2 = 1 + |x|^2/sqrt(d') + |x|^4/(2d');  J^T phi = x (1/sqrt(d') + |x|^2/d')
+                const float sn = fmaf(xx, fmaf(xx, p.k2, p.inv_c3), 1.f);
+                const float proj = sd_all / sn, jt = fmaf(xx, 2.f * p.k2, p.inv_c3);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) d8[c] = (d8[c] - proj * jt * x[8 * hh + c]) * rden;
+                if (valid)
+                    *reinterpret_cast<uint4 *>(dqrow + 8 * hh) =
+                        make_uint4(pack_bf16(d8[0], d8[1]), pack_bf16(d8[2], d8[3]), pack_bf16(d8[4], d8[5]),
+                                   pack_bf16(d8[6], d8[7]));
+            } else {
+                __nv_bfloat16 *dqrow = reinterpret_cast<__nv_bfloat16 *>(p.dq) + ((size_t)bh * N + t0 + i) * D;
+                float sd = 0.f, sn = 0.f;
 #pragma unroll 1
-            for (int c0 = hh * (F / 2); c0 < (hh + 1) * (F / 2); c0 += 16) {
-                float g[16], ph[16];
-                tmem_ld16(tX + lane + c0, g);
-                tmem_ld_wait();
-                unpack8_f16(lds128(aQ + sw128_off(i, c0)), ph);
-                unpack8_f16(lds128(aQ + sw128_off(i, c0 + 8)), ph + 8);
+                for (int c0 = hh * (F / 2); c0 < (hh + 1) * (F / 2); c0 += 16) {
+                    float g[16], ph[16];
+                    tmem_ld16(tX + lane + c0, g);
+                    tmem_ld_wait();
+                    unpack8_f16(lds128(aQ + sw128_off(i, c0)), ph);
+                    unpack8_f16(lds128(aQ + sw128_off(i, c0 + 8)), ph + 8);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) g[e] = (g[e] - proj * ph[e]) * fminf(ph[e], 1.f) * rden;
-                if (valid) {
+                    for (int e = 0; e < 16; ++e) {
+                        sd = fmaf(g[e], ph[e], sd);
+                        sn = fmaf(ph[e], ph[e], sn);
+                    }
+                }
+                red[2 * C + hh * C + i] = sd;
+                red[4 * C + hh * C + i] = sn;
+                __syncthreads();
+                sd = red[2 * C + i] + red[3 * C + i];
+                sn = red[4 * C + i] + red[5 * C + i];
+                const float proj = sd / sn;
+#pragma unroll 1
+                for (int c0 = hh * (F / 2); c0 < (hh + 1) * (F / 2); c0 += 16) {
+                    float g[16], ph[16];
+                    tmem_ld16(tX + lane + c0, g);
+                    tmem_ld_wait();
+                    unpack8_f16(lds128(aQ + sw128_off(i, c0)), ph);
+                    unpack8_f16(lds128(aQ + sw128_off(i, c0 + 8)), ph + 8);
 #pragma unroll
-                    for (int e = 0; e < 16; e += 8)
-                        *reinterpret_cast<uint4 *>(dqrow + c0 + e) =
-                            make_uint4(pack_bf16(g[e], g[e + 1]), pack_bf16(g[e + 2], g[e + 3]),
-                                       pack_bf16(g[e + 4], g[e + 5]), pack_bf16(g[e + 6], g[e + 7]));
+                    for (int e = 0; e < 16; ++e) g[e] = (g[e] - proj * ph[e]) * fminf(ph[e], 1.f) * rden;
+                    if (valid) {
+#pragma unroll
+                        for (int e = 0; e < 16; e += 8)
+                            *reinterpret_cast<uint4 *>(dqrow + c0 + e) =
+                                make_uint4(pack_bf16(g[e], g[e + 1]), pack_bf16(g[e + 2], g[e + 3]),
+                                           pack_bf16(g[e + 4], g[e + 5]), pack_bf16(g[e + 6], g[e + 7]));
+                    }
                 }
             }
             if (chunk + 1 < c_end) {
+#pragma unroll
+                for (int t = 0; t < NT; ++t) {
+                    if (!state_quadrant<Cfg>(t, wq)) continue;
+                    const int f = state_row<Cfg>(t, wq, l);
 #pragma unroll 1
-                for (int c0 = na_lo; c0 < na_hi; c0 += 16) {
-                    float v[16];
-                    tmem_ld16(tS + lane + c0, v);
-                    tmem_ld_wait();
-                    snap_cols_f16<F>(aS, aSL, row, c0, v);
+                    for (int c0 = na_lo; c0 < na_hi; c0 += 16) {
+                        float v[16];
+                        tmem_ld16(tS + t * NA + lane + c0, v);
+                        tmem_ld_wait();
+                        if (f >= 0) snap(f, c0, v);
+                    }
                 }
             }
         }
@@ -707,15 +1066,16 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
 // ---------------------------------------------------------------------------
 // State increments for the forward-order pass: for each segment but the
-// last, sum over its tokens of phi(k_j) [v_j | 1]^T, with fp16 operands like
+// last, sum over its tokens of phi(k_j) [v_j | 1]^T, with the operand type of
 // the pass that consumes them.
+template <class Cfg>
 __global__ void __launch_bounds__(128, 1)
 bwd_sstate_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const BwdParams p)
 {
     using namespace bwd_detail;
-    using Cfg = BwdCfg128;
-    constexpr int C = Cfg::C, D = Cfg::D, DV = Cfg::DV, NA = Cfg::NA, F = Cfg::F;
+    constexpr int C = Cfg::C, D = Cfg::D, DV = Cfg::DV, NA = Cfg::NA, F = Cfg::F, NT = Cfg::NT;
+    constexpr bool TAY = Cfg::TAYLOR, F16 = Cfg::F16;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *tma_bar = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
@@ -727,8 +1087,11 @@ bwd_sstate_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     if (seg == p.P - 1) return;   // the last segment's increment is never read
     const int c_begin = seg * p.cps, c_end = min(p.nchunks, c_begin + p.cps);
     const int N = p.N;
-    // two stages of [K | V_aug]: the Q and dO buffers, unused here, hold the second
-    uint8_t *sKs[2] = {smem + Cfg::OFF_K, smem + Cfg::OFF_Q}, *sVs[2] = {smem + Cfg::OFF_V, smem + Cfg::OFF_G};
+    // two stages of [K | V_aug]: elu: the K tiles in the K and Q regions;
+    // Taylor: the raw K tiles, and one phi(K) tile in the K region
+    uint8_t *sKs[2] = {smem + (TAY ? Cfg::OFF_RK : Cfg::OFF_K), smem + (TAY ? Cfg::OFF_RQ : Cfg::OFF_Q)};
+    uint8_t *sVs[2] = {smem + Cfg::OFF_V, smem + Cfg::OFF_G};
+    const uint32_t aPK = smem_addr(smem + Cfg::OFF_K);
     uint64_t *tma_b[2] = {tma_bar, tma_bar + 4};
     if (tid == 0) {
         mbar_init(tma_b[0], 1);
@@ -738,8 +1101,12 @@ bwd_sstate_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         mbar_init_fence();
     }
     if (warp == 0) tmem_alloc(tmem_slot, 256);
-    write_first_f16(sVs[0] + (DV / 16) * Cfg::BLK, tid, 1.f);
-    write_first_f16(sVs[1] + (DV / 16) * Cfg::BLK, tid, 1.f);
+    write_first<F16>(sVs[0] + (DV / 16) * Cfg::BLK, tid, 1.f);
+    write_first<F16>(sVs[1] + (DV / 16) * Cfg::BLK, tid, 1.f);
+    if constexpr (TAY) {
+#pragma unroll
+        for (int f0 = F; f0 < Cfg::FT; f0 += 8) sts128(aPK + sw128_off(tid, f0), make_uint4(0u, 0u, 0u, 0u));
+    }
     __syncthreads();
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane = (uint32_t)(warp * 32) << 16;
@@ -747,8 +1114,10 @@ bwd_sstate_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     // MMA has finished with the stage, a whole chunk ahead of their use
     auto issue = [&](int chunk) {
         const int st = (chunk - c_begin) & 1, t0 = chunk * C;
-        mbar_arrive_expect_tx(tma_b[st], Cfg::QK_TILE + C * DV * 2);
-        for (int x = 0; x < D; x += 64) tma_load_3d(sKs[st] + (x / 64) * C * 128, &tm_k, tma_b[st], x, t0, bh);
+        mbar_arrive_expect_tx(tma_b[st], (TAY ? Cfg::RAW : C * D * 2) + C * DV * 2);
+        if constexpr (TAY) tma_load_3d(sKs[st], &tm_k, tma_b[st], 0, t0, bh);
+        else
+            for (int x = 0; x < D; x += 64) tma_load_3d(sKs[st] + (x / 64) * C * 128, &tm_k, tma_b[st], x, t0, bh);
         for (int x = 0; x < DV; x += 16) tma_load_3d(sVs[st] + (x / 16) * Cfg::BLK, &tm_v, tma_b[st], x, t0, bh);
     };
     int issued = c_begin, waited = c_begin;   // thread 0: chunks whose loads went out / were waited for
@@ -757,23 +1126,38 @@ bwd_sstate_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     uint32_t mph = 0;
     for (int chunk = c_begin; chunk < c_end && !*abort_flag; ++chunk) {
         const int t0 = chunk * C, i = tid, st = (chunk - c_begin) & 1;
-        const uint32_t aK = smem_addr(sKs[st]), aV = smem_addr(sVs[st]);
+        const uint32_t aKs = smem_addr(sKs[st]), aV = smem_addr(sVs[st]);
         if (!mbar_wait(tma_b[st], (uint32_t)((chunk - c_begin) >> 1) & 1u)) *abort_flag = 1;
         waited = chunk + 1;
-        phi_row_f16(aK, i, t0 + i >= N);
+        if constexpr (TAY) {
+            float x[16];
+            raw_row16(aKs, i, x);
+            tay_phi_row<0, 20>(aPK, i, x, t0 + i >= N, p);
+        } else {
+            if (D == 128) phi_row_f16(aKs, i, t0 + i >= N);
+            else phi_block_f16(aKs, i, t0 + i >= N, 0);
 #pragma unroll
-        for (int c0 = 0; c0 < DV; c0 += 8) {
-            const uint32_t a = aV + sw32_off(i, c0, C);
-            const uint4 r = lds128(a);
-            sts128(a, make_uint4(bf16x2_to_f16x2(r.x), bf16x2_to_f16x2(r.y), bf16x2_to_f16x2(r.z), bf16x2_to_f16x2(r.w)));
+            for (int c0 = 0; c0 < DV; c0 += 8) {
+                const uint32_t a = aV + sw32_off(i, c0, C);
+                const uint4 r = lds128(a);
+                sts128(a, make_uint4(bf16x2_to_f16x2(r.x), bf16x2_to_f16x2(r.y), bf16x2_to_f16x2(r.z),
+                                     bf16x2_to_f16x2(r.w)));
+            }
         }
         full_sync();
         if (*abort_flag) break;
         if (tid == 0) {
+            const uint32_t aPhi = TAY ? aPK : aKs;
 #pragma unroll
-            for (int kk = 0; kk < C / 16; ++kk)
-                mma_bf16(tmem, smem_desc(aK + kk * 2048, C * 128, 1024, kSw128), smem_desc(aV + kk * 512, Cfg::BLK, 256, kSw32),
-                         idesc_f16(128, NA, 1, 1), chunk > c_begin || kk > 0);
+            for (int t = 0; t < NT; ++t) {
+                const int m = Cfg::tile_m(t);
+                const uint32_t a_base = aPhi + (Cfg::tile_f0(t) / 64) * (C * 128);
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    mma_bf16(tmem + t * NA, smem_desc(a_base + kk * 2048, C * 128, 1024, kSw128),
+                             smem_desc(aV + kk * 512, Cfg::BLK, 256, kSw32),
+                             F16 ? idesc_f16(m, NA, 1, 1) : idesc_bf16(m, NA, 1, 1), chunk > c_begin || kk > 0);
+            }
             mma_commit(mma_bar);
         }
         if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
@@ -786,14 +1170,20 @@ bwd_sstate_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         for (int c = waited; c < issued; ++c)
             mbar_wait(tma_b[(c - c_begin) & 1], (uint32_t)((c - c_begin) >> 1) & 1u, 100000000ull);
     if (!*abort_flag) {
-        float *dst = p.ws_s + ((size_t)(bh * p.P + seg) * F + tid) * NA;
-#pragma unroll 1
-        for (int c0 = 0; c0 < NA; c0 += 16) {
-            float v[16];
-            tmem_ld16(tmem + lane + c0, v);
-            tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 16; ++e) dst[c0 + e] = v[e];
+        for (int t = 0; t < NT; ++t) {
+            if (!state_quadrant<Cfg>(t, warp)) continue;
+            const int f = state_row<Cfg>(t, warp, tid & 31);
+            float *dst = p.ws_s + ((size_t)(bh * p.P + seg) * F + (f < 0 ? 0 : f)) * NA;
+#pragma unroll 1
+            for (int c0 = 0; c0 < NA; c0 += 16) {
+                float v[16];
+                tmem_ld16(tmem + t * NA + lane + c0, v);
+                tmem_ld_wait();
+                if (f >= 0)
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) dst[c0 + e] = v[e];
+            }
         }
     }
     full_sync();
@@ -803,13 +1193,14 @@ bwd_sstate_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
 // ---------------------------------------------------------------------------
 // R increments: for each segment but the first, sum over its tokens of
 // phi(q_i) G'_i^T (needs den_i, dden_i from the forward-order pass).
+template <class Cfg>
 __global__ void __launch_bounds__(128, 1)
 bwd_rstate_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                   const BwdParams p)
 {
     using namespace bwd_detail;
-    using Cfg = BwdCfg128;
-    constexpr int C = Cfg::C, D = Cfg::D, DV = Cfg::DV, NA = Cfg::NA, F = Cfg::F;
+    constexpr int C = Cfg::C, D = Cfg::D, DV = Cfg::DV, NA = Cfg::NA, F = Cfg::F, NT = Cfg::NT;
+    constexpr bool TAY = Cfg::TAYLOR;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *tma_bar = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
@@ -821,8 +1212,11 @@ bwd_rstate_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (seg == 0) return;   // the first segment's increment is never read
     const int c_begin = seg * p.cps, c_end = min(p.nchunks, c_begin + p.cps);
     const int N = p.N;
-    // two stages of [Q | G'_aug]: the K and V buffers, unused here, hold the second
-    uint8_t *sQs[2] = {smem + Cfg::OFF_Q, smem + Cfg::OFF_K}, *sGs[2] = {smem + Cfg::OFF_G, smem + Cfg::OFF_V};
+    // two stages of [Q | G'_aug]: elu: the Q tiles in the Q and K regions;
+    // Taylor: the raw Q tiles, and one phi(Q) tile in the Q region
+    uint8_t *sQs[2] = {smem + (TAY ? Cfg::OFF_RQ : Cfg::OFF_Q), smem + (TAY ? Cfg::OFF_RK : Cfg::OFF_K)};
+    uint8_t *sGs[2] = {smem + Cfg::OFF_G, smem + Cfg::OFF_V};
+    const uint32_t aPQ = smem_addr(smem + Cfg::OFF_Q);
     uint64_t *tma_b[2] = {tma_bar, tma_bar + 4};
     if (tid == 0) {
         mbar_init(tma_b[0], 1);
@@ -832,6 +1226,10 @@ bwd_rstate_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         mbar_init_fence();
     }
     if (warp == 0) tmem_alloc(tmem_slot, 256);
+    if constexpr (TAY) {
+#pragma unroll
+        for (int f0 = F; f0 < Cfg::FT; f0 += 8) sts128(aPQ + sw128_off(tid, f0), make_uint4(0u, 0u, 0u, 0u));
+    }
     __syncthreads();
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane = (uint32_t)(warp * 32) << 16;
@@ -839,8 +1237,10 @@ bwd_rstate_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     // MMA has finished with the stage
     auto issue = [&](int chunk) {
         const int st = (chunk - c_begin) & 1, t0 = chunk * C;
-        mbar_arrive_expect_tx(tma_b[st], Cfg::QK_TILE + C * DV * 2);
-        for (int x = 0; x < D; x += 64) tma_load_3d(sQs[st] + (x / 64) * C * 128, &tm_q, tma_b[st], x, t0, bh);
+        mbar_arrive_expect_tx(tma_b[st], (TAY ? Cfg::RAW : C * D * 2) + C * DV * 2);
+        if constexpr (TAY) tma_load_3d(sQs[st], &tm_q, tma_b[st], 0, t0, bh);
+        else
+            for (int x = 0; x < D; x += 64) tma_load_3d(sQs[st] + (x / 64) * C * 128, &tm_q, tma_b[st], x, t0, bh);
         for (int x = 0; x < DV; x += 16) tma_load_3d(sGs[st] + (x / 16) * Cfg::BLK, &tm_do, tma_b[st], x, t0, bh);
     };
     int issued = c_begin, waited = c_begin;
@@ -851,10 +1251,17 @@ bwd_rstate_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const int t0 = chunk * C, i = tid, st = (chunk - c_begin) & 1;
         const bool valid = t0 + i < N;
         uint8_t *sG = sGs[st];
-        const uint32_t aQ = smem_addr(sQs[st]), aG = smem_addr(sG);
+        const uint32_t aQs = smem_addr(sQs[st]), aG = smem_addr(sG);
         if (!mbar_wait(tma_b[st], (uint32_t)((chunk - c_begin) >> 1) & 1u)) *abort_flag = 1;
         waited = chunk + 1;
-        phi_row_inplace(aQ, i, false);
+        if constexpr (TAY) {
+            float x[16];
+            raw_row16(aQs, i, x);
+            tay_phi_row<0, 20>(aPQ, i, x, false, p);
+        } else {
+            if (D == 128) phi_row_inplace(aQs, i, false);
+            else phi_block_inplace(aQs, i, false, 0);
+        }
         {
             const float den = valid ? p.dd[((size_t)bh * N + t0 + i) * 2] : 1.f;
             const float dden = valid ? p.dd[((size_t)bh * N + t0 + i) * 2 + 1] : 0.f;
@@ -873,11 +1280,17 @@ bwd_rstate_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (*abort_flag) break;
         if (tid == 0) {
             // R_aug += phi(Q)^T G'   (M = F features, N = NA, K = tokens)
+            const uint32_t aPhi = TAY ? aPQ : aQs;
 #pragma unroll
-            for (int kk = 0; kk < C / 16; ++kk)
-                mma_bf16(tmem, smem_desc(aQ + kk * 2048, C * 128, 1024, kSw128),
-                         smem_desc(aG + kk * 512, Cfg::BLK, 256, kSw32), idesc_bf16(128, NA, 1, 1),
-                         chunk > c_begin || kk > 0);
+            for (int t = 0; t < NT; ++t) {
+                const int m = Cfg::tile_m(t);
+                const uint32_t a_base = aPhi + (Cfg::tile_f0(t) / 64) * (C * 128);
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    mma_bf16(tmem + t * NA, smem_desc(a_base + kk * 2048, C * 128, 1024, kSw128),
+                             smem_desc(aG + kk * 512, Cfg::BLK, 256, kSw32), idesc_bf16(m, NA, 1, 1),
+                             chunk > c_begin || kk > 0);
+            }
             mma_commit(mma_bar);
         }
         if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
@@ -889,14 +1302,20 @@ bwd_rstate_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         for (int c = waited; c < issued; ++c)
             mbar_wait(tma_b[(c - c_begin) & 1], (uint32_t)((c - c_begin) >> 1) & 1u, 100000000ull);
     if (!*abort_flag) {
-        float *dst = p.ws_r + ((size_t)(bh * p.P + seg) * F + tid) * NA;
-#pragma unroll 1
-        for (int c0 = 0; c0 < NA; c0 += 16) {
-            float v[16];
-            tmem_ld16(tmem + lane + c0, v);
-            tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 16; ++e) dst[c0 + e] = v[e];
+        for (int t = 0; t < NT; ++t) {
+            if (!state_quadrant<Cfg>(t, warp)) continue;
+            const int f = state_row<Cfg>(t, warp, tid & 31);
+            float *dst = p.ws_r + ((size_t)(bh * p.P + seg) * F + (f < 0 ? 0 : f)) * NA;
+#pragma unroll 1
+            for (int c0 = 0; c0 < NA; c0 += 16) {
+                float v[16];
+                tmem_ld16(tmem + t * NA + lane + c0, v);
+                tmem_ld_wait();
+                if (f >= 0)
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) dst[c0 + e] = v[e];
+            }
         }
     }
     full_sync();
@@ -907,29 +1326,31 @@ bwd_rstate_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 // Reverse-order pass: dk and dv.  256 threads: warps w and w + 4 share the
 // TMEM lanes of rows 32 (w % 4) .. + 31, and every per-row step is split
 // between them by columns (the first half of the columns to warps 0-3).
+template <class Cfg>
 __global__ void __launch_bounds__(256, 1)
 bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                 const BwdParams p)
 {
     using namespace bwd_detail;
-    using Cfg = BwdCfg128;
-    constexpr int C = Cfg::C, D = Cfg::D, DV = Cfg::DV, NA = Cfg::NA, F = Cfg::F;
+    constexpr int C = Cfg::C, D = Cfg::D, DV = Cfg::DV, NA = Cfg::NA, F = Cfg::F, NT = Cfg::NT;
+    constexpr bool TAY = Cfg::TAYLOR;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *tma_bar = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
     uint64_t *mma_bar = tma_bar + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tma_bar + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tma_bar + 3);
-    const int tid = threadIdx.x, warp = tid >> 5, wq = warp & 3, hh = warp >> 2;
-    const int row = wq * 32 + (tid & 31);   // this thread's token row / TMEM lane
+    const int tid = threadIdx.x, warp = tid >> 5, wq = warp & 3, hh = warp >> 2, l = tid & 31;
+    const int row = wq * 32 + l;   // this thread's token row / TMEM lane
+    float *red = reinterpret_cast<float *>(smem + Cfg::OFF_RED);
     const int bh = blockIdx.x / p.P, seg = blockIdx.x % p.P;
     const int c_begin = seg * p.cps, c_end = min(p.nchunks, c_begin + p.cps);
     const int N = p.N;
     uint8_t *sQ = smem + Cfg::OFF_Q, *sK = smem + Cfg::OFF_K, *sV = smem + Cfg::OFF_V, *sG = smem + Cfg::OFF_G,
             *sR = smem + Cfg::OFF_S, *sGL = smem + Cfg::OFF_SL;   // G' bf16 remainder
     const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV), aG = smem_addr(sG), aR = smem_addr(sR),
-                   aGL = smem_addr(sGL);
+                   aGL = smem_addr(sGL), aRQ = smem_addr(smem + Cfg::OFF_RQ), aRK = smem_addr(smem + Cfg::OFF_RK);
     if (tid == 0) {
         mbar_init(tma_bar, 1);
         mbar_init(mma_bar, 1);
@@ -938,30 +1359,41 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     if (warp == 0) tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
     if (hh == 0) write_ones_block(sV + (DV / 16) * Cfg::BLK, row);
+    if constexpr (TAY) {
+#pragma unroll
+        for (int f0 = F; f0 < Cfg::FT; f0 += 8)
+            sts128((hh ? aK : aQ) + sw128_off(row, f0), make_uint4(0u, 0u, 0u, 0u));
+    }
     __syncthreads();
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane = (uint32_t)(wq * 32) << 16;
-    const int na_lo = hh ? 80 : 0, na_hi = hh ? NA : 80;   // this thread's 16-column groups of R_aug
-    // TMEM: [0,64) P^T, [64,128) dP^T (packed); [0,128) holds A^T first;
-    // [128,256) dA^T, then dV, then dphi(K); [256,400) R_aug (M = 128);
-    // [400,464) the bf16 remainder of dP^T.
-    const uint32_t tA = tmem, tX = tmem + 128, tR = tmem + 256, tPL = tmem + 400;
+    const int na_lo = hh ? Cfg::NA_SPLIT : 0, na_hi = hh ? NA : Cfg::NA_SPLIT;   // this thread's columns of R_aug
+    const uint32_t tA = tmem, tX = tmem + Cfg::COL_X, tR = tmem + Cfg::COL_R, tPL = tmem + Cfg::COL_PL;
+    auto snap_r = [&](int f, int c0, const float *v) {
+        sts128(aR + sw32_off(f, c0, F), make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
+                                                   pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7])));
+        sts128(aR + sw32_off(f, c0 + 8, F), make_uint4(pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]),
+                                                       pack_bf16(v[12], v[13]), pack_bf16(v[14], v[15])));
+    };
 
     // ---- R entering the segment: sum of the later segments' increments
-    for (int c0 = na_lo; c0 < na_hi; c0 += 16) {
-        float v[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) v[e] = 0.f;
-        for (int s2 = seg + 1; s2 < p.P; ++s2) {
-            const float *src = p.ws_r + ((size_t)(bh * p.P + s2) * F + row) * NA + c0;
+    for (int t = 0; t < NT; ++t) {
+        if (!state_quadrant<Cfg>(t, wq)) continue;
+        const int f = state_row<Cfg>(t, wq, l);
+        for (int c0 = na_lo; c0 < na_hi; c0 += 16) {
+            float v[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] += src[e];
+            for (int e = 0; e < 16; ++e) v[e] = 0.f;
+            if (f >= 0)
+                for (int s2 = seg + 1; s2 < p.P; ++s2) {
+                    const float *src = p.ws_r + ((size_t)(bh * p.P + s2) * F + f) * NA + c0;
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) v[e] += src[e];
+                }
+            tmem_st16(tR + t * NA + lane + c0, v);
+            if (f >= 0) snap_r(f, c0, v);
         }
-        tmem_st16(tR + lane + c0, v);
-        sts128(aR + sw32_off(row, c0, F), make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
-                                                     pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7])));
-        sts128(aR + sw32_off(row, c0 + 8, F), make_uint4(pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]),
-                                                         pack_bf16(v[12], v[13]), pack_bf16(v[14], v[15])));
     }
     tmem_st_wait();
     full_sync();
@@ -971,10 +1403,15 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int t0 = chunk * C, j = row;
         const bool valid = t0 + j < N;
         if (tid == 0) {
-            mbar_arrive_expect_tx(tma_bar, 2 * Cfg::QK_TILE + 2 * C * DV * 2);
-            for (int x = 0; x < D; x += 64) {
-                tma_load_3d(sQ + (x / 64) * C * 128, &tm_q, tma_bar, x, t0, bh);
-                tma_load_3d(sK + (x / 64) * C * 128, &tm_k, tma_bar, x, t0, bh);
+            mbar_arrive_expect_tx(tma_bar, TAY ? 2 * Cfg::RAW + 2 * C * DV * 2 : 2 * C * D * 2 + 2 * C * DV * 2);
+            if constexpr (TAY) {
+                tma_load_3d(smem + Cfg::OFF_RQ, &tm_q, tma_bar, 0, t0, bh);
+                tma_load_3d(smem + Cfg::OFF_RK, &tm_k, tma_bar, 0, t0, bh);
+            } else {
+                for (int x = 0; x < D; x += 64) {
+                    tma_load_3d(sQ + (x / 64) * C * 128, &tm_q, tma_bar, x, t0, bh);
+                    tma_load_3d(sK + (x / 64) * C * 128, &tm_k, tma_bar, x, t0, bh);
+                }
             }
             for (int x = 0; x < DV; x += 16) {
                 tma_load_3d(sV + (x / 16) * Cfg::BLK, &tm_v, tma_bar, x, t0, bh);
@@ -983,8 +1420,25 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         if (!mbar_wait(tma_bar, tph)) *abort_flag = 1;
         tph ^= 1u;
-        phi_block_inplace(aQ, j, false, hh);
-        phi_block_inplace(aK, j, !valid, hh);
+        if constexpr (TAY) {
+            float xq[16], xk[16];
+            raw_row16(aRQ, j, xq);
+            raw_row16(aRK, j, xk);
+            if (hh == 0) {
+                tay_phi_row<0, 10>(aQ, j, xq, false, p);
+                tay_phi_row<0, 10>(aK, j, xk, !valid, p);
+            } else {
+                tay_phi_row<80, 10>(aQ, j, xq, false, p);
+                tay_phi_row<80, 10>(aK, j, xk, !valid, p);
+            }
+        } else if (D == 128) {
+            phi_block_inplace(aQ, j, false, hh);
+            phi_block_inplace(aK, j, !valid, hh);
+        } else if (hh == 0) {
+            phi_block_inplace(aQ, j, false, 0);
+        } else {
+            phi_block_inplace(aK, j, !valid, 0);
+        }
         {
             // G' row j (this thread's token as a query): [dO/den | dden] as bf16
             // plus its bf16 remainder (dA^T below uses both)
@@ -1014,13 +1468,18 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         full_sync();
         if (*abort_flag) break;
 
-        // A^T = phi(K) phi(Q)^T ;  dA^T = V_aug G'^T
+        // A^T = phi(K) phi(Q)^T (Taylor: raw K Q^T) ;  dA^T = V_aug G'^T
         if (tid == 0) {
+            if constexpr (TAY) {
+                mma_bf16(tA, smem_desc(aRK, 16, 256, kSw32), smem_desc(aRQ, 16, 256, kSw32), idesc_bf16(128, 128, 0, 0),
+                         false);
+            } else {
 #pragma unroll
-            for (int kk = 0; kk < F / 16; ++kk) {
-                const uint32_t off = (kk >> 2) * (C * 128) + (kk & 3) * 32;
-                mma_bf16(tA, smem_desc(aK + off, 16, 1024, kSw128), smem_desc(aQ + off, 16, 1024, kSw128),
-                         idesc_bf16(128, 128, 0, 0), kk > 0);
+                for (int kk = 0; kk < F / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * (C * 128) + (kk & 3) * 32;
+                    mma_bf16(tA, smem_desc(aK + off, 16, 1024, kSw128), smem_desc(aQ + off, 16, 1024, kSw128),
+                             idesc_bf16(128, 128, 0, 0), kk > 0);
+                }
             }
 #pragma unroll
             for (int kk = 0; kk < NA / 16; ++kk) {
@@ -1035,7 +1494,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mph ^= 1u;
         tc_fence_after();
         // row j keeps the queries i >= j
-        mask_pack_half(tA + lane, tA + lane, 64 * hh, [&](int i) { return i >= j; });
+        mask_pack_half_g<false, TAY>(tA + lane, tA + lane, 64 * hh, true, p.inv_c3, p.k2, [&](int i) { return i >= j; });
         mask_pack_half_hilo(tX + lane, tA + lane + 64, tPL + lane, 64 * hh, [&](int i) { return i >= j; });
         full_sync();
 
@@ -1087,9 +1546,14 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 mma_bf16(tX, smem_desc(aV + kk * Cfg::BLK, 16, 256, kSw32), smem_desc(aR + kk * Cfg::S_BLK, 16, 256, kSw32),
                          idesc_bf16(128, F, 0, 0), true);
 #pragma unroll
-            for (int kk = 0; kk < C / 16; ++kk)
-                mma_bf16(tR, smem_desc(aQ + kk * 2048, C * 128, 1024, kSw128),
-                         smem_desc(aG + kk * 512, Cfg::BLK, 256, kSw32), idesc_bf16(128, NA, 1, 1), true);
+            for (int t = 0; t < NT; ++t) {
+                const int m = Cfg::tile_m(t);
+                const uint32_t a_base = aQ + (Cfg::tile_f0(t) / 64) * (C * 128);
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    mma_bf16(tR + t * NA, smem_desc(a_base + kk * 2048, C * 128, 1024, kSw128),
+                             smem_desc(aG + kk * 512, Cfg::BLK, 256, kSw32), idesc_bf16(m, NA, 1, 1), true);
+            }
             mma_commit(mma_bar);
         }
         if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
@@ -1097,23 +1561,51 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc_fence_after();
         {
             __nv_bfloat16 *dkrow = reinterpret_cast<__nv_bfloat16 *>(p.dk) + ((size_t)bh * N + t0 + j) * D;
-#pragma unroll 1
-            for (int c0 = hh * (F / 2); c0 < (hh + 1) * (F / 2); c0 += 16) {
-                float g[16], ph[16];
-                tmem_ld16(tX + lane + c0, g);
-                tmem_ld_wait();
-                unpack8(lds128(aK + sw128_off(j, c0)), ph);
-                unpack8(lds128(aK + sw128_off(j, c0 + 8)), ph + 8);
-                if (valid)
+            if constexpr (TAY) {
+                float x[16], dx[16], sd = 0.f;
+                raw_row16(aRK, j, x);
 #pragma unroll
-                    for (int e = 0; e < 16; e += 8)
-                        *reinterpret_cast<uint4 *>(dkrow + c0 + e) = make_uint4(
-                            pack_bf16(g[e] * fminf(ph[e], 1.f), g[e + 1] * fminf(ph[e + 1], 1.f)),
-                            pack_bf16(g[e + 2] * fminf(ph[e + 2], 1.f), g[e + 3] * fminf(ph[e + 3], 1.f)),
-                            pack_bf16(g[e + 4] * fminf(ph[e + 4], 1.f), g[e + 5] * fminf(ph[e + 5], 1.f)),
-                            pack_bf16(g[e + 6] * fminf(ph[e + 6], 1.f), g[e + 7] * fminf(ph[e + 7], 1.f)));
+                for (int c = 0; c < 16; ++c) dx[c] = 0.f;
+                if (hh == 0) tay_vjp_half<0>(tX + lane, x, dx, sd, p);
+                else tay_vjp_half<1>(tX + lane, x, dx, sd, p);
+                float d8[8], sd_all;
+                tay_combine(red + 6 * C, red + 2 * C, hh, j, dx, sd, d8, sd_all);
+                if (valid)
+                    *reinterpret_cast<uint4 *>(dkrow + 8 * hh) =
+                        make_uint4(pack_bf16(d8[0], d8[1]), pack_bf16(d8[2], d8[3]), pack_bf16(d8[4], d8[5]),
+                                   pack_bf16(d8[6], d8[7]));
+            } else {
+#pragma unroll 1
+                for (int c0 = hh * (F / 2); c0 < (hh + 1) * (F / 2); c0 += 16) {
+                    float g[16], ph[16];
+                    tmem_ld16(tX + lane + c0, g);
+                    tmem_ld_wait();
+                    unpack8(lds128(aK + sw128_off(j, c0)), ph);
+                    unpack8(lds128(aK + sw128_off(j, c0 + 8)), ph + 8);
+                    if (valid)
+#pragma unroll
+                        for (int e = 0; e < 16; e += 8)
+                            *reinterpret_cast<uint4 *>(dkrow + c0 + e) = make_uint4(
+                                pack_bf16(g[e] * fminf(ph[e], 1.f), g[e + 1] * fminf(ph[e + 1], 1.f)),
+                                pack_bf16(g[e + 2] * fminf(ph[e + 2], 1.f), g[e + 3] * fminf(ph[e + 3], 1.f)),
+                                pack_bf16(g[e + 4] * fminf(ph[e + 4], 1.f), g[e + 5] * fminf(ph[e + 5], 1.f)),
+                                pack_bf16(g[e + 6] * fminf(ph[e + 6], 1.f), g[e + 7] * fminf(ph[e + 7], 1.f)));
+                }
             }
-            if (chunk > c_begin) snapshot_state<F, NA>(tR + lane, sR, nullptr, row, na_lo, na_hi);
+            if (chunk > c_begin) {
+#pragma unroll
+                for (int t = 0; t < NT; ++t) {
+                    if (!state_quadrant<Cfg>(t, wq)) continue;
+                    const int f = state_row<Cfg>(t, wq, l);
+#pragma unroll 1
+                    for (int c0 = na_lo; c0 < na_hi; c0 += 16) {
+                        float v[16];
+                        tmem_ld16(tR + t * NA + lane + c0, v);
+                        tmem_ld_wait();
+                        if (f >= 0) snap_r(f, c0, v);
+                    }
+                }
+            }
         }
         full_sync();
     }

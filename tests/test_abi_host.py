@@ -140,7 +140,20 @@ def test_kernel_plan_and_workspace(lib):
     # workspace: den/dden per token + S and R increments (4 segments x 128 x 144 fp32 each)
     assert la.la_backward_workspace_bytes(2, 16, 16384, 128, 128, 0, 1) == \
         32 * 16384 * 2 * 4 + 2 * 32 * 4 * 128 * 144 * 4
-    assert la.la_kernel_plan(1, 1, 2, 300, 64, 64, 0, 1) == (1, ["bwd_simt_kernel"])
+    # elu d=64 and both Taylor maps (d'=16, dv=64) take the tensor-core backward too:
+    # B=1 H=2 N=300 is 3 chunks, one segment each
+    assert la.la_kernel_plan(1, 1, 2, 300, 64, 64, 0, 1) == \
+        (4, ["bwd_sstate_kernel", "bwd_dq_kernel", "bwd_rstate_kernel", "bwd_dkdv_kernel"])
+    for fmap in (1, 2):
+        assert la.la_kernel_plan(1, 8, 16, 2048, 16, 64, fmap, 1) == (2, ["bwd_dq_kernel", "bwd_dkdv_kernel"])
+        # 128 heads: one segment per head, den/dden per token only
+        assert la.la_backward_workspace_bytes(8, 16, 2048, 16, 64, fmap, 1) == 128 * 2048 * 2 * 4
+        # 2 heads x 3 segments: plus S and R increments of 160 packed features x 80 columns
+        assert la.la_backward_workspace_bytes(1, 2, 300, 16, 64, fmap, 1) == 2 * 300 * 2 * 4 + 2 * 2 * 3 * 160 * 80 * 4
+    assert la.la_backward_workspace_bytes(1, 2, 300, 64, 64, 0, 1) == 2 * 300 * 2 * 4 + 2 * 2 * 3 * 64 * 80 * 4
+    # fp32 and the other shapes stay on the exact CUDA-core kernel
+    assert la.la_kernel_plan(1, 1, 2, 300, 32, 32, 0, 1) == (1, ["bwd_simt_kernel"])
+    assert la.la_kernel_plan(1, 1, 2, 300, 64, 64, 0, 0) == (1, ["bwd_simt_kernel"])
 
 
 def test_selftest_wait_limit_checked_before_launch(lib):

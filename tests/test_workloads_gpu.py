@@ -120,6 +120,29 @@ def test_workload_elu_bf16_train():
     assert ((lhs - rhs).norm() / rhs.norm()).item() < 1e-2
 
 
+def test_workload_taylor_bf16_train():
+    """The BASED Taylor training step at the Taylor prefill's shape: forward
+    and the tensor-core backward, every head against the oracle's recurrent
+    backward (the 273-feature map)."""
+    w = W.BY_NAME["taylor_bf16_train"]
+    q, k, v, do = W.make_inputs(w)
+    qd, kd, vd, dod = (t.to(DEV) for t in (q, k, v, do))
+    fr = la.la_forward(qd, kd, vd, w.fmap, den=True)
+    dq, dk, dvv = la.la_backward(qd, kd, vd, dod, w.fmap)
+    torch.cuda.synchronize()
+    la.la_get_device_status()
+    clk = _Clock()
+    o_ref, den_ref, _, _ = clk(orc.forward_recurrent, w.fmap, q, k, v)
+    rq, rk, rv = clk(orc.backward_recurrent, w.fmap, q, k, v, do)
+    errs = {n: orc.max_rel_l2(got.cpu(), ref) for n, got, ref in
+            (("o", fr["o"], o_ref), ("den", fr["den"], den_ref), ("dq", dq, rq), ("dk", dk, rk), ("dv", dvv, rv))}
+    _record("taylor_bf16_train", slices=w.B * w.H, oracle_s=round(clk.s, 2), **errs)
+    _check(errs, 1e-2)
+    lhs = dvv.float().sum(2)
+    rhs = dod.float().sum(2)
+    assert ((lhs - rhs).norm() / rhs.norm()).item() < 1e-2
+
+
 def test_workload_elu_bf16_decay_fwd():
     w = W.BY_NAME["elu_bf16_decay_fwd"]
     q, k, v, _ = W.make_inputs(w)

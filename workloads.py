@@ -4,19 +4,25 @@ This module only describes shapes and draws random inputs. It holds none of the
 method's arithmetic, so both the CUDA path and the CPU oracle can be fed from
 it without sharing any computation.
 
-Five workloads are defined, with the sizes used throughout the tests and the
-benchmark:
+The workloads, with the sizes used throughout the tests and the benchmark:
 
-  elu_fp32_fwd     elu(x)+1 forward, fp32 I/O, B=1 H=1 N=256 D=32
-  elu_bf16_fwd     elu(x)+1 chunked prefill, bf16 I/O, B=4 H=8 N=4096 D=64,
-                   inputs N(0,1)/sqrt(64)
-  taylor_bf16_fwd  BASED Taylor forward, bf16 I/O, B=8 H=16 N=2048 d'=16
-                   (273 features), Dv=64, inputs N(0,1)
-  elu_bf16_train   elu(x)+1 forward+backward, bf16 I/O, B=2 H=16 N=16384
-                   D=128, inputs and upstream grad N(0,1)/sqrt(128)
-  taylor_decode    BASED Taylor recurrent decode, fp32 I/O: 256 sequences,
-                   H=16, d'=16, Dv=64, state from a 2048-token prefill, then
-                   1024 one-token steps with fresh N(0,1) q/k/v
+  elu_fp32_fwd       elu(x)+1 forward, fp32 I/O, B=1 H=1 N=256 D=32
+  elu_bf16_fwd       elu(x)+1 chunked prefill, bf16 I/O, B=4 H=8 N=4096 D=64,
+                     inputs N(0,1)/sqrt(64)
+  taylor_bf16_fwd    BASED Taylor forward, bf16 I/O, B=8 H=16 N=2048 d'=16
+                     (273 features), Dv=64, inputs N(0,1)
+  elu_bf16_train     elu(x)+1 forward+backward, bf16 I/O, B=2 H=16 N=16384
+                     D=128, inputs and upstream grad N(0,1)/sqrt(128)
+  taylor_decode      BASED Taylor recurrent decode, fp32 I/O: 256 sequences,
+                     H=16, d'=16, Dv=64, state from a 2048-token prefill, then
+                     1024 one-token steps with fresh N(0,1) q/k/v
+  taylor_decode_sym  the same with the folded 153-row Taylor state
+  elu_bf16_varlen    16 packed prompts of seeded lengths in [1, 2048], H=8, D=64
+  elu_bf16_decay_fwd the headline shape with per-token forget gates
+  swa_bf16_fwd       sliding-window softmax attention, w=64, headline shape
+  swa_bf16_decode    its decode: 1024 x 16 heads, 64-token caches, 1024 steps
+  taylor_bf16_train  the Taylor forward's shape as a training step (forward +
+                     backward), inputs and upstream grad N(0,1)
 
 Random numbers come from torch's CPU Mersenne-Twister generator seeded with
 the workload's index; tensors are drawn in the order Q, K, V, dO (decode: the
@@ -111,6 +117,9 @@ WORKLOADS = [
     # (decode: 1024 sequences so that the 64-token bf16 caches, 268 MB, exceed L2; a 64-token
     # prompt fills each window, and a longer prompt would leave the same cache)
     Workload("swa_bf16_decode", 8, ELU1, BF16, 1024, 16, 64, 64, 64, 1.0, decode_steps=1024, window=64),
+    # the BASED Taylor shape as a training step: forward + backward, inputs and
+    # upstream gradient N(0,1)
+    Workload("taylor_bf16_train", 9, TAYLOR2, BF16, 8, 16, 2048, 16, 64, 1.0, backward=True),
 ]
 BY_NAME = {w.name: w for w in WORKLOADS}
 
