@@ -490,9 +490,13 @@ la_status forward_tc(const void *q, const void *k, const void *v, void *o, const
                                                       N, stream, false, cu, T, logdecay);
 }
 
-template <class Cfg>
+// Workspace of the tensor-core backward (floats): den_i, dden_i per token;
+// gated, c_i per token; when P > 1, the S and R increments per segment and,
+// gated, each segment's summed gate.
+template <class Cfg, bool GATED>
 la_status backward_tc(const void *q, const void *k, const void *v, const void *dout, void *dq, void *dk,
-                      void *dvp, void *workspace, int B, int H, int N, cudaStream_t stream)
+                      void *dvp, void *workspace, int B, int H, int N, cudaStream_t stream,
+                      const float *log_decay = nullptr, float *dlog_decay = nullptr)
 {
     const int BH = B * H;
     CUtensorMap tq, tk, tv, tdo;
@@ -506,10 +510,14 @@ la_status backward_tc(const void *q, const void *k, const void *v, const void *d
     tc_segments(B, H, N, &p.P, &p.cps, &p.nchunks);
     p.N = N;
     p.dd = (float *)workspace;
-    float *ws_s = p.dd + (size_t)BH * N * 2;
+    p.cvec = p.dd + (size_t)BH * N * 2;
+    float *ws_s = p.cvec + (GATED ? (size_t)BH * N : 0);
     float *ws_r = ws_s + (size_t)BH * p.P * Cfg::F * Cfg::NA;
     p.ws_s = ws_s;
     p.ws_r = ws_r;
+    p.ws_log = ws_r + (size_t)BH * p.P * Cfg::F * Cfg::NA;
+    p.logdecay = log_decay;
+    p.dg = dlog_decay;
     p.dq = dq;
     p.dk = dk;
     p.dv = dvp;
@@ -518,22 +526,25 @@ la_status backward_tc(const void *q, const void *k, const void *v, const void *d
     p.inv_c2 = (float)(1.0 / (sqrt(2.0) * sqrt(d)));
     p.inv_c3 = (float)(1.0 / sqrt(d));
     p.k2 = (float)(1.0 / (2.0 * d));
-    if (set_smem<bwd_sstate_kernel<Cfg>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
+    if (set_smem<bwd_sstate_kernel<Cfg, GATED>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
     if (p.P > 1) {
-        bwd_sstate_kernel<Cfg><<<BH * p.P, 128, Cfg::SMEM_ALLOC, stream>>>(tk, tv, p);
+        bwd_sstate_kernel<Cfg, GATED><<<BH * p.P, 128, Cfg::SMEM_ALLOC, stream>>>(tk, tv, p);
         if (launch_status() != LA_OK) return LA_ERR_CUDA;
     }
-    if (set_smem<bwd_dq_kernel<Cfg>>(Cfg::SMEM_ALLOC) != LA_OK ||
-        set_smem<bwd_dkdv_kernel<Cfg>>(Cfg::SMEM_ALLOC) != LA_OK ||
-        set_smem<bwd_rstate_kernel<Cfg>>(Cfg::SMEM_ALLOC) != LA_OK)
+    if (set_smem<bwd_dq_kernel<Cfg, GATED>>(Cfg::SMEM_ALLOC) != LA_OK ||
+        set_smem<bwd_dkdv_kernel<Cfg, GATED>>(Cfg::SMEM_ALLOC) != LA_OK ||
+        set_smem<bwd_rstate_kernel<Cfg, GATED>>(Cfg::SMEM_ALLOC) != LA_OK)
         return LA_ERR_CUDA;
-    bwd_dq_kernel<Cfg><<<BH * p.P, 256, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, p);
+    bwd_dq_kernel<Cfg, GATED><<<BH * p.P, 256, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, p);
     if (launch_status() != LA_OK) return LA_ERR_CUDA;
     if (p.P > 1) {
-        bwd_rstate_kernel<Cfg><<<BH * p.P, 128, Cfg::SMEM_ALLOC, stream>>>(tq, tdo, p);
+        bwd_rstate_kernel<Cfg, GATED><<<BH * p.P, 128, Cfg::SMEM_ALLOC, stream>>>(tq, tdo, p);
         if (launch_status() != LA_OK) return LA_ERR_CUDA;
     }
-    bwd_dkdv_kernel<Cfg><<<BH * p.P, 256, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, p);
+    bwd_dkdv_kernel<Cfg, GATED><<<BH * p.P, 256, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, p);
+    if (!GATED) return launch_status();
+    if (launch_status() != LA_OK) return LA_ERR_CUDA;
+    bwd_dg_kernel<<<BH, 1024, 0, stream>>>(p.cvec, p.dg, N);
     return launch_status();
 }
 
@@ -835,9 +846,9 @@ la_status la_backward(const void *q, const void *k, const void *v, const void *d
     cudaStream_t s = (cudaStream_t)stream;
     float *ws = (float *)workspace;
     switch (select_backward(B, H, N, dqk, dv, fmap, dtype) == Path::BwdTc ? bwd_tc_kind(dqk, dv, fmap, dtype) : 0) {
-    case 1: return backward_tc<BwdCfg128>(q, k, v, dout, dq, dk, dvp, workspace, B, H, N, s);
-    case 2: return backward_tc<BwdCfg64>(q, k, v, dout, dq, dk, dvp, workspace, B, H, N, s);
-    case 3: return backward_tc<BwdCfgT16>(q, k, v, dout, dq, dk, dvp, workspace, B, H, N, s);
+    case 1: return backward_tc<BwdCfg128, false>(q, k, v, dout, dq, dk, dvp, workspace, B, H, N, s);
+    case 2: return backward_tc<BwdCfg64, false>(q, k, v, dout, dq, dk, dvp, workspace, B, H, N, s);
+    case 3: return backward_tc<BwdCfgT16, false>(q, k, v, dout, dq, dk, dvp, workspace, B, H, N, s);
     default: break;
     }
     if (dtype == LA_F32)
@@ -892,7 +903,16 @@ size_t la_forward_decay_workspace_bytes(int B, int H, int N, int dqk, int dv, in
 size_t la_backward_decay_workspace_bytes(int B, int H, int N, int dqk, int dv, int fmap, int dtype)
 {
     if (check_shape(B, H, N, dqk, dv, fmap, dtype) != LA_OK) return 0;
-    return (size_t)B * H * N * 2 * sizeof(float);   // den_i, dden_i per token
+    const size_t BHN = (size_t)B * H * N;
+    const int kind = bwd_tc_kind(dqk, dv, fmap, dtype);
+    if (!kind) return BHN * 2 * sizeof(float);   // den_i, dden_i per token
+    // tensor cores: den_i, dden_i and c_i per token; per segment (P > 1) the S
+    // and R increments and the segment's summed gate
+    int P, cps, nc;
+    tc_segments(B, H, N, &P, &cps, &nc);
+    size_t floats = BHN * 3;
+    if (P > 1) floats += (size_t)B * H * P * (2 * bwd_increment_floats(kind) + 1);
+    return floats * sizeof(float);
 }
 
 la_status la_backward_decay(const void *q, const void *k, const void *v, const float *log_decay,
@@ -912,6 +932,12 @@ la_status la_backward_decay(const void *q, const void *k, const void *v, const f
     if (workspace_bytes < la_backward_decay_workspace_bytes(B, H, N, dqk, dv, fmap, dtype)) return LA_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
     float *ws = (float *)workspace;
+    switch (bwd_tc_kind(dqk, dv, fmap, dtype)) {
+    case 1: return backward_tc<BwdCfg128, true>(q, k, v, dout, dq, dk, dvp, workspace, B, H, N, st, log_decay, dlog_decay);
+    case 2: return backward_tc<BwdCfg64, true>(q, k, v, dout, dq, dk, dvp, workspace, B, H, N, st, log_decay, dlog_decay);
+    case 3: return backward_tc<BwdCfgT16, true>(q, k, v, dout, dq, dk, dvp, workspace, B, H, N, st, log_decay, dlog_decay);
+    default: break;
+    }
     if (dtype == LA_F32)
         return backward_simt<float>(q, k, v, dout, dq, dk, dvp, ws, B, H, N, dqk, dv, fmap, st, log_decay, dlog_decay);
     return backward_simt<__nv_bfloat16>(q, k, v, dout, dq, dk, dvp, ws, B, H, N, dqk, dv, fmap, st, log_decay,
@@ -1086,17 +1112,19 @@ int la_kernel_plan(int op, int B, int H, int N, int dqk, int dv, int fmap, int d
         }
         return P > 1 ? 2 : 1;
     }
-    else if (op == 1) p = select_backward(B, H, N, dqk, dv, fmap, dtype);
+    else if (op == 1 || op == 5) p = select_backward(B, H, N, dqk, dv, fmap, dtype);
     if (p == Path::BwdTc) {
         int P, cps, nc;
         tc_segments(B, H, N, &P, &cps, &nc);
-        const char *nm = P > 1 ? "bwd_sstate_kernel,bwd_dq_kernel,bwd_rstate_kernel,bwd_dkdv_kernel"
-                               : "bwd_dq_kernel,bwd_dkdv_kernel";
+        const bool g = op == 5;
+        const char *nm = P > 1 ? (g ? "bwd_sstate_kernel,bwd_dq_kernel,bwd_rstate_kernel,bwd_dkdv_kernel,bwd_dg_kernel"
+                                    : "bwd_sstate_kernel,bwd_dq_kernel,bwd_rstate_kernel,bwd_dkdv_kernel")
+                               : (g ? "bwd_dq_kernel,bwd_dkdv_kernel,bwd_dg_kernel" : "bwd_dq_kernel,bwd_dkdv_kernel");
         if (buf && buflen) {
             strncpy(buf, nm, buflen - 1);
             buf[buflen - 1] = 0;
         }
-        return P > 1 ? 4 : 2;
+        return (P > 1 ? 4 : 2) + (g ? 1 : 0);
     }
     else if (op == 2) p = select_decode(B, H, dqk, dv, fmap, dtype);
     const char *names[8];

@@ -104,7 +104,8 @@ struct BwdCfg {
     static constexpr int OFF_BAR = OFF_RK + RAW;
     static constexpr int OFF_RED = OFF_BAR + 128;        // per-row partial sums of the two threads of a row
     static constexpr int RED_FLOATS = 6 * C + (TAYLOR ? 2 * C * 16 : 0);
-    static constexpr int SMEM_ALLOC = OFF_RED + RED_FLOATS * 4 + 1024;
+    static constexpr int OFF_GATE = OFF_RED + RED_FLOATS * 4;   // gated form: [C] prefix sums, [4] quadrant totals
+    static constexpr int SMEM_ALLOC = OFF_GATE + (C + 8) * 4 + 1024;
     // TMEM columns.  Forward-order pass: [0, 128) scores -> P | dP; X: O_aug,
     // then dA, then dphi(Q); S: the state tiles; GL: the remainder of G''.
     // Reverse pass: [0, 128) scores -> P^T | dP^T; X: dA^T, then dV, then
@@ -136,6 +137,12 @@ struct BwdParams {
     // Taylor map: 1/d'^(1/4), 1/(sqrt2 sqrt d'), 1/sqrt(d') (pair features and
     // the score's linear term), 1/(2 d') (its square term)
     float inv_c1, inv_c2, inv_c3, k2;
+    // gated form (the GATED kernels only): log forget gate g_t per token
+    // [BH, N]; each segment's summed gate [BH, P] (written by the S pass);
+    // c_j = phi(k_j) . dphi(k_j) per token [BH, N] (written by the reverse
+    // pass) and dL/dg [BH, N] (its reverse prefix sum, negated)
+    const float *logdecay;
+    float *ws_log, *cvec, *dg;
 };
 
 namespace bwd_detail {
@@ -679,6 +686,135 @@ __device__ __forceinline__ void tay_combine(float *xred, float *sred, int hh, in
     sd_all = sred[i] + sred[128 + i];
 }
 
+
+// ---- gated form
+
+// Inclusive prefix sums L_r = g_{t0} + ... + g_{t0+r} of a chunk's log gates
+// for row r = 32 wq + l (rows at or past nvalid add 0; a gate below -80
+// counts as -80, as in the forward, which keeps every L finite so that no
+// difference of two L is inf - inf).  Writes gL[r] (when `writer`) and the
+// quadrant totals gL[C + wq]; returns L_r and the chunk's total L_last.
+// Every thread of the block calls it (it holds a barrier); the caller
+// synchronises again before reading another row's gL.
+__device__ __forceinline__ float gate_prefix(const float *g, int r, int nvalid, int wq, int l, bool writer, float *gL,
+                                             float &L_last)
+{
+    float x = r < nvalid ? fmaxf(g[r], -80.f) : 0.f;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, x, off);
+        if (l >= off) x += y;
+    }
+    if (writer && l == 31) gL[128 + wq] = x;
+    __syncthreads();
+    float before = 0.f, tot = 0.f;
+#pragma unroll
+    for (int w2 = 0; w2 < 4; ++w2) {
+        const float t = gL[128 + w2];
+        if (w2 < wq) before += t;
+        tot += t;
+    }
+    const float L = x + before;
+    if (writer) gL[r] = L;
+    L_last = tot;
+    return L;
+}
+
+// TMEM columns [c_lo, c_hi) (multiples of 16) of this thread's lane times s.
+__device__ __forceinline__ void tmem_scale(uint32_t t_lane, int c_lo, int c_hi, float s)
+{
+#pragma unroll 1
+    for (int c0 = c_lo; c0 < c_hi; c0 += 16) {
+        float v[16];
+        tmem_ld16(t_lane + c0, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] *= s;
+        tmem_st16(t_lane + c0, v);
+    }
+    tmem_st_wait();
+}
+
+// The state tiles' columns [c_lo, c_hi) of this thread's lane times s.
+template <class Cfg>
+__device__ __forceinline__ void decay_state_tiles(uint32_t t_state, uint32_t lane, int wq, int c_lo, int c_hi, float s)
+{
+#pragma unroll
+    for (int t = 0; t < Cfg::NT; ++t)
+        if (state_quadrant<Cfg>(t, wq)) tmem_scale(t_state + t * Cfg::NA + lane, c_lo, c_hi, s);
+}
+
+// Columns [c_lo, c_hi) (multiples of 8) of row r of a 128-row SW32 tile
+// (bf16 or fp16 pairs) times s.
+template <bool F16>
+__device__ __forceinline__ void scale_row_sw32(uint32_t tile, int r, int c_lo, int c_hi, float s)
+{
+#pragma unroll 1
+    for (int c0 = c_lo; c0 < c_hi; c0 += 8) {
+        const uint32_t a = tile + sw32_off(r, c0, 128);
+        float x[8];
+        if constexpr (F16) unpack8_f16(lds128(a), x);
+        else unpack8(lds128(a), x);
+        sts128(a, make_uint4(pack2<F16>(s * x[0], s * x[1]), pack2<F16>(s * x[2], s * x[3]),
+                             pack2<F16>(s * x[4], s * x[5]), pack2<F16>(s * x[6], s * x[7])));
+    }
+}
+
+// mask_pack_half_g with the gated weights: entry (i, j) of a row, i >= j,
+// is also multiplied by exp(L_i - L_j) (the gates a_{j+1} ... a_i); the
+// entries masked out are selected away, never multiplied, so an exp that
+// overflows there does no harm.  `rowL` is this row's L, `colL` the L of
+// column j (shared memory).
+template <bool F16, bool TAY, typename Keep>
+__device__ __forceinline__ void mask_pack_half_gate(uint32_t src, uint32_t dst, int j0, bool aliased, float k1, float k2,
+                                                    float rowL, const float *colL, bool row_is_query, Keep keep)
+{
+    float a[64];
+    tmem_ld32(src + j0, a);
+    tmem_ld32(src + j0 + 32, a + 32);
+    tmem_ld_wait();
+    if (aliased) {
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
+    if constexpr (TAY) {
+#pragma unroll
+        for (int e = 0; e < 64; ++e) a[e] = fmaf(a[e], fmaf(a[e], k2, k1), 1.f);
+    }
+#pragma unroll
+    for (int e = 0; e < 64; ++e) a[e] *= __expf(row_is_query ? rowL - colL[j0 + e] : colL[j0 + e] - rowL);
+    uint32_t pk[32];
+#pragma unroll
+    for (int e = 0; e < 64; e += 2) pk[e / 2] = pack2<F16>(keep(j0 + e) ? a[e] : 0.f, keep(j0 + e + 1) ? a[e + 1] : 0.f);
+    tmem_st32(dst + j0 / 2, pk);
+    tmem_st_wait();
+}
+
+// mask_pack_half_hilo with the gated weights (reverse pass: row j is a key,
+// column i a query, weight exp(L_i - L_j)).
+template <typename Keep>
+__device__ __forceinline__ void mask_pack_half_hilo_gate(uint32_t src, uint32_t dst_hi, uint32_t dst_lo, int j0,
+                                                         float rowL, const float *colL, Keep keep)
+{
+    float a[64];
+    tmem_ld32(src + j0, a);
+    tmem_ld32(src + j0 + 32, a + 32);
+    tmem_ld_wait();
+    uint32_t hi[32], lo[32];
+#pragma unroll
+    for (int e = 0; e < 64; e += 2) {
+        const float x0 = keep(j0 + e) ? a[e] * __expf(colL[j0 + e] - rowL) : 0.f;
+        const float x1 = keep(j0 + e + 1) ? a[e + 1] * __expf(colL[j0 + e + 1] - rowL) : 0.f;
+        hi[e / 2] = pack_bf16(x0, x1);
+        lo[e / 2] = pack_bf16(x0 - __bfloat162float(__float2bfloat16_rn(x0)),
+                              x1 - __bfloat162float(__float2bfloat16_rn(x1)));
+    }
+    tmem_st32(dst_hi + j0 / 2, hi);
+    tmem_st32(dst_lo + j0 / 2, lo);
+    tmem_st_wait();
+}
+
 }  // namespace bwd_detail
 
 // ---------------------------------------------------------------------------
@@ -691,7 +827,7 @@ __device__ __forceinline__ void tay_combine(float *xred, float *sred, int hh, in
 // for the inter-chunk term, and dphi(q) is projected orthogonal to phi(q).
 // Taylor: the same steps on bf16 operands, with the raw scores and the
 // feature-to-coordinate chain rule described at the top of the file.
-template <class Cfg>
+template <class Cfg, bool GATED = false>
 __global__ void __launch_bounds__(256, 1)
 bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -742,6 +878,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if constexpr (F16) snap_cols_f16<F>(aS, aSL, f, c0, v);
         else snap_cols<F>(aS, aSL, f, c0, v, true);
     };
+    float *gL = reinterpret_cast<float *>(smem + Cfg::OFF_GATE);   // gated: the chunk's prefix sums of the gates
 
     // ---- state entering the segment: sum of the earlier segments' increments
 #pragma unroll
@@ -755,8 +892,16 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             if (f >= 0)
                 for (int s2 = 0; s2 < seg; ++s2) {
                     const float *src = p.ws_s + ((size_t)(bh * p.P + s2) * F + f) * NA + c0;
+                    if constexpr (GATED) {
+                        // the state after segment s2 is its increment plus the earlier
+                        // state decayed by the segment's gates
+                        const float d = __expf(p.ws_log[(size_t)bh * p.P + s2]);
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) v[e] += src[e];
+                        for (int e = 0; e < 16; ++e) v[e] = fmaf(v[e], d, src[e]);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) v[e] += src[e];
+                    }
                 }
             tmem_st16(tS + t * NA + lane + c0, v);
             if (f >= 0) snap(f, c0, v);
@@ -787,6 +932,13 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
         if (!mbar_wait(tma_bar, tph)) *abort_flag = 1;
         tph ^= 1u;
+        // gated: L_i = g_{t0} + ... + g_i over the chunk; exp(L_i) scales the
+        // carried state's terms of row i, exp(L_last - L_j) the state update by key j
+        float Lrow = 0.f, Llast = 0.f;
+        if constexpr (GATED) {
+            Lrow = gate_prefix(p.logdecay + (size_t)bh * N + t0, row, min(C, N - t0), wq, l, hh == 0, gL, Llast);
+            if (hh == 0) write_first<F16>(sV + (DV / 16) * Cfg::BLK, row, 1.f);   // scaled by the last chunk's update
+        }
         if constexpr (TAY) {
             // phi(Q), phi(K): this thread's 80 of the 160 features of row i
             float xq[16], xk[16];
@@ -838,20 +990,44 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
         mph ^= 1u;
         tc_fence_after();
-        mask_pack_half_g<F16, TAY>(tA + lane, tA + lane, 64 * hh, true, p.inv_c3, p.k2, [&](int j) { return j <= i; });
+        if constexpr (GATED)
+            mask_pack_half_gate<F16, TAY>(tA + lane, tA + lane, 64 * hh, true, p.inv_c3, p.k2, Lrow, gL, true,
+                                          [&](int j) { return j <= i; });
+        else
+            mask_pack_half_g<F16, TAY>(tA + lane, tA + lane, 64 * hh, true, p.inv_c3, p.k2, [&](int j) { return j <= i; });
         full_sync();
 
-        // O_aug = P V_aug + phi(Q) S_aug
+        // O_aug = P V_aug + phi(Q) S_aug  (gated: the state term first, scaled
+        // per row by exp(L_i), then the chunk's own term added)
+        if constexpr (GATED) {
+            if (tid == 0) {
+                const uint32_t id_o = F16 ? idesc_f16(128, NA, 0, 1) : idesc_bf16(128, NA, 0, 1);
+#pragma unroll
+                for (int kk = 0; kk < F / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * (C * 128) + (kk & 3) * 32;
+                    mma_bf16(tX, smem_desc(aQ + off, 16, 1024, kSw128), smem_desc(aS + kk * 512, Cfg::S_BLK, 256, kSw32),
+                             id_o, kk > 0);
+                }
+                mma_commit(mma_bar);
+            }
+            if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
+            mph ^= 1u;
+            tc_fence_after();
+            tmem_scale(tX + lane, na_lo, na_hi, __expf(Lrow));
+            full_sync();
+        }
         if (tid == 0) {
             const uint32_t id_o = F16 ? idesc_f16(128, NA, 0, 1) : idesc_bf16(128, NA, 0, 1);
 #pragma unroll
             for (int kk = 0; kk < C / 16; ++kk)
-                mma_bf16_ts(tX, tA + kk * 8, smem_desc(aV + kk * 512, Cfg::BLK, 256, kSw32), id_o, kk > 0);
+                mma_bf16_ts(tX, tA + kk * 8, smem_desc(aV + kk * 512, Cfg::BLK, 256, kSw32), id_o, GATED || kk > 0);
+            if constexpr (!GATED) {
 #pragma unroll
-            for (int kk = 0; kk < F / 16; ++kk) {
-                const uint32_t off = (kk >> 2) * (C * 128) + (kk & 3) * 32;
-                mma_bf16(tX, smem_desc(aQ + off, 16, 1024, kSw128), smem_desc(aS + kk * 512, Cfg::S_BLK, 256, kSw32),
-                         id_o, true);
+                for (int kk = 0; kk < F / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * (C * 128) + (kk & 3) * 32;
+                    mma_bf16(tX, smem_desc(aQ + off, 16, 1024, kSw128),
+                             smem_desc(aS + kk * 512, Cfg::S_BLK, 256, kSw32), id_o, true);
+                }
             }
             mma_commit(mma_bar);
         }
@@ -939,8 +1115,41 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
         mph ^= 1u;
         tc_fence_after();
-        mask_pack_half_g<F16, false>(tX + lane, tA + lane + 64, 64 * hh, false, 0.f, 0.f, [&](int j) { return j <= i; });
+        if constexpr (GATED) {
+            mask_pack_half_gate<F16, false>(tX + lane, tA + lane + 64, 64 * hh, false, 0.f, 0.f, Lrow, gL, true,
+                                            [&](int j) { return j <= i; });
+            // V_aug's last use below is the state update: scale key row i by
+            // exp(L_last - L_i) (its ones column too), and decay the state by the
+            // chunk's whole gate
+            const float w = __expf(Llast - Lrow);
+            scale_row_sw32<F16>(aV, i, hh * (DV / 2), (hh + 1) * (DV / 2), w);
+            if (hh == 0) write_first<F16>(sV + (DV / 16) * Cfg::BLK, i, w);
+            decay_state_tiles<Cfg>(tS, lane, wq, na_lo, na_hi, __expf(Llast));
+        } else {
+            mask_pack_half_g<F16, false>(tX + lane, tA + lane + 64, 64 * hh, false, 0.f, 0.f,
+                                         [&](int j) { return j <= i; });
+        }
         full_sync();
+        if constexpr (GATED) {
+            // the carried state's term of dphi(Q) first, scaled per row by exp(L_i)
+            if (tid == 0) {
+                const uint32_t id_fk = F16 ? idesc_f16(128, F, 0, 0) : idesc_bf16(128, F, 0, 0);
+#pragma unroll
+                for (int kk = 0; kk < NA / 16; ++kk) {
+                    mma_bf16(tX, smem_desc(aG + kk * Cfg::BLK, 16, 256, kSw32),
+                             smem_desc(aS + kk * Cfg::S_BLK, 16, 256, kSw32), id_fk, kk > 0);
+                    mma_bf16(tX, smem_desc(aG + kk * Cfg::BLK, 16, 256, kSw32),
+                             smem_desc(aSL + kk * Cfg::S_BLK, 16, 256, kSw32), id_fk, true);
+                    mma_bf16_ts(tX, tGL + kk * 8, smem_desc(aS + kk * Cfg::S_BLK, 16, 256, kSw32), id_fk, true);
+                }
+                mma_commit(mma_bar);
+            }
+            if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
+            mph ^= 1u;
+            tc_fence_after();
+            tmem_scale(tX + lane, hh * (F / 2), (hh + 1) * (F / 2), __expf(Lrow));
+            full_sync();
+        }
 
         // dphi(Q) = dP phi(K) + G'' S_aug^T ;  then S_aug += phi(K)^T V_aug
         if (tid == 0) {
@@ -948,10 +1157,12 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const uint32_t id_fk = F16 ? idesc_f16(128, F, 0, 0) : idesc_bf16(128, F, 0, 0);
 #pragma unroll
             for (int kk = 0; kk < C / 16; ++kk)
-                mma_bf16_ts(tX, tA + 64 + kk * 8, smem_desc(aK + kk * 2048, C * 128, 1024, kSw128), id_f, kk > 0);
+                mma_bf16_ts(tX, tA + 64 + kk * 8, smem_desc(aK + kk * 2048, C * 128, 1024, kSw128), id_f,
+                            GATED || kk > 0);
             // inter-chunk term in ~16-bit precision: G''_hi S_hi^T + G''_hi S_lo^T + G''_lo S_hi^T
+            // (gated: issued above)
 #pragma unroll
-            for (int kk = 0; kk < NA / 16; ++kk) {
+            for (int kk = 0; kk < (GATED ? 0 : NA / 16); ++kk) {
                 mma_bf16(tX, smem_desc(aG + kk * Cfg::BLK, 16, 256, kSw32), smem_desc(aS + kk * Cfg::S_BLK, 16, 256, kSw32),
                          id_fk, true);
                 mma_bf16(tX, smem_desc(aG + kk * Cfg::BLK, 16, 256, kSw32), smem_desc(aSL + kk * Cfg::S_BLK, 16, 256, kSw32),
@@ -1068,7 +1279,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 // State increments for the forward-order pass: for each segment but the
 // last, sum over its tokens of phi(k_j) [v_j | 1]^T, with the operand type of
 // the pass that consumes them.
-template <class Cfg>
+template <class Cfg, bool GATED = false>
 __global__ void __launch_bounds__(128, 1)
 bwd_sstate_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const BwdParams p)
@@ -1124,9 +1335,16 @@ bwd_sstate_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     if (tid == 0)
         for (; issued < c_end && issued < c_begin + 2; ++issued) issue(issued);
     uint32_t mph = 0;
+    float *gL = reinterpret_cast<float *>(smem + Cfg::OFF_GATE);
+    float seg_log = 0.f;   // gated: sum of the segment's gates
     for (int chunk = c_begin; chunk < c_end && !*abort_flag; ++chunk) {
         const int t0 = chunk * C, i = tid, st = (chunk - c_begin) & 1;
         const uint32_t aKs = smem_addr(sKs[st]), aV = smem_addr(sVs[st]);
+        float Lrow = 0.f, Llast = 0.f;
+        if constexpr (GATED) {
+            Lrow = gate_prefix(p.logdecay + (size_t)bh * N + t0, i, min(C, N - t0), warp, tid & 31, true, gL, Llast);
+            seg_log += Llast;
+        }
         if (!mbar_wait(tma_b[st], (uint32_t)((chunk - c_begin) >> 1) & 1u)) *abort_flag = 1;
         waited = chunk + 1;
         if constexpr (TAY) {
@@ -1143,6 +1361,13 @@ bwd_sstate_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 sts128(a, make_uint4(bf16x2_to_f16x2(r.x), bf16x2_to_f16x2(r.y), bf16x2_to_f16x2(r.z),
                                      bf16x2_to_f16x2(r.w)));
             }
+        }
+        if constexpr (GATED) {
+            // S <- exp(L_last) S + sum_j exp(L_last - L_j) phi(k_j) [v_j | 1]^T
+            const float w = __expf(Llast - Lrow);
+            scale_row_sw32<F16>(aV, i, 0, DV, w);
+            write_first<F16>(sVs[st] + (DV / 16) * Cfg::BLK, i, w);
+            if (chunk > c_begin) decay_state_tiles<Cfg>(tmem, lane, warp, 0, NA, __expf(Llast));
         }
         full_sync();
         if (*abort_flag) break;
@@ -1170,6 +1395,7 @@ bwd_sstate_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         for (int c = waited; c < issued; ++c)
             mbar_wait(tma_b[(c - c_begin) & 1], (uint32_t)((c - c_begin) >> 1) & 1u, 100000000ull);
     if (!*abort_flag) {
+        if (GATED && tid == 0) p.ws_log[(size_t)bh * p.P + seg] = seg_log;
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
             if (!state_quadrant<Cfg>(t, warp)) continue;
@@ -1193,7 +1419,7 @@ bwd_sstate_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
 // ---------------------------------------------------------------------------
 // R increments: for each segment but the first, sum over its tokens of
 // phi(q_i) G'_i^T (needs den_i, dden_i from the forward-order pass).
-template <class Cfg>
+template <class Cfg, bool GATED = false>
 __global__ void __launch_bounds__(128, 1)
 bwd_rstate_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                   const BwdParams p)
@@ -1233,27 +1459,35 @@ bwd_rstate_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     __syncthreads();
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane = (uint32_t)(warp * 32) << 16;
-    // chunk c uses stage (c - c_begin) & 1; its loads go out when chunk c - 2's
-    // MMA has finished with the stage
-    auto issue = [&](int chunk) {
-        const int st = (chunk - c_begin) & 1, t0 = chunk * C;
+    // The it-th chunk taken (forward order; gated: from the segment's end, so
+    // that R can decay as it goes) uses stage it & 1; its loads go out when
+    // the (it - 2)-th chunk's MMA has finished with the stage.
+    const int nch = c_end - c_begin;
+    auto chunk_of = [&](int it) { return GATED ? c_end - 1 - it : c_begin + it; };
+    auto issue = [&](int it) {
+        const int st = it & 1, t0 = chunk_of(it) * C;
         mbar_arrive_expect_tx(tma_b[st], (TAY ? Cfg::RAW : C * D * 2) + C * DV * 2);
         if constexpr (TAY) tma_load_3d(sQs[st], &tm_q, tma_b[st], 0, t0, bh);
         else
             for (int x = 0; x < D; x += 64) tma_load_3d(sQs[st] + (x / 64) * C * 128, &tm_q, tma_b[st], x, t0, bh);
         for (int x = 0; x < DV; x += 16) tma_load_3d(sGs[st] + (x / 16) * Cfg::BLK, &tm_do, tma_b[st], x, t0, bh);
     };
-    int issued = c_begin, waited = c_begin;
+    int issued = 0, waited = 0;   // counts of chunks taken
     if (tid == 0)
-        for (; issued < c_end && issued < c_begin + 2; ++issued) issue(issued);
+        for (; issued < nch && issued < 2; ++issued) issue(issued);
     uint32_t mph = 0;
-    for (int chunk = c_begin; chunk < c_end && !*abort_flag; ++chunk) {
-        const int t0 = chunk * C, i = tid, st = (chunk - c_begin) & 1;
+    float *gL = reinterpret_cast<float *>(smem + Cfg::OFF_GATE);
+    for (int it = 0; it < nch && !*abort_flag; ++it) {
+        const int chunk = chunk_of(it);
+        const int t0 = chunk * C, i = tid, st = it & 1;
         const bool valid = t0 + i < N;
         uint8_t *sG = sGs[st];
         const uint32_t aQs = smem_addr(sQs[st]), aG = smem_addr(sG);
-        if (!mbar_wait(tma_b[st], (uint32_t)((chunk - c_begin) >> 1) & 1u)) *abort_flag = 1;
-        waited = chunk + 1;
+        float Lrow = 0.f, Llast = 0.f;
+        if constexpr (GATED)
+            Lrow = gate_prefix(p.logdecay + (size_t)bh * N + t0, i, min(C, N - t0), warp, tid & 31, true, gL, Llast);
+        if (!mbar_wait(tma_b[st], (uint32_t)(it >> 1) & 1u)) *abort_flag = 1;
+        waited = it + 1;
         if constexpr (TAY) {
             float x[16];
             raw_row16(aQs, i, x);
@@ -1263,9 +1497,11 @@ bwd_rstate_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             else phi_block_inplace(aQs, i, false, 0);
         }
         {
+            // gated: query row i enters R scaled by exp(L_i)
+            const float e = GATED ? __expf(Lrow) : 1.f;
             const float den = valid ? p.dd[((size_t)bh * N + t0 + i) * 2] : 1.f;
-            const float dden = valid ? p.dd[((size_t)bh * N + t0 + i) * 2 + 1] : 0.f;
-            const float inv = valid ? 1.f / den : 0.f;
+            const float dden = valid ? e * p.dd[((size_t)bh * N + t0 + i) * 2 + 1] : 0.f;
+            const float inv = valid ? e / den : 0.f;
 #pragma unroll 1
             for (int c0 = 0; c0 < DV; c0 += 8) {
                 float go[8];
@@ -1276,6 +1512,8 @@ bwd_rstate_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
             write_dden(sG + (DV / 16) * Cfg::BLK, i, dden);
         }
+        // gated: R <- exp(L_last) R + sum_i exp(L_i) phi(q_i) G'_i^T
+        if (GATED && it > 0) decay_state_tiles<Cfg>(tmem, lane, warp, 0, NA, __expf(Llast));
         full_sync();
         if (*abort_flag) break;
         if (tid == 0) {
@@ -1289,18 +1527,17 @@ bwd_rstate_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 for (int kk = 0; kk < C / 16; ++kk)
                     mma_bf16(tmem + t * NA, smem_desc(a_base + kk * 2048, C * 128, 1024, kSw128),
                              smem_desc(aG + kk * 512, Cfg::BLK, 256, kSw32), idesc_bf16(m, NA, 1, 1),
-                             chunk > c_begin || kk > 0);
+                             it > 0 || kk > 0);
             }
             mma_commit(mma_bar);
         }
         if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
         mph ^= 1u;
-        if (tid == 0 && !*abort_flag && issued < c_end) issue(issued++);
+        if (tid == 0 && !*abort_flag && issued < nch) issue(issued++);
         full_sync();
     }
     if (tid == 0 && *abort_flag)
-        for (int c = waited; c < issued; ++c)
-            mbar_wait(tma_b[(c - c_begin) & 1], (uint32_t)((c - c_begin) >> 1) & 1u, 100000000ull);
+        for (int c = waited; c < issued; ++c) mbar_wait(tma_b[c & 1], (uint32_t)(c >> 1) & 1u, 100000000ull);
     if (!*abort_flag) {
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
@@ -1326,7 +1563,7 @@ bwd_rstate_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 // Reverse-order pass: dk and dv.  256 threads: warps w and w + 4 share the
 // TMEM lanes of rows 32 (w % 4) .. + 31, and every per-row step is split
 // between them by columns (the first half of the columns to warps 0-3).
-template <class Cfg>
+template <class Cfg, bool GATED = false>
 __global__ void __launch_bounds__(256, 1)
 bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -1369,6 +1606,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t lane = (uint32_t)(wq * 32) << 16;
     const int na_lo = hh ? Cfg::NA_SPLIT : 0, na_hi = hh ? NA : Cfg::NA_SPLIT;   // this thread's columns of R_aug
     const uint32_t tA = tmem, tX = tmem + Cfg::COL_X, tR = tmem + Cfg::COL_R, tPL = tmem + Cfg::COL_PL;
+    float *gL = reinterpret_cast<float *>(smem + Cfg::OFF_GATE);   // gated: the chunk's prefix sums of the gates
     auto snap_r = [&](int f, int c0, const float *v) {
         sts128(aR + sw32_off(f, c0, F), make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
                                                    pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7])));
@@ -1385,12 +1623,24 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             float v[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) v[e] = 0.f;
-            if (f >= 0)
-                for (int s2 = seg + 1; s2 < p.P; ++s2) {
-                    const float *src = p.ws_r + ((size_t)(bh * p.P + s2) * F + f) * NA + c0;
+            if (f >= 0) {
+                if constexpr (GATED) {
+                    // R seen from the end of segment s2 - 1 is s2's increment plus
+                    // R at s2's end decayed by s2's gates; from the last segment down
+                    for (int s2 = p.P - 1; s2 > seg; --s2) {
+                        const float *src = p.ws_r + ((size_t)(bh * p.P + s2) * F + f) * NA + c0;
+                        const float d = s2 == p.P - 1 ? 0.f : __expf(p.ws_log[(size_t)bh * p.P + s2]);
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) v[e] += src[e];
+                        for (int e = 0; e < 16; ++e) v[e] = fmaf(v[e], d, src[e]);
+                    }
+                } else {
+                    for (int s2 = seg + 1; s2 < p.P; ++s2) {
+                        const float *src = p.ws_r + ((size_t)(bh * p.P + s2) * F + f) * NA + c0;
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) v[e] += src[e];
+                    }
                 }
+            }
             tmem_st16(tR + t * NA + lane + c0, v);
             if (f >= 0) snap_r(f, c0, v);
         }
@@ -1420,6 +1670,12 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         if (!mbar_wait(tma_bar, tph)) *abort_flag = 1;
         tph ^= 1u;
+        // gated: L over the chunk; exp(L_i - L_j) weights pair (i, j),
+        // exp(L_last - L_j) the later chunks' terms of key j, exp(L_i) query i's
+        // term of the R update
+        float Lrow = 0.f, Llast = 0.f;
+        if constexpr (GATED)
+            Lrow = gate_prefix(p.logdecay + (size_t)bh * N + t0, row, min(C, N - t0), wq, l, hh == 0, gL, Llast);
         if constexpr (TAY) {
             float xq[16], xk[16];
             raw_row16(aRQ, j, xq);
@@ -1439,11 +1695,13 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         } else {
             phi_block_inplace(aK, j, !valid, 0);
         }
+        float dden_row;
         {
             // G' row j (this thread's token as a query): [dO/den | dden] as bf16
             // plus its bf16 remainder (dA^T below uses both)
             const float den = valid ? p.dd[((size_t)bh * N + t0 + j) * 2] : 1.f;
-            const float dden = valid ? p.dd[((size_t)bh * N + t0 + j) * 2 + 1] : 0.f;
+            dden_row = valid ? p.dd[((size_t)bh * N + t0 + j) * 2 + 1] : 0.f;
+            const float dden = dden_row;
             const float inv = valid ? 1.f / den : 0.f;
 #pragma unroll 1
             for (int c0 = hh * (DV / 2); c0 < (hh + 1) * (DV / 2); c0 += 8) {
@@ -1494,18 +1752,44 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mph ^= 1u;
         tc_fence_after();
         // row j keeps the queries i >= j
-        mask_pack_half_g<false, TAY>(tA + lane, tA + lane, 64 * hh, true, p.inv_c3, p.k2, [&](int i) { return i >= j; });
-        mask_pack_half_hilo(tX + lane, tA + lane + 64, tPL + lane, 64 * hh, [&](int i) { return i >= j; });
+        if constexpr (GATED) {
+            mask_pack_half_gate<false, TAY>(tA + lane, tA + lane, 64 * hh, true, p.inv_c3, p.k2, Lrow, gL, false,
+                                            [&](int i) { return i >= j; });
+            mask_pack_half_hilo_gate(tX + lane, tA + lane + 64, tPL + lane, 64 * hh, Lrow, gL,
+                                     [&](int i) { return i >= j; });
+        } else {
+            mask_pack_half_g<false, TAY>(tA + lane, tA + lane, 64 * hh, true, p.inv_c3, p.k2,
+                                         [&](int i) { return i >= j; });
+            mask_pack_half_hilo(tX + lane, tA + lane + 64, tPL + lane, 64 * hh, [&](int i) { return i >= j; });
+        }
         full_sync();
+        if constexpr (GATED) {
+            // the later chunks' term of dV first, scaled per key row by exp(L_last - L_j)
+            if (tid == 0) {
+                const uint32_t id = idesc_bf16(128, DV, 0, 1);
+#pragma unroll
+                for (int kk = 0; kk < F / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * (C * 128) + (kk & 3) * 32;
+                    mma_bf16(tX, smem_desc(aK + off, 16, 1024, kSw128), smem_desc(aR + kk * 512, Cfg::S_BLK, 256, kSw32),
+                             id, kk > 0);
+                }
+                mma_commit(mma_bar);
+            }
+            if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
+            mph ^= 1u;
+            tc_fence_after();
+            tmem_scale(tX + lane, hh * (DV / 2), (hh + 1) * (DV / 2), __expf(Llast - Lrow));
+            full_sync();
+        }
 
         // dV = P^T G + phi(K) R
         if (tid == 0) {
             const uint32_t id = idesc_bf16(128, DV, 0, 1);
 #pragma unroll
             for (int kk = 0; kk < C / 16; ++kk)
-                mma_bf16_ts(tX, tA + kk * 8, smem_desc(aG + kk * 512, Cfg::BLK, 256, kSw32), id, kk > 0);
+                mma_bf16_ts(tX, tA + kk * 8, smem_desc(aG + kk * 512, Cfg::BLK, 256, kSw32), id, GATED || kk > 0);
 #pragma unroll
-            for (int kk = 0; kk < F / 16; ++kk) {
+            for (int kk = 0; kk < (GATED ? 0 : F / 16); ++kk) {
                 const uint32_t off = (kk >> 2) * (C * 128) + (kk & 3) * 32;
                 mma_bf16(tX, smem_desc(aK + off, 16, 1024, kSw128), smem_desc(aR + kk * 512, Cfg::S_BLK, 256, kSw32),
                          id, true);
@@ -1530,19 +1814,42 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                        pack_bf16(g[e + 4], g[e + 5]), pack_bf16(g[e + 6], g[e + 7]));
             }
         }
+        if constexpr (GATED) {
+            // G''s last use below is the R update: scale query row j by exp(L_j),
+            // and decay R by the chunk's whole gate
+            const float e = __expf(Lrow);
+            scale_row_sw32<false>(aG, j, hh * (DV / 2), (hh + 1) * (DV / 2), e);
+            if (hh == 0) write_dden(sG + (DV / 16) * Cfg::BLK, j, dden_row * e);
+            decay_state_tiles<Cfg>(tR, lane, wq, na_lo, na_hi, __expf(Llast));
+        }
         full_sync();
+        if constexpr (GATED) {
+            // the later chunks' term of dphi(K) first, scaled per key row by exp(L_last - L_j)
+            if (tid == 0) {
+#pragma unroll
+                for (int kk = 0; kk < NA / 16; ++kk)
+                    mma_bf16(tX, smem_desc(aV + kk * Cfg::BLK, 16, 256, kSw32),
+                             smem_desc(aR + kk * Cfg::S_BLK, 16, 256, kSw32), idesc_bf16(128, F, 0, 0), kk > 0);
+                mma_commit(mma_bar);
+            }
+            if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
+            mph ^= 1u;
+            tc_fence_after();
+            tmem_scale(tX + lane, hh * (F / 2), (hh + 1) * (F / 2), __expf(Llast - Lrow));
+            full_sync();
+        }
 
         // dphi(K) = dP^T phi(Q) + V_aug R_aug^T ;  then R_aug += phi(Q)^T G'
         if (tid == 0) {
 #pragma unroll
             for (int kk = 0; kk < C / 16; ++kk) {
                 mma_bf16_ts(tX, tA + 64 + kk * 8, smem_desc(aQ + kk * 2048, C * 128, 1024, kSw128),
-                            idesc_bf16(128, F, 0, 1), kk > 0);
+                            idesc_bf16(128, F, 0, 1), GATED || kk > 0);
                 mma_bf16_ts(tX, tPL + kk * 8, smem_desc(aQ + kk * 2048, C * 128, 1024, kSw128),
                             idesc_bf16(128, F, 0, 1), true);
             }
 #pragma unroll
-            for (int kk = 0; kk < NA / 16; ++kk)
+            for (int kk = 0; kk < (GATED ? 0 : NA / 16); ++kk)
                 mma_bf16(tX, smem_desc(aV + kk * Cfg::BLK, 16, 256, kSw32), smem_desc(aR + kk * Cfg::S_BLK, 16, 256, kSw32),
                          idesc_bf16(128, F, 0, 0), true);
 #pragma unroll
@@ -1570,11 +1877,13 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 else tay_vjp_half<1>(tX + lane, x, dx, sd, p);
                 float d8[8], sd_all;
                 tay_combine(red + 6 * C, red + 2 * C, hh, j, dx, sd, d8, sd_all);
+                if (GATED && hh == 0 && valid) p.cvec[(size_t)bh * N + t0 + j] = sd_all;   // phi(k_j) . dphi(k_j)
                 if (valid)
                     *reinterpret_cast<uint4 *>(dkrow + 8 * hh) =
                         make_uint4(pack_bf16(d8[0], d8[1]), pack_bf16(d8[2], d8[3]), pack_bf16(d8[4], d8[5]),
                                    pack_bf16(d8[6], d8[7]));
             } else {
+                float sd = 0.f;   // gated: phi(k_j) . dphi(k_j) over this thread's features
 #pragma unroll 1
                 for (int c0 = hh * (F / 2); c0 < (hh + 1) * (F / 2); c0 += 16) {
                     float g[16], ph[16];
@@ -1582,6 +1891,10 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     tmem_ld_wait();
                     unpack8(lds128(aK + sw128_off(j, c0)), ph);
                     unpack8(lds128(aK + sw128_off(j, c0 + 8)), ph + 8);
+                    if constexpr (GATED) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) sd = fmaf(g[e], ph[e], sd);
+                    }
                     if (valid)
 #pragma unroll
                         for (int e = 0; e < 16; e += 8)
@@ -1590,6 +1903,11 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                 pack_bf16(g[e + 2] * fminf(ph[e + 2], 1.f), g[e + 3] * fminf(ph[e + 3], 1.f)),
                                 pack_bf16(g[e + 4] * fminf(ph[e + 4], 1.f), g[e + 5] * fminf(ph[e + 5], 1.f)),
                                 pack_bf16(g[e + 6] * fminf(ph[e + 6], 1.f), g[e + 7] * fminf(ph[e + 7], 1.f)));
+                }
+                if constexpr (GATED) {
+                    red[2 * C + hh * C + j] = sd;
+                    __syncthreads();
+                    if (hh == 0 && valid) p.cvec[(size_t)bh * N + t0 + j] = red[2 * C + j] + red[3 * C + j];
                 }
             }
             if (chunk > c_begin) {
@@ -1611,6 +1929,44 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     full_sync();
     if (warp == 0) tmem_dealloc(tmem, Cfg::TMEM_COLS);
+}
+
+
+// ---------------------------------------------------------------------------
+// Gated form: dL/dg_l = - sum_{m >= l} c_m per head, c_m = phi(k_m) . dphi(k_m)
+// from the reverse pass.  (g_l scales every weight w_ij with j < l <= i; the
+// weights of a query sum to a constant in y_i's gradient, sum_j dL/dw_ij w_ij
+// = 0, which turns the sum over pairs into this suffix sum of per-key terms.)
+// One block per head walks the sequence from its end in tiles of 1024.
+__global__ void __launch_bounds__(1024, 1) bwd_dg_kernel(const float *c, float *dg, int N)
+{
+    __shared__ float wsum[32];
+    const int bh = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const float *cb = c + (size_t)bh * N;
+    float *db = dg + (size_t)bh * N;
+    float carry = 0.f;   // sum of c after the current tile
+    for (int end = N; end > 0; end -= 1024) {
+        const int idx = end - 1 - tid;   // thread t: position end-1-t
+        float x = idx >= 0 ? cb[idx] : 0.f;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, x, off);
+            if (lane >= off) x += y;
+        }
+        if (lane == 31) wsum[warp] = x;
+        __syncthreads();
+        float before = 0.f, total = 0.f;
+        for (int w2 = 0; w2 < 32; ++w2) {
+            const float t = wsum[w2];
+            if (w2 < warp) before += t;
+            total += t;
+        }
+        // position 0: no pair j < 0 <= i exists, so dL/dg_0 is zero by
+        // definition (the suffix sum is zero only up to rounding)
+        if (idx >= 0) db[idx] = idx == 0 ? 0.f : -(carry + before + x);
+        carry += total;
+        __syncthreads();
+    }
 }
 
 }  // namespace la

@@ -249,8 +249,13 @@ LA_API la_status la_forward_decay(const void *q, const void *k, const void *v, c
  * The weights of each output row sum to one, so
  *     dL/dg_l = sum over the pairs j < l <= i of w_ij dL/dw_ij
  *             = -sum_{j>=l} phi(k_j) . dL/dphi(k_j),
- * a suffix sum that the reverse-order pass accumulates.  Every shape runs on
- * the exact fp32 CUDA-core backward; workspace: la_backward_decay_workspace_bytes. */
+ * a suffix sum of per-key terms that the reverse-order pass produces.  bf16
+ * with a tensor-core shape (elu dqk = dv in {64, 128}; either Taylor map with
+ * dqk = 16, dv = 64) runs on the tensor-core backward with the gates inside
+ * each chunk's weights (a gate below e^-80 counts as e^-80, as in the
+ * forward) and a final suffix-sum kernel for dlog_decay; every other
+ * combination runs on the exact fp32 CUDA-core backward.  Workspace:
+ * la_backward_decay_workspace_bytes (its contents need no initialisation). */
 LA_API size_t la_backward_decay_workspace_bytes(int B, int H, int N, int dqk, int dv, int fmap, int dtype);
 
 LA_API la_status la_backward_decay(const void *q, const void *k, const void *v, const float *log_decay,
@@ -388,12 +393,14 @@ LA_API la_status la_feature_map(const void *x, void *phi, int64_t rows, int dqk,
 /* Which kernels a call would launch, without launching anything (for
  * launch accounting in benchmarks and tests).  op: 0 = la_forward,
  * 1 = la_backward, 2 = la_decode_step, 3 = la_forward_varlen (B = nseq,
- * N = max_seqlen), 4 = la_forward_decay.  Writes a comma-separated list of
+ * N = max_seqlen), 4 = la_forward_decay, 5 = la_backward_decay for the
+ * tensor-core shapes.  Writes a comma-separated list of
  * kernel names (truncated to buflen-1 characters, NUL-terminated) to buf
  * when buf is non-NULL, and returns the number of kernel launches the call
  * makes, or -1 for arguments the call itself would reject.  The gated
  * calls outside this list launch fixed kernels: la_decode_step_decay the
- * one op 2 reports for its shape, la_backward_decay one bwd_simt_kernel. */
+ * one op 2 reports for its shape, la_backward_decay on the other shapes one
+ * bwd_simt_kernel. */
 LA_API int la_kernel_plan(int op, int B, int H, int N, int dqk, int dv, int fmap, int dtype,
                           char *buf, size_t buflen);
 

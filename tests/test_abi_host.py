@@ -151,6 +151,16 @@ def test_kernel_plan_and_workspace(lib):
         # 2 heads x 3 segments: plus S and R increments of 160 packed features x 80 columns
         assert la.la_backward_workspace_bytes(1, 2, 300, 16, 64, fmap, 1) == 2 * 300 * 2 * 4 + 2 * 2 * 3 * 160 * 80 * 4
     assert la.la_backward_workspace_bytes(1, 2, 300, 64, 64, 0, 1) == 2 * 300 * 2 * 4 + 2 * 2 * 3 * 64 * 80 * 4
+    # the gated backward on the same shapes: plus the dL/dg suffix-sum kernel; its
+    # workspace holds den, dden and c per token, and per segment the S and R
+    # increments and the summed gate
+    assert la.la_kernel_plan(5, 1, 2, 300, 64, 64, 0, 1) == \
+        (5, ["bwd_sstate_kernel", "bwd_dq_kernel", "bwd_rstate_kernel", "bwd_dkdv_kernel", "bwd_dg_kernel"])
+    assert la.la_kernel_plan(5, 8, 16, 2048, 16, 64, 1, 1) == (3, ["bwd_dq_kernel", "bwd_dkdv_kernel", "bwd_dg_kernel"])
+    bd = la.load_library().la_backward_decay_workspace_bytes
+    assert bd(1, 2, 300, 64, 64, 0, 1) == (2 * 300 * 3 + 2 * 3 * (2 * 64 * 80 + 1)) * 4
+    assert bd(8, 16, 2048, 16, 64, 2, 1) == 128 * 2048 * 3 * 4
+    assert bd(1, 2, 300, 32, 32, 0, 1) == 2 * 300 * 2 * 4          # CUDA-core backward: den, dden
     # fp32 and the other shapes stay on the exact CUDA-core kernel
     assert la.la_kernel_plan(1, 1, 2, 300, 32, 32, 0, 1) == (1, ["bwd_simt_kernel"])
     assert la.la_kernel_plan(1, 1, 2, 300, 64, 64, 0, 0) == (1, ["bwd_simt_kernel"])

@@ -248,7 +248,8 @@ def test_forward_decay_full_forgetting(dtype, fmap, dqk, dv):
 
 
 @pytest.mark.parametrize("dtype", [W.F32, W.BF16])
-@pytest.mark.parametrize("fmap,dqk,dv", [(ELU1, 32, 32), (ELU1, 64, 64), (TAYLOR2_SYM, 16, 64), (TAYLOR2, 4, 8)])
+@pytest.mark.parametrize("fmap,dqk,dv", [(ELU1, 32, 32), (ELU1, 64, 64), (ELU1, 128, 128), (TAYLOR2, 16, 64),
+                                         (TAYLOR2_SYM, 16, 64), (TAYLOR2, 4, 8)])
 def test_backward_decay(fmap, dqk, dv, dtype):
     """Gated gradients, the gate's included, against the oracle's brute force."""
     for N in (1, 17, 64, 65, 200):
@@ -270,6 +271,26 @@ def test_backward_decay(fmap, dqk, dv, dtype):
             err = orc.max_rel_l2(got.cpu(), ref)
             assert err <= tol, (N, name, err)
         assert dg[..., 0].abs().max().item() <= 1e-4 * dg.abs().max().item()   # g_1 scales an empty state
+
+
+@pytest.mark.parametrize("fmap,dqk,dv", [(ELU1, 64, 64), (ELU1, 128, 128), (TAYLOR2, 16, 64), (TAYLOR2_SYM, 16, 64)])
+def test_backward_decay_segments(fmap, dqk, dv):
+    """The gated tensor-core backward with sequences cut into one-chunk
+    segments (2 heads, up to 1000 tokens: 8 segments), so that the S and R
+    increments, their gate-decayed sums and the suffix sum for dL/dg all run;
+    strong gates (down to e^-2 per token) and gates of exactly 0."""
+    for N, lo in ((300, -0.5), (1000, -0.05), (777, -2.0)):
+        q, k, v, do = W.random_qkv(9970 + N, 1, 2, N, dqk, dv, fmap=fmap, dtype=W.BF16,
+                                   scale=1.0 if fmap != ELU1 else dqk ** -0.5, with_dout=True)
+        g = _log_gates(9980 + N, 1, 2, N, lo=lo)
+        dq, dk, dvv, dg = la.la_backward_decay(q.to(DEV), k.to(DEV), v.to(DEV), g.to(DEV), do.to(DEV), fmap)
+        torch.cuda.synchronize()
+        la.la_get_device_status()
+        rq, rk, rv, rg = orc.backward_brute_decay(fmap, q, k, v, g, do)
+        for got, ref, name in ((dq, rq, "dq"), (dk, rk, "dk"), (dvv, rv, "dv"), (dg, rg, "dg")):
+            err = orc.max_rel_l2(got.cpu(), ref)
+            assert err <= 1e-2, (N, lo, name, err)
+        assert (dg[..., 0] == 0).all()
 
 
 def test_forward_decay_zero_gate_is_plain_forward():
