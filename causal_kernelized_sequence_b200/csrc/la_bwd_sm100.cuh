@@ -98,8 +98,10 @@ struct BwdCfg {
     static constexpr int OFF_V = OFF_K + PHI_TILE;
     static constexpr int OFF_G = OFF_V + VG_TILE;
     static constexpr int OFF_S = OFF_G + VG_TILE;
-    static constexpr int OFF_SL = OFF_S + S_TILE;        // low part of the state (forward-order pass) or of G'
-    static constexpr int OFF_RQ = OFF_SL + S_TILE;       // raw Q (Taylor)
+    // low part of the state (forward-order pass) or of G' (reverse pass)
+    static constexpr int SL_TILE = S_TILE > VG_TILE ? S_TILE : VG_TILE;
+    static constexpr int OFF_SL = OFF_S + S_TILE;
+    static constexpr int OFF_RQ = OFF_SL + SL_TILE;      // raw Q (Taylor)
     static constexpr int OFF_RK = OFF_RQ + RAW;          // raw K (Taylor)
     static constexpr int OFF_BAR = OFF_RK + RAW;
     static constexpr int OFF_RED = OFF_BAR + 128;        // per-row partial sums of the two threads of a row
@@ -121,6 +123,8 @@ struct BwdCfg {
     static_assert(NT * NA <= 256, "state tiles of the state passes");
     static_assert(PHI_TILE % 1024 == 0 && VG_TILE % 1024 == 0 && S_TILE % 256 == 0 && OFF_RQ % 1024 == 0,
                   "shared-memory alignment");
+    static_assert(SL_TILE >= S_TILE && SL_TILE >= VG_TILE && OFF_S + S_TILE >= OFF_G + VG_TILE,
+                  "the R snapshot fits the S region and the G' remainder the SL region");
     static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory");
 };
 
