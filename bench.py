@@ -279,7 +279,8 @@ class VarlenPrefill:
 
 
 class Train:
-    """One step = la_forward (o, den) + la_backward (dq, dk, dv)."""
+    """One step = la_forward (o, den) + la_backward (dq, dk, dv); for a gated
+    workload la_forward_decay + la_backward_decay (also dL/dg)."""
 
     def __init__(self, w, dev, seed_offset=0):
         import causal_kernelized_sequence_b200 as la
@@ -291,15 +292,23 @@ class Train:
         self.o = torch.empty_like(self.v)
         self.den = torch.empty(w.B, w.H, w.N, device=dev)
         self.dq, self.dk, self.dvv = torch.empty_like(self.q), torch.empty_like(self.k), torch.empty_like(self.v)
-        self.fws_bytes = la.la_forward_workspace_bytes(w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype)
-        self.bws_bytes = la.la_backward_workspace_bytes(w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype)
+        lib = la.load_library()
+        if w.decay:
+            self.gate = W.make_gates(w, device=dev, seed=replica_seed(w, seed_offset))
+            self.dgate = torch.empty_like(self.gate)
+            self.fws_bytes = lib.la_forward_decay_workspace_bytes(w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype)
+            self.bws_bytes = lib.la_backward_decay_workspace_bytes(w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype)
+        else:
+            self.fws_bytes = la.la_forward_workspace_bytes(w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype)
+            self.bws_bytes = la.la_backward_workspace_bytes(w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype)
         self.fws = torch.empty(max(1, self.fws_bytes), dtype=torch.uint8, device=dev)
         self.bws = torch.empty(max(1, self.bws_bytes), dtype=torch.uint8, device=dev)
         self.tokens = w.B * w.N
         e = 2
         BHN = w.B * w.H * w.N
-        self.fwd_bytes = BHN * (2 * w.dqk + 2 * w.dv) * e + BHN * 4
-        self.bwd_bytes = BHN * (2 * w.dqk + 2 * w.dv) * e + BHN * (2 * w.dqk + w.dv) * e
+        gb = 4 if w.decay else 0   # the gate, read by each pass; dL/dg written by the backward
+        self.fwd_bytes = BHN * (2 * w.dqk + 2 * w.dv) * e + BHN * 4 + BHN * gb
+        self.bwd_bytes = BHN * (2 * w.dqk + 2 * w.dv) * e + BHN * (2 * w.dqk + w.dv) * e + 2 * BHN * gb
         self.alg_bytes = self.fwd_bytes + self.bwd_bytes
         F = w.feature_dim
         self.alg_flops = (4.0 * F * (w.dv + 1) + 10.0 * F * w.dv + 6.0 * F) * BHN
@@ -311,6 +320,16 @@ class Train:
         import ctypes
         P = lambda t: ctypes.c_void_p(t.data_ptr())
         st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        if w.decay:
+            r = lib.la_forward_decay(P(self.q), P(self.k), P(self.v), P(self.gate), P(self.o), None, None, None, None,
+                                     P(self.den), P(self.fws), self.fws_bytes, w.B, w.H, w.N, w.dqk, w.dv, w.fmap,
+                                     w.dtype, st)
+            assert r == 0, r
+            r = lib.la_backward_decay(P(self.q), P(self.k), P(self.v), P(self.gate), P(self.do), P(self.dq),
+                                      P(self.dk), P(self.dvv), P(self.dgate), P(self.bws), self.bws_bytes,
+                                      w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype, st)
+            assert r == 0, r
+            return
         r = lib.la_forward(P(self.q), P(self.k), P(self.v), P(self.o), None, None, P(self.den), P(self.fws),
                            self.fws_bytes, w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype, st)
         assert r == 0, r
@@ -829,8 +848,9 @@ def main():
         # dram_x = DRAM bytes over algorithmic bytes (recorded ncu capture of
         # the current code, else absent).
         sec = {}
-        for name in ("elu_bf16_varlen", "elu_bf16_decay_fwd", "swa_bf16_fwd", "swa_bf16_decode",
-                     "taylor_decode_sym", "taylor_bf16_train", "taylor_decode", "elu_bf16_train", "taylor_bf16_fwd"):
+        for name in ("elu_bf16_varlen", "elu_bf16_decay_fwd", "elu_bf16_decay_train", "swa_bf16_fwd",
+                     "swa_bf16_decode", "taylor_decode_sym", "taylor_bf16_train", "taylor_decode", "elu_bf16_train",
+                     "taylor_bf16_fwd"):
             ws = W.BY_NAME[name]
             r2 = make_run(ws, dev, 0)
             st = 3 if ws.decode_steps else 50

@@ -478,7 +478,10 @@ def kernel_plan(w):
     op = 3 if getattr(w, "varlen", False) else 4 if getattr(w, "decay", False) else 0
     n, names = la_kernel_plan(op, w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype)
     if w.backward:
-        n2, names2 = la_kernel_plan(1, w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype)
+        decay = getattr(w, "decay", False)
+        n2, names2 = la_kernel_plan(5 if decay else 1, w.B, w.H, w.N, w.dqk, w.dv, w.fmap, w.dtype)
+        if n2 < 0:   # a gated backward outside the tensor-core shapes: the CUDA-core kernel
+            n2, names2 = 1, ["bwd_simt_kernel"]
         n, names = n + n2, names + names2
     return {"launches_per_step": n, "kernels": names}
 

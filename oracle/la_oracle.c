@@ -62,6 +62,15 @@
  *               The recurrent version scans s,z forward for dq and
  *               R_j = sum_{i>=j} phi(q_i) g_i^T, r_j = sum_{i>=j} phi(q_i) dden_i
  *               backward for dk, dv.
+ *   backward_brute_decay / backward_recurrent_decay -- the same for the
+ *               gated form, with w_ij = (prod_{l=j+1..i} a_l) a_ij in place of
+ *               a_ij, and dL/dg_l for the log gates.  The brute version sums
+ *               dL/dw_ij w_ij over the pairs j < l <= i that g_l scales.  The
+ *               recurrent version scans the gated s, z forward and the gated
+ *               R_j = phi(q_j) g_j^T + a_{j+1} R_{j+1} backward; with
+ *               B_m = g_1 + .. + g_m, w_ij = exp(B_i - B_j) a_ij, so
+ *               dL/dB_m = phi(q_m).dphiq_m - phi(k_m).dphik_m (the row sum of
+ *               w dL/dw minus the column sum) and dL/dg_l = sum_{m>=l} dL/dB_m.
  *
  * Parallelism: OpenMP over (b,h) slices only; each slice is computed in the
  * plain order above.
@@ -595,5 +604,89 @@ void orc_backward_brute_decay(int fmap, int B, int H, int N, int dqk, int dv,
             orc_phi_vjp(fmap, dqk, ks + (size_t)i * dqk, dphik + (size_t)i * F, dk + ((size_t)bh * N + i) * dqk);
         }
         free(phiq); free(phik); free(e); free(w); free(gi); free(dd); free(dphiq); free(dphik);
+    }
+}
+
+/* Gated gradients by scans (the header's backward_recurrent_decay). */
+void orc_backward_recurrent_decay(int fmap, int B, int H, int N, int dqk, int dv,
+                                  const double *q, const double *k, const double *v, const double *gate,
+                                  const double *dout, double *dq, double *dk, double *dvv, double *dgate)
+{
+    const int BH = B * H;
+    const int F = orc_feature_dim(fmap, dqk);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int bh = 0; bh < BH; ++bh) {
+        const double *qs = q + (size_t)bh * N * dqk;
+        const double *ks = k + (size_t)bh * N * dqk;
+        const double *vs = v + (size_t)bh * N * dv;
+        const double *gs = gate + (size_t)bh * N;
+        const double *dos = dout + (size_t)bh * N * dv;
+        double *dqs = dq + (size_t)bh * N * dqk;
+        double *dks = dk + (size_t)bh * N * dqk;
+        double *dvs = dvv + (size_t)bh * N * dv;
+        double *dgs = dgate + (size_t)bh * N;
+        double *s = (double *)calloc((size_t)F * dv, sizeof(double));
+        double *z = (double *)calloc((size_t)F, sizeof(double));
+        double *g = (double *)malloc(sizeof(double) * (size_t)N * dv);
+        double *dden = (double *)malloc(sizeof(double) * (size_t)N);
+        double *dB = (double *)malloc(sizeof(double) * (size_t)N);   /* dL/dB_m */
+        double *phiq = (double *)malloc(sizeof(double) * (size_t)F);
+        double *phik = (double *)malloc(sizeof(double) * (size_t)F);
+        double *dphi = (double *)malloc(sizeof(double) * (size_t)F);
+        /* Forward-order scan: the gated s_i, z_i include token i. */
+        for (int i = 0; i < N; ++i) {
+            orc_phi(fmap, dqk, qs + (size_t)i * dqk, phiq);
+            orc_phi(fmap, dqk, ks + (size_t)i * dqk, phik);
+            const double a = exp(gs[i]);
+            for (int f = 0; f < F; ++f) {
+                for (int c = 0; c < dv; ++c)
+                    s[(size_t)f * dv + c] = a * s[(size_t)f * dv + c] + phik[f] * vs[(size_t)i * dv + c];
+                z[f] = a * z[f] + phik[f];
+            }
+            const double d = dot(phiq, z, F);
+            double gy = 0.0;
+            for (int c = 0; c < dv; ++c) {
+                double n = 0.0;
+                for (int f = 0; f < F; ++f) n += phiq[f] * s[(size_t)f * dv + c];
+                g[(size_t)i * dv + c] = dos[(size_t)i * dv + c] / d;
+                gy += g[(size_t)i * dv + c] * (n / d);
+            }
+            dden[i] = -gy;
+            /* dphi(q_i) = s_i g_i + z_i dden_i */
+            for (int f = 0; f < F; ++f)
+                dphi[f] = dot(s + (size_t)f * dv, g + (size_t)i * dv, dv) + z[f] * dden[i];
+            dB[i] = dot(phiq, dphi, F);
+            orc_phi_vjp(fmap, dqk, qs + (size_t)i * dqk, dphi, dqs + (size_t)i * dqk);
+        }
+        /* Reverse-order scan: R_j = phi(q_j) g_j^T + a_{j+1} R_{j+1} (reusing s), r_j (reusing z). */
+        memset(s, 0, sizeof(double) * (size_t)F * dv);
+        memset(z, 0, sizeof(double) * (size_t)F);
+        for (int j = N - 1; j >= 0; --j) {
+            orc_phi(fmap, dqk, qs + (size_t)j * dqk, phiq);
+            orc_phi(fmap, dqk, ks + (size_t)j * dqk, phik);
+            const double a_next = j + 1 < N ? exp(gs[j + 1]) : 0.0;
+            for (int f = 0; f < F; ++f) {
+                for (int c = 0; c < dv; ++c)
+                    s[(size_t)f * dv + c] = a_next * s[(size_t)f * dv + c] + phiq[f] * g[(size_t)j * dv + c];
+                z[f] = a_next * z[f] + phiq[f] * dden[j];
+            }
+            /* dphi(k_j) = R_j v_j + r_j ; dv_j = R_j^T phi(k_j) */
+            for (int f = 0; f < F; ++f)
+                dphi[f] = dot(s + (size_t)f * dv, vs + (size_t)j * dv, dv) + z[f];
+            dB[j] -= dot(phik, dphi, F);
+            orc_phi_vjp(fmap, dqk, ks + (size_t)j * dqk, dphi, dks + (size_t)j * dqk);
+            for (int c = 0; c < dv; ++c) {
+                double acc = 0.0;
+                for (int f = 0; f < F; ++f) acc += s[(size_t)f * dv + c] * phik[f];
+                dvs[(size_t)j * dv + c] = acc;
+            }
+        }
+        /* dL/dg_l = sum_{m>=l} dL/dB_m */
+        double suffix = 0.0;
+        for (int l = N - 1; l >= 0; --l) {
+            suffix += dB[l];
+            dgs[l] = suffix;
+        }
+        free(s); free(z); free(g); free(dden); free(dB); free(phiq); free(phik); free(dphi);
     }
 }

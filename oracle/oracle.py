@@ -62,11 +62,12 @@ def _load():
             lib.orc_swa_forward.argtypes = [I, I, I, I, I, I, ctypes.c_double] + [_d] * 5
             lib.orc_backward_brute_decay.argtypes = [I, I, I, I, I, I] + [_d] * 9
             lib.orc_backward_recurrent.argtypes = [I, I, I, I, I, I, _d, _d, _d, _d, _d, _d, _d]
+            lib.orc_backward_recurrent_decay.argtypes = [I, I, I, I, I, I] + [_d] * 9
             for f in (lib.orc_phi, lib.orc_phi_vjp, lib.orc_forward_brute, lib.orc_forward_rows,
                       lib.orc_forward_recurrent, lib.orc_decode_step, lib.orc_backward_brute,
                       lib.orc_backward_recurrent, lib.orc_forward_recurrent_decay,
                       lib.orc_forward_brute_decay, lib.orc_decode_step_decay, lib.orc_swa_forward,
-                      lib.orc_backward_brute_decay):
+                      lib.orc_backward_brute_decay, lib.orc_backward_recurrent_decay):
                 f.restype = None
             _lib = lib
     return _lib
@@ -273,6 +274,20 @@ def backward_brute_decay(fmap: int, q, k, v, g, dout):
     dq = np.empty_like(q); dk = np.empty_like(k); dvv = np.empty_like(v); dg = np.empty_like(g)
     _load().orc_backward_brute_decay(fmap, B, H, N, dqk, dv, _p(q), _p(k), _p(v), _p(g), _p(dout),
                                      _p(dq), _p(dk), _p(dvv), _p(dg))
+    return dq, dk, dvv, dg
+
+
+def backward_recurrent_decay(fmap: int, q, k, v, g, dout):
+    """The gated gradients (dq, dk, dv, dg) by a forward scan of the gated
+    state (dq) and a backward scan of the gated R (dk, dv); dg from the
+    per-token dL/dB_m = phi(q_m).dphiq_m - phi(k_m).dphik_m, summed from the
+    end.  O(N F dv) per slice, for the full-size workloads."""
+    q, k, v, g, dout = _f64(q), _f64(k), _f64(v), _f64(g), _f64(dout)
+    B, H, N, dqk = q.shape
+    dv = v.shape[-1]
+    dq = np.empty_like(q); dk = np.empty_like(k); dvv = np.empty_like(v); dg = np.empty_like(g)
+    _load().orc_backward_recurrent_decay(fmap, B, H, N, dqk, dv, _p(q), _p(k), _p(v), _p(g), _p(dout),
+                                         _p(dq), _p(dk), _p(dvv), _p(dg))
     return dq, dk, dvv, dg
 
 

@@ -466,6 +466,23 @@ def test_decay_backward_autograd(orc):
         np.testing.assert_allclose(a, t.grad.numpy(), rtol=1e-9, atol=1e-11)
 
 
+@pytest.mark.parametrize("fmap,d,dv", [(ELU1, 5, 4), (TAYLOR2, 3, 4), (TAYLOR2_SYM, 4, 3)])
+def test_decay_backward_recurrent_equals_brute(orc, fmap, d, dv):
+    # The scan form (gated state forward, gated R backward, dL/dg from the
+    # per-token dL/dB_m) equals the pairwise brute force (pinned above by
+    # finite differences and autograd), with gates of 0 and of -inf among them.
+    N = 45
+    q = rnd(220, 2, 2, N, d, scale=0.7); k = rnd(221, 2, 2, N, d, scale=0.7)
+    v = rnd(222, 2, 2, N, dv); do = rnd(223, 2, 2, N, dv)
+    g = -np.abs(rnd(224, 2, 2, N)) * 0.6
+    g[..., ::6] = 0.0
+    g[0, 1, 17] = -np.inf
+    a = orc.backward_brute_decay(fmap, q, k, v, g, do)
+    b = orc.backward_recurrent_decay(fmap, q, k, v, g, do)
+    for x, y in zip(a, b):
+        np.testing.assert_allclose(y, x, rtol=1e-10, atol=1e-12 * np.abs(x).max())
+
+
 # ------------------------------------------------- sliding-window attention
 
 def test_swa_wide_window_is_causal_softmax_attention(orc):

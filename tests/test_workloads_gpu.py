@@ -143,6 +143,29 @@ def test_workload_taylor_bf16_train():
     assert ((lhs - rhs).norm() / rhs.norm()).item() < 1e-2
 
 
+def test_workload_elu_bf16_decay_train():
+    """The gated training step on the headline shape: gated forward and the
+    gated tensor-core backward, every head against the oracle's gated scans
+    (dq, dk, dv and dL/dg)."""
+    w = W.BY_NAME["elu_bf16_decay_train"]
+    q, k, v, do = W.make_inputs(w)
+    g = W.make_gates(w)
+    qd, kd, vd, dod, gd = (t.to(DEV) for t in (q, k, v, do, g))
+    fr = la.la_forward(qd, kd, vd, w.fmap, den=True, log_decay=gd)
+    dq, dk, dvv, dg = la.la_backward_decay(qd, kd, vd, gd, dod, w.fmap)
+    torch.cuda.synchronize()
+    la.la_get_device_status()
+    clk = _Clock()
+    o_ref, den_ref, _, _ = clk(orc.forward_recurrent_decay, w.fmap, q, k, v, g)
+    rq, rk, rv, rg = clk(orc.backward_recurrent_decay, w.fmap, q, k, v, g, do)
+    errs = {n: orc.max_rel_l2(got.cpu(), ref) for n, got, ref in
+            (("o", fr["o"], o_ref), ("den", fr["den"], den_ref), ("dq", dq, rq), ("dk", dk, rk), ("dv", dvv, rv),
+             ("dg", dg, rg))}
+    _record("elu_bf16_decay_train", slices=w.B * w.H, oracle_s=round(clk.s, 2), **errs)
+    _check(errs, 1e-2)
+    assert (dg[..., 0] == 0).all()
+
+
 def test_workload_elu_bf16_decay_fwd():
     w = W.BY_NAME["elu_bf16_decay_fwd"]
     q, k, v, _ = W.make_inputs(w)

@@ -23,6 +23,7 @@ The workloads, with the sizes used throughout the tests and the benchmark:
   swa_bf16_decode    its decode: 1024 x 16 heads, 64-token caches, 1024 steps
   taylor_bf16_train  the Taylor forward's shape as a training step (forward +
                      backward), inputs and upstream grad N(0,1)
+  elu_bf16_decay_train the gated form's training step on the headline shape
 
 Random numbers come from torch's CPU Mersenne-Twister generator seeded with
 the workload's index; tensors are drawn in the order Q, K, V, dO (decode: the
@@ -120,6 +121,9 @@ WORKLOADS = [
     # the BASED Taylor shape as a training step: forward + backward, inputs and
     # upstream gradient N(0,1)
     Workload("taylor_bf16_train", 9, TAYLOR2, BF16, 8, 16, 2048, 16, 64, 1.0, backward=True),
+    # the gated form as a training step on the headline shape (gates as elu_bf16_decay_fwd's)
+    Workload("elu_bf16_decay_train", 10, ELU1, BF16, 4, 8, 4096, 64, 64, 1.0 / math.sqrt(64), backward=True,
+             decay=True),
 ]
 BY_NAME = {w.name: w for w in WORKLOADS}
 
