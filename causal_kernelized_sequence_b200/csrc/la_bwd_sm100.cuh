@@ -819,6 +819,110 @@ __device__ __forceinline__ void mask_pack_half_hilo_gate(uint32_t src, uint32_t 
     tmem_st_wait();
 }
 
+
+// Reverse pass, gated: P^T and dP^T of this thread's 64 columns from j0 in one
+// step (row j is a key, column i a query; weight exp(L_i - L_j); with TAY the
+// raw scores s become 1 + s k1 + s^2 k2 first), and the row's part of
+// c_j = sum_i dL/dw_ij w_ij from the fp32 scores and dA^T (not from the
+// rounded operands of the later MMAs).  P^T overwrites the scores' columns,
+// so the block meets at a barrier between loading and storing (every thread
+// must call this).
+template <bool TAY, typename Keep>
+__device__ __forceinline__ float mask_pack_both_gate(uint32_t tA, uint32_t tX, uint32_t tPL, int j0, float k1, float k2,
+                                                     float rowL, const float *colL, Keep keep)
+{
+    float w[64];
+    tmem_ld32(tA + j0, w);
+    tmem_ld32(tA + j0 + 32, w + 32);
+    tmem_ld_wait();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+#pragma unroll
+    for (int e = 0; e < 64; ++e) {
+        float a = w[e];
+        if constexpr (TAY) a = fmaf(a, fmaf(a, k2, k1), 1.f);
+        w[e] = keep(j0 + e) ? a * __expf(colL[j0 + e] - rowL) : 0.f;
+    }
+    {
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 64; e += 2) pk[e / 2] = pack_bf16(w[e], w[e + 1]);
+        tmem_st32(tA + j0 / 2, pk);
+    }
+    float c = 0.f;
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+        float d[32];
+        tmem_ld32(tX + j0 + 32 * h2, d);
+        tmem_ld_wait();
+        uint32_t hi[16], lo[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+            const int i0 = j0 + 32 * h2 + e;
+            const float x0 = keep(i0) ? d[e] * __expf(colL[i0] - rowL) : 0.f;
+            const float x1 = keep(i0 + 1) ? d[e + 1] * __expf(colL[i0 + 1] - rowL) : 0.f;
+            c = fmaf(d[e], w[32 * h2 + e], c);          // w is 0 where masked
+            c = fmaf(d[e + 1], w[32 * h2 + e + 1], c);
+            hi[e / 2] = pack_bf16(x0, x1);
+            lo[e / 2] = pack_bf16(x0 - __bfloat162float(__float2bfloat16_rn(x0)),
+                                  x1 - __bfloat162float(__float2bfloat16_rn(x1)));
+        }
+        tmem_st16(tA + 64 + (j0 + 32 * h2) / 2, reinterpret_cast<const float *>(hi));
+        tmem_st16(tPL + (j0 + 32 * h2) / 2, reinterpret_cast<const float *>(lo));
+    }
+    tmem_st_wait();
+    return c;
+}
+
+// phi(k_j) . X_j over features [80 HALF, 80 HALF + 80) of the Taylor map, X
+// read from TMEM columns tcol + f, phi from the raw row x.
+template <int F0, int... E>
+__device__ __forceinline__ float tay_dot_seq(const float *g, const float *x, const BwdParams &p,
+                                             std::integer_sequence<int, E...>)
+{
+    float acc = 0.f;
+    ((acc = fmaf(g[E], tay_feat<F0 + E>(x, p), acc)), ...);
+    return acc;
+}
+template <int F0>
+__device__ __forceinline__ float tay_dot16(uint32_t tcol, const float *x, const BwdParams &p)
+{
+    float g[16];
+    tmem_ld16(tcol + F0, g);
+    tmem_ld_wait();
+    return tay_dot_seq<F0>(g, x, p, std::make_integer_sequence<int, 16>{});
+}
+template <int FB, int... G>
+__device__ __forceinline__ float tay_dot_groups(uint32_t tcol, const float *x, const BwdParams &p,
+                                                std::integer_sequence<int, G...>)
+{
+    return (tay_dot16<FB + 16 * G>(tcol, x, p) + ...);
+}
+template <int HALF>
+__device__ __forceinline__ float tay_dot_half(uint32_t tcol, const float *x, const BwdParams &p)
+{
+    return tay_dot_groups<80 * HALF>(tcol, x, p, std::make_integer_sequence<int, 5>{});
+}
+
+// phi(k_j) . X_j over feature columns [c_lo, c_hi) of an elu phi tile (bf16,
+// row j) and TMEM columns tcol + f.
+__device__ __forceinline__ float elu_dot_cols(uint32_t tcol, uint32_t phi_tile, int j, int c_lo, int c_hi)
+{
+    float acc = 0.f;
+#pragma unroll 1
+    for (int c0 = c_lo; c0 < c_hi; c0 += 16) {
+        float g[16], ph[16];
+        tmem_ld16(tcol + c0, g);
+        tmem_ld_wait();
+        unpack8(lds128(phi_tile + sw128_off(j, c0)), ph);
+        unpack8(lds128(phi_tile + sw128_off(j, c0 + 8)), ph + 8);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) acc = fmaf(g[e], ph[e], acc);
+    }
+    return acc;
+}
+
 }  // namespace bwd_detail
 
 // ---------------------------------------------------------------------------
@@ -1108,12 +1212,20 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
         full_sync();
 
-        // dA = G'' V_aug^T  (K = the NA augmented columns)
+        // dA = G'' V_aug^T  (K = the NA augmented columns).  bf16: the
+        // remainder of G'' too, so that dA_ij = dO_i . (v_j - y_i) keeps ~16 bits
+        // where its two terms cancel (with one token, y_1 = v_1 and dA_11 = 0)
         if (tid == 0) {
 #pragma unroll
             for (int kk = 0; kk < NA / 16; ++kk)
                 mma_bf16(tX, smem_desc(aG + kk * Cfg::BLK, 16, 256, kSw32), smem_desc(aV + kk * Cfg::BLK, 16, 256, kSw32),
                          F16 ? idesc_f16(128, 128, 0, 0) : idesc_bf16(128, 128, 0, 0), kk > 0);
+            if constexpr (!F16) {
+#pragma unroll
+                for (int kk = 0; kk < NA / 16; ++kk)
+                    mma_bf16_ts(tX, tGL + kk * 8, smem_desc(aV + kk * Cfg::BLK, 16, 256, kSw32),
+                                idesc_bf16(128, 128, 0, 0), true);
+            }
             mma_commit(mma_bar);
         }
         if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
@@ -1756,11 +1868,10 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mph ^= 1u;
         tc_fence_after();
         // row j keeps the queries i >= j
+        float c_part = 0.f;   // gated: this thread's part of c_j = sum_i dL/dw_ij w_ij
         if constexpr (GATED) {
-            mask_pack_half_gate<false, TAY>(tA + lane, tA + lane, 64 * hh, true, p.inv_c3, p.k2, Lrow, gL, false,
-                                            [&](int i) { return i >= j; });
-            mask_pack_half_hilo_gate(tX + lane, tA + lane + 64, tPL + lane, 64 * hh, Lrow, gL,
-                                     [&](int i) { return i >= j; });
+            c_part = mask_pack_both_gate<TAY>(tA + lane, tX + lane, tPL + lane, 64 * hh, p.inv_c3, p.k2, Lrow, gL,
+                                              [&](int i) { return i >= j; });
         } else {
             mask_pack_half_g<false, TAY>(tA + lane, tA + lane, 64 * hh, true, p.inv_c3, p.k2,
                                          [&](int i) { return i >= j; });
@@ -1839,7 +1950,18 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
             mph ^= 1u;
             tc_fence_after();
-            tmem_scale(tX + lane, hh * (F / 2), (hh + 1) * (F / 2), __expf(Llast - Lrow));
+            // the later chunks' part of c_j: phi(k_j) . (their term of dphi(k_j))
+            const float w = __expf(Llast - Lrow);
+            float dot;
+            if constexpr (TAY) {
+                float xk[16];
+                raw_row16(aRK, j, xk);
+                dot = hh == 0 ? tay_dot_half<0>(tX + lane, xk, p) : tay_dot_half<1>(tX + lane, xk, p);
+            } else {
+                dot = elu_dot_cols(tX + lane, aK, j, hh * (F / 2), (hh + 1) * (F / 2));
+            }
+            c_part = fmaf(w, dot, c_part);
+            tmem_scale(tX + lane, hh * (F / 2), (hh + 1) * (F / 2), w);
             full_sync();
         }
 
@@ -1881,13 +2003,11 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 else tay_vjp_half<1>(tX + lane, x, dx, sd, p);
                 float d8[8], sd_all;
                 tay_combine(red + 6 * C, red + 2 * C, hh, j, dx, sd, d8, sd_all);
-                if (GATED && hh == 0 && valid) p.cvec[(size_t)bh * N + t0 + j] = sd_all;   // phi(k_j) . dphi(k_j)
                 if (valid)
                     *reinterpret_cast<uint4 *>(dkrow + 8 * hh) =
                         make_uint4(pack_bf16(d8[0], d8[1]), pack_bf16(d8[2], d8[3]), pack_bf16(d8[4], d8[5]),
                                    pack_bf16(d8[6], d8[7]));
             } else {
-                float sd = 0.f;   // gated: phi(k_j) . dphi(k_j) over this thread's features
 #pragma unroll 1
                 for (int c0 = hh * (F / 2); c0 < (hh + 1) * (F / 2); c0 += 16) {
                     float g[16], ph[16];
@@ -1895,10 +2015,6 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     tmem_ld_wait();
                     unpack8(lds128(aK + sw128_off(j, c0)), ph);
                     unpack8(lds128(aK + sw128_off(j, c0 + 8)), ph + 8);
-                    if constexpr (GATED) {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) sd = fmaf(g[e], ph[e], sd);
-                    }
                     if (valid)
 #pragma unroll
                         for (int e = 0; e < 16; e += 8)
@@ -1908,11 +2024,12 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                 pack_bf16(g[e + 4] * fminf(ph[e + 4], 1.f), g[e + 5] * fminf(ph[e + 5], 1.f)),
                                 pack_bf16(g[e + 6] * fminf(ph[e + 6], 1.f), g[e + 7] * fminf(ph[e + 7], 1.f)));
                 }
-                if constexpr (GATED) {
-                    red[2 * C + hh * C + j] = sd;
-                    __syncthreads();
-                    if (hh == 0 && valid) p.cvec[(size_t)bh * N + t0 + j] = red[2 * C + j] + red[3 * C + j];
-                }
+            }
+            if constexpr (GATED) {
+                // c_j = phi(k_j) . dphi(k_j), summed over the row's two threads
+                red[4 * C + hh * C + j] = c_part;
+                __syncthreads();
+                if (hh == 0 && valid) p.cvec[(size_t)bh * N + t0 + j] = red[4 * C + j] + red[5 * C + j];
             }
             if (chunk > c_begin) {
 #pragma unroll
