@@ -106,8 +106,10 @@ struct BwdCfg {
     static constexpr int OFF_BAR = OFF_RK + RAW;
     static constexpr int OFF_RED = OFF_BAR + 128;        // per-row partial sums of the two threads of a row
     static constexpr int RED_FLOATS = 6 * C + (TAYLOR ? 2 * C * 16 : 0);
-    static constexpr int OFF_GATE = OFF_RED + RED_FLOATS * 4;   // gated form: [C] prefix sums, [4] quadrant totals
-    static constexpr int SMEM_ALLOC = OFF_GATE + (C + 8) * 4 + 1024;
+    // gated form: [C] prefix sums of the gates, [8] quadrant totals, then (reverse
+    // pass) [F] the bf16 remainder of R's normaliser column
+    static constexpr int OFF_GATE = OFF_RED + RED_FLOATS * 4;
+    static constexpr int SMEM_ALLOC = OFF_GATE + (C + 8 + F) * 4 + 1024;
     // TMEM columns.  Forward-order pass: [0, 128) scores -> P | dP; X: O_aug,
     // then dA, then dphi(Q); S: the state tiles; GL: the remainder of G''.
     // Reverse pass: [0, 128) scores -> P^T | dP^T; X: dA^T, then dV, then
@@ -820,6 +822,8 @@ __device__ __forceinline__ void mask_pack_half_hilo_gate(uint32_t src, uint32_t 
 }
 
 
+__device__ __forceinline__ float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+
 // Reverse pass, gated: P^T and dP^T of this thread's 64 columns from j0 in one
 // step (row j is a key, column i a query; weight exp(L_i - L_j); with TAY the
 // raw scores s become 1 + s k1 + s^2 k2 first), and the row's part of
@@ -827,7 +831,7 @@ __device__ __forceinline__ void mask_pack_half_hilo_gate(uint32_t src, uint32_t 
 // rounded operands of the later MMAs).  P^T overwrites the scores' columns,
 // so the block meets at a barrier between loading and storing (every thread
 // must call this).
-template <bool TAY, typename Keep>
+template <bool TAY, bool F16R, typename Keep>
 __device__ __forceinline__ float mask_pack_both_gate(uint32_t tA, uint32_t tX, uint32_t tPL, int j0, float k1, float k2,
                                                      float rowL, const float *colL, Keep keep)
 {
@@ -862,8 +866,11 @@ __device__ __forceinline__ float mask_pack_both_gate(uint32_t tA, uint32_t tX, u
             const int i0 = j0 + 32 * h2 + e;
             const float x0 = keep(i0) ? d[e] * __expf(colL[i0] - rowL) : 0.f;
             const float x1 = keep(i0 + 1) ? d[e + 1] * __expf(colL[i0 + 1] - rowL) : 0.f;
-            c = fmaf(d[e], w[32 * h2 + e], c);          // w is 0 where masked
-            c = fmaf(d[e + 1], w[32 * h2 + e + 1], c);
+            // the weights rounded as the forward-order pass rounded them for y
+            // (F16R: to fp16; 0 where masked)
+            c = fmaf(d[e], F16R ? __half2float(__float2half_rn(w[32 * h2 + e])) : bf16_round(w[32 * h2 + e]), c);
+            c = fmaf(d[e + 1], F16R ? __half2float(__float2half_rn(w[32 * h2 + e + 1])) : bf16_round(w[32 * h2 + e + 1]),
+                     c);
             hi[e / 2] = pack_bf16(x0, x1);
             lo[e / 2] = pack_bf16(x0 - __bfloat162float(__float2bfloat16_rn(x0)),
                                   x1 - __bfloat162float(__float2bfloat16_rn(x1)));
@@ -878,36 +885,38 @@ __device__ __forceinline__ float mask_pack_both_gate(uint32_t tA, uint32_t tX, u
 // phi(k_j) . X_j over features [80 HALF, 80 HALF + 80) of the Taylor map, X
 // read from TMEM columns tcol + f, phi from the raw row x.
 template <int F0, int... E>
-__device__ __forceinline__ float tay_dot_seq(const float *g, const float *x, const BwdParams &p,
+__device__ __forceinline__ float tay_dot_seq(const float *g, const float *x, const float *dr, const BwdParams &p,
                                              std::integer_sequence<int, E...>)
 {
     float acc = 0.f;
-    ((acc = fmaf(g[E], tay_feat<F0 + E>(x, p), acc)), ...);
+    ((acc = fmaf(g[E] + dr[F0 + E], tay_feat<F0 + E>(x, p), acc)), ...);
     return acc;
 }
 template <int F0>
-__device__ __forceinline__ float tay_dot16(uint32_t tcol, const float *x, const BwdParams &p)
+__device__ __forceinline__ float tay_dot16(uint32_t tcol, const float *x, const float *dr, const BwdParams &p)
 {
     float g[16];
     tmem_ld16(tcol + F0, g);
     tmem_ld_wait();
-    return tay_dot_seq<F0>(g, x, p, std::make_integer_sequence<int, 16>{});
+    return tay_dot_seq<F0>(g, x, dr, p, std::make_integer_sequence<int, 16>{});
 }
 template <int FB, int... G>
-__device__ __forceinline__ float tay_dot_groups(uint32_t tcol, const float *x, const BwdParams &p,
+__device__ __forceinline__ float tay_dot_groups(uint32_t tcol, const float *x, const float *dr, const BwdParams &p,
                                                 std::integer_sequence<int, G...>)
 {
-    return (tay_dot16<FB + 16 * G>(tcol, x, p) + ...);
+    return (tay_dot16<FB + 16 * G>(tcol, x, dr, p) + ...);
 }
+// ... plus dr_f per feature (the bf16 remainder of R's normaliser column).
 template <int HALF>
-__device__ __forceinline__ float tay_dot_half(uint32_t tcol, const float *x, const BwdParams &p)
+__device__ __forceinline__ float tay_dot_half(uint32_t tcol, const float *x, const float *dr, const BwdParams &p)
 {
-    return tay_dot_groups<80 * HALF>(tcol, x, p, std::make_integer_sequence<int, 5>{});
+    return tay_dot_groups<80 * HALF>(tcol, x, dr, p, std::make_integer_sequence<int, 5>{});
 }
 
-// phi(k_j) . X_j over feature columns [c_lo, c_hi) of an elu phi tile (bf16,
-// row j) and TMEM columns tcol + f.
-__device__ __forceinline__ float elu_dot_cols(uint32_t tcol, uint32_t phi_tile, int j, int c_lo, int c_hi)
+// phi(k_j) . (X_j + dr) over feature columns [c_lo, c_hi) of an elu phi tile
+// (bf16, row j), X from TMEM columns tcol + f.
+__device__ __forceinline__ float elu_dot_cols(uint32_t tcol, uint32_t phi_tile, int j, int c_lo, int c_hi,
+                                              const float *dr)
 {
     float acc = 0.f;
 #pragma unroll 1
@@ -918,7 +927,7 @@ __device__ __forceinline__ float elu_dot_cols(uint32_t tcol, uint32_t phi_tile, 
         unpack8(lds128(phi_tile + sw128_off(j, c0)), ph);
         unpack8(lds128(phi_tile + sw128_off(j, c0 + 8)), ph + 8);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) acc = fmaf(g[e], ph[e], acc);
+        for (int e = 0; e < 16; ++e) acc = fmaf(g[e] + dr[c0 + e], ph[e], acc);
     }
     return acc;
 }
@@ -1115,6 +1124,10 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     const uint32_t off = (kk >> 2) * (C * 128) + (kk & 3) * 32;
                     mma_bf16(tX, smem_desc(aQ + off, 16, 1024, kSw128), smem_desc(aS + kk * 512, Cfg::S_BLK, 256, kSw32),
                              id_o, kk > 0);
+                    // and its remainder: y_i, hence dden_i, must agree to ~16 bits with
+                    // the weights the reverse pass sums into dL/dg (see bwd_dg_kernel)
+                    mma_bf16(tX, smem_desc(aQ + off, 16, 1024, kSw128), smem_desc(aSL + kk * 512, Cfg::S_BLK, 256, kSw32),
+                             id_o, true);
                 }
                 mma_commit(mma_bar);
             }
@@ -1723,11 +1736,13 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int na_lo = hh ? Cfg::NA_SPLIT : 0, na_hi = hh ? NA : Cfg::NA_SPLIT;   // this thread's columns of R_aug
     const uint32_t tA = tmem, tX = tmem + Cfg::COL_X, tR = tmem + Cfg::COL_R, tPL = tmem + Cfg::COL_PL;
     float *gL = reinterpret_cast<float *>(smem + Cfg::OFF_GATE);   // gated: the chunk's prefix sums of the gates
+    float *dr = gL + C + 8;   // gated: r - bf16(r) per feature, r = R's normaliser column
     auto snap_r = [&](int f, int c0, const float *v) {
         sts128(aR + sw32_off(f, c0, F), make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
                                                    pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7])));
         sts128(aR + sw32_off(f, c0 + 8, F), make_uint4(pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]),
                                                        pack_bf16(v[12], v[13]), pack_bf16(v[14], v[15])));
+        if (GATED && c0 == DV) dr[f] = v[0] - bf16_round(v[0]);
     };
 
     // ---- R entering the segment: sum of the later segments' increments
@@ -1870,7 +1885,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // row j keeps the queries i >= j
         float c_part = 0.f;   // gated: this thread's part of c_j = sum_i dL/dw_ij w_ij
         if constexpr (GATED) {
-            c_part = mask_pack_both_gate<TAY>(tA + lane, tX + lane, tPL + lane, 64 * hh, p.inv_c3, p.k2, Lrow, gL,
+            c_part = mask_pack_both_gate<TAY, Cfg::F16>(tA + lane, tX + lane, tPL + lane, 64 * hh, p.inv_c3, p.k2, Lrow, gL,
                                               [&](int i) { return i >= j; });
         } else {
             mask_pack_half_g<false, TAY>(tA + lane, tA + lane, 64 * hh, true, p.inv_c3, p.k2,
@@ -1956,9 +1971,9 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if constexpr (TAY) {
                 float xk[16];
                 raw_row16(aRK, j, xk);
-                dot = hh == 0 ? tay_dot_half<0>(tX + lane, xk, p) : tay_dot_half<1>(tX + lane, xk, p);
+                dot = hh == 0 ? tay_dot_half<0>(tX + lane, xk, dr, p) : tay_dot_half<1>(tX + lane, xk, dr, p);
             } else {
-                dot = elu_dot_cols(tX + lane, aK, j, hh * (F / 2), (hh + 1) * (F / 2));
+                dot = elu_dot_cols(tX + lane, aK, j, hh * (F / 2), (hh + 1) * (F / 2), dr);
             }
             c_part = fmaf(w, dot, c_part);
             tmem_scale(tX + lane, hh * (F / 2), (hh + 1) * (F / 2), w);

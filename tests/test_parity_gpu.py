@@ -156,10 +156,13 @@ def test_forward_varlen(fmap, dqk, dv, dtype):
 
 def test_forward_varlen_matches_fixed_length():
     """Equal lengths packed are the fixed-length batch: same bits from the
-    same kernel (Taylor bf16, one launch either way)."""
+    same kernel (Taylor bf16).  A zero start state selects the one-launch
+    kernel for the fixed-length call, the one the packed call runs."""
     B, H, N = 3, 2, 700
     q, k, v, _ = W.random_qkv(8200, B, H, N, 16, 64, fmap=TAYLOR2, dtype=W.BF16)
-    fixed = gpu_forward(q, k, v, TAYLOR2, state=True, den=True)
+    F = la.la_feature_dim(TAYLOR2, 16)
+    fixed = gpu_forward(q, k, v, TAYLOR2, state=True, den=True, s_in=torch.zeros(B, H, F, 64, device=DEV),
+                        z_in=torch.zeros(B, H, F, device=DEV))
     pk = lambda t: t.permute(1, 0, 2, 3).reshape(H, B * N, t.shape[-1]).contiguous().to(DEV)
     cu = torch.arange(0, B * N + 1, N, dtype=torch.int32, device=DEV)
     r = la.la_forward_varlen(pk(q), pk(k), pk(v), cu, N, TAYLOR2, state=True, den=True)
