@@ -526,21 +526,35 @@ la_status backward_tc(const void *q, const void *k, const void *v, const void *d
     p.inv_c2 = (float)(1.0 / (sqrt(2.0) * sqrt(d)));
     p.inv_c3 = (float)(1.0 / sqrt(d));
     p.k2 = (float)(1.0 / (2.0 * d));
-    if (set_smem<bwd_sstate_kernel<Cfg, GATED>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
-    if (p.P > 1) {
-        bwd_sstate_kernel<Cfg, GATED><<<BH * p.P, 128, Cfg::SMEM_ALLOC, stream>>>(tk, tv, p);
-        if (launch_status() != LA_OK) return LA_ERR_CUDA;
-    }
+    // the S and R increment passes: elu on the three-stage kernels, Taylor on
+    // the two-stage ones (its phi tile is built from the raw tile in place)
+    auto state_pass = [&](bool s_pass) -> la_status {
+        if constexpr (Cfg::TAYLOR) {
+            if (s_pass) {
+                if (set_smem<bwd_sstate_kernel<Cfg, GATED>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
+                bwd_sstate_kernel<Cfg, GATED><<<BH * p.P, 128, Cfg::SMEM_ALLOC, stream>>>(tk, tv, p);
+            } else {
+                if (set_smem<bwd_rstate_kernel<Cfg, GATED>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
+                bwd_rstate_kernel<Cfg, GATED><<<BH * p.P, 128, Cfg::SMEM_ALLOC, stream>>>(tq, tdo, p);
+            }
+        } else {
+            if (s_pass) {
+                if (set_smem<bwd_sstate3_kernel<Cfg, GATED>>(Cfg::SP_SMEM) != LA_OK) return LA_ERR_CUDA;
+                bwd_sstate3_kernel<Cfg, GATED><<<BH * p.P, 256, Cfg::SP_SMEM, stream>>>(tk, tv, p);
+            } else {
+                if (set_smem<bwd_rstate3_kernel<Cfg, GATED>>(Cfg::SP_SMEM) != LA_OK) return LA_ERR_CUDA;
+                bwd_rstate3_kernel<Cfg, GATED><<<BH * p.P, 256, Cfg::SP_SMEM, stream>>>(tq, tdo, p);
+            }
+        }
+        return launch_status();
+    };
+    if (p.P > 1 && state_pass(true) != LA_OK) return LA_ERR_CUDA;
     if (set_smem<bwd_dq_kernel<Cfg, GATED>>(Cfg::SMEM_ALLOC) != LA_OK ||
-        set_smem<bwd_dkdv_kernel<Cfg, GATED>>(Cfg::SMEM_ALLOC) != LA_OK ||
-        set_smem<bwd_rstate_kernel<Cfg, GATED>>(Cfg::SMEM_ALLOC) != LA_OK)
+        set_smem<bwd_dkdv_kernel<Cfg, GATED>>(Cfg::SMEM_ALLOC) != LA_OK)
         return LA_ERR_CUDA;
     bwd_dq_kernel<Cfg, GATED><<<BH * p.P, 256, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, p);
     if (launch_status() != LA_OK) return LA_ERR_CUDA;
-    if (p.P > 1) {
-        bwd_rstate_kernel<Cfg, GATED><<<BH * p.P, 128, Cfg::SMEM_ALLOC, stream>>>(tq, tdo, p);
-        if (launch_status() != LA_OK) return LA_ERR_CUDA;
-    }
+    if (p.P > 1 && state_pass(false) != LA_OK) return LA_ERR_CUDA;
     bwd_dkdv_kernel<Cfg, GATED><<<BH * p.P, 256, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, p);
     if (!GATED) return launch_status();
     if (launch_status() != LA_OK) return LA_ERR_CUDA;
@@ -1116,10 +1130,13 @@ int la_kernel_plan(int op, int B, int H, int N, int dqk, int dv, int fmap, int d
     if (p == Path::BwdTc) {
         int P, cps, nc;
         tc_segments(B, H, N, &P, &cps, &nc);
-        const bool g = op == 5;
-        const char *nm = P > 1 ? (g ? "bwd_sstate_kernel,bwd_dq_kernel,bwd_rstate_kernel,bwd_dkdv_kernel,bwd_dg_kernel"
-                                    : "bwd_sstate_kernel,bwd_dq_kernel,bwd_rstate_kernel,bwd_dkdv_kernel")
-                               : (g ? "bwd_dq_kernel,bwd_dkdv_kernel,bwd_dg_kernel" : "bwd_dq_kernel,bwd_dkdv_kernel");
+        const bool g = op == 5, tay = bwd_tc_kind(dqk, dv, fmap, dtype) == 3;
+        const char *nm =
+            P == 1 ? (g ? "bwd_dq_kernel,bwd_dkdv_kernel,bwd_dg_kernel" : "bwd_dq_kernel,bwd_dkdv_kernel")
+            : tay  ? (g ? "bwd_sstate_kernel,bwd_dq_kernel,bwd_rstate_kernel,bwd_dkdv_kernel,bwd_dg_kernel"
+                        : "bwd_sstate_kernel,bwd_dq_kernel,bwd_rstate_kernel,bwd_dkdv_kernel")
+                   : (g ? "bwd_sstate3_kernel,bwd_dq_kernel,bwd_rstate3_kernel,bwd_dkdv_kernel,bwd_dg_kernel"
+                        : "bwd_sstate3_kernel,bwd_dq_kernel,bwd_rstate3_kernel,bwd_dkdv_kernel");
         if (buf && buflen) {
             strncpy(buf, nm, buflen - 1);
             buf[buflen - 1] = 0;

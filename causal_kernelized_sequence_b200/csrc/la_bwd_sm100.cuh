@@ -128,6 +128,15 @@ struct BwdCfg {
     static_assert(SL_TILE >= S_TILE && SL_TILE >= VG_TILE && OFF_S + S_TILE >= OFF_G + VG_TILE,
                   "the R snapshot fits the S region and the G' remainder the SL region");
     static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory");
+    // elu state passes (bwd_sstate3_kernel, bwd_rstate3_kernel): three stages of
+    // [K or Q tile | V_aug or G'_aug], then barriers and the gate prefix sums
+    static constexpr int SP_A = C * D * 2;
+    static constexpr int SP_STAGE = SP_A + VG_TILE;
+    static constexpr int SP_BAR = 3 * SP_STAGE;
+    static constexpr int SP_GATE = SP_BAR + 128;
+    static constexpr int SP_SMEM = SP_GATE + (C + 8) * 4 + 1024;
+    static_assert(TAYLOR || (SP_A % 1024 == 0 && SP_STAGE % 1024 == 0 && SP_SMEM <= 227 * 1024),
+                  "state-pass stages");
 };
 
 using BwdCfg128 = BwdCfg<128, 128, false>;
@@ -145,8 +154,8 @@ struct BwdParams {
     float inv_c1, inv_c2, inv_c3, k2;
     // gated form (the GATED kernels only): log forget gate g_t per token
     // [BH, N]; each segment's summed gate [BH, P] (written by the S pass);
-    // c_j = phi(k_j) . dphi(k_j) per token [BH, N] (written by the reverse
-    // pass) and dL/dg [BH, N] (its reverse prefix sum, negated)
+    // per token [BH, N]: r_i's part over earlier chunks (forward-order pass),
+    // then c_j - r_j (reverse pass); and dL/dg [BH, N], its reverse prefix sum, negated
     const float *logdecay;
     float *ws_log, *cvec, *dg;
 };
@@ -824,16 +833,37 @@ __device__ __forceinline__ void mask_pack_half_hilo_gate(uint32_t src, uint32_t 
 
 __device__ __forceinline__ float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
 
+// Column sums over a warp's 32 rows of a 32-column block held one row per
+// lane (v[c] = row lane's column c; v is overwritten): lane l returns the sum
+// of column l.  A reduce-scatter in five exchange steps (31 shuffles).
+__device__ __forceinline__ float warp_colsum32(float *v)
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int w = 16; w >= 1; w >>= 1) {
+        const bool up = (lane & w) != 0;
+#pragma unroll
+        for (int e = 0; e < w; ++e) {
+            const float send = up ? v[e] : v[e + w];
+            const float keep = up ? v[e + w] : v[e];
+            v[e] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+        }
+    }
+    return v[0];
+}
+
 // Reverse pass, gated: P^T and dP^T of this thread's 64 columns from j0 in one
 // step (row j is a key, column i a query; weight exp(L_i - L_j); with TAY the
-// raw scores s become 1 + s k1 + s^2 k2 first), and the row's part of
-// c_j = sum_i dL/dw_ij w_ij from the fp32 scores and dA^T (not from the
-// rounded operands of the later MMAs).  P^T overwrites the scores' columns,
-// so the block meets at a barrier between loading and storing (every thread
-// must call this).
-template <bool TAY, bool F16R, typename Keep>
+// raw scores s become 1 + s k1 + s^2 k2 first).  Also the pair terms
+// M_ij = dL/dw_ij w_ij of the chunk from the fp32 scores and dA^T: returns the
+// row's part of c_j = sum_i M_ij, and writes the warp's part of each
+// column's r_i = sum_j M_ij to rsum[i] (the two come from the same products,
+// so the chunk's pairs cancel exactly in the suffix sums of r - c).  P^T
+// overwrites the scores' columns, so the block meets at a barrier between
+// loading and storing (every thread must call this).
+template <bool TAY, typename Keep>
 __device__ __forceinline__ float mask_pack_both_gate(uint32_t tA, uint32_t tX, uint32_t tPL, int j0, float k1, float k2,
-                                                     float rowL, const float *colL, Keep keep)
+                                                     float rowL, const float *colL, float *rsum, Keep keep)
 {
     float w[64];
     tmem_ld32(tA + j0, w);
@@ -866,55 +896,57 @@ __device__ __forceinline__ float mask_pack_both_gate(uint32_t tA, uint32_t tX, u
             const int i0 = j0 + 32 * h2 + e;
             const float x0 = keep(i0) ? d[e] * __expf(colL[i0] - rowL) : 0.f;
             const float x1 = keep(i0 + 1) ? d[e + 1] * __expf(colL[i0 + 1] - rowL) : 0.f;
-            // the weights rounded as the forward-order pass rounded them for y
-            // (F16R: to fp16; 0 where masked)
-            c = fmaf(d[e], F16R ? __half2float(__float2half_rn(w[32 * h2 + e])) : bf16_round(w[32 * h2 + e]), c);
-            c = fmaf(d[e + 1], F16R ? __half2float(__float2half_rn(w[32 * h2 + e + 1])) : bf16_round(w[32 * h2 + e + 1]),
-                     c);
             hi[e / 2] = pack_bf16(x0, x1);
             lo[e / 2] = pack_bf16(x0 - __bfloat162float(__float2bfloat16_rn(x0)),
                                   x1 - __bfloat162float(__float2bfloat16_rn(x1)));
         }
         tmem_st16(tA + 64 + (j0 + 32 * h2) / 2, reinterpret_cast<const float *>(hi));
         tmem_st16(tPL + (j0 + 32 * h2) / 2, reinterpret_cast<const float *>(lo));
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            d[e] *= w[32 * h2 + e];   // M_ij (0 where masked)
+            c += d[e];
+        }
+        rsum[j0 + 32 * h2 + (threadIdx.x & 31)] = warp_colsum32(d);
     }
     tmem_st_wait();
     return c;
 }
 
-// phi(k_j) . X_j over features [80 HALF, 80 HALF + 80) of the Taylor map, X
-// read from TMEM columns tcol + f, phi from the raw row x.
-template <int F0, int... E>
+// phi(x) . (X + dr) over features [80 HALF, 80 HALF + 80) of the Taylor map,
+// X read from TMEM columns tcol + f, phi from the raw row x; dr_f (the bf16
+// remainder of R's normaliser column) only with DR.
+template <bool DR, int F0, int... E>
 __device__ __forceinline__ float tay_dot_seq(const float *g, const float *x, const float *dr, const BwdParams &p,
                                              std::integer_sequence<int, E...>)
 {
     float acc = 0.f;
-    ((acc = fmaf(g[E] + dr[F0 + E], tay_feat<F0 + E>(x, p), acc)), ...);
+    ((acc = fmaf(DR ? g[E] + dr[F0 + E] : g[E], tay_feat<F0 + E>(x, p), acc)), ...);
     return acc;
 }
-template <int F0>
+template <bool DR, int F0>
 __device__ __forceinline__ float tay_dot16(uint32_t tcol, const float *x, const float *dr, const BwdParams &p)
 {
     float g[16];
     tmem_ld16(tcol + F0, g);
     tmem_ld_wait();
-    return tay_dot_seq<F0>(g, x, dr, p, std::make_integer_sequence<int, 16>{});
+    return tay_dot_seq<DR, F0>(g, x, dr, p, std::make_integer_sequence<int, 16>{});
 }
-template <int FB, int... G>
+template <bool DR, int FB, int... G>
 __device__ __forceinline__ float tay_dot_groups(uint32_t tcol, const float *x, const float *dr, const BwdParams &p,
                                                 std::integer_sequence<int, G...>)
 {
-    return (tay_dot16<FB + 16 * G>(tcol, x, dr, p) + ...);
+    return (tay_dot16<DR, FB + 16 * G>(tcol, x, dr, p) + ...);
 }
-// ... plus dr_f per feature (the bf16 remainder of R's normaliser column).
-template <int HALF>
+template <bool DR, int HALF>
 __device__ __forceinline__ float tay_dot_half(uint32_t tcol, const float *x, const float *dr, const BwdParams &p)
 {
-    return tay_dot_groups<80 * HALF>(tcol, x, dr, p, std::make_integer_sequence<int, 5>{});
+    return tay_dot_groups<DR, 80 * HALF>(tcol, x, dr, p, std::make_integer_sequence<int, 5>{});
 }
 
-// phi(k_j) . (X_j + dr) over feature columns [c_lo, c_hi) of an elu phi tile
-// (bf16, row j), X from TMEM columns tcol + f.
+// phi_j . (X_j + dr) over feature columns [c_lo, c_hi) of an elu phi tile
+// (row j; fp16 or bf16 as F16), X from TMEM columns tcol + f; dr only with DR.
+template <bool F16, bool DR>
 __device__ __forceinline__ float elu_dot_cols(uint32_t tcol, uint32_t phi_tile, int j, int c_lo, int c_hi,
                                               const float *dr)
 {
@@ -924,10 +956,15 @@ __device__ __forceinline__ float elu_dot_cols(uint32_t tcol, uint32_t phi_tile, 
         float g[16], ph[16];
         tmem_ld16(tcol + c0, g);
         tmem_ld_wait();
-        unpack8(lds128(phi_tile + sw128_off(j, c0)), ph);
-        unpack8(lds128(phi_tile + sw128_off(j, c0 + 8)), ph + 8);
+        if constexpr (F16) {
+            unpack8_f16(lds128(phi_tile + sw128_off(j, c0)), ph);
+            unpack8_f16(lds128(phi_tile + sw128_off(j, c0 + 8)), ph + 8);
+        } else {
+            unpack8(lds128(phi_tile + sw128_off(j, c0)), ph);
+            unpack8(lds128(phi_tile + sw128_off(j, c0 + 8)), ph + 8);
+        }
 #pragma unroll
-        for (int e = 0; e < 16; ++e) acc = fmaf(g[e] + dr[c0 + e], ph[e], acc);
+        for (int e = 0; e < 16; ++e) acc = fmaf(DR ? g[e] + dr[c0 + e] : g[e], ph[e], acc);
     }
     return acc;
 }
@@ -1124,8 +1161,8 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     const uint32_t off = (kk >> 2) * (C * 128) + (kk & 3) * 32;
                     mma_bf16(tX, smem_desc(aQ + off, 16, 1024, kSw128), smem_desc(aS + kk * 512, Cfg::S_BLK, 256, kSw32),
                              id_o, kk > 0);
-                    // and its remainder: y_i, hence dden_i, must agree to ~16 bits with
-                    // the weights the reverse pass sums into dL/dg (see bwd_dg_kernel)
+                    // and its remainder: y_i, hence dden_i, to ~16 bits (dden_i enters
+                    // every pair term of row i in dL/dg)
                     mma_bf16(tX, smem_desc(aQ + off, 16, 1024, kSw128), smem_desc(aSL + kk * 512, Cfg::S_BLK, 256, kSw32),
                              id_o, true);
                 }
@@ -1276,8 +1313,21 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             if (!mbar_wait(mma_bar, mph)) *abort_flag = 1;
             mph ^= 1u;
             tc_fence_after();
+            // r_i's part over the earlier chunks' keys: sum over j < t0 of
+            // dL/dw_ij w_ij = phi(q_i) . (their term of dphi(q_i)), to cvec
+            float dot;
+            if constexpr (TAY) {
+                float xq[16];
+                raw_row16(aRQ, i, xq);
+                dot = hh == 0 ? tay_dot_half<false, 0>(tX + lane, xq, nullptr, p)
+                              : tay_dot_half<false, 1>(tX + lane, xq, nullptr, p);
+            } else {
+                dot = elu_dot_cols<F16, false>(tX + lane, aQ, i, hh * (F / 2), (hh + 1) * (F / 2), nullptr);
+            }
+            red[hh * C + i] = dot;
             tmem_scale(tX + lane, hh * (F / 2), (hh + 1) * (F / 2), __expf(Lrow));
             full_sync();
+            if (hh == 0 && valid) p.cvec[(size_t)bh * N + t0 + i] = (red[i] + red[C + i]) * __expf(Lrow) / den_row;
         }
 
         // dphi(Q) = dP phi(K) + G'' S_aug^T ;  then S_aug += phi(K)^T V_aug
@@ -1541,6 +1591,287 @@ bwd_sstate_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             }
         }
     }
+    full_sync();
+    if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+// ---------------------------------------------------------------------------
+// The elu state passes on a three-stage pipeline (256 threads).  Chunk k of a
+// segment uses stage k % 3; the two threads of row r (r and r + 128) convert
+// complementary parts of the row; once a chunk is converted one thread issues
+// its MMA into the TMEM accumulator and the block goes on to the next chunk,
+// whose conversion runs under that MMA.  Chunk k + 2's loads go out once the
+// MMA of chunk k - 1 has released its stage.  Gated: the accumulator decays by
+// the chunk's whole gate between two MMAs, so every thread waits for the
+// previous chunk's MMA after converting and before decaying.
+namespace bwd_detail {
+
+// Columns [c_lo, c_hi) (multiples of 8) of row r of a bf16 SW32 tile of 128
+// rows, rewritten as fp16 (times s with SCALE; without, the exact conversion).
+template <bool SCALE>
+__device__ __forceinline__ void row_to_f16(uint32_t tile, int r, int c_lo, int c_hi, float s)
+{
+#pragma unroll 1
+    for (int c0 = c_lo; c0 < c_hi; c0 += 8) {
+        const uint32_t a = tile + sw32_off(r, c0, 128);
+        const uint4 u = lds128(a);
+        if constexpr (SCALE) {
+            float f[8];
+            unpack8(u, f);
+            sts128(a, make_uint4(pack_f16(f[0] * s, f[1] * s), pack_f16(f[2] * s, f[3] * s), pack_f16(f[4] * s, f[5] * s),
+                                 pack_f16(f[6] * s, f[7] * s)));
+        } else {
+            sts128(a, make_uint4(bf16x2_to_f16x2(u.x), bf16x2_to_f16x2(u.y), bf16x2_to_f16x2(u.z), bf16x2_to_f16x2(u.w)));
+        }
+    }
+}
+
+// Columns [c_lo, c_hi) of row r of a bf16 SW32 tile of 128 rows times s.
+__device__ __forceinline__ void row_scale_bf16(uint32_t tile, int r, int c_lo, int c_hi, float s)
+{
+#pragma unroll 1
+    for (int c0 = c_lo; c0 < c_hi; c0 += 8) {
+        const uint32_t a = tile + sw32_off(r, c0, 128);
+        float f[8];
+        unpack8(lds128(a), f);
+        sts128(a, make_uint4(pack_bf16(f[0] * s, f[1] * s), pack_bf16(f[2] * s, f[3] * s), pack_bf16(f[4] * s, f[5] * s),
+                             pack_bf16(f[6] * s, f[7] * s)));
+    }
+}
+
+// The accumulated increment (one state tile of NA columns in TMEM) to
+// dst [F][NA]; this thread takes columns [c_lo, c_hi) of its lane's row.
+template <class Cfg>
+__device__ __forceinline__ void store_state_tile(float *dst, uint32_t t_lane, int wq, int l, int c_lo, int c_hi)
+{
+    if (!state_quadrant<Cfg>(0, wq)) return;
+    const int f = state_row<Cfg>(0, wq, l);
+    float *d = dst + (size_t)(f < 0 ? 0 : f) * Cfg::NA;
+#pragma unroll 1
+    for (int c0 = c_lo; c0 < c_hi; c0 += 16) {
+        float v[16];
+        tmem_ld16(t_lane + c0, v);
+        tmem_ld_wait();
+        if (f >= 0)
+#pragma unroll
+            for (int e = 0; e < 16; ++e) d[c0 + e] = v[e];
+    }
+}
+
+}  // namespace bwd_detail
+
+// S increments (elu): for each segment but the last, the sum over its tokens
+// of phi(k_j) [v_j | 1]^T (gated: key j weighted by exp(L_last - L_j) within
+// its chunk, the sum decayed by each later chunk's gate), fp16 operands like
+// the forward-order pass that consumes them.
+template <class Cfg, bool GATED = false>
+__global__ void __launch_bounds__(256, 1)
+bwd_sstate3_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                   const BwdParams p)
+{
+    using namespace bwd_detail;
+    static_assert(!Cfg::TAYLOR, "elu shapes");
+    constexpr int C = Cfg::C, D = Cfg::D, DV = Cfg::DV, NA = Cfg::NA;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *tma_b = reinterpret_cast<uint64_t *>(smem + Cfg::SP_BAR), *mma_b = tma_b + 3;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tma_b + 6);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tma_b + 7);
+    float *gL = reinterpret_cast<float *>(smem + Cfg::SP_GATE);
+    const int tid = threadIdx.x, warp = tid >> 5, wq = warp & 3, hh = warp >> 2, l = tid & 31;
+    const int row = wq * 32 + l;
+    const int bh = blockIdx.x / p.P, seg = blockIdx.x % p.P;
+    if (seg == p.P - 1) return;   // the last segment's increment is never read
+    const int c_begin = seg * p.cps, c_end = min(p.nchunks, c_begin + p.cps), n = c_end - c_begin;
+    const int N = p.N;
+    auto sA = [&](int st) { return smem + st * Cfg::SP_STAGE; };
+    auto sB = [&](int st) { return smem + st * Cfg::SP_STAGE + Cfg::SP_A; };
+    if (tid == 0) {
+        for (int s2 = 0; s2 < 3; ++s2) {
+            mbar_init(&tma_b[s2], 1);
+            mbar_init(&mma_b[s2], 1);
+        }
+        *abort_flag = 0;
+        mbar_init_fence();
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, 256);
+    if (!GATED && hh == 0)
+        for (int s2 = 0; s2 < 3; ++s2) write_first_f16(sB(s2) + (DV / 16) * Cfg::BLK, row, 1.f);
+    full_sync();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane = (uint32_t)(wq * 32) << 16;
+    const int na_lo = hh ? Cfg::NA_SPLIT : 0, na_hi = hh ? NA : Cfg::NA_SPLIT;
+    auto issue = [&](int k) {
+        const int st = k % 3, t0 = (c_begin + k) * C;
+        mbar_arrive_expect_tx(&tma_b[st], C * D * 2 + C * DV * 2);
+        for (int x = 0; x < D; x += 64) tma_load_3d(sA(st) + (x / 64) * C * 128, &tm_k, &tma_b[st], x, t0, bh);
+        for (int x = 0; x < DV; x += 16) tma_load_3d(sB(st) + (x / 16) * Cfg::BLK, &tm_v, &tma_b[st], x, t0, bh);
+    };
+    int issued = 0, waited = 0, mmas = 0;   // thread 0: chunks whose loads went out / were waited for / MMAs went out
+    if (tid == 0)
+        for (; issued < n && issued < 3; ++issued) issue(issued);
+    float seg_log = 0.f;
+    // every thread runs the same iterations and leaves only at the check after
+    // the barrier, so a flag thread 0 sets after that check is seen by all at
+    // the next one
+    for (int k = 0; k < n; ++k) {
+        const int st = k % 3, t0 = (c_begin + k) * C;
+        const uint32_t aK = smem_addr(sA(st)), aV = smem_addr(sB(st));
+        float Lrow = 0.f, Llast = 0.f;
+        if constexpr (GATED) {
+            Lrow = gate_prefix(p.logdecay + (size_t)bh * N + t0, row, min(C, N - t0), wq, l, hh == 0, gL, Llast);
+            seg_log += Llast;
+        }
+        if (!mbar_wait(&tma_b[st], (uint32_t)(k / 3) & 1u)) *abort_flag = 1;
+        if (tid == 0) waited = k + 1;
+        const bool zero = t0 + row >= N;
+        const float w = GATED ? __expf(Llast - Lrow) : 1.f;
+        // phi(K) and V_aug in fp16: d = 128, the row's two threads take one
+        // half of each; d = 64, one takes phi(K) and the other V_aug
+        if (D == 128 || hh == 0) phi_block_f16(aK, row, zero, D == 128 ? hh : 0);
+        if (D == 128 || hh == 1) {
+            const int c_lo = D == 128 ? 64 * hh : 0, c_hi = D == 128 ? 64 * hh + 64 : DV;
+            row_to_f16<GATED>(aV, row, c_lo, c_hi, w);
+            if (GATED && c_lo == 0) write_first_f16(sB(st) + (DV / 16) * Cfg::BLK, row, w);
+        }
+        if constexpr (GATED) {
+            if (k > 0) {
+                if (!mbar_wait(&mma_b[(k - 1) % 3], (uint32_t)((k - 1) / 3) & 1u)) *abort_flag = 1;
+                tc_fence_after();
+                decay_state_tiles<Cfg>(tmem, lane, wq, na_lo, na_hi, __expf(Llast));
+            }
+        }
+        full_sync();
+        if (*abort_flag) break;
+        if (tid == 0) {
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)
+                mma_bf16(tmem, smem_desc(aK + kk * 2048, C * 128, 1024, kSw128), smem_desc(aV + kk * 512, Cfg::BLK, 256, kSw32),
+                         idesc_f16(Cfg::tile_m(0), NA, 1, 1), k > 0 || kk > 0);
+            mma_commit(&mma_b[st]);
+            mmas = k + 1;
+            // the stage of chunk k - 1 takes chunk k + 2 once its MMA is done
+            if (k >= 1 && issued < n) {
+                if (mbar_wait(&mma_b[(k - 1) % 3], (uint32_t)((k - 1) / 3) & 1u)) issue(issued++);
+                else *abort_flag = 1;
+            }
+        }
+    }
+    // thread 0: let its own copies land and its MMAs finish (bounded), then all read
+    if (tid == 0) {
+        for (int c = waited; c < issued; ++c) mbar_wait(&tma_b[c % 3], (uint32_t)(c / 3) & 1u, 100000000ull);
+        if (mmas > 0 && !mbar_wait(&mma_b[(mmas - 1) % 3], (uint32_t)((mmas - 1) / 3) & 1u)) *abort_flag = 1;
+        if (mmas < n) *abort_flag = 1;
+    }
+    full_sync();
+    if (!*abort_flag) {
+        if (GATED && tid == 0) p.ws_log[(size_t)bh * p.P + seg] = seg_log;
+        store_state_tile<Cfg>(p.ws_s + (size_t)(bh * p.P + seg) * Cfg::F * NA, tmem + lane, wq, l, na_lo, na_hi);
+    }
+    full_sync();
+    if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+// R increments (elu): for each segment but the first, the sum over its tokens
+// of phi(q_i) G'_i^T (gated: chunks taken from the segment's end, query i
+// weighted by exp(L_i), the sum decayed by each earlier chunk's gate), on the
+// pipeline of bwd_sstate3_kernel with stages of [Q | G'_aug].
+template <class Cfg, bool GATED = false>
+__global__ void __launch_bounds__(256, 1)
+bwd_rstate3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                   const BwdParams p)
+{
+    using namespace bwd_detail;
+    static_assert(!Cfg::TAYLOR, "elu shapes");
+    constexpr int C = Cfg::C, D = Cfg::D, DV = Cfg::DV, NA = Cfg::NA;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *tma_b = reinterpret_cast<uint64_t *>(smem + Cfg::SP_BAR), *mma_b = tma_b + 3;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tma_b + 6);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tma_b + 7);
+    float *gL = reinterpret_cast<float *>(smem + Cfg::SP_GATE);
+    const int tid = threadIdx.x, warp = tid >> 5, wq = warp & 3, hh = warp >> 2, l = tid & 31;
+    const int row = wq * 32 + l;
+    const int bh = blockIdx.x / p.P, seg = blockIdx.x % p.P;
+    if (seg == 0) return;   // the first segment's increment is never read
+    const int c_begin = seg * p.cps, c_end = min(p.nchunks, c_begin + p.cps), n = c_end - c_begin;
+    const int N = p.N;
+    auto sA = [&](int st) { return smem + st * Cfg::SP_STAGE; };
+    auto sB = [&](int st) { return smem + st * Cfg::SP_STAGE + Cfg::SP_A; };
+    auto chunk_of = [&](int k) { return GATED ? c_end - 1 - k : c_begin + k; };
+    if (tid == 0) {
+        for (int s2 = 0; s2 < 3; ++s2) {
+            mbar_init(&tma_b[s2], 1);
+            mbar_init(&mma_b[s2], 1);
+        }
+        *abort_flag = 0;
+        mbar_init_fence();
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, 256);
+    full_sync();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane = (uint32_t)(wq * 32) << 16;
+    const int na_lo = hh ? Cfg::NA_SPLIT : 0, na_hi = hh ? NA : Cfg::NA_SPLIT;
+    auto issue = [&](int k) {
+        const int st = k % 3, t0 = chunk_of(k) * C;
+        mbar_arrive_expect_tx(&tma_b[st], C * D * 2 + C * DV * 2);
+        for (int x = 0; x < D; x += 64) tma_load_3d(sA(st) + (x / 64) * C * 128, &tm_q, &tma_b[st], x, t0, bh);
+        for (int x = 0; x < DV; x += 16) tma_load_3d(sB(st) + (x / 16) * Cfg::BLK, &tm_do, &tma_b[st], x, t0, bh);
+    };
+    int issued = 0, waited = 0, mmas = 0;
+    if (tid == 0)
+        for (; issued < n && issued < 3; ++issued) issue(issued);
+    for (int k = 0; k < n; ++k) {
+        const int st = k % 3, t0 = chunk_of(k) * C;
+        const bool valid = t0 + row < N;
+        const uint32_t aQ = smem_addr(sA(st)), aG = smem_addr(sB(st));
+        float Lrow = 0.f, Llast = 0.f;
+        if constexpr (GATED)
+            Lrow = gate_prefix(p.logdecay + (size_t)bh * N + t0, row, min(C, N - t0), wq, l, hh == 0, gL, Llast);
+        // den_i, dden_i of this row (they do not depend on the loads)
+        const float den = valid ? p.dd[((size_t)bh * N + t0 + row) * 2] : 1.f;
+        const float dden = valid ? p.dd[((size_t)bh * N + t0 + row) * 2 + 1] : 0.f;
+        if (!mbar_wait(&tma_b[st], (uint32_t)(k / 3) & 1u)) *abort_flag = 1;
+        if (tid == 0) waited = k + 1;
+        // phi(Q) in place, G' = [dO / den | dden] (gated: query row i times exp(L_i))
+        const float e = GATED ? __expf(Lrow) : 1.f;
+        if (D == 128 || hh == 0) phi_block_inplace(aQ, row, false, D == 128 ? hh : 0);
+        if (D == 128 || hh == 1) {
+            const int c_lo = D == 128 ? 64 * hh : 0, c_hi = D == 128 ? 64 * hh + 64 : DV;
+            row_scale_bf16(aG, row, c_lo, c_hi, valid ? e / den : 0.f);
+            if (c_lo == 0) write_dden(sB(st) + (DV / 16) * Cfg::BLK, row, valid ? e * dden : 0.f);
+        }
+        if constexpr (GATED) {
+            if (k > 0) {
+                if (!mbar_wait(&mma_b[(k - 1) % 3], (uint32_t)((k - 1) / 3) & 1u)) *abort_flag = 1;
+                tc_fence_after();
+                decay_state_tiles<Cfg>(tmem, lane, wq, na_lo, na_hi, __expf(Llast));
+            }
+        }
+        full_sync();
+        if (*abort_flag) break;
+        if (tid == 0) {
+            // R_aug += phi(Q)^T G'   (M = the D features, N = NA, K = tokens)
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)
+                mma_bf16(tmem, smem_desc(aQ + kk * 2048, C * 128, 1024, kSw128), smem_desc(aG + kk * 512, Cfg::BLK, 256, kSw32),
+                         idesc_bf16(Cfg::tile_m(0), NA, 1, 1), k > 0 || kk > 0);
+            mma_commit(&mma_b[st]);
+            mmas = k + 1;
+            if (k >= 1 && issued < n) {
+                if (mbar_wait(&mma_b[(k - 1) % 3], (uint32_t)((k - 1) / 3) & 1u)) issue(issued++);
+                else *abort_flag = 1;
+            }
+        }
+    }
+    if (tid == 0) {
+        for (int c = waited; c < issued; ++c) mbar_wait(&tma_b[c % 3], (uint32_t)(c / 3) & 1u, 100000000ull);
+        if (mmas > 0 && !mbar_wait(&mma_b[(mmas - 1) % 3], (uint32_t)((mmas - 1) / 3) & 1u)) *abort_flag = 1;
+        if (mmas < n) *abort_flag = 1;
+    }
+    full_sync();
+    if (!*abort_flag)
+        store_state_tile<Cfg>(p.ws_r + (size_t)(bh * p.P + seg) * Cfg::F * NA, tmem + lane, wq, l, na_lo, na_hi);
     full_sync();
     if (warp == 0) tmem_dealloc(tmem, 256);
 }
@@ -1885,14 +2216,17 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // row j keeps the queries i >= j
         float c_part = 0.f;   // gated: this thread's part of c_j = sum_i dL/dw_ij w_ij
         if constexpr (GATED) {
-            c_part = mask_pack_both_gate<TAY, Cfg::F16>(tA + lane, tX + lane, tPL + lane, 64 * hh, p.inv_c3, p.k2, Lrow, gL,
-                                              [&](int i) { return i >= j; });
+            c_part = mask_pack_both_gate<TAY>(tA + lane, tX + lane, tPL + lane, 64 * hh, p.inv_c3, p.k2, Lrow, gL,
+                                              red + wq * C, [&](int i) { return i >= j; });
         } else {
             mask_pack_half_g<false, TAY>(tA + lane, tA + lane, 64 * hh, true, p.inv_c3, p.k2,
                                          [&](int i) { return i >= j; });
             mask_pack_half_hilo(tX + lane, tA + lane + 64, tPL + lane, 64 * hh, [&](int i) { return i >= j; });
         }
         full_sync();
+        // gated: r_j's part over this chunk's keys (token j as a query), from the
+        // four quadrants' column sums
+        const float r_chunk = GATED ? red[j] + red[C + j] + red[2 * C + j] + red[3 * C + j] : 0.f;
         if constexpr (GATED) {
             // the later chunks' term of dV first, scaled per key row by exp(L_last - L_j)
             if (tid == 0) {
@@ -1971,9 +2305,9 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if constexpr (TAY) {
                 float xk[16];
                 raw_row16(aRK, j, xk);
-                dot = hh == 0 ? tay_dot_half<0>(tX + lane, xk, dr, p) : tay_dot_half<1>(tX + lane, xk, dr, p);
+                dot = hh == 0 ? tay_dot_half<true, 0>(tX + lane, xk, dr, p) : tay_dot_half<true, 1>(tX + lane, xk, dr, p);
             } else {
-                dot = elu_dot_cols(tX + lane, aK, j, hh * (F / 2), (hh + 1) * (F / 2), dr);
+                dot = elu_dot_cols<false, true>(tX + lane, aK, j, hh * (F / 2), (hh + 1) * (F / 2), dr);
             }
             c_part = fmaf(w, dot, c_part);
             tmem_scale(tX + lane, hh * (F / 2), (hh + 1) * (F / 2), w);
@@ -2041,10 +2375,15 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
             }
             if constexpr (GATED) {
-                // c_j = phi(k_j) . dphi(k_j), summed over the row's two threads
+                // c_j - r_j: c_j = phi(k_j) . dphi(k_j) summed over the row's two
+                // threads; r_j = the chunk's part above plus the earlier chunks'
+                // part the forward-order pass left in cvec
                 red[4 * C + hh * C + j] = c_part;
                 __syncthreads();
-                if (hh == 0 && valid) p.cvec[(size_t)bh * N + t0 + j] = red[4 * C + j] + red[5 * C + j];
+                if (hh == 0 && valid) {
+                    float *cj = p.cvec + (size_t)bh * N + t0 + j;
+                    *cj = red[4 * C + j] + red[5 * C + j] - r_chunk - *cj;
+                }
             }
             if (chunk > c_begin) {
 #pragma unroll
@@ -2069,10 +2408,13 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
 
 // ---------------------------------------------------------------------------
-// Gated form: dL/dg_l = - sum_{m >= l} c_m per head, c_m = phi(k_m) . dphi(k_m)
-// from the reverse pass.  (g_l scales every weight w_ij with j < l <= i; the
-// weights of a query sum to a constant in y_i's gradient, sum_j dL/dw_ij w_ij
-// = 0, which turns the sum over pairs into this suffix sum of per-key terms.)
+// Gated form: dL/dg_l = - sum_{m >= l} x_m per head, x_m = c_m - r_m from the
+// two passes.  g_l scales every weight w_ij with j < l <= i, so dL/dg_l is the
+// sum of M_ij = dL/dw_ij w_ij over those pairs; with r_m = sum_j M_mj (a row)
+// and c_m = sum_i M_im (a column), sum_{m >= l} (r_m - c_m) is exactly that sum
+// for any M.  (In exact arithmetic r_m = 0, the weights of a query entering y_m
+// as a ratio; the kernels' own r_m is kept because their c_m and r_m then come
+// from the same rounded pair terms for the pairs inside a chunk.)
 // One block per head walks the sequence from its end in tiles of 1024.
 __global__ void __launch_bounds__(1024, 1) bwd_dg_kernel(const float *c, float *dg, int N)
 {

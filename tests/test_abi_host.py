@@ -142,7 +142,10 @@ def test_kernel_plan_and_workspace(lib):
         32 * 16384 * 2 * 4 + 2 * 32 * 4 * 128 * 144 * 4
     # elu d=64 and both Taylor maps (d'=16, dv=64) take the tensor-core backward too:
     # B=1 H=2 N=300 is 3 chunks, one segment each
+    # (the elu increment passes run on the three-stage kernels, Taylor's on the two-stage ones)
     assert la.la_kernel_plan(1, 1, 2, 300, 64, 64, 0, 1) == \
+        (4, ["bwd_sstate3_kernel", "bwd_dq_kernel", "bwd_rstate3_kernel", "bwd_dkdv_kernel"])
+    assert la.la_kernel_plan(1, 1, 2, 300, 16, 64, 1, 1) == \
         (4, ["bwd_sstate_kernel", "bwd_dq_kernel", "bwd_rstate_kernel", "bwd_dkdv_kernel"])
     for fmap in (1, 2):
         assert la.la_kernel_plan(1, 8, 16, 2048, 16, 64, fmap, 1) == (2, ["bwd_dq_kernel", "bwd_dkdv_kernel"])
@@ -155,7 +158,7 @@ def test_kernel_plan_and_workspace(lib):
     # workspace holds den, dden and c per token, and per segment the S and R
     # increments and the summed gate
     assert la.la_kernel_plan(5, 1, 2, 300, 64, 64, 0, 1) == \
-        (5, ["bwd_sstate_kernel", "bwd_dq_kernel", "bwd_rstate_kernel", "bwd_dkdv_kernel", "bwd_dg_kernel"])
+        (5, ["bwd_sstate3_kernel", "bwd_dq_kernel", "bwd_rstate3_kernel", "bwd_dkdv_kernel", "bwd_dg_kernel"])
     assert la.la_kernel_plan(5, 8, 16, 2048, 16, 64, 1, 1) == (3, ["bwd_dq_kernel", "bwd_dkdv_kernel", "bwd_dg_kernel"])
     bd = la.load_library().la_backward_decay_workspace_bytes
     assert bd(1, 2, 300, 64, 64, 0, 1) == (2 * 300 * 3 + 2 * 3 * (2 * 64 * 80 + 1)) * 4
