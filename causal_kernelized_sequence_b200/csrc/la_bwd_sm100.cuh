@@ -59,10 +59,12 @@
 // l < 16); the elu d = 64 state is one M = 64 tile in the same layout.
 // bwd_dq_kernel and bwd_dkdv_kernel run 256 threads: warps w and w + 4 share
 // the lanes of one 32-row quadrant and split every per-row step by columns,
-// exchanging row reductions through shared memory.  bwd_sstate_kernel and
-// bwd_rstate_kernel run 128 threads, one per row, and load the next chunk
-// while the current one is summed.  Each block takes a chunk's steps in
-// order; every mbarrier wait is bounded.
+// exchanging row reductions through shared memory.  The S and R increment
+// passes run 256 threads on three load stages for the elu shapes
+// (bwd_sstate3_kernel, bwd_rstate3_kernel: a chunk's MMA runs under the next
+// chunk's conversion) and 128 threads, one per row, on two stages for the
+// Taylor map (bwd_sstate_kernel, bwd_rstate_kernel).  Each block takes a
+// chunk's steps in order; every mbarrier wait is bounded.
 #pragma once
 
 #include <type_traits>
@@ -174,27 +176,43 @@ __device__ __forceinline__ void full_sync()
     tc_fence_after();
 }
 
-// elu(x)+1 in place on row `row` of a [128 x 128] bf16 SW128 tile; rows at or
-// beyond `nvalid` are zeroed when `zero_tail`.
-__device__ __forceinline__ void phi_row_inplace(uint32_t tile, int row, bool zero)
+__device__ __forceinline__ uint32_t pack_f16(float a, float b)
 {
-#pragma unroll
-    for (int blk = 0; blk < 2; ++blk) {
-        uint4 raw[8];
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) raw[cc] = lds128(tile + sw128_off(row, blk * 64 + cc * 8));
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-            uint4 r = raw[cc];
-            r = zero ? make_uint4(0u, 0u, 0u, 0u)
-                     : make_uint4(elu1_bf16x2(r.x), elu1_bf16x2(r.y), elu1_bf16x2(r.z), elu1_bf16x2(r.w));
-            sts128(tile + sw128_off(row, blk * 64 + cc * 8), r);
-        }
-    }
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&h);
 }
 
-// elu(x)+1 in place on the 64-column block `blk` of row `row` (one half of
-// phi_row_inplace, for two threads per row).
+// elu(x)+1 of two bf16 values evaluated in fp32 (its exp through __expf,
+// ~2^-21 relative) and rounded to nearest once, as a bf16 pair.  The packed
+// bf16 form (elu1_bf16x2: argument and exp2 each in 8-bit bf16) left the
+// reverse pass's pair terms ~0.17 % low on average against fp64, while the
+// packed fp16 form below showed no such offset; the gated reverse passes sum
+// per-token differences of those terms over the whole sequence for dL/dg,
+// where a one-sided error accumulates, so they take this form.
+__device__ __forceinline__ float elu1_f32(float x) { return x > 0.f ? x + 1.f : __expf(x); }
+
+__device__ __forceinline__ uint32_t elu1_rn_bf16x2(uint32_t x)
+{
+    return pack_bf16(elu1_f32(__uint_as_float(x << 16)), elu1_f32(__uint_as_float(x & 0xFFFF0000u)));
+}
+
+// elu(x)+1 of two bf16 values, as fp16: max(x,0) + 2^(min(x,0) log2 e), the
+// exponent argument rounded once to fp16 and the packed exp2 in fp16 (11
+// significant bits, so phi - 1 keeps ~8 bits for |x| ~ 0.1).
+__device__ __forceinline__ uint32_t elu1_f16x2_from_bf16x2(uint32_t x)
+{
+    const float lo = __uint_as_float(x << 16), hi = __uint_as_float(x & 0xFFFF0000u);
+    const uint32_t arg = pack_f16(fminf(lo, 0.f) * 1.4426950408889634f, fminf(hi, 0.f) * 1.4426950408889634f);
+    const uint32_t pos = pack_f16(fmaxf(lo, 0.f), fmaxf(hi, 0.f));
+    uint32_t ex, r;
+    asm("ex2.approx.f16x2 %0, %1;" : "=r"(ex) : "r"(arg));
+    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(pos), "r"(ex));
+    return r;
+}
+
+// elu(x)+1 in place (bf16) on the 64-column block `blk` of row `row` of a
+// bf16 SW128 tile; zeros when `zero`.  EXACT: the fp32 form rounded once.
+template <bool EXACT>
 __device__ __forceinline__ void phi_block_inplace(uint32_t tile, int row, bool zero, int blk)
 {
     uint4 raw[8];
@@ -204,8 +222,36 @@ __device__ __forceinline__ void phi_block_inplace(uint32_t tile, int row, bool z
     for (int cc = 0; cc < 8; ++cc) {
         uint4 r = raw[cc];
         r = zero ? make_uint4(0u, 0u, 0u, 0u)
-                 : make_uint4(elu1_bf16x2(r.x), elu1_bf16x2(r.y), elu1_bf16x2(r.z), elu1_bf16x2(r.w));
+                 : EXACT ? make_uint4(elu1_rn_bf16x2(r.x), elu1_rn_bf16x2(r.y), elu1_rn_bf16x2(r.z), elu1_rn_bf16x2(r.w))
+                         : make_uint4(elu1_bf16x2(r.x), elu1_bf16x2(r.y), elu1_bf16x2(r.z), elu1_bf16x2(r.w));
         sts128(tile + sw128_off(row, blk * 64 + cc * 8), r);
+    }
+}
+
+// phi(x) s in place (bf16) on the 64-column block `blk` of row `row` of a bf16
+// SW128 tile.  EXACT: phi in fp32 times s, rounded once; otherwise the packed
+// bf16 phi times s (two roundings).
+template <bool EXACT>
+__device__ __forceinline__ void phi_block_scaled(uint32_t tile, int row, float s, int blk)
+{
+    uint4 raw[8];
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) raw[cc] = lds128(tile + sw128_off(row, blk * 64 + cc * 8));
+    const uint32_t s2 = pack_bf16(s, s);
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) {
+        uint32_t w[4] = {raw[cc].x, raw[cc].y, raw[cc].z, raw[cc].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            if constexpr (EXACT) {
+                w[e] = pack_bf16(elu1_f32(__uint_as_float(w[e] << 16)) * s,
+                                 elu1_f32(__uint_as_float(w[e] & 0xFFFF0000u)) * s);
+            } else {
+                const uint32_t ph = elu1_bf16x2(w[e]);
+                asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(w[e]) : "r"(ph), "r"(s2));
+            }
+        }
+        sts128(tile + sw128_off(row, blk * 64 + cc * 8), make_uint4(w[0], w[1], w[2], w[3]));
     }
 }
 
@@ -286,12 +332,6 @@ __device__ __forceinline__ void mask_pack_row(uint32_t src, uint32_t dst, Keep k
 
 // ---- fp16 operand helpers (the forward-order pass runs its MMAs on fp16)
 
-__device__ __forceinline__ uint32_t pack_f16(float a, float b)
-{
-    __half2 h = __floats2half2_rn(a, b);
-    return *reinterpret_cast<uint32_t *>(&h);
-}
-
 __device__ __forceinline__ void unpack8_f16(uint4 u, float *f)
 {
     const __half2 *h = reinterpret_cast<const __half2 *>(&u);
@@ -311,39 +351,9 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t x)
     return pack_f16(__uint_as_float(x << 16), __uint_as_float(x & 0xFFFF0000u));
 }
 
-// elu(x)+1 of two bf16 values, as fp16: max(x,0) + 2^(min(x,0) log2 e), the
-// exponent argument rounded once to fp16 and the packed exp2 in fp16 (11
-// significant bits, so phi - 1 keeps ~8 bits for |x| ~ 0.1).
-__device__ __forceinline__ uint32_t elu1_f16x2_from_bf16x2(uint32_t x)
-{
-    const float lo = __uint_as_float(x << 16), hi = __uint_as_float(x & 0xFFFF0000u);
-    const uint32_t arg = pack_f16(fminf(lo, 0.f) * 1.4426950408889634f, fminf(hi, 0.f) * 1.4426950408889634f);
-    const uint32_t pos = pack_f16(fmaxf(lo, 0.f), fmaxf(hi, 0.f));
-    uint32_t ex, r;
-    asm("ex2.approx.f16x2 %0, %1;" : "=r"(ex) : "r"(arg));
-    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(pos), "r"(ex));
-    return r;
-}
-
-__device__ __forceinline__ void phi_row_f16(uint32_t tile, int row, bool zero)
-{
-#pragma unroll
-    for (int blk = 0; blk < 2; ++blk) {
-        uint4 raw[8];
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) raw[cc] = lds128(tile + sw128_off(row, blk * 64 + cc * 8));
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-            const uint4 r = raw[cc];
-            sts128(tile + sw128_off(row, blk * 64 + cc * 8),
-                   zero ? make_uint4(0u, 0u, 0u, 0u)
-                        : make_uint4(elu1_f16x2_from_bf16x2(r.x), elu1_f16x2_from_bf16x2(r.y),
-                                     elu1_f16x2_from_bf16x2(r.z), elu1_f16x2_from_bf16x2(r.w)));
-        }
-    }
-}
-
-// phi_row_f16 on the 64-column block `blk` only (two threads per row).
+// elu(x)+1 of the 64-column block `blk` of row `row` of a bf16 SW128 tile,
+// rewritten in place as fp16 (the forward-order pass's operands); zeros when
+// `zero`.
 __device__ __forceinline__ void phi_block_f16(uint32_t tile, int row, bool zero, int blk)
 {
     uint4 raw[8];
@@ -832,6 +842,28 @@ __device__ __forceinline__ void mask_pack_half_hilo_gate(uint32_t src, uint32_t 
 
 
 __device__ __forceinline__ float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+
+// Columns [c_lo, c_hi) (multiples of 8) of row r of a bf16 head tile and its
+// bf16 remainder tile (128-row SW32): (head + remainder) times s, split again
+// into a head and a remainder.
+__device__ __forceinline__ void scale_row_hilo(uint32_t thi, uint32_t tlo, int r, int c_lo, int c_hi, float s)
+{
+#pragma unroll 1
+    for (int c0 = c_lo; c0 < c_hi; c0 += 8) {
+        const uint32_t off = sw32_off(r, c0, 128);
+        float h[8], lo[8];
+        unpack8(lds128(thi + off), h);
+        unpack8(lds128(tlo + off), lo);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            h[e] = (h[e] + lo[e]) * s;
+            lo[e] = h[e] - bf16_round(h[e]);
+        }
+        sts128(thi + off, make_uint4(pack_bf16(h[0], h[1]), pack_bf16(h[2], h[3]), pack_bf16(h[4], h[5]), pack_bf16(h[6], h[7])));
+        sts128(tlo + off,
+               make_uint4(pack_bf16(lo[0], lo[1]), pack_bf16(lo[2], lo[3]), pack_bf16(lo[4], lo[5]), pack_bf16(lo[6], lo[7])));
+    }
+}
 
 // Column sums over a warp's 32 rows of a 32-column block held one row per
 // lane (v[c] = row lane's column c; v is overwritten): lane l returns the sum
@@ -1455,17 +1487,18 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 }
 
 // ---------------------------------------------------------------------------
-// State increments for the forward-order pass: for each segment but the
-// last, sum over its tokens of phi(k_j) [v_j | 1]^T, with the operand type of
-// the pass that consumes them.
+// State increments for the forward-order pass, Taylor map: for each segment
+// but the last, sum over its tokens of phi(k_j) [v_j | 1]^T (bf16 operands,
+// like the pass that consumes them).  128 threads, one per row, two load
+// stages; the phi(K) tile is built from the raw tile of the stage.
 template <class Cfg, bool GATED = false>
 __global__ void __launch_bounds__(128, 1)
 bwd_sstate_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const BwdParams p)
 {
     using namespace bwd_detail;
-    constexpr int C = Cfg::C, D = Cfg::D, DV = Cfg::DV, NA = Cfg::NA, F = Cfg::F, NT = Cfg::NT;
-    constexpr bool TAY = Cfg::TAYLOR, F16 = Cfg::F16;
+    static_assert(Cfg::TAYLOR, "the elu shapes take bwd_sstate3_kernel");
+    constexpr int C = Cfg::C, DV = Cfg::DV, NA = Cfg::NA, F = Cfg::F, NT = Cfg::NT;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *tma_bar = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
@@ -1477,9 +1510,8 @@ bwd_sstate_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     if (seg == p.P - 1) return;   // the last segment's increment is never read
     const int c_begin = seg * p.cps, c_end = min(p.nchunks, c_begin + p.cps);
     const int N = p.N;
-    // two stages of [K | V_aug]: elu: the K tiles in the K and Q regions;
-    // Taylor: the raw K tiles, and one phi(K) tile in the K region
-    uint8_t *sKs[2] = {smem + (TAY ? Cfg::OFF_RK : Cfg::OFF_K), smem + (TAY ? Cfg::OFF_RQ : Cfg::OFF_Q)};
+    // two stages of [raw K | V_aug], and one phi(K) tile in the K region
+    uint8_t *sKs[2] = {smem + Cfg::OFF_RK, smem + Cfg::OFF_RQ};
     uint8_t *sVs[2] = {smem + Cfg::OFF_V, smem + Cfg::OFF_G};
     const uint32_t aPK = smem_addr(smem + Cfg::OFF_K);
     uint64_t *tma_b[2] = {tma_bar, tma_bar + 4};
@@ -1491,12 +1523,10 @@ bwd_sstate_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         mbar_init_fence();
     }
     if (warp == 0) tmem_alloc(tmem_slot, 256);
-    write_first<F16>(sVs[0] + (DV / 16) * Cfg::BLK, tid, 1.f);
-    write_first<F16>(sVs[1] + (DV / 16) * Cfg::BLK, tid, 1.f);
-    if constexpr (TAY) {
+    write_first<false>(sVs[0] + (DV / 16) * Cfg::BLK, tid, 1.f);
+    write_first<false>(sVs[1] + (DV / 16) * Cfg::BLK, tid, 1.f);
 #pragma unroll
-        for (int f0 = F; f0 < Cfg::FT; f0 += 8) sts128(aPK + sw128_off(tid, f0), make_uint4(0u, 0u, 0u, 0u));
-    }
+    for (int f0 = F; f0 < Cfg::FT; f0 += 8) sts128(aPK + sw128_off(tid, f0), make_uint4(0u, 0u, 0u, 0u));
     __syncthreads();
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane = (uint32_t)(warp * 32) << 16;
@@ -1504,10 +1534,8 @@ bwd_sstate_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     // MMA has finished with the stage, a whole chunk ahead of their use
     auto issue = [&](int chunk) {
         const int st = (chunk - c_begin) & 1, t0 = chunk * C;
-        mbar_arrive_expect_tx(tma_b[st], (TAY ? Cfg::RAW : C * D * 2) + C * DV * 2);
-        if constexpr (TAY) tma_load_3d(sKs[st], &tm_k, tma_b[st], 0, t0, bh);
-        else
-            for (int x = 0; x < D; x += 64) tma_load_3d(sKs[st] + (x / 64) * C * 128, &tm_k, tma_b[st], x, t0, bh);
+        mbar_arrive_expect_tx(tma_b[st], Cfg::RAW + C * DV * 2);
+        tma_load_3d(sKs[st], &tm_k, tma_b[st], 0, t0, bh);
         for (int x = 0; x < DV; x += 16) tma_load_3d(sVs[st] + (x / 16) * Cfg::BLK, &tm_v, tma_b[st], x, t0, bh);
     };
     int issued = c_begin, waited = c_begin;   // thread 0: chunks whose loads went out / were waited for
@@ -1526,41 +1554,30 @@ bwd_sstate_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         }
         if (!mbar_wait(tma_b[st], (uint32_t)((chunk - c_begin) >> 1) & 1u)) *abort_flag = 1;
         waited = chunk + 1;
-        if constexpr (TAY) {
+        {
             float x[16];
             raw_row16(aKs, i, x);
             tay_phi_row<0, 20>(aPK, i, x, t0 + i >= N, p);
-        } else {
-            if (D == 128) phi_row_f16(aKs, i, t0 + i >= N);
-            else phi_block_f16(aKs, i, t0 + i >= N, 0);
-#pragma unroll
-            for (int c0 = 0; c0 < DV; c0 += 8) {
-                const uint32_t a = aV + sw32_off(i, c0, C);
-                const uint4 r = lds128(a);
-                sts128(a, make_uint4(bf16x2_to_f16x2(r.x), bf16x2_to_f16x2(r.y), bf16x2_to_f16x2(r.z),
-                                     bf16x2_to_f16x2(r.w)));
-            }
         }
         if constexpr (GATED) {
             // S <- exp(L_last) S + sum_j exp(L_last - L_j) phi(k_j) [v_j | 1]^T
             const float w = __expf(Llast - Lrow);
-            scale_row_sw32<F16>(aV, i, 0, DV, w);
-            write_first<F16>(sVs[st] + (DV / 16) * Cfg::BLK, i, w);
+            scale_row_sw32<false>(aV, i, 0, DV, w);
+            write_first<false>(sVs[st] + (DV / 16) * Cfg::BLK, i, w);
             if (chunk > c_begin) decay_state_tiles<Cfg>(tmem, lane, warp, 0, NA, __expf(Llast));
         }
         full_sync();
         if (*abort_flag) break;
         if (tid == 0) {
-            const uint32_t aPhi = TAY ? aPK : aKs;
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
                 const int m = Cfg::tile_m(t);
-                const uint32_t a_base = aPhi + (Cfg::tile_f0(t) / 64) * (C * 128);
+                const uint32_t a_base = aPK + (Cfg::tile_f0(t) / 64) * (C * 128);
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
                     mma_bf16(tmem + t * NA, smem_desc(a_base + kk * 2048, C * 128, 1024, kSw128),
-                             smem_desc(aV + kk * 512, Cfg::BLK, 256, kSw32),
-                             F16 ? idesc_f16(m, NA, 1, 1) : idesc_bf16(m, NA, 1, 1), chunk > c_begin || kk > 0);
+                             smem_desc(aV + kk * 512, Cfg::BLK, 256, kSw32), idesc_bf16(m, NA, 1, 1),
+                             chunk > c_begin || kk > 0);
             }
             mma_commit(mma_bar);
         }
@@ -1623,19 +1640,6 @@ __device__ __forceinline__ void row_to_f16(uint32_t tile, int r, int c_lo, int c
         } else {
             sts128(a, make_uint4(bf16x2_to_f16x2(u.x), bf16x2_to_f16x2(u.y), bf16x2_to_f16x2(u.z), bf16x2_to_f16x2(u.w)));
         }
-    }
-}
-
-// Columns [c_lo, c_hi) of row r of a bf16 SW32 tile of 128 rows times s.
-__device__ __forceinline__ void row_scale_bf16(uint32_t tile, int r, int c_lo, int c_hi, float s)
-{
-#pragma unroll 1
-    for (int c0 = c_lo; c0 < c_hi; c0 += 8) {
-        const uint32_t a = tile + sw32_off(r, c0, 128);
-        float f[8];
-        unpack8(lds128(a), f);
-        sts128(a, make_uint4(pack_bf16(f[0] * s, f[1] * s), pack_bf16(f[2] * s, f[3] * s), pack_bf16(f[4] * s, f[5] * s),
-                             pack_bf16(f[6] * s, f[7] * s)));
     }
 }
 
@@ -1775,7 +1779,7 @@ bwd_sstate3_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 // R increments (elu): for each segment but the first, the sum over its tokens
 // of phi(q_i) G'_i^T (gated: chunks taken from the segment's end, query i
 // weighted by exp(L_i), the sum decayed by each earlier chunk's gate), on the
-// pipeline of bwd_sstate3_kernel with stages of [Q | G'_aug].
+// pipeline of bwd_sstate3_kernel with stages of [Q | dO_aug].
 template <class Cfg, bool GATED = false>
 __global__ void __launch_bounds__(256, 1)
 bwd_rstate3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
@@ -1833,14 +1837,14 @@ bwd_rstate3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const float dden = valid ? p.dd[((size_t)bh * N + t0 + row) * 2 + 1] : 0.f;
         if (!mbar_wait(&tma_b[st], (uint32_t)(k / 3) & 1u)) *abort_flag = 1;
         if (tid == 0) waited = k + 1;
-        // phi(Q) in place, G' = [dO / den | dden] (gated: query row i times exp(L_i))
-        const float e = GATED ? __expf(Lrow) : 1.f;
-        if (D == 128 || hh == 0) phi_block_inplace(aQ, row, false, D == 128 ? hh : 0);
-        if (D == 128 || hh == 1) {
-            const int c_lo = D == 128 ? 64 * hh : 0, c_hi = D == 128 ? 64 * hh + 64 : DV;
-            row_scale_bf16(aG, row, c_lo, c_hi, valid ? e / den : 0.f);
-            if (c_lo == 0) write_dden(sB(st) + (DV / 16) * Cfg::BLK, row, valid ? e * dden : 0.f);
-        }
+        // phi(q_i) G'_i^T with G'_i = [dO_i / den_i | dden_i] (gated: times
+        // exp(L_i)), taken as (phi(q_i) s_i) [dO_i | den_i dden_i]^T with
+        // s_i = exp(L_i) / den_i: dO stays exact in bf16 and the scale rounds
+        // once, with phi
+        const float si = valid ? (GATED ? __expf(Lrow) : 1.f) / den : 0.f;
+        if (D == 128 || hh == 0) phi_block_scaled<GATED>(aQ, row, si, D == 128 ? hh : 0);
+        if ((D == 128 && hh == 0) || (D != 128 && hh == 1))
+            write_dden(sB(st) + (DV / 16) * Cfg::BLK, row, valid ? den * dden : 0.f);
         if constexpr (GATED) {
             if (k > 0) {
                 if (!mbar_wait(&mma_b[(k - 1) % 3], (uint32_t)((k - 1) / 3) & 1u)) *abort_flag = 1;
@@ -1877,16 +1881,17 @@ bwd_rstate3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 }
 
 // ---------------------------------------------------------------------------
-// R increments: for each segment but the first, sum over its tokens of
-// phi(q_i) G'_i^T (needs den_i, dden_i from the forward-order pass).
+// R increments, Taylor map: for each segment but the first, sum over its
+// tokens of phi(q_i) G'_i^T (needs den_i, dden_i from the forward-order pass);
+// the pipeline of bwd_sstate_kernel with stages of [raw Q | G'_aug].
 template <class Cfg, bool GATED = false>
 __global__ void __launch_bounds__(128, 1)
 bwd_rstate_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                   const BwdParams p)
 {
     using namespace bwd_detail;
-    constexpr int C = Cfg::C, D = Cfg::D, DV = Cfg::DV, NA = Cfg::NA, F = Cfg::F, NT = Cfg::NT;
-    constexpr bool TAY = Cfg::TAYLOR;
+    static_assert(Cfg::TAYLOR, "the elu shapes take bwd_rstate3_kernel");
+    constexpr int C = Cfg::C, DV = Cfg::DV, NA = Cfg::NA, F = Cfg::F, NT = Cfg::NT;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *tma_bar = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
@@ -1898,9 +1903,8 @@ bwd_rstate_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (seg == 0) return;   // the first segment's increment is never read
     const int c_begin = seg * p.cps, c_end = min(p.nchunks, c_begin + p.cps);
     const int N = p.N;
-    // two stages of [Q | G'_aug]: elu: the Q tiles in the Q and K regions;
-    // Taylor: the raw Q tiles, and one phi(Q) tile in the Q region
-    uint8_t *sQs[2] = {smem + (TAY ? Cfg::OFF_RQ : Cfg::OFF_Q), smem + (TAY ? Cfg::OFF_RK : Cfg::OFF_K)};
+    // two stages of [raw Q | G'_aug], and one phi(Q) tile in the Q region
+    uint8_t *sQs[2] = {smem + Cfg::OFF_RQ, smem + Cfg::OFF_RK};
     uint8_t *sGs[2] = {smem + Cfg::OFF_G, smem + Cfg::OFF_V};
     const uint32_t aPQ = smem_addr(smem + Cfg::OFF_Q);
     uint64_t *tma_b[2] = {tma_bar, tma_bar + 4};
@@ -1912,10 +1916,8 @@ bwd_rstate_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         mbar_init_fence();
     }
     if (warp == 0) tmem_alloc(tmem_slot, 256);
-    if constexpr (TAY) {
 #pragma unroll
-        for (int f0 = F; f0 < Cfg::FT; f0 += 8) sts128(aPQ + sw128_off(tid, f0), make_uint4(0u, 0u, 0u, 0u));
-    }
+    for (int f0 = F; f0 < Cfg::FT; f0 += 8) sts128(aPQ + sw128_off(tid, f0), make_uint4(0u, 0u, 0u, 0u));
     __syncthreads();
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane = (uint32_t)(warp * 32) << 16;
@@ -1926,10 +1928,8 @@ bwd_rstate_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     auto chunk_of = [&](int it) { return GATED ? c_end - 1 - it : c_begin + it; };
     auto issue = [&](int it) {
         const int st = it & 1, t0 = chunk_of(it) * C;
-        mbar_arrive_expect_tx(tma_b[st], (TAY ? Cfg::RAW : C * D * 2) + C * DV * 2);
-        if constexpr (TAY) tma_load_3d(sQs[st], &tm_q, tma_b[st], 0, t0, bh);
-        else
-            for (int x = 0; x < D; x += 64) tma_load_3d(sQs[st] + (x / 64) * C * 128, &tm_q, tma_b[st], x, t0, bh);
+        mbar_arrive_expect_tx(tma_b[st], Cfg::RAW + C * DV * 2);
+        tma_load_3d(sQs[st], &tm_q, tma_b[st], 0, t0, bh);
         for (int x = 0; x < DV; x += 16) tma_load_3d(sGs[st] + (x / 16) * Cfg::BLK, &tm_do, tma_b[st], x, t0, bh);
     };
     int issued = 0, waited = 0;   // counts of chunks taken
@@ -1948,13 +1948,10 @@ bwd_rstate_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             Lrow = gate_prefix(p.logdecay + (size_t)bh * N + t0, i, min(C, N - t0), warp, tid & 31, true, gL, Llast);
         if (!mbar_wait(tma_b[st], (uint32_t)(it >> 1) & 1u)) *abort_flag = 1;
         waited = it + 1;
-        if constexpr (TAY) {
+        {
             float x[16];
             raw_row16(aQs, i, x);
             tay_phi_row<0, 20>(aPQ, i, x, false, p);
-        } else {
-            if (D == 128) phi_row_inplace(aQs, i, false);
-            else phi_block_inplace(aQs, i, false, 0);
         }
         {
             // gated: query row i enters R scaled by exp(L_i)
@@ -1978,11 +1975,10 @@ bwd_rstate_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (*abort_flag) break;
         if (tid == 0) {
             // R_aug += phi(Q)^T G'   (M = F features, N = NA, K = tokens)
-            const uint32_t aPhi = TAY ? aPQ : aQs;
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
                 const int m = Cfg::tile_m(t);
-                const uint32_t a_base = aPhi + (Cfg::tile_f0(t) / 64) * (C * 128);
+                const uint32_t a_base = aPQ + (Cfg::tile_f0(t) / 64) * (C * 128);
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
                     mma_bf16(tmem + t * NA, smem_desc(a_base + kk * 2048, C * 128, 1024, kSw128),
@@ -2150,12 +2146,12 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tay_phi_row<80, 10>(aK, j, xk, !valid, p);
             }
         } else if (D == 128) {
-            phi_block_inplace(aQ, j, false, hh);
-            phi_block_inplace(aK, j, !valid, hh);
+            phi_block_inplace<GATED>(aQ, j, false, hh);
+            phi_block_inplace<GATED>(aK, j, !valid, hh);
         } else if (hh == 0) {
-            phi_block_inplace(aQ, j, false, 0);
+            phi_block_inplace<GATED>(aQ, j, false, 0);
         } else {
-            phi_block_inplace(aK, j, !valid, 0);
+            phi_block_inplace<GATED>(aK, j, !valid, 0);
         }
         float dden_row;
         {
@@ -2279,11 +2275,17 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
         }
         if constexpr (GATED) {
-            // G''s last use below is the R update: scale query row j by exp(L_j),
+            // G''s last use below is the R update: scale query row j by exp(L_j)
+            // (head and remainder: dL/dg sums phi(k) . dphi(k) over the sequence,
+            // and a bf16 G' in R leaves ~2^-9 of noise in each of those terms),
             // and decay R by the chunk's whole gate
             const float e = __expf(Lrow);
-            scale_row_sw32<false>(aG, j, hh * (DV / 2), (hh + 1) * (DV / 2), e);
-            if (hh == 0) write_dden(sG + (DV / 16) * Cfg::BLK, j, dden_row * e);
+            scale_row_hilo(aG, aGL, j, hh * (DV / 2), (hh + 1) * (DV / 2), e);
+            if (hh == 0) {
+                const float x = dden_row * e;
+                write_dden(sG + (DV / 16) * Cfg::BLK, j, x);
+                write_dden(sGL + (DV / 16) * Cfg::BLK, j, x - bf16_round(x));
+            }
             decay_state_tiles<Cfg>(tR, lane, wq, na_lo, na_hi, __expf(Llast));
         }
         full_sync();
@@ -2332,9 +2334,13 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const int m = Cfg::tile_m(t);
                 const uint32_t a_base = aQ + (Cfg::tile_f0(t) / 64) * (C * 128);
 #pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk)
+                for (int kk = 0; kk < C / 16; ++kk) {
                     mma_bf16(tR + t * NA, smem_desc(a_base + kk * 2048, C * 128, 1024, kSw128),
                              smem_desc(aG + kk * 512, Cfg::BLK, 256, kSw32), idesc_bf16(m, NA, 1, 1), true);
+                    if constexpr (GATED)
+                        mma_bf16(tR + t * NA, smem_desc(a_base + kk * 2048, C * 128, 1024, kSw128),
+                                 smem_desc(aGL + kk * 512, Cfg::BLK, 256, kSw32), idesc_bf16(m, NA, 1, 1), true);
+                }
             }
             mma_commit(mma_bar);
         }
