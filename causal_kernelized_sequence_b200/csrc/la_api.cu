@@ -370,10 +370,10 @@ la_status forward_tc_run(const CUtensorMap &tq, const CUtensorMap &tk, const CUt
     if (set_smem<fwd_tc_kernel<Cfg, 0, GATED>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
     if (p.P > 1) {
         if (set_smem<fwd_tc_kernel<Cfg, 1, GATED>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
-        fwd_tc_kernel<Cfg, 1, GATED><<<BH * p.P, 256, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+        fwd_tc_kernel<Cfg, 1, GATED><<<BH * p.P, 288, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
         if (launch_status() != LA_OK) return LA_ERR_CUDA;
     }
-    fwd_tc_kernel<Cfg, 0, GATED><<<BH * p.P, 256, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+    fwd_tc_kernel<Cfg, 0, GATED><<<BH * p.P, 288, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
     return launch_status();
 }
 

@@ -10,8 +10,9 @@
 // (DV + 16 columns), so S_aug = [S | z] and one accumulator row holds both
 // numerator and denominator, rounded identically.
 //
-// Per chunk (one CTA of 256 threads; token i <-> TMEM lane i, whose row two
-// threads share, warps w and w + 4 each taking half of its columns):
+// Per chunk (one CTA of 256 worker threads plus one warp whose first thread
+// issues the MMAs and the refill loads; token i <-> TMEM lane i, whose row two
+// workers share, warps w and w + 4 each taking half of its columns):
 //   TMA     Q_c, K_c (SW128, or SW32 for d'=16) and V_c (SW32) into a
 //           2-stage ring (one stage for d = 128).  Rows past the slice's
 //           end read as zeros (fixed length) or hold the next packed
@@ -235,7 +236,7 @@ __device__ __forceinline__ void taylor_sym_to_full(int f, int &r1, int &r2, floa
 // each segment only (written to p.ws).  GATED: the gated form (p.logdecay);
 // a template flag, so the ungated kernels carry none of its work.
 template <class Cfg, int MODE, bool GATED>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(288, 1)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const FwdParams p)
 {
@@ -251,10 +252,14 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tma_bar + 3);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tma_bar + 4);
 
-    // 256 threads: warp w reaches TMEM lanes 32 (w % 4) .. + 31 and takes
-    // column half w / 4 of the row it owns there.
+    // 288 threads.  Workers 0..255: warp w reaches TMEM lanes 32 (w % 4) .. + 31
+    // and takes column half w / 4 of the row it owns there.  Warp 8: its first
+    // thread issues the MMAs and refills the load stages, so that no worker
+    // stalls behind the tensor pipe's issue queue; every thread meets at the
+    // block barriers.
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wq = warp & 3, half = warp >> 2, row = wq * 32 + lane;
+    const bool worker = tid < 256, issuer = tid == 256;
     const int bh = blockIdx.x / p.P, seg = blockIdx.x % p.P;   // bh: the state slice
     // This slice's tokens: fixed length N at rows bh*N.. of a [BH, N, *] tensor
     // (TMA coordinates (x, t, bh)), or packed sequence n at rows h*T + cu[n]..
@@ -336,7 +341,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     // earlier term first decays by the gates of the segments after it:
     // acc <- exp(L_seg) acc + dS_seg, from the entering state through seg - 1
     if (MODE == 0 && (seg > 0 || p.s_in)) {
-        for (int t = 0; t < Cfg::NT; ++t) {
+        for (int t = 0; t < (worker ? Cfg::NT : 0); ++t) {
             const int m = Cfg::tile_m(t);
             const int r = (m == 128) ? row : ((lane < 16) ? wq * 16 + lane : -1);
             const int f = r < 0 ? -1 : Cfg::tile_f0(t) + r;
@@ -471,13 +476,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (gated) {
             // gates below e^-80 count as e^-80: zero next to any surviving term
             // in fp32, and it keeps L finite, so differences of L never meet inf - inf
-            float x = row < nvalid ? fmaxf(p.logdecay[row0 + t0 + row], -80.f) : 0.f;
+            float x = worker && row < nvalid ? fmaxf(p.logdecay[row0 + t0 + row], -80.f) : 0.f;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
                 const float y = __shfl_up_sync(0xffffffffu, x, off);
                 if (lane >= off) x += y;
             }
-            if (half == 0 && lane == 31) gTot[wq] = x;
+            if (worker && half == 0 && lane == 31) gTot[wq] = x;
             __syncthreads();
             float before = 0.f;
 #pragma unroll
@@ -491,6 +496,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             gate_w = __expf(gate_last - gate_L);
             seg_log += gate_last;
         }
+        // (the issuer waits too: its MMAs read the stage)
         if (!mbar_wait(&tma_bar[s], tphase)) *abort_flag = 1;
         uint8_t *sQ = smem + Cfg::OFF_Q + s * Cfg::QK_TILE;
         uint8_t *sK = smem + Cfg::OFF_K + s * Cfg::QK_TILE;
@@ -499,7 +505,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         uint8_t *sPK = Cfg::TAYLOR ? smem + Cfg::OFF_PK : sK;
 
         // ---- feature maps (token row `row`, column half `half`)
-        {
+        if (worker) {
             const int i = row;
             const bool kvalid = i < nvalid;
             if (!Cfg::TAYLOR) {
@@ -548,7 +554,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
         }
         // segment pass, gated: the carried state decays before MMA3 adds to it
-        if (MODE == 1 && gated && have_state) decay_state(gate_last);
+        if (worker && MODE == 1 && gated && have_state) decay_state(gate_last);
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
@@ -556,7 +562,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (*abort_flag) break;
 
         // ---- MMA1 (scores) and MMA3 (state update)
-        if (tid == 0) {
+        if (issuer) {
             const uint32_t aQ = smem_addr(sPQ), aK = smem_addr(sPK), aV = smem_addr(sV);
             if (MODE == 0) {
                 if (Cfg::TAYLOR) {
@@ -578,7 +584,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             if (MODE == 1) mma_commit(mma_bar);
         }
         if (MODE == 0) {
-            if (!mbar_wait(x_bar, x_phase)) *abort_flag = 1;
+            if (worker && !mbar_wait(x_bar, x_phase)) *abort_flag = 1;
             x_phase ^= 1u;
         } else {
             if (!mbar_wait(mma_bar, mma_phase)) *abort_flag = 1;
@@ -589,13 +595,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
         if (MODE == 1) {
             __syncthreads();
-            if (tid == 0 && it + STAGES < c_end - c_begin) issue_tma(chunk + STAGES, s);
+            if (issuer && it + STAGES < c_end - c_begin) issue_tma(chunk + STAGES, s);
             if (*abort_flag) break;
             continue;
         }
 
         // ---- causal mask -> P (bf16, K-major SW128); keys of this thread's half
-        {
+        if (worker) {
             const int i = row;
             uint8_t *sP = smem + Cfg::OFF_P;
 #pragma unroll 1
@@ -618,7 +624,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                                    pack_bf16(a[e + 4], a[e + 5]), pack_bf16(a[e + 6], a[e + 7]));
             }
         }
-        if (gated) {
+        if (gated && worker) {
             // elu: phi tiles are also MMA1's operands, so they are scaled only
             // now that MMA1 has completed (Taylor scaled them when computing them)
             if (!Cfg::TAYLOR) {
@@ -634,7 +640,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tc_fence_after();
 
         // ---- MMA2: O_aug = P V_aug + phi(Q) S_snap
-        if (tid == 0) {
+        if (issuer) {
             const uint32_t aP = smem_addr(smem + Cfg::OFF_P), aV = smem_addr(sV);
             const uint32_t idesc = idesc_bf16(128, NA, 0, 1);
 #pragma unroll
@@ -659,10 +665,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         mma_phase ^= 1u;
         tc_fence_after();
         if (gated) have_state = true;
-        if (tid == 0 && it + STAGES < c_end - c_begin) issue_tma(chunk + STAGES, s);
+        if (issuer && it + STAGES < c_end - c_begin) issue_tma(chunk + STAGES, s);
 
         // ---- outputs: y = num / den (this thread's half of the value columns)
-        {
+        if (worker) {
             const int i = row;
             constexpr int DH = DV / 2;
             float o[DH], d16[16];
@@ -683,7 +689,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
         }
         // ---- state snapshot for the next chunk (bf16, MN-major SW32)
-        if (chunk + 1 < c_end) {
+        if (worker && chunk + 1 < c_end) {
             uint8_t *sS = smem + Cfg::OFF_S;
 #pragma unroll
             for (int t = 0; t < Cfg::NT; ++t) {
@@ -720,7 +726,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     // gated: the entering state's antisymmetric part (restored below) has
     // decayed by every gate of the sequence
     const float skew_decay = gated ? __expf(lsum_before + seg_log) : 1.f;
-    if ((write_ws || write_final) && !*abort_flag) {
+    if (worker && (write_ws || write_final) && !*abort_flag) {
 #pragma unroll 1
         for (int t = 0; t < Cfg::NT; ++t) {
             const int m = Cfg::tile_m(t);
