@@ -364,16 +364,16 @@ bool make_map(CUtensorMap *m, const void *base, int inner, int N, int BH, int bo
 
 // The segment-state launch (P > 1) and the main launch of fwd_tc_kernel.
 template <class Cfg, bool GATED>
-la_status forward_tc_run(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv, const FwdParams &p,
-                         int BH, cudaStream_t stream)
+la_status forward_tc_run(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &to,
+                         const FwdParams &p, int BH, cudaStream_t stream)
 {
     if (set_smem<fwd_tc_kernel<Cfg, 0, GATED>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
     if (p.P > 1) {
         if (set_smem<fwd_tc_kernel<Cfg, 1, GATED>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
-        fwd_tc_kernel<Cfg, 1, GATED><<<BH * p.P, 288, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+        fwd_tc_kernel<Cfg, 1, GATED><<<BH * p.P, 288, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, to, p);
         if (launch_status() != LA_OK) return LA_ERR_CUDA;
     }
-    fwd_tc_kernel<Cfg, 0, GATED><<<BH * p.P, 288, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+    fwd_tc_kernel<Cfg, 0, GATED><<<BH * p.P, 288, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, to, p);
     return launch_status();
 }
 
@@ -387,13 +387,17 @@ la_status forward_tc_launch(const void *q, const void *k, const void *v, void *o
     // sequences (cu != null): B sequences of at most N tokens, tensors [H, T, *].
     const int BH = B * H;
     const int map_rows = cu ? T : N, map_slices = cu ? H : BH;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     const CUtensorMapSwizzle qsw = Cfg::TAYLOR ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_128B;
     const int qbox = Cfg::TAYLOR ? 16 : 64;
     if (!make_map(&tq, q, Cfg::DQK, map_rows, map_slices, qbox, qsw) ||
         !make_map(&tk, k, Cfg::DQK, map_rows, map_slices, qbox, qsw) ||
         !make_map(&tv, v, Cfg::DV, map_rows, map_slices, 16, CU_TENSOR_MAP_SWIZZLE_32B))
         return LA_ERR_CUDA;
+    // y leaves by TMA stores of 64-column SW128 boxes (fixed length; packed
+    // sequences store rows directly and never read this map)
+    if (cu) to = tv;
+    else if (!make_map(&to, o, Cfg::DV, N, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return LA_ERR_CUDA;
     FwdParams p;
     p.s_in = s_in;
     p.z_in = z_in;
@@ -415,8 +419,8 @@ la_status forward_tc_launch(const void *q, const void *k, const void *v, void *o
     p.inv_c2 = (float)(1.0 / (sqrt(2.0) * sqrt(d)));
     p.k1 = (float)(1.0 / sqrt(d));
     p.k2 = (float)(1.0 / (2.0 * d));
-    if (logdecay) return forward_tc_run<Cfg, true>(tq, tk, tv, p, BH, stream);
-    return forward_tc_run<Cfg, false>(tq, tk, tv, p, BH, stream);
+    if (logdecay) return forward_tc_run<Cfg, true>(tq, tk, tv, to, p, BH, stream);
+    return forward_tc_run<Cfg, false>(tq, tk, tv, to, p, BH, stream);
 }
 
 // Chunk-parallel forward (elu, d_qk = d_v = 64): state launch, then output launch.

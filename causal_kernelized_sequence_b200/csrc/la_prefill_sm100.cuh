@@ -238,7 +238,7 @@ __device__ __forceinline__ void taylor_sym_to_full(int f, int &r1, int &r2, floa
 template <class Cfg, int MODE, bool GATED>
 __global__ void __launch_bounds__(288, 1)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-              const __grid_constant__ CUtensorMap tm_v, const FwdParams p)
+              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, const FwdParams p)
 {
     using namespace sm100;
     using namespace fwd_detail;
@@ -294,6 +294,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
+        if (MODE == 0 && !p.cu) prefetch_tensormap(&tm_o);
     }
     if (warp == 0) tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
     // Constant normaliser block of every V stage: column DV of V_aug = 1.
@@ -555,6 +556,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
         // segment pass, gated: the carried state decays before MMA3 adds to it
         if (worker && MODE == 1 && gated && have_state) decay_state(gate_last);
+        // the previous chunk's y store has read its staging tile (the P tile,
+        // which the mask below writes again)
+        if (MODE == 0 && issuer && !p.cu && it > 0) bulk_wait_read();
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
@@ -667,7 +671,12 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (gated) have_state = true;
         if (issuer && it + STAGES < c_end - c_begin) issue_tma(chunk + STAGES, s);
 
-        // ---- outputs: y = num / den (this thread's half of the value columns)
+        // ---- outputs: y = num / den (this thread's half of the value columns).
+        // Fixed length: y goes to the P tile (free once MMA2 has completed) as
+        // SW128 rows and leaves by one TMA store after the chunk's last barrier
+        // (rows past the slice's end are clipped by the tensor map).  Packed
+        // sequences: plain stores of the rows that belong to this sequence.
+        const bool tma_y = !p.cu;
         if (worker) {
             const int i = row;
             constexpr int DH = DV / 2;
@@ -678,15 +687,24 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             tmem_ld_wait();
             const float den = d16[0];
             const float inv = 1.f / den;
-            if (i < nvalid) {
+            if (tma_y) {
+                uint8_t *sY = smem + Cfg::OFF_P;
+#pragma unroll
+                for (int c0 = 0; c0 < DH; c0 += 8) {
+                    const int col = half * DH + c0;
+                    *reinterpret_cast<uint4 *>(sY + (col / 64) * (C * 128) + sw128_off(i, col % 64)) =
+                        make_uint4(pack_bf16(o[c0] * inv, o[c0 + 1] * inv), pack_bf16(o[c0 + 2] * inv, o[c0 + 3] * inv),
+                                   pack_bf16(o[c0 + 4] * inv, o[c0 + 5] * inv), pack_bf16(o[c0 + 6] * inv, o[c0 + 7] * inv));
+                }
+            } else if (i < nvalid) {
                 __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + (size_t)(row0 + t0 + i) * DV + half * DH;
 #pragma unroll
                 for (int c0 = 0; c0 < DH; c0 += 8)
                     *reinterpret_cast<uint4 *>(orow + c0) =
                         make_uint4(pack_bf16(o[c0] * inv, o[c0 + 1] * inv), pack_bf16(o[c0 + 2] * inv, o[c0 + 3] * inv),
                                    pack_bf16(o[c0 + 4] * inv, o[c0 + 5] * inv), pack_bf16(o[c0 + 6] * inv, o[c0 + 7] * inv));
-                if (p.den_out && half == 0) p.den_out[row0 + t0 + i] = den;
             }
+            if (p.den_out && half == 0 && i < nvalid) p.den_out[row0 + t0 + i] = den;
         }
         // ---- state snapshot for the next chunk (bf16, MN-major SW32)
         if (worker && chunk + 1 < c_end) {
@@ -716,8 +734,16 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+        if (MODE == 0 && issuer && tma_y && !*abort_flag) {
+            for (int x = 0; x < DV; x += 64)
+                tma_store_3d(&tm_o, smem + Cfg::OFF_P + (x / 64) * (C * 128), x, t_base + t0, tz);
+            bulk_commit();
+        }
         if (*abort_flag) break;
     }
+    // the last y stores have completed (their staging tile and the block's
+    // shared memory outlive them)
+    if (MODE == 0 && issuer && !p.cu) bulk_wait_all();
 
     // ---- segment increment (MODE 1) or final state (MODE 0, last segment)
     const bool write_ws = (MODE == 1);
