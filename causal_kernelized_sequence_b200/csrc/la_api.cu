@@ -394,10 +394,9 @@ la_status forward_tc_launch(const void *q, const void *k, const void *v, void *o
         !make_map(&tk, k, Cfg::DQK, map_rows, map_slices, qbox, qsw) ||
         !make_map(&tv, v, Cfg::DV, map_rows, map_slices, 16, CU_TENSOR_MAP_SWIZZLE_32B))
         return LA_ERR_CUDA;
-    // y leaves by TMA stores of 64-column SW128 boxes (fixed length; packed
-    // sequences store rows directly and never read this map)
-    if (cu) to = tv;
-    else if (!make_map(&to, o, Cfg::DV, N, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return LA_ERR_CUDA;
+    // y leaves by TMA stores of 64-column SW128 boxes ([BH, N, DV], or the
+    // packed [H, T, DV])
+    if (!make_map(&to, o, Cfg::DV, map_rows, map_slices, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return LA_ERR_CUDA;
     FwdParams p;
     p.s_in = s_in;
     p.z_in = z_in;

@@ -294,7 +294,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
-        if (MODE == 0 && !p.cu) prefetch_tensormap(&tm_o);
+        if (MODE == 0) prefetch_tensormap(&tm_o);
     }
     if (warp == 0) tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
     // Constant normaliser block of every V stage: column DV of V_aug = 1.
@@ -558,7 +558,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (worker && MODE == 1 && gated && have_state) decay_state(gate_last);
         // the previous chunk's y store has read its staging tile (the P tile,
         // which the mask below writes again)
-        if (MODE == 0 && issuer && !p.cu && it > 0) bulk_wait_read();
+        if (MODE == 0 && issuer && it > 0) bulk_wait_read();
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
@@ -672,11 +672,12 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (issuer && it + STAGES < c_end - c_begin) issue_tma(chunk + STAGES, s);
 
         // ---- outputs: y = num / den (this thread's half of the value columns).
-        // Fixed length: y goes to the P tile (free once MMA2 has completed) as
-        // SW128 rows and leaves by one TMA store after the chunk's last barrier
-        // (rows past the slice's end are clipped by the tensor map).  Packed
-        // sequences: plain stores of the rows that belong to this sequence.
-        const bool tma_y = !p.cu;
+        // y goes to the P tile (free once MMA2 has completed) as SW128 rows and
+        // leaves by one TMA store after the chunk's last barrier: at fixed
+        // length rows past the slice's end are clipped by the tensor map; a
+        // packed sequence's partial last chunk would reach into the next
+        // sequence's rows, so there the rows of this sequence are stored directly.
+        const bool tma_y = !p.cu || nvalid == C;
         if (worker) {
             const int i = row;
             constexpr int DH = DV / 2;
@@ -743,7 +744,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     }
     // the last y stores have completed (their staging tile and the block's
     // shared memory outlive them)
-    if (MODE == 0 && issuer && !p.cu) bulk_wait_all();
+    if (MODE == 0 && issuer) bulk_wait_all();
 
     // ---- segment increment (MODE 1) or final state (MODE 0, last segment)
     const bool write_ws = (MODE == 1);
