@@ -502,12 +502,15 @@ la_status backward_tc(const void *q, const void *k, const void *v, const void *d
                       const float *log_decay = nullptr, float *dlog_decay = nullptr)
 {
     const int BH = B * H;
-    CUtensorMap tq, tk, tv, tdo;
+    CUtensorMap tq, tk, tv, tdo, tdq, tdk;
     const int qbox = Cfg::TAYLOR ? 16 : 64;
     const CUtensorMapSwizzle qsw = Cfg::TAYLOR ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_128B;
+    // dq and dk leave through maps of Q's and K's geometry (stores of the tiles
+    // their inputs were loaded into)
     if (!make_map(&tq, q, Cfg::D, N, BH, qbox, qsw) || !make_map(&tk, k, Cfg::D, N, BH, qbox, qsw) ||
         !make_map(&tv, v, Cfg::DV, N, BH, 16, CU_TENSOR_MAP_SWIZZLE_32B) ||
-        !make_map(&tdo, dout, Cfg::DV, N, BH, 16, CU_TENSOR_MAP_SWIZZLE_32B))
+        !make_map(&tdo, dout, Cfg::DV, N, BH, 16, CU_TENSOR_MAP_SWIZZLE_32B) ||
+        !make_map(&tdq, dq, Cfg::D, N, BH, qbox, qsw) || !make_map(&tdk, dk, Cfg::D, N, BH, qbox, qsw))
         return LA_ERR_CUDA;
     BwdParams p;
     tc_segments(B, H, N, &p.P, &p.cps, &p.nchunks);
@@ -555,10 +558,10 @@ la_status backward_tc(const void *q, const void *k, const void *v, const void *d
     if (set_smem<bwd_dq_kernel<Cfg, GATED>>(Cfg::SMEM_ALLOC) != LA_OK ||
         set_smem<bwd_dkdv_kernel<Cfg, GATED>>(Cfg::SMEM_ALLOC) != LA_OK)
         return LA_ERR_CUDA;
-    bwd_dq_kernel<Cfg, GATED><<<BH * p.P, 256, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, p);
+    bwd_dq_kernel<Cfg, GATED><<<BH * p.P, 256, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, tdq, p);
     if (launch_status() != LA_OK) return LA_ERR_CUDA;
     if (p.P > 1 && state_pass(false) != LA_OK) return LA_ERR_CUDA;
-    bwd_dkdv_kernel<Cfg, GATED><<<BH * p.P, 256, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, p);
+    bwd_dkdv_kernel<Cfg, GATED><<<BH * p.P, 256, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, tdk, p);
     if (!GATED) return launch_status();
     if (launch_status() != LA_OK) return LA_ERR_CUDA;
     bwd_dg_kernel<<<BH, 1024, 0, stream>>>(p.cvec, p.dg, N);
@@ -601,10 +604,11 @@ static la_status swa_tc_launch(const void *q, const void *k, const void *v, void
                                cudaStream_t stream)
 {
     using Cfg = SwaCfg<W>;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     if (!make_map(&tq, q, 64, N, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&tk, k, 64, N, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B, Cfg::KW) ||
-        !make_map(&tv, v, 64, N, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B, Cfg::KW))
+        !make_map(&tv, v, 64, N, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B, Cfg::KW) ||
+        !make_map(&to, o, 64, N, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B))
         return LA_ERR_CUDA;
     SwaParams p;
     p.o = (__nv_bfloat16 *)o;
@@ -618,7 +622,7 @@ static la_status swa_tc_launch(const void *q, const void *k, const void *v, void
     const int per_sm = Cfg::TMEM_COLS == 256 ? 2 : 1;   // TMEM: 512 columns per SM
     const int grid = (int)(ntiles < (long long)per_sm * kNumSms ? ntiles : per_sm * kNumSms);
     if (set_smem<swa_fwd_tc_kernel<Cfg>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
-    swa_fwd_tc_kernel<Cfg><<<grid, Cfg::THREADS, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+    swa_fwd_tc_kernel<Cfg><<<grid, Cfg::THREADS, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, to, p);
     return launch_status();
 }
 

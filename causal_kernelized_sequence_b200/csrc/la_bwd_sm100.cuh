@@ -1017,7 +1017,7 @@ template <class Cfg, bool GATED = false>
 __global__ void __launch_bounds__(256, 1)
 bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-              const BwdParams p)
+              const __grid_constant__ CUtensorMap tm_dq, const BwdParams p)
 {
     using namespace bwd_detail;
     constexpr int C = Cfg::C, D = Cfg::D, DV = Cfg::DV, NA = Cfg::NA, F = Cfg::F, NT = Cfg::NT;
@@ -1101,6 +1101,8 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const int t0 = chunk * C, i = row;
         const bool valid = t0 + i < N;
         if (tid == 0) {
+            // the previous chunk's dq left from the Q tile (its raw tile for Taylor)
+            if (chunk > c_begin) bulk_wait_read();
             mbar_arrive_expect_tx(tma_bar, TAY ? 2 * Cfg::RAW + 2 * C * DV * 2 : 2 * C * D * 2 + 2 * C * DV * 2);
             if constexpr (TAY) {
                 tma_load_3d(smem + Cfg::OFF_RQ, &tm_q, tma_bar, 0, t0, bh);
@@ -1404,7 +1406,6 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         {
             const float rden = valid ? 1.f / den_row : 0.f;
             if constexpr (TAY) {
-                __nv_bfloat16 *dqrow = reinterpret_cast<__nv_bfloat16 *>(p.dq) + ((size_t)bh * N + t0 + i) * D;
                 float x[16], dx[16], sd = 0.f;
                 raw_row16(aRQ, i, x);
 #pragma unroll
@@ -1421,12 +1422,11 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 const float proj = sd_all / sn, jt = fmaf(xx, 2.f * p.k2, p.inv_c3);
 #pragma unroll
                 for (int c = 0; c < 8; ++c) d8[c] = (d8[c] - proj * jt * x[8 * hh + c]) * rden;
-                if (valid)
-                    *reinterpret_cast<uint4 *>(dqrow + 8 * hh) =
-                        make_uint4(pack_bf16(d8[0], d8[1]), pack_bf16(d8[2], d8[3]), pack_bf16(d8[4], d8[5]),
-                                   pack_bf16(d8[6], d8[7]));
+                // dq over its own raw q in the raw Q tile (both threads of the row
+                // read it before tay_combine's barrier); one TMA store per chunk
+                sts128(aRQ + sw32_off(i, 8 * hh, 128), make_uint4(pack_bf16(d8[0], d8[1]), pack_bf16(d8[2], d8[3]),
+                                                                  pack_bf16(d8[4], d8[5]), pack_bf16(d8[6], d8[7])));
             } else {
-                __nv_bfloat16 *dqrow = reinterpret_cast<__nv_bfloat16 *>(p.dq) + ((size_t)bh * N + t0 + i) * D;
                 float sd = 0.f, sn = 0.f;
 #pragma unroll 1
                 for (int c0 = hh * (F / 2); c0 < (hh + 1) * (F / 2); c0 += 16) {
@@ -1456,13 +1456,13 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     unpack8_f16(lds128(aQ + sw128_off(i, c0 + 8)), ph + 8);
 #pragma unroll
                     for (int e = 0; e < 16; ++e) g[e] = (g[e] - proj * ph[e]) * fminf(ph[e], 1.f) * rden;
-                    if (valid) {
+                    // dq over the thread's own phi(q) entries (same SW128 layout); one
+                    // TMA store per chunk
 #pragma unroll
-                        for (int e = 0; e < 16; e += 8)
-                            *reinterpret_cast<uint4 *>(dqrow + c0 + e) =
-                                make_uint4(pack_bf16(g[e], g[e + 1]), pack_bf16(g[e + 2], g[e + 3]),
-                                           pack_bf16(g[e + 4], g[e + 5]), pack_bf16(g[e + 6], g[e + 7]));
-                    }
+                    for (int e = 0; e < 16; e += 8)
+                        sts128(aQ + sw128_off(i, c0 + e),
+                               make_uint4(pack_bf16(g[e], g[e + 1]), pack_bf16(g[e + 2], g[e + 3]),
+                                          pack_bf16(g[e + 4], g[e + 5]), pack_bf16(g[e + 6], g[e + 7])));
                 }
             }
             if (chunk + 1 < c_end) {
@@ -1481,7 +1481,16 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
         }
         full_sync();
+        // the chunk's dq (over phi(Q), or over the raw Q tile for Taylor) leaves
+        // by TMA; rows past the slice's end are clipped by the tensor map
+        if (tid == 0 && !*abort_flag) {
+            if constexpr (TAY) tma_store_3d(&tm_dq, smem + Cfg::OFF_RQ, 0, t0, bh);
+            else
+                for (int x = 0; x < D; x += 64) tma_store_3d(&tm_dq, sQ + (x / 64) * C * 128, x, t0, bh);
+            bulk_commit();
+        }
     }
+    if (tid == 0) bulk_wait_all();
     full_sync();
     if (warp == 0) tmem_dealloc(tmem, Cfg::TMEM_COLS);
 }
@@ -2023,7 +2032,7 @@ template <class Cfg, bool GATED = false>
 __global__ void __launch_bounds__(256, 1)
 bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                const BwdParams p)
+                const __grid_constant__ CUtensorMap tm_dk, const BwdParams p)
 {
     using namespace bwd_detail;
     constexpr int C = Cfg::C, D = Cfg::D, DV = Cfg::DV, NA = Cfg::NA, F = Cfg::F, NT = Cfg::NT;
@@ -2111,6 +2120,8 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int t0 = chunk * C, j = row;
         const bool valid = t0 + j < N;
         if (tid == 0) {
+            // the previous chunk's dk left from the K tile (its raw tile for Taylor)
+            if (chunk < c_end - 1) bulk_wait_read();
             mbar_arrive_expect_tx(tma_bar, TAY ? 2 * Cfg::RAW + 2 * C * DV * 2 : 2 * C * D * 2 + 2 * C * DV * 2);
             if constexpr (TAY) {
                 tma_load_3d(smem + Cfg::OFF_RQ, &tm_q, tma_bar, 0, t0, bh);
@@ -2348,7 +2359,6 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mph ^= 1u;
         tc_fence_after();
         {
-            __nv_bfloat16 *dkrow = reinterpret_cast<__nv_bfloat16 *>(p.dk) + ((size_t)bh * N + t0 + j) * D;
             if constexpr (TAY) {
                 float x[16], dx[16], sd = 0.f;
                 raw_row16(aRK, j, x);
@@ -2358,10 +2368,10 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 else tay_vjp_half<1>(tX + lane, x, dx, sd, p);
                 float d8[8], sd_all;
                 tay_combine(red + 6 * C, red + 2 * C, hh, j, dx, sd, d8, sd_all);
-                if (valid)
-                    *reinterpret_cast<uint4 *>(dkrow + 8 * hh) =
-                        make_uint4(pack_bf16(d8[0], d8[1]), pack_bf16(d8[2], d8[3]), pack_bf16(d8[4], d8[5]),
-                                   pack_bf16(d8[6], d8[7]));
+                // dk over its own raw k (read by both threads of the row before the
+                // barrier in tay_combine); one TMA store per chunk
+                sts128(aRK + sw32_off(j, 8 * hh, 128), make_uint4(pack_bf16(d8[0], d8[1]), pack_bf16(d8[2], d8[3]),
+                                                                  pack_bf16(d8[4], d8[5]), pack_bf16(d8[6], d8[7])));
             } else {
 #pragma unroll 1
                 for (int c0 = hh * (F / 2); c0 < (hh + 1) * (F / 2); c0 += 16) {
@@ -2370,14 +2380,14 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     tmem_ld_wait();
                     unpack8(lds128(aK + sw128_off(j, c0)), ph);
                     unpack8(lds128(aK + sw128_off(j, c0 + 8)), ph + 8);
-                    if (valid)
+                    // dk over the thread's own phi(k) entries (same SW128 layout)
 #pragma unroll
-                        for (int e = 0; e < 16; e += 8)
-                            *reinterpret_cast<uint4 *>(dkrow + c0 + e) = make_uint4(
-                                pack_bf16(g[e] * fminf(ph[e], 1.f), g[e + 1] * fminf(ph[e + 1], 1.f)),
-                                pack_bf16(g[e + 2] * fminf(ph[e + 2], 1.f), g[e + 3] * fminf(ph[e + 3], 1.f)),
-                                pack_bf16(g[e + 4] * fminf(ph[e + 4], 1.f), g[e + 5] * fminf(ph[e + 5], 1.f)),
-                                pack_bf16(g[e + 6] * fminf(ph[e + 6], 1.f), g[e + 7] * fminf(ph[e + 7], 1.f)));
+                    for (int e = 0; e < 16; e += 8)
+                        sts128(aK + sw128_off(j, c0 + e), make_uint4(
+                            pack_bf16(g[e] * fminf(ph[e], 1.f), g[e + 1] * fminf(ph[e + 1], 1.f)),
+                            pack_bf16(g[e + 2] * fminf(ph[e + 2], 1.f), g[e + 3] * fminf(ph[e + 3], 1.f)),
+                            pack_bf16(g[e + 4] * fminf(ph[e + 4], 1.f), g[e + 5] * fminf(ph[e + 5], 1.f)),
+                            pack_bf16(g[e + 6] * fminf(ph[e + 6], 1.f), g[e + 7] * fminf(ph[e + 7], 1.f))));
                 }
             }
             if constexpr (GATED) {
@@ -2407,7 +2417,15 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
         }
         full_sync();
+        // the chunk's dk leaves by TMA (rows past the slice's end clipped)
+        if (tid == 0 && !*abort_flag) {
+            if constexpr (TAY) tma_store_3d(&tm_dk, smem + Cfg::OFF_RK, 0, t0, bh);
+            else
+                for (int x = 0; x < D; x += 64) tma_store_3d(&tm_dk, sK + (x / 64) * C * 128, x, t0, bh);
+            bulk_commit();
+        }
     }
+    if (tid == 0) bulk_wait_all();
     full_sync();
     if (warp == 0) tmem_dealloc(tmem, Cfg::TMEM_COLS);
 }

@@ -46,7 +46,8 @@ struct SwaCfg {
     static constexpr int OFF_V = REGION_A;
     static constexpr int OFF_BAR = OFF_V + (KV_TILE + 1023) / 1024 * 1024;
     static constexpr int OFF_RED = OFF_BAR + 64;     // row max and row sum of each half: 4 x 128 floats
-    static constexpr int SMEM = OFF_RED + 4 * C * 4;
+    static constexpr int OFF_Y = (OFF_RED + 4 * C * 4 + 1023) / 1024 * 1024;   // o tile (SW128), stored by TMA
+    static constexpr int SMEM = OFF_Y + C * 128;
     static constexpr int COL_S = 0;
     static constexpr int COL_O = (KW + 31) / 32 * 32;
     static constexpr int TMEM_COLS = COL_O + D <= 256 ? 256 : 512;
@@ -76,7 +77,7 @@ struct SwaParams {
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, Cfg::MIN_BLOCKS)
 swa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const SwaParams p)
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, const SwaParams p)
 {
     using namespace sm100;
     using namespace fwd_detail;
@@ -102,6 +103,7 @@ swa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
+        prefetch_tensormap(&tm_o);
     }
     if (warp == 0) tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
     tc_fence_before();
@@ -122,6 +124,15 @@ swa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
     uint32_t load_phase = 0, mma_phase = 0;
     bool load_pending = false;   // thread 0: a tile's loads issued and not yet waited for
+    // A tile's o goes to the o tile in shared memory and leaves by one TMA store,
+    // issued by thread 0 once every thread has passed the next barrier (rows past
+    // the slice's end are clipped by the tensor map)
+    int y_bh = -1, y_t0 = 0;     // thread 0: the tile whose o waits in the o tile
+    auto store_y = [&]() {
+        tma_store_3d(&tm_o, smem + Cfg::OFF_Y, 0, y_t0, y_bh);
+        bulk_commit();
+        y_bh = -1;
+    };
     if (tid == 0 && (int)blockIdx.x < ntiles) {
         issue_loads(blockIdx.x);
         load_pending = true;
@@ -166,6 +177,7 @@ swa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (c < nh && c0 + c >= lo && c0 + c <= hi) m = fmaxf(m, sv[c]);
             red_m[hh * C + i] = m;
             __syncthreads();
+            if (tid == 0 && y_bh >= 0) store_y();   // the previous tile's o
             rowmax = fmaxf(red_m[i], red_m[C + i]);
             float sum = 0.f;
 #pragma unroll
@@ -195,8 +207,10 @@ swa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         tc_fence_after();
         if (*abort_flag) break;
 
-        // ---- MMA2: O = P V
+        // ---- MMA2: O = P V   (its epilogue rewrites the o tile: the previous
+        // tile's store must have read it)
         if (tid == 0) {
+            bulk_wait_read();
             const uint32_t id = idesc_bf16(128, Cfg::D, 0, 1);
 #pragma unroll
             for (int kk = 0; kk < KW / 16; ++kk) {
@@ -224,15 +238,17 @@ swa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
             for (int c = 0; c < DH; c += 16) tmem_ld16(tmem + lane_base + Cfg::COL_O + hh * DH + c, ov + c);
             tmem_ld_wait();
-            if (t0 + i < p.N) {
-                const float inv = 1.f / rowsum;
-                __nv_bfloat16 *orow = p.o + ((size_t)bh * p.N + t0 + i) * Cfg::D + hh * DH;
+            const float inv = 1.f / rowsum;
 #pragma unroll
-                for (int c = 0; c < DH; c += 8)
-                    *reinterpret_cast<uint4 *>(orow + c) =
-                        make_uint4(pack_bf16(ov[c] * inv, ov[c + 1] * inv), pack_bf16(ov[c + 2] * inv, ov[c + 3] * inv),
-                                   pack_bf16(ov[c + 4] * inv, ov[c + 5] * inv), pack_bf16(ov[c + 6] * inv, ov[c + 7] * inv));
-                if (p.lse && hh == 0) p.lse[(size_t)bh * p.N + t0 + i] = rowmax * p.scale + logf(rowsum);
+            for (int c = 0; c < DH; c += 8)
+                sts128(smem_addr(smem + Cfg::OFF_Y) + sw128_off(i, hh * DH + c),
+                       make_uint4(pack_bf16(ov[c] * inv, ov[c + 1] * inv), pack_bf16(ov[c + 2] * inv, ov[c + 3] * inv),
+                                  pack_bf16(ov[c + 4] * inv, ov[c + 5] * inv), pack_bf16(ov[c + 6] * inv, ov[c + 7] * inv)));
+            if (t0 + i < p.N && p.lse && hh == 0) p.lse[(size_t)bh * p.N + t0 + i] = rowmax * p.scale + logf(rowsum);
+            fence_proxy_async();
+            if (tid == 0) {
+                y_bh = bh;
+                y_t0 = t0;
             }
         }
         tc_fence_before();
@@ -242,6 +258,10 @@ swa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (tid == 0) {
+        if (y_bh >= 0 && !*abort_flag) store_y();   // the last tile's o
+        bulk_wait_all();
+    }
     if (warp == 0) tmem_dealloc(tmem, Cfg::TMEM_COLS);
 }
 
