@@ -502,7 +502,7 @@ la_status backward_tc(const void *q, const void *k, const void *v, const void *d
                       const float *log_decay = nullptr, float *dlog_decay = nullptr)
 {
     const int BH = B * H;
-    CUtensorMap tq, tk, tv, tdo, tdq, tdk;
+    CUtensorMap tq, tk, tv, tdo, tdq, tdk, tdv;
     const int qbox = Cfg::TAYLOR ? 16 : 64;
     const CUtensorMapSwizzle qsw = Cfg::TAYLOR ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_128B;
     // dq and dk leave through maps of Q's and K's geometry (stores of the tiles
@@ -510,7 +510,8 @@ la_status backward_tc(const void *q, const void *k, const void *v, const void *d
     if (!make_map(&tq, q, Cfg::D, N, BH, qbox, qsw) || !make_map(&tk, k, Cfg::D, N, BH, qbox, qsw) ||
         !make_map(&tv, v, Cfg::DV, N, BH, 16, CU_TENSOR_MAP_SWIZZLE_32B) ||
         !make_map(&tdo, dout, Cfg::DV, N, BH, 16, CU_TENSOR_MAP_SWIZZLE_32B) ||
-        !make_map(&tdq, dq, Cfg::D, N, BH, qbox, qsw) || !make_map(&tdk, dk, Cfg::D, N, BH, qbox, qsw))
+        !make_map(&tdq, dq, Cfg::D, N, BH, qbox, qsw) || !make_map(&tdk, dk, Cfg::D, N, BH, qbox, qsw) ||
+        !make_map(&tdv, dvp, Cfg::DV, N, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B))
         return LA_ERR_CUDA;
     BwdParams p;
     tc_segments(B, H, N, &p.P, &p.cps, &p.nchunks);
@@ -561,7 +562,7 @@ la_status backward_tc(const void *q, const void *k, const void *v, const void *d
     bwd_dq_kernel<Cfg, GATED><<<BH * p.P, 256, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, tdq, p);
     if (launch_status() != LA_OK) return LA_ERR_CUDA;
     if (p.P > 1 && state_pass(false) != LA_OK) return LA_ERR_CUDA;
-    bwd_dkdv_kernel<Cfg, GATED><<<BH * p.P, 256, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, tdk, p);
+    bwd_dkdv_kernel<Cfg, GATED><<<BH * p.P, 256, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, tdk, tdv, p);
     if (!GATED) return launch_status();
     if (launch_status() != LA_OK) return LA_ERR_CUDA;
     bwd_dg_kernel<<<BH, 1024, 0, stream>>>(p.cvec, p.dg, N);

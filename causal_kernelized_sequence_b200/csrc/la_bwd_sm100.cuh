@@ -129,6 +129,7 @@ struct BwdCfg {
                   "shared-memory alignment");
     static_assert(SL_TILE >= S_TILE && SL_TILE >= VG_TILE && OFF_S + S_TILE >= OFF_G + VG_TILE,
                   "the R snapshot fits the S region and the G' remainder the SL region");
+    static_assert(SL_TILE >= C * DV * 2 && OFF_SL % 1024 == 0, "dv staged in the SL region (SW128)");
     static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory");
     // elu state passes (bwd_sstate3_kernel, bwd_rstate3_kernel): three stages of
     // [K or Q tile | V_aug or G'_aug], then barriers and the gate prefix sums
@@ -2032,7 +2033,8 @@ template <class Cfg, bool GATED = false>
 __global__ void __launch_bounds__(256, 1)
 bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                const __grid_constant__ CUtensorMap tm_dk, const BwdParams p)
+                const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
+                const BwdParams p)
 {
     using namespace bwd_detail;
     constexpr int C = Cfg::C, D = Cfg::D, DV = Cfg::DV, NA = Cfg::NA, F = Cfg::F, NT = Cfg::NT;
@@ -2271,18 +2273,25 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mph ^= 1u;
         tc_fence_after();
         {
+            // ungated: dv goes as SW128 rows to the G' remainder tile (read only by
+            // dA^T above) and leaves by TMA with dk; gated: row stores (that tile
+            // still feeds the R update)
             __nv_bfloat16 *dvrow = reinterpret_cast<__nv_bfloat16 *>(p.dv) + ((size_t)bh * N + t0 + j) * DV;
 #pragma unroll 1
             for (int c0 = hh * (DV / 2); c0 < (hh + 1) * (DV / 2); c0 += 16) {
                 float g[16];
                 tmem_ld16(tX + lane + c0, g);
                 tmem_ld_wait();
-                if (valid)
 #pragma unroll
-                    for (int e = 0; e < 16; e += 8)
-                        *reinterpret_cast<uint4 *>(dvrow + c0 + e) =
-                            make_uint4(pack_bf16(g[e], g[e + 1]), pack_bf16(g[e + 2], g[e + 3]),
-                                       pack_bf16(g[e + 4], g[e + 5]), pack_bf16(g[e + 6], g[e + 7]));
+                for (int e = 0; e < 16; e += 8) {
+                    const uint4 u = make_uint4(pack_bf16(g[e], g[e + 1]), pack_bf16(g[e + 2], g[e + 3]),
+                                               pack_bf16(g[e + 4], g[e + 5]), pack_bf16(g[e + 6], g[e + 7]));
+                    if constexpr (GATED) {
+                        if (valid) *reinterpret_cast<uint4 *>(dvrow + c0 + e) = u;
+                    } else {
+                        sts128(aGL + sw128_off(j, c0 + e), u);
+                    }
+                }
             }
         }
         if constexpr (GATED) {
@@ -2417,11 +2426,14 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
         }
         full_sync();
-        // the chunk's dk leaves by TMA (rows past the slice's end clipped)
+        // the chunk's dk (and, ungated, dv) leave by TMA (rows past the slice's
+        // end clipped)
         if (tid == 0 && !*abort_flag) {
             if constexpr (TAY) tma_store_3d(&tm_dk, smem + Cfg::OFF_RK, 0, t0, bh);
             else
                 for (int x = 0; x < D; x += 64) tma_store_3d(&tm_dk, sK + (x / 64) * C * 128, x, t0, bh);
+            if constexpr (!GATED)
+                for (int x = 0; x < DV; x += 64) tma_store_3d(&tm_dv, sGL + (x / 64) * C * 128, x, t0, bh);
             bulk_commit();
         }
     }
