@@ -66,7 +66,9 @@ struct FwdCfg {
     // TMEM columns
     static constexpr int COL_O = 0;
     static constexpr int COL_S = (C > NA ? C : NA);
-    static constexpr int TMEM_USED = COL_S + NT * NA;
+    // Taylor: phi(Q) as bf16 pairs (the A operand of MMA2's state term)
+    static constexpr int COL_PQ = COL_S + NT * NA;
+    static constexpr int TMEM_USED = COL_PQ + (TAYLOR ? FP / 2 : 0);
     static constexpr int TMEM_COLS = TMEM_USED <= 256 ? 256 : 512;
     // Shared memory (bytes; every region 1024-aligned)
     static constexpr int QK_TILE = TAYLOR ? C * 32 : C * DQK * 2;   // one raw Q or K tile
@@ -79,6 +81,8 @@ struct FwdCfg {
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + STAGES * QK_TILE;
     static constexpr int OFF_V = OFF_K + STAGES * QK_TILE;
+    // Taylor: two phi(K) tiles (phi(Q) lives in TMEM): the next chunk's is built
+    // while this chunk's MMA2 runs (ungated full forward)
     static constexpr int OFF_PQ = OFF_V + ((STAGES * V_TILE + 1023) / 1024) * 1024;
     static constexpr int OFF_PK = OFF_PQ + PHI_TILE;
     static constexpr int OFF_P = OFF_PK + PHI_TILE;
@@ -464,6 +468,48 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
     };
 
+    // Taylor, full forward: phi(Q) goes to TMEM (columns COL_PQ + 40 h for the
+    // row's half h: K-step kk of MMA2's state term takes columns 8 kk .. 8 kk + 7);
+    // ungated, the next chunk's phi(K) is built into the other phi(K) tile while
+    // this chunk's MMA2 runs.
+    constexpr bool EARLYK = Cfg::TAYLOR && MODE == 0 && !GATED;
+    auto phi_k_tile = [&](int itk) {   // the phi(K) tile of the range's chunk itk
+        return smem + ((EARLYK && (itk & 1)) ? Cfg::OFF_PQ : Cfg::OFF_PK);
+    };
+    // this thread's half of phi(x) (times rs) for row `row` into an SW128 phi tile
+    auto taylor_tile_half = [&](uint8_t *dst, const float *x, bool zero, float rs) {
+        auto features = [&](auto h) {
+            constexpr int F0 = decltype(h)::value * (Cfg::FT / 2);
+#pragma unroll
+            for (int f0 = F0; f0 < F0 + Cfg::FT / 2; f0 += 8) {
+                float v8[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    v8[e] = zero ? 0.f : rs * taylor_sym_feature<16>(x, f0 + e, inv_c1, inv_c2, r2_inv_c2);
+                *reinterpret_cast<uint4 *>(dst + sw128_off(row, f0)) =
+                    make_uint4(pack_bf16(v8[0], v8[1]), pack_bf16(v8[2], v8[3]), pack_bf16(v8[4], v8[5]),
+                               pack_bf16(v8[6], v8[7]));
+            }
+        };
+        if (half == 0) features(std::integral_constant<int, 0>{});
+        else features(std::integral_constant<int, 1>{});
+    };
+    auto taylor_q_tmem = [&](const float *x, float rs) {
+        uint32_t w[40];
+        auto features = [&](auto h) {
+            constexpr int F0 = decltype(h)::value * 80;
+#pragma unroll
+            for (int e = 0; e < 80; e += 2)
+                w[e / 2] = pack_bf16(rs * taylor_sym_feature<16>(x, F0 + e, inv_c1, inv_c2, r2_inv_c2),
+                                     rs * taylor_sym_feature<16>(x, F0 + e + 1, inv_c1, inv_c2, r2_inv_c2));
+        };
+        if (half == 0) features(std::integral_constant<int, 0>{});
+        else features(std::integral_constant<int, 1>{});
+        tmem_st32(tmem + lane_base + Cfg::COL_PQ + 40 * half, w);
+        tmem_st8(tmem + lane_base + Cfg::COL_PQ + 40 * half + 32, w + 32);
+        tmem_st_wait();
+    };
+
     for (int chunk = c_begin; chunk < c_end; ++chunk) {
         const int it = chunk - c_begin;
         const int s = it % STAGES;
@@ -502,8 +548,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         uint8_t *sQ = smem + Cfg::OFF_Q + s * Cfg::QK_TILE;
         uint8_t *sK = smem + Cfg::OFF_K + s * Cfg::QK_TILE;
         uint8_t *sV = smem + Cfg::OFF_V + s * Cfg::V_TILE;
-        uint8_t *sPQ = Cfg::TAYLOR ? smem + Cfg::OFF_PQ : sQ;
-        uint8_t *sPK = Cfg::TAYLOR ? smem + Cfg::OFF_PK : sK;
+        uint8_t *sPQ = sQ;   // elu: phi in place (Taylor: phi(Q) in TMEM)
+        uint8_t *sPK = Cfg::TAYLOR ? phi_k_tile(it) : sK;
 
         // ---- feature maps (token row `row`, column half `half`)
         if (worker) {
@@ -526,31 +572,16 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 // segment pass, gated: phi(K) feeds only MMA3 here, scale it now
                 if (MODE == 1 && gated) scale_row_half(sK, gate_w);
             } else {
-#pragma unroll 1
-                for (int m = (MODE == 0 ? 0 : 1); m < 2; ++m) {
-                    const uint8_t *raw = m == 0 ? sQ : sK;
-                    uint8_t *dst = m == 0 ? sPQ : sPK;
-                    const bool zero = (m == 1) && !kvalid;
-                    const float rs = m == 0 ? gate_e : gate_w;   // 1 ungated
-                    float x[16];
-                    unpack8(*reinterpret_cast<const uint4 *>(raw + sw32_off(i, 0, C)), x);
-                    unpack8(*reinterpret_cast<const uint4 *>(raw + sw32_off(i, 8, C)), x + 8);
-                    // two unrolled copies so every feature index is a compile-time constant
-                    auto features = [&](auto h) {
-                        constexpr int F0 = decltype(h)::value * (Cfg::FT / 2);
-#pragma unroll
-                        for (int f0 = F0; f0 < F0 + Cfg::FT / 2; f0 += 8) {
-                            float v8[8];
-#pragma unroll
-                            for (int e = 0; e < 8; ++e)
-                                v8[e] = zero ? 0.f : rs * taylor_sym_feature<16>(x, f0 + e, inv_c1, inv_c2, r2_inv_c2);
-                            *reinterpret_cast<uint4 *>(dst + sw128_off(i, f0)) =
-                                make_uint4(pack_bf16(v8[0], v8[1]), pack_bf16(v8[2], v8[3]),
-                                           pack_bf16(v8[4], v8[5]), pack_bf16(v8[6], v8[7]));
-                        }
-                    };
-                    if (half == 0) features(std::integral_constant<int, 0>{});
-                    else features(std::integral_constant<int, 1>{});
+                float x[16];
+                if (MODE == 0) {
+                    unpack8(*reinterpret_cast<const uint4 *>(sQ + sw32_off(i, 0, C)), x);
+                    unpack8(*reinterpret_cast<const uint4 *>(sQ + sw32_off(i, 8, C)), x + 8);
+                    taylor_q_tmem(x, gate_e);   // gate_e = 1 ungated
+                }
+                if (!(EARLYK && it > 0)) {   // EARLYK: built during the previous chunk
+                    unpack8(*reinterpret_cast<const uint4 *>(sK + sw32_off(i, 0, C)), x);
+                    unpack8(*reinterpret_cast<const uint4 *>(sK + sw32_off(i, 8, C)), x + 8);
+                    taylor_tile_half(sPK, x, !kvalid, gate_w);
                 }
             }
         }
@@ -658,12 +689,27 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
                 for (int kk = 0; kk < FP / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * (C * 128) + (kk & 3) * 32;
-                    mma_bf16(tmem + Cfg::COL_O, smem_desc(aQ + off, 16, 1024, kSw128),
-                             smem_desc(aS + kk * 512, Cfg::S_BLK, 256, kSw32), idesc, true);
+                    if constexpr (Cfg::TAYLOR)
+                        mma_bf16_ts(tmem + Cfg::COL_O, tmem + Cfg::COL_PQ + kk * 8,
+                                    smem_desc(aS + kk * 512, Cfg::S_BLK, 256, kSw32), idesc, true);
+                    else
+                        mma_bf16(tmem + Cfg::COL_O, smem_desc(aQ + off, 16, 1024, kSw128),
+                                 smem_desc(aS + kk * 512, Cfg::S_BLK, 256, kSw32), idesc, true);
                 }
             }
             if (gated) issue_state_mma(smem_addr(sPK), aV, have_state);
             mma_commit(mma_bar);
+        }
+        if (EARLYK && worker && chunk + 1 < c_end) {
+            // the next chunk's phi(K) into the other tile (MMA3 two chunks back
+            // read it last and has finished) while MMA2 runs
+            const int s1 = (it + 1) % STAGES;
+            if (!mbar_wait(&tma_bar[s1], (uint32_t)((it + 1) / STAGES) & 1u)) *abort_flag = 1;
+            const uint8_t *sK1 = smem + Cfg::OFF_K + s1 * Cfg::QK_TILE;
+            float x[16];
+            unpack8(*reinterpret_cast<const uint4 *>(sK1 + sw32_off(row, 0, C)), x);
+            unpack8(*reinterpret_cast<const uint4 *>(sK1 + sw32_off(row, 8, C)), x + 8);
+            taylor_tile_half(phi_k_tile(it + 1), x, row >= min(C, N - t0 - C), 1.f);
         }
         if (!mbar_wait(mma_bar, mma_phase)) *abort_flag = 1;
         mma_phase ^= 1u;
