@@ -473,6 +473,26 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     // ungated, the next chunk's phi(K) is built into the other phi(K) tile while
     // this chunk's MMA2 runs.
     constexpr bool EARLYK = Cfg::TAYLOR && MODE == 0 && !GATED;
+    // elu with two load stages, full forward: the next chunk's phi(Q) and phi(K)
+    // are formed in place in its stage (already landed) while this chunk's MMA2
+    // runs (the gated form scales them after MMA1, as before)
+    constexpr bool EARLYPHI = !Cfg::TAYLOR && MODE == 0 && STAGES == 2;
+    // elu(x)+1 in place on this thread's half of row `row` of Q and K (K rows
+    // past `kvalid_rows` zeroed)
+    auto elu_phi_in_place = [&](uint8_t *tq, uint8_t *tk, int kvalid_rows, bool do_q) {
+#pragma unroll 1
+        for (int m = do_q ? 0 : 1; m < 2; ++m) {
+            uint8_t *tile = m == 0 ? tq : tk;
+            const bool zero = m == 1 && row >= kvalid_rows;
+#pragma unroll
+            for (int col = half * (DQK / 2); col < (half + 1) * (DQK / 2); col += 8) {
+                const uint32_t a = smem_addr(tile + sw128_off(row, col));
+                const uint4 r = lds128(a);
+                sts128(a, zero ? make_uint4(0u, 0u, 0u, 0u)
+                               : make_uint4(elu1_bf16x2(r.x), elu1_bf16x2(r.y), elu1_bf16x2(r.z), elu1_bf16x2(r.w)));
+            }
+        }
+    };
     auto phi_k_tile = [&](int itk) {   // the phi(K) tile of the range's chunk itk
         return smem + ((EARLYK && (itk & 1)) ? Cfg::OFF_PQ : Cfg::OFF_PK);
     };
@@ -556,19 +576,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const int i = row;
             const bool kvalid = i < nvalid;
             if (!Cfg::TAYLOR) {
-#pragma unroll 1
-                for (int m = 0; m < (MODE == 0 ? 2 : 1); ++m) {
-                    uint8_t *tile = (MODE == 0 && m == 0) ? sQ : sK;
-                    const bool zero = (tile == sK) && !kvalid;
-#pragma unroll
-                    for (int col = half * (DQK / 2); col < (half + 1) * (DQK / 2); col += 8) {
-                        const uint32_t a = smem_addr(tile + sw128_off(i, col));
-                        const uint4 r = lds128(a);
-                        sts128(a, zero ? make_uint4(0u, 0u, 0u, 0u)
-                                       : make_uint4(elu1_bf16x2(r.x), elu1_bf16x2(r.y), elu1_bf16x2(r.z),
-                                                    elu1_bf16x2(r.w)));
-                    }
-                }
+                // EARLYPHI: chunks after the first were converted during the previous one
+                if (!(EARLYPHI && it > 0)) elu_phi_in_place(sQ, sK, nvalid, MODE == 0);
                 // segment pass, gated: phi(K) feeds only MMA3 here, scale it now
                 if (MODE == 1 && gated) scale_row_half(sK, gate_w);
             } else {
@@ -699,6 +708,12 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             if (gated) issue_state_mma(smem_addr(sPK), aV, have_state);
             mma_commit(mma_bar);
+        }
+        if (EARLYPHI && worker && chunk + 1 < c_end) {
+            const int s1 = (it + 1) % STAGES;
+            if (!mbar_wait(&tma_bar[s1], (uint32_t)((it + 1) / STAGES) & 1u)) *abort_flag = 1;
+            elu_phi_in_place(smem + Cfg::OFF_Q + s1 * Cfg::QK_TILE, smem + Cfg::OFF_K + s1 * Cfg::QK_TILE,
+                             min(C, N - t0 - C), true);
         }
         if (EARLYK && worker && chunk + 1 < c_end) {
             // the next chunk's phi(K) into the other tile (MMA3 two chunks back
