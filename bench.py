@@ -463,8 +463,8 @@ def timed(run, steps, warmup, dist_on, device_index, graph_len=None, repeats=1):
     """Run warm-up, then `repeats` timed regions of exactly `steps` steps each,
     replayed from CUDA graphs, each bracketed by a barrier and a device
     synchronisation and timed with CUDA events on the launching stream (max
-    over ranks).  Returns (median ms per step, [min, max] ms per step over the
-    repeats, clocks sampled over all of them)."""
+    over ranks).  Returns (median ms per step, [min, mean, max] ms per step
+    over the repeats, clocks sampled over all of them)."""
     stream = torch.cuda.Stream()
     # eager warm-up: also configures kernels before any capture
     with torch.cuda.stream(stream):
@@ -499,7 +499,7 @@ def timed(run, steps, warmup, dist_on, device_index, graph_len=None, repeats=1):
                 torch.distributed.barrier()
             per_step.append(max_over_ranks(start.elapsed_time(end), dist_on, "cuda") / steps)
     del g, gr
-    return statistics.median(per_step), [min(per_step), max(per_step)], clk.summary()
+    return statistics.median(per_step), [min(per_step), statistics.fmean(per_step), max(per_step)], clk.summary()
 
 
 def _e2e_buffers(w, dev, rank, nsets):
@@ -818,7 +818,8 @@ def main():
         "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if w.dtype == W.BF16 else "f32", "data": "synthetic",
         "config": base_config(w, world),
-        "repeats": args.repeats, "ms_per_step_min_max": [round(x, 6) for x in spread],
+        "repeats": args.repeats, "ms_per_step_min_max": [round(spread[0], 6), round(spread[2], 6)],
+        "ms_per_step_mean": round(spread[1], 6),
         "timing": f"median of {args.repeats} timed regions of {args.steps} steps (CUDA graphs, CUDA events)",
         "l2": run.l2_note(),
         "roofline": dict(roofline_entry("hbm", achieved, hbm, "GB/s", load_traffic("forward:" + w.name)),
@@ -864,7 +865,7 @@ def main():
                 ent["dram_x"] = round(tr / r2.alg_bytes, 3)
             sec[name] = ent
             print(f"[bench] {ws.describe()}: {ent['v'] / 1e6:.2f} M tokens/s, {ms2:.4f} ms/step "
-                  f"(min {spread2[0]:.4f}, max {spread2[1]:.4f}), {ent['hbm'] * 100:.1f} % HBM, "
+                  f"(min {spread2[0]:.4f}, mean {spread2[1]:.4f}, max {spread2[2]:.4f}), {ent['hbm'] * 100:.1f} % HBM, "
                   f"{ent['tc'] * 100:.1f} % bf16 peak, clocks {clk2.get('sm_mhz')} MHz {clk2.get('reasons')}",
                   file=sys.stderr, flush=True)
             del r2
