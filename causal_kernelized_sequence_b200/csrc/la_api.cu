@@ -10,10 +10,12 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 #include <atomic>
+#include <utility>
 #include <mutex>
 
 #include "../../include/la.h"
 #include <cstdio>
+#include <utility>
 
 #include "la_device.cuh"
 #include "la_simt.cuh"
@@ -93,6 +95,31 @@ la_status check_on_current_device(const void *p)
 la_status launch_status()
 {
     const cudaError_t e = cudaGetLastError();
+#ifdef LA_DEBUG_LAUNCH
+    if (e != cudaSuccess) fprintf(stderr, "libla launch error: %s\n", cudaGetErrorString(e));
+#endif
+    return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+// Launch as a programmatic dependent of the previous kernel in the stream:
+// the grid may be scheduled onto SMs that kernel has left once all its blocks
+// have started (every tensor-core forward kernel triggers at its start), and
+// each of these kernels waits for the previous one to complete (its writes
+// visible) before it touches global memory.
+template <typename... KArgs, typename... Args>
+la_status launch_pdl(void (*kernel)(KArgs...), int grid, int threads, int smem, cudaStream_t stream, Args &&...args)
+{
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 #ifdef LA_DEBUG_LAUNCH
     if (e != cudaSuccess) fprintf(stderr, "libla launch error: %s\n", cudaGetErrorString(e));
 #endif
@@ -370,11 +397,10 @@ la_status forward_tc_run(const CUtensorMap &tq, const CUtensorMap &tk, const CUt
     if (set_smem<fwd_tc_kernel<Cfg, 0, GATED>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
     if (p.P > 1) {
         if (set_smem<fwd_tc_kernel<Cfg, 1, GATED>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
-        fwd_tc_kernel<Cfg, 1, GATED><<<BH * p.P, 288, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, to, p);
-        if (launch_status() != LA_OK) return LA_ERR_CUDA;
+        if (launch_pdl(fwd_tc_kernel<Cfg, 1, GATED>, BH * p.P, 288, Cfg::SMEM_ALLOC, stream, tq, tk, tv, to, p) != LA_OK)
+            return LA_ERR_CUDA;
     }
-    fwd_tc_kernel<Cfg, 0, GATED><<<BH * p.P, 288, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, to, p);
-    return launch_status();
+    return launch_pdl(fwd_tc_kernel<Cfg, 0, GATED>, BH * p.P, 288, Cfg::SMEM_ALLOC, stream, tq, tk, tv, to, p);
 }
 
 template <class Cfg>
@@ -454,28 +480,14 @@ la_status forward_split64(const void *q, const void *k, const void *v, void *o, 
 #endif
         return LA_ERR_CUDA;
     }
-    fwd_split_state_kernel<<<p.G, Cfg::S_THREADS, Cfg::S_SMEM_ALLOC, stream>>>(tk, tv, p);
-    if (launch_status() != LA_OK) return LA_ERR_CUDA;
-    // The output launch may start on SMs the state launch has left (programmatic
-    // dependent launch); it waits for the state launch before using its results.
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.G);
-    cfg.blockDim = dim3(Cfg::O_THREADS);
-    cfg.dynamicSmemBytes = Cfg::O_SMEM_ALLOC;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    const cudaError_t le = cudaLaunchKernelEx(&cfg, fwd_split_out_kernel, tq, tv, to, p);
-    if (le != cudaSuccess) {
-#ifdef LA_DEBUG_LAUNCH
-        fprintf(stderr, "libla launch error (output launch): %s\n", cudaGetErrorString(le));
-#endif
+    // Both launches are programmatic dependents of the kernel before them in
+    // the stream: the state launch sets up on SMs the previous kernel has left
+    // and waits for it to complete before touching global memory; the output
+    // launch may start on SMs the state launch has left and waits for the
+    // state launch before using its results.
+    if (launch_pdl(fwd_split_state_kernel, p.G, Cfg::S_THREADS, Cfg::S_SMEM_ALLOC, stream, tk, tv, p) != LA_OK)
         return LA_ERR_CUDA;
-    }
-    return launch_status();
+    return launch_pdl(fwd_split_out_kernel, p.G, Cfg::O_THREADS, Cfg::O_SMEM_ALLOC, stream, tq, tv, to, p);
 }
 
 la_status forward_tc(const void *q, const void *k, const void *v, void *o, const float *s_in, const float *z_in,
@@ -623,8 +635,7 @@ static la_status swa_tc_launch(const void *q, const void *k, const void *v, void
     const int per_sm = Cfg::TMEM_COLS == 256 ? 2 : 1;   // TMEM: 512 columns per SM
     const int grid = (int)(ntiles < (long long)per_sm * kNumSms ? ntiles : per_sm * kNumSms);
     if (set_smem<swa_fwd_tc_kernel<Cfg>>(Cfg::SMEM_ALLOC) != LA_OK) return LA_ERR_CUDA;
-    swa_fwd_tc_kernel<Cfg><<<grid, Cfg::THREADS, Cfg::SMEM_ALLOC, stream>>>(tq, tk, tv, to, p);
-    return launch_status();
+    return launch_pdl(swa_fwd_tc_kernel<Cfg>, grid, Cfg::THREADS, Cfg::SMEM_ALLOC, stream, tq, tk, tv, to, p);
 }
 
 template <typename T>

@@ -215,6 +215,12 @@ fwd_split_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     auto fail = [&]() { *abort_flag = 1; };
+    // This launch may begin while the previous kernel of the stream finishes
+    // (programmatic dependent launch): the setup above overlaps its tail, and
+    // nothing is read or written in global memory before that kernel has
+    // completed (its writes are then visible; the previous forward's output
+    // launch may still read the workspace written below until then).
+    grid_dependency_wait();
     // The output launch may take each SM as soon as this block leaves it; it
     // waits for this whole grid before reading anything written here.
     launch_dependents();
@@ -487,6 +493,10 @@ fwd_split_out_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         return opens ? p.s_in != nullptr : it > 0;
     };
     auto has_carry = [&](int it) { return carry_in && it < first_len; };
+    // The next kernel of the stream may take each SM this block leaves; a
+    // dependent launch of the state kernel (the next forward) waits for this
+    // whole grid before it touches global memory.
+    launch_dependents();
     LA_TLB(1, 0);
     if (tid == 0) LA_TLS(1, 15, 0);
 

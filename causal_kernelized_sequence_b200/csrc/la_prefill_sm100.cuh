@@ -261,6 +261,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     // thread issues the MMAs and refills the load stages, so that no worker
     // stalls behind the tensor pipe's issue queue; every thread meets at the
     // block barriers.
+    // Launched as a programmatic dependent: nothing in global memory is read
+    // or written before the previous kernel of the stream has completed; the
+    // next one may then take the SMs this grid leaves.
+    sm100::grid_dependency_wait();
+    sm100::launch_dependents();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wq = warp & 3, half = warp >> 2, row = wq * 32 + lane;
     const bool worker = tid < 256, issuer = tid == 256;

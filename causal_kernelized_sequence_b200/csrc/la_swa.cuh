@@ -89,6 +89,11 @@ swa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(load_bar + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(load_bar + 3);
 
+    // Launched as a programmatic dependent: nothing in global memory is read
+    // or written before the previous kernel of the stream has completed; the
+    // next one may then take the SMs this grid leaves.
+    grid_dependency_wait();
+    launch_dependents();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wq = warp & 3, hh = warp >> 2, row = wq * 32 + lane;   // TMEM lane quadrant, row half
     const int ntiles = p.BH * p.tiles_per_bh;
