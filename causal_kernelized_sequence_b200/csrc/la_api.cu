@@ -339,22 +339,13 @@ la_status decode_vec(const void *q, const void *k, const void *v, void *y, float
     // state rows per pass: 256 threads / (dv / 4) float4 groups per row
     const int passes = (fp.F + kDecodeThreads / (dv / 4) - 1) / (kDecodeThreads / (dv / 4));
     const bool short_state = passes <= 10;
+    auto go = [&](auto kernel) { return launch_pdl(kernel, B * H, kDecodeThreads, 0, stream, qq, kk, vv, yy, s, z, fp, g); };
     switch (dv) {
-    case 32:
-        if (short_state) decode_vec_kernel<T, 32, 10, 3><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp, g);
-        else decode_vec_kernel<T, 32, 18, 2><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp, g);
-        break;
-    case 64:
-        if (short_state) decode_vec_kernel<T, 64, 10, 3><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp, g);
-        else decode_vec_kernel<T, 64, 18, 2><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp, g);
-        break;
-    case 128:
-        if (short_state) decode_vec_kernel<T, 128, 10, 3><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp, g);
-        else decode_vec_kernel<T, 128, 18, 2><<<B * H, kDecodeThreads, 0, stream>>>(qq, kk, vv, yy, s, z, fp, g);
-        break;
+    case 32: return short_state ? go(decode_vec_kernel<T, 32, 10, 3>) : go(decode_vec_kernel<T, 32, 18, 2>);
+    case 64: return short_state ? go(decode_vec_kernel<T, 64, 10, 3>) : go(decode_vec_kernel<T, 64, 18, 2>);
+    case 128: return short_state ? go(decode_vec_kernel<T, 128, 10, 3>) : go(decode_vec_kernel<T, 128, 18, 2>);
     default: return LA_ERR_UNSUPPORTED;
     }
-    return launch_status();
 }
 
 // ---------------------------------------------------------- tensor maps
@@ -1083,14 +1074,11 @@ la_status la_swa_decode_step(const void *q, const void *k, const void *v, void *
                      aligned(k_cache, 16) && aligned(v_cache, 16);
     if (vec) {
         if (dtype == LA_F32)
-            swa_decode64_kernel<float><<<B * H, 128, 0, st>>>((const float *)q, (const float *)k, (const float *)v,
-                                                              (float *)y, (float *)k_cache, (float *)v_cache, pos,
-                                                              H, window, scale);
-        else
-            swa_decode64_kernel<__nv_bfloat16><<<B * H, 128, 0, st>>>(
-                (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, (__nv_bfloat16 *)y,
-                (__nv_bfloat16 *)k_cache, (__nv_bfloat16 *)v_cache, pos, H, window, scale);
-        return launch_status();
+            return launch_pdl(swa_decode64_kernel<float>, B * H, 128, 0, st, (const float *)q, (const float *)k,
+                              (const float *)v, (float *)y, (float *)k_cache, (float *)v_cache, pos, H, window, scale);
+        return launch_pdl(swa_decode64_kernel<__nv_bfloat16>, B * H, 128, 0, st, (const __nv_bfloat16 *)q,
+                          (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, (__nv_bfloat16 *)y,
+                          (__nv_bfloat16 *)k_cache, (__nv_bfloat16 *)v_cache, pos, H, window, scale);
     }
     if (dtype == LA_F32) {
         if (set_smem<swa_decode_kernel<float>>(bytes) != LA_OK) return LA_ERR_CUDA;

@@ -24,6 +24,7 @@
 #pragma once
 
 #include "la_device.cuh"
+#include "sm100.cuh"
 
 namespace la {
 
@@ -47,6 +48,11 @@ decode_vec_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__r
     __shared__ float red[NW][DV];
     __shared__ float dred[NW];
 
+    // Launched as a programmatic dependent: the previous step's state and
+    // outputs are complete and visible once this returns; the next step's
+    // blocks may then take the SMs this grid leaves.
+    sm100::grid_dependency_wait();
+    sm100::launch_dependents();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int c4 = tid % CPR, r0 = tid / CPR;
     const int F = fp.F, dqk = fp.dqk;

@@ -437,6 +437,11 @@ swa_decode64_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *_
     __shared__ float p_s[64];
     __shared__ float part[16][64];
     __shared__ float red[8];
+    // Launched as a programmatic dependent: the previous step's cache writes
+    // and outputs are complete and visible once this returns; the next step's
+    // blocks may then take the SMs this grid leaves.
+    sm100::grid_dependency_wait();
+    sm100::launch_dependents();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const size_t bh = blockIdx.x;
     const int t = pos[bh / H];
