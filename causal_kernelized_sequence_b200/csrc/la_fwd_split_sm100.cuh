@@ -267,8 +267,15 @@ fwd_split_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
                 mma_commit(&ds_full[b]);
                 bulk_store_hint(p.phik + (size_t)(rg.tb + it) * Cfg::TILE, st, Cfg::TILE, keep);
                 bulk_commit();
-                bulk_wait_read();
-                mma_commit(&stage_free[s]);
+                // Free the previous chunk's stage once its phi(K) store has read it
+                // (every bulk group but this chunk's has been read), not this one's:
+                // the issue of the next chunk's MMA does not wait for the store.
+                // The commit also covers this chunk's MMA, issued after the previous
+                // one's; the range's last stage is never needed again.
+                if (it >= 1) {
+                    bulk_wait_read_le1();
+                    mma_commit(&stage_free[(it - 1) % NS]);
+                }
             }
             asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
         }
