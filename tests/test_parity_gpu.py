@@ -479,3 +479,53 @@ def test_forward_deterministic():
     b = gpu_forward(q, k, v, TAYLOR2, state=True)
     for n in a:
         assert torch.equal(a[n], b[n]), n
+
+
+def _chain(sync):
+    """Calls on one stream whose inputs are the previous calls' outputs:
+    the split forward (its state launch reading k and v that the previous
+    output launch wrote, its output launch reading q), the window prefill,
+    the Taylor prefill and a run of decode steps on a resident state."""
+    def step():
+        if sync:
+            torch.cuda.synchronize()
+    q, k, v, _ = W.random_qkv(8100, 4, 8, 4096, 64, 64, dtype=W.BF16)
+    q, k, v = q.to(DEV), k.to(DEV), v.to(DEV)
+    o1 = la.la_forward(q, k, v, ELU1)["o"]
+    step()
+    o2 = la.la_forward(o1, o1, o1, ELU1)["o"]
+    step()
+    o3 = la.la_swa_forward(o2, o2, o2, 64)["o"]
+    step()
+    o4 = la.la_forward(o3, o3, o3, ELU1)["o"]
+    step()
+    qt, kt, vt, _ = W.random_qkv(8101, 8, 16, 2048, 16, 64, fmap=TAYLOR2, dtype=W.BF16)
+    qt, kt, vt = qt.to(DEV), kt.to(DEV), vt.to(DEV)
+    t1 = la.la_forward(qt, kt, vt, TAYLOR2)["o"]
+    step()
+    t2 = la.la_forward(qt, kt, t1, TAYLOR2)["o"]
+    step()
+    r = la.la_forward(qt[:, :, :1000].contiguous(), kt[:, :, :1000].contiguous(), vt[:, :, :1000].contiguous(),
+                      TAYLOR2, state=True)
+    s, z = r["s"], r["z"]
+    ys = []
+    for t in range(1000, 1016):
+        step()
+        ys.append(la.la_decode_step(qt[:, :, t].contiguous(), kt[:, :, t].contiguous(), vt[:, :, t].contiguous(),
+                                    s, z, TAYLOR2))
+    torch.cuda.synchronize()
+    la.la_get_device_status()
+    out = {"o1": o1, "o2": o2, "o3": o3, "o4": o4, "t1": t1, "t2": t2, "s": s, "z": z}
+    out.update({f"y{i}": y for i, y in enumerate(ys)})
+    return {n: x.cpu() for n, x in out.items()}
+
+
+def test_back_to_back_calls_see_previous_results():
+    """The tensor-core forward and decode kernels are launched as programmatic
+    dependents of the kernel before them; each must wait for it before reading
+    its results.  Every kernel here is deterministic, so the chain run without
+    host synchronisation must match the synchronised one bit for bit."""
+    a = _chain(sync=True)
+    b = _chain(sync=False)
+    for n in a:
+        assert torch.equal(a[n], b[n]), n
