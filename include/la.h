@@ -38,7 +38,14 @@
  *    never allocates or frees device memory and never synchronises, except
  *    la_get_device_status.  Work is enqueued on `stream` (a cudaStream_t,
  *    passed as void*; NULL is the legacy default stream) and runs
- *    asynchronously.
+ *    asynchronously.  The tensor-core forward kernels and the decode kernels
+ *    are launched with programmatic stream serialization: each waits for the
+ *    kernel before it in the stream to complete before it touches memory,
+ *    and lets the kernel after it be scheduled while it drains.  A kernel of
+ *    the caller that follows one of these calls and is itself launched with
+ *    programmatic stream serialization must wait for its prerequisite grid
+ *    (griddepcontrol.wait) before it reads this call's results, as that
+ *    launch attribute requires of every kernel.
  *  - Layouts are dense row-major: q, k [B,H,N,dqk]; v, o [B,H,N,dv];
  *    gradients like their primal; den [B,H,N] fp32; state S [B,H,F,dv] fp32
  *    and z [B,H,F] fp32 with the feature order above and no padding.
