@@ -247,9 +247,18 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     using namespace sm100;
     using namespace fwd_detail;
     constexpr int C = Cfg::C, DV = Cfg::DV, NA = Cfg::NA, DQK = Cfg::DQK, FP = Cfg::FP;
-    constexpr int STAGES = Cfg::STAGES;
+    // The d = 128 segment pass reads only K and V, so it takes a second K/V
+    // stage in the regions the main pass uses for Q and for P (and the state
+    // snapshot), which it leaves unused.
+    constexpr bool SEG2 = MODE == 1 && DQK == 128;
+    constexpr int STAGES = SEG2 ? 2 : Cfg::STAGES;
+    static_assert(!SEG2 || (Cfg::STAGES == 1 && Cfg::OFF_Q + Cfg::QK_TILE <= Cfg::OFF_K &&
+                            Cfg::OFF_P % 1024 == 0 && Cfg::OFF_P + Cfg::V_TILE <= Cfg::OFF_BAR),
+                  "second segment-pass stage");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    auto stage_k = [&](int s) { return (SEG2 && s == 1) ? smem + Cfg::OFF_Q : smem + Cfg::OFF_K + s * Cfg::QK_TILE; };
+    auto stage_v = [&](int s) { return (SEG2 && s == 1) ? smem + Cfg::OFF_P : smem + Cfg::OFF_V + s * Cfg::V_TILE; };
     uint64_t *tma_bar = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
     uint64_t *mma_bar = tma_bar + 2;
     uint64_t *x_bar = tma_bar + 5;   // MODE 0: the scores (MMA1) alone, so the mask need not wait for MMA3
@@ -308,7 +317,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (warp == 0) tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
     // Constant normaliser block of every V stage: column DV of V_aug = 1.
     for (int s = 0; s < STAGES && tid < C; ++s) {
-        uint8_t *blk = smem + Cfg::OFF_V + s * Cfg::V_TILE + (DV / 16) * Cfg::V_BLK;
+        uint8_t *blk = stage_v(s) + (DV / 16) * Cfg::V_BLK;
         const int r = tid;  // C == 128 rows
         uint4 *row = reinterpret_cast<uint4 *>(blk + (r >> 3) * 256 + (r & 7) * 32);
         const int one_chunk = 0 ^ ((r >> 2) & 1);
@@ -326,14 +335,14 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const int t0 = chunk * C;
         mbar_arrive_expect_tx(&tma_bar[s], MODE == 0 ? Cfg::TX_BYTES : Cfg::TX_BYTES - C * DQK * 2);
         uint8_t *q_dst = smem + Cfg::OFF_Q + s * Cfg::QK_TILE;
-        uint8_t *k_dst = smem + Cfg::OFF_K + s * Cfg::QK_TILE;
+        uint8_t *k_dst = stage_k(s);
         constexpr int QBOX = Cfg::TAYLOR ? 16 : 64;
         for (int x = 0; x < DQK; x += QBOX) {
             const int off = Cfg::TAYLOR ? 0 : (x / 64) * C * 128;
             if (MODE == 0) tma_load_3d(q_dst + off, &tm_q, &tma_bar[s], x, t_base + t0, tz);
             tma_load_3d(k_dst + off, &tm_k, &tma_bar[s], x, t_base + t0, tz);
         }
-        uint8_t *v_dst = smem + Cfg::OFF_V + s * Cfg::V_TILE;
+        uint8_t *v_dst = stage_v(s);
         for (int x = 0; x < DV; x += 16)
             tma_load_3d(v_dst + (x / 16) * Cfg::V_BLK, &tm_v, &tma_bar[s], x, t_base + t0, tz);
     };
@@ -571,8 +580,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         // (the issuer waits too: its MMAs read the stage)
         if (!mbar_wait(&tma_bar[s], tphase)) *abort_flag = 1;
         uint8_t *sQ = smem + Cfg::OFF_Q + s * Cfg::QK_TILE;
-        uint8_t *sK = smem + Cfg::OFF_K + s * Cfg::QK_TILE;
-        uint8_t *sV = smem + Cfg::OFF_V + s * Cfg::V_TILE;
+        uint8_t *sK = stage_k(s);
+        uint8_t *sV = stage_v(s);
         uint8_t *sPQ = sQ;   // elu: phi in place (Taylor: phi(Q) in TMEM)
         uint8_t *sPK = Cfg::TAYLOR ? phi_k_tile(it) : sK;
 
