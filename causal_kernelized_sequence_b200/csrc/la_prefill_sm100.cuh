@@ -262,6 +262,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     uint64_t *tma_bar = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
     uint64_t *mma_bar = tma_bar + 2;
     uint64_t *x_bar = tma_bar + 5;   // MODE 0: the scores (MMA1) alone, so the mask need not wait for MMA3
+    uint64_t *k_bar = tma_bar + 6;   // MODE 0, d = 128, ungated: MMA1 and MMA3 done with the K tile
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tma_bar + 3);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tma_bar + 4);
 
@@ -307,6 +308,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (int s = 0; s < STAGES; ++s) mbar_init(&tma_bar[s], 1);
         mbar_init(mma_bar, 1);
         mbar_init(x_bar, 1);
+        mbar_init(k_bar, 1);
         *abort_flag = 0;
         mbar_init_fence();
         prefetch_tensormap(&tm_q);
@@ -346,6 +348,25 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (int x = 0; x < DV; x += 16)
             tma_load_3d(v_dst + (x / 16) * Cfg::V_BLK, &tm_v, &tma_bar[s], x, t_base + t0, tz);
     };
+    // The d = 128 full forward (one stage, ungated) loads a chunk's K as soon as
+    // MMA1 and MMA3 have finished with the previous chunk's phi(K), and its Q
+    // and V once MMA2 has completed: the K bytes are added to the phase ahead
+    // of the arrival that the Q and V copies bring.
+    constexpr bool EARLYK128 = MODE == 0 && DQK == 128 && !GATED && STAGES == 1;
+    auto issue_k = [&](int chunk, int s) {
+        mbar_expect_tx(&tma_bar[s], C * DQK * 2);
+        for (int x = 0; x < DQK; x += 64)
+            tma_load_3d(stage_k(s) + (x / 64) * C * 128, &tm_k, &tma_bar[s], x, t_base + chunk * C, tz);
+    };
+    auto issue_qv = [&](int chunk, int s) {
+        const int t0 = chunk * C;
+        mbar_arrive_expect_tx(&tma_bar[s], Cfg::TX_BYTES - C * DQK * 2);
+        for (int x = 0; x < DQK; x += 64)
+            tma_load_3d(smem + Cfg::OFF_Q + s * Cfg::QK_TILE + (x / 64) * C * 128, &tm_q, &tma_bar[s], x, t_base + t0, tz);
+        for (int x = 0; x < DV; x += 16)
+            tma_load_3d(stage_v(s) + (x / 16) * Cfg::V_BLK, &tm_v, &tma_bar[s], x, t_base + t0, tz);
+    };
+    uint32_t k_phase = 0;
 
     bool have_state = false;
     constexpr bool gated = GATED;
@@ -639,6 +660,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             if (MODE == 0) mma_commit(x_bar);
             // MMA3 runs under the mask step; the commit after MMA2 covers it
             if (!gated || MODE == 1) issue_state_mma(aK, aV, have_state);
+            if (EARLYK128) mma_commit(k_bar);
             if (MODE == 1) mma_commit(mma_bar);
         }
         if (MODE == 0) {
@@ -722,6 +744,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             if (gated) issue_state_mma(smem_addr(sPK), aV, have_state);
             mma_commit(mma_bar);
+            if (EARLYK128 && it + 1 < c_end - c_begin) {
+                if (!mbar_wait(k_bar, k_phase)) *abort_flag = 1;
+                k_phase ^= 1u;
+                issue_k(chunk + 1, s);
+            }
         }
         if (EARLYPHI && worker && chunk + 1 < c_end) {
             const int s1 = (it + 1) % STAGES;
@@ -744,7 +771,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         mma_phase ^= 1u;
         tc_fence_after();
         if (gated) have_state = true;
-        if (issuer && it + STAGES < c_end - c_begin) issue_tma(chunk + STAGES, s);
+        if (issuer && it + STAGES < c_end - c_begin) {
+            if (EARLYK128) issue_qv(chunk + STAGES, s);
+            else issue_tma(chunk + STAGES, s);
+        }
 
         // ---- outputs: y = num / den (this thread's half of the value columns).
         // y goes to the P tile (free once MMA2 has completed) as SW128 rows and

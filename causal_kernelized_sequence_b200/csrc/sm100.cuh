@@ -30,6 +30,14 @@ __device__ __forceinline__ void mbar_init_fence()
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
+// Raise the transaction count of the current phase without arriving: bytes of
+// a copy issued ahead of the arrival that will complete the phase.
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes)
 {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
