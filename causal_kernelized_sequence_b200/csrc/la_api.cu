@@ -120,10 +120,12 @@ la_status launch_pdl(void (*kernel)(KArgs...), int grid, int threads, int smem, 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    if (e == cudaSuccess) return LA_OK;
 #ifdef LA_DEBUG_LAUNCH
-    if (e != cudaSuccess) fprintf(stderr, "libla launch error: %s\n", cudaGetErrorString(e));
+    fprintf(stderr, "libla launch error: %s\n", cudaGetErrorString(e));
 #endif
-    return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+    (void)cudaGetLastError();   // consume it, as launch_status does for the other launches
+    return LA_ERR_CUDA;
 }
 
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device) and
