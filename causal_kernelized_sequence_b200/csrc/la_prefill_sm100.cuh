@@ -14,7 +14,9 @@
 // issues the MMAs and the refill loads; token i <-> TMEM lane i, whose row two
 // workers share, warps w and w + 4 each taking half of its columns):
 //   TMA     Q_c, K_c (SW128, or SW32 for d'=16) and V_c (SW32) into a
-//           2-stage ring (one stage for d = 128).  Rows past the slice's
+//           2-stage ring (d = 128: one stage, with the next chunk's K loaded
+//           once MMA1 and MMA3 are done with this one's; the segment pass,
+//           which reads only K and V, two).  Rows past the slice's
 //           end read as zeros (fixed length) or hold the next packed
 //           sequence's tokens; either way they are kept out of the state
 //           and out of every stored row.
